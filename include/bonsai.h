@@ -1,0 +1,159 @@
+/*
+ * bonsai.h -- C ABI of libbonsai, the B200 (sm_100a) ternary linear layer of
+ * Bonsai 2-style ternary language models.
+ *
+ * The layer computes  y = x' . Wdeq^T  where
+ *   - W is N x K (out x in) with trits t in {-1, 0, +1} and one FP16 scale per
+ *     run of 128 weights along K:  Wdeq[n][k] = s[n][k/128] * t[n][k];
+ *     source: "27B 模型压到 5.95GB，推理能力还保住 98%" (allhereai.com), the
+ *     paragraph describing the method (ternary weights, a shared FP16 scale per
+ *     128 weights, a block Hadamard rotation folded into storage);
+ *   - x' = blockdiag(Hn) x is the online block-Hadamard rotation of the
+ *     activations, Hn = H_128 / sqrt(128) with H_128 the Sylvester matrix
+ *     (Hn[i][j] = (-1)^popcount(i & j) / sqrt(128)), applied to each run of 128
+ *     activations starting at a multiple of 128; sources: the same page, the
+ *     paragraph on running the files (a Hadamard activation runtime is needed,
+ *     without it the output is garbage), and "Bonsai 2，把27B压进6个G"
+ *     (10100.com), section 它怎么做到的 (the input must get the matching transform).
+ *
+ * Layouts (all row-major, all buffers owned by the caller):
+ *   x       M x K   FP16 (IEEE binary16 bit patterns in uint16_t)
+ *   y       M x N   FP16, round-to-nearest-even from an FP32 accumulator
+ *   scales  N x K/128  FP16
+ *   trits   N x K   int8 in {-1, 0, +1}
+ *   packed  the trit plane of one of the two packings of the allhereai.com page
+ *           (paragraph on the two file packings):
+ *     BONSAI_FMT_PTQ1_0  "compact trits", 1.75 bits/weight with the scale:
+ *         row n, group g (128 weights) occupies 26 bytes at (n*K/128 + g)*26;
+ *         byte b < 25 holds weights 128g+5b .. 128g+5b+4, byte 25 the last
+ *         three, as  byte = sum_i (t_i + 1) * 3^i  (first weight least
+ *         significant; padding digits zero, so byte 25 < 27; bytes >= 243
+ *         are invalid).  Trit plane size N * K/128 * 26 bytes.
+ *     BONSAI_FMT_PQ2_0   one trit per 2-bit slot, 2.125 bits/weight with the
+ *         scale: weight k of row n is code t+1 in bits 2(k%4), 2(k%4)+1 of byte
+ *         n*K/4 + k/4 (code 3 is invalid).  Trit plane size N * K/4 bytes.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are CUDA device pointers (any allocator) and must be 16-byte
+ *     aligned; sizes are element counts.  K must be a positive multiple of 128;
+ *     M and N must be >= 1 (M = 0 or N = 0 is accepted and launches nothing).
+ *   - stream is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Calls are asynchronous on it.  The return value reports argument
+ *     validation and launch only: on a non-zero return nothing was launched
+ *     (validation) or the launch failed (BONSAI_ERR_CUDA).  Faults inside a
+ *     kernel surface at the caller's next synchronisation.
+ *   - The library keeps one internal workspace per device (FP32 split-K
+ *     partials and an FP16 copy of x' for the prefill GEMM).  It is allocated
+ *     with cudaMalloc on the first call that needs it, grown when a larger
+ *     call arrives (after a device synchronisation), and released by
+ *     bonsai_shutdown().  Calls that use it must not overlap on the GPU (keep
+ *     them on one stream); bonsai_reserve() sizes it ahead of stream capture.
+ *   - Invalid codes in a packed plane (PTQ1_0 bytes >= 243, PQ2_0 code 3)
+ *     produce unspecified output values but never out-of-bounds accesses.
+ */
+#ifndef BONSAI_H
+#define BONSAI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BONSAI_FMT_PTQ1_0 = 1,
+    BONSAI_FMT_PQ2_0 = 2
+} bonsai_fmt;
+
+typedef enum {
+    BONSAI_OK = 0,
+    BONSAI_ERR_NULL = -1,   /* a required pointer is NULL                          */
+    BONSAI_ERR_SHAPE = -2,  /* M, N or K negative, K not a multiple of 128, or too large */
+    BONSAI_ERR_FMT = -3,    /* unknown packing format                             */
+    BONSAI_ERR_ALIGN = -4,  /* a pointer is not 16-byte aligned                   */
+    BONSAI_ERR_CUDA = -5,   /* a CUDA runtime call or kernel launch failed        */
+    BONSAI_ERR_ARCH = -6,   /* the current device is not compute capability 10.0  */
+    BONSAI_ERR_NOMEM = -7,  /* the internal workspace could not be allocated      */
+    BONSAI_ERR_ALGO = -8    /* the requested kernel cannot run this shape         */
+} bonsai_status;
+
+/* Kernel selection for bonsai_ternary_linear_algo (bonsai_ternary_linear uses AUTO). */
+typedef enum {
+    BONSAI_ALGO_AUTO = 0,
+    BONSAI_ALGO_SIMPLE = 1,  /* one warp per output row; any M (slow, plain)              */
+    BONSAI_ALGO_GEMV = 2,    /* batch-1 lookup-table GEMV with split-K; M == 1 only       */
+    BONSAI_ALGO_SKINNY = 3,  /* register-dequant tensor-core kernel; 1 <= M <= 16         */
+    BONSAI_ALGO_GEMM = 4     /* tcgen05/TMEM prefill GEMM on FP16 tiles; any M            */
+} bonsai_algo;
+
+/* Library version, (major << 16) | (minor << 8) | patch. */
+int bonsai_version(void);
+
+/* Human-readable text for a bonsai_status value (static storage). */
+const char *bonsai_status_string(int status);
+
+/* BONSAI_OK if the current CUDA device is an sm_100 part this build can run on,
+ * BONSAI_ERR_ARCH if it is another architecture, BONSAI_ERR_CUDA if there is no
+ * usable device. */
+int bonsai_check_device(void);
+
+/* Bytes of the packed trit plane for N x K weights (scales excluded: they are
+ * always N * K/128 FP16 values).  Returns BONSAI_ERR_SHAPE / BONSAI_ERR_FMT
+ * (negative) on a bad argument. */
+int64_t bonsai_packed_bytes(int fmt, int64_t N, int64_t K);
+
+/* Packs N x K trits into the PTQ1_0 plane (layout above).  A trit outside
+ * {-1, 0, +1} makes its byte 0xFF, an invalid code, so a bad input is
+ * detectable by bonsai_unpack.  Packing is an offline step; its cost is not on
+ * the inference path.  Source: allhereai.com page, paragraph on the packings. */
+int bonsai_pack_ptq1(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K, void *stream);
+
+/* Packs N x K trits into the PQ2_0 plane (layout above).  A trit outside
+ * {-1, 0, +1} is stored as the invalid code 3.  Same source. */
+int bonsai_pack_pq2(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K, void *stream);
+
+/* Unpacks a plane of format fmt back into N x K int8 trits.  Invalid codes
+ * unpack to -128 (every trit of an invalid PTQ1_0 byte).  Test hook: it makes
+ * the packed layout checkable byte for byte. */
+int bonsai_unpack(int fmt, const uint8_t *packed, int8_t *trits, int64_t N, int64_t K,
+                  void *stream);
+
+/* x_out = blockdiag(Hn) x for an M x K FP16 matrix (the rotation defined above),
+ * computed in FP32 and rounded to FP16 (nearest even).  x_out may equal x (in
+ * place) but must not otherwise overlap it.  This is the same transform
+ * bonsai_ternary_linear applies internally; it is exported for callers that
+ * keep rotated activations and as a test hook. */
+int bonsai_hadamard128(const uint16_t *x, uint16_t *x_out, int64_t M, int64_t K, void *stream);
+
+/* y = x' . Wdeq^T (definitions above) for un-rotated FP16 x: the Hadamard
+ * rotation of x is applied inside the call.  Dispatch on M: M == 1 -> GEMV,
+ * 2 <= M <= 16 -> skinny tensor-core kernel, larger M -> tcgen05 GEMM.  y must
+ * not overlap x, packed or scales.  Source of the operation: allhereai.com page,
+ * method paragraph and packings paragraph. */
+int bonsai_ternary_linear(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                          uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, void *stream);
+
+/* As bonsai_ternary_linear with an explicit kernel choice (bonsai_algo) and an
+ * explicit split-K factor for the GEMV / skinny kernels (0 = automatic, 1 = no
+ * split, otherwise the number of K slices, clamped to what the shape allows).
+ * Returns BONSAI_ERR_ALGO if the chosen kernel cannot run the shape (e.g.
+ * BONSAI_ALGO_GEMV with M > 1).  For measurement and testing of each kernel. */
+int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                               uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int algo,
+                               int split_k, void *stream);
+
+/* Grows the calling device's workspace so that calls up to M x N x K (any
+ * format and kernel) need no further allocation; call before capturing calls
+ * into a CUDA graph.  Synchronises the device if it reallocates. */
+int bonsai_reserve(int64_t M, int64_t N, int64_t K);
+
+/* Frees the workspaces of every device (after synchronising each).  The
+ * library stays usable: the next call allocates again. */
+void bonsai_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BONSAI_H */

@@ -1,0 +1,81 @@
+// common.cuh -- device helpers shared by the libbonsai kernels.
+//
+// The block Hadamard rotation (source: "27B 模型压到 5.95GB，推理能力还保住 98%",
+// allhereai.com, the method paragraph and the paragraph on running the files;
+// "Bonsai 2，把27B压进6个G", 10100.com, section 它怎么做到的) is applied to each run
+// of 128 activations: x'[i] = sum_j Hn[i][j] x[j], Hn[i][j] = (-1)^popcount(i&j)/sqrt(128).
+// The fast Walsh-Hadamard transform below computes it with 7 butterfly stages
+// (one per index bit), which is the Sylvester matrix in natural order.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace bonsai {
+
+constexpr int kGroup = 128;           // weights per FP16 scale == Hadamard block size
+constexpr int kPtq1GroupBytes = 26;   // 25 bytes x 5 trits + 1 byte x 3 trits
+constexpr int kPq2GroupBytes = 32;    // 128 trits x 2 bits
+constexpr float kHadamardNorm = 0.088388347648318440550f;  // 1/sqrt(128)
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
+    return __half2float(__ushort_as_half(h));
+}
+
+__device__ __forceinline__ uint16_t float_to_half_bits(float f) {
+    return __half_as_ushort(__float2half_rn(f));
+}
+
+// One 128-block held by a warp, lane l holding elements 4l .. 4l+3 in v[0..3].
+// On return v holds the same positions of Hn * block (FP32 throughout).
+__device__ __forceinline__ void fwht128_warp(float v[4], int lane) {
+    // index bits 0 and 1 live inside the lane
+    const float a0 = v[0] + v[1], a1 = v[0] - v[1];
+    const float a2 = v[2] + v[3], a3 = v[2] - v[3];
+    v[0] = a0 + a2;
+    v[2] = a0 - a2;
+    v[1] = a1 + a3;
+    v[3] = a1 - a3;
+    // index bits 2..6 are lane bits 0..4: butterfly (a, b) -> (a + b, a - b)
+#pragma unroll
+    for (int b = 0; b < 5; b++) {
+        const int mask = 1 << b;
+        const bool upper = (lane & mask) != 0;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float p = __shfl_xor_sync(0xffffffffu, v[i], mask);
+            v[i] = upper ? (p - v[i]) : (v[i] + p);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; i++) v[i] *= kHadamardNorm;
+}
+
+// Loads 4 consecutive FP16 values (8 bytes, 8-byte aligned) as floats.
+__device__ __forceinline__ void load_half4(const uint16_t *p, float v[4]) {
+    const uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    const __half2 h01 = *reinterpret_cast<const __half2 *>(&raw.x);
+    const __half2 h23 = *reinterpret_cast<const __half2 *>(&raw.y);
+    const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+    v[0] = f01.x;
+    v[1] = f01.y;
+    v[2] = f23.x;
+    v[3] = f23.y;
+}
+
+__device__ __forceinline__ void store_half4(uint16_t *p, const float v[4]) {
+    const __half2 h01 = __floats2half2_rn(v[0], v[1]);
+    const __half2 h23 = __floats2half2_rn(v[2], v[3]);
+    uint2 raw;
+    raw.x = *reinterpret_cast<const uint32_t *>(&h01);
+    raw.y = *reinterpret_cast<const uint32_t *>(&h23);
+    *reinterpret_cast<uint2 *>(p) = raw;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+}  // namespace bonsai

@@ -1,0 +1,72 @@
+// internal.h -- launchers shared between the C-ABI layer (bonsai_api.cu) and the
+// kernel files.  Not part of the public interface.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace bonsai {
+
+struct DeviceInfo {
+    int sm_count = 0;
+    int major = 0, minor = 0;
+    int smem_optin = 0;  // max dynamic shared memory per block (opt-in), bytes
+    int l2_bytes = 0;
+};
+
+// Split-K bookkeeping lives at the start of the workspace: kMaxTiles arrival
+// counters, zero when the workspace is created and returned to zero by the
+// last CTA of each tile, so consecutive calls need no memset.
+constexpr int kMaxTiles = 65536;
+constexpr size_t kCounterBytes = kMaxTiles * sizeof(unsigned int);
+
+struct Workspace {
+    unsigned int *counters = nullptr;  // kMaxTiles entries
+    uint8_t *data = nullptr;           // the rest, 256-byte aligned
+    size_t data_bytes = 0;
+};
+
+// ---- pack.cu
+cudaError_t launch_pack_ptq1(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K,
+                             cudaStream_t s, const DeviceInfo &dev);
+cudaError_t launch_pack_pq2(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K,
+                            cudaStream_t s, const DeviceInfo &dev);
+cudaError_t launch_unpack(int fmt, const uint8_t *packed, int8_t *trits, int64_t N, int64_t K,
+                          cudaStream_t s, const DeviceInfo &dev);
+
+// ---- hadamard.cu
+cudaError_t launch_hadamard_f16(const uint16_t *x, uint16_t *out, int64_t M, int64_t K,
+                                cudaStream_t s, const DeviceInfo &dev);
+cudaError_t launch_hadamard_f32(const uint16_t *x, float *out, int64_t M, int64_t K,
+                                cudaStream_t s, const DeviceInfo &dev);
+
+// ---- linear_simple.cu: x' (FP32, M x K) in the workspace, then one warp per row
+size_t simple_workspace_bytes(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_linear_simple(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                                 uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt,
+                                 const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
+
+// ---- gemv_lut.cu: M == 1
+bool gemv_supported(int64_t M, int64_t N, int64_t K, int fmt);
+size_t gemv_workspace_bytes(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev);
+cudaError_t launch_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                        uint16_t *y, int64_t N, int64_t K, int fmt, int split_k,
+                        const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
+
+// ---- skinny_mma.cu: 1 <= M <= 16
+bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt);
+size_t skinny_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int split_k,
+                              const DeviceInfo &dev);
+cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                          uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int split_k,
+                          const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
+
+// ---- gemm_tcgen05.cu: prefill
+bool gemm_supported(int64_t M, int64_t N, int64_t K, int fmt);
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt);
+cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                        uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt,
+                        const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
+
+}  // namespace bonsai

@@ -1,0 +1,90 @@
+"""The C-ABI library without a GPU: it loads, exports every declared entry
+point, and rejects bad arguments on the host before touching CUDA."""
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bonsai.h")
+
+
+@pytest.fixture(scope="module")
+def bz():
+    from ternary_weight_02_b200 import build
+    build.build()
+    from ternary_weight_02_b200 import bonsai
+    return bonsai
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(bonsai_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("bonsai_pack_ptq1", "bonsai_pack_pq2", "bonsai_hadamard128",
+                     "bonsai_ternary_linear", "bonsai_unpack", "bonsai_packed_bytes"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(bz):
+    lib = bz.raw()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    with open("/proc/self/maps") as f:
+        assert any(bz.LIB_PATH in line for line in f)
+
+
+def test_packed_bytes_host_arithmetic(bz):
+    assert bz.bonsai_packed_bytes(bz.BONSAI_FMT_PTQ1_0, 5120, 17408) == 5120 * 136 * 26
+    assert bz.bonsai_packed_bytes(bz.BONSAI_FMT_PQ2_0, 34816, 5120) == 34816 * 1280
+    assert bz.raw().bonsai_packed_bytes(bz.BONSAI_FMT_PQ2_0, 4, 100) == bz.BONSAI_ERR_SHAPE
+    assert bz.raw().bonsai_packed_bytes(7, 4, 128) == bz.BONSAI_ERR_FMT
+    assert bz.raw().bonsai_packed_bytes(1, -1, 128) == bz.BONSAI_ERR_SHAPE
+
+
+def test_host_validation_needs_no_gpu(bz):
+    L = bz.raw()
+    good = 1 << 20  # an aligned non-null value; validation rejects before it is used
+    # NULL pointers
+    assert L.bonsai_ternary_linear(None, good, good, good, 1, 8, 128, 2, None) == bz.BONSAI_ERR_NULL
+    assert L.bonsai_pack_pq2(good, None, 4, 128, None) == bz.BONSAI_ERR_NULL
+    assert L.bonsai_hadamard128(None, good, 1, 128, None) == bz.BONSAI_ERR_NULL
+    # shapes
+    assert L.bonsai_ternary_linear(good, good, good, good, 1, 8, 100, 2, None) == bz.BONSAI_ERR_SHAPE
+    assert L.bonsai_ternary_linear(good, good, good, good, -1, 8, 128, 2, None) == bz.BONSAI_ERR_SHAPE
+    assert L.bonsai_ternary_linear(good, good, good, good, 1, 8, 0, 2, None) == bz.BONSAI_ERR_SHAPE
+    assert L.bonsai_hadamard128(good, good, 2, 64, None) == bz.BONSAI_ERR_SHAPE
+    # format
+    assert L.bonsai_ternary_linear(good, good, good, good, 1, 8, 128, 0, None) == bz.BONSAI_ERR_FMT
+    assert L.bonsai_unpack(3, good, good, 1, 128, None) == bz.BONSAI_ERR_FMT
+    # alignment
+    assert L.bonsai_ternary_linear(good + 2, good, good, good, 1, 8, 128, 2, None) == bz.BONSAI_ERR_ALIGN
+    assert L.bonsai_pack_ptq1(good, good + 8, 4, 128, None) == bz.BONSAI_ERR_ALIGN
+    # algorithm choice that cannot take the shape
+    assert (L.bonsai_ternary_linear_algo(good, good, good, good, 1, 8, 128, 2, 99, 0, None)
+            == bz.BONSAI_ERR_ALGO)
+    # empty problems are accepted and launch nothing
+    assert L.bonsai_ternary_linear(None, None, None, None, 0, 8, 128, 2, None) == bz.BONSAI_OK
+    assert L.bonsai_pack_pq2(None, None, 0, 128, None) == bz.BONSAI_OK
+
+
+def test_status_strings(bz):
+    for code in range(-8, 1):
+        s = bz.bonsai_status_string(code)
+        assert s and s != "unknown status"
+    assert bz.bonsai_status_string(-99) == "unknown status"
+    assert bz.bonsai_version() >= (0 << 16) | (1 << 8)
+
+
+def test_no_device_reports_cuda_error(bz):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    good = 1 << 20
+    assert bz.bonsai_check_device() == bz.BONSAI_ERR_CUDA
+    assert bz.raw().bonsai_ternary_linear(good, good, good, good, 1, 8, 128, 2, None) == bz.BONSAI_ERR_CUDA

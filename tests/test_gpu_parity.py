@@ -1,0 +1,148 @@
+"""GPU parity through the C ABI against the CPU checker.
+
+Integer work (packing, unpacking) must be bit-exact; the linear layer must meet
+rel-L2 <= 1e-3 and max|y - y_ref| <= 1e-2 * rms(y_ref) against the float64
+checker on the same seeded inputs."""
+import numpy as np
+import pytest
+
+import oracle
+from tests.gpu_util import Problem, to_numpy_f16
+
+pytestmark = pytest.mark.gpu
+
+PTQ1, PQ2 = oracle.FMT_PTQ1_0, oracle.FMT_PQ2_0
+
+
+@pytest.fixture(scope="module")
+def bz():
+    import torch
+    from ternary_weight_02_b200 import bonsai
+    assert bonsai.bonsai_check_device() == bonsai.BONSAI_OK
+    torch.cuda.init()
+    return bonsai
+
+
+# ------------------------------------------------------------ codec
+
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("N,K", [(1, 128), (3, 384), (37, 1024), (64, 5120), (5, 17408)])
+def test_pack_bit_exact(bz, fmt, N, K):
+    import torch
+    p = Problem(0, N, K, fmt, seed=N + K)
+    packed = bz.pack(fmt, torch.from_numpy(p.trits).cuda())
+    torch.cuda.synchronize()
+    want = p.oracle_packed()
+    got = packed.cpu().numpy().reshape(want.shape)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+def test_unpack_bit_exact_and_invalid_codes(bz, fmt):
+    import torch
+    N, K = 9, 640
+    p = Problem(0, N, K, fmt, seed=3)
+    packed = p.oracle_packed().copy()
+    # plant invalid codes in the host-side plane before upload
+    flat = packed.reshape(-1)
+    if fmt == PTQ1:
+        flat[[5, 77, 300]] = [243, 255, 250]
+    else:
+        flat[[5, 77, 300]] = [0xFF, 0x03, 0xC0]
+    want, bad = oracle.unpack(fmt, packed, N, K)
+    assert bad > 0
+    t = torch.empty((N, K), dtype=torch.int8, device="cuda")
+    bz.bonsai_unpack(fmt, torch.from_numpy(packed).cuda(), t, N, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(t.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+def test_pack_marks_invalid_trits(bz, fmt):
+    import torch
+    t = np.zeros((2, 256), dtype=np.int8)
+    t[1, 77] = 3
+    t[0, 200] = -2
+    got = bz.pack(fmt, torch.from_numpy(t).cuda()).cpu().numpy()
+    assert np.array_equal(got.reshape(-1), oracle.pack(fmt, t).reshape(-1))
+    assert oracle.check(fmt, got, 2, 256) == 2
+
+
+# ------------------------------------------------------------ Hadamard
+
+@pytest.mark.parametrize("M,K", [(1, 128), (3, 1024), (17, 5120), (2, 17408)])
+def test_hadamard128(bz, M, K):
+    import torch
+    p = Problem(M, 1, K, PQ2, seed=M)
+    x, _, _ = p.device()
+    out = torch.empty_like(x)
+    bz.bonsai_hadamard128(x, out, M, K)
+    torch.cuda.synchronize()
+    got = to_numpy_f16(out)
+    ref = oracle.hadamard128(p.x.astype(np.float64))
+    ok, rel, mx = oracle.compare(got, ref)
+    assert ok, (rel, mx)
+    # FP32 butterflies then one rounding: within one FP16 ulp of the exact value
+    ref16 = ref.astype(np.float16).astype(np.float64)
+    ulp = np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64)
+    assert np.all(np.abs(got - ref16) <= ulp)
+    assert np.mean(got == ref16) > 0.99
+    # in place gives the same bits
+    bz.bonsai_hadamard128(x, x, M, K)
+    torch.cuda.synchronize()
+    assert torch.equal(x, out)
+
+
+# ------------------------------------------------------------ linear
+
+def _run(bz, p, algo, split_k=0):
+    import torch
+    x, packed, scales = p.device()
+    y = torch.full((p.M, p.N), float("nan"), dtype=torch.float16, device="cuda")
+    bz.bonsai_ternary_linear_algo(x, packed, scales, y, p.M, p.N, p.K, p.fmt, algo, split_k)
+    torch.cuda.synchronize()
+    return to_numpy_f16(y)
+
+
+SIMPLE_CASES = [(1, 1, 128), (1, 33, 384), (3, 100, 1024), (17, 65, 640), (1, 1024, 1024)]
+
+
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("M,N,K", SIMPLE_CASES)
+def test_linear_simple(bz, fmt, M, N, K):
+    p = Problem(M, N, K, fmt, seed=M * 7 + N)
+    got = _run(bz, p, bz.BONSAI_ALGO_SIMPLE)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+def test_linear_auto_config1(bz, fmt):
+    """Single ternary linear, M=1, K=1024 -> N=1024, seed 0, through the default entry point."""
+    import torch
+    p = Problem(1, 1024, 1024, fmt, seed=0)
+    x, packed, scales = p.device()
+    y = torch.empty((1, 1024), dtype=torch.float16, device="cuda")
+    bz.bonsai_ternary_linear(x, packed, scales, y, 1, 1024, 1024, fmt)
+    torch.cuda.synchronize()
+    got = to_numpy_f16(y)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+    # negative: the same output is far from the product without the rotation
+    bad_ok, bad_rel, _ = oracle.compare(got, p.oracle_y(apply_hadamard=False))
+    assert not bad_ok and bad_rel > 0.5
+
+
+def test_argument_errors_on_device(bz):
+    import torch
+    x = torch.zeros((1, 256), dtype=torch.float16, device="cuda")
+    y = torch.zeros((1, 16), dtype=torch.float16, device="cuda")
+    s = torch.zeros((16, 2), dtype=torch.float16, device="cuda")
+    w = torch.zeros((16, 64), dtype=torch.uint8, device="cuda")
+    L = bz.raw()
+    stream = torch.cuda.current_stream().cuda_stream
+    assert L.bonsai_ternary_linear(x.data_ptr() + 2, w.data_ptr(), s.data_ptr(), y.data_ptr(), 1,
+                                   16, 256, 2, stream) == bz.BONSAI_ERR_ALIGN
+    assert L.bonsai_ternary_linear_algo(x.data_ptr(), w.data_ptr(), s.data_ptr(), y.data_ptr(), 2,
+                                        16, 256, 2, bz.BONSAI_ALGO_GEMV, 0, stream) in (
+        bz.BONSAI_ERR_ALGO,)
