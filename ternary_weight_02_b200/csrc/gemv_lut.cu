@@ -15,22 +15,29 @@
 //   it covers: PQ2_0 byte (4 two-bit codes) -> sum_i (c_i - 1) x'_i over 4
 //   activations; PTQ1_0 byte (base-3 number, 5 digits) -> sum_i (d_i - 1) x'_i over 5
 //   (3 in the last byte of a group).  One byte costs a byte permute (which forms the
-//   shared-memory offset), one shared load and half a paired FP32 add.
-// * K is cut into 512-wide slices (4 scale groups).  A CTA rotates its slice of x with
-//   the warp FWHT (FP32, in registers), builds the slice's tables (128 tables x 256
-//   FP32 entries = 128 KB), then its 16 warps stream rows of the slice.
+//   absolute shared-memory address) and one shared load, plus the FP32 adds.
+// * K is cut into 512-wide slices (4 scale groups); one slice's tables are 128 tables
+//   x 256 FP32 entries = 128 KB of shared memory.
 // * Bank-conflict-free lookups: lane l of every warp reads only tables stored in bank
 //   l, so the 32 random lookups of one instruction hit 32 different banks.  Lane l
 //   owns bytes 4l..4l+3 of a 128-byte PQ2_0 row slice (one 32-bit load per lane); for
 //   PTQ1_0 the 8 lanes of a scale group load 7 aligned words covering the group's 26
 //   bytes (the 2 bytes of a neighbouring group and the 8th lane map to all-zero
-//   tables), so each group is again exactly 8 lanes.
-// * Reduction: a warp handles 32 rows; lane L keeps row (i XOR L) in register i, which
-//   makes the 32-row transpose-reduction select-free (31 shuffles per lane).  Scales
-//   are applied after the 8 lanes of a group are summed (4 multiplies per lane).
-// * Split-K: each (slice, 32-row block) task writes an FP32 partial; the warp that
-//   finishes a row block last (arrival counter in the workspace) sums the partials in
-//   slice order (deterministic), writes FP16 y and resets the counter.
+//   "phantom" tables), so each group is again exactly 8 lanes.
+// * A warp task is 16 rows of one slice, loaded in natural order (each 32-bit load
+//   instruction reads one row's contiguous slice segment), with further tasks' words
+//   and scales in flight.  A transpose-reduction over the 8 lanes of a scale group is
+//   followed by the scale multiply and two more shuffle stages.
+// * Two schedules:
+//   - rows mode (large N): a CTA owns a range of rows, rotates all of x once, and walks
+//     the K slices, rebuilding the tables per slice and keeping each row's sum in
+//     registers.  No split-K and no tail.
+//   - split mode (small N): a CTA owns one slice and a range of rows and writes FP32
+//     partials; the warp that brings a row block's last slice (arrival counter in the
+//     workspace) sums the partials in slice order (deterministic) and writes y.
+// * Programmatic dependent launch: a kernel lets the next kernel on the stream start
+//   at once; the next kernel prefetches its own weights and then waits for this one to
+//   finish before it reads x, the workspace or y.
 #include "common.cuh"
 #include "internal.h"
 
@@ -39,12 +46,23 @@ namespace {
 
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kSliceK = 512;     // activations per K slice
-constexpr int kRows = 32;        // rows per warp task
-constexpr int kTableRegion = 65536;  // 256 entries x 256 bytes (64 banks-words per entry)
-constexpr int kTableBytes = 2 * kTableRegion;
-constexpr int kMiscBytes = 4096;     // x' of the slice (2 KB) + padding
-constexpr int kSmemBytes = kMiscBytes + kTableBytes;
+constexpr int kSliceK = 512;         // activations per K slice
+constexpr int kRows = 16;            // rows per warp task
+constexpr int kTableRegion = 65536;  // 256 entries x 256 bytes
+// Shared-memory layout.  The tables live at shared-window addresses [0x10000, 0x30000)
+// so that a byte permute alone forms a lookup's absolute address (byte 2 = 1 + region,
+// byte 1 = the weight byte, byte 0 = lane slot).  The dynamic allocation starts at a
+// small window address b (after the per-block reserved area) and spans 0x30000 bytes,
+// which covers the table range for any b <= 0x10000 - kMiscBytes; x' (FP32) lives at
+// its start: one slice in split mode, all of K in rows mode.
+constexpr uint32_t kTableAddr = 0x10000u;
+constexpr int kMiscBytes = 0x10000 - 2048;  // room for x' below the tables
+constexpr int kSmemBytes = 0x30000;
+constexpr int kRowsModeMaxK = 12288;        // x' of all K must fit below the tables
+constexpr int kMaxTasksPerWarp = 32;        // split mode: row blocks per warp (host-checked)
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 template <int kFmt>
 struct Fmt;
@@ -53,7 +71,7 @@ template <>
 struct Fmt<2> {  // PQ2_0
     static constexpr int kSliceBytes = 128;
     __device__ static int64_t row_bytes(int64_t K) { return K / 4; }
-    // byte offset of lane's word inside the slice-row, or -1 if the lane loads nothing
+    // byte offset of the lane's word inside a row's slice segment
     __device__ static int lane_offset(int lane) { return 4 * lane; }
 };
 
@@ -61,15 +79,15 @@ template <>
 struct Fmt<1> {  // PTQ1_0
     static constexpr int kSliceBytes = 4 * kPtq1GroupBytes;  // 104
     __device__ static int64_t row_bytes(int64_t K) { return (K / kGroup) * kPtq1GroupBytes; }
+    // the 8th lane of a group reads a valid word too; its tables are all zero
     __device__ static int lane_offset(int lane) {
         const int g = lane >> 3, k = lane & 7;
-        if (k == 7) return -1;
-        return kPtq1GroupBytes * g - 2 * (g & 1) + 4 * k;  // 4-byte aligned
+        return kPtq1GroupBytes * g - 2 * (g & 1) + 4 * (k == 7 ? 0 : k);  // 4-byte aligned
     }
 };
 
 // PTQ1_0: position (inside its group) of byte slot j of lane, or -1 for a slot that
-// belongs to a neighbouring group / an idle lane.
+// belongs to a neighbouring group / an idle lane (a phantom slot).
 __device__ __forceinline__ int ptq1_slot_pos(int lane, int j) {
     const int g = lane >> 3, k = lane & 7;
     if (k == 7) return -1;
@@ -83,186 +101,386 @@ __device__ __forceinline__ uint32_t table_offset(int lane, int j, int e) {
     return (uint32_t)((j >> 1) * kTableRegion + e * 256 + (j & 1) * 128 + lane * 4);
 }
 
-// Builds the slice's tables from x' (FP32 in shared memory).  Thread t: lane (bank)
-// t & 31, slot j = (t >> 5) & 3, top digit q = t >> 7 (threads with q == 3 idle).
+__device__ __forceinline__ float signed_term(int digit, float xv) {
+    return digit == 0 ? -xv : (digit == 1 ? 0.f : xv);
+}
+
+// Builds one slice's tables from its x' (FP32 in shared memory).  Thread t serves table
+// (lane = t & 31, slot j = (t >> 5) & 3) and, of that table's 3^(n-2) settings of its
+// high digits, those congruent to t >> 7 (mod 4); each setting is 9 entries.
 template <int kFmt>
 __device__ __forceinline__ void build_tables(const float *xr, uint8_t *tables, int t) {
     const int lane = t & 31, j = (t >> 5) & 3, q = t >> 7;
-    if (q > 2) return;
+    const float *xa;
+    int n, place;  // trits in the chunk, place value of one digit (4: 2-bit slots, 3: base 3)
     if (kFmt == 2) {
-        const int c = 4 * lane + j;  // chunk: activations 4c .. 4c+3 of the slice
-        const float x0 = xr[4 * c], x1 = xr[4 * c + 1], x2 = xr[4 * c + 2], x3 = xr[4 * c + 3];
-        const float base3 = q == 0 ? -x3 : (q == 1 ? 0.f : x3);
-#pragma unroll
-        for (int c2 = 0; c2 < 3; c2++) {
-            const float b2 = base3 + (c2 == 0 ? -x2 : (c2 == 1 ? 0.f : x2));
-#pragma unroll
-            for (int c1 = 0; c1 < 3; c1++) {
-                const float b1 = b2 + (c1 == 0 ? -x1 : (c1 == 1 ? 0.f : x1));
-#pragma unroll
-                for (int c0 = 0; c0 < 3; c0++) {
-                    const float v = b1 + (c0 == 0 ? -x0 : (c0 == 1 ? 0.f : x0));
-                    const int e = c0 | (c1 << 2) | (c2 << 4) | (q << 6);
-                    *reinterpret_cast<float *>(tables + table_offset(lane, j, e)) = v;
-                }
-            }
-        }
+        xa = xr + 4 * (4 * lane + j);  // chunk 4*lane + j covers activations 4c .. 4c+3
+        n = 4;
+        place = 4;
     } else {
         const int p = ptq1_slot_pos(lane, j);
-        if (p < 0) return;
-        const int g = lane >> 3;
-        const float *xa = xr + kGroup * g + 5 * p;
-        if (p == kPtq1GroupBytes - 1) {  // last byte of a group: three trits, digits 3,4 zero
-            if (q != 0) return;
-            const float x0 = xa[0], x1 = xa[1], x2 = xa[2];
+        if (p < 0) return;  // phantom slot: its table stays zero
+        xa = xr + kGroup * (lane >> 3) + 5 * p;
+        n = p == kPtq1GroupBytes - 1 ? 3 : 5;
+        place = 3;
+    }
+    int combos = 1;
+    for (int i = 2; i < n; i++) combos *= 3;
+    float xs[5];
+    if (kFmt == 2) {
+        const float4 q4 = *reinterpret_cast<const float4 *>(xa);
+        xs[0] = q4.x, xs[1] = q4.y, xs[2] = q4.z, xs[3] = q4.w, xs[4] = 0.f;
+    } else {
 #pragma unroll
-            for (int d2 = 0; d2 < 3; d2++) {
-                const float b2 = d2 == 0 ? -x2 : (d2 == 1 ? 0.f : x2);
+        for (int i = 0; i < 5; i++) xs[i] = i < n ? xa[i] : 0.f;
+    }
+    const float x0 = xs[0], x1 = xs[1];
+    for (int c = q; c < combos; c += kThreads / 128) {
+        float base = 0.f;
+        int e = 0, rest = c, pw = place * place;
 #pragma unroll
-                for (int d1 = 0; d1 < 3; d1++) {
-                    const float b1 = b2 + (d1 == 0 ? -x1 : (d1 == 1 ? 0.f : x1));
-#pragma unroll
-                    for (int d0 = 0; d0 < 3; d0++) {
-                        const float v = b1 + (d0 == 0 ? -x0 : (d0 == 1 ? 0.f : x0));
-                        *reinterpret_cast<float *>(tables + table_offset(lane, j, d0 + 3 * d1 + 9 * d2)) = v;
-                    }
-                }
+        for (int i = 2; i < 5; i++) {
+            if (i < n) {
+                const int d = rest % 3;
+                rest /= 3;
+                base += signed_term(d, xs[i]);
+                e += d * pw;
+                pw *= place;
             }
-            return;
         }
-        const float x0 = xa[0], x1 = xa[1], x2 = xa[2], x3 = xa[3], x4 = xa[4];
-        const float base4 = q == 0 ? -x4 : (q == 1 ? 0.f : x4);
 #pragma unroll
-        for (int d3 = 0; d3 < 3; d3++) {
-            const float b3 = base4 + (d3 == 0 ? -x3 : (d3 == 1 ? 0.f : x3));
+        for (int d1 = 0; d1 < 3; d1++) {
+            const float b1 = base + signed_term(d1, x1);
 #pragma unroll
-            for (int d2 = 0; d2 < 3; d2++) {
-                const float b2 = b3 + (d2 == 0 ? -x2 : (d2 == 1 ? 0.f : x2));
-#pragma unroll
-                for (int d1 = 0; d1 < 3; d1++) {
-                    const float b1 = b2 + (d1 == 0 ? -x1 : (d1 == 1 ? 0.f : x1));
-#pragma unroll
-                    for (int d0 = 0; d0 < 3; d0++) {
-                        const float v = b1 + (d0 == 0 ? -x0 : (d0 == 1 ? 0.f : x0));
-                        const int e = d0 + 3 * d1 + 9 * d2 + 27 * d3 + 81 * q;
-                        *reinterpret_cast<float *>(tables + table_offset(lane, j, e)) = v;
-                    }
-                }
-            }
+            for (int d0 = 0; d0 < 3; d0++)
+                *reinterpret_cast<float *>(tables + table_offset(lane, j, e + d1 * place + d0)) =
+                    b1 + signed_term(d0, x0);
         }
     }
 }
 
+// PTQ1_0 phantom tables (idle 8th lane of each group, slots that belong to a
+// neighbouring group) must read as zero for any byte.  Each lane clears its own
+// phantom tables, so every store instruction hits 32 different banks.  PQ2_0 needs
+// nothing: a valid byte never reaches an unwritten entry.
 template <int kFmt>
-__global__ void __launch_bounds__(kThreads, 1) gemv_lut_kernel(
+__device__ __forceinline__ void zero_phantom_tables(uint8_t *tables, int lane, int warp) {
+    if (kFmt != 1) return;
+    for (int e = warp; e < 256; e += kWarps)
+#pragma unroll
+        for (int j = 0; j < 4; j++)
+            if (ptq1_slot_pos(lane, j) < 0) *reinterpret_cast<float *>(tables + table_offset(lane, j, e)) = 0.f;
+}
+
+// Loads one warp task: register i <- the lane's word of row n0 + i (each load
+// instruction reads one row's contiguous slice segment), and the two scales the lane
+// applies after the group reduction: rows (lane & 7) + 8m of group lane >> 3.
+template <int kFmt>
+__device__ __forceinline__ void load_task(uint32_t (&w)[kRows], float (&sc)[2], const uint8_t *slice_base,
+                                          const uint16_t *scales, int64_t n0, int64_t N, int64_t G,
+                                          int64_t gcol, uint32_t row_bytes, int lane_off, int lane) {
+    const uint8_t *p = slice_base + n0 * row_bytes + lane_off;
+    const uint16_t *sp = scales + (n0 + (lane & 7)) * G + gcol;
+    if (N - n0 >= kRows) {  // full task: no predicates
+#pragma unroll
+        for (int i = 0; i < kRows; i++)
+            w[i] = __ldcs(reinterpret_cast<const unsigned int *>(p + (size_t)i * row_bytes));
+        sc[0] = half_bits_to_float(__ldg(sp));
+        sc[1] = half_bits_to_float(__ldg(sp + 8 * G));
+        return;
+    }
+    const int nvalid = (int)(N - n0);
+#pragma unroll
+    for (int i = 0; i < kRows; i++)
+        w[i] = i < nvalid ? __ldcs(reinterpret_cast<const unsigned int *>(p + (size_t)i * row_bytes)) : 0u;
+    sc[0] = (lane & 7) < nvalid ? half_bits_to_float(__ldg(sp)) : 0.f;
+    sc[1] = (lane & 7) + 8 < nvalid ? half_bits_to_float(__ldg(sp + 8 * G)) : 0.f;
+}
+
+__device__ __forceinline__ float lds_abs(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+    return v;
+}
+
+// One stage of the transpose-reduction over lane bit b: of each register pair
+// (2m, 2m+1) -- the same rows except row bit b -- the lane keeps the one whose row
+// bit b equals its lane bit b and adds the partner lane's copy of that row.
+template <int kHalf>
+__device__ __forceinline__ void transpose_stage(float (&v)[kRows], int lane, int b) {
+    const bool hi = (lane >> b) & 1;
+#pragma unroll
+    for (int m = 0; m < kHalf; m++) {
+        const float keep = hi ? v[2 * m + 1] : v[2 * m];
+        const float send = hi ? v[2 * m] : v[2 * m + 1];
+        v[m] = keep + __shfl_xor_sync(0xffffffffu, send, 1 << b);
+    }
+}
+
+// Lookups of one task and the reduction over the 8 lanes of each scale group:
+// returns, scaled, rows (lane & 7) + 8m (m = 0, 1) of this lane's group.
+__device__ __forceinline__ float2 task_group_sums(const uint32_t (&w)[kRows], const float (&sc)[2],
+                                                  const uint32_t (&pbase)[4], int lane) {
+    float v[kRows];
+#pragma unroll
+    for (int i = 0; i < kRows; i++) {
+        const float t0 = lds_abs(__byte_perm(w[i], pbase[0], 0x7604));
+        const float t1 = lds_abs(__byte_perm(w[i], pbase[1], 0x7614));
+        const float t2 = lds_abs(__byte_perm(w[i], pbase[2], 0x7624));
+        const float t3 = lds_abs(__byte_perm(w[i], pbase[3], 0x7634));
+        v[i] = (t0 + t1) + (t2 + t3);
+    }
+    transpose_stage<8>(v, lane, 0);
+    transpose_stage<4>(v, lane, 1);
+    transpose_stage<2>(v, lane, 2);
+    return make_float2(v[0] * sc[0], v[1] * sc[1]);
+}
+
+// Sum of the four groups: lanes L and L + 16 end with row L & 15 of the task.
+__device__ __forceinline__ float groups_total(float2 g, int lane) {
+    const bool hi = (lane >> 3) & 1;
+    const float keep = hi ? g.y : g.x;
+    const float send = hi ? g.x : g.y;
+    const float r = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    return r + __shfl_xor_sync(0xffffffffu, r, 16);
+}
+
+__device__ __forceinline__ void make_pbase(uint32_t (&pbase)[4], int lane) {
+    // byte 0 = (j & 1) * 128 + 4 * lane, byte 2 = 1 + region (absolute address 0x10000 + ...)
+#pragma unroll
+    for (int j = 0; j < 4; j++)
+        pbase[j] = (kTableAddr + ((uint32_t)(j >> 1) << 16)) | ((uint32_t)(j & 1) << 7) | ((uint32_t)lane << 2);
+}
+
+// ---------------------------------------------------------------- split mode
+
+template <int kFmt>
+__global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
     const uint16_t *__restrict__ x, const uint8_t *__restrict__ packed,
     const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
-    unsigned int *__restrict__ counters, int64_t N, int64_t K) {
+    unsigned int *__restrict__ counters, int64_t N, int64_t K, int parts) {
     extern __shared__ __align__(16) uint8_t smem[];
     float *xr = reinterpret_cast<float *>(smem);
-    uint8_t *tables = smem + kMiscBytes;
+    const uint32_t smem_addr = (uint32_t)__cvta_generic_to_shared(smem);
+    if (smem_addr + kMiscBytes > kTableAddr) return;  // layout assumption violated (host checks it)
+    uint8_t *tables = smem + (kTableAddr - smem_addr);
+    pdl_launch_dependents();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t G = K / kGroup;
     const int S = (int)(K / kSliceK);
     const int64_t RB = (N + kRows - 1) / kRows;
-    const int64_t T = (int64_t)S * RB;
-    const int64_t t_begin = T * blockIdx.x / gridDim.x;
-    const int64_t t_end = T * (blockIdx.x + 1) / gridDim.x;
-    const int64_t row_bytes = Fmt<kFmt>::row_bytes(K);
+    // CTA = (slice, part): the row blocks of one part of the rows, for one K slice
+    const int slice = blockIdx.x / parts, part = blockIdx.x - slice * parts;
+    const int64_t rb_begin = RB * part / parts, rb_end = RB * (part + 1) / parts;
+    const uint32_t row_bytes = (uint32_t)Fmt<kFmt>::row_bytes(K);
     const int lane_off = Fmt<kFmt>::lane_offset(lane);
+    const uint8_t *slice_base = packed + (int64_t)slice * Fmt<kFmt>::kSliceBytes;
+    const int64_t gcol = (int64_t)slice * (kSliceK / kGroup) + (lane >> 3);
 
-    // zero every table once: entries that no valid byte can reach, and the tables of
-    // PTQ1_0 padding slots, then stay zero for the whole launch
-    for (int i = tid; i < kTableBytes / 16; i += kThreads)
-        reinterpret_cast<uint4 *>(tables)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // weights are not written by earlier kernels of this library: prefetch before the wait
+    int64_t rb = rb_begin + warp;
+    uint32_t wa[kRows], wb[kRows], wc[kRows];
+    float sa[2], sb[2], sc2[2];
+    if (rb < rb_end) load_task<kFmt>(wa, sa, slice_base, scales, rb * kRows, N, G, gcol, row_bytes, lane_off, lane);
+    if (rb + kWarps < rb_end)
+        load_task<kFmt>(wb, sb, slice_base, scales, (rb + kWarps) * kRows, N, G, gcol, row_bytes, lane_off, lane);
+    zero_phantom_tables<kFmt>(tables, lane, warp);
 
-    // per-lane byte-permute operands: byte 0 = (j & 1) * 128 + 4 * lane, byte 2 = region
-    uint32_t pbase[4];
-#pragma unroll
-    for (int j = 0; j < 4; j++) pbase[j] = ((uint32_t)(j >> 1) << 16) | ((uint32_t)(j & 1) << 7) | ((uint32_t)lane << 2);
-
-    for (int64_t seg = t_begin; seg < t_end;) {
-        const int slice = (int)(seg / RB);
-        const int64_t seg_end = ((int64_t)slice + 1) * RB < t_end ? ((int64_t)slice + 1) * RB : t_end;
-        __syncthreads();  // previous slice's lookups are done (and the zeroing above)
-        if (warp >= 12) {  // rotate the slice of x: 4 blocks of 128
-            const int b = warp - 12;
-            float v[4];
-            load_half4(x + (int64_t)slice * kSliceK + b * kGroup + 4 * lane, v);
-            fwht128_warp(v, lane);
-            *reinterpret_cast<float4 *>(xr + b * kGroup + 4 * lane) = make_float4(v[0], v[1], v[2], v[3]);
-        }
-        __syncthreads();
-        build_tables<kFmt>(xr, tables, tid);
-        __syncthreads();
-
-        const uint8_t *slice_base = packed + (int64_t)slice * Fmt<kFmt>::kSliceBytes;
-        for (int64_t task = seg + warp; task < seg_end; task += kWarps) {
-            const int64_t rb = task - (int64_t)slice * RB;
-            const int64_t n0 = rb * kRows;
-            const int nvalid = (int)(N - n0 < kRows ? N - n0 : kRows);
-            const uint8_t *lane_base = slice_base + n0 * row_bytes + lane_off;
-
-            uint32_t w[kRows];
-#pragma unroll
-            for (int i = 0; i < kRows; i++) {
-                const int r = i ^ lane;
-                w[i] = 0u;
-                if (lane_off >= 0 && r < nvalid)
-                    w[i] = __ldcs(reinterpret_cast<const unsigned int *>(lane_base + (int64_t)r * row_bytes));
-            }
-            float v[kRows];
-#pragma unroll
-            for (int i = 0; i < kRows; i++) {
-                const float t0 = *reinterpret_cast<const float *>(tables + __byte_perm(w[i], pbase[0], 0x7604));
-                const float t1 = *reinterpret_cast<const float *>(tables + __byte_perm(w[i], pbase[1], 0x7614));
-                const float t2 = *reinterpret_cast<const float *>(tables + __byte_perm(w[i], pbase[2], 0x7624));
-                const float t3 = *reinterpret_cast<const float *>(tables + __byte_perm(w[i], pbase[3], 0x7634));
-                v[i] = (t0 + t2) + (t1 + t3);
-            }
-            // sum over the 8 lanes of each scale group (lane bits 0..2 <-> row bits 0..2)
-#pragma unroll
-            for (int b = 0; b < 3; b++) {
-#pragma unroll
-                for (int i = 0; i < kRows; i++)
-                    if ((i & ((2 << b) - 1)) == 0) v[i] += __shfl_xor_sync(0xffffffffu, v[i | (1 << b)], 1 << b);
-            }
-            // scale: register i (i in {0, 8, 16, 24}) holds row i ^ lane of group lane >> 3
-            const int64_t gcol = (int64_t)slice * (kSliceK / kGroup) + (lane >> 3);
-#pragma unroll
-            for (int i = 0; i < kRows; i += 8) {
-                const int r = i ^ lane;
-                const float sc = r < nvalid ? half_bits_to_float(__ldg(scales + (n0 + r) * G + gcol)) : 0.f;
-                v[i] *= sc;
-            }
-            // sum over the 4 groups (lane bits 3, 4 <-> row bits 3, 4)
-            v[0] += __shfl_xor_sync(0xffffffffu, v[8], 8);
-            v[16] += __shfl_xor_sync(0xffffffffu, v[24], 8);
-            v[0] += __shfl_xor_sync(0xffffffffu, v[16], 16);
-            // lane L now holds row n0 + L
-            const bool mine = lane < nvalid;
-            if (S == 1) {
-                if (mine) y[n0 + lane] = float_to_half_bits(v[0]);
-                continue;
-            }
-            if (mine) partials[(int64_t)slice * N + n0 + lane] = v[0];
-            __threadfence();
-            __syncwarp();
-            unsigned int arrived = 0;
-            if (lane == 0) arrived = atomicAdd(counters + rb, 1u);
-            arrived = __shfl_sync(0xffffffffu, arrived, 0);
-            if (arrived == (unsigned int)(S - 1)) {
-                __threadfence();
-                float acc = 0.f;
-                if (mine)
-                    for (int s = 0; s < S; s++) acc += __ldcg(partials + (int64_t)s * N + n0 + lane);
-                if (mine) y[n0 + lane] = float_to_half_bits(acc);
-                if (lane == 0) counters[rb] = 0u;
-            }
-        }
-        seg = seg_end;
+    pdl_wait();  // x, the workspace and y may belong to the previous kernel
+    if (warp < 4) {  // rotate the slice of x: 4 blocks of 128
+        float xv[4];
+        load_half4(x + (int64_t)slice * kSliceK + warp * kGroup + 4 * lane, xv);
+        fwht128_warp(xv, lane);
+        *reinterpret_cast<float4 *>(xr + warp * kGroup + 4 * lane) = make_float4(xv[0], xv[1], xv[2], xv[3]);
     }
+    __syncthreads();
+    build_tables<kFmt>(xr, tables, tid);
+    __syncthreads();
+    uint32_t pbase[4];
+    make_pbase(pbase, lane);
+
+    int ntasks = 0;
+    auto finish = [&](float2 gs, int64_t task_rb) {
+        const float total = groups_total(gs, lane);
+        const int64_t n0 = task_rb * kRows;
+        const int row = lane & 15;
+        if (lane < 16 && n0 + row < N) {
+            if (S == 1)
+                y[n0 + row] = float_to_half_bits(total);
+            else
+                partials[(int64_t)slice * N + n0 + row] = total;
+        }
+        ntasks++;
+    };
+    // three rotating task buffers: while one task is reduced, the next two are in flight
+    while (rb < rb_end) {
+        if (rb + 2 * kWarps < rb_end)
+            load_task<kFmt>(wc, sc2, slice_base, scales, (rb + 2 * kWarps) * kRows, N, G, gcol, row_bytes, lane_off, lane);
+        finish(task_group_sums(wa, sa, pbase, lane), rb);
+        rb += kWarps;
+        if (rb >= rb_end) break;
+        if (rb + 2 * kWarps < rb_end)
+            load_task<kFmt>(wa, sa, slice_base, scales, (rb + 2 * kWarps) * kRows, N, G, gcol, row_bytes, lane_off, lane);
+        finish(task_group_sums(wb, sb, pbase, lane), rb);
+        rb += kWarps;
+        if (rb >= rb_end) break;
+        if (rb + 2 * kWarps < rb_end)
+            load_task<kFmt>(wb, sb, slice_base, scales, (rb + 2 * kWarps) * kRows, N, G, gcol, row_bytes, lane_off, lane);
+        finish(task_group_sums(wc, sc2, pbase, lane), rb);
+        rb += kWarps;
+    }
+    if (S == 1 || ntasks == 0) return;
+
+    // publish this warp's partials, count arrivals (one lane per task), and finish the
+    // row blocks for which this warp brought the last slice
+    __threadfence();
+    __syncwarp();
+    const int64_t my_rb0 = rb_begin + warp;
+    bool last = false;
+    if (lane < ntasks) last = atomicAdd(counters + my_rb0 + (int64_t)lane * kWarps, 1u) == (unsigned int)(S - 1);
+    unsigned int last_mask = __ballot_sync(0xffffffffu, last);
+    if (last_mask == 0u) return;
+    __threadfence();
+    const int half = lane >> 4, row = lane & 15;
+    const int s_lo = half ? S / 2 : 0, s_hi = half ? S : S / 2;
+    while (last_mask) {
+        const int k = __ffs(last_mask) - 1;
+        last_mask &= last_mask - 1;
+        const int64_t rbk = my_rb0 + (int64_t)k * kWarps;
+        const int64_t n0 = rbk * kRows;
+        float acc = 0.f;
+        if (n0 + row < N) {
+            const float *pp = partials + n0 + row;
+            for (int s0 = s_lo; s0 < s_hi; s0 += 8) {
+                float tmp[8];
+#pragma unroll
+                for (int u = 0; u < 8; u++) tmp[u] = s0 + u < s_hi ? __ldcg(pp + (int64_t)(s0 + u) * N) : 0.f;
+#pragma unroll
+                for (int u = 0; u < 8; u++) acc += tmp[u];
+            }
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 16);
+        if (lane < 16 && n0 + row < N) y[n0 + row] = float_to_half_bits(acc);
+        if (lane == 0) counters[rbk] = 0u;
+    }
+}
+
+// ---------------------------------------------------------------- rows mode
+
+// A CTA owns row blocks [rb_begin, rb_end); in rounds of kWarps blocks (one per warp)
+// it walks all K slices.  Each warp keeps the scaled group sums of its block in two
+// registers across slices and reduces over the groups once at the end.
+template <int kFmt>
+__global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(
+    const uint16_t *__restrict__ x, const uint8_t *__restrict__ packed,
+    const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, int64_t N, int64_t K) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    float *xr = reinterpret_cast<float *>(smem);  // x' of all K (K <= kRowsModeMaxK)
+    const uint32_t smem_addr = (uint32_t)__cvta_generic_to_shared(smem);
+    if (smem_addr + kMiscBytes > kTableAddr) return;  // layout assumption violated (host checks it)
+    uint8_t *tables = smem + (kTableAddr - smem_addr);
+    pdl_launch_dependents();
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t G = K / kGroup;
+    const int S = (int)(K / kSliceK);
+    const int64_t RB = (N + kRows - 1) / kRows;
+    const int64_t rb_begin = RB * blockIdx.x / gridDim.x, rb_end = RB * (blockIdx.x + 1) / gridDim.x;
+    const uint32_t row_bytes = (uint32_t)Fmt<kFmt>::row_bytes(K);
+    const int lane_off = Fmt<kFmt>::lane_offset(lane);
+    uint32_t pbase[4];
+    make_pbase(pbase, lane);
+
+    bool first = true;
+    for (int64_t round = rb_begin; round < rb_end; round += kWarps) {
+        const int64_t rb = round + warp;
+        const bool active = rb < rb_end;
+        // four slice buffers: slice s uses buffer s % 4, slices s+1 .. s+3 are in flight
+        uint32_t wq[4][kRows];
+        float sq[4][2];
+        auto fetch = [&](int sl, uint32_t (&wt)[kRows], float (&st)[2]) {
+            if (active && sl < S)
+                load_task<kFmt>(wt, st, packed + (int64_t)sl * Fmt<kFmt>::kSliceBytes, scales, rb * kRows, N, G,
+                                (int64_t)sl * (kSliceK / kGroup) + (lane >> 3), row_bytes, lane_off, lane);
+        };
+        fetch(0, wq[0], sq[0]);
+        fetch(1, wq[1], sq[1]);
+        fetch(2, wq[2], sq[2]);
+        if (first) {
+            zero_phantom_tables<kFmt>(tables, lane, warp);
+            pdl_wait();  // x and y may belong to the previous kernel
+            for (int64_t b = warp; b < G; b += kWarps) {  // rotate all of x once
+                float xv[4];
+                load_half4(x + b * kGroup + 4 * lane, xv);
+                fwht128_warp(xv, lane);
+                *reinterpret_cast<float4 *>(xr + b * kGroup + 4 * lane) = make_float4(xv[0], xv[1], xv[2], xv[3]);
+            }
+            first = false;
+        }
+        float2 acc = make_float2(0.f, 0.f);
+        for (int s = 0; s < S; s += 4) {
+#pragma unroll
+            for (int h = 0; h < 4; h++) {
+                if (s + h < S) {
+                    fetch(s + h + 3, wq[(h + 3) & 3], sq[(h + 3) & 3]);
+                    __syncthreads();  // the previous slice's lookups are done (and x' is written)
+                    build_tables<kFmt>(xr + (int64_t)(s + h) * kSliceK, tables, tid);
+                    __syncthreads();
+                    if (active) {
+                        const float2 gs = task_group_sums(wq[h], sq[h], pbase, lane);
+                        acc.x += gs.x;
+                        acc.y += gs.y;
+                    }
+                }
+            }
+        }
+        const float total = groups_total(acc, lane);
+        const int64_t n0 = rb * kRows;
+        const int row = lane & 15;
+        if (active && lane < 16 && n0 + row < N) y[n0 + row] = float_to_half_bits(total);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+// Rows mode when every CTA gets enough row blocks to keep most warps busy per slice.
+// (PTQ1_0 tables cost ~3x more to build per slice, so PTQ1_0 always splits K.)
+bool use_rows_mode(int64_t N, int64_t K, int fmt, const DeviceInfo &dev) {
+    if (fmt != 2 || K > kRowsModeMaxK || K / kSliceK < 2) return false;
+    const int64_t RB = (N + kRows - 1) / kRows;
+    return RB >= (int64_t)dev.sm_count * 12;
+}
+
+// Split mode: rows of the weight matrix are split into `parts` ranges per K slice so that
+// the grid (slices x parts) fills the SMs once.
+int gemv_parts(int64_t N, int64_t K, const DeviceInfo &dev) {
+    const int64_t S = K / kSliceK;
+    const int64_t RB = (N + kRows - 1) / kRows;
+    int64_t parts = dev.sm_count / S;
+    if (parts < 1) parts = 1;
+    // every warp of a CTA handles at most kMaxTasksPerWarp row blocks
+    const int64_t min_parts = (RB + (int64_t)kWarps * kMaxTasksPerWarp - 1) / ((int64_t)kWarps * kMaxTasksPerWarp);
+    if (parts < min_parts) parts = min_parts;
+    if (parts > RB) parts = RB;
+    return (int)parts;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args... args) {
+    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 }  // namespace
@@ -275,31 +493,35 @@ bool gemv_supported(int64_t M, int64_t N, int64_t K, int fmt) {
 }
 
 size_t gemv_workspace_bytes(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev) {
-    (void)fmt;
     (void)split_k;
-    (void)dev;
     const int64_t S = K / kSliceK;
-    return S > 1 ? (size_t)S * (size_t)N * sizeof(float) : 0;
+    if (S <= 1 || use_rows_mode(N, K, fmt, dev)) return 0;
+    return (size_t)S * (size_t)N * sizeof(float);
 }
 
 cudaError_t launch_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                         uint16_t *y, int64_t N, int64_t K, int fmt, int split_k,
                         const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
-    (void)split_k;  // the K split is fixed by the 512-wide table slice
-    const int64_t tasks = (K / kSliceK) * ((N + kRows - 1) / kRows);
-    const int grid = (int)(tasks < dev.sm_count ? tasks : dev.sm_count);
-    float *partials = reinterpret_cast<float *>(ws.data);
-    cudaError_t err;
-    if (fmt == 1) {
-        err = cudaFuncSetAttribute(gemv_lut_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (err != cudaSuccess) return err;
-        gemv_lut_kernel<1><<<grid, kThreads, kSmemBytes, s>>>(x, packed, scales, y, partials, ws.counters, N, K);
-    } else {
-        err = cudaFuncSetAttribute(gemv_lut_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (err != cudaSuccess) return err;
-        gemv_lut_kernel<2><<<grid, kThreads, kSmemBytes, s>>>(x, packed, scales, y, partials, ws.counters, N, K);
+    (void)split_k;  // the schedule is chosen from the shape
+    // the dynamic allocation must start below kTableAddr - kMiscBytes in the shared
+    // window; it starts right after the per-block reserved area (no static shared memory)
+    static int reserved = -1;
+    if (reserved < 0 && cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, 0) != cudaSuccess)
+        return cudaErrorUnknown;
+    if (reserved + kMiscBytes > (int)kTableAddr) return cudaErrorNotSupported;
+    if (use_rows_mode(N, K, fmt, dev)) {
+        const int64_t RB = (N + kRows - 1) / kRows;
+        const int grid = (int)(RB < dev.sm_count ? RB : dev.sm_count);
+        if (fmt == 1) return launch_pdl(gemv_rows_kernel<1>, grid, s, x, packed, scales, y, N, K);
+        return launch_pdl(gemv_rows_kernel<2>, grid, s, x, packed, scales, y, N, K);
     }
-    return cudaGetLastError();
+    const int parts = gemv_parts(N, K, dev);
+    const int64_t grid = (K / kSliceK) * parts;
+    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+    float *partials = reinterpret_cast<float *>(ws.data);
+    if (fmt == 1)
+        return launch_pdl(gemv_split_kernel<1>, (int)grid, s, x, packed, scales, y, partials, ws.counters, N, K, parts);
+    return launch_pdl(gemv_split_kernel<2>, (int)grid, s, x, packed, scales, y, partials, ws.counters, N, K, parts);
 }
 
 }  // namespace bonsai
