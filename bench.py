@@ -1,0 +1,406 @@
+"""Benchmark of the ternary linear layer on B200: one JSON line on rank 0.
+
+A step is one decoded token (M = 1) through a synthetic 64-layer stack of 27B-class
+ternary projections: per layer qkv (5120 -> 7168), o (5120 -> 5120), fused gate/up
+(5120 -> 34816) and down (17408 -> 5120), every projection with its own weights
+resident in HBM (64 distinct copies per shape: 5.6 GB PQ2_0 / 4.6 GB PTQ1_0, far
+larger than the 126 MB L2, so nothing is served from cache between steps).  Each
+projection is one bonsai_ternary_linear call: fused block-Hadamard rotation of x,
+trit decode, group scales, reduction.  The 256 calls of a step are replayed from a
+CUDA graph.
+
+  value      whole-job HBM GB/s: algorithmic bytes of all ranks' steps (trit planes +
+             FP16 scales + x + y) / max-over-ranks device time.
+  roofline   the dominant kernel (the gate/up GEMV), timed live with CUDA events on
+             its stream, against the measured HBM copy bandwidth.
+  e2e        the same metric through the C ABI with pinned host buffers: every step
+             copies the step's activations host -> device and its outputs back.
+  cpu_baseline  the float64 CPU checker on a bounded sample (one layer), rank 0, N=1.
+
+Multi-GPU: one process per GPU (torchrun); each rank decodes its own token stream
+through its own copy of the stack (replicas, weak scaling, no collective on the
+data path).  `--impl reference` times the CPU checker itself on the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "batch-1 ternary GEMV HBM GB/s (% of 8 TB/s); prefill GEMM TFLOPS (% peak)"
+SHAPES = [("qkv", 5120, 7168), ("o", 5120, 5120), ("gate_up", 5120, 34816), ("down", 17408, 5120)]
+LAYERS = 64
+FMT_NAMES = {1: "PTQ1_0", 2: "PQ2_0"}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def plane_bytes(fmt, N, K):
+    trit = N * (K // 128) * 26 if fmt == 1 else N * K // 4
+    return trit + N * (K // 128) * 2
+
+
+def step_bytes(fmt):
+    """Algorithmic bytes of one token through the stack: weights + scales + x + y."""
+    per_layer = sum(plane_bytes(fmt, N, K) + 2 * K + 2 * N for _, K, N in SHAPES)
+    return LAYERS * per_layer
+
+
+class Clocks:
+    """Samples nvidia-smi during the timed region (SM clock, throttle reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def kernel_traffic(fmt):
+    """DRAM bytes per gate/up launch from the committed ncu summary, if it was taken on
+    the kernel source as it is now (matched by hash); else None."""
+    path = os.path.join(ROOT, "profiles", "gemv_traffic.json")
+    src = os.path.join(ROOT, "ternary_weight_02_b200", "csrc", "gemv_lut.cu")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    with open(src, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:16]
+    ent = d.get(FMT_NAMES[fmt])
+    if not ent or ent.get("source_sha256_16") != h:
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args):
+    """The CPU checker as it stands, timed on this host's cores: each step is one layer
+    (the four projections) of the stack at M = 1, a bounded sample of the workload."""
+    import oracle
+    from ternary_weight_02_b200 import inputs
+    fmt = {"ptq1": 1, "pq2": 2}[args.fmt]
+    probs = []
+    for i, (name, K, N) in enumerate(SHAPES):
+        t = inputs.trits(i, N, K)
+        probs.append((inputs.activations(i, 1, K), oracle.pack(fmt, t), inputs.scales(i, N, K), N, K))
+    threads = oracle.max_threads()
+
+    def one_step():
+        for x, p, s, N, K in probs:
+            oracle.ternary_linear(x, p, s, N, K, fmt)
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one_step()
+    dt = (time.perf_counter() - t0) / args.steps
+    sample_bytes = step_bytes(fmt) / LAYERS
+    value = sample_bytes / dt / 1e9
+    sample = f"one layer (qkv, o, gate/up, down at M=1, {FMT_NAMES[fmt]}) of the 64-layer stack per step"
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "impl": "reference",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"27B-class decode projections, M=1, {FMT_NAMES[fmt]}, one layer per step",
+                   "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------ our arm
+
+def build_stack(fmt, dev, bz, torch):
+    """Weights of the 64-layer stack: seeded trits/scales per shape, packed on the GPU,
+    copied into 64 distinct buffers per shape; x per shape."""
+    from ternary_weight_02_b200 import inputs
+    stack = []
+    xs, ys = [], []
+    for i, (name, K, N) in enumerate(SHAPES):
+        t = torch.from_numpy(inputs.trits(i, N, K)).to(dev)
+        packed = bz.pack(fmt, t)
+        del t
+        s = torch.from_numpy(inputs.scales(i, N, K).view(np.int16)).to(dev).view(torch.float16)
+        copies = [(packed.clone(), s.clone()) for _ in range(LAYERS)]
+        del packed, s
+        stack.append(copies)
+        xs.append(torch.from_numpy(inputs.activations(i, 1, K).view(np.int16)).to(dev).view(torch.float16))
+        ys.append(torch.empty((1, N), dtype=torch.float16, device=dev))
+    return stack, xs, ys
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from ternary_weight_02_b200 import bonsai as bz
+
+    world, rank, local = dist_setup()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if bz.bonsai_check_device() != bz.BONSAI_OK:
+        raise RuntimeError("libbonsai: not an sm_100 device")
+    peaks, peak_kind = measured_peaks()
+    fmt = {"ptq1": 1, "pq2": 2}[args.fmt]
+    bz.bonsai_reserve(1, 34816, 17408)
+
+    results = {}
+    for f in ([fmt] + [o for o in (2, 1) if o != fmt]) if args.both else [fmt]:
+        stack, xs, ys = build_stack(f, dev, bz, torch)
+        stream = torch.cuda.Stream(device=dev)
+        sp = stream.cuda_stream
+
+        def enqueue(only=None):
+            for layer in range(LAYERS):
+                for i, (name, K, N) in enumerate(SHAPES):
+                    if only is not None and i != only:
+                        continue
+                    p, s = stack[i][layer]
+                    bz.bonsai_ternary_linear(xs[i], p, s, ys[i], 1, N, K, f, sp)
+
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                enqueue()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                enqueue()
+            g_dom = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_dom, stream=stream):
+                enqueue(only=2)
+        torch.cuda.synchronize()
+
+        # ---- device-resident timing
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                g.replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        clocks = Clocks(local)
+        clocks.start()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        clk = clocks.stop()
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        value = world * step_bytes(f) / (ms * 1e-3) / 1e9
+
+        # ---- dominant kernel (gate/up GEMV), 64 launches per replay
+        with torch.cuda.stream(stream):
+            g_dom.replay()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(max(3, args.steps)):
+                g_dom.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        dom_launches = LAYERS * max(3, args.steps)
+        dom_us = e0.elapsed_time(e1) * 1e3 / dom_launches
+        _, Kd, Nd = SHAPES[2]
+        dom_bytes = plane_bytes(f, Nd, Kd) + 2 * Kd + 2 * Nd
+        dom_gbs = dom_bytes / (dom_us * 1e-6) / 1e9
+        traffic = kernel_traffic(f)
+
+        # ---- end to end through the C ABI with host buffers
+        hx = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in xs]
+        for h, x in zip(hx, xs):
+            h.copy_(x.cpu())
+        hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
+        h2d = sum(h.numel() * h.element_size() for h in hx)
+        d2h = sum(h.numel() * h.element_size() for h in hy)
+
+        def e2e_step():
+            for h, x in zip(hx, xs):
+                x.copy_(h, non_blocking=True)
+            g.replay()
+            for h, y in zip(hy, ys):
+                h.copy_(y, non_blocking=True)
+
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                e2e_step()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(args.steps):
+                e2e_step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = e0.elapsed_time(e1) / args.steps
+        if world > 1:
+            t = torch.tensor([ms_e2e], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = world * step_bytes(f) / (ms_e2e * 1e-3) / 1e9
+
+        results[f] = {
+            "value": value, "ms": ms, "clocks": clk, "dom_us": dom_us, "dom_gbs": dom_gbs,
+            "dom_bytes": dom_bytes, "traffic": traffic, "e2e": e2e, "h2d": h2d, "d2h": d2h,
+        }
+        del stack, g, g_dom
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+    r = results[fmt]
+    line = None
+    if rank == 0:
+        hbm = float(peaks["hbm_gbs"])
+        line = {
+            "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms"], 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded SplitMix64 trits P(0)=.38, FP16 scales U[.01,.05], FP16 x N(0,1))",
+            "config": {
+                "workload": (f"64-layer 27B-class linear stack at M=1 (qkv 5120->7168, o 5120->5120, "
+                             f"gate/up 5120->34816, down 17408->5120), {FMT_NAMES[fmt]}, one token per step"),
+                "packing": FMT_NAMES[fmt], "layers": LAYERS, "tokens_per_step": 1,
+                "bytes_per_step": step_bytes(fmt), "l2": "inputs larger than L2 (weights re-read every step)",
+                "per_token_us": round(r["ms"] * 1e3, 2), "frac_of_8TBps": round(r["value"] / 8000.0, 4),
+                "frac_of_measured_hbm": round(r["value"] / hbm, 4), "parallelism": f"replicas x{world}",
+            },
+            "roofline": {
+                "bound": "hbm", "kernel": "gemv gate/up 5120->34816", "achieved": round(r["dom_gbs"], 1),
+                "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(r["dom_gbs"] / hbm, 4),
+                "traffic": r["traffic"], "algorithmic_bytes_per_launch": r["dom_bytes"],
+                "avg_launch_us": round(r["dom_us"], 3),
+            },
+            "e2e": {"value": round(r["e2e"], 1), "unit": "GB/s", "h2d_bytes_per_step": r["h2d"],
+                    "d2h_bytes_per_step": r["d2h"]},
+            "gpu_launches": LAYERS * len(SHAPES) * args.steps,
+            "clocks": r["clocks"],
+        }
+        others = {FMT_NAMES[k]: {"value": round(v["value"], 1), "unit": "GB/s",
+                                 "per_token_us": round(v["ms"] * 1e3, 2),
+                                 "gate_up_gbs": round(v["dom_gbs"], 1), "e2e": round(v["e2e"], 1)}
+                  for k, v in results.items() if k != fmt}
+        if others:
+            line["other_packings"] = others
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def cpu_baseline(fmt):
+    """The checker on one layer of the stack (rank 0, N = 1): bounded CPU sample."""
+    import oracle
+    from ternary_weight_02_b200 import inputs
+    probs = []
+    for i, (name, K, N) in enumerate(SHAPES):
+        probs.append((inputs.activations(i, 1, K), oracle.pack(fmt, inputs.trits(i, N, K)),
+                      inputs.scales(i, N, K), N, K))
+    t0 = time.perf_counter()
+    for x, p, s, N, K in probs:
+        oracle.ternary_linear(x, p, s, N, K, fmt)
+    dt = time.perf_counter() - t0
+    return {"value": round(step_bytes(fmt) / LAYERS / dt / 1e9, 3), "unit": "GB/s",
+            "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"one layer (4 projections, M=1, {FMT_NAMES[fmt]}) of the 64-layer stack, float64"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--fmt", choices=["pq2", "ptq1"], default="pq2")
+    ap.add_argument("--both", type=int, default=1, help="also measure the other packing")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, _ = dist_setup()
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args)), flush=True)
+        return
+    line = run_ours(args)
+    if rank == 0 and line is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline({"ptq1": 1, "pq2": 2}[args.fmt])
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()
