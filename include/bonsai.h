@@ -75,7 +75,8 @@ typedef enum {
     BONSAI_ERR_CUDA = -5,   /* a CUDA runtime call or kernel launch failed        */
     BONSAI_ERR_ARCH = -6,   /* the current device is not compute capability 10.0  */
     BONSAI_ERR_NOMEM = -7,  /* the internal workspace could not be allocated      */
-    BONSAI_ERR_ALGO = -8    /* the requested kernel cannot run this shape         */
+    BONSAI_ERR_ALGO = -8,   /* the requested kernel cannot run this shape         */
+    BONSAI_ERR_TOO_LARGE = -9 /* beyond the fixed scratch of bonsai_ternary_linear_noalloc */
 } bonsai_status;
 
 /* Kernel selection for bonsai_ternary_linear_algo (bonsai_ternary_linear uses AUTO). */
@@ -147,6 +148,32 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
  * format and kernel) need no further allocation; call before capturing calls
  * into a CUDA graph.  Synchronises the device if it reallocates. */
 int bonsai_reserve(int64_t M, int64_t N, int64_t K);
+
+/* Batch-1 ternary linear layer that allocates nothing.
+ *
+ * Some callers cannot call cudaMalloc: code that runs while a CUDA graph is being
+ * captured, allocators that must own every byte on the device, or hosts that forbid
+ * allocation after start-up.  This entry point computes the same y as
+ * bonsai_ternary_linear for M == 1 (the split-K lookup-table GEMV) but takes its
+ * scratch -- split-K arrival counters and FP32 partial sums -- from one fixed array in
+ * device memory that is part of the library image, instead of the per-device
+ * workspace.  It never calls cudaMalloc, cudaFree or any allocating routine.  The
+ * pages this library follows describe no such variant: it exists only for these
+ * callers.
+ *
+ * Limits: M must be 1, K a multiple of 512, N <= 1048576, and (K / 512) * N <= 1048576
+ * (the array holds 65536 counters and 2^20 FP32 partials, 4.25 MiB, kept by every
+ * GPU that loads the library until the process exits); larger problems return
+ * BONSAI_ERR_TOO_LARGE and launch nothing.  Inputs and output are caller-owned
+ * device memory as for bonsai_ternary_linear.
+ *
+ * Set-up: the first call on each device looks up that device's copy of the array
+ * (with that device current); make that first call before capturing any stream.
+ * Every call shares the one array: it clears the counters it uses on `stream` before
+ * its kernel, and calls whose work overlaps on the GPU (different streams, or
+ * concurrent host threads) race on the array -- serialise them. */
+int bonsai_ternary_linear_noalloc(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                                  uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, void *stream);
 
 /* Frees the workspaces of every device (after synchronising each).  The
  * library stays usable: the next call allocates again. */

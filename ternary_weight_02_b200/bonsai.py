@@ -28,6 +28,7 @@ BONSAI_ERR_CUDA = -5
 BONSAI_ERR_ARCH = -6
 BONSAI_ERR_NOMEM = -7
 BONSAI_ERR_ALGO = -8
+BONSAI_ERR_TOO_LARGE = -9
 
 BONSAI_ALGO_AUTO = 0
 BONSAI_ALGO_SIMPLE = 1
@@ -56,6 +57,7 @@ _SIGS = {
     "bonsai_hadamard128": (_int, [_p, _p, _i64, _i64, _p]),
     "bonsai_ternary_linear": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _p]),
     "bonsai_ternary_linear_algo": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _int, _int, _p]),
+    "bonsai_ternary_linear_noalloc": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _p]),
     "bonsai_reserve": (_int, [_i64, _i64, _i64]),
     "bonsai_shutdown": (None, []),
 }
@@ -149,6 +151,13 @@ def bonsai_ternary_linear_algo(x, packed, scales, y, M: int, N: int, K: int, fmt
     _check(_lib.bonsai_ternary_linear_algo(_ptr(x), _ptr(packed), _ptr(scales), _ptr(y), M, N, K,
                                            fmt, algo, split_k, _stream(stream)),
            "bonsai_ternary_linear_algo")
+
+
+def bonsai_ternary_linear_noalloc(x, packed, scales, y, M: int, N: int, K: int, fmt: int,
+                                  stream=None) -> None:
+    """Batch-1 layer on the library's fixed device scratch: allocates nothing."""
+    _check(_lib.bonsai_ternary_linear_noalloc(_ptr(x), _ptr(packed), _ptr(scales), _ptr(y), M, N, K,
+                                              fmt, _stream(stream)), "bonsai_ternary_linear_noalloc")
 
 
 def bonsai_reserve(M: int, N: int, K: int) -> None:

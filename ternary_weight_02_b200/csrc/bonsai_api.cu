@@ -137,6 +137,16 @@ size_t workspace_for(int algo, int64_t M, int64_t N, int64_t K, int fmt, int spl
 }
 
 }  // namespace
+
+int current_device_info(DeviceInfo *out) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int dev;
+    DeviceState *st;
+    const int rc = probe_current(&dev, &st);
+    if (rc == BONSAI_OK) *out = st->info;
+    return rc;
+}
+
 }  // namespace bonsai
 
 using namespace bonsai;
@@ -156,6 +166,7 @@ const char *bonsai_status_string(int status) {
         case BONSAI_ERR_ARCH: return "current device is not an sm_100 (B200-class) GPU";
         case BONSAI_ERR_NOMEM: return "could not allocate the device workspace";
         case BONSAI_ERR_ALGO: return "the requested kernel cannot run this shape";
+        case BONSAI_ERR_TOO_LARGE: return "the problem needs more than the fixed device scratch of the no-allocation entry point";
         default: return "unknown status";
     }
 }

@@ -524,4 +524,29 @@ cudaError_t launch_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t
     return launch_pdl(gemv_split_kernel<2>, (int)grid, s, x, packed, scales, y, partials, ws.counters, N, K, parts);
 }
 
+// Split-mode launch with caller-provided scratch (counters and partials), whatever the
+// shape; used by the no-allocation entry point.  partial_floats is the space the
+// scratch holds after its counters; returns cudaErrorInvalidValue if the shape needs more.
+size_t gemv_split_partial_floats(int64_t N, int64_t K) {
+    const int64_t S = K / kSliceK;
+    return S > 1 ? (size_t)S * (size_t)N : 0;
+}
+
+cudaError_t launch_gemv_split_scratch(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                                      uint16_t *y, int64_t N, int64_t K, int fmt, unsigned int *counters,
+                                      float *partials, size_t partial_floats, cudaStream_t s,
+                                      const DeviceInfo &dev) {
+    if (gemv_split_partial_floats(N, K) > partial_floats) return cudaErrorInvalidValue;
+    static int reserved = -1;
+    if (reserved < 0 && cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, 0) != cudaSuccess)
+        return cudaErrorUnknown;
+    if (reserved + kMiscBytes > (int)kTableAddr) return cudaErrorNotSupported;
+    const int parts = gemv_parts(N, K, dev);
+    const int64_t grid = (K / kSliceK) * parts;
+    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+    if (fmt == 1)
+        return launch_pdl(gemv_split_kernel<1>, (int)grid, s, x, packed, scales, y, partials, counters, N, K, parts);
+    return launch_pdl(gemv_split_kernel<2>, (int)grid, s, x, packed, scales, y, partials, counters, N, K, parts);
+}
+
 }  // namespace bonsai

@@ -54,6 +54,15 @@ cudaError_t launch_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t
                         uint16_t *y, int64_t N, int64_t K, int fmt, int split_k,
                         const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
 
+// split-mode GEMV on caller-provided scratch (no-allocation entry point)
+size_t gemv_split_partial_floats(int64_t N, int64_t K);
+cudaError_t launch_gemv_split_scratch(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                                      uint16_t *y, int64_t N, int64_t K, int fmt, unsigned int *counters,
+                                      float *partials, size_t partial_floats, cudaStream_t s,
+                                      const DeviceInfo &dev);
+// current device's properties (the same probe the other entry points use)
+int current_device_info(DeviceInfo *out);
+
 // ---- skinny_mma.cu: 1 <= M <= 16
 bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t skinny_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int split_k,

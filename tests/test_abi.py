@@ -74,7 +74,7 @@ def test_host_validation_needs_no_gpu(bz):
 
 
 def test_status_strings(bz):
-    for code in range(-8, 1):
+    for code in range(-9, 1):
         s = bz.bonsai_status_string(code)
         assert s and s != "unknown status"
     assert bz.bonsai_status_string(-99) == "unknown status"
