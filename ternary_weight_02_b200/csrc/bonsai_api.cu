@@ -114,7 +114,7 @@ int resolve_algo(int algo, int64_t M, int64_t N, int64_t K, int fmt) {
     if (algo == BONSAI_ALGO_AUTO) {
         if (M == 1 && gemv_supported(M, N, K, fmt)) return BONSAI_ALGO_GEMV;
         if (M <= 16 && skinny_supported(M, N, K, fmt)) return BONSAI_ALGO_SKINNY;
-        if (M > 16 && gemm_supported(M, N, K, fmt)) return BONSAI_ALGO_GEMM;
+        if (gemm_supported(M, N, K, fmt)) return BONSAI_ALGO_GEMM;
         return BONSAI_ALGO_SIMPLE;
     }
     switch (algo) {

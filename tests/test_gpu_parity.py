@@ -213,3 +213,59 @@ def test_gemv_rejects_batches(bz):
     w = torch.zeros((8, 128), dtype=torch.uint8, device="cuda")
     with pytest.raises(bz.BonsaiError):
         bz.bonsai_ternary_linear_algo(x, w, s, y, 2, 8, 512, PQ2, bz.BONSAI_ALGO_GEMV)
+
+
+# ------------------------------------------------------------ prefill GEMM (tcgen05 / TMEM)
+
+GEMM_SMALL = [(1, 64, 128), (17, 256, 128), (130, 300, 384), (256, 512, 1024), (300, 1000, 640)]
+
+
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("M,N,K", GEMM_SMALL)
+def test_gemm_small(bz, fmt, M, N, K):
+    p = Problem(M, N, K, fmt, seed=M + N + K)
+    got = _run(bz, p, bz.BONSAI_ALGO_GEMM)
+    assert np.all(np.isfinite(got))
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+def _sampled_reference(fmt, M, N, K, seed, ms, ns):
+    """Checker values of y at the (m, n) pairs of ms x ns, from regenerated input rows."""
+    from ternary_weight_02_b200 import inputs
+    um, un = np.unique(ms), np.unique(ns)
+    x = inputs.normal_rows(seed, K, um)
+    t = inputs.trits_rows(seed, K, un)
+    s = inputs.scales_rows(seed, K // 128, un)
+    y = oracle.ternary_linear(x, oracle.pack(fmt, t), s, len(un), K, fmt)
+    return y, um, un
+
+
+# prefill: M tokens x 27B-class projections (K -> N)
+PREFILL = [(2048, 5120, 34816), (512, 17408, 5120), (8192, 5120, 7168)]
+
+
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("M,K,N", PREFILL)
+def test_gemm_prefill_full_size_sampled(bz, fmt, M, K, N):
+    """Full-size GEMM on the device; 64 x 64 sampled outputs against the checker."""
+    import torch
+    from ternary_weight_02_b200 import inputs
+    seed = 5
+    dev = torch.device("cuda")
+    t = torch.from_numpy(inputs.trits(seed, N, K)).to(dev)
+    packed = bz.pack(fmt, t)
+    del t
+    s = torch.from_numpy(inputs.scales(seed, N, K).view(np.int16)).to(dev).view(torch.float16)
+    x = torch.from_numpy(inputs.activations(seed, M, K).view(np.int16)).to(dev).view(torch.float16)
+    y = torch.full((M, N), float("nan"), dtype=torch.float16, device=dev)
+    bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(M + N)
+    ms = np.concatenate([[0, M - 1], rng.integers(0, M, 62)])
+    ns = np.concatenate([[0, N - 1], rng.integers(0, N, 62)])
+    ref, um, un = _sampled_reference(fmt, M, N, K, seed, ms, ns)
+    got = y[torch.from_numpy(um).to(dev)][:, torch.from_numpy(un).to(dev)].float().cpu().numpy()
+    ok, rel, mx = oracle.compare(got, ref)
+    assert ok, (rel, mx)
+    assert bool(torch.isfinite(y).all())
