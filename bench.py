@@ -320,6 +320,9 @@ def run_ours(args):
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
 
+    prefill = run_prefill(fmt, args.prefill_m, dev, bz, torch, peaks, peak_kind, max(3, args.steps // 20)) \
+        if args.prefill_m > 0 else None
+
     r = results[fmt]
     line = None
     if rank == 0:
@@ -354,10 +357,59 @@ def run_ours(args):
                   for k, v in results.items() if k != fmt}
         if others:
             line["other_packings"] = others
+        if prefill is not None:
+            line["prefill"] = prefill
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return line
+
+
+def run_prefill(fmt, M, dev, bz, torch, peaks, peak_kind, steps):
+    """Prefill: M tokens through one layer's four projections (tcgen05 GEMM + FWHT pass)."""
+    from ternary_weight_02_b200 import inputs
+    stream = torch.cuda.Stream(device=dev)
+    items = []
+    for i, (name, K, N) in enumerate(SHAPES):
+        t = torch.from_numpy(inputs.trits(i, N, K)).to(dev)
+        packed = bz.pack(fmt, t)
+        del t
+        s = torch.from_numpy(inputs.scales(i, N, K).view(np.int16)).to(dev).view(torch.float16)
+        x = torch.randn((M, K), device=dev, generator=torch.Generator(device=dev).manual_seed(i)).half()
+        items.append((name, K, N, packed, s, x, torch.empty((M, N), dtype=torch.float16, device=dev)))
+        bz.bonsai_reserve(M, N, K)
+    sp = stream.cuda_stream
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    per = {}
+    total_flop = 0
+    with torch.cuda.stream(stream):
+        for name, K, N, packed, s, x, y in items:
+            for _ in range(2):
+                bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt, sp)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(steps):
+                bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt, sp)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / steps
+            flop = 2 * M * N * K
+            total_flop += flop
+            per[name] = {"us": round(us, 1), "tflops": round(flop / us / 1e6, 1)}
+    layer_us = sum(v["us"] for v in per.values())
+    burst = float(peaks["bf16_tflops"])
+    dom = per["gate_up"]
+    return {
+        "metric": "prefill GEMM TFLOP/s", "value": round(total_flop / layer_us / 1e6, 1), "unit": "TFLOP/s",
+        "workload": f"M={M} tokens x the four 27B-class projections, {FMT_NAMES[fmt]}, FP16 x FP16 -> FP32 (tcgen05)",
+        "us_per_layer": round(layer_us, 1), "per_projection": per,
+        "roofline": {"bound": "tensor", "kernel": "gemm gate/up 5120->34816 (incl. FWHT pass)",
+                     "achieved": dom["tflops"], "peak": burst, "peak_kind": f"{peak_kind} bf16 burst (fp16 same dense rate)",
+                     "unit": "TFLOP/s", "frac": round(dom["tflops"] / burst, 4),
+                     "frac_of_sustained": round(dom["tflops"] / float(peaks["bf16_tflops_sustained"]), 4),
+                     "traffic": None},
+    }
 
 
 def cpu_baseline(fmt):
@@ -377,6 +429,36 @@ def cpu_baseline(fmt):
             "sample": f"one layer (4 projections, M=1, {FMT_NAMES[fmt]}) of the 64-layer stack, float64"}
 
 
+def run_case(args):
+    """One projection, `reps` calls (a small case for profilers: python bench.py --case ...)."""
+    import torch
+    from ternary_weight_02_b200 import bonsai as bz
+    from ternary_weight_02_b200 import inputs
+    fmt = {"ptq1": 1, "pq2": 2}[args.fmt]
+    i = [n for n, _, _ in SHAPES].index(args.shape)
+    _, K, N = SHAPES[i]
+    M = 1 if args.case == "gemv" else args.m
+    dev = torch.device("cuda")
+    t = torch.from_numpy(inputs.trits(i, N, K)).to(dev)
+    packed = bz.pack(fmt, t)
+    del t
+    s = torch.from_numpy(inputs.scales(i, N, K).view(np.int16)).to(dev).view(torch.float16)
+    x = torch.from_numpy(inputs.activations(i, M, K).view(np.int16)).to(dev).view(torch.float16)
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    algo = bz.BONSAI_ALGO_GEMV if args.case == "gemv" else bz.BONSAI_ALGO_GEMM
+    bz.bonsai_reserve(M, N, K)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.reps):
+        bz.bonsai_ternary_linear_algo(x, packed, s, y, M, N, K, fmt, algo)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / args.reps
+    print(json.dumps({"case": args.case, "shape": args.shape, "fmt": FMT_NAMES[fmt], "M": M, "K": K, "N": N,
+                      "reps": args.reps, "us_per_call": round(us, 2)}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -386,10 +468,18 @@ def main():
     ap.add_argument("--fmt", choices=["pq2", "ptq1"], default="pq2")
     ap.add_argument("--both", type=int, default=1, help="also measure the other packing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-m", type=int, default=2048, help="tokens of the prefill GEMM line (0: skip)")
+    ap.add_argument("--case", choices=["gemv", "gemm"], help="run one projection only (profiler case)")
+    ap.add_argument("--shape", choices=[n for n, _, _ in SHAPES], default="gate_up")
+    ap.add_argument("--m", type=int, default=2048, help="tokens for --case gemm")
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     world, rank, _ = dist_setup()
+    if args.case:
+        run_case(args)
+        return
     if args.impl == "reference":
         if rank != 0:
             return

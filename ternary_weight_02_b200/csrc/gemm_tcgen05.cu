@@ -161,42 +161,59 @@ __device__ __forceinline__ void st_chunk(uint8_t *stage, int r, int chunk, const
     *p = make_uint4(v[0], v[1], v[2], v[3]);
 }
 
-// Codes of one 128-weight group of row n as 8 words (word i: weights 16i .. 16i+15).
+// Raw packed bytes of one 128-weight group of row n (PQ2_0: 32 bytes; PTQ1_0: 26 bytes
+// in 7 words) and its FP16 scale, loaded a group ahead of their decode.
+struct GroupRaw {
+    uint32_t w[8];
+    uint16_t scale;
+};
+
 template <int kFmt>
-__device__ __forceinline__ void group_codes(const uint8_t *packed, int64_t n, int64_t G, int64_t g,
-                                            const uint32_t *lut, uint32_t (&cw)[8]) {
+__device__ __forceinline__ void load_group(const uint8_t *packed, const uint16_t *scales, int64_t n, int64_t G,
+                                           int64_t g, GroupRaw &raw) {
+    raw.scale = __ldg(scales + n * G + g);
     if (kFmt == 2) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(packed + n * G * kPq2GroupBytes + g * kPq2GroupBytes);
+        const uint4 *p = reinterpret_cast<const uint4 *>(packed + (n * G + g) * kPq2GroupBytes);
         const uint4 a = __ldg(p), b = __ldg(p + 1);
-        cw[0] = a.x, cw[1] = a.y, cw[2] = a.z, cw[3] = a.w;
-        cw[4] = b.x, cw[5] = b.y, cw[6] = b.z, cw[7] = b.w;
+        raw.w[0] = a.x, raw.w[1] = a.y, raw.w[2] = a.z, raw.w[3] = a.w;
+        raw.w[4] = b.x, raw.w[5] = b.y, raw.w[6] = b.z, raw.w[7] = b.w;
     } else {
         // 26 bytes at an even address: 6 aligned words and one aligned half-word
         const uint8_t *src = packed + (n * G + g) * kPtq1GroupBytes;
-        uint32_t bytes[7];
         if ((reinterpret_cast<uintptr_t>(src) & 3u) == 0) {
             const uint32_t *q = reinterpret_cast<const uint32_t *>(src);
 #pragma unroll
-            for (int i = 0; i < 6; i++) bytes[i] = __ldg(q + i);
-            bytes[6] = __ldg(reinterpret_cast<const unsigned short *>(src + 24));
+            for (int i = 0; i < 6; i++) raw.w[i] = __ldg(q + i);
+            raw.w[6] = __ldg(reinterpret_cast<const unsigned short *>(src + 24));
         } else {
             const uint32_t lo = __ldg(reinterpret_cast<const unsigned short *>(src));
             const uint32_t *q = reinterpret_cast<const uint32_t *>(src + 2);
             uint32_t t[6];
 #pragma unroll
             for (int i = 0; i < 6; i++) t[i] = __ldg(q + i);
-            bytes[0] = lo | (t[0] << 16);
+            raw.w[0] = lo | (t[0] << 16);
 #pragma unroll
-            for (int i = 1; i < 6; i++) bytes[i] = __funnelshift_r(t[i - 1], t[i], 16);
-            bytes[6] = t[5] >> 16;
+            for (int i = 1; i < 6; i++) raw.w[i] = __funnelshift_r(t[i - 1], t[i], 16);
+            raw.w[6] = t[5] >> 16;
         }
+        raw.w[7] = 0u;
+    }
+}
+
+// Codes of the group as 8 words (word i: weights 16i .. 16i+15, code = trit + 1).
+template <int kFmt>
+__device__ __forceinline__ void group_codes(const GroupRaw &raw, const uint32_t *lut, uint32_t (&cw)[8]) {
+    if (kFmt == 2) {
+#pragma unroll
+        for (int i = 0; i < 8; i++) cw[i] = raw.w[i];
+    } else {
 #pragma unroll
         for (int i = 0; i < 8; i++) cw[i] = 0u;
         // byte b's five digits become codes 5b .. 5b+4 (2 bits each, bit 10b of the
         // 256-bit code stream); the padding digits of byte 25 fall past bit 255
 #pragma unroll
         for (int b = 0; b < kPtq1GroupBytes; b++) {
-            const uint32_t f = lut[(bytes[b >> 2] >> (8 * (b & 3))) & 0xFFu];
+            const uint32_t f = lut[(raw.w[b >> 2] >> (8 * (b & 3))) & 0xFFu];
             const int pos = 10 * b, wi = pos >> 5, sh = pos & 31;
             cw[wi] |= f << sh;
             if (sh > 22 && wi + 1 < 8) cw[wi + 1] |= f >> (32 - sh);
@@ -301,15 +318,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
         const int r = tid - 64;                      // 0 .. 255: row of the B tile
         const int64_t n = (int64_t)tile_n * BN + r;  // weight row
         const bool valid = n < N;
+        GroupRaw cur, nxt;
+        if (valid) load_group<kFmt>(packed, scales, n, G, 0, cur);
         for (int g = 0; g < (int)G; g++) {
             const int ks0 = 2 * g;  // the group fills stages ks0 and ks0 + 1
             const int s0 = ks0 % STAGES, s1 = (ks0 + 1) % STAGES;
             const uint32_t ph0 = (uint32_t)(ks0 / STAGES) & 1u, ph1 = (uint32_t)((ks0 + 1) / STAGES) & 1u;
+            if (valid && g + 1 < (int)G) load_group<kFmt>(packed, scales, n, G, g + 1, nxt);  // in flight
             uint32_t cw[8];
             __half2 s2 = __float2half2_rn(0.f);
             if (valid) {
-                group_codes<kFmt>(packed, n, G, g, lut, cw);
-                const __half sh = __ushort_as_half(__ldg(scales + n * G + g));
+                group_codes<kFmt>(cur, lut, cw);
+                const __half sh = __ushort_as_half(cur.scale);
                 s2 = __halves2half2(sh, sh);
             } else {
 #pragma unroll
@@ -339,6 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                 mbar_arrive(full_b + s0);
                 mbar_arrive(full_b + s1);
             }
+            cur = nxt;
         }
 
         // ------------------------------------------------ epilogue

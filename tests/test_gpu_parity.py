@@ -269,3 +269,49 @@ def test_gemm_prefill_full_size_sampled(bz, fmt, M, K, N):
     ok, rel, mx = oracle.compare(got, ref)
     assert ok, (rel, mx)
     assert bool(torch.isfinite(y).all())
+
+
+# ------------------------------------------------------------ skinny batches (mma.sync, PQ2_0)
+
+SKINNY_SMALL = [(2, 64, 128), (3, 129, 384), (8, 300, 1024), (9, 100, 640), (16, 257, 2048)]
+
+
+@pytest.mark.parametrize("M,N,K", SKINNY_SMALL)
+@pytest.mark.parametrize("split_k", [0, 1, 3])
+def test_skinny_small(bz, M, N, K, split_k):
+    p = Problem(M, N, K, PQ2, seed=M * 31 + N)
+    got = _run(bz, p, bz.BONSAI_ALGO_SKINNY, split_k)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+@pytest.mark.parametrize("M", [2, 4, 8, 16])
+@pytest.mark.parametrize("K,N", [(5120, 5120), (17408, 5120), (5120, 34816)])
+def test_skinny_decode_shapes_full(bz, M, K, N):
+    """Skinny decode batches on 27B-class projections, every output against the checker."""
+    p = Problem(M, N, K, PQ2, seed=M)
+    got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+def test_skinny_split_is_deterministic(bz):
+    import torch
+    p = Problem(8, 5120, 17408, PQ2, seed=3)
+    x, packed, scales = p.device()
+    outs = []
+    for sk in (0, 0, 5, 5):
+        y = torch.empty((8, 5120), dtype=torch.float16, device="cuda")
+        bz.bonsai_ternary_linear_algo(x, packed, scales, y, 8, 5120, 17408, PQ2, bz.BONSAI_ALGO_SKINNY, sk)
+        outs.append(y)
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[2], outs[3])
+    assert oracle.compare(to_numpy_f16(outs[2]), to_numpy_f16(outs[0]))[0]
+
+
+@pytest.mark.parametrize("M", [2, 5, 16])
+def test_small_batches_ptq1_take_the_gemm(bz, M):
+    p = Problem(M, 300, 1024, PTQ1, seed=M)
+    got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
