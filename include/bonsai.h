@@ -136,8 +136,11 @@ int bonsai_ternary_linear(const uint16_t *x, const uint8_t *packed, const uint16
                           uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, void *stream);
 
 /* As bonsai_ternary_linear with an explicit kernel choice (bonsai_algo) and an
- * explicit split-K factor for the GEMV / skinny kernels (0 = automatic, 1 = no
- * split, otherwise the number of K slices, clamped to what the shape allows).
+ * explicit split-K factor for the skinny kernel (0 = automatic, 1 = no split,
+ * otherwise the number of K chunks, clamped to what the shape allows).  For
+ * BONSAI_ALGO_GEMM the same argument picks the M tile instead: 1 = 128 rows per CTA,
+ * 2 = 256 rows (two TMEM accumulators sharing each expanded weight tile), 0 =
+ * automatic.  The batch-1 GEMV ignores it (its K split follows its table slice).
  * Returns BONSAI_ERR_ALGO if the chosen kernel cannot run the shape (e.g.
  * BONSAI_ALGO_GEMV with M > 1).  For measurement and testing of each kernel. */
 int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,

@@ -279,7 +279,7 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
             e = launch_skinny(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, st->info);
             break;
         case BONSAI_ALGO_GEMM:
-            e = launch_gemm(x, packed, scales, y, M, N, K, fmt, ws, s, st->info);
+            e = launch_gemm(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, st->info);
             break;
         default:
             e = launch_linear_simple(x, packed, scales, y, M, N, K, fmt, ws, s, st->info);

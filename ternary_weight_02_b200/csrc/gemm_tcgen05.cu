@@ -32,22 +32,30 @@
 namespace bonsai {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128, BN = 256, BK = 64;  // BM: rows of one MMA / one TMEM accumulator
 constexpr int kExpandWarps = 8;
 constexpr int kThreads = (2 + kExpandWarps) * 32;  // 320
-constexpr int A_STAGE_BYTES = BM * BK * 2;         // 16 KB
 constexpr int B_STAGE_BYTES = BN * BK * 2;         // 32 KB
-constexpr int kTmemCols = 256;
 constexpr uint32_t kSpinLimit = 1u << 22;
-// shared memory: [A stages][B stages][barriers][tmem slot][abort flag][PTQ1_0 LUT]
-constexpr int kOffA = 0;
-constexpr int kOffB = STAGES * A_STAGE_BYTES;
-constexpr int kOffBar = kOffB + STAGES * B_STAGE_BYTES;
-constexpr int kNumBars = 3 * STAGES + 1;  // full_a, full_b, empty, done
-constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-constexpr int kOffAbort = kOffTmemSlot + 8;
-constexpr int kOffLut = kOffAbort + 8;
-constexpr int kSmemBytes = kOffLut + 256 * 4 + 1024;  // + alignment slack for the 1024-B tile base
+
+// Tile configuration: kAcc accumulators of 128 rows each share every B stage (the
+// expanded weights), so the CTA covers 128 * kAcc rows of y.
+template <int kAcc>
+struct Cfg {
+    static constexpr int kStages = kAcc == 2 ? 3 : 4;
+    static constexpr int kTileM = BM * kAcc;
+    static constexpr int kAStage = kTileM * BK * 2;  // 16 or 32 KB
+    static constexpr int kTmemCols = 256 * kAcc;
+    // shared memory: [A stages][B stages][barriers][tmem slot][abort flag][PTQ1_0 LUT]
+    static constexpr int kOffA = 0;
+    static constexpr int kOffB = kStages * kAStage;
+    static constexpr int kOffBar = kOffB + kStages * B_STAGE_BYTES;
+    static constexpr int kNumBars = 3 * kStages + 1;  // full_a, full_b, empty, done
+    static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
+    static constexpr int kOffAbort = kOffTmemSlot + 8;
+    static constexpr int kOffLut = kOffAbort + 8;
+    static constexpr int kSmemBytes = kOffLut + 256 * 4 + 1024;  // + slack for the 1024-B tile base
+};
 
 // ---------------------------------------------------------------- PTX wrappers
 
@@ -223,20 +231,22 @@ __device__ __forceinline__ void group_codes(const GroupRaw &raw, const uint32_t 
 
 // ---------------------------------------------------------------- kernel
 
-template <int kFmt>
+template <int kFmt, int kAcc>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap a_map, const uint8_t *__restrict__ packed,
     const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, int M, int N, int K) {
+    using C = Cfg<kAcc>;
+    constexpr int STAGES = C::kStages;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment of the tile area (128-byte swizzle atoms)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem + kOffA;
-    uint8_t *sB = smem + kOffB;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint8_t *sA = smem + C::kOffA;
+    uint8_t *sB = smem + C::kOffB;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint64_t *full_a = bars, *full_b = bars + STAGES, *empty = bars + 2 * STAGES, *done = bars + 3 * STAGES;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmemSlot);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffAbort);
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem + kOffLut);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffAbort);
+    uint32_t *lut = reinterpret_cast<uint32_t *>(smem + C::kOffLut);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int tile_m = blockIdx.x, tile_n = blockIdx.y;
@@ -244,10 +254,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     const int64_t G = K / kGroup;
 
     if (tid == 0) {
-        for (int s = 0; s < STAGES; s++) {
-            mbar_init(full_a + s, 1);
-            mbar_init(full_b + s, kExpandWarps);
-            mbar_init(empty + s, 1);
+        for (int st = 0; st < STAGES; st++) {
+            mbar_init(full_a + st, 1);
+            mbar_init(full_b + st, kExpandWarps);
+            mbar_init(empty + st, 1);
         }
         mbar_init(done, 1);
         *abort_flag = 0;
@@ -266,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)),
-                     "r"(kTmemCols)
+                     "r"(C::kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -280,14 +290,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
         if (lane == 0) {
             int issued = 0;
             for (int ks = 0; ks < num_k; ks++) {
-                const int s = ks % STAGES;
+                const int st = ks % STAGES;
                 const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-                if (*abort_flag || !mbar_wait(empty + s, ph ^ 1u)) {
+                if (*abort_flag || !mbar_wait(empty + st, ph ^ 1u)) {
                     *abort_flag = 1;
                     break;
                 }
-                mbar_arrive_expect_tx(full_a + s, A_STAGE_BYTES);
-                tma_load_2d(sA + s * A_STAGE_BYTES, &a_map, full_a + s, ks * BK, tile_m * BM);
+                mbar_arrive_expect_tx(full_a + st, C::kAStage);
+#pragma unroll
+                for (int a = 0; a < kAcc; a++)
+                    tma_load_2d(sA + st * C::kAStage + a * (BM * BK * 2), &a_map, full_a + st, ks * BK,
+                                tile_m * C::kTileM + a * BM);
                 issued = ks + 1;
             }
             // the copies this thread started land before the CTA may exit
@@ -298,18 +311,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             for (int ks = 0; ks < num_k; ks++) {
-                const int s = ks % STAGES;
+                const int st = ks % STAGES;
                 const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-                if (*abort_flag || !mbar_wait(full_a + s, ph) || !mbar_wait(full_b + s, ph)) {
+                if (*abort_flag || !mbar_wait(full_a + st, ph) || !mbar_wait(full_b + st, ph)) {
                     *abort_flag = 1;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a0 = saddr(sA + s * A_STAGE_BYTES), b0 = saddr(sB + s * B_STAGE_BYTES);
+                const uint32_t b0 = saddr(sB + st * B_STAGE_BYTES);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; kk++)
-                    mma_f16(tmem, desc_sw128(a0 + kk * 32), desc_sw128(b0 + kk * 32), (ks > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(empty + s);  // frees the stage when these MMAs have read it
+                for (int kk = 0; kk < BK / 16; kk++) {
+                    const uint64_t bdesc = desc_sw128(b0 + kk * 32);
+#pragma unroll
+                    for (int a = 0; a < kAcc; a++) {
+                        const uint32_t a0 = saddr(sA + st * C::kAStage + a * (BM * BK * 2));
+                        mma_f16(tmem + (uint32_t)(a * 256), desc_sw128(a0 + kk * 32), bdesc,
+                                (ks > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                mma_commit(empty + st);  // frees the stage when these MMAs have read it
             }
             mma_commit(done);  // all MMAs issued by this thread are complete
         }
@@ -320,76 +340,76 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
         const bool valid = n < N;
         GroupRaw cur, nxt;
         if (valid) load_group<kFmt>(packed, scales, n, G, 0, cur);
-        for (int g = 0; g < (int)G; g++) {
-            const int ks0 = 2 * g;  // the group fills stages ks0 and ks0 + 1
-            const int s0 = ks0 % STAGES, s1 = (ks0 + 1) % STAGES;
-            const uint32_t ph0 = (uint32_t)(ks0 / STAGES) & 1u, ph1 = (uint32_t)((ks0 + 1) / STAGES) & 1u;
-            if (valid && g + 1 < (int)G) load_group<kFmt>(packed, scales, n, G, g + 1, nxt);  // in flight
-            uint32_t cw[8];
-            __half2 s2 = __float2half2_rn(0.f);
-            if (valid) {
-                group_codes<kFmt>(cur, lut, cw);
-                const __half sh = __ushort_as_half(cur.scale);
-                s2 = __halves2half2(sh, sh);
-            } else {
+        uint32_t cw[8];
+        __half2 s2 = __float2half2_rn(0.f);
+        for (int ks = 0; ks < num_k; ks++) {
+            const int g = ks >> 1, hf = ks & 1;  // a 128-weight group fills two 64-wide stages
+            if (hf == 0) {
+                if (valid && g + 1 < (int)G) load_group<kFmt>(packed, scales, n, G, g + 1, nxt);  // in flight
+                if (valid) {
+                    group_codes<kFmt>(cur, lut, cw);
+                    const __half sh = __ushort_as_half(cur.scale);
+                    s2 = __halves2half2(sh, sh);
+                } else {
 #pragma unroll
-                for (int i = 0; i < 8; i++) cw[i] = 0x55555555u;  // all trits zero
+                    for (int i = 0; i < 8; i++) cw[i] = 0x55555555u;  // all trits zero
+                }
             }
+            const int st = ks % STAGES;
+            const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
             // every lane acquires the stage itself; the verdict is made warp-uniform
-            const bool free_ok = !*abort_flag && mbar_wait(empty + s0, ph0 ^ 1u) && mbar_wait(empty + s1, ph1 ^ 1u);
+            const bool free_ok = !*abort_flag && mbar_wait(empty + st, ph ^ 1u);
             if (!__all_sync(0xffffffffu, free_ok)) {
                 *abort_flag = 1;
                 break;
             }
-            uint8_t *st0 = sB + s0 * B_STAGE_BYTES, *st1 = sB + s1 * B_STAGE_BYTES;
+            uint8_t *stage = sB + st * B_STAGE_BYTES;
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
+            for (int i = 0; i < 4; i++) {
                 uint32_t out[8];
-                expand_word(cw[i], s2, out);
-                // word i covers weights 16i .. 16i+15 = chunks 2i, 2i+1 of the group
-                uint8_t *st = i < 4 ? st0 : st1;
-                const int c = (2 * i) & 7;
-                st_chunk(st, r, c, out);
-                st_chunk(st, r, c + 1, out + 4);
+                expand_word(hf ? cw[4 + i] : cw[i], s2, out);  // weights 64hf + 16i .. +15
+                st_chunk(stage, r, 2 * i, out);
+                st_chunk(stage, r, 2 * i + 1, out + 4);
             }
             // make the generic-proxy stores visible to the tensor core, then signal
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(full_b + s0);
-                mbar_arrive(full_b + s1);
-            }
-            cur = nxt;
+            if (lane == 0) mbar_arrive(full_b + st);
+            if (hf == 1) cur = nxt;
         }
 
         // ------------------------------------------------ epilogue
         const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0)) && !*abort_flag;
         tc_fence_after();
-        const int q = warp & 3;                  // TMEM lane quadrant this warp may read
-        const int half = (warp - 2) >> 2;        // which 128 columns
-        const int m = tile_m * BM + 32 * q + lane;
+        const int q = warp & 3;            // TMEM lane quadrant this warp may read
+        const int half = (warp - 2) >> 2;  // which 128 columns
 #pragma unroll 1
-        for (int c = 0; c < 4; c++) {
-            const int col = half * 128 + 32 * c;
-            uint32_t v[32];
-            __syncwarp();
-            tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)col, v);
-            if (m >= M) continue;
-            const int64_t n0 = (int64_t)tile_n * BN + col;
-            uint16_t *yr = y + (int64_t)m * N + n0;
-            if (ok && n0 + 32 <= N && (N & 7) == 0) {
-                uint32_t h[16];
+        for (int a = 0; a < kAcc; a++) {
+            const int m = tile_m * C::kTileM + a * BM + 32 * q + lane;
+#pragma unroll 1
+            for (int c = 0; c < 4; c++) {
+                const int col = half * 128 + 32 * c;
+                uint32_t v[32];
+                __syncwarp();
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 256 + col), v);
+                if (m >= M) continue;
+                const int64_t n0 = (int64_t)tile_n * BN + col;
+                uint16_t *yr = y + (int64_t)m * N + n0;
+                if (ok && n0 + 32 <= N && (N & 7) == 0) {
+                    uint32_t h[16];
 #pragma unroll
-                for (int i = 0; i < 16; i++) {
-                    const __half2 p2 = __floats2half2_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                    h[i] = *reinterpret_cast<const uint32_t *>(&p2);
+                    for (int i = 0; i < 16; i++) {
+                        const __half2 p2 =
+                            __floats2half2_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                        h[i] = *reinterpret_cast<const uint32_t *>(&p2);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(yr);
+#pragma unroll
+                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+                } else {
+                    for (int i = 0; i < 32; i++)
+                        if (n0 + i < N) yr[i] = ok ? float_to_half_bits(__uint_as_float(v[i])) : (uint16_t)0x7E00u;
                 }
-                uint4 *dst = reinterpret_cast<uint4 *>(yr);
-#pragma unroll
-                for (int i = 0; i < 4; i++) dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
-            } else {
-                for (int i = 0; i < 32; i++)
-                    if (n0 + i < N) yr[i] = ok ? float_to_half_bits(__uint_as_float(v[i])) : (uint16_t)0x7E00u;
             }
         }
     }
@@ -399,7 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
+                     : "memory");
     }
 }
 
@@ -436,7 +457,7 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt) {
 }
 
 cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
-                        uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt,
+                        uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int tile_hint,
                         const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
     uint16_t *xr = reinterpret_cast<uint16_t *>(ws.data);
     cudaError_t err = launch_hadamard_f16(x, xr, M, K, s, dev);
@@ -454,17 +475,25 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
 
-    const dim3 grid((unsigned)((M + BM - 1) / BM), (unsigned)((N + BN - 1) / BN));
-    if (fmt == 1) {
-        err = cudaFuncSetAttribute(gemm_tcgen05_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (err != cudaSuccess) return err;
-        gemm_tcgen05_kernel<1><<<grid, kThreads, kSmemBytes, s>>>(map, packed, scales, y, (int)M, (int)N, (int)K);
-    } else {
-        err = cudaFuncSetAttribute(gemm_tcgen05_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (err != cudaSuccess) return err;
-        gemm_tcgen05_kernel<2><<<grid, kThreads, kSmemBytes, s>>>(map, packed, scales, y, (int)M, (int)N, (int)K);
-    }
-    return cudaGetLastError();
+    // one or two 128-row accumulators per CTA: two halve the trit expansion per FLOP; pick
+    // the one whose grid wastes less of the last wave
+    const int64_t nt = (N + BN - 1) / BN;
+    auto wave_eff = [&](int64_t tiles) {
+        const int64_t waves = (tiles + dev.sm_count - 1) / dev.sm_count;
+        return (double)tiles / (double)(waves * dev.sm_count);
+    };
+    const int64_t t1 = ((M + BM - 1) / BM) * nt, t2 = ((M + 2 * BM - 1) / (2 * BM)) * nt;
+    const bool two = tile_hint == 2 || (tile_hint != 1 && M > BM && wave_eff(t2) * 1.35 >= wave_eff(t1));
+    auto go = [&](auto kern, int acc, int smem) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        const dim3 grid((unsigned)((M + (int64_t)BM * acc - 1) / ((int64_t)BM * acc)), (unsigned)nt);
+        kern<<<grid, kThreads, smem, s>>>(map, packed, scales, y, (int)M, (int)N, (int)K);
+        return cudaGetLastError();
+    };
+    if (fmt == 1)
+        return two ? go(gemm_tcgen05_kernel<1, 2>, 2, Cfg<2>::kSmemBytes) : go(gemm_tcgen05_kernel<1, 1>, 1, Cfg<1>::kSmemBytes);
+    return two ? go(gemm_tcgen05_kernel<2, 2>, 2, Cfg<2>::kSmemBytes) : go(gemm_tcgen05_kernel<2, 1>, 1, Cfg<1>::kSmemBytes);
 }
 
 }  // namespace bonsai

@@ -222,9 +222,11 @@ GEMM_SMALL = [(1, 64, 128), (17, 256, 128), (130, 300, 384), (256, 512, 1024), (
 
 @pytest.mark.parametrize("fmt", [PTQ1, PQ2])
 @pytest.mark.parametrize("M,N,K", GEMM_SMALL)
-def test_gemm_small(bz, fmt, M, N, K):
+@pytest.mark.parametrize("tile", [1, 2])
+def test_gemm_small(bz, fmt, M, N, K, tile):
+    """tile 1: one 128-row TMEM accumulator per CTA; tile 2: two (256 rows)."""
     p = Problem(M, N, K, fmt, seed=M + N + K)
-    got = _run(bz, p, bz.BONSAI_ALGO_GEMM)
+    got = _run(bz, p, bz.BONSAI_ALGO_GEMM, tile)
     assert np.all(np.isfinite(got))
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
