@@ -312,7 +312,9 @@ def run_ours(args):
             ms_e2e = float(t.item())
         e2e = world * step_bytes(f) / (ms_e2e * 1e-3) / 1e9
 
+        launches_per_layer = sum(bz.bonsai_launch_count(1, N, K, f) for _, K, N in SHAPES)
         results[f] = {
+            "launches_per_layer": launches_per_layer,
             "value": value, "ms": ms, "clocks": clk, "dom_us": dom_us, "dom_gbs": dom_gbs,
             "dom_bytes": dom_bytes, "traffic": traffic, "e2e": e2e, "h2d": h2d, "d2h": d2h,
         }
@@ -348,7 +350,7 @@ def run_ours(args):
             },
             "e2e": {"value": round(r["e2e"], 1), "unit": "GB/s", "h2d_bytes_per_step": r["h2d"],
                     "d2h_bytes_per_step": r["d2h"]},
-            "gpu_launches": LAYERS * len(SHAPES) * args.steps,
+            "gpu_launches": LAYERS * r["launches_per_layer"] * args.steps,
             "clocks": r["clocks"],
         }
         others = {FMT_NAMES[k]: {"value": round(v["value"], 1), "unit": "GB/s",

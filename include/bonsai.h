@@ -140,12 +140,20 @@ int bonsai_ternary_linear(const uint16_t *x, const uint8_t *packed, const uint16
  * otherwise the number of K chunks, clamped to what the shape allows).  For
  * BONSAI_ALGO_GEMM the same argument picks the M tile instead: 1 = 128 rows per CTA,
  * 2 = 256 rows (two TMEM accumulators sharing each expanded weight tile), 0 =
- * automatic.  The batch-1 GEMV ignores it (its K split follows its table slice).
+ * automatic.  For BONSAI_ALGO_GEMV it picks the schedule: 1 = each CTA walks all K
+ * slices of its rows (no split-K), >= 2 = one 512-wide K slice per CTA with split-K
+ * partials, 0 = automatic.
  * Returns BONSAI_ERR_ALGO if the chosen kernel cannot run the shape (e.g.
  * BONSAI_ALGO_GEMV with M > 1).  For measurement and testing of each kernel. */
 int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                                uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int algo,
                                int split_k, void *stream);
+
+/* Number of kernels one bonsai_ternary_linear_algo call with these arguments launches
+ * on the current device (the batch-1 GEMV: 1, or 2 when its split-K partials are
+ * summed by a second kernel; the other kernels: 2, the rotation pass and the kernel),
+ * or a negative bonsai_status.  Launches nothing. */
+int bonsai_launch_count(int64_t M, int64_t N, int64_t K, int fmt, int algo, int split_k);
 
 /* Grows the calling device's workspace so that calls up to M x N x K (any
  * format and kernel) need no further allocation; call before capturing calls

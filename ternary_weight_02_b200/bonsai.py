@@ -58,6 +58,7 @@ _SIGS = {
     "bonsai_ternary_linear": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _p]),
     "bonsai_ternary_linear_algo": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _int, _int, _p]),
     "bonsai_ternary_linear_noalloc": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _p]),
+    "bonsai_launch_count": (_int, [_i64, _i64, _i64, _int, _int, _int]),
     "bonsai_reserve": (_int, [_i64, _i64, _i64]),
     "bonsai_shutdown": (None, []),
 }
@@ -158,6 +159,14 @@ def bonsai_ternary_linear_noalloc(x, packed, scales, y, M: int, N: int, K: int, 
     """Batch-1 layer on the library's fixed device scratch: allocates nothing."""
     _check(_lib.bonsai_ternary_linear_noalloc(_ptr(x), _ptr(packed), _ptr(scales), _ptr(y), M, N, K,
                                               fmt, _stream(stream)), "bonsai_ternary_linear_noalloc")
+
+
+def bonsai_launch_count(M: int, N: int, K: int, fmt: int, algo: int = BONSAI_ALGO_AUTO,
+                        split_k: int = 0) -> int:
+    n = _lib.bonsai_launch_count(M, N, K, fmt, algo, split_k)
+    if n < 0:
+        raise BonsaiError(n, "bonsai_launch_count")
+    return n
 
 
 def bonsai_reserve(M: int, N: int, K: int) -> None:

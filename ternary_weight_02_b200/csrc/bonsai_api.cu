@@ -294,6 +294,25 @@ int bonsai_ternary_linear(const uint16_t *x, const uint8_t *packed, const uint16
                                       stream);
 }
 
+int bonsai_launch_count(int64_t M, int64_t N, int64_t K, int fmt, int algo, int split_k) {
+    int rc = check_fmt(fmt);
+    if (rc != BONSAI_OK) return rc;
+    rc = check_shape(M, N, K);
+    if (rc != BONSAI_OK) return rc;
+    if (M == 0 || N == 0) return 0;
+    const int chosen = resolve_algo(algo, M, N, K, fmt);
+    if (chosen < 0) return chosen;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int dev;
+    DeviceState *st;
+    rc = probe_current(&dev, &st);
+    if (rc != BONSAI_OK) return rc;
+    switch (chosen) {
+        case BONSAI_ALGO_GEMV: return gemv_launches(N, K, fmt, split_k, st->info);
+        default: return 2;  // the rotation pass, then the kernel
+    }
+}
+
 int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
     int rc = check_shape(M, N, K);
     if (rc != BONSAI_OK) return rc;

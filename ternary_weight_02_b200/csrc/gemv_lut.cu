@@ -29,12 +29,14 @@
 //   and scales in flight.  A transpose-reduction over the 8 lanes of a scale group is
 //   followed by the scale multiply and two more shuffle stages.
 // * Two schedules:
-//   - rows mode (large N): a CTA owns a range of rows, rotates all of x once, and walks
-//     the K slices, rebuilding the tables per slice and keeping each row's sum in
-//     registers.  No split-K and no tail.
-//   - split mode (small N): a CTA owns one slice and a range of rows and writes FP32
-//     partials; the warp that brings a row block's last slice (arrival counter in the
-//     workspace) sums the partials in slice order (deterministic) and writes y.
+//   - rows mode (on request): a CTA owns a range of rows, rotates all of x once, and
+//     walks the K slices, rebuilding the tables per slice and keeping each row's sum
+//     in registers.  No split-K, but ten table builds per CTA for K = 5120.
+//   - split mode (the default): a CTA owns one slice and a range of rows and writes FP32
+//     partials; a small second kernel (launched behind it with programmatic dependent
+//     launch) sums each row's partials in slice order (deterministic) and writes y.
+//     In this mode x is loaded before the weight prefetch, so that its few loads are
+//     not queued behind the CTA's weight traffic.
 // * Programmatic dependent launch: a kernel lets the next kernel on the stream start
 //   at once; the next kernel prefetches its own weights and then waits for this one to
 //   finish before it reads x, the workspace or y.
@@ -173,10 +175,12 @@ __device__ __forceinline__ void zero_phantom_tables(uint8_t *tables, int lane, i
 }
 
 // Loads one warp task: register i <- the lane's word of row n0 + i (each load
-// instruction reads one row's contiguous slice segment), and the two scales the lane
-// applies after the group reduction: rows (lane & 7) + 8m of group lane >> 3.
+// instruction reads one row's contiguous slice segment), and the two FP16 scales the
+// lane applies after the group reduction: rows (lane & 7) + 8m of group lane >> 3.
+// Nothing here consumes the loaded values, so the loads stay in flight until the
+// task is processed (the scales are converted only there).
 template <int kFmt>
-__device__ __forceinline__ void load_task(uint32_t (&w)[kRows], float (&sc)[2], const uint8_t *slice_base,
+__device__ __forceinline__ void load_task(uint32_t (&w)[kRows], uint16_t (&sc)[2], const uint8_t *slice_base,
                                           const uint16_t *scales, int64_t n0, int64_t N, int64_t G,
                                           int64_t gcol, uint32_t row_bytes, int lane_off, int lane) {
     const uint8_t *p = slice_base + n0 * row_bytes + lane_off;
@@ -185,16 +189,16 @@ __device__ __forceinline__ void load_task(uint32_t (&w)[kRows], float (&sc)[2], 
 #pragma unroll
         for (int i = 0; i < kRows; i++)
             w[i] = __ldcs(reinterpret_cast<const unsigned int *>(p + (size_t)i * row_bytes));
-        sc[0] = half_bits_to_float(__ldg(sp));
-        sc[1] = half_bits_to_float(__ldg(sp + 8 * G));
+        sc[0] = __ldg(sp);
+        sc[1] = __ldg(sp + 8 * G);
         return;
     }
     const int nvalid = (int)(N - n0);
 #pragma unroll
     for (int i = 0; i < kRows; i++)
         w[i] = i < nvalid ? __ldcs(reinterpret_cast<const unsigned int *>(p + (size_t)i * row_bytes)) : 0u;
-    sc[0] = (lane & 7) < nvalid ? half_bits_to_float(__ldg(sp)) : 0.f;
-    sc[1] = (lane & 7) + 8 < nvalid ? half_bits_to_float(__ldg(sp + 8 * G)) : 0.f;
+    sc[0] = (lane & 7) < nvalid ? __ldg(sp) : (uint16_t)0;
+    sc[1] = (lane & 7) + 8 < nvalid ? __ldg(sp + 8 * G) : (uint16_t)0;
 }
 
 __device__ __forceinline__ float lds_abs(uint32_t addr) {
@@ -219,7 +223,7 @@ __device__ __forceinline__ void transpose_stage(float (&v)[kRows], int lane, int
 
 // Lookups of one task and the reduction over the 8 lanes of each scale group:
 // returns, scaled, rows (lane & 7) + 8m (m = 0, 1) of this lane's group.
-__device__ __forceinline__ float2 task_group_sums(const uint32_t (&w)[kRows], const float (&sc)[2],
+__device__ __forceinline__ float2 task_group_sums(const uint32_t (&w)[kRows], const uint16_t (&sc)[2],
                                                   const uint32_t (&pbase)[4], int lane) {
     float v[kRows];
 #pragma unroll
@@ -228,12 +232,13 @@ __device__ __forceinline__ float2 task_group_sums(const uint32_t (&w)[kRows], co
         const float t1 = lds_abs(__byte_perm(w[i], pbase[1], 0x7614));
         const float t2 = lds_abs(__byte_perm(w[i], pbase[2], 0x7624));
         const float t3 = lds_abs(__byte_perm(w[i], pbase[3], 0x7634));
-        v[i] = (t0 + t1) + (t2 + t3);
+        const float2 u = __fadd2_rn(make_float2(t0, t1), make_float2(t2, t3));
+        v[i] = u.x + u.y;
     }
     transpose_stage<8>(v, lane, 0);
     transpose_stage<4>(v, lane, 1);
     transpose_stage<2>(v, lane, 2);
-    return make_float2(v[0] * sc[0], v[1] * sc[1]);
+    return make_float2(v[0] * half_bits_to_float(sc[0]), v[1] * half_bits_to_float(sc[1]));
 }
 
 // Sum of the four groups: lanes L and L + 16 end with row L & 15 of the task.
@@ -257,8 +262,8 @@ __device__ __forceinline__ void make_pbase(uint32_t (&pbase)[4], int lane) {
 template <int kFmt>
 __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
     const uint16_t *__restrict__ x, const uint8_t *__restrict__ packed,
-    const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
-    unsigned int *__restrict__ counters, int64_t N, int64_t K, int parts) {
+    const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials, int64_t N,
+    int64_t K, int parts) {
     extern __shared__ __align__(16) uint8_t smem[];
     float *xr = reinterpret_cast<float *>(smem);
     const uint32_t smem_addr = (uint32_t)__cvta_generic_to_shared(smem);
@@ -278,19 +283,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
     const uint8_t *slice_base = packed + (int64_t)slice * Fmt<kFmt>::kSliceBytes;
     const int64_t gcol = (int64_t)slice * (kSliceK / kGroup) + (lane >> 3);
 
-    // weights are not written by earlier kernels of this library: prefetch before the wait
+    zero_phantom_tables<kFmt>(tables, lane, warp);
+    pdl_wait();  // x, the workspace and y may belong to the previous kernel
+    // x first, so that its loads are not queued behind this CTA's weight loads
+    float xv[4];
+    if (warp < 4) load_half4(x + (int64_t)slice * kSliceK + warp * kGroup + 4 * lane, xv);
     int64_t rb = rb_begin + warp;
     uint32_t wa[kRows], wb[kRows], wc[kRows];
-    float sa[2], sb[2], sc2[2];
+    uint16_t sa[2], sb[2], sc2[2];
     if (rb < rb_end) load_task<kFmt>(wa, sa, slice_base, scales, rb * kRows, N, G, gcol, row_bytes, lane_off, lane);
     if (rb + kWarps < rb_end)
         load_task<kFmt>(wb, sb, slice_base, scales, (rb + kWarps) * kRows, N, G, gcol, row_bytes, lane_off, lane);
-    zero_phantom_tables<kFmt>(tables, lane, warp);
-
-    pdl_wait();  // x, the workspace and y may belong to the previous kernel
     if (warp < 4) {  // rotate the slice of x: 4 blocks of 128
-        float xv[4];
-        load_half4(x + (int64_t)slice * kSliceK + warp * kGroup + 4 * lane, xv);
         fwht128_warp(xv, lane);
         *reinterpret_cast<float4 *>(xr + warp * kGroup + 4 * lane) = make_float4(xv[0], xv[1], xv[2], xv[3]);
     }
@@ -300,7 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
     uint32_t pbase[4];
     make_pbase(pbase, lane);
 
-    int ntasks = 0;
+    // one slice's sums go straight to y (S == 1) or to the FP32 partials, which
+    // gemv_reduce_kernel adds up in slice order
     auto finish = [&](float2 gs, int64_t task_rb) {
         const float total = groups_total(gs, lane);
         const int64_t n0 = task_rb * kRows;
@@ -311,7 +316,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
             else
                 partials[(int64_t)slice * N + n0 + row] = total;
         }
-        ntasks++;
     };
     // three rotating task buffers: while one task is reduced, the next two are in flight
     while (rb < rb_end) {
@@ -330,39 +334,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
         finish(task_group_sums(wc, sc2, pbase, lane), rb);
         rb += kWarps;
     }
-    if (S == 1 || ntasks == 0) return;
+}
 
-    // publish this warp's partials, count arrivals (one lane per task), and finish the
-    // row blocks for which this warp brought the last slice
-    __threadfence();
-    __syncwarp();
-    const int64_t my_rb0 = rb_begin + warp;
-    bool last = false;
-    if (lane < ntasks) last = atomicAdd(counters + my_rb0 + (int64_t)lane * kWarps, 1u) == (unsigned int)(S - 1);
-    unsigned int last_mask = __ballot_sync(0xffffffffu, last);
-    if (last_mask == 0u) return;
-    __threadfence();
-    const int half = lane >> 4, row = lane & 15;
-    const int s_lo = half ? S / 2 : 0, s_hi = half ? S : S / 2;
-    while (last_mask) {
-        const int k = __ffs(last_mask) - 1;
-        last_mask &= last_mask - 1;
-        const int64_t rbk = my_rb0 + (int64_t)k * kWarps;
-        const int64_t n0 = rbk * kRows;
+// y[n] = sum over slices s (in order) of partials[s][n]; launched right after the split
+// kernel, it waits for that kernel to finish before reading.
+__global__ void __launch_bounds__(256) gemv_reduce_kernel(const float *__restrict__ partials,
+                                                          uint16_t *__restrict__ y, int64_t N, int S) {
+    pdl_launch_dependents();
+    pdl_wait();
+    for (int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; n < N; n += (int64_t)gridDim.x * blockDim.x) {
         float acc = 0.f;
-        if (n0 + row < N) {
-            const float *pp = partials + n0 + row;
-            for (int s0 = s_lo; s0 < s_hi; s0 += 8) {
-                float tmp[8];
+        int s = 0;
+        for (; s + 8 <= S; s += 8) {
+            float t[8];
 #pragma unroll
-                for (int u = 0; u < 8; u++) tmp[u] = s0 + u < s_hi ? __ldcg(pp + (int64_t)(s0 + u) * N) : 0.f;
+            for (int u = 0; u < 8; u++) t[u] = __ldcg(partials + (int64_t)(s + u) * N + n);
 #pragma unroll
-                for (int u = 0; u < 8; u++) acc += tmp[u];
-            }
+            for (int u = 0; u < 8; u++) acc += t[u];
         }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 16);
-        if (lane < 16 && n0 + row < N) y[n0 + row] = float_to_half_bits(acc);
-        if (lane == 0) counters[rbk] = 0u;
+        for (; s < S; s++) acc += __ldcg(partials + (int64_t)s * N + n);
+        y[n] = float_to_half_bits(acc);
     }
 }
 
@@ -398,8 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(
         const bool active = rb < rb_end;
         // four slice buffers: slice s uses buffer s % 4, slices s+1 .. s+3 are in flight
         uint32_t wq[4][kRows];
-        float sq[4][2];
-        auto fetch = [&](int sl, uint32_t (&wt)[kRows], float (&st)[2]) {
+        uint16_t sq[4][2];
+        auto fetch = [&](int sl, uint32_t (&wt)[kRows], uint16_t (&st)[2]) {
             if (active && sl < S)
                 load_task<kFmt>(wt, st, packed + (int64_t)sl * Fmt<kFmt>::kSliceBytes, scales, rb * kRows, N, G,
                                 (int64_t)sl * (kSliceK / kGroup) + (lane >> 3), row_bytes, lane_off, lane);
@@ -444,12 +435,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_rows_kernel(
 
 // ---------------------------------------------------------------- host side
 
-// Rows mode when every CTA gets enough row blocks to keep most warps busy per slice.
-// (PTQ1_0 tables cost ~3x more to build per slice, so PTQ1_0 always splits K.)
+// Rows mode (no split-K) is kept for measurement: with the split-K partials summed by a
+// second kernel, split mode is as fast or faster at every measured decode shape, so it
+// is the default.
 bool use_rows_mode(int64_t N, int64_t K, int fmt, const DeviceInfo &dev) {
-    if (fmt != 2 || K > kRowsModeMaxK || K / kSliceK < 2) return false;
-    const int64_t RB = (N + kRows - 1) / kRows;
-    return RB >= (int64_t)dev.sm_count * 12;
+    (void)N;
+    (void)K;
+    (void)fmt;
+    (void)dev;
+    return false;
 }
 
 // Split mode: rows of the weight matrix are split into `parts` ranges per K slice so that
@@ -467,13 +461,16 @@ int gemv_parts(int64_t N, int64_t K, const DeviceInfo &dev) {
 }
 
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args... args) {
-    cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (err != cudaSuccess) return err;
+cudaError_t launch_pdl_cfg(void (*kernel)(KArgs...), int grid, int threads, int smem, cudaStream_t s,
+                           Args... args) {
+    if (smem > 0) {
+        cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (err != cudaSuccess) return err;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -481,6 +478,26 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args.
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args... args) {
+    return launch_pdl_cfg(kernel, grid, kThreads, kSmemBytes, s, args...);
+}
+
+// Split mode: the slice kernel, then (K > 512) the in-order reduction of its partials.
+cudaError_t launch_split(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
+                         float *partials, int64_t N, int64_t K, int fmt, cudaStream_t s, const DeviceInfo &dev) {
+    const int parts = gemv_parts(N, K, dev);
+    const int64_t grid = (K / kSliceK) * parts;
+    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+    cudaError_t e = fmt == 1
+        ? launch_pdl(gemv_split_kernel<1>, (int)grid, s, x, packed, scales, y, partials, N, K, parts)
+        : launch_pdl(gemv_split_kernel<2>, (int)grid, s, x, packed, scales, y, partials, N, K, parts);
+    if (e != cudaSuccess || K / kSliceK == 1) return e;
+    const int64_t rgrid64 = (N + 255) / 256;
+    const int rgrid = (int)(rgrid64 < 4 * (int64_t)dev.sm_count ? rgrid64 : 4 * (int64_t)dev.sm_count);
+    return launch_pdl_cfg(gemv_reduce_kernel, rgrid, 256, 0, s, (const float *)partials, y, N, (int)(K / kSliceK));
 }
 
 }  // namespace
@@ -492,36 +509,40 @@ bool gemv_supported(int64_t M, int64_t N, int64_t K, int fmt) {
     return true;
 }
 
+// Schedule: split_k 0 = automatic, 1 = rows mode (when the shape allows it), >= 2 = split mode.
+bool pick_rows_mode(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev) {
+    if (split_k == 1) return K <= kRowsModeMaxK && K / kSliceK >= 2;
+    if (split_k >= 2) return false;
+    return use_rows_mode(N, K, fmt, dev);
+}
+
+int gemv_launches(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev) {
+    if (pick_rows_mode(N, K, fmt, split_k, dev) || K / kSliceK <= 1) return 1;
+    return 2;
+}
+
 size_t gemv_workspace_bytes(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev) {
-    (void)split_k;
     const int64_t S = K / kSliceK;
-    if (S <= 1 || use_rows_mode(N, K, fmt, dev)) return 0;
+    if (S <= 1 || pick_rows_mode(N, K, fmt, split_k, dev)) return 0;
     return (size_t)S * (size_t)N * sizeof(float);
 }
 
 cudaError_t launch_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                         uint16_t *y, int64_t N, int64_t K, int fmt, int split_k,
                         const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
-    (void)split_k;  // the schedule is chosen from the shape
     // the dynamic allocation must start below kTableAddr - kMiscBytes in the shared
     // window; it starts right after the per-block reserved area (no static shared memory)
     static int reserved = -1;
     if (reserved < 0 && cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, 0) != cudaSuccess)
         return cudaErrorUnknown;
     if (reserved + kMiscBytes > (int)kTableAddr) return cudaErrorNotSupported;
-    if (use_rows_mode(N, K, fmt, dev)) {
+    if (pick_rows_mode(N, K, fmt, split_k, dev)) {
         const int64_t RB = (N + kRows - 1) / kRows;
         const int grid = (int)(RB < dev.sm_count ? RB : dev.sm_count);
         if (fmt == 1) return launch_pdl(gemv_rows_kernel<1>, grid, s, x, packed, scales, y, N, K);
         return launch_pdl(gemv_rows_kernel<2>, grid, s, x, packed, scales, y, N, K);
     }
-    const int parts = gemv_parts(N, K, dev);
-    const int64_t grid = (K / kSliceK) * parts;
-    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-    float *partials = reinterpret_cast<float *>(ws.data);
-    if (fmt == 1)
-        return launch_pdl(gemv_split_kernel<1>, (int)grid, s, x, packed, scales, y, partials, ws.counters, N, K, parts);
-    return launch_pdl(gemv_split_kernel<2>, (int)grid, s, x, packed, scales, y, partials, ws.counters, N, K, parts);
+    return launch_split(x, packed, scales, y, reinterpret_cast<float *>(ws.data), N, K, fmt, s, dev);
 }
 
 // Split-mode launch with caller-provided scratch (counters and partials), whatever the
@@ -541,12 +562,8 @@ cudaError_t launch_gemv_split_scratch(const uint16_t *x, const uint8_t *packed, 
     if (reserved < 0 && cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, 0) != cudaSuccess)
         return cudaErrorUnknown;
     if (reserved + kMiscBytes > (int)kTableAddr) return cudaErrorNotSupported;
-    const int parts = gemv_parts(N, K, dev);
-    const int64_t grid = (K / kSliceK) * parts;
-    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-    if (fmt == 1)
-        return launch_pdl(gemv_split_kernel<1>, (int)grid, s, x, packed, scales, y, partials, counters, N, K, parts);
-    return launch_pdl(gemv_split_kernel<2>, (int)grid, s, x, packed, scales, y, partials, counters, N, K, parts);
+    (void)counters;  // the in-order reduction kernel needs no arrival counters
+    return launch_split(x, packed, scales, y, partials, N, K, fmt, s, dev);
 }
 
 }  // namespace bonsai

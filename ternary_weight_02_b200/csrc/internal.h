@@ -50,6 +50,7 @@ cudaError_t launch_linear_simple(const uint16_t *x, const uint8_t *packed, const
 // ---- gemv_lut.cu: M == 1
 bool gemv_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t gemv_workspace_bytes(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev);
+int gemv_launches(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev);
 cudaError_t launch_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                         uint16_t *y, int64_t N, int64_t K, int fmt, int split_k,
                         const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
