@@ -119,6 +119,22 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(ms: float, device=None) -> float:
+    """Max of a per-rank time over all ranks (the job's time); identity without a group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank_step: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: all ranks' bytes of one step over the slowest rank's step time."""
+    return world * bytes_per_rank_step / (ms_max * 1e-3) / 1e9
+
+
 def kernel_traffic(fmt):
     """DRAM bytes per gate/up launch from the committed ncu summary, if it was taken on
     the kernel source as it is now (matched by hash); else None."""
@@ -259,11 +275,8 @@ def run_ours(args):
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / args.steps
         clk = clocks.stop()
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        value = world * step_bytes(f) / (ms * 1e-3) / 1e9
+        ms = max_over_ranks(ms, dev)
+        value = whole_job_gbs(step_bytes(f), world, ms)
 
         # ---- dominant kernel (gate/up GEMV), 64 launches per replay
         with torch.cuda.stream(stream):
@@ -305,12 +318,8 @@ def run_ours(args):
                 e2e_step()
             e1.record(stream)
         torch.cuda.synchronize()
-        ms_e2e = e0.elapsed_time(e1) / args.steps
-        if world > 1:
-            t = torch.tensor([ms_e2e], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e2e = float(t.item())
-        e2e = world * step_bytes(f) / (ms_e2e * 1e-3) / 1e9
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+        e2e = whole_job_gbs(step_bytes(f), world, ms_e2e)
 
         launches_per_layer = sum(bz.bonsai_launch_count(1, N, K, f) for _, K, N in SHAPES)
         results[f] = {

@@ -1,0 +1,64 @@
+"""The multi-rank bench path on CPU: two gloo ranks, the job time is the max over
+ranks and the whole-job throughput counts every rank's bytes; the reference arm runs
+on rank 0 only."""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms = 2.0 + rank  # rank 1 is the slower one
+        m = bench.max_over_ranks(ms)
+        gbs = bench.whole_job_gbs(1_000_000, world, m)
+        q.put((rank, m, gbs))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_whole_job_value():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    out = sorted(q.get(timeout=5) for _ in range(2))
+    for rank, m, gbs in out:
+        assert m == 3.0  # the slowest rank's time, on every rank
+        assert abs(gbs - 2 * 1_000_000 / 3e-3 / 1e9) < 1e-9
+
+
+def test_single_process_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(4.5) == 4.5
+    assert abs(bench.whole_job_gbs(6_000_000_000, 1, 1.0) - 6000.0) < 1e-9
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                       env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == ""
