@@ -41,6 +41,10 @@ METRIC = "batch-1 ternary GEMV HBM GB/s (% of 8 TB/s); prefill GEMM TFLOPS (% pe
 SHAPES = [("qkv", 5120, 7168), ("o", 5120, 5120), ("gate_up", 5120, 34816), ("down", 17408, 5120)]
 LAYERS = 64
 FMT_NAMES = {1: "PTQ1_0", 2: "PQ2_0"}
+# the kernel a batch-1 call runs for each packing, and its source file
+DOM_KERNEL = {1: "lookup-table GEMV (gemv_split_kernel + in-order reduction)",
+              2: "integer tensor-core GEMV (gemv_imma_kernel)"}
+DOM_SOURCE = {1: "gemv_lut.cu", 2: "gemv_imma.cu"}
 
 
 def measured_peaks():
@@ -139,7 +143,7 @@ def kernel_traffic(fmt):
     """DRAM bytes per gate/up launch from the committed ncu summary, if it was taken on
     the kernel source as it is now (matched by hash); else None."""
     path = os.path.join(ROOT, "profiles", "gemv_traffic.json")
-    src = os.path.join(ROOT, "ternary_weight_02_b200", "csrc", "gemv_lut.cu")
+    src = os.path.join(ROOT, "ternary_weight_02_b200", "csrc", DOM_SOURCE[fmt])
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -352,7 +356,7 @@ def run_ours(args):
                 "frac_of_measured_hbm": round(r["value"] / hbm, 4), "parallelism": f"replicas x{world}",
             },
             "roofline": {
-                "bound": "hbm", "kernel": "gemv gate/up 5120->34816", "achieved": round(r["dom_gbs"], 1),
+                "bound": "hbm", "kernel": f"{DOM_KERNEL[fmt]}, gate/up 5120->34816", "achieved": round(r["dom_gbs"], 1),
                 "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(r["dom_gbs"] / hbm, 4),
                 "traffic": r["traffic"], "algorithmic_bytes_per_launch": r["dom_bytes"],
                 "avg_launch_us": round(r["dom_us"], 3),
@@ -448,7 +452,7 @@ def run_case(args):
     fmt = {"ptq1": 1, "pq2": 2}[args.fmt]
     i = [n for n, _, _ in SHAPES].index(args.shape)
     _, K, N = SHAPES[i]
-    M = 1 if args.case == "gemv" else args.m
+    M = 1 if args.case in ("gemv", "imma") else args.m
     dev = torch.device("cuda")
     t = torch.from_numpy(inputs.trits(i, N, K)).to(dev)
     packed = bz.pack(fmt, t)
@@ -456,7 +460,7 @@ def run_case(args):
     s = torch.from_numpy(inputs.scales(i, N, K).view(np.int16)).to(dev).view(torch.float16)
     x = torch.from_numpy(inputs.activations(i, M, K).view(np.int16)).to(dev).view(torch.float16)
     y = torch.empty((M, N), dtype=torch.float16, device=dev)
-    algo = bz.BONSAI_ALGO_GEMV if args.case == "gemv" else bz.BONSAI_ALGO_GEMM
+    algo = {"gemv": bz.BONSAI_ALGO_GEMV, "imma": bz.BONSAI_ALGO_IMMA, "gemm": bz.BONSAI_ALGO_GEMM}[args.case]
     bz.bonsai_reserve(M, N, K)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -480,7 +484,7 @@ def main():
     ap.add_argument("--both", type=int, default=1, help="also measure the other packing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-m", type=int, default=2048, help="tokens of the prefill GEMM line (0: skip)")
-    ap.add_argument("--case", choices=["gemv", "gemm"], help="run one projection only (profiler case)")
+    ap.add_argument("--case", choices=["gemv", "imma", "gemm"], help="run one projection only (profiler case)")
     ap.add_argument("--shape", choices=[n for n, _, _ in SHAPES], default="gate_up")
     ap.add_argument("--m", type=int, default=2048, help="tokens for --case gemm")
     ap.add_argument("--reps", type=int, default=3)

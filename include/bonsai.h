@@ -85,7 +85,8 @@ typedef enum {
     BONSAI_ALGO_SIMPLE = 1,  /* one warp per output row; any M (slow, plain)              */
     BONSAI_ALGO_GEMV = 2,    /* batch-1 lookup-table GEMV with split-K; M == 1 only       */
     BONSAI_ALGO_SKINNY = 3,  /* register-dequant tensor-core kernel; 1 <= M <= 16         */
-    BONSAI_ALGO_GEMM = 4     /* tcgen05/TMEM prefill GEMM on FP16 tiles; any M            */
+    BONSAI_ALGO_GEMM = 4,    /* tcgen05/TMEM prefill GEMM on FP16 tiles; any M            */
+    BONSAI_ALGO_IMMA = 5     /* batch-1 GEMV on the integer tensor cores; M == 1, PQ2_0   */
 } bonsai_algo;
 
 /* Library version, (major << 16) | (minor << 8) | patch. */
@@ -128,8 +129,12 @@ int bonsai_unpack(int fmt, const uint8_t *packed, int8_t *trits, int64_t N, int6
 int bonsai_hadamard128(const uint16_t *x, uint16_t *x_out, int64_t M, int64_t K, void *stream);
 
 /* y = x' . Wdeq^T (definitions above) for un-rotated FP16 x: the Hadamard
- * rotation of x is applied inside the call.  Dispatch on M: M == 1 -> GEMV,
- * 2 <= M <= 16 -> skinny tensor-core kernel, larger M -> tcgen05 GEMM.  y must
+ * rotation of x is applied inside the call.  Dispatch on M: M == 1 -> the
+ * integer tensor-core GEMV (PQ2_0, K <= 24576) or the lookup-table GEMV (PTQ1_0),
+ * 2 <= M <= 16 -> skinny tensor-core kernel, larger M -> tcgen05 GEMM.  The
+ * integer GEMV holds each 128-group of x' as 16-bit fixed point with a power-of-two
+ * scale (|x~| <= 2^14) before the exact integer products; the other kernels round
+ * x' to FP16 (GEMM, skinny) or keep it in FP32 (lookup tables, plain kernel).  y must
  * not overlap x, packed or scales.  Source of the operation: allhereai.com page,
  * method paragraph and packings paragraph. */
 int bonsai_ternary_linear(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
@@ -142,7 +147,8 @@ int bonsai_ternary_linear(const uint16_t *x, const uint8_t *packed, const uint16
  * 2 = 256 rows (two TMEM accumulators sharing each expanded weight tile), 0 =
  * automatic.  For BONSAI_ALGO_GEMV it picks the schedule: 1 = each CTA walks all K
  * slices of its rows (no split-K), >= 2 = one 512-wide K slice per CTA with split-K
- * partials, 0 = automatic.
+ * partials, 0 = automatic.  BONSAI_ALGO_IMMA ignores it (its work split is fixed
+ * by the shape and the SM count, so results are bitwise repeatable).
  * Returns BONSAI_ERR_ALGO if the chosen kernel cannot run the shape (e.g.
  * BONSAI_ALGO_GEMV with M > 1).  For measurement and testing of each kernel. */
 int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
@@ -150,8 +156,9 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
                                int split_k, void *stream);
 
 /* Number of kernels one bonsai_ternary_linear_algo call with these arguments launches
- * on the current device (the batch-1 GEMV: 1, or 2 when its split-K partials are
- * summed by a second kernel; the other kernels: 2, the rotation pass and the kernel),
+ * on the current device (the lookup-table GEMV: 1, or 2 when its split-K partials are
+ * summed by a second kernel; the integer tensor-core GEMV: 2, its rotation and
+ * quantisation of x, then the GEMV; the other kernels: 2, the rotation pass and the kernel),
  * or a negative bonsai_status.  Launches nothing. */
 int bonsai_launch_count(int64_t M, int64_t N, int64_t K, int fmt, int algo, int split_k);
 

@@ -35,6 +35,7 @@ BONSAI_ALGO_SIMPLE = 1
 BONSAI_ALGO_GEMV = 2
 BONSAI_ALGO_SKINNY = 3
 BONSAI_ALGO_GEMM = 4
+BONSAI_ALGO_IMMA = 5
 
 FORMATS = {"ptq1": BONSAI_FMT_PTQ1_0, "pq2": BONSAI_FMT_PQ2_0}
 

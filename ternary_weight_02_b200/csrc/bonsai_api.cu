@@ -112,6 +112,7 @@ int cuda_status(cudaError_t e) {
 // Picks the kernel for AUTO, or checks an explicit choice.
 int resolve_algo(int algo, int64_t M, int64_t N, int64_t K, int fmt) {
     if (algo == BONSAI_ALGO_AUTO) {
+        if (M == 1 && gemv_imma_supported(M, N, K, fmt)) return BONSAI_ALGO_IMMA;
         if (M == 1 && gemv_supported(M, N, K, fmt)) return BONSAI_ALGO_GEMV;
         if (M <= 16 && skinny_supported(M, N, K, fmt)) return BONSAI_ALGO_SKINNY;
         if (gemm_supported(M, N, K, fmt)) return BONSAI_ALGO_GEMM;
@@ -122,6 +123,7 @@ int resolve_algo(int algo, int64_t M, int64_t N, int64_t K, int fmt) {
         case BONSAI_ALGO_GEMV: return gemv_supported(M, N, K, fmt) ? algo : BONSAI_ERR_ALGO;
         case BONSAI_ALGO_SKINNY: return skinny_supported(M, N, K, fmt) ? algo : BONSAI_ERR_ALGO;
         case BONSAI_ALGO_GEMM: return gemm_supported(M, N, K, fmt) ? algo : BONSAI_ERR_ALGO;
+        case BONSAI_ALGO_IMMA: return gemv_imma_supported(M, N, K, fmt) ? algo : BONSAI_ERR_ALGO;
         default: return BONSAI_ERR_ALGO;
     }
 }
@@ -132,6 +134,7 @@ size_t workspace_for(int algo, int64_t M, int64_t N, int64_t K, int fmt, int spl
         case BONSAI_ALGO_GEMV: return gemv_workspace_bytes(N, K, fmt, split_k, info);
         case BONSAI_ALGO_SKINNY: return skinny_workspace_bytes(M, N, K, fmt, split_k, info);
         case BONSAI_ALGO_GEMM: return gemm_workspace_bytes(M, N, K, fmt);
+        case BONSAI_ALGO_IMMA: return gemv_imma_workspace_bytes(N, K);
         default: return simple_workspace_bytes(M, N, K);
     }
 }
@@ -281,6 +284,9 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
         case BONSAI_ALGO_GEMM:
             e = launch_gemm(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, st->info);
             break;
+        case BONSAI_ALGO_IMMA:
+            e = launch_gemv_imma(x, packed, scales, y, N, K, ws, s, st->info);
+            break;
         default:
             e = launch_linear_simple(x, packed, scales, y, M, N, K, fmt, ws, s, st->info);
             break;
@@ -309,6 +315,7 @@ int bonsai_launch_count(int64_t M, int64_t N, int64_t K, int fmt, int algo, int 
     if (rc != BONSAI_OK) return rc;
     switch (chosen) {
         case BONSAI_ALGO_GEMV: return gemv_launches(N, K, fmt, split_k, st->info);
+        case BONSAI_ALGO_IMMA: return 2;  // x -> x~ fragments, then the GEMV
         default: return 2;  // the rotation pass, then the kernel
     }
 }
@@ -326,6 +333,10 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
         size_t v;
         if (M <= 1 && gemv_supported(1, N, K, fmt)) {
             v = gemv_workspace_bytes(N, K, fmt, 0, st->info);
+            need = v > need ? v : need;
+        }
+        if (M <= 1 && gemv_imma_supported(1, N, K, fmt)) {
+            v = gemv_imma_workspace_bytes(N, K);
             need = v > need ? v : need;
         }
         if (skinny_supported(M < 16 ? M : 16, N, K, fmt)) {

@@ -1,0 +1,557 @@
+// gemv_imma.cu -- batch-1 (M == 1) ternary GEMV for PQ2_0 on the integer tensor cores,
+// with the block Hadamard rotation of x fused in.
+//
+// Operation: y[n] = sum_g s[n][g] * sum_j t[n][128g+j] * x'[128g+j], x' = blockdiag(Hn) x.
+// Sources: "27B 模型压到 5.95GB，推理能力还保住 98%" (allhereai.com): method paragraph
+// (trits, FP16 scale per 128 weights, block Hadamard), paragraph on running the files
+// (activation-side Hadamard), paragraph on the two packings (PQ2_0: one trit per 2-bit
+// slot); "Bonsai 2，把27B压进6个G" (10100.com), section 它怎么做到的.
+//
+// Design (B200, HBM-bound: 34 bytes per 128 weights):
+//
+// * At ~6.5 TB/s an SM must take in ~22 weight bytes per clock.  mma.sync issues at
+//   ~0.38 per clock per SM on this part, so one MMA has to cover well over 64 bytes.
+//   The u8 x s8 m16n8k32 MMA covers 16 rows x 32 weights = 128 bytes once its eight
+//   columns are used for (4 scale groups) x (high byte, low byte) of the activations:
+//   the weights of group gl meet a B operand that is non-zero in columns 2gl, 2gl+1
+//   only, so four groups accumulate side by side in one fragment.
+// * Activations as 16-bit block fixed point.  Per 128-group, x~ = rint(x' * 2^e) with
+//   the power of two chosen so that |x~| <= 2^14, stored as signed bytes hi * 256 + lo.
+//   With c = t + 1 the PQ2_0 code of a weight, the MMA gives sum c*hi and sum c*lo
+//   exactly in int32, so sum t*x~ = 256*Dhi + Dlo - sum x~ exactly; one FP32 multiply by
+//   s * 2^-e per (row, group) follows.  (The rounding of x' to x~ is the only
+//   approximation; it is finer than FP16 for every element of the group.)
+// * Two launches, chained with programmatic dependent launch:
+//   1. gemv_imma_prep_kernel rotates and quantises x once (8 lanes per group) into
+//      the fragment order the MMAs read, in the workspace;
+//   2. gemv_imma_kernel: 16 warps per CTA, each feeding its own ring of item buffers
+//      (a TMA box of trits, and the item's scale words by cp.async).  The first item
+//      of every warp is requested before waiting for the previous kernel; the x~
+//      fragments are copied next, ahead of the remaining weight traffic.
+// * Decode.  A 32-bit weight word holds 16 codes; (w >> 2j) & 0x03030303 is code j of
+//   its four bytes as four u8 lanes of an A register.  The three shifts are done as
+//   multiply-high by 2^(32-2j) (FMA pipe), the masks on the ALU pipe.
+// * A work item is 32 rows x 512 weights: one TMA box of the trit plane (4 KB, 128-byte
+//   swizzle).  MMA row gid reads shared-memory row 2*gid (gid < 4) or 2*gid - 7, so
+//   that the eight rows one 64-bit load touches fall in distinct swizzle phases (no
+//   bank conflicts).
+// * Work split.  Items are ordered (row tile, K chunk); each CTA takes one contiguous
+//   range, dealt round-robin to its consumer warps.  Every item's 32 row sums go to a
+//   slot in shared memory; at the end each row tile's slots are added in K order.  A
+//   tile shared with a neighbouring CTA goes through FP32 partials in the workspace:
+//   the CTA whose arrival completes the tile adds the pieces in K order (deterministic)
+//   and resets the tile's counter to zero for the next call.
+// * Every mbarrier wait is bounded.  A warp whose wait gives up stops refilling, turns
+//   its results into NaN (keeping the partial-sum protocol intact) and, before the
+//   CTA exits, waits (again bounded) for the copies it had started.
+#include "common.cuh"
+#include "internal.h"
+#include "tma.cuh"
+
+namespace bonsai {
+namespace {
+
+constexpr int kConsumers = 16;                          // warps; each feeds its own ring
+constexpr int kThreads = kConsumers * 32;
+constexpr int kItemRows = 32;
+constexpr int kItemK = 512;
+constexpr int kItemRowBytes = kItemK / 4;               // 128 bytes of PQ2_0 codes
+constexpr int kItemBytes = kItemRows * kItemRowBytes;   // 4096
+constexpr int kScaleRingBytes = kItemRows * 8;          // per stage: the item's 4 scales of each row
+constexpr int kXHalfBytes = 144;                        // one part (hi or lo) of a group's fragments, padded
+constexpr int kXGroupBytes = 2 * kXHalfBytes;
+constexpr int kStages = 2;
+constexpr int kPreStages = 1;                           // issued before the wait on the previous kernel
+constexpr int kMaxCtaItems = 160;                       // slot buffer: 160 x 32 floats
+constexpr int64_t kMaxK = 24576;  // the layout below then fits the 227 KB a CTA may use
+constexpr uint32_t kCodeMask = 0x03030303u;
+
+// Shared memory, from a 1024-byte aligned base (each 4 KB weight buffer stays 1024-byte
+// aligned, as the 128-byte swizzle of its TMA box requires):
+// [weight rings: kConsumers x kStages x 4096][scale rings: kConsumers x kStages x 256]
+// [x~ fragments G4 x 288][(64 sum x~, 2^-e / 64) x G4][slots kMaxCtaItems x 128][256 zero bytes]
+// [full barriers][x barrier]
+struct Layout {
+    int sring, xfrag, sxf, slots, zero, full, xbar, total;
+};
+
+__host__ __device__ inline Layout make_layout(int K) {
+    Layout L;
+    const int G4 = ((K + kItemK - 1) / kItemK) * 4;
+    L.sring = kConsumers * kStages * kItemBytes;
+    L.xfrag = L.sring + kConsumers * kStages * kScaleRingBytes;
+    L.sxf = L.xfrag + G4 * kXGroupBytes;
+    L.slots = L.sxf + G4 * 8;
+    L.zero = L.slots + kMaxCtaItems * kItemRows * 4;
+    L.full = L.zero + 256;
+    L.xbar = L.full + kConsumers * kStages * 8;
+    L.total = L.xbar + 8 + 1024;  // + room to align the base
+    return L;
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(saddr(dst)), "l"(src), "r"(bytes), "r"(saddr(bar))
+        : "memory");
+}
+
+
+// D += A * B, A 16 x 32 u8 (row-major fragments), B 32 x 8 s8, D int32.
+__device__ __forceinline__ void imma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                     uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------- 1. x -> x~ fragments
+
+// Eight lanes per 128-group, four groups per warp; lane l (0..7) of a group holds
+// elements k = 16l + m, m = 0..15.  Fragment layout of group g, part p (0: high byte,
+// 1: low byte), B-operand slot (s, j) of the MMA that meets code slot j of the weights'
+// 8-byte subslot s: element k = 32*s + 16*hb + 4*i + j is byte (8*(j & 1) + 4*hb + i) of
+// 16-byte chunk 2*s + (j >> 1) in the 144-byte half-block (2g + p).  The 16 bytes of
+// padding per half-block put the eight lanes that load one chunk of four consecutive
+// groups on distinct shared-memory banks.  Lane l = 2*s + hb writes whole words.
+__global__ void __launch_bounds__(128) gemv_imma_prep_kernel(const uint16_t *__restrict__ x,
+                                                             uint8_t *__restrict__ xfrag, int2 *__restrict__ sxf,
+                                                             int K) {
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int l = lane & 7;
+    const int g = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + (lane >> 3);
+    const int G = K / kGroup;
+    const int G4 = ((K + kItemK - 1) / kItemK) * 4;
+    pdl_wait();  // x and the fragment buffer may belong to the previous kernel
+    if (g >= G4) return;  // whole 8-lane groups leave together (G4 is a multiple of 4)
+    const unsigned int gmask = 0xffu << (lane & 24);
+    float v[16];
+    if (g < G) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)g * kGroup + 16 * l);
+        const uint4 r0 = src[0], r1 = src[1];
+        const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
+            v[2 * i] = f.x;
+            v[2 * i + 1] = f.y;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; i++) v[i] = 0.f;
+    }
+    // index bits 0..3 inside the lane
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 16; i++)
+            if ((i & h) == 0) {
+                const float a = v[i], b = v[i + h];
+                v[i] = a + b;
+                v[i + h] = a - b;
+            }
+    // index bits 4..6 are lane bits 0..2
+#pragma unroll
+    for (int b = 0; b < 3; b++) {
+        const int mask = 1 << b;
+        const bool upper = (l & mask) != 0;
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            const float p = __shfl_xor_sync(gmask, v[i], mask);
+            v[i] = upper ? (p - v[i]) : (v[i] + p);
+        }
+    }
+    float am = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        v[i] *= kHadamardNorm;
+        am = fmaxf(am, fabsf(v[i]));
+    }
+#pragma unroll
+    for (int b = 1; b < 8; b <<= 1) am = fmaxf(am, __shfl_xor_sync(gmask, am, b));
+    const uint32_t mb = __float_as_uint(am);
+    const int E = (int)(mb >> 23) - 127;  // am < 2^(E+1)
+    int e = mb == 0u ? 0 : 13 - E;        // am * 2^e < 2^14
+    e = e < -126 ? -126 : (e > 100 ? 100 : e);
+    const float sc = __int_as_float((e + 127) << 23);
+    // 2^-e / 64: the GEMV's sums come out 64 times too large (code slots weighted 4^(3-j))
+    const float f = E == 128 ? __int_as_float(0x7fc00000) : __int_as_float((121 - e) << 23);  // Inf/NaN -> NaN
+    int q[16];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < 16; i++) {
+        q[i] = __float2int_rn(v[i] * sc);
+        sum += q[i];
+    }
+#pragma unroll
+    for (int b = 1; b < 8; b <<= 1) sum += __shfl_xor_sync(gmask, sum, b);
+    // lane l = 2s + hb: chunk 2s + (j >> 1), byte 8 (j & 1) + 4 hb + i
+    uint8_t *dst = xfrag + (int64_t)g * kXGroupBytes + (l >> 1) * 32 + (l & 1) * 4;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        uint32_t whi = 0u, wlo = 0u;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int qq = q[4 * i + j];
+            const int hi = (qq + 128) >> 8;
+            const int lo = qq - (hi << 8);
+            whi |= ((uint32_t)hi & 0xffu) << (8 * i);
+            wlo |= ((uint32_t)lo & 0xffu) << (8 * i);
+        }
+        const int off = (j >> 1) * 16 + (j & 1) * 8;
+        *reinterpret_cast<uint32_t *>(dst + off) = whi;
+        *reinterpret_cast<uint32_t *>(dst + kXHalfBytes + off) = wlo;
+    }
+    if (l == 0) sxf[g] = make_int2(sum * 64, __float_as_int(f));
+}
+
+// ---------------------------------------------------------------- 2. the GEMV
+
+__device__ __forceinline__ void cp_async8(void *dst, const void *src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(saddr(dst)), "l"(src), "r"(valid ? 8 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// kAsyncScales: K is a multiple of 512, so an item's four scales of a row are 8 aligned
+// bytes, copied with cp.async as part of the item's copy; otherwise each lane loads the
+// scales it needs when it processes the item.
+template <bool kAsyncScales>
+__global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
+    const __grid_constant__ CUtensorMap wmap, const uint8_t *__restrict__ xprep, const uint16_t *__restrict__ scales,
+    uint16_t *__restrict__ y, float *__restrict__ partials, unsigned int *__restrict__ counters, int N, int K,
+    uint32_t mul2, uint32_t mul4, uint32_t mul6) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int gid = lane >> 2, tig = lane & 3;
+    const Layout L = make_layout(K);
+    const int G = K / kGroup;
+    const int KC = (K + kItemK - 1) / kItemK;
+    const int G4 = KC * 4;
+    const int RT = (N + kItemRows - 1) / kItemRows;
+    const int I = RT * KC;  // items (host-checked to fit)
+    const int C = gridDim.x;
+    const int c0 = (int)((int64_t)I * blockIdx.x / C), c1 = (int)((int64_t)I * (blockIdx.x + 1) / C);
+    const int nq = c1 - c0 > warp ? (c1 - c0 - warp + kConsumers - 1) / kConsumers : 0;  // this warp's items
+
+    uint8_t *wring = smem + warp * kStages * kItemBytes;
+    uint8_t *sring = smem + L.sring + warp * kStages * kScaleRingBytes;  // [stage][item row][4 scales]
+    uint8_t *xf = smem + L.xfrag;
+    const int2 *sxf = reinterpret_cast<const int2 *>(smem + L.sxf);
+    float *slots = reinterpret_cast<float *>(smem + L.slots);
+    uint8_t *zero = smem + L.zero;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full) + warp * kStages;
+    uint64_t *xbar = reinterpret_cast<uint64_t *>(smem + L.xbar);
+
+    // item q of this warp: c0 + warp + q * kConsumers -> ring stage q % kStages.  Lane 0
+    // starts the TMA box; lane r copies the item's four scales of row r (cp.async); one
+    // cp.async group per item (empty past the end) keeps the group count in step.
+    // (row tile, K chunk) of an item, advanced by kConsumers items per step
+    const int step_rt = kConsumers / KC, step_kc = kConsumers - step_rt * KC;
+    auto advance = [&](int &rt, int &kc) {
+        kc += step_kc;
+        rt += step_rt;
+        if (kc >= KC) kc -= KC, rt++;
+    };
+    int n_issued = 0;
+    int i_rt = (c0 + warp) / KC, i_kc = (c0 + warp) - ((c0 + warp) / KC) * KC;  // next item to issue
+    auto issue = [&](int q) {
+        if (q < nq) {
+            const int rt = i_rt, kc = i_kc;
+            advance(i_rt, i_kc);
+            const int st = q % kStages;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(full + st, kItemBytes);
+                tma_load_2d(wring + st * kItemBytes, &wmap, full + st, kc * kItemRowBytes, rt * kItemRows);
+            }
+            if (kAsyncScales) {
+                const int row = rt * kItemRows + lane;
+                const bool v = row < N;
+                cp_async8(sring + st * kScaleRingBytes + lane * 8, scales + (v ? (int64_t)row * G + kc * 4 : 0), v);
+            }
+            n_issued++;
+        }
+        if (kAsyncScales) cp_async_commit();
+    };
+
+    if (lane == 0) {
+        for (int st = 0; st < kStages; st++) mbar_init(full + st, 1);
+        if (tid == 0) mbar_init(xbar, 1);
+        mbar_init_fence();
+    }
+    if (tid < 64) reinterpret_cast<uint32_t *>(zero)[tid] = 0u;
+    __syncthreads();
+    // weights and scales do not depend on the previous kernel: start some before waiting
+    for (int q = 0; q < kPreStages; q++) issue(q);
+    pdl_launch_dependents();
+    pdl_wait();  // the x~ fragments come from the prep kernel
+    if (tid == 0) {  // before the remaining weight copies, so that it is not queued behind them
+        mbar_arrive_expect_tx(xbar, (uint32_t)G4 * (kXGroupBytes + 8));
+        bulk_load(xf, xprep, (uint32_t)G4 * (kXGroupBytes + 8), xbar);
+    }
+    __syncthreads();
+    for (int q = kPreStages; q < kStages; q++) issue(q);
+
+    // Lane (gid, tig) works on scale group tig of the item: MMA rows gid and gid + 8 of
+    // each 16-row tile t are shared-memory rows r = 16t + gid (+ 8), whose group tig is
+    // logical 16-byte chunks 2tig and 2tig + 1, stored at chunk ^ (r & 7) = chunk ^ gid.
+    const uint32_t loff0 = (uint32_t)(gid * kItemRowBytes + (((2 * tig) ^ gid) << 4));
+    const uint32_t loff1 = (uint32_t)(gid * kItemRowBytes + (((2 * tig + 1) ^ gid) << 4));
+    // B columns 2gq, 2gq + 1 carry group gq's high and low bytes; lane (gid, tig) supplies
+    // column gid for the k of lane quad tig, i.e. group tig: non-zero iff gid >> 1 == tig.
+    const bool bactive = (gid >> 1) == tig;
+    const uint8_t *xb_lane = bactive ? xf + (2 * tig + (gid & 1)) * kXHalfBytes : zero;
+    const int xb_stride = bactive ? kXGroupBytes : 0;
+    const int R = 8 * tig + gid;  // the item row this lane reports: (t, h) = (tig >> 1, tig & 1)
+
+    bool ok = __all_sync(0xffffffffu, mbar_wait(xbar, 0));
+    int n_waited = 0;
+    int st = 0;
+    uint32_t phase = 0;
+    int rt = (c0 + warp) / KC, kc = (c0 + warp) - ((c0 + warp) / KC) * KC;
+    for (int q = 0; q < nq; q++) {
+        const int i = c0 + warp + q * kConsumers;
+        if (ok) {
+            ok = __all_sync(0xffffffffu, mbar_wait(full + st, phase));
+            if (ok) n_waited++;
+        }
+        const uint8_t *sb = wring + st * kItemBytes;
+        uint4 raw[2][2][2];  // [t][h][16-byte half of the lane's 32 bytes]
+#pragma unroll
+        for (int t = 0; t < 2; t++)
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                raw[t][h][0] = *reinterpret_cast<const uint4 *>(sb + loff0 + 2048 * t + 1024 * h);
+                raw[t][h][1] = *reinterpret_cast<const uint4 *>(sb + loff1 + 2048 * t + 1024 * h);
+            }
+        const int g0 = kc * 4;
+        uint32_t sc[4];  // (t, h) = (e >> 1, e & 1): scale of row 16t + 8h + gid, group g0 + tig
+        if (kAsyncScales) {
+            cp_async_wait<kStages - 1>();  // this item's scales have landed (own copies)
+            __syncwarp();                  // ... and every lane's
+            const uint8_t *sp = sring + st * kScaleRingBytes + gid * 8 + tig * 2;
+#pragma unroll
+            for (int e = 0; e < 4; e++) sc[e] = *reinterpret_cast<const uint16_t *>(sp + e * 64);
+        } else {
+            const int g = g0 + tig;
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const int row = rt * kItemRows + 8 * e + gid;
+                sc[e] = (row < N && g < G) ? (uint32_t)__ldg(scales + (int64_t)row * G + g) : 0u;
+            }
+        }
+        __syncwarp();
+        if (ok) {  // refill this buffer with the warp's item q + kStages
+            if (lane == 0) fence_proxy_async();
+            issue(q + kStages);
+        } else if (kAsyncScales) {
+            cp_async_commit();
+        }
+
+        // Codes stay in place: (w & 0x03030303 << 2j) gives code slot j of the four bytes of
+        // a word as u8 values c * 4^j.  One accumulator per (tile, j); the 4^j factors are
+        // undone once per item (the sums come out 64 times too large, folded into 2^-e).
+        int d[2][4][4];
+#pragma unroll
+        for (int t = 0; t < 2; t++)
+#pragma unroll
+            for (int j = 0; j < 4; j++)
+#pragma unroll
+                for (int e = 0; e < 4; e++) d[t][j][e] = 0;
+        const uint8_t *xb = xb_lane + g0 * xb_stride;
+#pragma unroll
+        for (int s = 0; s < 4; s++) {
+            const uint4 b01 = *reinterpret_cast<const uint4 *>(xb + 32 * s);       // code slots 0, 1
+            const uint4 b23 = *reinterpret_cast<const uint4 *>(xb + 32 * s + 16);  // code slots 2, 3
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const uint32_t mask = kCodeMask << (2 * j);
+                const uint32_t bx = j == 0 ? b01.x : (j == 1 ? b01.z : (j == 2 ? b23.x : b23.z));
+                const uint32_t by = j == 0 ? b01.y : (j == 1 ? b01.w : (j == 2 ? b23.y : b23.w));
+#pragma unroll
+                for (int t = 0; t < 2; t++) {
+                    // subslot s: bytes 8s..8s+7 of the group; a0/a2 = row gid bytes 0-3 / 4-7, a1/a3 = row gid + 8
+                    const uint4 &r0 = raw[t][0][s >> 1], &r1 = raw[t][1][s >> 1];
+                    const uint32_t w0 = (s & 1) ? r0.z : r0.x, w2 = (s & 1) ? r0.w : r0.y;
+                    const uint32_t w1 = (s & 1) ? r1.z : r1.x, w3 = (s & 1) ? r1.w : r1.y;
+                    imma(d[t][j], w0 & mask, w1 & mask, w2 & mask, w3 & mask, bx, by);
+                }
+            }
+        }
+        // lane (gid, tig) holds columns 2tig (hi) and 2tig+1 (lo): group g0 + tig of rows
+        // gid (d[t][j][0..1]) and gid + 8 (d[t][j][2..3])
+        const int2 sf = sxf[g0 + tig];  // (64 * sum x~, 2^-e / 64)
+        const float fg = __int_as_float(sf.y);
+        float v[4];  // (t, h) = (e >> 1, e & 1)
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+            const int t = e >> 1, h = e & 1;
+            const int H = ((d[t][0][2 * h] * 4 + d[t][1][2 * h]) * 4 + d[t][2][2 * h]) * 4 + d[t][3][2 * h];
+            const int Lo = ((d[t][0][2 * h + 1] * 4 + d[t][1][2 * h + 1]) * 4 + d[t][2][2 * h + 1]) * 4 +
+                           d[t][3][2 * h + 1];
+            const int T64 = H * 256 + Lo - sf.x;
+            v[e] = (float)T64 * (half_bits_to_float((uint16_t)sc[e]) * fg);
+        }
+        // sum over the four groups (lanes of the quad) and leave (t, h) = (tig >> 1, tig & 1)
+        // in lane tig: keep the pair whose h is the lane's, then the t
+        {
+            const bool b0 = tig & 1;
+            const float k0 = b0 ? v[1] : v[0], s0 = b0 ? v[0] : v[1];
+            const float k1 = b0 ? v[3] : v[2], s1 = b0 ? v[2] : v[3];
+            const float u0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 1);  // t = 0
+            const float u1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 1);  // t = 1
+            const bool b1 = tig & 2;
+            const float kk = b1 ? u1 : u0, ss = b1 ? u0 : u1;
+            v[0] = kk + __shfl_xor_sync(0xffffffffu, ss, 2);
+        }
+        float mine = v[0];
+        if (!ok) mine = __int_as_float(0x7fc00000);
+        slots[(i - c0) * kItemRows + R] = mine;
+        if (++st == kStages) st = 0, phase ^= 1u;
+        advance(rt, kc);
+    }
+    if (kAsyncScales) cp_async_wait_all();
+    // after a wait gave up: let the box copies already started land before the CTA exits
+    if (!ok && lane == 0) {
+        int dst = n_waited % kStages;
+        uint32_t dph = (uint32_t)((n_waited / kStages) & 1);
+        for (int q = n_waited; q < n_issued; q++) {
+            mbar_wait(full + dst, dph);
+            if (++dst == kStages) dst = 0, dph ^= 1u;
+        }
+    }
+    __syncthreads();  // every slot is written
+
+    // ---- row tiles: add each tile's items in K order; tiles shared with a neighbouring
+    // CTA go through the workspace partials (one warp per tile, one lane per row)
+    const int rt_first = c0 / KC, rt_last = c1 > c0 ? (c1 - 1) / KC : rt_first - 1;
+    for (int rt = rt_first + warp; rt <= rt_last; rt += kConsumers) {
+        const int tile_first = rt * KC, tile_end = tile_first + KC;
+        const int a = c0 > tile_first ? c0 : tile_first;
+        const int b = c1 < tile_end ? c1 : tile_end;
+        float sum = 0.f;
+        for (int i = a; i < b; i++) sum += slots[(i - c0) * kItemRows + lane];
+        const int row = rt * kItemRows + lane;
+        if (a == tile_first && b == tile_end) {
+            if (row < N) y[row] = float_to_half_bits(sum);
+            continue;
+        }
+        partials[(int64_t)a * kItemRows + lane] = sum;
+        __threadfence();
+        __syncwarp();
+        const unsigned int cover = (unsigned int)(b - a);
+        unsigned int old = 0u;
+        if (lane == 0) old = atomicAdd(counters + rt, cover);
+        old = __shfl_sync(0xffffffffu, old, 0);
+        if (old + cover != (unsigned int)KC) continue;
+        __threadfence();  // this CTA completes the tile: add the pieces in K order
+        float total = 0.f;
+        int s = tile_first;
+        while (s < tile_end) {
+            // the CTA whose range holds item s, and where its range ends
+            const int c2 = (int)(((int64_t)(s + 1) * C - 1) / I);
+            int e2 = (int)((int64_t)I * (c2 + 1) / C);
+            e2 = e2 < tile_end ? e2 : tile_end;
+            total += c2 == (int)blockIdx.x ? sum : __ldcg(partials + (int64_t)s * kItemRows + lane);
+            s = e2;
+        }
+        if (row < N) y[row] = float_to_half_bits(total);
+        if (lane == 0) counters[rt] = 0u;
+    }
+}
+
+struct Shape {
+    int KC, G4, RT, I, grid;
+};
+
+Shape shape_of(int64_t N, int64_t K, int sm_count) {
+    Shape s;
+    s.KC = (int)((K + kItemK - 1) / kItemK);
+    s.G4 = s.KC * 4;
+    s.RT = (int)((N + kItemRows - 1) / kItemRows);
+    s.I = s.RT * s.KC;
+    int64_t grid = (s.I + kMaxCtaItems - 1) / kMaxCtaItems;  // every CTA's slots fit
+    const int64_t want = (s.I + kConsumers - 1) / kConsumers;  // no idle consumer warps
+    int64_t g2 = want < sm_count ? want : sm_count;
+    if (grid < g2) grid = g2;
+    s.grid = (int)grid;
+    return s;
+}
+
+}  // namespace
+
+static_assert(kConsumers * kStages * (kItemBytes + kScaleRingBytes) + (kMaxK / kItemK) * 4 * (kXGroupBytes + 8) +
+                  kMaxCtaItems * kItemRows * 4 + 256 + kConsumers * kStages * 8 + 8 + 1024 <= 232448,
+              "shared-memory layout exceeds the per-CTA limit at the largest K");
+
+bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt) {
+    if (fmt != 2 || M != 1 || N < 1 || K < kGroup || K % kGroup != 0 || K > kMaxK) return false;
+    const int64_t RT = (N + kItemRows - 1) / kItemRows;
+    return RT <= kMaxTiles && RT * ((K + kItemK - 1) / kItemK) < ((int64_t)1 << 30);
+}
+
+// workspace: [x~ fragments G4 x 256][(sum, 2^-e) x G4][pad to 256][partials: items x 32 floats]
+size_t gemv_imma_workspace_bytes(int64_t N, int64_t K) {
+    const int64_t KC = (K + kItemK - 1) / kItemK;
+    const int64_t items = ((N + kItemRows - 1) / kItemRows) * KC;
+    const size_t xbytes = ((size_t)(KC * 4) * (kXGroupBytes + 8) + 255) / 256 * 256;
+    return xbytes + (size_t)items * kItemRows * sizeof(float);
+}
+
+cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
+                             int64_t N, int64_t K, const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
+    const Layout lay = make_layout((int)K);
+    if (lay.total > dev.smem_optin) return cudaErrorInvalidValue;
+    EncodeTiledFn encode = encode_fn();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap wmap;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
+        const cuuint64_t strides[1] = {(cuuint64_t)(K / 4)};
+        const cuuint32_t box[2] = {kItemRowBytes, kItemRows};
+        const cuuint32_t estr[2] = {1, 1};
+        if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    const Shape sh = shape_of(N, K, dev.sm_count);
+    uint8_t *xprep = ws.data;
+    int2 *sxf = reinterpret_cast<int2 *>(xprep + (size_t)sh.G4 * kXGroupBytes);
+    float *partials = reinterpret_cast<float *>(
+        ws.data + ((size_t)sh.G4 * (kXGroupBytes + 8) + 255) / 256 * 256);
+
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // 1. x -> x~ fragments: four groups per warp, four warps per CTA
+    cfg.gridDim = dim3((unsigned)((sh.G4 + 15) / 16));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_imma_prep_kernel, x, xprep, sxf, (int)K);
+    if (e != cudaSuccess) return e;
+    // 2. the GEMV
+    // K a multiple of 512: an item's scales of a row are 8 aligned bytes, copied with the item
+    auto kern = K % kItemK == 0 ? gemv_imma_kernel<true> : gemv_imma_kernel<false>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3((unsigned)sh.grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = lay.total;
+    return cudaLaunchKernelEx(&cfg, kern, wmap, (const uint8_t *)xprep, scales, y, partials, ws.counters,
+                              (int)N, (int)K, 1u << 30, 1u << 28, 1u << 26);
+}
+
+}  // namespace bonsai

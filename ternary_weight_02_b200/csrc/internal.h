@@ -64,6 +64,12 @@ cudaError_t launch_gemv_split_scratch(const uint16_t *x, const uint8_t *packed, 
 // current device's properties (the same probe the other entry points use)
 int current_device_info(DeviceInfo *out);
 
+// ---- gemv_imma.cu: M == 1, PQ2_0, integer tensor cores
+bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt);
+size_t gemv_imma_workspace_bytes(int64_t N, int64_t K);
+cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
+                             int64_t N, int64_t K, const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
+
 // ---- skinny_mma.cu: 1 <= M <= 16
 bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t skinny_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int split_k,

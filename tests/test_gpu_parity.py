@@ -174,13 +174,13 @@ def test_gemv_decode_shapes_full(bz, fmt, K, N):
     got = _run(bz, p, bz.BONSAI_ALGO_GEMV)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
-    # through the default entry point too (M == 1 dispatches to this kernel)
-    import torch
-    x, packed, scales = p.device()
-    y = torch.empty((1, N), dtype=torch.float16, device="cuda")
-    bz.bonsai_ternary_linear(x, packed, scales, y, 1, N, K, fmt)
-    torch.cuda.synchronize()
-    assert np.array_equal(to_numpy_f16(y), got)
+    if fmt == PTQ1:  # through the default entry point too (M == 1 PTQ1_0 dispatches here)
+        import torch
+        x, packed, scales = p.device()
+        y = torch.empty((1, N), dtype=torch.float16, device="cuda")
+        bz.bonsai_ternary_linear(x, packed, scales, y, 1, N, K, fmt)
+        torch.cuda.synchronize()
+        assert np.array_equal(to_numpy_f16(y), got)
 
 
 @pytest.mark.parametrize("fmt", [PTQ1, PQ2])
@@ -213,6 +213,90 @@ def test_gemv_rejects_batches(bz):
     w = torch.zeros((8, 128), dtype=torch.uint8, device="cuda")
     with pytest.raises(bz.BonsaiError):
         bz.bonsai_ternary_linear_algo(x, w, s, y, 2, 8, 512, PQ2, bz.BONSAI_ALGO_GEMV)
+
+
+# ------------------------------------------------------------ batch-1 GEMV (integer tensor cores)
+
+# ragged N (not a multiple of the 32-row item) and ragged K (not a multiple of the
+# 512-weight item), one item, many items, the largest K the kernel takes
+IMMA_CASES = [(1, 128), (33, 384), (31, 640), (100, 1024), (1024, 1024), (1000, 2048), (5000, 1152),
+              (37, 17408), (70, 24576),
+              # enough items that every consumer warp walks its ring several times, with
+              # ragged N / K, and K not a multiple of 1024 (scales loaded without TMA)
+              (6000, 6144), (4099, 8192), (9000, 2560), (4000, 9728),
+              # more items per warp than ring buffers: the producer waits for released buffers
+              (20000, 8192), (12000, 10752)]
+
+
+@pytest.mark.parametrize("N,K", IMMA_CASES)
+def test_imma_small(bz, N, K):
+    p = Problem(1, N, K, PQ2, seed=N + 5 * K)
+    got = _run(bz, p, bz.BONSAI_ALGO_IMMA)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+@pytest.mark.parametrize("K,N", DECODE_SHAPES)
+def test_imma_decode_shapes_full(bz, K, N):
+    """Every output of the full-size M=1 PQ2_0 projections against the float64 checker,
+    and the default entry point (which dispatches M == 1 PQ2_0 here) bit-equal to it."""
+    import torch
+    p = Problem(1, N, K, PQ2, seed=0)
+    got = _run(bz, p, bz.BONSAI_ALGO_IMMA)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+    x, packed, scales = p.device()
+    y = torch.empty((1, N), dtype=torch.float16, device="cuda")
+    bz.bonsai_ternary_linear(x, packed, scales, y, 1, N, K, PQ2)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_numpy_f16(y), got)
+    assert bz.bonsai_launch_count(1, N, K, PQ2) == 2
+
+
+def test_imma_repeatable_and_counters_reset(bz):
+    """Row tiles split between warps are summed through partials and arrival counters;
+    the counters return to zero, so back-to-back calls on shapes with different splits
+    give bit-identical results."""
+    import torch
+    probs = [Problem(1, 3000, 5120, PQ2, seed=1), Problem(1, 77, 17408, PQ2, seed=2),
+             Problem(1, 5120, 17408, PQ2, seed=3)]
+    devs = [p.device() for p in probs]
+    outs = []
+    for _ in range(3):
+        for p, (x, packed, scales) in zip(probs, devs):
+            y = torch.empty((1, p.N), dtype=torch.float16, device="cuda")
+            bz.bonsai_ternary_linear_algo(x, packed, scales, y, 1, p.N, p.K, PQ2, bz.BONSAI_ALGO_IMMA, 0)
+            outs.append(y)
+    torch.cuda.synchronize()
+    for i in range(3, 9):
+        assert torch.equal(outs[i], outs[i % 3])
+    for i, p in enumerate(probs):
+        assert oracle.compare(to_numpy_f16(outs[i]), p.oracle_y())[0]
+
+
+def test_imma_input_with_large_and_small_groups(bz):
+    """Groups of x whose magnitudes differ by 2^20 get their own power-of-two scales."""
+    import torch
+    p = Problem(1, 256, 2048, PQ2, seed=9)
+    xs = p.x.astype(np.float32)
+    for g in range(16):
+        xs[:, 128 * g:128 * (g + 1)] *= 2.0 ** (5 if g % 2 else -15)
+    p.x = xs.astype(np.float16)
+    got = _run(bz, p, bz.BONSAI_ALGO_IMMA)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+def test_imma_rejects_what_it_cannot_run(bz):
+    import torch
+    x = torch.zeros((2, 512), dtype=torch.float16, device="cuda")
+    y = torch.zeros((2, 8), dtype=torch.float16, device="cuda")
+    s = torch.zeros((8, 4), dtype=torch.float16, device="cuda")
+    w = torch.zeros((8, 128), dtype=torch.uint8, device="cuda")
+    with pytest.raises(bz.BonsaiError):  # a batch
+        bz.bonsai_ternary_linear_algo(x, w, s, y, 2, 8, 512, PQ2, bz.BONSAI_ALGO_IMMA)
+    with pytest.raises(bz.BonsaiError):  # PTQ1_0
+        bz.bonsai_ternary_linear_algo(x[:1], w, s, y[:1], 1, 8, 512, PTQ1, bz.BONSAI_ALGO_IMMA)
 
 
 # ------------------------------------------------------------ prefill GEMM (tcgen05 / TMEM)
