@@ -157,8 +157,8 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
 
 /* Number of kernels one bonsai_ternary_linear_algo call with these arguments launches
  * on the current device (the lookup-table GEMV: 1, or 2 when its split-K partials are
- * summed by a second kernel; the integer tensor-core GEMV: 2, its rotation and
- * quantisation of x, then the GEMV; the other kernels: 2, the rotation pass and the kernel),
+ * summed by a second kernel; the integer tensor-core GEMV: 1; the other kernels: 2,
+ * the rotation pass and the kernel),
  * or a negative bonsai_status.  Launches nothing. */
 int bonsai_launch_count(int64_t M, int64_t N, int64_t K, int fmt, int algo, int split_k);
 

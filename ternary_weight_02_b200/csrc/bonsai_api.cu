@@ -315,7 +315,7 @@ int bonsai_launch_count(int64_t M, int64_t N, int64_t K, int fmt, int algo, int 
     if (rc != BONSAI_OK) return rc;
     switch (chosen) {
         case BONSAI_ALGO_GEMV: return gemv_launches(N, K, fmt, split_k, st->info);
-        case BONSAI_ALGO_IMMA: return 2;  // x -> x~ fragments, then the GEMV
+        case BONSAI_ALGO_IMMA: return 1;  // the rotation and quantisation of x are fused
         default: return 2;  // the rotation pass, then the kernel
     }
 }

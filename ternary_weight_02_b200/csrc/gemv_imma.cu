@@ -21,13 +21,11 @@
 //   exactly in int32, so sum t*x~ = 256*Dhi + Dlo - sum x~ exactly; one FP32 multiply by
 //   s * 2^-e per (row, group) follows.  (The rounding of x' to x~ is the only
 //   approximation; it is finer than FP16 for every element of the group.)
-// * Two launches, chained with programmatic dependent launch:
-//   1. gemv_imma_prep_kernel rotates and quantises x once (8 lanes per group) into
-//      the fragment order the MMAs read, in the workspace;
-//   2. gemv_imma_kernel: 16 warps per CTA, each feeding its own ring of item buffers
-//      (a TMA box of trits, and the item's scale words by cp.async).  The first item
-//      of every warp is requested before waiting for the previous kernel; the x~
-//      fragments are copied next, ahead of the remaining weight traffic.
+// * One launch.  16 warps per CTA, each feeding its own ring of item buffers (a TMA
+//   box of trits, and the item's scales by cp.async).  The first item of every warp is
+//   requested before waiting for the previous kernel (weights do not depend on it);
+//   then every CTA rotates and quantises all of x into x~ fragments in shared memory
+//   (8 lanes per group), with its x loads issued ahead of the remaining weight copies.
 // * Decode.  A 32-bit weight word holds 16 codes; (w >> 2j) & 0x03030303 is code j of
 //   its four bytes as four u8 lanes of an A register.  The three shifts are done as
 //   multiply-high by 2^(32-2j) (FMA pipe), the masks on the ALU pipe.
@@ -70,9 +68,9 @@ constexpr uint32_t kCodeMask = 0x03030303u;
 // aligned, as the 128-byte swizzle of its TMA box requires):
 // [weight rings: kConsumers x kStages x 4096][scale rings: kConsumers x kStages x 256]
 // [x~ fragments G4 x 288][(64 sum x~, 2^-e / 64) x G4][slots kMaxCtaItems x 128][256 zero bytes]
-// [full barriers][x barrier]
+// [full barriers]
 struct Layout {
-    int sring, xfrag, sxf, slots, zero, full, xbar, total;
+    int sring, xfrag, sxf, slots, zero, full, total;
 };
 
 __host__ __device__ inline Layout make_layout(int K) {
@@ -84,21 +82,12 @@ __host__ __device__ inline Layout make_layout(int K) {
     L.slots = L.sxf + G4 * 8;
     L.zero = L.slots + kMaxCtaItems * kItemRows * 4;
     L.full = L.zero + 256;
-    L.xbar = L.full + kConsumers * kStages * 8;
-    L.total = L.xbar + 8 + 1024;  // + room to align the base
+    L.total = L.full + kConsumers * kStages * 8 + 1024;  // + room to align the base
     return L;
 }
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
-
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(saddr(dst)), "l"(src), "r"(bytes), "r"(saddr(bar))
-        : "memory");
-}
-
 
 // D += A * B, A 16 x 32 u8 (row-major fragments), B 32 x 8 s8, D int32.
 __device__ __forceinline__ void imma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -108,7 +97,18 @@ __device__ __forceinline__ void imma(int (&d)[4], uint32_t a0, uint32_t a1, uint
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// ---------------------------------------------------------------- 1. x -> x~ fragments
+// ---------------------------------------------------------------- x -> x~ fragments
+
+// Loads the 32 bytes of x lane l of group g holds (zeros past the last group).
+__device__ __forceinline__ void load_x8(const uint16_t *__restrict__ x, int g, int G, int l, uint4 &r0, uint4 &r1) {
+    if (g < G) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)g * kGroup + 16 * l);
+        r0 = src[0];
+        r1 = src[1];
+    } else {
+        r0 = r1 = make_uint4(0u, 0u, 0u, 0u);
+    }
+}
 
 // Eight lanes per 128-group, four groups per warp; lane l (0..7) of a group holds
 // elements k = 16l + m, m = 0..15.  Fragment layout of group g, part p (0: high byte,
@@ -117,22 +117,13 @@ __device__ __forceinline__ void imma(int (&d)[4], uint32_t a0, uint32_t a1, uint
 // 16-byte chunk 2*s + (j >> 1) in the 144-byte half-block (2g + p).  The 16 bytes of
 // padding per half-block put the eight lanes that load one chunk of four consecutive
 // groups on distinct shared-memory banks.  Lane l = 2*s + hb writes whole words.
-__global__ void __launch_bounds__(128) gemv_imma_prep_kernel(const uint16_t *__restrict__ x,
-                                                             uint8_t *__restrict__ xfrag, int2 *__restrict__ sxf,
-                                                             int K) {
-    pdl_launch_dependents();
-    const int lane = threadIdx.x & 31;
+// Rotates and quantises group g (its x in r0, r1 of the group's 8 lanes) into the
+// fragment area and (64 * sum x~, 2^-e / 64) into sxf[g].
+__device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag, int2 *sxf, int g, int lane) {
     const int l = lane & 7;
-    const int g = (blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + (lane >> 3);
-    const int G = K / kGroup;
-    const int G4 = ((K + kItemK - 1) / kItemK) * 4;
-    pdl_wait();  // x and the fragment buffer may belong to the previous kernel
-    if (g >= G4) return;  // whole 8-lane groups leave together (G4 is a multiple of 4)
     const unsigned int gmask = 0xffu << (lane & 24);
     float v[16];
-    if (g < G) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(x + (int64_t)g * kGroup + 16 * l);
-        const uint4 r0 = src[0], r1 = src[1];
+    {
         const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
 #pragma unroll
         for (int i = 0; i < 8; i++) {
@@ -140,9 +131,6 @@ __global__ void __launch_bounds__(128) gemv_imma_prep_kernel(const uint16_t *__r
             v[2 * i] = f.x;
             v[2 * i + 1] = f.y;
         }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 16; i++) v[i] = 0.f;
     }
     // index bits 0..3 inside the lane
 #pragma unroll
@@ -190,7 +178,7 @@ __global__ void __launch_bounds__(128) gemv_imma_prep_kernel(const uint16_t *__r
 #pragma unroll
     for (int b = 1; b < 8; b <<= 1) sum += __shfl_xor_sync(gmask, sum, b);
     // lane l = 2s + hb: chunk 2s + (j >> 1), byte 8 (j & 1) + 4 hb + i
-    uint8_t *dst = xfrag + (int64_t)g * kXGroupBytes + (l >> 1) * 32 + (l & 1) * 4;
+    uint8_t *dst = xfrag + g * kXGroupBytes + (l >> 1) * 32 + (l & 1) * 4;
 #pragma unroll
     for (int j = 0; j < 4; j++) {
         uint32_t whi = 0u, wlo = 0u;
@@ -209,7 +197,22 @@ __global__ void __launch_bounds__(128) gemv_imma_prep_kernel(const uint16_t *__r
     if (l == 0) sxf[g] = make_int2(sum * 64, __float_as_int(f));
 }
 
-// ---------------------------------------------------------------- 2. the GEMV
+// ---------------------------------------------------------------- the GEMV
+
+__device__ __forceinline__ void st_release(unsigned int *p, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Bounded wait for another CTA's release of *p (which that CTA sets before it waits on
+// anything itself): false if it did not come within kSpinLimit polls.
+__device__ __forceinline__ bool wait_flag(const unsigned int *p) {
+    for (uint32_t i = 0; i < kSpinLimit; i++) {
+        unsigned int v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        if (v != 0u) return true;
+        __nanosleep(64);
+    }
+    return false;
+}
 
 __device__ __forceinline__ void cp_async8(void *dst, const void *src, bool valid) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(saddr(dst)), "l"(src), "r"(valid ? 8 : 0)
@@ -225,8 +228,8 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // scales it needs when it processes the item.
 template <bool kAsyncScales>
 __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
-    const __grid_constant__ CUtensorMap wmap, const uint8_t *__restrict__ xprep, const uint16_t *__restrict__ scales,
-    uint16_t *__restrict__ y, float *__restrict__ partials, unsigned int *__restrict__ counters, int N, int K,
+    const __grid_constant__ CUtensorMap wmap, const uint16_t *__restrict__ x, const uint16_t *__restrict__ scales,
+    uint16_t *__restrict__ y, float *__restrict__ partials, unsigned int *__restrict__ flags, int N, int K,
     uint32_t mul2, uint32_t mul4, uint32_t mul6) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u);
@@ -249,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     float *slots = reinterpret_cast<float *>(smem + L.slots);
     uint8_t *zero = smem + L.zero;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full) + warp * kStages;
-    uint64_t *xbar = reinterpret_cast<uint64_t *>(smem + L.xbar);
 
     // item q of this warp: c0 + warp + q * kConsumers -> ring stage q % kStages.  Lane 0
     // starts the TMA box; lane r copies the item's four scales of row r (cp.async); one
@@ -284,7 +286,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
 
     if (lane == 0) {
         for (int st = 0; st < kStages; st++) mbar_init(full + st, 1);
-        if (tid == 0) mbar_init(xbar, 1);
         mbar_init_fence();
     }
     if (tid < 64) reinterpret_cast<uint32_t *>(zero)[tid] = 0u;
@@ -292,13 +293,25 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     // weights and scales do not depend on the previous kernel: start some before waiting
     for (int q = 0; q < kPreStages; q++) issue(q);
     pdl_launch_dependents();
-    pdl_wait();  // the x~ fragments come from the prep kernel
-    if (tid == 0) {  // before the remaining weight copies, so that it is not queued behind them
-        mbar_arrive_expect_tx(xbar, (uint32_t)G4 * (kXGroupBytes + 8));
-        bulk_load(xf, xprep, (uint32_t)G4 * (kXGroupBytes + 8), xbar);
+    pdl_wait();  // x, y and the workspace may belong to the previous kernel
+    // x -> x~ fragments, four groups per warp and round: all of this warp's x first
+    {
+        constexpr int kRounds = (int)((kMaxK / kItemK) * 4 / 4 + kConsumers - 1) / kConsumers;
+        uint4 xr[kRounds][2];
+#pragma unroll
+        for (int r = 0; r < kRounds; r++) {
+            const int g = (warp + r * kConsumers) * 4 + (lane >> 3);
+            if (g < G4) load_x8(x, g, G, lane & 7, xr[r][0], xr[r][1]);
+        }
+        for (int q = kPreStages; q < kStages; q++) issue(q);
+#pragma unroll
+        for (int r = 0; r < kRounds; r++) {
+            const int g = (warp + r * kConsumers) * 4 + (lane >> 3);
+            if ((warp + r * kConsumers) * 4 < G4)  // whole warps: G4 is a multiple of 4
+                build_group8(xr[r][0], xr[r][1], xf, reinterpret_cast<int2 *>(smem + L.sxf), g, lane);
+        }
     }
     __syncthreads();
-    for (int q = kPreStages; q < kStages; q++) issue(q);
 
     // Lane (gid, tig) works on scale group tig of the item: MMA rows gid and gid + 8 of
     // each 16-row tile t are shared-memory rows r = 16t + gid (+ 8), whose group tig is
@@ -312,12 +325,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const int xb_stride = bactive ? kXGroupBytes : 0;
     const int R = 8 * tig + gid;  // the item row this lane reports: (t, h) = (tig >> 1, tig & 1)
 
-    bool ok = __all_sync(0xffffffffu, mbar_wait(xbar, 0));
+    bool ok = true;
     int n_waited = 0;
     int st = 0;
     uint32_t phase = 0;
     int rt = (c0 + warp) / KC, kc = (c0 + warp) - ((c0 + warp) / KC) * KC;
-    for (int q = 0; q < nq; q++) {
+    auto process = [&](int q) {
         const int i = c0 + warp + q * kConsumers;
         if (ok) {
             ok = __all_sync(0xffffffffu, mbar_wait(full + st, phase));
@@ -417,7 +430,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
         slots[(i - c0) * kItemRows + R] = mine;
         if (++st == kStages) st = 0, phase ^= 1u;
         advance(rt, kc);
+    };
+
+    // Row tiles split between CTAs: the CTA holding a tile's first item owns the tile and
+    // adds the other pieces, which the CTAs that follow publish (partial sums + a release
+    // flag).  A CTA's first tile, when it is such a later piece, is published as soon as
+    // its items are done, so that its owner -- which reaches that tile last -- does not wait.
+    const int rt_first = c0 / KC, rt_last = c1 > c0 ? (c1 - 1) / KC : rt_first - 1;
+    const int first_end = c1 < (rt_first + 1) * KC ? c1 : (rt_first + 1) * KC;
+    const bool early = c0 > rt_first * KC && first_end < c1;
+    const int q_pub = early ? (first_end - c0 - 1) / kConsumers : -1;  // the round of its last item
+    auto publish = [&](int a, float v) {  // piece starting at item a; one lane per row
+        partials[(int64_t)a * kItemRows + lane] = v;
+        __syncwarp();  // the warp's stores are ordered before lane 0's release
+        if (lane == 0) st_release(flags + a, 1u);
+    };
+    if (early) {
+        for (int q = 0; q <= q_pub; q++)
+            if (q < nq) process(q);
+        __syncthreads();  // the first tile's slots are written
+        if (warp == 0) {
+            float v = 0.f;
+            for (int i = c0; i < first_end; i++) v += slots[(i - c0) * kItemRows + lane];
+            publish(c0, v);
+        }
     }
+    for (int q = q_pub + 1; q < nq; q++) process(q);
     if (kAsyncScales) cp_async_wait_all();
     // after a wait gave up: let the box copies already started land before the CTA exits
     if (!ok && lane == 0) {
@@ -430,41 +468,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     }
     __syncthreads();  // every slot is written
 
-    // ---- row tiles: add each tile's items in K order; tiles shared with a neighbouring
-    // CTA go through the workspace partials (one warp per tile, one lane per row)
-    const int rt_first = c0 / KC, rt_last = c1 > c0 ? (c1 - 1) / KC : rt_first - 1;
+    // ---- row tiles: add each tile's items in K order (one warp per tile, one lane per row)
     for (int rt = rt_first + warp; rt <= rt_last; rt += kConsumers) {
         const int tile_first = rt * KC, tile_end = tile_first + KC;
         const int a = c0 > tile_first ? c0 : tile_first;
         const int b = c1 < tile_end ? c1 : tile_end;
+        if (rt == rt_first && early) continue;  // published already
         float sum = 0.f;
         for (int i = a; i < b; i++) sum += slots[(i - c0) * kItemRows + lane];
-        const int row = rt * kItemRows + lane;
-        if (a == tile_first && b == tile_end) {
-            if (row < N) y[row] = float_to_half_bits(sum);
+        if (a > tile_first) {  // a later piece of a tile owned by an earlier CTA
+            publish(a, sum);
             continue;
         }
-        partials[(int64_t)a * kItemRows + lane] = sum;
-        __threadfence();
-        __syncwarp();
-        const unsigned int cover = (unsigned int)(b - a);
-        unsigned int old = 0u;
-        if (lane == 0) old = atomicAdd(counters + rt, cover);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        if (old + cover != (unsigned int)KC) continue;
-        __threadfence();  // this CTA completes the tile: add the pieces in K order
-        float total = 0.f;
-        int s = tile_first;
+        // owned: add the pieces of the CTAs that follow, in K order
+        int s = b, c2 = (int)blockIdx.x + 1;
         while (s < tile_end) {
-            // the CTA whose range holds item s, and where its range ends
-            const int c2 = (int)(((int64_t)(s + 1) * C - 1) / I);
-            int e2 = (int)((int64_t)I * (c2 + 1) / C);
+            int e2 = (int)((int64_t)I * (c2 + 1) / C);  // the piece of CTA c2 is [s, e2)
             e2 = e2 < tile_end ? e2 : tile_end;
-            total += c2 == (int)blockIdx.x ? sum : __ldcg(partials + (int64_t)s * kItemRows + lane);
+            bool got = true;
+            if (lane == 0) got = wait_flag(flags + s);
+            got = __shfl_sync(0xffffffffu, got, 0);
+            __syncwarp();  // lane 0's acquire is ordered before the warp's loads
+            sum += got ? __ldcg(partials + (int64_t)s * kItemRows + lane) : __int_as_float(0x7fc00000);
+            if (lane == 0) flags[s] = 0u;  // ready for the next call
             s = e2;
+            c2++;
         }
-        if (row < N) y[row] = float_to_half_bits(total);
-        if (lane == 0) counters[rt] = 0u;
+        const int row = rt * kItemRows + lane;
+        if (row < N) y[row] = float_to_half_bits(sum);
     }
 }
 
@@ -489,21 +520,20 @@ Shape shape_of(int64_t N, int64_t K, int sm_count) {
 }  // namespace
 
 static_assert(kConsumers * kStages * (kItemBytes + kScaleRingBytes) + (kMaxK / kItemK) * 4 * (kXGroupBytes + 8) +
-                  kMaxCtaItems * kItemRows * 4 + 256 + kConsumers * kStages * 8 + 8 + 1024 <= 232448,
+                  kMaxCtaItems * kItemRows * 4 + 256 + kConsumers * kStages * 8 + 1024 <= 232448,
               "shared-memory layout exceeds the per-CTA limit at the largest K");
 
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt) {
     if (fmt != 2 || M != 1 || N < 1 || K < kGroup || K % kGroup != 0 || K > kMaxK) return false;
     const int64_t RT = (N + kItemRows - 1) / kItemRows;
-    return RT <= kMaxTiles && RT * ((K + kItemK - 1) / kItemK) < ((int64_t)1 << 30);
+    return RT * ((K + kItemK - 1) / kItemK) <= kMaxTiles;  // one flag per item in the counter block
 }
 
-// workspace: [x~ fragments G4 x 256][(sum, 2^-e) x G4][pad to 256][partials: items x 32 floats]
+// workspace: the partial sums of row tiles shared by two CTAs, items x 32 floats
 size_t gemv_imma_workspace_bytes(int64_t N, int64_t K) {
     const int64_t KC = (K + kItemK - 1) / kItemK;
     const int64_t items = ((N + kItemRows - 1) / kItemRows) * KC;
-    const size_t xbytes = ((size_t)(KC * 4) * (kXGroupBytes + 8) + 255) / 256 * 256;
-    return xbytes + (size_t)items * kItemRows * sizeof(float);
+    return (size_t)items * kItemRows * sizeof(float);
 }
 
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
@@ -524,34 +554,23 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
             return cudaErrorInvalidValue;
     }
     const Shape sh = shape_of(N, K, dev.sm_count);
-    uint8_t *xprep = ws.data;
-    int2 *sxf = reinterpret_cast<int2 *>(xprep + (size_t)sh.G4 * kXGroupBytes);
-    float *partials = reinterpret_cast<float *>(
-        ws.data + ((size_t)sh.G4 * (kXGroupBytes + 8) + 255) / 256 * 256);
-
+    float *partials = reinterpret_cast<float *>(ws.data);
+    // K a multiple of 512: an item's scales of a row are 8 aligned bytes, copied with the item
+    auto kern = K % kItemK == 0 ? gemv_imma_kernel<true> : gemv_imma_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+    if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    // 1. x -> x~ fragments: four groups per warp, four warps per CTA
-    cfg.gridDim = dim3((unsigned)((sh.G4 + 15) / 16));
-    cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_imma_prep_kernel, x, xprep, sxf, (int)K);
-    if (e != cudaSuccess) return e;
-    // 2. the GEMV
-    // K a multiple of 512: an item's scales of a row are 8 aligned bytes, copied with the item
-    auto kern = K % kItemK == 0 ? gemv_imma_kernel<true> : gemv_imma_kernel<false>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
-    if (e != cudaSuccess) return e;
     cfg.gridDim = dim3((unsigned)sh.grid);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = lay.total;
-    return cudaLaunchKernelEx(&cfg, kern, wmap, (const uint8_t *)xprep, scales, y, partials, ws.counters,
-                              (int)N, (int)K, 1u << 30, 1u << 28, 1u << 26);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, wmap, x, scales, y, partials, ws.counters, (int)N, (int)K, 1u << 30,
+                              1u << 28, 1u << 26);
 }
 
 }  // namespace bonsai

@@ -250,7 +250,7 @@ def test_imma_decode_shapes_full(bz, K, N):
     bz.bonsai_ternary_linear(x, packed, scales, y, 1, N, K, PQ2)
     torch.cuda.synchronize()
     assert np.array_equal(to_numpy_f16(y), got)
-    assert bz.bonsai_launch_count(1, N, K, PQ2) == 2
+    assert bz.bonsai_launch_count(1, N, K, PQ2) == 1
 
 
 def test_imma_repeatable_and_counters_reset(bz):
