@@ -294,21 +294,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     for (int q = 0; q < kPreStages; q++) issue(q);
     pdl_launch_dependents();
     pdl_wait();  // x, y and the workspace may belong to the previous kernel
-    // x -> x~ fragments, four groups per warp and round: all of this warp's x first
+    // x -> x~ fragments, four groups (a quad) per warp and round: all of this warp's x
+    // first.  Every CTA reads all of x at the same moment, so each starts at a different
+    // quad: the simultaneous requests spread over the lines of x instead of piling up.
     {
         constexpr int kRounds = (int)((kMaxK / kItemK) * 4 / 4 + kConsumers - 1) / kConsumers;
+        const int nquads = G4 / 4;
+        const int rot = (int)(blockIdx.x % (unsigned)nquads);
         uint4 xr[kRounds][2];
 #pragma unroll
         for (int r = 0; r < kRounds; r++) {
-            const int g = (warp + r * kConsumers) * 4 + (lane >> 3);
-            if (g < G4) load_x8(x, g, G, lane & 7, xr[r][0], xr[r][1]);
+            const int quad = warp + r * kConsumers;
+            int pq = quad + rot;
+            if (pq >= nquads) pq -= nquads;
+            if (quad < nquads) load_x8(x, pq * 4 + (lane >> 3), G, lane & 7, xr[r][0], xr[r][1]);
         }
         for (int q = kPreStages; q < kStages; q++) issue(q);
 #pragma unroll
         for (int r = 0; r < kRounds; r++) {
-            const int g = (warp + r * kConsumers) * 4 + (lane >> 3);
-            if ((warp + r * kConsumers) * 4 < G4)  // whole warps: G4 is a multiple of 4
-                build_group8(xr[r][0], xr[r][1], xf, reinterpret_cast<int2 *>(smem + L.sxf), g, lane);
+            const int quad = warp + r * kConsumers;
+            int pq = quad + rot;
+            if (pq >= nquads) pq -= nquads;
+            if (quad < nquads)  // whole warps
+                build_group8(xr[r][0], xr[r][1], xf, reinterpret_cast<int2 *>(smem + L.sxf), pq * 4 + (lane >> 3),
+                             lane);
         }
     }
     __syncthreads();
