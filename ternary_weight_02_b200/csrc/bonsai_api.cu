@@ -27,6 +27,8 @@ struct DeviceState {
     DeviceInfo info;
     void *ws_base = nullptr;
     size_t ws_bytes = 0;  // total allocation (counters + data)
+    void *zb_base = nullptr;
+    size_t zb_bytes = 0;  // the zero-initialised region
 };
 
 std::mutex g_mutex;
@@ -62,7 +64,7 @@ int probe_current(int *dev_out, DeviceState **st_out) {
 // Makes sure the current device's workspace holds at least data_bytes after the
 // counter block.  Grows by reallocating (after a device synchronisation, since
 // work in flight may still use the old buffer).
-int ensure_workspace(DeviceState &st, size_t data_bytes, Workspace *ws) {
+int ensure_workspace(DeviceState &st, size_t data_bytes, size_t zeroed_bytes, Workspace *ws) {
     const size_t need = kCounterBytes + ((data_bytes + 255) / 256) * 256;
     if (st.ws_bytes < need) {
         if (st.ws_base) {
@@ -85,6 +87,28 @@ int ensure_workspace(DeviceState &st, size_t data_bytes, Workspace *ws) {
         st.ws_base = p;
         st.ws_bytes = grow;
     }
+    if (st.zb_bytes < zeroed_bytes) {
+        if (st.zb_base) {
+            if (cudaDeviceSynchronize() != cudaSuccess) return BONSAI_ERR_CUDA;
+            cudaFree(st.zb_base);
+            st.zb_base = nullptr;
+            st.zb_bytes = 0;
+        }
+        const size_t grow = zeroed_bytes < (size_t(16) << 20) ? (size_t(16) << 20) : zeroed_bytes;
+        void *p = nullptr;
+        if (cudaMalloc(&p, grow) != cudaSuccess) {
+            cudaGetLastError();
+            return BONSAI_ERR_NOMEM;
+        }
+        if (cudaMemset(p, 0, grow) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+            cudaFree(p);
+            return BONSAI_ERR_CUDA;
+        }
+        st.zb_base = p;
+        st.zb_bytes = grow;
+    }
+    ws->zeroed = static_cast<uint8_t *>(st.zb_base);
+    ws->zeroed_bytes = st.zb_bytes;
     ws->counters = static_cast<unsigned int *>(st.ws_base);
     ws->data = static_cast<uint8_t *>(st.ws_base) + kCounterBytes;
     ws->data_bytes = st.ws_bytes - kCounterBytes;
@@ -134,7 +158,7 @@ size_t workspace_for(int algo, int64_t M, int64_t N, int64_t K, int fmt, int spl
         case BONSAI_ALGO_GEMV: return gemv_workspace_bytes(N, K, fmt, split_k, info);
         case BONSAI_ALGO_SKINNY: return skinny_workspace_bytes(M, N, K, fmt, split_k, info);
         case BONSAI_ALGO_GEMM: return gemm_workspace_bytes(M, N, K, fmt);
-        case BONSAI_ALGO_IMMA: return gemv_imma_workspace_bytes(N, K);
+        case BONSAI_ALGO_IMMA: return 0;
         default: return simple_workspace_bytes(M, N, K);
     }
 }
@@ -270,7 +294,8 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
     rc = probe_current(&dev, &st);
     if (rc != BONSAI_OK) return rc;
     Workspace ws;
-    rc = ensure_workspace(*st, workspace_for(chosen, M, N, K, fmt, split_k, st->info), &ws);
+    rc = ensure_workspace(*st, workspace_for(chosen, M, N, K, fmt, split_k, st->info),
+                          chosen == BONSAI_ALGO_IMMA ? gemv_imma_zeroed_bytes(N, K) : 0, &ws);
     if (rc != BONSAI_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
@@ -328,7 +353,7 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
     DeviceState *st;
     rc = probe_current(&dev, &st);
     if (rc != BONSAI_OK) return rc;
-    size_t need = simple_workspace_bytes(M, N, K);
+    size_t need = simple_workspace_bytes(M, N, K), zneed = 0;
     for (int fmt = BONSAI_FMT_PTQ1_0; fmt <= BONSAI_FMT_PQ2_0; fmt++) {
         size_t v;
         if (M <= 1 && gemv_supported(1, N, K, fmt)) {
@@ -336,8 +361,8 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
             need = v > need ? v : need;
         }
         if (M <= 1 && gemv_imma_supported(1, N, K, fmt)) {
-            v = gemv_imma_workspace_bytes(N, K);
-            need = v > need ? v : need;
+            v = gemv_imma_zeroed_bytes(N, K);
+            zneed = v > zneed ? v : zneed;
         }
         if (skinny_supported(M < 16 ? M : 16, N, K, fmt)) {
             v = skinny_workspace_bytes(M < 16 ? M : 16, N, K, fmt, 0, st->info);
@@ -349,7 +374,7 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
         }
     }
     Workspace ws;
-    return ensure_workspace(*st, need, &ws);
+    return ensure_workspace(*st, need, zneed, &ws);
 }
 
 void bonsai_shutdown(void) {
@@ -363,6 +388,13 @@ void bonsai_shutdown(void) {
             cudaFree(g_dev[d].ws_base);
             g_dev[d].ws_base = nullptr;
             g_dev[d].ws_bytes = 0;
+        }
+        if (g_dev[d].zb_base) {
+            cudaSetDevice(d);
+            cudaDeviceSynchronize();
+            cudaFree(g_dev[d].zb_base);
+            g_dev[d].zb_base = nullptr;
+            g_dev[d].zb_bytes = 0;
         }
     }
     if (current >= 0) cudaSetDevice(current);

@@ -60,7 +60,7 @@ constexpr int kXHalfBytes = 144;                        // one part (hi or lo) o
 constexpr int kXGroupBytes = 2 * kXHalfBytes;
 constexpr int kStages = 2;
 constexpr int kPreStages = 1;                           // issued before the wait on the previous kernel
-constexpr int kMaxCtaItems = 160;                       // slot buffer: 160 x 32 floats
+constexpr int kMaxCtaItems = 96;                        // slot buffer: 96 x 32 floats
 constexpr int64_t kMaxK = 24576;  // the layout below then fits the 227 KB a CTA may use
 constexpr uint32_t kCodeMask = 0x03030303u;
 
@@ -199,19 +199,32 @@ __device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag,
 
 // ---------------------------------------------------------------- the GEMV
 
-__device__ __forceinline__ void st_release(unsigned int *p, unsigned int v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+// A later piece's partial sums travel as 64-bit (value, epoch) pairs, one per row: an
+// aligned 64-bit access is single-copy atomic, so a reader that sees epoch 1 sees the
+// value stored with it -- no fence on either side.
+__device__ __forceinline__ void st_pair(uint64_t *p, float v) {
+    const uint64_t w = (uint64_t)__float_as_uint(v) | ((uint64_t)1 << 32);
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
-// Bounded wait for another CTA's release of *p (which that CTA sets before it waits on
-// anything itself): false if it did not come within kSpinLimit polls.
-__device__ __forceinline__ bool wait_flag(const unsigned int *p) {
+__device__ __forceinline__ uint64_t ld_pair(const uint64_t *p) {
+    uint64_t w;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+    return w;
+}
+// Bounded wait, by the whole warp, for the 32 pairs at p (one per lane) to carry epoch 1;
+// returns this lane's value, or NaN if they did not all come within kSpinLimit polls.
+// The pairs are written by a CTA with a higher index, which writes them before it waits
+// on anything itself.
+__device__ __forceinline__ float wait_pairs(uint64_t *p, int lane) {
     for (uint32_t i = 0; i < kSpinLimit; i++) {
-        unsigned int v;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-        if (v != 0u) return true;
-        __nanosleep(64);
+        const uint64_t w = ld_pair(p + lane);
+        if (__all_sync(0xffffffffu, (w >> 32) == 1u)) {
+            asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p + lane), "l"((uint64_t)0) : "memory");
+            return __uint_as_float((uint32_t)w);  // (cleared for the next call)
+        }
+        __nanosleep(32);
     }
-    return false;
+    return __int_as_float(0x7fc00000);
 }
 
 __device__ __forceinline__ void cp_async8(void *dst, const void *src, bool valid) {
@@ -229,7 +242,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 template <bool kAsyncScales>
 __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const __grid_constant__ CUtensorMap wmap, const uint16_t *__restrict__ x, const uint16_t *__restrict__ scales,
-    uint16_t *__restrict__ y, float *__restrict__ partials, unsigned int *__restrict__ flags, int N, int K,
+    uint16_t *__restrict__ y, uint64_t *__restrict__ partials, int N, int K,
     uint32_t mul2, uint32_t mul4, uint32_t mul6) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u);
@@ -442,23 +455,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     };
 
     // Row tiles split between CTAs: the CTA holding a tile's first item owns the tile and
-    // adds the other pieces, which the CTAs that follow publish (partial sums + a release
-    // flag).  A CTA's first tile, when it is such a later piece, is published as soon as
-    // its items are done, so that its owner -- which reaches that tile last -- does not wait.
+    // adds the other pieces, which the CTAs that follow store as (value, epoch) pairs.  The
+    // owner reaches its piece last (the end of its range), while the later pieces open
+    // their CTAs' ranges: a CTA's first tile, when it is such a piece, is stored as soon as
+    // its items are done.  Waits only go from a CTA to higher ones, which store before
+    // they wait on anything: all CTAs of the grid fit on the GPU at once (one per SM).
     const int rt_first = c0 / KC, rt_last = c1 > c0 ? (c1 - 1) / KC : rt_first - 1;
     const int first_end = c1 < (rt_first + 1) * KC ? c1 : (rt_first + 1) * KC;
     const bool early = c0 > rt_first * KC && first_end < c1;
     const int q_pub = early ? (first_end - c0 - 1) / kConsumers : -1;  // the round of its last item
-    auto publish = [&](int a, float v) {  // piece starting at item a; one lane per row
-        partials[(int64_t)a * kItemRows + lane] = v;
-        __syncwarp();  // the warp's stores are ordered before lane 0's release
-        if (lane == 0) st_release(flags + a, 1u);
-    };
+    auto publish = [&](int a, float v) { st_pair(partials + (int64_t)a * kItemRows + lane, v); };
     if (early) {
         for (int q = 0; q <= q_pub; q++)
             if (q < nq) process(q);
         __syncthreads();  // the first tile's slots are written
-        if (warp == 0) {
+        if (warp == kConsumers - 1) {  // the last warp has the fewest items (round-robin)
             float v = 0.f;
             for (int i = c0; i < first_end; i++) v += slots[(i - c0) * kItemRows + lane];
             publish(c0, v);
@@ -482,24 +493,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
         const int tile_first = rt * KC, tile_end = tile_first + KC;
         const int a = c0 > tile_first ? c0 : tile_first;
         const int b = c1 < tile_end ? c1 : tile_end;
-        if (rt == rt_first && early) continue;  // published already
+        if (rt == rt_first && early) continue;  // stored already
         float sum = 0.f;
         for (int i = a; i < b; i++) sum += slots[(i - c0) * kItemRows + lane];
         if (a > tile_first) {  // a later piece of a tile owned by an earlier CTA
             publish(a, sum);
             continue;
         }
-        // owned: add the pieces of the CTAs that follow, in K order
+        // owned (or whole): add the pieces of the CTAs that follow, in K order
         int s = b, c2 = (int)blockIdx.x + 1;
         while (s < tile_end) {
             int e2 = (int)((int64_t)I * (c2 + 1) / C);  // the piece of CTA c2 is [s, e2)
             e2 = e2 < tile_end ? e2 : tile_end;
-            bool got = true;
-            if (lane == 0) got = wait_flag(flags + s);
-            got = __shfl_sync(0xffffffffu, got, 0);
-            __syncwarp();  // lane 0's acquire is ordered before the warp's loads
-            sum += got ? __ldcg(partials + (int64_t)s * kItemRows + lane) : __int_as_float(0x7fc00000);
-            if (lane == 0) flags[s] = 0u;  // ready for the next call
+            sum += wait_pairs(partials + (int64_t)s * kItemRows, lane);
             s = e2;
             c2++;
         }
@@ -535,14 +541,16 @@ static_assert(kConsumers * kStages * (kItemBytes + kScaleRingBytes) + (kMaxK / k
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt) {
     if (fmt != 2 || M != 1 || N < 1 || K < kGroup || K % kGroup != 0 || K > kMaxK) return false;
     const int64_t RT = (N + kItemRows - 1) / kItemRows;
-    return RT * ((K + kItemK - 1) / kItemK) <= kMaxTiles;  // one flag per item in the counter block
+    return RT * ((K + kItemK - 1) / kItemK) < ((int64_t)1 << 30);
 }
 
-// workspace: the partial sums of row tiles shared by two CTAs, items x 32 floats
-size_t gemv_imma_workspace_bytes(int64_t N, int64_t K) {
+// the zero-initialised workspace region: (value, epoch) pairs of the pieces of row tiles
+// split between CTAs, indexed by the piece's first item: items x 32 x 8 bytes.  Every
+// pair a call stores is cleared again by its reader.
+size_t gemv_imma_zeroed_bytes(int64_t N, int64_t K) {
     const int64_t KC = (K + kItemK - 1) / kItemK;
     const int64_t items = ((N + kItemRows - 1) / kItemRows) * KC;
-    return (size_t)items * kItemRows * sizeof(float);
+    return (size_t)items * kItemRows * sizeof(uint64_t);
 }
 
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
@@ -563,10 +571,14 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
             return cudaErrorInvalidValue;
     }
     const Shape sh = shape_of(N, K, dev.sm_count);
-    float *partials = reinterpret_cast<float *>(ws.data);
+    if (ws.zeroed_bytes < gemv_imma_zeroed_bytes(N, K)) return cudaErrorInvalidValue;
+    uint64_t *partials = reinterpret_cast<uint64_t *>(ws.zeroed);
     // K a multiple of 512: an item's scales of a row are 8 aligned bytes, copied with the item
     auto kern = K % kItemK == 0 ? gemv_imma_kernel<true> : gemv_imma_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lay.total);
+    // the attribute is set to the largest layout any K takes, so that launches of several
+    // sizes captured into one graph all stay within it
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         make_layout((int)kMaxK).total);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -578,7 +590,7 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, wmap, x, scales, y, partials, ws.counters, (int)N, (int)K, 1u << 30,
+    return cudaLaunchKernelEx(&cfg, kern, wmap, x, scales, y, partials, (int)N, (int)K, 1u << 30,
                               1u << 28, 1u << 26);
 }
 

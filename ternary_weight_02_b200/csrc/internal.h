@@ -25,6 +25,10 @@ struct Workspace {
     unsigned int *counters = nullptr;  // kMaxTiles entries
     uint8_t *data = nullptr;           // the rest, 256-byte aligned
     size_t data_bytes = 0;
+    // a separate region that is zero when created and that its one user (the integer
+    // GEMV's split row tiles) returns to zero after every call
+    uint8_t *zeroed = nullptr;
+    size_t zeroed_bytes = 0;
 };
 
 // ---- pack.cu
@@ -66,7 +70,7 @@ int current_device_info(DeviceInfo *out);
 
 // ---- gemv_imma.cu: M == 1, PQ2_0, integer tensor cores
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt);
-size_t gemv_imma_workspace_bytes(int64_t N, int64_t K);
+size_t gemv_imma_zeroed_bytes(int64_t N, int64_t K);  // of Workspace::zeroed
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
                              int64_t N, int64_t K, const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
 
