@@ -22,10 +22,10 @@
 //   s * 2^-e per (row, group) follows.  (The rounding of x' to x~ is the only
 //   approximation; it is finer than FP16 for every element of the group.)
 // * One launch.  16 warps per CTA, each feeding its own ring of item buffers (a TMA
-//   box of trits, and the item's scales by cp.async).  The first item of every warp is
-//   requested before waiting for the previous kernel (weights do not depend on it);
-//   then every CTA rotates and quantises all of x into x~ fragments in shared memory
-//   (8 lanes per group), with its x loads issued ahead of the remaining weight copies.
+//   box of trits, and the item's scales by cp.async).  After waiting for the previous
+//   kernel, every CTA loads all of x (each CTA starting at a different group quad), then
+//   starts its weight copies, then rotates and quantises x into x~ fragments in shared
+//   memory (8 lanes per group) while the first items arrive.
 // * Decode.  A 32-bit weight word holds 16 codes; (w >> 2j) & 0x03030303 is code j of
 //   its four bytes as four u8 lanes of an A register.  The three shifts are done as
 //   multiply-high by 2^(32-2j) (FMA pipe), the masks on the ALU pipe.
@@ -59,7 +59,6 @@ constexpr int kScaleRingBytes = kItemRows * 8;          // per stage: the item's
 constexpr int kXHalfBytes = 144;                        // one part (hi or lo) of a group's fragments, padded
 constexpr int kXGroupBytes = 2 * kXHalfBytes;
 constexpr int kStages = 2;
-constexpr int kPreStages = 1;                           // issued before the wait on the previous kernel
 constexpr int kMaxCtaItems = 96;                        // slot buffer: 96 x 32 floats
 constexpr int64_t kMaxK = 24576;  // the layout below then fits the 227 KB a CTA may use
 constexpr uint32_t kCodeMask = 0x03030303u;
@@ -95,6 +94,14 @@ __device__ __forceinline__ void imma(int (&d)[4], uint32_t a0, uint32_t a1, uint
     asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// D = A * B (C = 0): the first MMA of an accumulator chain, so no register is zeroed.
+__device__ __forceinline__ void imma0(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                      uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
 // ---------------------------------------------------------------- x -> x~ fragments
@@ -146,11 +153,11 @@ __device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag,
 #pragma unroll
     for (int b = 0; b < 3; b++) {
         const int mask = 1 << b;
-        const bool upper = (l & mask) != 0;
+        const float sgn = (l & mask) ? -1.f : 1.f;  // upper half: partner - own; lower: own + partner
 #pragma unroll
         for (int i = 0; i < 16; i++) {
             const float p = __shfl_xor_sync(gmask, v[i], mask);
-            v[i] = upper ? (p - v[i]) : (v[i] + p);
+            v[i] = fmaf(sgn, v[i], p);  // exact sign flip, one rounding: same as the add or subtract
         }
     }
     float am = 0.f;
@@ -303,8 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     }
     if (tid < 64) reinterpret_cast<uint32_t *>(zero)[tid] = 0u;
     __syncthreads();
-    // weights and scales do not depend on the previous kernel: start some before waiting
-    for (int q = 0; q < kPreStages; q++) issue(q);
+    // Nothing is requested before the wait: a CTA that starts late (its SM freed late by
+    // the previous kernel) would otherwise queue its x loads behind its own weight copies,
+    // and the call's time is set by its slowest CTA (measured: faster on every shape).
     pdl_launch_dependents();
     pdl_wait();  // x, y and the workspace may belong to the previous kernel
     // x -> x~ fragments, four groups (a quad) per warp and round: all of this warp's x
@@ -322,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
             if (pq >= nquads) pq -= nquads;
             if (quad < nquads) load_x8(x, pq * 4 + (lane >> 3), G, lane & 7, xr[r][0], xr[r][1]);
         }
-        for (int q = kPreStages; q < kStages; q++) issue(q);
+        for (int q = 0; q < kStages; q++) issue(q);
 #pragma unroll
         for (int r = 0; r < kRounds; r++) {
             const int quad = warp + r * kConsumers;
@@ -395,12 +403,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
         // a word as u8 values c * 4^j.  One accumulator per (tile, j); the 4^j factors are
         // undone once per item (the sums come out 64 times too large, folded into 2^-e).
         int d[2][4][4];
-#pragma unroll
-        for (int t = 0; t < 2; t++)
-#pragma unroll
-            for (int j = 0; j < 4; j++)
-#pragma unroll
-                for (int e = 0; e < 4; e++) d[t][j][e] = 0;
         const uint8_t *xb = xb_lane + g0 * xb_stride;
 #pragma unroll
         for (int s = 0; s < 4; s++) {
@@ -417,7 +419,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
                     const uint4 &r0 = raw[t][0][s >> 1], &r1 = raw[t][1][s >> 1];
                     const uint32_t w0 = (s & 1) ? r0.z : r0.x, w2 = (s & 1) ? r0.w : r0.y;
                     const uint32_t w1 = (s & 1) ? r1.z : r1.x, w3 = (s & 1) ? r1.w : r1.y;
-                    imma(d[t][j], w0 & mask, w1 & mask, w2 & mask, w3 & mask, bx, by);
+                    if (s == 0)
+                        imma0(d[t][j], w0 & mask, w1 & mask, w2 & mask, w3 & mask, bx, by);
+                    else
+                        imma(d[t][j], w0 & mask, w1 & mask, w2 & mask, w3 & mask, bx, by);
                 }
             }
         }
