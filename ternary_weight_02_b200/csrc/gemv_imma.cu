@@ -60,6 +60,7 @@ constexpr int kXHalfBytes = 144;                        // one part (hi or lo) o
 constexpr int kXGroupBytes = 2 * kXHalfBytes;
 constexpr int kStages = 2;
 constexpr int kMaxCtaItems = 96;                        // slot buffer: 96 x 32 floats
+constexpr int kMaxCtaTiles = kMaxCtaItems + 2;          // row tiles one CTA's items touch
 constexpr int64_t kMaxK = 24576;  // the layout below then fits the 227 KB a CTA may use
 constexpr uint32_t kCodeMask = 0x03030303u;
 
@@ -69,9 +70,11 @@ constexpr uint32_t kCodeMask = 0x03030303u;
 // [x~ fragments G4 x 288][(64 sum x~, 2^-e / 64) x G4][slots kMaxCtaItems x 128][256 zero bytes]
 // [full barriers]
 struct Layout {
-    int sring, xfrag, sxf, slots, zero, full, total;
+    int sring, xfrag, sxf, slots, tcnt, zero, full, total;
 };
 
+// Alignment: the weight buffers 1024 bytes (swizzled TMA destinations), the fragment,
+// slot and zero areas 16 bytes (128-bit loads), the barriers 8 bytes.
 __host__ __device__ inline Layout make_layout(int K) {
     Layout L;
     const int G4 = ((K + kItemK - 1) / kItemK) * 4;
@@ -79,7 +82,8 @@ __host__ __device__ inline Layout make_layout(int K) {
     L.xfrag = L.sring + kConsumers * kStages * kScaleRingBytes;
     L.sxf = L.xfrag + G4 * kXGroupBytes;
     L.slots = L.sxf + G4 * 8;
-    L.zero = L.slots + kMaxCtaItems * kItemRows * 4;
+    L.tcnt = L.slots + kMaxCtaItems * kItemRows * 4;
+    L.zero = (L.tcnt + kMaxCtaTiles * 4 + 15) & ~15;  // 128-bit loads read the zero bytes
     L.full = L.zero + 256;
     L.total = L.full + kConsumers * kStages * 8 + 1024;  // + room to align the base
     return L;
@@ -270,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     uint8_t *xf = smem + L.xfrag;
     const int2 *sxf = reinterpret_cast<const int2 *>(smem + L.sxf);
     float *slots = reinterpret_cast<float *>(smem + L.slots);
+    int *tile_cnt = reinterpret_cast<int *>(smem + L.tcnt);  // items done, per row tile of the range
     uint8_t *zero = smem + L.zero;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full) + warp * kStages;
 
@@ -309,6 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
         mbar_init_fence();
     }
     if (tid < 64) reinterpret_cast<uint32_t *>(zero)[tid] = 0u;
+    for (int i = tid; i < kMaxCtaTiles; i += kThreads) tile_cnt[i] = 0;
     __syncthreads();
     // Nothing is requested before the wait: a CTA that starts late (its SM freed late by
     // the previous kernel) would otherwise queue its x loads behind its own weight copies,
@@ -360,6 +366,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     int st = 0;
     uint32_t phase = 0;
     int rt = (c0 + warp) / KC, kc = (c0 + warp) - ((c0 + warp) / KC) * KC;
+    // Row tiles split between CTAs: the CTA holding a tile's first item owns the tile and
+    // adds the other pieces, which the CTAs that follow store as (value, epoch) pairs.  The
+    // owner reaches its piece last (the end of its range), while the later pieces open
+    // their CTAs' ranges and are stored as soon as their items are done.  Waits only go
+    // from a CTA to higher ones, which store before they wait on anything: all CTAs of the
+    // grid fit on the GPU at once (one per SM).
+    const int rt_first = c0 / KC;
+    // One warp per tile, one lane per row: add the CTA's items of tile rt ([a, b)) in K
+    // order, then write y (whole tile), store the piece (a later piece) or collect the
+    // later pieces and write y (owned).
+    auto finish_tile = [&](int rt, int a, int b) {
+        const int tile_first = rt * KC, tile_end = tile_first + KC;
+        float sum = 0.f;
+        for (int i = a; i < b; i++) sum += slots[(i - c0) * kItemRows + lane];
+        if (a > tile_first) {
+            st_pair(partials + (int64_t)a * kItemRows + lane, sum);
+            return;
+        }
+        int s = b, c2 = (int)blockIdx.x + 1;
+        while (s < tile_end) {
+            int e2 = (int)((int64_t)I * (c2 + 1) / C);  // the piece of CTA c2 is [s, e2)
+            e2 = e2 < tile_end ? e2 : tile_end;
+            sum += wait_pairs(partials + (int64_t)s * kItemRows, lane);
+            s = e2;
+            c2++;
+        }
+        const int row = rt * kItemRows + lane;
+        if (row < N) y[row] = float_to_half_bits(sum);
+    };
+
     auto process = [&](int q) {
         const int i = c0 + warp + q * kConsumers;
         if (ok) {
@@ -455,32 +491,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
         float mine = v[0];
         if (!ok) mine = __int_as_float(0x7fc00000);
         slots[(i - c0) * kItemRows + R] = mine;
+        // the warp that completes the CTA's part of a row tile finalises it
+        __syncwarp();
+        int done = 0;
+        if (lane == 0) {
+            __threadfence_block();  // this warp's slot stores before the count
+            done = atomicAdd(tile_cnt + (rt - rt_first), 1) + 1;
+            __threadfence_block();  // the other warps' slot stores before the reads below
+        }
+        done = __shfl_sync(0xffffffffu, done, 0);
+        const int tile_first = rt * KC;
+        const int a = c0 > tile_first ? c0 : tile_first;
+        const int b = c1 < tile_first + KC ? c1 : tile_first + KC;
+        if (done == b - a) finish_tile(rt, a, b);
         if (++st == kStages) st = 0, phase ^= 1u;
         advance(rt, kc);
     };
 
-    // Row tiles split between CTAs: the CTA holding a tile's first item owns the tile and
-    // adds the other pieces, which the CTAs that follow store as (value, epoch) pairs.  The
-    // owner reaches its piece last (the end of its range), while the later pieces open
-    // their CTAs' ranges: a CTA's first tile, when it is such a piece, is stored as soon as
-    // its items are done.  Waits only go from a CTA to higher ones, which store before
-    // they wait on anything: all CTAs of the grid fit on the GPU at once (one per SM).
-    const int rt_first = c0 / KC, rt_last = c1 > c0 ? (c1 - 1) / KC : rt_first - 1;
-    const int first_end = c1 < (rt_first + 1) * KC ? c1 : (rt_first + 1) * KC;
-    const bool early = c0 > rt_first * KC && first_end < c1;
-    const int q_pub = early ? (first_end - c0 - 1) / kConsumers : -1;  // the round of its last item
-    auto publish = [&](int a, float v) { st_pair(partials + (int64_t)a * kItemRows + lane, v); };
-    if (early) {
-        for (int q = 0; q <= q_pub; q++)
-            if (q < nq) process(q);
-        __syncthreads();  // the first tile's slots are written
-        if (warp == kConsumers - 1) {  // the last warp has the fewest items (round-robin)
-            float v = 0.f;
-            for (int i = c0; i < first_end; i++) v += slots[(i - c0) * kItemRows + lane];
-            publish(c0, v);
-        }
-    }
-    for (int q = q_pub + 1; q < nq; q++) process(q);
+    for (int q = 0; q < nq; q++) process(q);
     if (kAsyncScales) cp_async_wait_all();
     // after a wait gave up: let the box copies already started land before the CTA exits
     if (!ok && lane == 0) {
@@ -490,32 +518,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
             mbar_wait(full + dst, dph);
             if (++dst == kStages) dst = 0, dph ^= 1u;
         }
-    }
-    __syncthreads();  // every slot is written
-
-    // ---- row tiles: add each tile's items in K order (one warp per tile, one lane per row)
-    for (int rt = rt_first + warp; rt <= rt_last; rt += kConsumers) {
-        const int tile_first = rt * KC, tile_end = tile_first + KC;
-        const int a = c0 > tile_first ? c0 : tile_first;
-        const int b = c1 < tile_end ? c1 : tile_end;
-        if (rt == rt_first && early) continue;  // stored already
-        float sum = 0.f;
-        for (int i = a; i < b; i++) sum += slots[(i - c0) * kItemRows + lane];
-        if (a > tile_first) {  // a later piece of a tile owned by an earlier CTA
-            publish(a, sum);
-            continue;
-        }
-        // owned (or whole): add the pieces of the CTAs that follow, in K order
-        int s = b, c2 = (int)blockIdx.x + 1;
-        while (s < tile_end) {
-            int e2 = (int)((int64_t)I * (c2 + 1) / C);  // the piece of CTA c2 is [s, e2)
-            e2 = e2 < tile_end ? e2 : tile_end;
-            sum += wait_pairs(partials + (int64_t)s * kItemRows, lane);
-            s = e2;
-            c2++;
-        }
-        const int row = rt * kItemRows + lane;
-        if (row < N) y[row] = float_to_half_bits(sum);
     }
 }
 
@@ -540,7 +542,8 @@ Shape shape_of(int64_t N, int64_t K, int sm_count) {
 }  // namespace
 
 static_assert(kConsumers * kStages * (kItemBytes + kScaleRingBytes) + (kMaxK / kItemK) * 4 * (kXGroupBytes + 8) +
-                  kMaxCtaItems * kItemRows * 4 + 256 + kConsumers * kStages * 8 + 1024 <= 232448,
+                  kMaxCtaItems * kItemRows * 4 + kMaxCtaTiles * 4 + 15 + 256 + kConsumers * kStages * 8 + 1024 <=
+                  232448,
               "shared-memory layout exceeds the per-CTA limit at the largest K");
 
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt) {
@@ -562,6 +565,9 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
                              int64_t N, int64_t K, const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
     const Layout lay = make_layout((int)K);
     if (lay.total > dev.smem_optin) return cudaErrorInvalidValue;
+    // the kernel's 128-bit and barrier accesses rely on these alignments
+    if ((lay.sring | lay.xfrag | lay.sxf | lay.slots | lay.zero) % 16 != 0 || lay.full % 8 != 0)
+        return cudaErrorInvalidValue;
     EncodeTiledFn encode = encode_fn();
     if (!encode) return cudaErrorNotSupported;
     CUtensorMap wmap;
