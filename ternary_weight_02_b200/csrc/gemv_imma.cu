@@ -59,6 +59,9 @@ constexpr int kScaleRingBytes = kItemRows * 8;          // per stage: the item's
 constexpr int kXHalfBytes = 144;                        // one part (hi or lo) of a group's fragments, padded
 constexpr int kXGroupBytes = 2 * kXHalfBytes;
 constexpr int kStages = 2;
+// Items each warp requests before building x~; the rest of its ring after: every
+// warp's first item then arrives in the first half of the start-up burst.
+constexpr int kFirstIssue = 1;
 constexpr int kMaxCtaItems = 96;                        // slot buffer: 96 x 32 floats
 constexpr int kMaxCtaTiles = kMaxCtaItems + 2;          // row tiles one CTA's items touch
 constexpr int64_t kMaxK = 24576;  // the layout below then fits the 227 KB a CTA may use
@@ -164,43 +167,43 @@ __device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag,
             v[i] = fmaf(sgn, v[i], p);  // exact sign flip, one rounding: same as the add or subtract
         }
     }
+    // v holds the unnormalised transform: 1/sqrt(128) is folded into the quantisation
     float am = 0.f;
 #pragma unroll
-    for (int i = 0; i < 16; i++) {
-        v[i] *= kHadamardNorm;
-        am = fmaxf(am, fabsf(v[i]));
-    }
+    for (int i = 0; i < 16; i++) am = fmaxf(am, fabsf(v[i]));
 #pragma unroll
     for (int b = 1; b < 8; b <<= 1) am = fmaxf(am, __shfl_xor_sync(gmask, am, b));
-    const uint32_t mb = __float_as_uint(am);
-    const int E = (int)(mb >> 23) - 127;  // am < 2^(E+1)
-    int e = mb == 0u ? 0 : 13 - E;        // am * 2^e < 2^14
+    const uint32_t mb = __float_as_uint(am * kHadamardNorm);  // max |x'| of the group
+    const int E = (int)(mb >> 23) - 127;  // max |x'| < 2^(E+1)
+    int e = mb == 0u ? 0 : 13 - E;        // max |x'| * 2^e < 2^14
     e = e < -126 ? -126 : (e > 100 ? 100 : e);
-    const float sc = __int_as_float((e + 127) << 23);
+    const float sc = __int_as_float((e + 127) << 23) * kHadamardNorm;
     // 2^-e / 64: the GEMV's sums come out 64 times too large (code slots weighted 4^(3-j))
     const float f = E == 128 ? __int_as_float(0x7fc00000) : __int_as_float((121 - e) << 23);  // Inf/NaN -> NaN
-    int q[16];
+    // q = rint(v * sc) by the magic-number rounding: v*sc + (1.5*2^23 + 128) lands in
+    // [2^23, 2^24), where floats are the integers, so its bits minus those of 1.5*2^23
+    // are q + 128 (|q| <= 2^14 + 1).  Then the high byte hi = (q + 128) >> 8 is byte 1
+    // of qa = q + 128 and the low byte lo = q - 256 hi is byte 0 of qa with its top bit
+    // flipped.
+    int qa[16];
     int sum = 0;
 #pragma unroll
     for (int i = 0; i < 16; i++) {
-        q[i] = __float2int_rn(v[i] * sc);
-        sum += q[i];
+        qa[i] = (int)(__float_as_uint(fmaf(v[i], sc, 12583040.0f)) - 0x4B400000u);
+        sum += qa[i];
     }
 #pragma unroll
     for (int b = 1; b < 8; b <<= 1) sum += __shfl_xor_sync(gmask, sum, b);
-    // lane l = 2s + hb: chunk 2s + (j >> 1), byte 8 (j & 1) + 4 hb + i
+    sum -= 128 * kGroup;  // the 128 added to each of the group's q
+    // lane l = 2s + hb: chunk 2s + (j >> 1), byte 8 (j & 1) + 4 hb + i (element 16l + 4i + j)
     uint8_t *dst = xfrag + g * kXGroupBytes + (l >> 1) * 32 + (l & 1) * 4;
 #pragma unroll
     for (int j = 0; j < 4; j++) {
-        uint32_t whi = 0u, wlo = 0u;
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            const int qq = q[4 * i + j];
-            const int hi = (qq + 128) >> 8;
-            const int lo = qq - (hi << 8);
-            whi |= ((uint32_t)hi & 0xffu) << (8 * i);
-            wlo |= ((uint32_t)lo & 0xffu) << (8 * i);
-        }
+        const uint32_t a0 = (uint32_t)qa[j], a1 = (uint32_t)qa[4 + j];
+        const uint32_t a2 = (uint32_t)qa[8 + j], a3 = (uint32_t)qa[12 + j];
+        const uint32_t whi = __byte_perm(__byte_perm(a0, a1, 0x0051), __byte_perm(a2, a3, 0x0051), 0x5410);
+        const uint32_t wlo =
+            __byte_perm(__byte_perm(a0, a1, 0x0040), __byte_perm(a2, a3, 0x0040), 0x5410) ^ 0x80808080u;
         const int off = (j >> 1) * 16 + (j & 1) * 8;
         *reinterpret_cast<uint32_t *>(dst + off) = whi;
         *reinterpret_cast<uint32_t *>(dst + kXHalfBytes + off) = wlo;
@@ -336,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
             if (pq >= nquads) pq -= nquads;
             if (quad < nquads) load_x8(x, pq * 4 + (lane >> 3), G, lane & 7, xr[r][0], xr[r][1]);
         }
-        for (int q = 0; q < kStages; q++) issue(q);
+        for (int q = 0; q < kFirstIssue; q++) issue(q);
 #pragma unroll
         for (int r = 0; r < kRounds; r++) {
             const int quad = warp + r * kConsumers;
@@ -346,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
                 build_group8(xr[r][0], xr[r][1], xf, reinterpret_cast<int2 *>(smem + L.sxf), pq * 4 + (lane >> 3),
                              lane);
         }
+        for (int q = kFirstIssue; q < kStages; q++) issue(q);
     }
     __syncthreads();
 
