@@ -157,7 +157,7 @@ size_t workspace_for(int algo, int64_t M, int64_t N, int64_t K, int fmt, int spl
     switch (algo) {
         case BONSAI_ALGO_GEMV: return gemv_workspace_bytes(N, K, fmt, split_k, info);
         case BONSAI_ALGO_SKINNY: return skinny_workspace_bytes(M, N, K, fmt, split_k, info);
-        case BONSAI_ALGO_GEMM: return gemm_workspace_bytes(M, N, K, fmt);
+        case BONSAI_ALGO_GEMM: return gemm_workspace_bytes(M, N, K, fmt, info);
         case BONSAI_ALGO_IMMA: return 0;
         default: return simple_workspace_bytes(M, N, K);
     }
@@ -369,7 +369,7 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
             need = v > need ? v : need;
         }
         if (gemm_supported(M, N, K, fmt)) {
-            v = gemm_workspace_bytes(M, N, K, fmt);
+            v = gemm_workspace_bytes(M, N, K, fmt, st->info);
             need = v > need ? v : need;
         }
     }

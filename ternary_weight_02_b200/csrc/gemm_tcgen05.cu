@@ -12,18 +12,22 @@
 //     (hadamard.cu).  Rotating inside the GEMM would redo each 128 x 128 A tile's FWHT
 //     for every one of the N/256 column tiles; as a pass it costs one read and one
 //     write of x, under 1% of the GEMM's time at these shapes.
-//  2. this kernel.  A CTA computes one 128 x 256 tile of y over all of K in 64-wide
-//     stages (4-stage ring):
+//  2. this kernel, persistent: at most one CTA per SM, each taking whole tiles in waves
+//     and then an even share of the last tiles' 64-wide K stages (stream-K, below), so
+//     that no SM idles in a partial last wave.  A tile is kAcc x 128 rows x 256
+//     columns of y; per stage (3- or 4-deep rings):
 //     - warp 0 (one thread): TMA loads of the x' tile (128 rows x 64, 128-byte swizzle);
-//     - warp 1: allocates 256 TMEM columns; one thread issues tcgen05.mma
+//     - warp 1: allocates the TMEM accumulators; one thread issues tcgen05.mma
 //       (M=128, N=256, K=16, kind::f16, FP32 accumulate) and commits each stage back;
 //     - warps 2..9 (256 threads, one weight row each): expand the packed trits of a
 //       128-weight group times its FP16 scale into two 64-wide FP16 B stages, written
 //       in the same 128-byte-swizzled K-major layout the MMA descriptors describe
-//       (t * s is exact in FP16); then the epilogue: tcgen05.ld of the accumulator,
-//       FP32 -> FP16 (nearest even), stores to y.
+//       (t * s is exact in FP16); after each piece of a tile, the epilogue:
+//       tcgen05.ld of the accumulator, then FP16 (nearest even) stores to y, or the
+//       FP32 hand-over of a split tile.
 // Every wait is bounded: if one gives up, the CTA stops issuing work, waits for the
-// copies and MMAs it started, frees its tensor memory and writes NaN to its tile.
+// copies and MMAs it started, frees its tensor memory and writes NaN to its tiles (and
+// hands NaN over for a split one).
 #include <cuda.h>
 
 #include "common.cuh"
@@ -50,7 +54,7 @@ struct Cfg {
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kStages * kAStage;
     static constexpr int kOffBar = kOffB + kStages * B_STAGE_BYTES;
-    static constexpr int kNumBars = 3 * kStages + 1;  // full_a, full_b, empty, done
+    static constexpr int kNumBars = 3 * kStages + 3;  // full_a, full_b, empty, done, tmem_free, fin
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 8;
     static constexpr int kOffLut = kOffAbort + 8;
@@ -90,16 +94,25 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// 64 columns of this warp's 32 TMEM lanes (lane i of the warp: TMEM lane 32q + i) in one
+// load; the wait is in the same statement, so no use of r can be scheduled before it.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, "
+        "%35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, "
+        "%56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+          "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+          "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
 }
 
 // ---------------------------------------------------------------- trit expansion
@@ -193,29 +206,104 @@ __device__ __forceinline__ void group_codes(const GroupRaw &raw, const uint32_t 
     }
 }
 
+// ---------------------------------------------------------------- cross-CTA hand-over
+
+// A tile piece's FP32 partial sums go to the CTA's own slot in the workspace; a flag
+// word per CTA (zero at rest) says that the slot is complete.  The writer's threads
+// fence, meet at a named barrier, and one of them releases the flag; the owner acquires
+// it (every lane polls, bounded), reads the slot through L2 and later clears the flag.
+__device__ __forceinline__ void flag_release(unsigned int *p, unsigned int v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned int flag_acquire(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// Bounded wait of a whole warp for *p == 1.
+__device__ __forceinline__ bool flag_wait(const unsigned int *p) {
+    for (uint32_t i = 0; i < kSpinLimit; i++) {
+        if (__all_sync(0xffffffffu, flag_acquire(p) == 1u)) return true;
+        __nanosleep(64);
+    }
+    return false;
+}
+// The eight expansion/epilogue warps (256 threads) meet here; barrier 0 is __syncthreads.
+__device__ __forceinline__ void expand_warps_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 // ---------------------------------------------------------------- kernel
 
+// Work split (whole-tile waves, then stream-K).  The T tiles of y (kAcc*128 rows x 256
+// columns, numbered with the row tile fastest) are taken by C persistent CTAs:
+//  1. W = floor(T/C) - 1 waves of whole tiles (none if T < 2C): CTA b takes tiles b,
+//     b + C, ..., so that the C tiles in flight at once are consecutive and share x' row
+//     tiles and weight columns in L2;
+//  2. the remaining tiles (one to two waves' worth) are cut into units of one 64-wide K
+//     stage, unit u being stage u % nk of remaining tile u / nk, and CTA b takes units
+//     [Ur*b/C, Ur*(b+1)/C) in order, as a run of "pieces" (its units of one tile).  Only
+//     the first of these pieces can continue a tile that an earlier CTA started, and only
+//     the last can be a tile's start that a later CTA continues:
+//     - a whole tile is written to y directly;
+//     - a continuing piece stores its FP32 sums in the CTA's slot and raises its flag;
+//     - a tile's first piece (its "owner") waits for the flags of the CTAs that continue
+//       the tile, adds their slots in K order, writes y and clears those flags.
+// A continuing piece comes before anything else of its CTA's split share, and the owner's
+// piece last: the waits are short, and they only go from a CTA to later ones, which never
+// wait before they have stored (all CTAs of the grid are resident at once, one per SM).
 template <int kFmt, int kAcc>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap a_map, const uint8_t *__restrict__ packed,
-    const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, int M, int N, int K) {
+    const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
+    unsigned int *__restrict__ flags, int M, int N, int K, int mt) {
     using C = Cfg<kAcc>;
     constexpr int STAGES = C::kStages;
+    constexpr int kSlotFloats = C::kTileM * BN;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment of the tile area (128-byte swizzle atoms)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem + C::kOffA;
     uint8_t *sB = smem + C::kOffB;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
-    uint64_t *full_a = bars, *full_b = bars + STAGES, *empty = bars + 2 * STAGES, *done = bars + 3 * STAGES;
+    uint64_t *full_a = bars, *full_b = bars + STAGES, *empty = bars + 2 * STAGES;
+    uint64_t *done = bars + 3 * STAGES, *tmem_free = done + 1, *fin = done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffAbort);
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem + C::kOffLut);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tile_m = blockIdx.x, tile_n = blockIdx.y;
-    const int num_k = K / BK;
+    const int nk = K / BK;
     const int64_t G = K / kGroup;
+    const int nctas = (int)gridDim.x, cta = (int)blockIdx.x;
+    // whole-tile waves first (CTA b: tiles b, b + C, ...), then the last one or two
+    // waves' worth of tiles split by units
+    const int T = mt * ((N + BN - 1) / BN);
+    const int W = T / nctas >= 2 ? T / nctas - 1 : 0;
+    const int Tdp = W * nctas;
+    const int Ur = (T - Tdp) * nk;
+    auto range_end = [&](int c) { return (int)((int64_t)Ur * (c + 1) / nctas); };
+    const int u_begin = (int)((int64_t)Ur * cta / nctas), u_end = range_end(cta);
+    const int n_mine = W * nk + (u_end - u_begin);  // this CTA's units
+    // the piece that starts at this CTA's unit v: tile s (row tile fastest), stages
+    // [kb, ke); tr: the tile's index among the split ones (-1 for a whole-tile wave)
+    struct Piece {
+        int s, kb, ke, tr;
+    };
+    auto piece_at = [&](int v) {
+        Piece p;
+        if (v < W * nk) {
+            p.s = cta + (v / nk) * nctas;
+            p.kb = 0;
+            p.ke = nk;
+            p.tr = -1;
+        } else {
+            const int u = u_begin + (v - W * nk);
+            p.tr = u / nk;
+            p.kb = u - p.tr * nk;
+            p.ke = p.kb + (u_end - u) < nk ? p.kb + (u_end - u) : nk;
+            p.s = Tdp + p.tr;
+        }
+        return p;
+    };
 
     if (tid == 0) {
         for (int st = 0; st < STAGES; st++) {
@@ -224,6 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
             mbar_init(empty + st, 1);
         }
         mbar_init(done, 1);
+        mbar_init(tmem_free, kExpandWarps);
+        mbar_init(fin, 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -252,128 +342,243 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (x' tiles)
         if (lane == 0) {
-            int issued = 0;
-            for (int ks = 0; ks < num_k; ks++) {
-                const int st = ks % STAGES;
-                const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-                if (*abort_flag || !mbar_wait(empty + st, ph ^ 1u)) {
-                    *abort_flag = 1;
-                    break;
-                }
-                mbar_arrive_expect_tx(full_a + st, C::kAStage);
+            int it = 0;  // units issued: ring position
+            for (int v = 0; v < n_mine && !*abort_flag;) {
+                const Piece p = piece_at(v);
+                const int tm = p.s % mt;
+                for (int ks = p.kb; ks < p.ke; ks++, it++) {
+                    const int st = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    if (*abort_flag || !mbar_wait(empty + st, ph ^ 1u)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(full_a + st, C::kAStage);
 #pragma unroll
-                for (int a = 0; a < kAcc; a++)
-                    tma_load_2d(sA + st * C::kAStage + a * (BM * BK * 2), &a_map, full_a + st, ks * BK,
-                                tile_m * C::kTileM + a * BM);
-                issued = ks + 1;
+                    for (int a = 0; a < kAcc; a++)
+                        tma_load_2d(sA + st * C::kAStage + a * (BM * BK * 2), &a_map, full_a + st, ks * BK,
+                                    tm * C::kTileM + a * BM);
+                }
+                v += p.ke - p.kb;
             }
             // the copies this thread started land before the CTA may exit
-            for (int ks = issued - STAGES < 0 ? 0 : issued - STAGES; ks < issued; ks++)
-                mbar_wait(full_a + (ks % STAGES), (uint32_t)(ks / STAGES) & 1u);
+            for (int i = it - STAGES < 0 ? 0 : it - STAGES; i < it; i++)
+                mbar_wait(full_a + (i % STAGES), (uint32_t)(i / STAGES) & 1u);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            for (int ks = 0; ks < num_k; ks++) {
-                const int st = ks % STAGES;
-                const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-                if (*abort_flag || !mbar_wait(full_a + st, ph) || !mbar_wait(full_b + st, ph)) {
+            int it = 0, pc = 0;
+            for (int v = 0; v < n_mine && !*abort_flag; pc++) {
+                const Piece p = piece_at(v);
+                v += p.ke - p.kb;
+                // the accumulator is free once the previous piece's epilogue has read it
+                if (pc > 0 && !mbar_wait(tmem_free, (uint32_t)(pc - 1) & 1u)) {
                     *abort_flag = 1;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t b0 = saddr(sB + st * B_STAGE_BYTES);
-#pragma unroll
-                for (int kk = 0; kk < BK / 16; kk++) {
-                    const uint64_t bdesc = desc_sw128(b0 + kk * 32);
-#pragma unroll
-                    for (int a = 0; a < kAcc; a++) {
-                        const uint32_t a0 = saddr(sA + st * C::kAStage + a * (BM * BK * 2));
-                        mma_f16(tmem + (uint32_t)(a * 256), desc_sw128(a0 + kk * 32), bdesc,
-                                (ks > 0 || kk > 0) ? 1u : 0u);
+                for (int ks = p.kb; ks < p.ke; ks++, it++) {
+                    const int st = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    if (*abort_flag || !mbar_wait(full_a + st, ph) || !mbar_wait(full_b + st, ph)) {
+                        *abort_flag = 1;
+                        break;
                     }
+                    tc_fence_after();
+                    const uint32_t b0 = saddr(sB + st * B_STAGE_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; kk++) {
+                        const uint64_t bdesc = desc_sw128(b0 + kk * 32);
+#pragma unroll
+                        for (int a = 0; a < kAcc; a++) {
+                            const uint32_t a0 = saddr(sA + st * C::kAStage + a * (BM * BK * 2));
+                            mma_f16(tmem + (uint32_t)(a * 256), desc_sw128(a0 + kk * 32), bdesc,
+                                    (ks > p.kb || kk > 0) ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(empty + st);  // frees the stage when these MMAs have read it
                 }
-                mma_commit(empty + st);  // frees the stage when these MMAs have read it
+                if (*abort_flag) break;
+                mma_commit(done);  // the piece's sums are complete in tensor memory
             }
-            mma_commit(done);  // all MMAs issued by this thread are complete
+            // every MMA this thread issued has completed before tensor memory is freed
+            mma_commit(fin);
+            mbar_wait(fin, 0);
         }
     } else {
-        // ------------------------------------------------ trit expansion (one row per thread)
-        const int r = tid - 64;                      // 0 .. 255: row of the B tile
-        const int64_t n = (int64_t)tile_n * BN + r;  // weight row
-        const bool valid = n < N;
-        GroupRaw cur, nxt;
-        if (valid) load_group<kFmt>(packed, scales, n, G, 0, cur);
-        uint32_t cw[8];
-        __half2 s2 = __float2half2_rn(0.f);
-        for (int ks = 0; ks < num_k; ks++) {
-            const int g = ks >> 1, hf = ks & 1;  // a 128-weight group fills two 64-wide stages
-            if (hf == 0) {
-                if (valid && g + 1 < (int)G) load_group<kFmt>(packed, scales, n, G, g + 1, nxt);  // in flight
-                if (valid) {
-                    group_codes<kFmt>(cur, lut, cw);
-                    const __half sh = __ushort_as_half(cur.scale);
-                    s2 = __halves2half2(sh, sh);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 8; i++) cw[i] = 0x55555555u;  // all trits zero
-                }
-            }
-            const int st = ks % STAGES;
-            const uint32_t ph = (uint32_t)(ks / STAGES) & 1u;
-            // every lane acquires the stage itself; the verdict is made warp-uniform
-            const bool free_ok = !*abort_flag && mbar_wait(empty + st, ph ^ 1u);
-            if (!__all_sync(0xffffffffu, free_ok)) {
-                *abort_flag = 1;
-                break;
-            }
-            uint8_t *stage = sB + st * B_STAGE_BYTES;
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                uint32_t out[8];
-                expand_word(hf ? cw[4 + i] : cw[i], s2, out);  // weights 64hf + 16i .. +15
-                st_chunk(stage, r, 2 * i, out);
-                st_chunk(stage, r, 2 * i + 1, out + 4);
-            }
-            // make the generic-proxy stores visible to the tensor core, then signal
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(full_b + st);
-            if (hf == 1) cur = nxt;
-        }
-
-        // ------------------------------------------------ epilogue
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(done, 0)) && !*abort_flag;
-        tc_fence_after();
+        // ------------------------------------------------ trit expansion (one row per thread), epilogues
+        const int r = tid - 64;            // 0 .. 255: row of the B tile
         const int q = warp & 3;            // TMEM lane quadrant this warp may read
-        const int half = (warp - 2) >> 2;  // which 128 columns
-#pragma unroll 1
-        for (int a = 0; a < kAcc; a++) {
-            const int m = tile_m * C::kTileM + a * BM + 32 * q + lane;
-#pragma unroll 1
-            for (int c = 0; c < 4; c++) {
-                const int col = half * 128 + 32 * c;
-                uint32_t v[32];
-                __syncwarp();
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 256 + col), v);
-                if (m >= M) continue;
-                const int64_t n0 = (int64_t)tile_n * BN + col;
-                uint16_t *yr = y + (int64_t)m * N + n0;
-                if (ok && n0 + 32 <= N && (N & 7) == 0) {
-                    uint32_t h[16];
+        const int half = (warp - 2) >> 2;  // which 128 columns of the tile it writes
+        int it = 0, pc = 0;
+        bool live = true;
+        for (int v = 0; v < n_mine; pc++) {
+            const Piece p = piece_at(v);
+            v += p.ke - p.kb;
+            const int tm = p.s % mt, tn = p.s / mt;
+            const int64_t n = (int64_t)tn * BN + r;  // weight row
+            const bool valid = n < N;
+            if (live) {
+                GroupRaw cur, nxt;
+                if (valid) load_group<kFmt>(packed, scales, n, G, p.kb >> 1, cur);
+                const int g_last = (p.ke - 1) >> 1;
+                uint32_t cw[8];
+                __half2 s2 = __float2half2_rn(0.f);
+                for (int ks = p.kb; ks < p.ke; ks++, it++) {
+                    const int g = ks >> 1, hf = ks & 1;  // a 128-weight group fills two 64-wide stages
+                    if (ks == p.kb || hf == 0) {
+                        if (valid && g < g_last) load_group<kFmt>(packed, scales, n, G, g + 1, nxt);  // in flight
+                        if (valid) {
+                            group_codes<kFmt>(cur, lut, cw);
+                            const __half sh = __ushort_as_half(cur.scale);
+                            s2 = __halves2half2(sh, sh);
+                        } else {
 #pragma unroll
-                    for (int i = 0; i < 16; i++) {
-                        const __half2 p2 =
-                            __floats2half2_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                        h[i] = *reinterpret_cast<const uint32_t *>(&p2);
+                            for (int i = 0; i < 8; i++) cw[i] = 0x55555555u;  // all trits zero
+                        }
                     }
-                    uint4 *dst = reinterpret_cast<uint4 *>(yr);
+                    const int st = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    // every lane acquires the stage itself; the verdict is made warp-uniform
+                    const bool free_ok = !*abort_flag && mbar_wait(empty + st, ph ^ 1u);
+                    if (!__all_sync(0xffffffffu, free_ok)) {
+                        *abort_flag = 1;
+                        live = false;
+                        break;
+                    }
+                    uint8_t *stage = sB + st * B_STAGE_BYTES;
 #pragma unroll
-                    for (int i = 0; i < 4; i++) dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
-                } else {
-                    for (int i = 0; i < 32; i++)
-                        if (n0 + i < N) yr[i] = ok ? float_to_half_bits(__uint_as_float(v[i])) : (uint16_t)0x7E00u;
+                    for (int i = 0; i < 4; i++) {
+                        uint32_t out[8];
+                        expand_word(hf ? cw[4 + i] : cw[i], s2, out);  // weights 64hf + 16i .. +15
+                        st_chunk(stage, r, 2 * i, out);
+                        st_chunk(stage, r, 2 * i + 1, out + 4);
+                    }
+                    // make the generic-proxy stores visible to the tensor core, then signal
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(full_b + st);
+                    if (hf == 1) cur = nxt;
                 }
+            }
+
+            // ---------------------------------------------- epilogue of the piece
+            if (live) live = __all_sync(0xffffffffu, mbar_wait(done, (uint32_t)pc & 1u)) && !*abort_flag;
+            const bool ok = live;
+            tc_fence_after();
+            const bool continues = p.kb > 0;                  // a later piece of a tile
+            const bool owner = p.kb == 0 && p.ke < nk;        // first piece, others follow
+            const int tile_end = (p.tr + 1) * nk;  // in split units
+            bool got = true;  // the later pieces all arrived (owner)
+            if (owner)
+                for (int c2 = cta + 1, s = u_end; s < tile_end; s = range_end(c2), c2++)
+                    got = flag_wait(flags + c2) && got;
+            // Hand-over slots are kept in the order of the accumulator fragments (accumulator a,
+            // warp, 32-column chunk c, float4 i, lane), so that writer and owner, which use the
+            // same thread mapping, both move 512 contiguous bytes per warp instruction.
+            const int w8 = warp - 2;
+            auto slot_at = [&](int c2, int a, int c) {
+                return reinterpret_cast<float4 *>(partials + (size_t)c2 * kSlotFloats) +
+                       ((size_t)((a * kExpandWarps + w8) * 4 + c) * 8) * 32 + lane;
+            };
+            // y goes out through this warp's 8 KB of the B ring (idle until the next piece's
+            // expansion): 32 rows x 128 FP16 columns, 16-byte chunks swizzled by the row.
+            uint8_t *stage_y = sB + w8 * 8192;
+#pragma unroll 1
+            for (int a = 0; a < kAcc; a++) {
+#pragma unroll 1
+                for (int cp = 0; cp < 2; cp++) {
+                    uint32_t v[64];
+                    __syncwarp();
+                    if (ok) {
+                        tmem_ld64(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 256 + half * 128 + 64 * cp), v);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 64; i++) v[i] = 0x7fc00000u;
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < 2; cc++) {
+                        const int c = 2 * cp + cc;  // 32-column chunk of this warp's 128 columns
+                        uint32_t *vc = v + 32 * cc;
+                        if (continues) {
+                            float4 *dst = slot_at(cta, a, c);
+#pragma unroll
+                            for (int i = 0; i < 8; i++)
+                                dst[32 * i] = make_float4(__uint_as_float(vc[4 * i]), __uint_as_float(vc[4 * i + 1]),
+                                                          __uint_as_float(vc[4 * i + 2]), __uint_as_float(vc[4 * i + 3]));
+                            continue;
+                        }
+                        if (owner) {
+                            for (int c2 = cta + 1, s = u_end; s < tile_end; s = range_end(c2), c2++) {
+                                const float4 *src = slot_at(c2, a, c);
+                                float4 w[8];
+#pragma unroll
+                                for (int i = 0; i < 8; i++) w[i] = __ldcg(src + 32 * i);
+#pragma unroll
+                                for (int i = 0; i < 8; i++) {
+                                    vc[4 * i] = __float_as_uint(__uint_as_float(vc[4 * i]) + w[i].x);
+                                    vc[4 * i + 1] = __float_as_uint(__uint_as_float(vc[4 * i + 1]) + w[i].y);
+                                    vc[4 * i + 2] = __float_as_uint(__uint_as_float(vc[4 * i + 2]) + w[i].z);
+                                    vc[4 * i + 3] = __float_as_uint(__uint_as_float(vc[4 * i + 3]) + w[i].w);
+                                }
+                            }
+                            if (!got)
+#pragma unroll
+                                for (int i = 0; i < 32; i++) vc[i] = 0x7fc00000u;
+                        }
+                        // FP16 (nearest even) into the staging row of this lane
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            uint32_t h[4];
+#pragma unroll
+                            for (int e = 0; e < 4; e++) {
+                                const __half2 p2 = __floats2half2_rn(__uint_as_float(vc[8 * j + 2 * e]),
+                                                                     __uint_as_float(vc[8 * j + 2 * e + 1]));
+                                h[e] = *reinterpret_cast<const uint32_t *>(&p2);
+                            }
+                            *reinterpret_cast<uint4 *>(stage_y + lane * 256 + (((4 * c + j) ^ (lane & 7)) << 4)) =
+                                make_uint4(h[0], h[1], h[2], h[3]);
+                        }
+                    }
+                }
+                if (continues) continue;
+                __syncwarp();
+                // two rows of 256 bytes per instruction: lane (row parity, 16-byte chunk)
+                const int ch = lane & 15;
+                const int64_t n0 = (int64_t)tn * BN + half * 128 + ch * 8;
+#pragma unroll 4
+                for (int i = 0; i < 16; i++) {
+                    const int row = 2 * i + (lane >> 4);
+                    const int m = tm * C::kTileM + a * BM + 32 * q + row;
+                    const uint4 val = *reinterpret_cast<const uint4 *>(stage_y + row * 256 + ((ch ^ (row & 7)) << 4));
+                    if (m >= M || n0 >= N) continue;
+                    uint16_t *yr = y + (int64_t)m * N + n0;
+                    if (n0 + 8 <= N && (N & 7) == 0) {
+                        *reinterpret_cast<uint4 *>(yr) = val;
+                    } else {
+                        const uint32_t wv[4] = {val.x, val.y, val.z, val.w};
+                        for (int e = 0; e < 8 && n0 + e < N; e++) yr[e] = (uint16_t)(wv[e >> 1] >> (16 * (e & 1)));
+                    }
+                }
+                __syncwarp();  // the staging rows are rewritten by the next accumulator
+            }
+            // tensor memory has been read: the next piece's MMAs may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tmem_free);
+            if (continues) {
+                __threadfence();
+                expand_warps_sync();
+                if (r == 0) flag_release(flags + cta, 1u);
+            } else if (owner) {
+                expand_warps_sync();  // every warp has read the later pieces and its staging rows
+                if (r == 0)
+                    for (int c2 = cta + 1, s = u_end; s < tile_end; s = range_end(c2), c2++) flags[c2] = 0u;
+            } else {
+                // the next piece's expansion writes the B ring, where other warps may still
+                // be reading their staging rows
+                expand_warps_sync();
             }
         }
     }
@@ -390,24 +595,56 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
 
 // ---------------------------------------------------------------- host side
 
+// Tile and grid of one call.  Stream-K leaves no partial last wave, so two 128-row
+// accumulators (half the trit expansion per FLOP) are used whenever M > 128.
+struct GemmPlan {
+    int acc, mt, nt, nk, ctas;
+    int64_t units;
+};
+GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K, int tile_hint, int sm_count) {
+    GemmPlan p;
+    p.acc = tile_hint == 1 ? 1 : tile_hint == 2 ? 2 : (M > BM ? 2 : 1);
+    p.mt = (int)((M + (int64_t)BM * p.acc - 1) / ((int64_t)BM * p.acc));
+    p.nt = (int)((N + BN - 1) / BN);
+    p.nk = (int)(K / BK);
+    p.units = (int64_t)p.mt * p.nt * p.nk;
+    // at least kMinUnits stages per CTA, at most one CTA per SM (all resident at once)
+    constexpr int64_t kMinUnits = 4;
+    int64_t c = (p.units + kMinUnits - 1) / kMinUnits;
+    c = c < sm_count ? c : sm_count;
+    p.ctas = (int)(c > 0 ? c : 1);
+    return p;
+}
+
+constexpr size_t kSlotBytes = (size_t)2 * BM * BN * 4;  // one CTA's FP32 partial tile (two accumulators)
+
+size_t x_rot_bytes(int64_t M, int64_t K) { return (((size_t)M * (size_t)K * 2) + 255) / 256 * 256; }
+
 }  // namespace
 
 bool gemm_supported(int64_t M, int64_t N, int64_t K, int fmt) {
     (void)fmt;
-    // TMA coordinates and the grid are 32-bit; the rows of x' must be 16-byte multiples
-    return M >= 1 && M < (int64_t)1 << 30 && N < (int64_t)1 << 30 && K % kGroup == 0 && K < (int64_t)1 << 30;
+    // TMA coordinates are 32-bit; the unit count of the work split must fit an int
+    if (!(M >= 1 && M < (int64_t)1 << 30 && N >= 1 && N < (int64_t)1 << 30 && K % kGroup == 0 &&
+          K < (int64_t)1 << 30))
+        return false;
+    return ((M + BM - 1) / BM) * ((N + BN - 1) / BN) * (K / BK) < ((int64_t)1 << 31) / 4;
 }
 
-size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt) {
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, const DeviceInfo &dev) {
     (void)N;
     (void)fmt;
-    return (size_t)M * (size_t)K * 2;  // x' in FP16
+    // x' in FP16, then one partial tile per CTA
+    return x_rot_bytes(M, K) + (size_t)dev.sm_count * kSlotBytes;
 }
 
 cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                         uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int tile_hint,
                         const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
+    const GemmPlan plan = gemm_plan(M, N, K, tile_hint, dev.sm_count);
+    if (ws.data_bytes < gemm_workspace_bytes(M, N, K, fmt, dev) || plan.ctas > kMaxTiles) return cudaErrorInvalidValue;
     uint16_t *xr = reinterpret_cast<uint16_t *>(ws.data);
+    float *partials = reinterpret_cast<float *>(ws.data + x_rot_bytes(M, K));
     cudaError_t err = launch_hadamard_f16(x, xr, M, K, s, dev);
     if (err != cudaSuccess) return err;
 
@@ -423,25 +660,18 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
 
-    // one or two 128-row accumulators per CTA: two halve the trit expansion per FLOP; pick
-    // the one whose grid wastes less of the last wave
-    const int64_t nt = (N + BN - 1) / BN;
-    auto wave_eff = [&](int64_t tiles) {
-        const int64_t waves = (tiles + dev.sm_count - 1) / dev.sm_count;
-        return (double)tiles / (double)(waves * dev.sm_count);
-    };
-    const int64_t t1 = ((M + BM - 1) / BM) * nt, t2 = ((M + 2 * BM - 1) / (2 * BM)) * nt;
-    const bool two = tile_hint == 2 || (tile_hint != 1 && M > BM && wave_eff(t2) * 1.35 >= wave_eff(t1));
-    auto go = [&](auto kern, int acc, int smem) -> cudaError_t {
+    auto go = [&](auto kern, int smem) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        const dim3 grid((unsigned)((M + (int64_t)BM * acc - 1) / ((int64_t)BM * acc)), (unsigned)nt);
-        kern<<<grid, kThreads, smem, s>>>(map, packed, scales, y, (int)M, (int)N, (int)K);
+        kern<<<plan.ctas, kThreads, smem, s>>>(map, packed, scales, y, partials, ws.counters, (int)M, (int)N,
+                                               (int)K, plan.mt);
         return cudaGetLastError();
     };
     if (fmt == 1)
-        return two ? go(gemm_tcgen05_kernel<1, 2>, 2, Cfg<2>::kSmemBytes) : go(gemm_tcgen05_kernel<1, 1>, 1, Cfg<1>::kSmemBytes);
-    return two ? go(gemm_tcgen05_kernel<2, 2>, 2, Cfg<2>::kSmemBytes) : go(gemm_tcgen05_kernel<2, 1>, 1, Cfg<1>::kSmemBytes);
+        return plan.acc == 2 ? go(gemm_tcgen05_kernel<1, 2>, Cfg<2>::kSmemBytes)
+                             : go(gemm_tcgen05_kernel<1, 1>, Cfg<1>::kSmemBytes);
+    return plan.acc == 2 ? go(gemm_tcgen05_kernel<2, 2>, Cfg<2>::kSmemBytes)
+                         : go(gemm_tcgen05_kernel<2, 1>, Cfg<1>::kSmemBytes);
 }
 
 }  // namespace bonsai

@@ -84,8 +84,9 @@ cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16
 
 // ---- gemm_tcgen05.cu: prefill
 bool gemm_supported(int64_t M, int64_t N, int64_t K, int fmt);
-size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt);
-// tile_hint: 0 automatic, 1 one 128-row accumulator per CTA, 2 two (256 rows)
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, const DeviceInfo &dev);
+// tile_hint: 0 automatic, 1 one 128-row accumulator per CTA, 2 two (256 rows).  Uses
+// Workspace::counters[0, SMs) as hand-over flags (zero at rest).
 cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                         uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int tile_hint,
                         const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);

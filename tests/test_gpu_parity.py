@@ -301,7 +301,13 @@ def test_imma_rejects_what_it_cannot_run(bz):
 
 # ------------------------------------------------------------ prefill GEMM (tcgen05 / TMEM)
 
-GEMM_SMALL = [(1, 64, 128), (17, 256, 128), (130, 300, 384), (256, 512, 1024), (300, 1000, 640)]
+# The last one or two waves of tiles are split over the CTAs by 64-wide K stages (at
+# least 4 per CTA): these shapes put a tile on 1 to ~5 CTAs, so split tiles are handed
+# over through chains of one to four later pieces, and some CTAs hold several tiles.
+# (2000, 9500, 256) has more than two waves of tiles on 148 SMs: whole-tile waves first,
+# then the split remainder.
+GEMM_SMALL = [(1, 64, 128), (17, 256, 128), (130, 300, 384), (256, 512, 1024), (300, 1000, 640),
+              (600, 2000, 1152), (1000, 3000, 2048), (2000, 9500, 256)]
 
 
 @pytest.mark.parametrize("fmt", [PTQ1, PQ2])
@@ -314,6 +320,22 @@ def test_gemm_small(bz, fmt, M, N, K, tile):
     assert np.all(np.isfinite(got))
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
+
+
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+def test_gemm_split_tiles_repeatable(bz, fmt):
+    """Split tiles hand their partial sums over through flags that the owner clears:
+    the same call twice, and after a differently split shape, gives the same bits."""
+    import torch
+    p = Problem(2048, 8192, 384, fmt, seed=11)
+    q = Problem(300, 1000, 640, fmt, seed=12)
+    a = _run(bz, p, bz.BONSAI_ALGO_GEMM)
+    _run(bz, q, bz.BONSAI_ALGO_GEMM)
+    b = _run(bz, p, bz.BONSAI_ALGO_GEMM)
+    assert np.array_equal(a, b)
+    ok, rel, mx = oracle.compare(a, p.oracle_y())
+    assert ok, (rel, mx)
+    del torch
 
 
 def _sampled_reference(fmt, M, N, K, seed, ms, ns):
