@@ -9,7 +9,7 @@
 //
 // Two launches per call:
 //  1. the block-Hadamard rotation x -> x' (FP16, round to nearest) into the workspace
-//     (hadamard.cu).  Rotating inside the GEMM would redo each 128 x 128 A tile's FWHT
+//     (hadamard.cu), each 8 columns in the K order of the expanded weights.  Rotating inside the GEMM would redo each 128 x 128 A tile's FWHT
 //     for every one of the N/256 column tiles; as a pass it costs one read and one
 //     write of x, under 1% of the GEMM's time at these shapes.
 //  2. this kernel, persistent: at most one CTA per SM, each taking whole tiles in waves
@@ -118,25 +118,19 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
 // ---------------------------------------------------------------- trit expansion
 
 // One 32-bit word of 2-bit codes (code c_i = trit + 1 at bits 2i, weights w0 .. w0+15)
-// times the scale, as two 16-byte chunks of FP16: out[0..3] = weights w0..w0+7,
-// out[4..7] = weights w0+8..w0+15.  A code placed in the mantissa of 1024.0
-// (0x6400) reads as 1024 + c; subtracting 1025 gives the trit exactly and the
-// multiply by the FP16 scale is exact (the product is 0 or +-s).
-__device__ __forceinline__ void expand_word(uint32_t w, __half2 s2, uint32_t (&out)[8]) {
-    const __half2 bias = __halves2half2(__ushort_as_half(0x6401), __ushort_as_half(0x6401));  // 1025
-    uint32_t h[8];
+// times the scale s, as two 16-byte chunks of FP16: out[0..3] = weights w0 .. w0+7 and
+// out[4..7] = weights w0+8 .. w0+15, each 8 in the order [0, 4, 1, 5, 2, 6, 3, 7] (x' is
+// stored in the same order).  The value of code c is byte pair (2c, 2c+1) of the table
+// {tneg = -s | 0 << 16, tpos = +s}: -s, 0 or +s, exactly t * s.  With m = the codes j,
+// j+4, j+8, j+12 of the word as bytes, m * 0x22 + 0x10 per byte is the selector nibble
+// pair (2c, 2c+1) of each, so one byte permute makes two weights.
+__device__ __forceinline__ void expand_word(uint32_t w, uint32_t tneg, uint32_t tpos, uint32_t (&out)[8]) {
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-        // low half: code i, high half: code i + 8
-        const uint32_t m = ((w >> (2 * i)) & 0x00030003u) | 0x64006400u;
-        __half2 v = __hsub2(*reinterpret_cast<const __half2 *>(&m), bias);
-        v = __hmul2(v, s2);
-        h[i] = *reinterpret_cast<const uint32_t *>(&v);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        out[i] = __byte_perm(h[2 * i], h[2 * i + 1], 0x5410);      // low halves: codes 2i, 2i+1
-        out[4 + i] = __byte_perm(h[2 * i], h[2 * i + 1], 0x7632);  // high halves: codes 2i+8, 2i+9
+    for (int j = 0; j < 4; j++) {
+        const uint32_t m = (w >> (2 * j)) & 0x03030303u;
+        const uint32_t sel = m * 0x22u + 0x10101010u;
+        out[j] = __byte_perm(tneg, tpos, sel);            // codes j, j + 4
+        out[4 + j] = __byte_perm(tneg, tpos, sel >> 16);  // codes j + 8, j + 12
     }
 }
 
@@ -424,15 +418,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                 if (valid) load_group<kFmt>(packed, scales, n, G, p.kb >> 1, cur);
                 const int g_last = (p.ke - 1) >> 1;
                 uint32_t cw[8];
-                __half2 s2 = __float2half2_rn(0.f);
+                uint32_t tneg = 0u, tpos = 0u;  // the group's value table {-s, 0, +s}
                 for (int ks = p.kb; ks < p.ke; ks++, it++) {
                     const int g = ks >> 1, hf = ks & 1;  // a 128-weight group fills two 64-wide stages
                     if (ks == p.kb || hf == 0) {
                         if (valid && g < g_last) load_group<kFmt>(packed, scales, n, G, g + 1, nxt);  // in flight
                         if (valid) {
                             group_codes<kFmt>(cur, lut, cw);
-                            const __half sh = __ushort_as_half(cur.scale);
-                            s2 = __halves2half2(sh, sh);
+                            tneg = (uint32_t)cur.scale ^ 0x8000u;
+                            tpos = (uint32_t)cur.scale;
                         } else {
 #pragma unroll
                             for (int i = 0; i < 8; i++) cw[i] = 0x55555555u;  // all trits zero
@@ -451,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
 #pragma unroll
                     for (int i = 0; i < 4; i++) {
                         uint32_t out[8];
-                        expand_word(hf ? cw[4 + i] : cw[i], s2, out);  // weights 64hf + 16i .. +15
+                        expand_word(hf ? cw[4 + i] : cw[i], tneg, tpos, out);  // weights 64hf + 16i .. +15
                         st_chunk(stage, r, 2 * i, out);
                         st_chunk(stage, r, 2 * i + 1, out + 4);
                     }
@@ -645,7 +639,7 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
     if (ws.data_bytes < gemm_workspace_bytes(M, N, K, fmt, dev) || plan.ctas > kMaxTiles) return cudaErrorInvalidValue;
     uint16_t *xr = reinterpret_cast<uint16_t *>(ws.data);
     float *partials = reinterpret_cast<float *>(ws.data + x_rot_bytes(M, K));
-    cudaError_t err = launch_hadamard_f16(x, xr, M, K, s, dev);
+    cudaError_t err = launch_hadamard_f16_perm8(x, xr, M, K, s, dev);  // in the expansion's K order
     if (err != cudaSuccess) return err;
 
     EncodeTiledFn encode = encode_fn();

@@ -15,7 +15,11 @@
 namespace bonsai {
 namespace {
 
-template <bool kOutF32>
+// kPerm8 (FP16 output only): each 8 consecutive outputs are stored in the order
+// [0, 4, 1, 5, 2, 6, 3, 7].  The prefill GEMM expands its weights in the same order
+// within each 8 (a contraction does not depend on the order of its terms), which lets it
+// build two FP16 weights with one byte permute.
+template <bool kOutF32, bool kPerm8>
 __global__ void __launch_bounds__(256) hadamard128_kernel(const uint16_t *x, void *out,
                                                           int64_t nblocks) {
     const int lane = threadIdx.x & 31;
@@ -29,12 +33,27 @@ __global__ void __launch_bounds__(256) hadamard128_kernel(const uint16_t *x, voi
             float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + blk * kGroup) + lane;
             *o = make_float4(v[0], v[1], v[2], v[3]);
         } else {
-            store_half4(static_cast<uint16_t *>(out) + blk * kGroup + 4 * lane, v);
+            if (kPerm8) {
+                // lanes 2b, 2b + 1 hold outputs 8b .. 8b + 7; the even lane stores
+                // (0, 4, 1, 5), the odd one (2, 6, 3, 7)
+                const bool odd = lane & 1;
+                const float r0 = __shfl_xor_sync(0xffffffffu, odd ? v[0] : v[2], 1);
+                const float r1 = __shfl_xor_sync(0xffffffffu, odd ? v[1] : v[3], 1);
+                float o[4];
+                if (odd) {
+                    o[0] = r0, o[1] = v[2], o[2] = r1, o[3] = v[3];
+                } else {
+                    o[0] = v[0], o[1] = r0, o[2] = v[1], o[3] = r1;
+                }
+                store_half4(static_cast<uint16_t *>(out) + blk * kGroup + 4 * lane, o);
+            } else {
+                store_half4(static_cast<uint16_t *>(out) + blk * kGroup + 4 * lane, v);
+            }
         }
     }
 }
 
-template <bool kOutF32>
+template <bool kOutF32, bool kPerm8 = false>
 cudaError_t launch(const uint16_t *x, void *out, int64_t M, int64_t K, cudaStream_t s,
                    const DeviceInfo &dev) {
     const int64_t nblocks = M * (K / kGroup);
@@ -42,7 +61,7 @@ cudaError_t launch(const uint16_t *x, void *out, int64_t M, int64_t K, cudaStrea
     const int64_t want = (nblocks + 7) / 8;  // 8 warps per CTA
     const int64_t cap = (int64_t)dev.sm_count * 8;
     const int grid = (int)(want < cap ? want : cap);
-    hadamard128_kernel<kOutF32><<<grid, 256, 0, s>>>(x, out, nblocks);
+    hadamard128_kernel<kOutF32, kPerm8><<<grid, 256, 0, s>>>(x, out, nblocks);
     return cudaGetLastError();
 }
 
@@ -51,6 +70,11 @@ cudaError_t launch(const uint16_t *x, void *out, int64_t M, int64_t K, cudaStrea
 cudaError_t launch_hadamard_f16(const uint16_t *x, uint16_t *out, int64_t M, int64_t K,
                                 cudaStream_t s, const DeviceInfo &dev) {
     return launch<false>(x, out, M, K, s, dev);
+}
+
+cudaError_t launch_hadamard_f16_perm8(const uint16_t *x, uint16_t *out, int64_t M, int64_t K,
+                                      cudaStream_t s, const DeviceInfo &dev) {
+    return launch<false, true>(x, out, M, K, s, dev);
 }
 
 cudaError_t launch_hadamard_f32(const uint16_t *x, float *out, int64_t M, int64_t K,

@@ -44,6 +44,10 @@ cudaError_t launch_hadamard_f16(const uint16_t *x, uint16_t *out, int64_t M, int
                                 cudaStream_t s, const DeviceInfo &dev);
 cudaError_t launch_hadamard_f32(const uint16_t *x, float *out, int64_t M, int64_t K,
                                 cudaStream_t s, const DeviceInfo &dev);
+// As launch_hadamard_f16, each 8 outputs stored in the order [0, 4, 1, 5, 2, 6, 3, 7]
+// (the K order of the prefill GEMM's expanded weight tiles).
+cudaError_t launch_hadamard_f16_perm8(const uint16_t *x, uint16_t *out, int64_t M, int64_t K,
+                                      cudaStream_t s, const DeviceInfo &dev);
 
 // ---- linear_simple.cu: x' (FP32, M x K) in the workspace, then one warp per row
 size_t simple_workspace_bytes(int64_t M, int64_t N, int64_t K);
