@@ -41,6 +41,7 @@ constexpr int BM = 128, BN = 256, BK = 64;  // BM: rows of one MMA / one TMEM ac
 constexpr int kExpandWarps = 8;
 constexpr int kThreads = (2 + kExpandWarps) * 32;  // 320
 constexpr int B_STAGE_BYTES = BN * BK * 2;         // 32 KB
+constexpr int CODE_STAGE_BYTES = BN * BK / 4;      // PQ2_0 codes of a B stage: 256 rows x 16 bytes
 
 // Tile configuration: kAcc accumulators of 128 rows each share every B stage (the
 // expanded weights), so the CTA covers 128 * kAcc rows of y.
@@ -50,10 +51,12 @@ struct Cfg {
     static constexpr int kTileM = BM * kAcc;
     static constexpr int kAStage = kTileM * BK * 2;  // 16 or 32 KB
     static constexpr int kTmemCols = 256 * kAcc;
-    // shared memory: [A stages][B stages][barriers][tmem slot][abort flag][PTQ1_0 LUT]
+    // shared memory: [A stages][B stages][PQ2_0 code stages][barriers][tmem slot][abort
+    // flag][PTQ1_0 LUT]
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kStages * kAStage;
-    static constexpr int kOffBar = kOffB + kStages * B_STAGE_BYTES;
+    static constexpr int kOffCodes = kOffB + kStages * B_STAGE_BYTES;
+    static constexpr int kOffBar = kOffCodes + kStages * CODE_STAGE_BYTES;
     static constexpr int kNumBars = 3 * kStages + 3;  // full_a, full_b, empty, done, tmem_free, fin
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 8;
@@ -246,7 +249,8 @@ __device__ __forceinline__ void expand_warps_sync() { asm volatile("bar.sync 1, 
 // wait before they have stored (all CTAs of the grid are resident at once, one per SM).
 template <int kFmt, int kAcc>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
-    const __grid_constant__ CUtensorMap a_map, const uint8_t *__restrict__ packed,
+    const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap w_map,
+    const uint8_t *__restrict__ packed,
     const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
     unsigned int *__restrict__ flags, int M, int N, int K, int mt) {
     using C = Cfg<kAcc>;
@@ -257,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem + C::kOffA;
     uint8_t *sB = smem + C::kOffB;
+    const uint8_t *sCodes = smem + C::kOffCodes;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint64_t *full_a = bars, *full_b = bars + STAGES, *empty = bars + 2 * STAGES;
     uint64_t *done = bars + 3 * STAGES, *tmem_free = done + 1, *fin = done + 2;
@@ -339,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
             int it = 0;  // units issued: ring position
             for (int v = 0; v < n_mine && !*abort_flag;) {
                 const Piece p = piece_at(v);
-                const int tm = p.s % mt;
+                const int tm = p.s % mt, tn = p.s / mt;
                 for (int ks = p.kb; ks < p.ke; ks++, it++) {
                     const int st = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -347,11 +352,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                         *abort_flag = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(full_a + st, C::kAStage);
+                    mbar_arrive_expect_tx(full_a + st, C::kAStage + (kFmt == 2 ? CODE_STAGE_BYTES : 0));
 #pragma unroll
                     for (int a = 0; a < kAcc; a++)
                         tma_load_2d(sA + st * C::kAStage + a * (BM * BK * 2), &a_map, full_a + st, ks * BK,
                                     tm * C::kTileM + a * BM);
+                    // PQ2_0: the stage's codes, 16 bytes of each of the tile's 256 weight rows
+                    if (kFmt == 2)
+                        tma_load_2d(const_cast<uint8_t *>(sCodes) + st * CODE_STAGE_BYTES, &w_map, full_a + st,
+                                    ks * (BK / 4), tn * BN);
                 }
                 v += p.ke - p.kb;
             }
@@ -414,46 +423,68 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
             const int64_t n = (int64_t)tn * BN + r;  // weight row
             const bool valid = n < N;
             if (live) {
+                // PTQ1_0: the packed bytes of the group being expanded and of the next one (in
+                // flight) come by plain loads; PQ2_0: the codes come with the stage's x' tiles
+                // (TMA), only the scale by a plain load, one group ahead
                 GroupRaw cur, nxt;
-                if (valid) load_group<kFmt>(packed, scales, n, G, p.kb >> 1, cur);
                 const int g_last = (p.ke - 1) >> 1;
+                uint32_t sc = 0u;
+                if (kFmt == 1 && valid) load_group<kFmt>(packed, scales, n, G, p.kb >> 1, cur);
+                if (kFmt == 2 && valid) sc = __ldg(scales + n * G + (p.kb >> 1));
                 uint32_t cw[8];
                 uint32_t tneg = 0u, tpos = 0u;  // the group's value table {-s, 0, +s}
                 for (int ks = p.kb; ks < p.ke; ks++, it++) {
                     const int g = ks >> 1, hf = ks & 1;  // a 128-weight group fills two 64-wide stages
                     if (ks == p.kb || hf == 0) {
-                        if (valid && g < g_last) load_group<kFmt>(packed, scales, n, G, g + 1, nxt);  // in flight
-                        if (valid) {
-                            group_codes<kFmt>(cur, lut, cw);
-                            tneg = (uint32_t)cur.scale ^ 0x8000u;
-                            tpos = (uint32_t)cur.scale;
+                        if (kFmt == 2) {
+                            tneg = valid ? sc ^ 0x8000u : 0u;
+                            tpos = valid ? sc : 0u;
+                            if (valid && g < g_last) sc = __ldg(scales + n * G + g + 1);
                         } else {
+                            if (valid && g < g_last) load_group<kFmt>(packed, scales, n, G, g + 1, nxt);
+                            if (valid) {
+                                group_codes<kFmt>(cur, lut, cw);
+                                tneg = (uint32_t)cur.scale ^ 0x8000u;
+                                tpos = (uint32_t)cur.scale;
+                            } else {
 #pragma unroll
-                            for (int i = 0; i < 8; i++) cw[i] = 0x55555555u;  // all trits zero
+                                for (int i = 0; i < 8; i++) cw[i] = 0x55555555u;  // all trits zero
+                            }
                         }
                     }
                     const int st = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    // every lane acquires the stage itself; the verdict is made warp-uniform
-                    const bool free_ok = !*abort_flag && mbar_wait(empty + st, ph ^ 1u);
+                    // every lane acquires the stage itself (and, PQ2_0, its codes); the verdict
+                    // is made warp-uniform
+                    const bool free_ok = !*abort_flag && mbar_wait(empty + st, ph ^ 1u) &&
+                                         (kFmt != 2 || mbar_wait(full_a + st, ph));
                     if (!__all_sync(0xffffffffu, free_ok)) {
                         *abort_flag = 1;
                         live = false;
                         break;
                     }
+                    uint32_t w4[4];
+                    if (kFmt == 2) {
+                        const uint4 c4 = *reinterpret_cast<const uint4 *>(sCodes + st * CODE_STAGE_BYTES + r * 16);
+                        w4[0] = c4.x, w4[1] = c4.y, w4[2] = c4.z, w4[3] = c4.w;
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; i++) w4[i] = hf ? cw[4 + i] : cw[i];
+                    }
                     uint8_t *stage = sB + st * B_STAGE_BYTES;
 #pragma unroll
                     for (int i = 0; i < 4; i++) {
                         uint32_t out[8];
-                        expand_word(hf ? cw[4 + i] : cw[i], tneg, tpos, out);  // weights 64hf + 16i .. +15
+                        expand_word(w4[i], tneg, tpos, out);  // weights 64ks + 16i .. +15
                         st_chunk(stage, r, 2 * i, out);
                         st_chunk(stage, r, 2 * i + 1, out + 4);
                     }
-                    // make the generic-proxy stores visible to the tensor core, then signal
+                    // make the generic-proxy accesses (these stores, the code loads) ordered
+                    // before later async-proxy ones, then signal
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                     if (lane == 0) mbar_arrive(full_b + st);
-                    if (hf == 1) cur = nxt;
+                    if (kFmt == 1 && hf == 1) cur = nxt;
                 }
             }
 
@@ -654,10 +685,21 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
 
+    // PQ2_0 codes: rows of K/4 bytes, a box of 16 bytes x 256 rows per 64-wide stage
+    CUtensorMap wmap = map;  // (unused by PTQ1_0)
+    if (fmt == 2) {
+        const cuuint64_t wdims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
+        const cuuint64_t wstrides[1] = {(cuuint64_t)(K / 4)};
+        const cuuint32_t wbox[2] = {BK / 4, BN};
+        if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), wdims, wstrides, wbox,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
     auto go = [&](auto kern, int smem) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        kern<<<plan.ctas, kThreads, smem, s>>>(map, packed, scales, y, partials, ws.counters, (int)M, (int)N,
+        kern<<<plan.ctas, kThreads, smem, s>>>(map, wmap, packed, scales, y, partials, ws.counters, (int)M, (int)N,
                                                (int)K, plan.mt);
         return cudaGetLastError();
     };
