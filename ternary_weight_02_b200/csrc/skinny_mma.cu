@@ -15,12 +15,15 @@
 //   where an FP16 bit pattern with a zero exponent reads as c * 4^j * 2^-24.  The
 //   matching activations are stored pre-scaled by 4^-j (exact), so each MMA adds
 //   2^-24 * sum c * x' in FP32.  The lane's k slots are permuted (the same
-//   permutation on both operands) so that its four slots are one byte of the word.
+//   permutation on both operands) so that its four slots are one byte of a word.
 // * Per 128-weight group the MMA starts from zero; the epilogue adds
 //   s[n][g] * (2^24 * D - sum_j x'[m][j]) (the second term turns codes into trits).
+// * Each lane loads only the 8 bytes of a row's group that its MMA slots use (words 2tq,
+//   2tq + 1), and keeps kRing groups in flight in a ring of registers whose slots are
+//   addressed by constants (no register copies that would wait for a load).
 // * x' (FWHT prepass, FP16) of the CTA's K chunk sits in shared memory as
-//   [k-step][token][16 halves], 4^-(k mod 4)-scaled, so a lane's B fragment is one
-//   8-byte load from a contiguous 256-byte row.
+//   [k-step][token][16 halves], 4^-(k mod 4)-scaled and in the MMAs' K order, so a
+//   lane's B fragment is one 8-byte load from a contiguous 256-byte row.
 // * A warp owns 16 weight rows; a CTA 128 rows and one K chunk.  Split-K: chunks
 //   write FP32 partials; the warp that brings a row block's last chunk sums them in
 //   chunk order (deterministic) and writes y.
@@ -33,10 +36,17 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kRowsPerCta = kWarps * 16;
-constexpr int kSubGroups = 16;  // groups of x' staged in shared memory at a time
+constexpr int kRing = 8;  // groups of weights in flight per warp
 
-struct Raw {
-    uint4 a, b;  // 32 bytes: one 128-weight group of one row
+// groups of x' staged in shared memory at a time: 96 KB for either token tile count
+template <int NT>
+constexpr int sub_groups() { return NT == 1 ? 48 : 24; }
+
+// One 128-weight group of the warp's rows r0 = gid and r1 = gid + 8, as lane (gid, tq)
+// holds it: words 2tq and 2tq + 1 (8 bytes) of each row, and the two FP16 scales.
+struct Grp {
+    uint2 a, b;
+    uint32_t s0, s1;
 };
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -48,21 +58,64 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(d[0]), "f"(d[1]), "f"(d[2]), "f"(d[3]));
 }
 
-__device__ __forceinline__ uint32_t word_of(const Raw &r, int i) {
-    const uint4 &v = i < 4 ? r.a : r.b;
-    const int j = i & 3;
-    return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
+// K order of the MMAs: MMA i of a group takes, from lane quad member tq, byte (i & 3) of
+// group word 2tq + (i >> 2), i.e. the four weights 32tq + 16(i >> 2) + 4(i & 3) + c,
+// c = 0..3, which sit at B slots 4tq + c of the MMA's 16-half row of x'.
+__device__ __forceinline__ int64_t skinny_k(int64_t group, int step, int tq) {
+    return group * kGroup + 32 * tq + 16 * (step >> 2) + 4 * (step & 3);
+}
+
+// The rotation pass of this kernel: one warp per (group g, token m < MT).  It writes x'
+// (FP16, nearest) of the block in the layout the MMAs read, [g][step][token][16] with
+// slot 4tq + c = element skinny_k(g, step, tq) + c scaled by 4^-c, zeros for the padding
+// tokens m >= M, and the FP32 sum of the block's FP16 x' values to gsum[g][m].
+template <int MT>
+__global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ xs,
+                                                          float *__restrict__ gsum, int M, int64_t K) {
+    const int lane = threadIdx.x & 31;
+    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // (g, m) = (w / MT, w % MT)
+    const int64_t G = K / kGroup;
+    if (w >= G * MT) return;
+    const int64_t g = w / MT;
+    const int m = (int)(w % MT);
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (m < M) {
+        load_half4(x + (int64_t)m * K + g * kGroup + 4 * lane, v);
+        fwht128_warp(v, lane);
+    }
+    const __half2 h01 = __floats2half2_rn(v[0], v[1]), h23 = __floats2half2_rn(v[2], v[3]);
+    const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+    const float sum = warp_sum((f01.x + f01.y) + (f23.x + f23.y));
+    // lane l holds elements 4l .. 4l+3 = skinny_k(g, i, tq) + c with tq = l >> 3 and
+    // i = 4 ((l >> 2) & 1) + (l & 3)
+    const int tq = lane >> 3, i = 4 * ((lane >> 2) & 1) + (lane & 3);
+    const __half2 s01 = __hmul2(h01, __floats2half2_rn(1.f, 0.25f));
+    const __half2 s23 = __hmul2(h23, __floats2half2_rn(0.0625f, 0.015625f));
+    uint2 out;
+    out.x = *reinterpret_cast<const uint32_t *>(&s01);
+    out.y = *reinterpret_cast<const uint32_t *>(&s23);
+    *reinterpret_cast<uint2 *>(xs + ((g * 8 + i) * MT + m) * 16 + 4 * tq) = out;
+    if (lane == 0) gsum[g * MT + m] = sum;
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
 }
 
 template <int NT>  // n8 token tiles: 1 (M <= 8) or 2 (M <= 16)
 __global__ void __launch_bounds__(kThreads) skinny_kernel(
-    const uint16_t *__restrict__ xr, const uint8_t *__restrict__ packed, const uint16_t *__restrict__ scales,
-    uint16_t *__restrict__ y, float *__restrict__ partials, unsigned int *__restrict__ counters, int M, int64_t N,
-    int64_t K, int S, int gpc) {
+    const uint16_t *__restrict__ xsg, const float *__restrict__ gsg, const uint8_t *__restrict__ packed,
+    const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
+    unsigned int *__restrict__ counters, int M, int64_t N, int64_t K, int S, int gpc) {
     constexpr int MT = NT * 8;  // tokens padded
+    static_assert(sub_groups<NT>() % kRing == 0, "ring slots follow the group index");
+    // groups staged at a time: the whole chunk when it fits (shared memory is sized so)
+    const int kSub = gpc < sub_groups<NT>() ? gpc : sub_groups<NT>();
     extern __shared__ __align__(16) uint8_t smem[];
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [kSubGroups * 8 k-steps][MT][16]
-    float *gsum = reinterpret_cast<float *>(smem + kSubGroups * 8 * MT * 32);  // [MT][kSubGroups]
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [kSub * 8 steps][MT][16]
+    float *gsum = reinterpret_cast<float *>(smem + kSub * 8 * MT * 32);  // [MT][kSub]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tq = lane & 3;
@@ -73,7 +126,6 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
     const int64_t n0 = (int64_t)blockIdx.x * kRowsPerCta + warp * 16;
     const int64_t r0 = n0 + gid, r1 = n0 + gid + 8;
     const bool v0 = r0 < N, v1 = r1 < N;
-    const uint32_t sel = 0x4040u | (uint32_t)tq | ((uint32_t)tq << 8);  // [byte tq, 0, byte tq, 0]
 
     float acc[NT][4];
 #pragma unroll
@@ -81,97 +133,87 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
 #pragma unroll
         for (int e = 0; e < 4; e++) acc[nt][e] = 0.f;
 
-    auto load_raw = [&](int g, Raw &ra, Raw &rb, float &s0, float &s1) {
-        const uint4 z = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);  // trits 0
+    auto load = [&](int g, Grp &q) {
         if (v0) {
-            const uint4 *p = reinterpret_cast<const uint4 *>(packed + (r0 * G + g) * kPq2GroupBytes);
-            ra.a = __ldcs(p);
-            ra.b = __ldcs(p + 1);
-            s0 = half_bits_to_float(__ldg(scales + r0 * G + g));
+            q.a = __ldcs(reinterpret_cast<const uint2 *>(packed + (r0 * G + g) * kPq2GroupBytes) + tq);
+            q.s0 = __ldg(scales + r0 * G + g);
         } else {
-            ra.a = z, ra.b = z, s0 = 0.f;
+            q.a = make_uint2(0x55555555u, 0x55555555u), q.s0 = 0u;  // trits 0
         }
         if (v1) {
-            const uint4 *p = reinterpret_cast<const uint4 *>(packed + (r1 * G + g) * kPq2GroupBytes);
-            rb.a = __ldcs(p);
-            rb.b = __ldcs(p + 1);
-            s1 = half_bits_to_float(__ldg(scales + r1 * G + g));
+            q.b = __ldcs(reinterpret_cast<const uint2 *>(packed + (r1 * G + g) * kPq2GroupBytes) + tq);
+            q.s1 = __ldg(scales + r1 * G + g);
         } else {
-            rb.a = z, rb.b = z, s1 = 0.f;
+            q.b = make_uint2(0x55555555u, 0x55555555u), q.s1 = 0u;
         }
     };
 
-    Raw ca, cb, na, nb;
-    float cs0 = 0.f, cs1 = 0.f, ns0 = 0.f, ns1 = 0.f;
-    if (g_begin < g_end) load_raw(g_begin, ca, cb, cs0, cs1);
+    // group g of the chunk lives in ring slot (g - g_begin) % kRing; the first kRing are
+    // requested before x' is staged
+    Grp ring[kRing];
+#pragma unroll
+    for (int u = 0; u < kRing; u++)
+        if (g_begin + u < g_end) load(g_begin + u, ring[u]);
 
-    for (int sub = g_begin; sub < g_end; sub += kSubGroups) {
-        const int nsub = g_end - sub < kSubGroups ? g_end - sub : kSubGroups;
+    for (int sub = g_begin; sub < g_end; sub += kSub) {
+        const int nsub = g_end - sub < kSub ? g_end - sub : kSub;
         __syncthreads();  // the previous sub-chunk's x' is no longer read
-        // stage x'[m][128*sub .. 128*(sub+nsub)) as [k-step][token][16], element k scaled 4^-(k mod 4)
-        for (int idx = tid; idx < nsub * 8 * MT * 4; idx += kThreads) {
-            const int q4 = idx & 3;            // which 4 halves of the 16
-            const int m = (idx >> 2) % MT;
-            const int ks = (idx >> 2) / MT;    // k-step within the sub-chunk
-            const int64_t k = (int64_t)sub * kGroup + ks * 16 + q4 * 4;
-            uint2 out = make_uint2(0u, 0u);
-            if (m < M) {
-                const uint2 raw = *reinterpret_cast<const uint2 *>(xr + (int64_t)m * K + k);
-                const __half2 lo = *reinterpret_cast<const __half2 *>(&raw.x);
-                const __half2 hi = *reinterpret_cast<const __half2 *>(&raw.y);
-                const __half2 f01 = __hmul2(lo, __floats2half2_rn(1.f, 0.25f));
-                const __half2 f23 = __hmul2(hi, __floats2half2_rn(0.0625f, 0.015625f));
-                out.x = *reinterpret_cast<const uint32_t *>(&f01);
-                out.y = *reinterpret_cast<const uint32_t *>(&f23);
+        // the sub-chunk's x' (laid out by the rotation pass as read here) and group sums
+        {
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(xsg + (int64_t)sub * 8 * MT * 16);
+            const int bytes = nsub * 8 * MT * 32;
+            for (int off = tid * 16; off < bytes; off += kThreads * 16)
+                cp_async16(reinterpret_cast<uint8_t *>(xs) + off, src + off);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            for (int idx = tid; idx < nsub * MT; idx += kThreads) {
+                const int gl = idx / MT, m = idx % MT;
+                gsum[m * kSub + gl] = gsg[(int64_t)(sub + gl) * MT + m];
             }
-            *reinterpret_cast<uint2 *>(xs + ((ks * MT + m) * 16 + q4 * 4)) = out;
-        }
-        // group sums of x' per token (FP32 sum of the FP16 values)
-        for (int pair = warp; pair < MT * nsub; pair += kWarps) {
-            const int m = pair % MT, gl = pair / MT;
-            float v = 0.f;
-            if (m < M) {
-                float f[4];
-                load_half4(xr + (int64_t)m * K + (int64_t)(sub + gl) * kGroup + 4 * lane, f);
-                v = (f[0] + f[1]) + (f[2] + f[3]);
-            }
-            v = warp_sum(v);
-            if (lane == 0) gsum[m * kSubGroups + gl] = v;
+            asm volatile("cp.async.wait_all;" ::: "memory");
         }
         __syncthreads();
 
-        for (int gl = 0; gl < nsub; gl++) {
-            const int g = sub + gl;
-            if (g + 1 < g_end) load_raw(g + 1, na, nb, ns0, ns1);  // next group in flight
-            float d[NT][4];
+        for (int gl0 = 0; gl0 < nsub; gl0 += kRing) {
 #pragma unroll
-            for (int nt = 0; nt < NT; nt++)
+            for (int u = 0; u < kRing; u++) {
+                const int gl = gl0 + u;
+                if (gl >= nsub) break;
+                Grp &cur = ring[u];
+                float d[NT][4];
 #pragma unroll
-                for (int e = 0; e < 4; e++) d[nt][e] = 0.f;
+                for (int nt = 0; nt < NT; nt++)
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const uint32_t p0 = __byte_perm(word_of(ca, i), 0u, sel);
-                const uint32_t p1 = __byte_perm(word_of(cb, i), 0u, sel);
-                const uint32_t a0 = p0 & 0x000C0003u, a1 = p1 & 0x000C0003u;
-                const uint32_t a2 = p0 & 0x00C00030u, a3 = p1 & 0x00C00030u;
-                const int ks = gl * 8 + i;
+                    for (int e = 0; e < 4; e++) d[nt][e] = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    // byte (i & 3) of the lane's word i >> 2, in both halves: (c0, c1) and
+                    // (c2, c3) left in place as FP16 subnormals c * 4^j * 2^-24
+                    const uint32_t sel = 0x4040u | (uint32_t)(i & 3) | ((uint32_t)(i & 3) << 8);
+                    const uint32_t p0 = __byte_perm((i >> 2) ? cur.a.y : cur.a.x, 0u, sel);
+                    const uint32_t p1 = __byte_perm((i >> 2) ? cur.b.y : cur.b.x, 0u, sel);
+                    const uint32_t a0 = p0 & 0x000C0003u, a1 = p1 & 0x000C0003u;
+                    const uint32_t a2 = p0 & 0x00C00030u, a3 = p1 & 0x00C00030u;
+                    const int ks = gl * 8 + i;
+#pragma unroll
+                    for (int nt = 0; nt < NT; nt++) {
+                        const uint2 b = *reinterpret_cast<const uint2 *>(xs + ((ks * MT + nt * 8 + gid) * 16 + tq * 4));
+                        mma16816(d[nt], a0, a1, a2, a3, b.x, b.y);
+                    }
+                }
+                const float cs0 = half_bits_to_float((uint16_t)cur.s0), cs1 = half_bits_to_float((uint16_t)cur.s1);
 #pragma unroll
                 for (int nt = 0; nt < NT; nt++) {
-                    const uint2 b = *reinterpret_cast<const uint2 *>(xs + ((ks * MT + nt * 8 + gid) * 16 + tq * 4));
-                    mma16816(d[nt], a0, a1, a2, a3, b.x, b.y);
+                    const int m0 = nt * 8 + 2 * tq;
+                    const float gs0 = gsum[m0 * kSub + gl], gs1 = gsum[(m0 + 1) * kSub + gl];
+                    // d[0], d[1]: row r0, tokens m0, m0+1; d[2], d[3]: row r1
+                    acc[nt][0] = fmaf(cs0, fmaf(d[nt][0], 16777216.f, -gs0), acc[nt][0]);
+                    acc[nt][1] = fmaf(cs0, fmaf(d[nt][1], 16777216.f, -gs1), acc[nt][1]);
+                    acc[nt][2] = fmaf(cs1, fmaf(d[nt][2], 16777216.f, -gs0), acc[nt][2]);
+                    acc[nt][3] = fmaf(cs1, fmaf(d[nt][3], 16777216.f, -gs1), acc[nt][3]);
                 }
+                const int g = sub + gl;
+                if (g + kRing < g_end) load(g + kRing, cur);  // refill the slot
             }
-#pragma unroll
-            for (int nt = 0; nt < NT; nt++) {
-                const int m0 = nt * 8 + 2 * tq;
-                const float gs0 = gsum[m0 * kSubGroups + gl], gs1 = gsum[(m0 + 1) * kSubGroups + gl];
-                // d[0], d[1]: row r0, tokens m0, m0+1; d[2], d[3]: row r1
-                acc[nt][0] = fmaf(cs0, fmaf(d[nt][0], 16777216.f, -gs0), acc[nt][0]);
-                acc[nt][1] = fmaf(cs0, fmaf(d[nt][1], 16777216.f, -gs1), acc[nt][1]);
-                acc[nt][2] = fmaf(cs1, fmaf(d[nt][2], 16777216.f, -gs0), acc[nt][2]);
-                acc[nt][3] = fmaf(cs1, fmaf(d[nt][3], 16777216.f, -gs1), acc[nt][3]);
-            }
-            ca = na, cb = nb, cs0 = ns0, cs1 = ns1;
         }
     }
 
@@ -216,18 +258,34 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
     if (lane == 0) counters[rb] = 0u;
 }
 
-int smem_bytes(int NT) { return kSubGroups * 8 * NT * 8 * 32 + NT * 8 * kSubGroups * 4; }
+int smem_bytes(int NT, int gpc) {
+    int sub = NT == 1 ? sub_groups<1>() : sub_groups<2>();
+    sub = gpc < sub ? gpc : sub;
+    return sub * 8 * NT * 8 * 32 + NT * 8 * sub * 4;
+}
 
-// K chunks: enough CTAs for about two waves, unless split_k (> 0) says otherwise.
+// K chunks: about as many CTAs as fit on the GPU at once (one wave; a CTA's registers
+// allow two per SM), unless split_k (> 0) says otherwise.
 void choose_split(int64_t N, int64_t K, int split_k, const DeviceInfo &dev, int *S, int *gpc) {
     const int64_t G = K / kGroup;
     const int64_t rb = (N + kRowsPerCta - 1) / kRowsPerCta;
-    int64_t s = split_k > 0 ? split_k : (2 * (int64_t)dev.sm_count + rb - 1) / rb;
+    int64_t s = split_k > 0 ? split_k : (2 * (int64_t)dev.sm_count) / rb;
     if (s < 1) s = 1;
     if (s > G) s = G;
     const int64_t per = (G + s - 1) / s;
     *gpc = (int)per;
     *S = (int)((G + per - 1) / per);
+}
+
+// Workspace: the staged x' ([G][8][MT][16] FP16), the group sums ([G][MT] FP32), then the
+// split-K partials.
+size_t staged_bytes(int64_t M, int64_t K) {
+    const int64_t MT = M <= 8 ? 8 : 16;
+    return ((size_t)(K / kGroup) * 8 * MT * 32 + 255) / 256 * 256;
+}
+size_t gsum_bytes(int64_t M, int64_t K) {
+    const int64_t MT = M <= 8 ? 8 : 16;
+    return ((size_t)(K / kGroup) * MT * 4 + 255) / 256 * 256;
 }
 
 }  // namespace
@@ -241,30 +299,32 @@ size_t skinny_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int spli
     (void)fmt;
     int S, gpc;
     choose_split(N, K, split_k, dev, &S, &gpc);
-    const size_t xbytes = ((size_t)M * (size_t)K * 2 + 255) / 256 * 256;
-    return xbytes + (S > 1 ? (size_t)S * (size_t)M * (size_t)N * sizeof(float) : 0);
+    return staged_bytes(M, K) + gsum_bytes(M, K) + (S > 1 ? (size_t)S * (size_t)M * (size_t)N * sizeof(float) : 0);
 }
 
 cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                           uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int split_k,
                           const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
     (void)fmt;
-    uint16_t *xr = reinterpret_cast<uint16_t *>(ws.data);
-    cudaError_t err = launch_hadamard_f16(x, xr, M, K, s, dev);
-    if (err != cudaSuccess) return err;
+    uint16_t *xsg = reinterpret_cast<uint16_t *>(ws.data);
+    float *gsg = reinterpret_cast<float *>(ws.data + staged_bytes(M, K));
+    float *partials = reinterpret_cast<float *>(ws.data + staged_bytes(M, K) + gsum_bytes(M, K));
     int S, gpc;
     choose_split(N, K, split_k, dev, &S, &gpc);
-    float *partials = reinterpret_cast<float *>(ws.data + ((size_t)M * (size_t)K * 2 + 255) / 256 * 256);
     const dim3 grid((unsigned)((N + kRowsPerCta - 1) / kRowsPerCta), (unsigned)S);
+    const int64_t G = K / kGroup;
+    cudaError_t err;
     if (M <= 8) {
-        err = cudaFuncSetAttribute(skinny_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(1));
+        skinny_prep_kernel<8><<<(unsigned)((G * 8 + 7) / 8), 256, 0, s>>>(x, xsg, gsg, (int)M, K);
+        err = cudaFuncSetAttribute(skinny_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(1, gpc));
         if (err != cudaSuccess) return err;
-        skinny_kernel<1><<<grid, kThreads, smem_bytes(1), s>>>(xr, packed, scales, y, partials, ws.counters,
+        skinny_kernel<1><<<grid, kThreads, smem_bytes(1, gpc), s>>>(xsg, gsg, packed, scales, y, partials, ws.counters,
                                                                (int)M, N, K, S, gpc);
     } else {
-        err = cudaFuncSetAttribute(skinny_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(2));
+        skinny_prep_kernel<16><<<(unsigned)((G * 16 + 7) / 8), 256, 0, s>>>(x, xsg, gsg, (int)M, K);
+        err = cudaFuncSetAttribute(skinny_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(2, gpc));
         if (err != cudaSuccess) return err;
-        skinny_kernel<2><<<grid, kThreads, smem_bytes(2), s>>>(xr, packed, scales, y, partials, ws.counters,
+        skinny_kernel<2><<<grid, kThreads, smem_bytes(2, gpc), s>>>(xsg, gsg, packed, scales, y, partials, ws.counters,
                                                                (int)M, N, K, S, gpc);
     }
     return cudaGetLastError();
