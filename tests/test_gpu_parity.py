@@ -254,12 +254,14 @@ def test_imma_decode_shapes_full(bz, K, N):
 
 
 def test_imma_repeatable_and_counters_reset(bz):
-    """Row tiles split between warps are summed through partials and arrival counters;
-    the counters return to zero, so back-to-back calls on shapes with different splits
-    give bit-identical results."""
+    """Row tiles split between CTAs are summed through (value, epoch) pairs that their
+    reader clears, so back-to-back calls on shapes with different splits (among them the
+    34816 x 5120 and 20000 x 8192 ones, many row tiles per CTA) give bit-identical
+    results."""
     import torch
     probs = [Problem(1, 3000, 5120, PQ2, seed=1), Problem(1, 77, 17408, PQ2, seed=2),
-             Problem(1, 5120, 17408, PQ2, seed=3)]
+             Problem(1, 34816, 5120, PQ2, seed=4), Problem(1, 5120, 17408, PQ2, seed=3),
+             Problem(1, 20000, 8192, PQ2, seed=5)]
     devs = [p.device() for p in probs]
     outs = []
     for _ in range(3):
@@ -268,8 +270,9 @@ def test_imma_repeatable_and_counters_reset(bz):
             bz.bonsai_ternary_linear_algo(x, packed, scales, y, 1, p.N, p.K, PQ2, bz.BONSAI_ALGO_IMMA, 0)
             outs.append(y)
     torch.cuda.synchronize()
-    for i in range(3, 9):
-        assert torch.equal(outs[i], outs[i % 3])
+    n = len(probs)
+    for i in range(n, 3 * n):
+        assert torch.equal(outs[i], outs[i % n])
     for i, p in enumerate(probs):
         assert oracle.compare(to_numpy_f16(outs[i]), p.oracle_y())[0]
 
