@@ -22,6 +22,7 @@ LIB = os.path.join(HERE, "liboracle.so")
 
 FMT_PTQ1_0 = 1
 FMT_PQ2_0 = 2
+FMT_Q1_0 = 3
 GROUP = 128
 INVALID_TRIT = -128
 
@@ -48,11 +49,11 @@ def lib():
         ll, p, i = ctypes.c_longlong, ctypes.c_void_p, ctypes.c_int
         L.oracle_packed_bytes.restype = ll
         L.oracle_packed_bytes.argtypes = [i, ll, ll]
-        for name in ("oracle_pack_ptq1", "oracle_pack_pq2", "oracle_unpack_ptq1",
-                     "oracle_unpack_pq2"):
+        for name in ("oracle_pack_ptq1", "oracle_pack_pq2", "oracle_pack_q1", "oracle_unpack_ptq1",
+                     "oracle_unpack_pq2", "oracle_unpack_q1"):
             getattr(L, name).restype = ll
             getattr(L, name).argtypes = [p, p, ll, ll]
-        for name in ("oracle_check_ptq1", "oracle_check_pq2"):
+        for name in ("oracle_check_ptq1", "oracle_check_pq2", "oracle_check_q1"):
             getattr(L, name).restype = ll
             getattr(L, name).argtypes = [p, ll, ll]
         L.oracle_unpack.restype = ll
@@ -80,14 +81,16 @@ def packed_bytes(fmt: int, N: int, K: int) -> int:
 
 
 def pack(fmt: int, trits: np.ndarray) -> np.ndarray:
-    """N x K int8 trits -> packed uint8 plane (PTQ1_0: N x (K/128*26); PQ2_0: N x K/4)."""
+    """N x K int8 trits -> packed uint8 plane (PTQ1_0: N x (K/128*26); PQ2_0: N x K/4;
+    Q1_0: N x K/8, weights +-1)."""
     t = np.ascontiguousarray(trits, dtype=np.int8)
     N, K = t.shape
     nbytes = packed_bytes(fmt, N, K)
     if nbytes < 0:
         raise ValueError("bad format or shape")
     out = np.zeros(nbytes, dtype=np.uint8)
-    fn = lib().oracle_pack_ptq1 if fmt == FMT_PTQ1_0 else lib().oracle_pack_pq2
+    fn = {FMT_PTQ1_0: lib().oracle_pack_ptq1, FMT_PQ2_0: lib().oracle_pack_pq2,
+          FMT_Q1_0: lib().oracle_pack_q1}[fmt]
     fn(_ptr(t), _ptr(out), N, K)
     return out.reshape(N, -1) if N else out.reshape(0, 0)
 
@@ -107,7 +110,8 @@ def unpack(fmt: int, packed: np.ndarray, N: int, K: int):
 def check(fmt: int, packed: np.ndarray, N: int, K: int) -> int:
     """Number of non-canonical codes in a packed plane (0 for a valid one)."""
     p = np.ascontiguousarray(packed, dtype=np.uint8).reshape(-1)
-    fn = lib().oracle_check_ptq1 if fmt == FMT_PTQ1_0 else lib().oracle_check_pq2
+    fn = {FMT_PTQ1_0: lib().oracle_check_ptq1, FMT_PQ2_0: lib().oracle_check_pq2,
+          FMT_Q1_0: lib().oracle_check_q1}[fmt]
     return int(fn(_ptr(p), N, K))
 
 

@@ -17,6 +17,11 @@
  *      "each trit in a 2-bit slot", 2.13 bits/weight); and "Bonsai把 27B 大模型
  *      塞进手机的极端量化方案到底靠不靠谱" (wmrh.cn), section 关键机制 (the
  *      5 trits / 8 bits storage bound).
+ *      Q1_0   -- the 1-bit sibling: weights w in {-1, +1}, one bit each, 16 bytes
+ *                per group of 128.  Source: "Bonsai把 27B 大模型塞进手机的极端量化
+ *                方案到底靠不靠谱" (wmrh.cn), section 核心观点 (1-bit Bonsai, about
+ *                1.125 bits/weight, 3.9 GB) and section 关键机制 (weights held to
+ *                {-1, 1} or {-1, 0, 1} with an FP16 group-wise scale).
  *   2. the block Hadamard rotation of the activations, x' = blockdiag(Hn) x,
  *      with Hn = H_128 / sqrt(128) and H_128 the Sylvester matrix, written out
  *      as an explicit 128 x 128 matrix.  Source: allhereai.com page, the
@@ -32,8 +37,9 @@
  * Readings where the pages are silent (block size of the rotation, Sylvester
  * order and 1/sqrt(128) normalisation, base-3 digit order least significant
  * first, 2-bit slot order least significant first, code = trit + 1, padding
- * digits zero) are fixed here exactly as the CUDA library's header states
- * them, and are listed with their reasons in the design notes.
+ * digits zero, 1-bit order least significant first with bit 1 = +1) are fixed here
+ * exactly as the CUDA library's header states them, and are listed with their
+ * reasons in the design notes.
  *
  * Build: gcc -O2 -fopenmp -shared -fPIC -o liboracle.so bonsai_oracle.c -lm
  */
@@ -49,6 +55,7 @@
 #define ORACLE_GROUP 128
 #define ORACLE_FMT_PTQ1_0 1
 #define ORACLE_FMT_PQ2_0 2
+#define ORACLE_FMT_Q1_0 3
 #define ORACLE_PTQ1_GROUP_BYTES 26 /* 25 bytes x 5 trits + 1 byte x 3 trits */
 #define ORACLE_INVALID_TRIT (-128) /* written by the unpackers for an invalid code */
 
@@ -60,6 +67,7 @@ long long oracle_packed_bytes(int fmt, long long N, long long K)
     if (N < 0 || K < 0 || K % ORACLE_GROUP != 0) return -1;
     if (fmt == ORACLE_FMT_PTQ1_0) return N * (K / ORACLE_GROUP) * ORACLE_PTQ1_GROUP_BYTES;
     if (fmt == ORACLE_FMT_PQ2_0) return N * (K / 4);
+    if (fmt == ORACLE_FMT_Q1_0) return N * (K / 8);
     return -1;
 }
 
@@ -199,10 +207,55 @@ long long oracle_check_pq2(const uint8_t *packed, long long N, long long K)
     return bad;
 }
 
+/* ------------------------------------------------------------------ Q1_0 */
+
+/* Weight k of a row is bit (k mod 8) of byte k/8 of the row: 1 for +1, 0 for -1.  One
+ * bit has no invalid value, so a weight other than +1 or -1 is stored as -1 and counted
+ * in the return value. */
+long long oracle_pack_q1(const int8_t *trits, uint8_t *packed, long long N, long long K)
+{
+    long long bad = 0;
+    for (long long n = 0; n < N; n++)
+        for (long long byte = 0; byte < K / 8; byte++) {
+            int v = 0;
+            for (int i = 0; i < 8; i++) {
+                int t = trits[n * K + 8 * byte + i];
+                if (t == 1)
+                    v |= 1 << i;
+                else if (t != -1)
+                    bad++;
+            }
+            packed[n * (K / 8) + byte] = (uint8_t)v;
+        }
+    return bad;
+}
+
+static long long q1_unpack_row(const uint8_t *row, int8_t *t, long long K)
+{
+    for (long long k = 0; k < K; k++) t[k] = ((row[k / 8] >> (k % 8)) & 1) ? 1 : -1;
+    return 0;
+}
+
+long long oracle_unpack_q1(const uint8_t *packed, int8_t *trits, long long N, long long K)
+{
+    for (long long n = 0; n < N; n++) q1_unpack_row(packed + n * (K / 8), trits + n * K, K);
+    return 0;
+}
+
+/* Validator: every bit pattern is a valid Q1_0 plane. */
+long long oracle_check_q1(const uint8_t *packed, long long N, long long K)
+{
+    (void)packed;
+    (void)N;
+    (void)K;
+    return 0;
+}
+
 long long oracle_unpack(int fmt, const uint8_t *packed, int8_t *trits, long long N, long long K)
 {
     if (fmt == ORACLE_FMT_PTQ1_0) return oracle_unpack_ptq1(packed, trits, N, K);
     if (fmt == ORACLE_FMT_PQ2_0) return oracle_unpack_pq2(packed, trits, N, K);
+    if (fmt == ORACLE_FMT_Q1_0) return oracle_unpack_q1(packed, trits, N, K);
     return -1;
 }
 
@@ -295,8 +348,10 @@ long long oracle_ternary_linear(const double *x, const uint8_t *packed, const do
         int8_t *t = (int8_t *)malloc((size_t)(K > 0 ? K : 1));
         if (fmt == ORACLE_FMT_PTQ1_0)
             bad += ptq1_unpack_row(packed + n * row_bytes, t, K);
-        else
+        else if (fmt == ORACLE_FMT_PQ2_0)
             bad += pq2_unpack_row(packed + n * row_bytes, t, K);
+        else
+            bad += q1_unpack_row(packed + n * row_bytes, t, K);
         for (long long m = 0; m < M; m++) {
             double acc = 0.0;
             for (long long g = 0; g < G; g++) {

@@ -16,6 +16,7 @@ Distributions (the workload of the Bonsai 2 ternary linear layers: ternary
 trits with one FP16 scale per 128 weights and FP16 activations):
 
 * trits: u < 0.38 -> 0, u < 0.69 -> -1, else +1  (P(0)=.38, P(+-1)=.31);
+* signs (the 1-bit Q1_0 weights): u < 0.5 -> -1, else +1;
 * scales: 0.01 + 0.04 u in float64, rounded to FP16 (round to nearest even);
 * x: standard normal by the Box-Muller transform in float64, rounded to FP16.
 
@@ -34,6 +35,7 @@ _M2 = np.uint64(0x94D049BB133111EB)
 STREAM_TRITS = 1
 STREAM_SCALES = 2
 STREAM_X = 3
+STREAM_SIGNS = 4
 
 P_ZERO = 0.38
 P_MINUS = 0.31
@@ -95,6 +97,23 @@ def trits_rows(seed: int, K: int, rows, stream_id: int = STREAM_TRITS) -> np.nda
 def trits(seed: int, N: int, K: int, stream_id: int = STREAM_TRITS) -> np.ndarray:
     """N x K int8 trits, row-major."""
     return trits_rows(seed, K, np.arange(N), stream_id)
+
+
+def signs_rows(seed: int, K: int, rows, stream_id: int = STREAM_SIGNS) -> np.ndarray:
+    """1-bit weights (int8 in {-1, +1}) of the given rows of an N x K weight matrix."""
+    rows = np.asarray(rows, dtype=np.int64).reshape(-1)
+    key = stream_key(seed, stream_id)
+    out = np.empty((rows.size, K), dtype=np.int8)
+    step = max(1, _CHUNK // max(K, 1))
+    for r0 in range(0, rows.size, step):
+        u = uniform(key, _indices(rows[r0:r0 + step], K))
+        out[r0:r0 + step] = np.where(u < 0.5, -1, 1).astype(np.int8)
+    return out
+
+
+def signs(seed: int, N: int, K: int, stream_id: int = STREAM_SIGNS) -> np.ndarray:
+    """N x K int8 weights in {-1, +1}, row-major."""
+    return signs_rows(seed, K, np.arange(N), stream_id)
 
 
 def scales_rows(seed: int, G: int, rows, stream_id: int = STREAM_SCALES) -> np.ndarray:

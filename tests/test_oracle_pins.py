@@ -17,7 +17,12 @@ import oracle
 from ternary_weight_02_b200 import inputs
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
-PTQ1, PQ2 = oracle.FMT_PTQ1_0, oracle.FMT_PQ2_0
+PTQ1, PQ2, Q1 = oracle.FMT_PTQ1_0, oracle.FMT_PQ2_0, oracle.FMT_Q1_0
+
+
+def _weights(fmt, seed, N, K):
+    """Seeded weights a format can hold: trits, or signs for the 1-bit Q1_0."""
+    return inputs.signs(seed, N, K) if fmt == Q1 else inputs.trits(seed, N, K)
 
 
 def _golden_codec():
@@ -193,8 +198,43 @@ def test_bits_per_weight_match_pages():
 
 def test_packed_bytes_bad_shapes():
     assert oracle.packed_bytes(PTQ1, 4, 100) == -1
-    assert oracle.packed_bytes(3, 4, 128) == -1
+    assert oracle.packed_bytes(4, 4, 128) == -1
     assert oracle.packed_bytes(PQ2, 0, 128) == 0
+    assert oracle.packed_bytes(Q1, 4, 256) == 128 and oracle.packed_bytes(Q1, 1, 64) == -1
+
+
+def test_q1_bits_per_weight_match_pages():
+    # one bit per weight plus one FP16 scale per 128: 1.125, the 1-bit family's figure
+    pages = _golden_sizes()
+    K = 5120
+    bpw = oracle.packed_bytes(Q1, 1, K) * 8 / K + 16 / 128
+    assert bpw == 1.125 == pages["q1_bits_per_weight"]
+    # the 3.9 GB file then holds ~27.7e9 weights at that rate: the 27B model (the file
+    # also carries the unquantised parts, so the count is an upper bound)
+    n = pages["q1_file_gb"] * 8e9 / bpw
+    assert 26.5e9 < n < 28.5e9
+
+
+def test_q1_all_256_bytes_round_trip():
+    # bit i of byte b is weight 8b + i: 1 -> +1, 0 -> -1 (least significant first)
+    for v in range(256):
+        t, bad = oracle.unpack(Q1, np.full((1, 16), v, dtype=np.uint8), 1, 128)
+        assert bad == 0
+        want = np.array([1 if (v >> i) & 1 else -1 for i in range(8)] * 16, dtype=np.int8)
+        assert np.array_equal(t[0], want)
+        assert np.array_equal(oracle.pack(Q1, t), np.full((1, 16), v, dtype=np.uint8))
+        assert oracle.check(Q1, np.full((1, 16), v, dtype=np.uint8), 1, 128) == 0
+
+
+def test_q1_pack_counts_non_binary_and_stores_minus_one():
+    t = np.ones((2, 128), dtype=np.int8)
+    t[0, 3] = 0
+    t[1, 127] = 2
+    p = oracle.pack(Q1, t)
+    assert p[0, 0] == 0xF7 and p[1, 15] == 0x7F
+    u, bad = oracle.unpack(Q1, p, 2, 128)
+    assert u[0, 3] == -1 and u[1, 127] == -1 and bad == 0
+    assert int(oracle.lib().oracle_pack_q1(oracle._ptr(t), oracle._ptr(np.zeros(32, np.uint8)), 2, 128)) == 2
 
 
 # ---------------------------------------------------------------- Hadamard
@@ -268,10 +308,10 @@ def _dense(trits, scales):
     return trits.astype(np.float64) * np.repeat(scales.astype(np.float64), 128, axis=1)
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
 @pytest.mark.parametrize("N,K,M", [(1, 128, 1), (3, 256, 2), (8, 128, 3), (5, 384, 1)])
 def test_linear_brute_force_dense(fmt, N, K, M):
-    t = inputs.trits(11, N, K)
+    t = _weights(fmt, 11, N, K)
     s = inputs.scales(11, N, K)
     x = inputs.activations(11, M, K)
     y = oracle.ternary_linear(x, oracle.pack(fmt, t), s, N, K, fmt)
@@ -305,6 +345,39 @@ def test_linear_hand_cases(fmt):
     t = np.ones((1, K), dtype=np.int8)
     y = oracle.ternary_linear(xd, oracle.pack(fmt, t), s, 1, K, fmt)
     assert np.isclose(y[0, 0], 0.25 * np.sqrt(128.0), rtol=1e-14)
+
+
+def test_linear_q1_hand_cases():
+    K = 256
+    s = np.array([[0.5, 0.25]], dtype=np.float16)
+    x = inputs.activations(3, 1, K)
+    xr = oracle.hadamard128(x.astype(np.float64))
+    full = 0.5 * xr[0, :128].sum() + 0.25 * xr[0, 128:].sum()
+    t = np.ones((1, K), dtype=np.int8)
+    assert np.isclose(oracle.ternary_linear(x, oracle.pack(Q1, t), s, 1, K, Q1)[0, 0], full, rtol=1e-13)
+    # all -1: the negation
+    assert np.isclose(oracle.ternary_linear(x, oracle.pack(Q1, -t), s, 1, K, Q1)[0, 0], -full, rtol=1e-13)
+    # one weight flipped to -1 at k = 200 (group 1): y = full - 2 * 0.25 * x'[200]
+    t[0, 200] = -1
+    y = oracle.ternary_linear(x, oracle.pack(Q1, t), s, 1, K, Q1)
+    assert np.isclose(y[0, 0], full - 0.5 * xr[0, 200], rtol=1e-12)
+
+
+def test_linear_q1_agrees_with_ternary_formats_on_signs():
+    # weights +-1 are valid in all three packings: the three decodes give one result
+    N, K, M = 17, 384, 3
+    t = inputs.signs(6, N, K)
+    s = inputs.scales(6, N, K)
+    x = inputs.activations(6, M, K)
+    yq = oracle.ternary_linear(x, oracle.pack(Q1, t), s, N, K, Q1)
+    for fmt in (PTQ1, PQ2):
+        assert np.array_equal(yq, oracle.ternary_linear(x, oracle.pack(fmt, t), s, N, K, fmt))
+
+
+def test_signs_generator():
+    t = inputs.signs(1, 64, 1024)
+    assert set(np.unique(t)) == {-1, 1} and abs(float((t == 1).mean()) - 0.5) < 0.01
+    assert np.array_equal(inputs.signs_rows(1, 1024, [5, 63]), t[[5, 63]])
 
 
 def test_linear_formats_agree_and_threads_agree():
