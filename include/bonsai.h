@@ -32,6 +32,11 @@
  *     BONSAI_FMT_PQ2_0   one trit per 2-bit slot, 2.125 bits/weight with the
  *         scale: weight k of row n is code t+1 in bits 2(k%4), 2(k%4)+1 of byte
  *         n*K/4 + k/4 (code 3 is invalid).  Trit plane size N * K/4 bytes.
+ *     BONSAI_FMT_Q1_0    the 1-bit sibling of the wmrh.cn page (section 核心观点,
+ *         ~1.125 bits/weight; section 关键机制, weights in {-1, +1} with an FP16
+ *         group scale): weight k of row n is bit k%8 of byte n*K/8 + k/8, 1 for +1
+ *         and 0 for -1 (every byte is valid).  Plane size N * K/8 bytes.  Same
+ *         scale plane and the same rotation of x as the ternary packings.
  *
  * Conventions for every entry point:
  *   - Pointers are CUDA device pointers (any allocator) and must be 16-byte
@@ -63,7 +68,8 @@ extern "C" {
 
 typedef enum {
     BONSAI_FMT_PTQ1_0 = 1,
-    BONSAI_FMT_PQ2_0 = 2
+    BONSAI_FMT_PQ2_0 = 2,
+    BONSAI_FMT_Q1_0 = 3
 } bonsai_fmt;
 
 typedef enum {
@@ -114,6 +120,10 @@ int bonsai_pack_ptq1(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K,
 /* Packs N x K trits into the PQ2_0 plane (layout above).  A trit outside
  * {-1, 0, +1} is stored as the invalid code 3.  Same source. */
 int bonsai_pack_pq2(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K, void *stream);
+
+/* Packs N x K weights into the Q1_0 plane (layout above): +1 -> bit 1, any other
+ * value -> bit 0 (-1).  Source: wmrh.cn page, sections 核心观点 and 关键机制. */
+int bonsai_pack_q1(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K, void *stream);
 
 /* Unpacks a plane of format fmt back into N x K int8 trits.  Invalid codes
  * unpack to -128 (every trit of an invalid PTQ1_0 byte).  Test hook: it makes

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(PKG, "libbonsai.so")
 
 BONSAI_FMT_PTQ1_0 = 1
 BONSAI_FMT_PQ2_0 = 2
+BONSAI_FMT_Q1_0 = 3
 
 BONSAI_OK = 0
 BONSAI_ERR_NULL = -1
@@ -37,7 +38,7 @@ BONSAI_ALGO_SKINNY = 3
 BONSAI_ALGO_GEMM = 4
 BONSAI_ALGO_IMMA = 5
 
-FORMATS = {"ptq1": BONSAI_FMT_PTQ1_0, "pq2": BONSAI_FMT_PQ2_0}
+FORMATS = {"ptq1": BONSAI_FMT_PTQ1_0, "pq2": BONSAI_FMT_PQ2_0, "q1": BONSAI_FMT_Q1_0}
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -54,6 +55,7 @@ _SIGS = {
     "bonsai_packed_bytes": (_i64, [_int, _i64, _i64]),
     "bonsai_pack_ptq1": (_int, [_p, _p, _i64, _i64, _p]),
     "bonsai_pack_pq2": (_int, [_p, _p, _i64, _i64, _p]),
+    "bonsai_pack_q1": (_int, [_p, _p, _i64, _i64, _p]),
     "bonsai_unpack": (_int, [_int, _p, _p, _i64, _i64, _p]),
     "bonsai_hadamard128": (_int, [_p, _p, _i64, _i64, _p]),
     "bonsai_ternary_linear": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _p]),
@@ -134,6 +136,10 @@ def bonsai_pack_pq2(trits, packed, N: int, K: int, stream=None) -> None:
     _check(_lib.bonsai_pack_pq2(_ptr(trits), _ptr(packed), N, K, _stream(stream)), "bonsai_pack_pq2")
 
 
+def bonsai_pack_q1(trits, packed, N: int, K: int, stream=None) -> None:
+    _check(_lib.bonsai_pack_q1(_ptr(trits), _ptr(packed), N, K, _stream(stream)), "bonsai_pack_q1")
+
+
 def bonsai_unpack(fmt: int, packed, trits, N: int, K: int, stream=None) -> None:
     _check(_lib.bonsai_unpack(fmt, _ptr(packed), _ptr(trits), N, K, _stream(stream)), "bonsai_unpack")
 
@@ -185,7 +191,8 @@ def pack(fmt: int, trits, stream=None):
     import torch
     N, K = trits.shape
     out = torch.empty(bonsai_packed_bytes(fmt, N, K), dtype=torch.uint8, device=trits.device)
-    fn = bonsai_pack_ptq1 if fmt == BONSAI_FMT_PTQ1_0 else bonsai_pack_pq2
+    fn = {BONSAI_FMT_PTQ1_0: bonsai_pack_ptq1, BONSAI_FMT_PQ2_0: bonsai_pack_pq2,
+          BONSAI_FMT_Q1_0: bonsai_pack_q1}[fmt]
     fn(trits, out, N, K, stream)
     return out.view(N, -1) if N else out
 

@@ -124,7 +124,8 @@ int check_shape(int64_t M, int64_t N, int64_t K) {
 }
 
 int check_fmt(int fmt) {
-    return (fmt == BONSAI_FMT_PTQ1_0 || fmt == BONSAI_FMT_PQ2_0) ? BONSAI_OK : BONSAI_ERR_FMT;
+    return (fmt == BONSAI_FMT_PTQ1_0 || fmt == BONSAI_FMT_PQ2_0 || fmt == BONSAI_FMT_Q1_0) ? BONSAI_OK
+                                                                                         : BONSAI_ERR_FMT;
 }
 
 int cuda_status(cudaError_t e) {
@@ -209,6 +210,7 @@ int64_t bonsai_packed_bytes(int fmt, int64_t N, int64_t K) {
     if (check_fmt(fmt) != BONSAI_OK) return BONSAI_ERR_FMT;
     if (check_shape(0, N, K) != BONSAI_OK) return BONSAI_ERR_SHAPE;
     if (fmt == BONSAI_FMT_PTQ1_0) return N * (K / kGroup) * kPtq1GroupBytes;
+    if (fmt == BONSAI_FMT_Q1_0) return N * (K / 8);
     return N * (K / 4);
 }
 
@@ -228,6 +230,7 @@ static int pack_common(const int8_t *trits, uint8_t *packed, int64_t N, int64_t 
     if (rc != BONSAI_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (fmt == BONSAI_FMT_PTQ1_0) return cuda_status(launch_pack_ptq1(trits, packed, N, K, s, st->info));
+    if (fmt == BONSAI_FMT_Q1_0) return cuda_status(launch_pack_q1(trits, packed, N, K, s, st->info));
     return cuda_status(launch_pack_pq2(trits, packed, N, K, s, st->info));
 }
 
@@ -237,6 +240,10 @@ int bonsai_pack_ptq1(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K,
 
 int bonsai_pack_pq2(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K, void *stream) {
     return pack_common(trits, packed, N, K, stream, BONSAI_FMT_PQ2_0);
+}
+
+int bonsai_pack_q1(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K, void *stream) {
+    return pack_common(trits, packed, N, K, stream, BONSAI_FMT_Q1_0);
 }
 
 int bonsai_unpack(int fmt, const uint8_t *packed, int8_t *trits, int64_t N, int64_t K, void *stream) {
@@ -354,7 +361,7 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
     rc = probe_current(&dev, &st);
     if (rc != BONSAI_OK) return rc;
     size_t need = simple_workspace_bytes(M, N, K), zneed = 0;
-    for (int fmt = BONSAI_FMT_PTQ1_0; fmt <= BONSAI_FMT_PQ2_0; fmt++) {
+    for (int fmt = BONSAI_FMT_PTQ1_0; fmt <= BONSAI_FMT_Q1_0; fmt++) {
         size_t v;
         if (M <= 1 && gemv_supported(1, N, K, fmt)) {
             v = gemv_workspace_bytes(N, K, fmt, 0, st->info);

@@ -16,6 +16,7 @@ namespace bonsai {
 constexpr int kGroup = 128;           // weights per FP16 scale == Hadamard block size
 constexpr int kPtq1GroupBytes = 26;   // 25 bytes x 5 trits + 1 byte x 3 trits
 constexpr int kPq2GroupBytes = 32;    // 128 trits x 2 bits
+constexpr int kQ1GroupBytes = 16;     // 128 signs x 1 bit
 constexpr float kHadamardNorm = 0.088388347648318440550f;  // 1/sqrt(128)
 
 __device__ __forceinline__ float half_bits_to_float(uint16_t h) {

@@ -137,6 +137,22 @@ __device__ __forceinline__ void expand_word(uint32_t w, uint32_t tneg, uint32_t 
     }
 }
 
+// Q1_0: one 32-bit word of signs (bit i = weight w0+i, 1 for +1) times the scale s, as
+// four 16-byte chunks of FP16: out[0..3] = weights [0,8,1,9,2,10,3,11], out[4..7] =
+// [4,12,..,7,15], out[8..11] = 16 + [0,8,..], out[12..15] = 16 + [4,12,..] (x' is stored
+// in the same order within each 16).  The value of bit b is byte pair (2b, 2b+1) of the
+// table tab = -s | +s << 16.
+__device__ __forceinline__ void expand_word_q1(uint32_t w, uint32_t tab, uint32_t (&out)[16]) {
+#pragma unroll
+    for (int j = 0; j < 8; j++) {
+        const uint32_t m = (w >> j) & 0x01010101u;  // weights j, j + 8, j + 16, j + 24
+        const uint32_t sel = m * 0x22u + 0x10101010u;
+        const int c = (j >> 2) * 4 + (j & 3);
+        out[c] = __byte_perm(tab, 0u, sel);             // weights j, j + 8
+        out[8 + c] = __byte_perm(tab, 0u, sel >> 16);   // weights j + 16, j + 24
+    }
+}
+
 // Stores one 16-byte chunk (8 halves) of row r of a B stage at its swizzled place.
 __device__ __forceinline__ void st_chunk(uint8_t *stage, int r, int chunk, const uint32_t *v) {
     uint4 *p = reinterpret_cast<uint4 *>(stage + r * 128 + ((chunk ^ (r & 7)) << 4));
@@ -159,6 +175,10 @@ __device__ __forceinline__ void load_group(const uint8_t *packed, const uint16_t
         const uint4 a = __ldg(p), b = __ldg(p + 1);
         raw.w[0] = a.x, raw.w[1] = a.y, raw.w[2] = a.z, raw.w[3] = a.w;
         raw.w[4] = b.x, raw.w[5] = b.y, raw.w[6] = b.z, raw.w[7] = b.w;
+    } else if (kFmt == 3) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(packed + (n * G + g) * kQ1GroupBytes));
+        raw.w[0] = a.x, raw.w[1] = a.y, raw.w[2] = a.z, raw.w[3] = a.w;
+        raw.w[4] = raw.w[5] = raw.w[6] = raw.w[7] = 0u;
     } else {
         // 26 bytes at an even address: 6 aligned words and one aligned half-word
         const uint8_t *src = packed + (n * G + g) * kPtq1GroupBytes;
@@ -185,7 +205,7 @@ __device__ __forceinline__ void load_group(const uint8_t *packed, const uint16_t
 // Codes of the group as 8 words (word i: weights 16i .. 16i+15, code = trit + 1).
 template <int kFmt>
 __device__ __forceinline__ void group_codes(const GroupRaw &raw, const uint32_t *lut, uint32_t (&cw)[8]) {
-    if (kFmt == 2) {
+    if (kFmt == 2 || kFmt == 3) {  // (Q1_0: sign words 0..3)
 #pragma unroll
         for (int i = 0; i < 8; i++) cw[i] = raw.w[i];
     } else {
@@ -423,13 +443,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
             const int64_t n = (int64_t)tn * BN + r;  // weight row
             const bool valid = n < N;
             if (live) {
-                // PTQ1_0: the packed bytes of the group being expanded and of the next one (in
+                // PTQ1_0, Q1_0: the packed bytes of the group being expanded and of the next one (in
                 // flight) come by plain loads; PQ2_0: the codes come with the stage's x' tiles
                 // (TMA), only the scale by a plain load, one group ahead
                 GroupRaw cur, nxt;
                 const int g_last = (p.ke - 1) >> 1;
                 uint32_t sc = 0u;
-                if (kFmt == 1 && valid) load_group<kFmt>(packed, scales, n, G, p.kb >> 1, cur);
+                if (kFmt != 2 && valid) load_group<kFmt>(packed, scales, n, G, p.kb >> 1, cur);
                 if (kFmt == 2 && valid) sc = __ldg(scales + n * G + (p.kb >> 1));
                 uint32_t cw[8];
                 uint32_t tneg = 0u, tpos = 0u;  // the group's value table {-s, 0, +s}
@@ -450,6 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
 #pragma unroll
                                 for (int i = 0; i < 8; i++) cw[i] = 0x55555555u;  // all trits zero
                             }
+                            if (kFmt == 3)  // Q1_0: one table {-s, +s}
+                                tneg = valid ? ((uint32_t)cur.scale ^ 0x8000u) | ((uint32_t)cur.scale << 16) : 0u;
                         }
                     }
                     const int st = it % STAGES;
@@ -472,19 +494,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                         for (int i = 0; i < 4; i++) w4[i] = hf ? cw[4 + i] : cw[i];
                     }
                     uint8_t *stage = sB + st * B_STAGE_BYTES;
+                    if (kFmt == 3) {
+                        const uint32_t wq[2] = {hf ? cw[2] : cw[0], hf ? cw[3] : cw[1]};  // no dynamic index
 #pragma unroll
-                    for (int i = 0; i < 4; i++) {
-                        uint32_t out[8];
-                        expand_word(w4[i], tneg, tpos, out);  // weights 64ks + 16i .. +15
-                        st_chunk(stage, r, 2 * i, out);
-                        st_chunk(stage, r, 2 * i + 1, out + 4);
+                        for (int i = 0; i < 2; i++) {
+                            uint32_t out[16];
+                            expand_word_q1(wq[i], tneg, out);  // weights 64ks + 32i .. +31
+#pragma unroll
+                            for (int c = 0; c < 4; c++) st_chunk(stage, r, 4 * i + c, out + 4 * c);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; i++) {
+                            uint32_t out[8];
+                            expand_word(w4[i], tneg, tpos, out);  // weights 64ks + 16i .. +15
+                            st_chunk(stage, r, 2 * i, out);
+                            st_chunk(stage, r, 2 * i + 1, out + 4);
+                        }
                     }
                     // make the generic-proxy accesses (these stores, the code loads) ordered
                     // before later async-proxy ones, then signal
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                     if (lane == 0) mbar_arrive(full_b + st);
-                    if (kFmt == 1 && hf == 1) cur = nxt;
+                    if (kFmt != 2 && hf == 1) cur = nxt;
                 }
             }
 
@@ -648,7 +681,7 @@ size_t x_rot_bytes(int64_t M, int64_t K) { return (((size_t)M * (size_t)K * 2) +
 }  // namespace
 
 bool gemm_supported(int64_t M, int64_t N, int64_t K, int fmt) {
-    (void)fmt;
+    if (fmt != 1 && fmt != 2 && fmt != 3) return false;
     // TMA coordinates are 32-bit; the unit count of the work split must fit an int
     if (!(M >= 1 && M < (int64_t)1 << 30 && N >= 1 && N < (int64_t)1 << 30 && K % kGroup == 0 &&
           K < (int64_t)1 << 30))
@@ -670,7 +703,9 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
     if (ws.data_bytes < gemm_workspace_bytes(M, N, K, fmt, dev) || plan.ctas > kMaxTiles) return cudaErrorInvalidValue;
     uint16_t *xr = reinterpret_cast<uint16_t *>(ws.data);
     float *partials = reinterpret_cast<float *>(ws.data + x_rot_bytes(M, K));
-    cudaError_t err = launch_hadamard_f16_perm8(x, xr, M, K, s, dev);  // in the expansion's K order
+    // x' in the expansion's K order
+    cudaError_t err = fmt == 3 ? launch_hadamard_f16_perm16(x, xr, M, K, s, dev)
+                               : launch_hadamard_f16_perm8(x, xr, M, K, s, dev);
     if (err != cudaSuccess) return err;
 
     EncodeTiledFn encode = encode_fn();
@@ -706,6 +741,9 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
     if (fmt == 1)
         return plan.acc == 2 ? go(gemm_tcgen05_kernel<1, 2>, Cfg<2>::kSmemBytes)
                              : go(gemm_tcgen05_kernel<1, 1>, Cfg<1>::kSmemBytes);
+    if (fmt == 3)
+        return plan.acc == 2 ? go(gemm_tcgen05_kernel<3, 2>, Cfg<2>::kSmemBytes)
+                             : go(gemm_tcgen05_kernel<3, 1>, Cfg<1>::kSmemBytes);
     return plan.acc == 2 ? go(gemm_tcgen05_kernel<2, 2>, Cfg<2>::kSmemBytes)
                          : go(gemm_tcgen05_kernel<2, 1>, Cfg<1>::kSmemBytes);
 }

@@ -1,5 +1,7 @@
-// gemv_lut.cu -- batch-1 (M == 1) ternary GEMV for both packings, with the block
-// Hadamard rotation of x fused in.
+// gemv_lut.cu -- batch-1 (M == 1) ternary GEMV for the packings, with the block
+// Hadamard rotation of x fused in.  Q1_0 (1-bit, "Bonsai把 27B 大模型塞进手机的极端量化方案
+// 到底靠不靠谱" (wmrh.cn), sections 核心观点 and 关键机制): a byte holds 8 signs, so its
+// table covers 8 activations and a 128-byte row slice covers 1024 (split mode only).
 //
 // Operation: y[n] = sum_g s[n][g] * sum_j t[n][128g+j] * x'[128g+j], x' = blockdiag(Hn) x.
 // Sources: "27B 模型压到 5.95GB，推理能力还保住 98%" (allhereai.com): method paragraph
@@ -71,6 +73,8 @@ struct Fmt;
 
 template <>
 struct Fmt<2> {  // PQ2_0
+    static constexpr int kSliceK = 512;       // activations per K slice
+    static constexpr int kLanesPerGroup = 8;  // lanes whose words cover one scale group
     static constexpr int kSliceBytes = 128;
     __device__ static int64_t row_bytes(int64_t K) { return K / 4; }
     // byte offset of the lane's word inside a row's slice segment
@@ -79,6 +83,8 @@ struct Fmt<2> {  // PQ2_0
 
 template <>
 struct Fmt<1> {  // PTQ1_0
+    static constexpr int kSliceK = 512;
+    static constexpr int kLanesPerGroup = 8;
     static constexpr int kSliceBytes = 4 * kPtq1GroupBytes;  // 104
     __device__ static int64_t row_bytes(int64_t K) { return (K / kGroup) * kPtq1GroupBytes; }
     // the 8th lane of a group reads a valid word too; its tables are all zero
@@ -86,6 +92,15 @@ struct Fmt<1> {  // PTQ1_0
         const int g = lane >> 3, k = lane & 7;
         return kPtq1GroupBytes * g - 2 * (g & 1) + 4 * (k == 7 ? 0 : k);  // 4-byte aligned
     }
+};
+
+template <>
+struct Fmt<3> {  // Q1_0: a byte holds 8 signs, so a 128-byte row slice covers 1024 activations
+    static constexpr int kSliceK = 1024;
+    static constexpr int kLanesPerGroup = 4;
+    static constexpr int kSliceBytes = 128;
+    __device__ static int64_t row_bytes(int64_t K) { return K / 8; }
+    __device__ static int lane_offset(int lane) { return 4 * lane; }
 };
 
 // PTQ1_0: position (inside its group) of byte slot j of lane, or -1 for a slot that
@@ -107,11 +122,44 @@ __device__ __forceinline__ float signed_term(int digit, float xv) {
     return digit == 0 ? -xv : (digit == 1 ? 0.f : xv);
 }
 
+// Q1_0: table (lane, j) belongs to byte 4 lane + j of the row slice, i.e. activations
+// 8(4 lane + j) .. +7; entry e = sum_i (bit i of e ? +x'_i : -x'_i), as a sum of two
+// halves L[e & 15] + H[e >> 4].  Thread t serves table (lane = t & 31, j = (t >> 5) & 3)
+// and its 64 entries e >> 6 == t >> 7.
+__device__ __forceinline__ void build_tables_q1(const float *xr, uint8_t *tables, int t) {
+    const int lane = t & 31, j = (t >> 5) & 3, q = t >> 7;
+    const float *xa = xr + 8 * (4 * lane + j);
+    const float4 a = *reinterpret_cast<const float4 *>(xa), b = *reinterpret_cast<const float4 *>(xa + 4);
+    const float lo[4] = {a.x, a.y, a.z, a.w}, hi[4] = {b.x, b.y, b.z, b.w};
+    float L[16];
+#pragma unroll
+    for (int e = 0; e < 16; e++) {
+        float v = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; i++) v += ((e >> i) & 1) ? lo[i] : -lo[i];
+        L[e] = v;
+    }
+#pragma unroll
+    for (int hh = 0; hh < 4; hh++) {
+        const int h = 4 * q + hh;  // high nibble
+        float H = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; i++) H += ((h >> i) & 1) ? hi[i] : -hi[i];
+#pragma unroll
+        for (int l = 0; l < 16; l++)
+            *reinterpret_cast<float *>(tables + table_offset(lane, j, 16 * h + l)) = L[l] + H;
+    }
+}
+
 // Builds one slice's tables from its x' (FP32 in shared memory).  Thread t serves table
 // (lane = t & 31, slot j = (t >> 5) & 3) and, of that table's 3^(n-2) settings of its
 // high digits, those congruent to t >> 7 (mod 4); each setting is 9 entries.
 template <int kFmt>
 __device__ __forceinline__ void build_tables(const float *xr, uint8_t *tables, int t) {
+    if (kFmt == 3) {
+        build_tables_q1(xr, tables, t);
+        return;
+    }
     const int lane = t & 31, j = (t >> 5) & 3, q = t >> 7;
     const float *xa;
     int n, place;  // trits in the chunk, place value of one digit (4: 2-bit slots, 3: base 3)
@@ -179,26 +227,29 @@ __device__ __forceinline__ void zero_phantom_tables(uint8_t *tables, int lane, i
 // lane applies after the group reduction: rows (lane & 7) + 8m of group lane >> 3.
 // Nothing here consumes the loaded values, so the loads stay in flight until the
 // task is processed (the scales are converted only there).
-template <int kFmt>
-__device__ __forceinline__ void load_task(uint32_t (&w)[kRows], uint16_t (&sc)[2], const uint8_t *slice_base,
+// kNS = kRows / kLanesPerGroup scales per lane: rows (lane % lpg) + lpg m of group
+// lane / lpg (lpg = lanes per scale group: 8, or 4 for Q1_0).
+template <int kFmt, int kNS = kRows / Fmt<kFmt>::kLanesPerGroup>
+__device__ __forceinline__ void load_task(uint32_t (&w)[kRows], uint16_t (&sc)[kNS], const uint8_t *slice_base,
                                           const uint16_t *scales, int64_t n0, int64_t N, int64_t G,
                                           int64_t gcol, uint32_t row_bytes, int lane_off, int lane) {
+    constexpr int lpg = Fmt<kFmt>::kLanesPerGroup;
     const uint8_t *p = slice_base + n0 * row_bytes + lane_off;
-    const uint16_t *sp = scales + (n0 + (lane & 7)) * G + gcol;
+    const uint16_t *sp = scales + (n0 + (lane % lpg)) * G + gcol;
     if (N - n0 >= kRows) {  // full task: no predicates
 #pragma unroll
         for (int i = 0; i < kRows; i++)
             w[i] = __ldcs(reinterpret_cast<const unsigned int *>(p + (size_t)i * row_bytes));
-        sc[0] = __ldg(sp);
-        sc[1] = __ldg(sp + 8 * G);
+#pragma unroll
+        for (int m = 0; m < kNS; m++) sc[m] = __ldg(sp + (int64_t)lpg * m * G);
         return;
     }
     const int nvalid = (int)(N - n0);
 #pragma unroll
     for (int i = 0; i < kRows; i++)
         w[i] = i < nvalid ? __ldcs(reinterpret_cast<const unsigned int *>(p + (size_t)i * row_bytes)) : 0u;
-    sc[0] = (lane & 7) < nvalid ? __ldg(sp) : (uint16_t)0;
-    sc[1] = (lane & 7) + 8 < nvalid ? __ldg(sp + 8 * G) : (uint16_t)0;
+#pragma unroll
+    for (int m = 0; m < kNS; m++) sc[m] = (lane % lpg) + lpg * m < nvalid ? __ldg(sp + (int64_t)lpg * m * G) : (uint16_t)0;
 }
 
 __device__ __forceinline__ float lds_abs(uint32_t addr) {
@@ -241,6 +292,30 @@ __device__ __forceinline__ float2 task_group_sums(const uint32_t (&w)[kRows], co
     return make_float2(v[0] * half_bits_to_float(sc[0]), v[1] * half_bits_to_float(sc[1]));
 }
 
+// Q1_0: lookups of one task, the reduction over the 4 lanes of each of the slice's 8
+// scale groups, the scales, then the sum over the groups.  Lanes L and L + 16 end with
+// row L & 15 of the task.
+__device__ __forceinline__ float task_total_q1(const uint32_t (&w)[kRows], const uint16_t (&sc)[4],
+                                               const uint32_t (&pbase)[4], int lane) {
+    float v[kRows];
+#pragma unroll
+    for (int i = 0; i < kRows; i++) {
+        const float t0 = lds_abs(__byte_perm(w[i], pbase[0], 0x7604));
+        const float t1 = lds_abs(__byte_perm(w[i], pbase[1], 0x7614));
+        const float t2 = lds_abs(__byte_perm(w[i], pbase[2], 0x7624));
+        const float t3 = lds_abs(__byte_perm(w[i], pbase[3], 0x7634));
+        const float2 u = __fadd2_rn(make_float2(t0, t1), make_float2(t2, t3));
+        v[i] = u.x + u.y;
+    }
+    transpose_stage<8>(v, lane, 0);
+    transpose_stage<4>(v, lane, 1);  // v[m]: row (lane & 3) + 4m of group lane >> 2
+#pragma unroll
+    for (int m = 0; m < 4; m++) v[m] *= half_bits_to_float(sc[m]);
+    transpose_stage<2>(v, lane, 2);
+    transpose_stage<1>(v, lane, 3);  // v[0]: row lane & 15, summed over lane bits 2, 3
+    return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 16);
+}
+
 // Sum of the four groups: lanes L and L + 16 end with row L & 15 of the task.
 __device__ __forceinline__ float groups_total(float2 g, int lane) {
     const bool hi = (lane >> 3) & 1;
@@ -273,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t G = K / kGroup;
-    const int S = (int)(K / kSliceK);
+    constexpr int kSK = Fmt<kFmt>::kSliceK, kLPG = Fmt<kFmt>::kLanesPerGroup, kNS = kRows / kLPG;
+    const int S = (int)(K / kSK);
     const int64_t RB = (N + kRows - 1) / kRows;
     // CTA = (slice, part): the row blocks of one part of the rows, for one K slice
     const int slice = blockIdx.x / parts, part = blockIdx.x - slice * parts;
@@ -281,20 +357,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
     const uint32_t row_bytes = (uint32_t)Fmt<kFmt>::row_bytes(K);
     const int lane_off = Fmt<kFmt>::lane_offset(lane);
     const uint8_t *slice_base = packed + (int64_t)slice * Fmt<kFmt>::kSliceBytes;
-    const int64_t gcol = (int64_t)slice * (kSliceK / kGroup) + (lane >> 3);
+    const int64_t gcol = (int64_t)slice * (kSK / kGroup) + lane / kLPG;
 
     zero_phantom_tables<kFmt>(tables, lane, warp);
     pdl_wait();  // x, the workspace and y may belong to the previous kernel
     // x first, so that its loads are not queued behind this CTA's weight loads
     float xv[4];
-    if (warp < 4) load_half4(x + (int64_t)slice * kSliceK + warp * kGroup + 4 * lane, xv);
+    if (warp < kSK / kGroup) load_half4(x + (int64_t)slice * kSK + warp * kGroup + 4 * lane, xv);
     int64_t rb = rb_begin + warp;
     uint32_t wa[kRows], wb[kRows], wc[kRows];
-    uint16_t sa[2], sb[2], sc2[2];
+    uint16_t sa[kNS], sb[kNS], sc2[kNS];
     if (rb < rb_end) load_task<kFmt>(wa, sa, slice_base, scales, rb * kRows, N, G, gcol, row_bytes, lane_off, lane);
     if (rb + kWarps < rb_end)
         load_task<kFmt>(wb, sb, slice_base, scales, (rb + kWarps) * kRows, N, G, gcol, row_bytes, lane_off, lane);
-    if (warp < 4) {  // rotate the slice of x: 4 blocks of 128
+    if (warp < kSK / kGroup) {  // rotate the slice of x: 4 (Q1_0: 8) blocks of 128
         fwht128_warp(xv, lane);
         *reinterpret_cast<float4 *>(xr + warp * kGroup + 4 * lane) = make_float4(xv[0], xv[1], xv[2], xv[3]);
     }
@@ -306,8 +382,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
 
     // one slice's sums go straight to y (S == 1) or to the FP32 partials, which
     // gemv_reduce_kernel adds up in slice order
-    auto finish = [&](float2 gs, int64_t task_rb) {
-        const float total = groups_total(gs, lane);
+    auto task_total = [&](const uint32_t(&w)[kRows], const uint16_t(&sc)[kNS]) -> float {
+        if constexpr (kFmt == 3)
+            return task_total_q1(w, sc, pbase, lane);
+        else
+            return groups_total(task_group_sums(w, sc, pbase, lane), lane);
+    };
+    auto finish = [&](float total, int64_t task_rb) {
         const int64_t n0 = task_rb * kRows;
         const int row = lane & 15;
         if (lane < 16 && n0 + row < N) {
@@ -321,17 +402,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
     while (rb < rb_end) {
         if (rb + 2 * kWarps < rb_end)
             load_task<kFmt>(wc, sc2, slice_base, scales, (rb + 2 * kWarps) * kRows, N, G, gcol, row_bytes, lane_off, lane);
-        finish(task_group_sums(wa, sa, pbase, lane), rb);
+        finish(task_total(wa, sa), rb);
         rb += kWarps;
         if (rb >= rb_end) break;
         if (rb + 2 * kWarps < rb_end)
             load_task<kFmt>(wa, sa, slice_base, scales, (rb + 2 * kWarps) * kRows, N, G, gcol, row_bytes, lane_off, lane);
-        finish(task_group_sums(wb, sb, pbase, lane), rb);
+        finish(task_total(wb, sb), rb);
         rb += kWarps;
         if (rb >= rb_end) break;
         if (rb + 2 * kWarps < rb_end)
             load_task<kFmt>(wb, sb, slice_base, scales, (rb + 2 * kWarps) * kRows, N, G, gcol, row_bytes, lane_off, lane);
-        finish(task_group_sums(wc, sc2, pbase, lane), rb);
+        finish(task_total(wc, sc2), rb);
         rb += kWarps;
     }
 }
@@ -448,8 +529,10 @@ bool use_rows_mode(int64_t N, int64_t K, int fmt, const DeviceInfo &dev) {
 
 // Split mode: rows of the weight matrix are split into `parts` ranges per K slice so that
 // the grid (slices x parts) fills the SMs once.
-int gemv_parts(int64_t N, int64_t K, const DeviceInfo &dev) {
-    const int64_t S = K / kSliceK;
+int slice_k(int fmt) { return fmt == 3 ? Fmt<3>::kSliceK : kSliceK; }
+
+int gemv_parts(int64_t N, int64_t K, int fmt, const DeviceInfo &dev) {
+    const int64_t S = K / slice_k(fmt);
     const int64_t RB = (N + kRows - 1) / kRows;
     int64_t parts = dev.sm_count / S;
     if (parts < 1) parts = 1;
@@ -488,41 +571,42 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args.
 // Split mode: the slice kernel, then (K > 512) the in-order reduction of its partials.
 cudaError_t launch_split(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
                          float *partials, int64_t N, int64_t K, int fmt, cudaStream_t s, const DeviceInfo &dev) {
-    const int parts = gemv_parts(N, K, dev);
-    const int64_t grid = (K / kSliceK) * parts;
+    const int parts = gemv_parts(N, K, fmt, dev);
+    const int64_t S = K / slice_k(fmt);
+    const int64_t grid = S * parts;
     if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-    cudaError_t e = fmt == 1
-        ? launch_pdl(gemv_split_kernel<1>, (int)grid, s, x, packed, scales, y, partials, N, K, parts)
-        : launch_pdl(gemv_split_kernel<2>, (int)grid, s, x, packed, scales, y, partials, N, K, parts);
-    if (e != cudaSuccess || K / kSliceK == 1) return e;
+    cudaError_t e = fmt == 1   ? launch_pdl(gemv_split_kernel<1>, (int)grid, s, x, packed, scales, y, partials, N, K, parts)
+                    : fmt == 3 ? launch_pdl(gemv_split_kernel<3>, (int)grid, s, x, packed, scales, y, partials, N, K, parts)
+                               : launch_pdl(gemv_split_kernel<2>, (int)grid, s, x, packed, scales, y, partials, N, K, parts);
+    if (e != cudaSuccess || S == 1) return e;
     const int64_t rgrid64 = (N + 255) / 256;
     const int rgrid = (int)(rgrid64 < 4 * (int64_t)dev.sm_count ? rgrid64 : 4 * (int64_t)dev.sm_count);
-    return launch_pdl_cfg(gemv_reduce_kernel, rgrid, 256, 0, s, (const float *)partials, y, N, (int)(K / kSliceK));
+    return launch_pdl_cfg(gemv_reduce_kernel, rgrid, 256, 0, s, (const float *)partials, y, N, (int)S);
 }
 
 }  // namespace
 
 bool gemv_supported(int64_t M, int64_t N, int64_t K, int fmt) {
-    if (M != 1 || K % kSliceK != 0) return false;
+    if (M != 1 || (fmt != 1 && fmt != 2 && fmt != 3) || K % slice_k(fmt) != 0) return false;
     if ((N + kRows - 1) / kRows > kMaxTiles) return false;
-    (void)fmt;
     return true;
 }
 
 // Schedule: split_k 0 = automatic, 1 = rows mode (when the shape allows it), >= 2 = split mode.
 bool pick_rows_mode(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev) {
+    if (fmt == 3) return false;  // Q1_0: split mode only
     if (split_k == 1) return K <= kRowsModeMaxK && K / kSliceK >= 2;
     if (split_k >= 2) return false;
     return use_rows_mode(N, K, fmt, dev);
 }
 
 int gemv_launches(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev) {
-    if (pick_rows_mode(N, K, fmt, split_k, dev) || K / kSliceK <= 1) return 1;
+    if (pick_rows_mode(N, K, fmt, split_k, dev) || K / slice_k(fmt) <= 1) return 1;
     return 2;
 }
 
 size_t gemv_workspace_bytes(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev) {
-    const int64_t S = K / kSliceK;
+    const int64_t S = K / slice_k(fmt);
     if (S <= 1 || pick_rows_mode(N, K, fmt, split_k, dev)) return 0;
     return (size_t)S * (size_t)N * sizeof(float);
 }
@@ -549,7 +633,7 @@ cudaError_t launch_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t
 // shape; used by the no-allocation entry point.  partial_floats is the space the
 // scratch holds after its counters; returns cudaErrorInvalidValue if the shape needs more.
 size_t gemv_split_partial_floats(int64_t N, int64_t K) {
-    const int64_t S = K / kSliceK;
+    const int64_t S = K / kSliceK;  // PTQ1_0 / PQ2_0 (the no-allocation entry point's formats)
     return S > 1 ? (size_t)S * (size_t)N : 0;
 }
 

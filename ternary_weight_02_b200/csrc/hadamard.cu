@@ -15,11 +15,12 @@
 namespace bonsai {
 namespace {
 
-// kPerm8 (FP16 output only): each 8 consecutive outputs are stored in the order
-// [0, 4, 1, 5, 2, 6, 3, 7].  The prefill GEMM expands its weights in the same order
-// within each 8 (a contraction does not depend on the order of its terms), which lets it
-// build two FP16 weights with one byte permute.
-template <bool kOutF32, bool kPerm8>
+// kPerm (FP16 output only): 0 natural order; 8: each 8 consecutive outputs in the order
+// [0, 4, 1, 5, 2, 6, 3, 7]; 16: each 16 in the order [0, 8, 1, 9, ..., 7, 15].  The
+// prefill GEMM expands its PQ2_0 (8) or Q1_0 (16) weights in the same order within each
+// block (a contraction does not depend on the order of its terms), which lets it build
+// two FP16 weights with one byte permute.
+template <bool kOutF32, int kPerm>
 __global__ void __launch_bounds__(256) hadamard128_kernel(const uint16_t *x, void *out,
                                                           int64_t nblocks) {
     const int lane = threadIdx.x & 31;
@@ -33,7 +34,26 @@ __global__ void __launch_bounds__(256) hadamard128_kernel(const uint16_t *x, voi
             float4 *o = reinterpret_cast<float4 *>(static_cast<float *>(out) + blk * kGroup) + lane;
             *o = make_float4(v[0], v[1], v[2], v[3]);
         } else {
-            if (kPerm8) {
+            if (kPerm == 16) {
+                // lanes 4b .. 4b+3 hold outputs 16b .. 16b+15; lane r of the four stores
+                // (e, e + 8, e + 1, e + 9) with e = 4 (r >> 1) + 2 (r & 1): elements e, e + 1
+                // of lane r >> 1 and of lane 2 + (r >> 1)
+                const int base = lane & ~3, r = lane & 3;
+                const int la = base + (r >> 1), lb = base + 2 + (r >> 1);
+                float a[4], b[4];
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    a[k] = __shfl_sync(0xffffffffu, v[k], la);
+                    b[k] = __shfl_sync(0xffffffffu, v[k], lb);
+                }
+                const bool odd = r & 1;
+                float o[4];
+                o[0] = odd ? a[2] : a[0];
+                o[1] = odd ? b[2] : b[0];
+                o[2] = odd ? a[3] : a[1];
+                o[3] = odd ? b[3] : b[1];
+                store_half4(static_cast<uint16_t *>(out) + blk * kGroup + 4 * lane, o);
+            } else if (kPerm == 8) {
                 // lanes 2b, 2b + 1 hold outputs 8b .. 8b + 7; the even lane stores
                 // (0, 4, 1, 5), the odd one (2, 6, 3, 7)
                 const bool odd = lane & 1;
@@ -53,7 +73,7 @@ __global__ void __launch_bounds__(256) hadamard128_kernel(const uint16_t *x, voi
     }
 }
 
-template <bool kOutF32, bool kPerm8 = false>
+template <bool kOutF32, int kPerm = 0>
 cudaError_t launch(const uint16_t *x, void *out, int64_t M, int64_t K, cudaStream_t s,
                    const DeviceInfo &dev) {
     const int64_t nblocks = M * (K / kGroup);
@@ -61,7 +81,7 @@ cudaError_t launch(const uint16_t *x, void *out, int64_t M, int64_t K, cudaStrea
     const int64_t want = (nblocks + 7) / 8;  // 8 warps per CTA
     const int64_t cap = (int64_t)dev.sm_count * 8;
     const int grid = (int)(want < cap ? want : cap);
-    hadamard128_kernel<kOutF32, kPerm8><<<grid, 256, 0, s>>>(x, out, nblocks);
+    hadamard128_kernel<kOutF32, kPerm><<<grid, 256, 0, s>>>(x, out, nblocks);
     return cudaGetLastError();
 }
 
@@ -74,7 +94,12 @@ cudaError_t launch_hadamard_f16(const uint16_t *x, uint16_t *out, int64_t M, int
 
 cudaError_t launch_hadamard_f16_perm8(const uint16_t *x, uint16_t *out, int64_t M, int64_t K,
                                       cudaStream_t s, const DeviceInfo &dev) {
-    return launch<false, true>(x, out, M, K, s, dev);
+    return launch<false, 8>(x, out, M, K, s, dev);
+}
+
+cudaError_t launch_hadamard_f16_perm16(const uint16_t *x, uint16_t *out, int64_t M, int64_t K,
+                                       cudaStream_t s, const DeviceInfo &dev) {
+    return launch<false, 16>(x, out, M, K, s, dev);
 }
 
 cudaError_t launch_hadamard_f32(const uint16_t *x, float *out, int64_t M, int64_t K,

@@ -36,6 +36,8 @@ cudaError_t launch_pack_ptq1(const int8_t *trits, uint8_t *packed, int64_t N, in
                              cudaStream_t s, const DeviceInfo &dev);
 cudaError_t launch_pack_pq2(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K,
                             cudaStream_t s, const DeviceInfo &dev);
+cudaError_t launch_pack_q1(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K,
+                           cudaStream_t s, const DeviceInfo &dev);
 cudaError_t launch_unpack(int fmt, const uint8_t *packed, int8_t *trits, int64_t N, int64_t K,
                           cudaStream_t s, const DeviceInfo &dev);
 
@@ -48,6 +50,9 @@ cudaError_t launch_hadamard_f32(const uint16_t *x, float *out, int64_t M, int64_
 // (the K order of the prefill GEMM's expanded weight tiles).
 cudaError_t launch_hadamard_f16_perm8(const uint16_t *x, uint16_t *out, int64_t M, int64_t K,
                                       cudaStream_t s, const DeviceInfo &dev);
+// The same, each 16 outputs in the order [0, 8, 1, 9, ..., 7, 15] (Q1_0 tiles).
+cudaError_t launch_hadamard_f16_perm16(const uint16_t *x, uint16_t *out, int64_t M, int64_t K,
+                                       cudaStream_t s, const DeviceInfo &dev);
 
 // ---- linear_simple.cu: x' (FP32, M x K) in the workspace, then one warp per row
 size_t simple_workspace_bytes(int64_t M, int64_t N, int64_t K);

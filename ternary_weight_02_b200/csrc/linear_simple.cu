@@ -1,4 +1,4 @@
-// linear_simple.cu -- the plain CUDA ternary linear layer (any M, both packings).
+// linear_simple.cu -- the plain CUDA ternary linear layer (any M, every packing).
 //
 // y[m][n] = sum_g s[n][g] * sum_j t[n][128g+j] * x'[m][128g+j], x' the block
 // Hadamard rotation of x.  Source: "27B 模型压到 5.95GB，推理能力还保住 98%"
@@ -40,6 +40,9 @@ __global__ void __launch_bounds__(256) linear_simple_kernel(
                     int v = packed[(n * G + g) * kPtq1GroupBytes + j / 5];
                     for (int d = 0; d < j % 5; d++) v /= 3;
                     t = v % 3 - 1;
+                } else if (kFmt == 3) {
+                    const int v = packed[n * (K / 8) + g * kQ1GroupBytes + j / 8];
+                    t = ((v >> (j % 8)) & 1) ? 1 : -1;
                 } else {
                     const int v = packed[n * (K / 4) + g * kPq2GroupBytes + j / 4];
                     t = ((v >> (2 * (j % 4))) & 3) - 1;
@@ -76,6 +79,8 @@ cudaError_t launch_linear_simple(const uint16_t *x, const uint8_t *packed, const
     const int grid = (int)(want < cap ? want : cap);
     if (fmt == 1)
         linear_simple_kernel<1><<<grid, 256, 0, s>>>(xr, packed, scales, y, M, N, K);
+    else if (fmt == 3)
+        linear_simple_kernel<3><<<grid, 256, 0, s>>>(xr, packed, scales, y, M, N, K);
     else
         linear_simple_kernel<2><<<grid, 256, 0, s>>>(xr, packed, scales, y, M, N, K);
     return cudaGetLastError();

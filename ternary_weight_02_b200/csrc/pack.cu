@@ -52,6 +52,33 @@ __global__ void pack_pq2_kernel(const int8_t *__restrict__ trits, uint8_t *__res
     }
 }
 
+__global__ void pack_q1_kernel(const int8_t *__restrict__ trits, uint8_t *__restrict__ packed,
+                               int64_t total) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        // byte i of the plane holds weights 8i .. 8i+7, bit j = (weight 8i+j == +1)
+        const int2 t8 = *reinterpret_cast<const int2 *>(trits + 8 * i);
+        int value = 0;
+        for (int j = 0; j < 8; j++) {
+            const int t = (int8_t)(((j < 4 ? t8.x : t8.y) >> (8 * (j & 3))) & 0xFF);
+            value |= (t == 1 ? 1 : 0) << j;
+        }
+        packed[i] = (uint8_t)value;
+    }
+}
+
+__global__ void unpack_q1_kernel(const uint8_t *__restrict__ packed, int8_t *__restrict__ trits,
+                                 int64_t total) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int v = packed[i];
+        int8_t out[8];
+        for (int j = 0; j < 8; j++) out[j] = ((v >> j) & 1) ? (int8_t)1 : (int8_t)-1;
+        *reinterpret_cast<char4 *>(trits + 8 * i) = make_char4(out[0], out[1], out[2], out[3]);
+        *reinterpret_cast<char4 *>(trits + 8 * i + 4) = make_char4(out[4], out[5], out[6], out[7]);
+    }
+}
+
 __global__ void unpack_ptq1_kernel(const uint8_t *__restrict__ packed, int8_t *__restrict__ trits,
                                    int64_t total, int64_t K) {
     const int64_t G = K / kGroup;
@@ -109,9 +136,21 @@ cudaError_t launch_pack_pq2(const int8_t *trits, uint8_t *packed, int64_t N, int
     return cudaGetLastError();
 }
 
+cudaError_t launch_pack_q1(const int8_t *trits, uint8_t *packed, int64_t N, int64_t K,
+                           cudaStream_t s, const DeviceInfo &dev) {
+    const int64_t total = N * (K / 8);
+    if (total == 0) return cudaSuccess;
+    pack_q1_kernel<<<grid_for(total, 256, dev), 256, 0, s>>>(trits, packed, total);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_unpack(int fmt, const uint8_t *packed, int8_t *trits, int64_t N, int64_t K,
                           cudaStream_t s, const DeviceInfo &dev) {
-    if (fmt == 1) {
+    if (fmt == 3) {
+        const int64_t total = N * (K / 8);
+        if (total == 0) return cudaSuccess;
+        unpack_q1_kernel<<<grid_for(total, 256, dev), 256, 0, s>>>(packed, trits, total);
+    } else if (fmt == 1) {
         const int64_t total = N * (K / kGroup) * kPtq1GroupBytes;
         if (total == 0) return cudaSuccess;
         unpack_ptq1_kernel<<<grid_for(total, 256, dev), 256, 0, s>>>(packed, trits, total, K);

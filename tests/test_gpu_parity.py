@@ -11,7 +11,7 @@ from tests.gpu_util import Problem, to_numpy_f16
 
 pytestmark = pytest.mark.gpu
 
-PTQ1, PQ2 = oracle.FMT_PTQ1_0, oracle.FMT_PQ2_0
+PTQ1, PQ2, Q1 = oracle.FMT_PTQ1_0, oracle.FMT_PQ2_0, oracle.FMT_Q1_0
 
 
 @pytest.fixture(scope="module")
@@ -25,7 +25,7 @@ def bz():
 
 # ------------------------------------------------------------ codec
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
 @pytest.mark.parametrize("N,K", [(1, 128), (3, 384), (37, 1024), (64, 5120), (5, 17408)])
 def test_pack_bit_exact(bz, fmt, N, K):
     import torch
@@ -68,6 +68,24 @@ def test_pack_marks_invalid_trits(bz, fmt):
     assert oracle.check(fmt, got, 2, 256) == 2
 
 
+def test_q1_unpack_every_byte_and_pack_non_binary(bz):
+    import torch
+    N, K = 2, 2048  # 512 bytes: every byte value twice
+    packed = np.tile(np.arange(256, dtype=np.uint8), 2).reshape(N, K // 8)
+    want, bad = oracle.unpack(Q1, packed, N, K)
+    assert bad == 0
+    t = torch.empty((N, K), dtype=torch.int8, device="cuda")
+    bz.bonsai_unpack(Q1, torch.from_numpy(packed).cuda(), t, N, K)
+    torch.cuda.synchronize()
+    assert np.array_equal(t.cpu().numpy(), want)
+    # weights other than +-1 are stored as -1, as the checker's packer does
+    w = np.ones((2, 256), dtype=np.int8)
+    w[0, 5] = 0
+    w[1, 200] = 3
+    got = bz.pack(Q1, torch.from_numpy(w).cuda()).cpu().numpy()
+    assert np.array_equal(got.reshape(-1), oracle.pack(Q1, w).reshape(-1))
+
+
 # ------------------------------------------------------------ Hadamard
 
 @pytest.mark.parametrize("M,K", [(1, 128), (3, 1024), (17, 5120), (2, 17408)])
@@ -107,7 +125,7 @@ def _run(bz, p, algo, split_k=0):
 SIMPLE_CASES = [(1, 1, 128), (1, 33, 384), (3, 100, 1024), (17, 65, 640), (1, 1024, 1024)]
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
 @pytest.mark.parametrize("M,N,K", SIMPLE_CASES)
 def test_linear_simple(bz, fmt, M, N, K):
     p = Problem(M, N, K, fmt, seed=M * 7 + N)
@@ -116,7 +134,7 @@ def test_linear_simple(bz, fmt, M, N, K):
     assert ok, (rel, mx)
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
 def test_linear_auto_config1(bz, fmt):
     """Single ternary linear, M=1, K=1024 -> N=1024, seed 0, through the default entry point."""
     import torch
@@ -162,11 +180,33 @@ def test_gemv_small(bz, fmt, N, K):
     assert ok, (rel, mx)
 
 
+# Q1_0 (1-bit): a byte covers 8 activations, so the lookup-table GEMV's K slice is 1024
+Q1_GEMV_CASES = [(1, 1024), (33, 1024), (100, 3072), (1000, 2048), (37, 17408)]
+
+
+@pytest.mark.parametrize("N,K", Q1_GEMV_CASES)
+def test_gemv_small_q1(bz, N, K):
+    p = Problem(1, N, K, Q1, seed=N + 5 * K)
+    got = _run(bz, p, bz.BONSAI_ALGO_GEMV)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+def test_q1_k_not_multiple_of_1024(bz):
+    """The lookup-table GEMV refuses Q1_0 at K % 1024 != 0; the default entry point then
+    takes the plain kernel, still against the checker."""
+    p = Problem(1, 50, 640, Q1, seed=4)
+    with pytest.raises(bz.BonsaiError):
+        _run(bz, p, bz.BONSAI_ALGO_GEMV)
+    ok, rel, mx = oracle.compare(_run(bz, p, bz.BONSAI_ALGO_AUTO), p.oracle_y())
+    assert ok, (rel, mx)
+
+
 # 27B-class decode projections (K -> N): qkv, o, fused gate/up, down
 DECODE_SHAPES = [(5120, 7168), (5120, 5120), (5120, 34816), (17408, 5120)]
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
 @pytest.mark.parametrize("K,N", DECODE_SHAPES)
 def test_gemv_decode_shapes_full(bz, fmt, K, N):
     """Every output of the full-size M=1 projections against the float64 checker."""
@@ -174,7 +214,7 @@ def test_gemv_decode_shapes_full(bz, fmt, K, N):
     got = _run(bz, p, bz.BONSAI_ALGO_GEMV)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
-    if fmt == PTQ1:  # through the default entry point too (M == 1 PTQ1_0 dispatches here)
+    if fmt in (PTQ1, Q1):  # through the default entry point too (M == 1 PTQ1_0, Q1_0 dispatch here)
         import torch
         x, packed, scales = p.device()
         y = torch.empty((1, N), dtype=torch.float16, device="cuda")
@@ -183,7 +223,7 @@ def test_gemv_decode_shapes_full(bz, fmt, K, N):
         assert np.array_equal(to_numpy_f16(y), got)
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
 def test_gemv_repeatable_and_counters_reset(bz, fmt):
     """Split-K arrival counters return to zero: back-to-back calls on different shapes
     give bit-identical results (the slice-ordered reduction is deterministic)."""
@@ -313,7 +353,7 @@ GEMM_SMALL = [(1, 64, 128), (17, 256, 128), (130, 300, 384), (256, 512, 1024), (
               (600, 2000, 1152), (1000, 3000, 2048), (2000, 9500, 256)]
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
 @pytest.mark.parametrize("M,N,K", GEMM_SMALL)
 @pytest.mark.parametrize("tile", [1, 2])
 def test_gemm_small(bz, fmt, M, N, K, tile):
@@ -325,7 +365,7 @@ def test_gemm_small(bz, fmt, M, N, K, tile):
     assert ok, (rel, mx)
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
 def test_gemm_split_tiles_repeatable(bz, fmt):
     """Split tiles hand their partial sums over through flags that the owner clears:
     the same call twice, and after a differently split shape, gives the same bits."""
@@ -346,7 +386,7 @@ def _sampled_reference(fmt, M, N, K, seed, ms, ns):
     from ternary_weight_02_b200 import inputs
     um, un = np.unique(ms), np.unique(ns)
     x = inputs.normal_rows(seed, K, um)
-    t = inputs.trits_rows(seed, K, un)
+    t = inputs.signs_rows(seed, K, un) if fmt == Q1 else inputs.trits_rows(seed, K, un)
     s = inputs.scales_rows(seed, K // 128, un)
     y = oracle.ternary_linear(x, oracle.pack(fmt, t), s, len(un), K, fmt)
     return y, um, un
@@ -356,7 +396,7 @@ def _sampled_reference(fmt, M, N, K, seed, ms, ns):
 PREFILL = [(2048, 5120, 34816), (512, 17408, 5120), (8192, 5120, 7168)]
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
 @pytest.mark.parametrize("M,K,N", PREFILL)
 def test_gemm_prefill_full_size_sampled(bz, fmt, M, K, N):
     """Full-size GEMM on the device; 64 x 64 sampled outputs against the checker."""
@@ -364,7 +404,9 @@ def test_gemm_prefill_full_size_sampled(bz, fmt, M, K, N):
     from ternary_weight_02_b200 import inputs
     seed = 5
     dev = torch.device("cuda")
-    t = torch.from_numpy(inputs.trits(seed, N, K)).to(dev)
+    w = inputs.signs(seed, N, K) if fmt == Q1 else inputs.trits(seed, N, K)
+    t = torch.from_numpy(w).to(dev)
+    del w
     packed = bz.pack(fmt, t)
     del t
     s = torch.from_numpy(inputs.scales(seed, N, K).view(np.int16)).to(dev).view(torch.float16)
@@ -421,8 +463,9 @@ def test_skinny_split_is_deterministic(bz):
 
 
 @pytest.mark.parametrize("M", [2, 5, 16])
-def test_small_batches_ptq1_take_the_gemm(bz, M):
-    p = Problem(M, 300, 1024, PTQ1, seed=M)
+@pytest.mark.parametrize("fmt", [PTQ1, Q1])
+def test_small_batches_ptq1_take_the_gemm(bz, M, fmt):
+    p = Problem(M, 300, 1024, fmt, seed=M)
     got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
