@@ -40,11 +40,19 @@ sys.path.insert(0, ROOT)
 METRIC = "batch-1 ternary GEMV HBM GB/s (% of 8 TB/s); prefill GEMM TFLOPS (% peak)"
 SHAPES = [("qkv", 5120, 7168), ("o", 5120, 5120), ("gate_up", 5120, 34816), ("down", 17408, 5120)]
 LAYERS = 64
-FMT_NAMES = {1: "PTQ1_0", 2: "PQ2_0"}
+FMT_NAMES = {1: "PTQ1_0", 2: "PQ2_0", 3: "Q1_0"}
+FMTS = {"ptq1": 1, "pq2": 2, "q1": 3}
 # the kernel a batch-1 call runs for each packing, and its source file
 DOM_KERNEL = {1: "lookup-table GEMV (gemv_split_kernel + in-order reduction)",
-              2: "integer tensor-core GEMV (gemv_imma_kernel)"}
-DOM_SOURCE = {1: "gemv_lut.cu", 2: "gemv_imma.cu"}
+              2: "integer tensor-core GEMV (gemv_imma_kernel)",
+              3: "lookup-table GEMV (gemv_split_kernel, 1-bit tables + in-order reduction)"}
+DOM_SOURCE = {1: "gemv_lut.cu", 2: "gemv_imma.cu", 3: "gemv_lut.cu"}
+
+
+def weights(fmt, seed, N, K):
+    """Seeded weights of the workload: trits, or signs for the 1-bit Q1_0 packing."""
+    from ternary_weight_02_b200 import inputs
+    return inputs.signs(seed, N, K) if fmt == 3 else inputs.trits(seed, N, K)
 
 
 def measured_peaks():
@@ -57,7 +65,7 @@ def measured_peaks():
 
 
 def plane_bytes(fmt, N, K):
-    trit = N * (K // 128) * 26 if fmt == 1 else N * K // 4
+    trit = N * (K // 128) * 26 if fmt == 1 else (N * K // 8 if fmt == 3 else N * K // 4)
     return trit + N * (K // 128) * 2
 
 
@@ -163,10 +171,10 @@ def run_reference(args):
     (the four projections) of the stack at M = 1, a bounded sample of the workload."""
     import oracle
     from ternary_weight_02_b200 import inputs
-    fmt = {"ptq1": 1, "pq2": 2}[args.fmt]
+    fmt = FMTS[args.fmt]
     probs = []
     for i, (name, K, N) in enumerate(SHAPES):
-        t = inputs.trits(i, N, K)
+        t = weights(fmt, i, N, K)
         probs.append((inputs.activations(i, 1, K), oracle.pack(fmt, t), inputs.scales(i, N, K), N, K))
     threads = oracle.max_threads()
 
@@ -205,7 +213,7 @@ def build_stack(fmt, dev, bz, torch):
     stack = []
     xs, ys = [], []
     for i, (name, K, N) in enumerate(SHAPES):
-        t = torch.from_numpy(inputs.trits(i, N, K)).to(dev)
+        t = torch.from_numpy(weights(fmt, i, N, K)).to(dev)
         packed = bz.pack(fmt, t)
         del t
         s = torch.from_numpy(inputs.scales(i, N, K).view(np.int16)).to(dev).view(torch.float16)
@@ -230,11 +238,11 @@ def run_ours(args):
     if bz.bonsai_check_device() != bz.BONSAI_OK:
         raise RuntimeError("libbonsai: not an sm_100 device")
     peaks, peak_kind = measured_peaks()
-    fmt = {"ptq1": 1, "pq2": 2}[args.fmt]
+    fmt = FMTS[args.fmt]
     bz.bonsai_reserve(1, 34816, 17408)
 
     results = {}
-    for f in ([fmt] + [o for o in (2, 1) if o != fmt]) if args.both else [fmt]:
+    for f in ([fmt] + [o for o in (2, 1, 3) if o != fmt]) if args.both else [fmt]:
         stack, xs, ys = build_stack(f, dev, bz, torch)
         stream = torch.cuda.Stream(device=dev)
         sp = stream.cuda_stream
@@ -386,7 +394,7 @@ def run_prefill(fmt, M, dev, bz, torch, peaks, peak_kind, steps):
     stream = torch.cuda.Stream(device=dev)
     items = []
     for i, (name, K, N) in enumerate(SHAPES):
-        t = torch.from_numpy(inputs.trits(i, N, K)).to(dev)
+        t = torch.from_numpy(weights(fmt, i, N, K)).to(dev)
         packed = bz.pack(fmt, t)
         del t
         s = torch.from_numpy(inputs.scales(i, N, K).view(np.int16)).to(dev).view(torch.float16)
@@ -433,7 +441,7 @@ def cpu_baseline(fmt):
     from ternary_weight_02_b200 import inputs
     probs = []
     for i, (name, K, N) in enumerate(SHAPES):
-        probs.append((inputs.activations(i, 1, K), oracle.pack(fmt, inputs.trits(i, N, K)),
+        probs.append((inputs.activations(i, 1, K), oracle.pack(fmt, weights(fmt, i, N, K)),
                       inputs.scales(i, N, K), N, K))
     t0 = time.perf_counter()
     for x, p, s, N, K in probs:
@@ -449,12 +457,12 @@ def run_case(args):
     import torch
     from ternary_weight_02_b200 import bonsai as bz
     from ternary_weight_02_b200 import inputs
-    fmt = {"ptq1": 1, "pq2": 2}[args.fmt]
+    fmt = FMTS[args.fmt]
     i = [n for n, _, _ in SHAPES].index(args.shape)
     _, K, N = SHAPES[i]
     M = 1 if args.case in ("gemv", "imma") else args.m
     dev = torch.device("cuda")
-    t = torch.from_numpy(inputs.trits(i, N, K)).to(dev)
+    t = torch.from_numpy(weights(fmt, i, N, K)).to(dev)
     packed = bz.pack(fmt, t)
     del t
     s = torch.from_numpy(inputs.scales(i, N, K).view(np.int16)).to(dev).view(torch.float16)
@@ -480,7 +488,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--fmt", choices=["pq2", "ptq1"], default="pq2")
+    ap.add_argument("--fmt", choices=["pq2", "ptq1", "q1"], default="pq2")
     ap.add_argument("--both", type=int, default=1, help="also measure the other packing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-m", type=int, default=2048, help="tokens of the prefill GEMM line (0: skip)")
@@ -503,7 +511,7 @@ def main():
     line = run_ours(args)
     if rank == 0 and line is not None:
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline({"ptq1": 1, "pq2": 2}[args.fmt])
+            line["cpu_baseline"] = cpu_baseline(FMTS[args.fmt])
         print(json.dumps(line), flush=True)
 
 
