@@ -66,6 +66,8 @@ def lib():
         L.oracle_fwht_recursive.argtypes = [p, ll]
         L.oracle_ternary_linear.restype = ll
         L.oracle_ternary_linear.argtypes = [p, p, p, p, ll, ll, ll, i, i, i]
+        L.oracle_swiglu.restype = None
+        L.oracle_swiglu.argtypes = [p, p, ll, ll]
         L.oracle_max_threads.restype = i
         L.oracle_max_threads.argtypes = []
         _lib = L
@@ -152,6 +154,23 @@ def ternary_linear(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, N: int
     if bad < 0:
         raise ValueError("bad argument")
     return y
+
+
+def swiglu(y: np.ndarray) -> np.ndarray:
+    """h = silu(y[:, :F]) * y[:, F:] for an M x 2F float array (float64 result)."""
+    yd = np.ascontiguousarray(y, dtype=np.float64)
+    M, F2 = yd.shape
+    if F2 % 2:
+        raise ValueError("the fused gate/up output has an even number of columns")
+    h = np.zeros((M, F2 // 2), dtype=np.float64)
+    lib().oracle_swiglu(_ptr(yd), _ptr(h), M, F2 // 2)
+    return h
+
+
+def swiglu_linear(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, F: int, K: int, fmt: int,
+                  nthreads: int = 0) -> np.ndarray:
+    """The fused gate/up layer (2F weight rows: gate, then up) followed by SwiGLU: M x F."""
+    return swiglu(ternary_linear(x, packed, scales, 2 * F, K, fmt, nthreads=nthreads))
 
 
 def max_threads() -> int:

@@ -33,6 +33,7 @@
  *      one FP16 scale per 128 weights.  Source: allhereai.com page, the
  *      paragraph describing the method (ternary weights, one FP16 scale shared
  *      by every 128 weights).
+ *   4. the SwiGLU step after a fused gate/up product, h = silu(gate) * up.
  *
  * Readings where the pages are silent (block size of the rotation, Sylvester
  * order and 1/sqrt(128) normalisation, base-3 digit order least significant
@@ -366,6 +367,22 @@ long long oracle_ternary_linear(const double *x, const uint8_t *packed, const do
     }
     free(xr);
     return bad;
+}
+
+/* ------------------------------------------------------------------ SwiGLU */
+
+/* The MLP step that follows the fused gate/up projection: with y the M x 2F output of
+ * one linear layer whose rows 0 .. F-1 are the gate projection and F .. 2F-1 the up
+ * projection, h[m][f] = silu(y[m][f]) * y[m][F + f], silu(z) = z / (1 + e^-z).  Written
+ * out in float64.  Source of the fused gate/up projection (N = 2 x 17408): the 27B-class
+ * shapes this layer is built for (d = 5120, ffn = 17408). */
+void oracle_swiglu(const double *y, double *h, long long M, long long F)
+{
+    for (long long m = 0; m < M; m++)
+        for (long long f = 0; f < F; f++) {
+            double g = y[m * 2 * F + f], u = y[m * 2 * F + F + f];
+            h[m * F + f] = g / (1.0 + exp(-g)) * u;
+        }
 }
 
 /* Threads an OpenMP region would use by default (1 without OpenMP). */

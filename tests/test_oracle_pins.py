@@ -380,6 +380,50 @@ def test_signs_generator():
     assert np.array_equal(inputs.signs_rows(1, 1024, [5, 63]), t[[5, 63]])
 
 
+# ---------------------------------------------------------------- SwiGLU
+
+def test_swiglu_closed_forms():
+    z = np.array([[0.0, 1.0, -1.0, 40.0, -40.0, 2.0,  # gate
+                   3.0, 1.0, 2.0, 0.5, 7.0, -1.0]])   # up
+    h = oracle.swiglu(z)[0]
+    e1 = np.exp(-1.0)
+    assert h[0] == 0.0
+    assert h[1] == 1.0 / (1.0 + e1) * 1.0           # silu(1) = sigma(1)
+    assert np.isclose(h[2], -1.0 * (1.0 - 1.0 / (1.0 + e1)) * 2.0, rtol=1e-15)
+    assert np.isclose(h[3], 40.0 * 0.5, rtol=1e-15)  # sigma(40) = 1 to double precision
+    assert np.isclose(h[4], -280.0 * np.exp(-40.0), rtol=1e-14)  # sigma(-40) = e^-40 (1 - e^-40 ...)
+    assert np.isclose(h[5], 2.0 / (1.0 + np.exp(-2.0)) * -1.0, rtol=1e-15)
+
+
+def test_swiglu_odd_identity_and_layout():
+    # silu(z) - silu(-z) = z for every z; gate is the first half of the columns
+    rng = np.random.default_rng(0)
+    g = rng.normal(0, 3, (3, 50))
+    ones = np.ones_like(g)
+    hp = oracle.swiglu(np.concatenate([g, ones], axis=1))
+    hm = oracle.swiglu(np.concatenate([-g, ones], axis=1))
+    assert np.allclose(hp - hm, g, rtol=0, atol=1e-13)
+    # swapping the halves changes the result (the layout is pinned, not symmetric)
+    u = rng.normal(0, 3, (3, 50))
+    assert not np.allclose(oracle.swiglu(np.concatenate([g, u], 1)), oracle.swiglu(np.concatenate([u, g], 1)))
+
+
+@pytest.mark.parametrize("fmt", [PQ2, PTQ1])
+def test_swiglu_linear_brute_force(fmt):
+    F, K, M = 6, 256, 3
+    t = _weights(fmt, 9, 2 * F, K)
+    s = inputs.scales(9, 2 * F, K)
+    x = inputs.activations(9, M, K)
+    h = oracle.swiglu_linear(x, oracle.pack(fmt, t), s, F, K, fmt)
+    H = oracle.sylvester128()
+    xr = (x.astype(np.float64).reshape(M, K // 128, 128) @ H.T).reshape(M, K)
+    y = xr @ _dense(t, s).T
+    gate, up = y[:, :F], y[:, F:]
+    want = gate * (1.0 / (1.0 + np.exp(-gate))) * up
+    assert h.shape == (M, F)
+    assert np.allclose(h, want, rtol=1e-12, atol=1e-13)
+
+
 def test_linear_formats_agree_and_threads_agree():
     N, K, M = 33, 640, 2
     t = inputs.trits(5, N, K)
