@@ -165,6 +165,23 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
                                uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int algo,
                                int split_k, void *stream);
 
+/* The SwiGLU step of the MLP after a fused gate/up projection: for y, the M x 2F FP16
+ * output of a linear layer whose weight rows 0 .. F-1 are the gate projection and
+ * F .. 2F-1 the up projection, h[m][f] = silu(y[m][f]) * y[m][F + f] with
+ * silu(z) = z / (1 + e^-z), computed in FP32 and rounded to FP16 (nearest even).  h is
+ * M x F; y and h must not overlap.  Source of the fused gate/up projection: the
+ * 27B-class layer shapes (d = 5120, ffn = 17408, gate/up N = 34816). */
+int bonsai_swiglu(const uint16_t *y, uint16_t *h, int64_t M, int64_t F, void *stream);
+
+/* The fused gate/up linear layer followed by SwiGLU: packed and scales hold 2F weight rows
+ * (gate rows first, then up rows: the N = 2F plane of bonsai_ternary_linear) and h gets
+ * the M x F result of bonsai_swiglu applied to their product with x'.  On the integer
+ * tensor-core GEMV (M = 1 PQ2_0) and the prefill GEMM the step runs in the kernel's
+ * epilogue on the FP32 sums; the lookup-table GEMV, the skinny and the plain kernel write
+ * the product to the library's workspace in FP16 and bonsai_swiglu follows. */
+int bonsai_ternary_linear_swiglu(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                                 uint16_t *h, int64_t M, int64_t F, int64_t K, int fmt, void *stream);
+
 /* Number of kernels one bonsai_ternary_linear_algo call with these arguments launches
  * on the current device (the lookup-table GEMV: 1, or 2 when its split-K partials are
  * summed by a second kernel; the integer tensor-core GEMV: 1; the other kernels: 2,

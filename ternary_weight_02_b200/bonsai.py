@@ -62,6 +62,8 @@ _SIGS = {
     "bonsai_ternary_linear_algo": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _int, _int, _p]),
     "bonsai_ternary_linear_noalloc": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _p]),
     "bonsai_launch_count": (_int, [_i64, _i64, _i64, _int, _int, _int]),
+    "bonsai_swiglu": (_int, [_p, _p, _i64, _i64, _p]),
+    "bonsai_ternary_linear_swiglu": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _p]),
     "bonsai_reserve": (_int, [_i64, _i64, _i64]),
     "bonsai_shutdown": (None, []),
 }
@@ -185,6 +187,15 @@ def bonsai_shutdown() -> None:
 
 
 # ---------------------------------------------------------------- conveniences
+
+def bonsai_swiglu(y, h, M: int, F: int, stream=None) -> None:
+    _check(_lib.bonsai_swiglu(_ptr(y), _ptr(h), M, F, _stream(stream)), "bonsai_swiglu")
+
+
+def bonsai_ternary_linear_swiglu(x, packed, scales, h, M: int, F: int, K: int, fmt: int, stream=None) -> None:
+    _check(_lib.bonsai_ternary_linear_swiglu(_ptr(x), _ptr(packed), _ptr(scales), _ptr(h), M, F, K, fmt,
+                                             _stream(stream)), "bonsai_ternary_linear_swiglu")
+
 
 def pack(fmt: int, trits, stream=None):
     """Packs an N x K int8 CUDA tensor of trits; returns the uint8 plane (N x bytes/row)."""

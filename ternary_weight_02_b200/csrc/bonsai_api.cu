@@ -153,6 +153,19 @@ int resolve_algo(int algo, int64_t M, int64_t N, int64_t K, int fmt) {
     }
 }
 
+// Launches the chosen kernel (argument checks and the workspace are the caller's).
+cudaError_t run_linear(int chosen, const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
+                       int64_t M, int64_t N, int64_t K, int fmt, int split_k, const Workspace &ws, cudaStream_t s,
+                       const DeviceInfo &info) {
+    switch (chosen) {
+        case BONSAI_ALGO_GEMV: return launch_gemv(x, packed, scales, y, N, K, fmt, split_k, ws, s, info);
+        case BONSAI_ALGO_SKINNY: return launch_skinny(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, info);
+        case BONSAI_ALGO_GEMM: return launch_gemm(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, info);
+        case BONSAI_ALGO_IMMA: return launch_gemv_imma(x, packed, scales, y, N, K, ws, s, info);
+        default: return launch_linear_simple(x, packed, scales, y, M, N, K, fmt, ws, s, info);
+    }
+}
+
 size_t workspace_for(int algo, int64_t M, int64_t N, int64_t K, int fmt, int split_k,
                      const DeviceInfo &info) {
     switch (algo) {
@@ -304,32 +317,71 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
     rc = ensure_workspace(*st, workspace_for(chosen, M, N, K, fmt, split_k, st->info),
                           chosen == BONSAI_ALGO_IMMA ? gemv_imma_zeroed_bytes(N, K) : 0, &ws);
     if (rc != BONSAI_OK) return rc;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    switch (chosen) {
-        case BONSAI_ALGO_GEMV:
-            e = launch_gemv(x, packed, scales, y, N, K, fmt, split_k, ws, s, st->info);
-            break;
-        case BONSAI_ALGO_SKINNY:
-            e = launch_skinny(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, st->info);
-            break;
-        case BONSAI_ALGO_GEMM:
-            e = launch_gemm(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, st->info);
-            break;
-        case BONSAI_ALGO_IMMA:
-            e = launch_gemv_imma(x, packed, scales, y, N, K, ws, s, st->info);
-            break;
-        default:
-            e = launch_linear_simple(x, packed, scales, y, M, N, K, fmt, ws, s, st->info);
-            break;
-    }
-    return cuda_status(e);
+    return cuda_status(run_linear(chosen, x, packed, scales, y, M, N, K, fmt, split_k, ws,
+                                  static_cast<cudaStream_t>(stream), st->info));
 }
 
 int bonsai_ternary_linear(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                           uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, void *stream) {
     return bonsai_ternary_linear_algo(x, packed, scales, y, M, N, K, fmt, BONSAI_ALGO_AUTO, 0,
                                       stream);
+}
+
+int bonsai_swiglu(const uint16_t *y, uint16_t *h, int64_t M, int64_t F, void *stream) {
+    if (M < 0 || F < 0 || M > kMaxDim || F > kMaxDim) return BONSAI_ERR_SHAPE;
+    if (M == 0 || F == 0) return BONSAI_OK;
+    if (!y || !h) return BONSAI_ERR_NULL;
+    if (!aligned16(y) || !aligned16(h)) return BONSAI_ERR_ALIGN;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int dev;
+    DeviceState *st;
+    const int rc = probe_current(&dev, &st);
+    if (rc != BONSAI_OK) return rc;
+    return cuda_status(launch_swiglu(y, h, M, F, static_cast<cudaStream_t>(stream), st->info));
+}
+
+int bonsai_ternary_linear_swiglu(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                                 uint16_t *h, int64_t M, int64_t F, int64_t K, int fmt, void *stream) {
+    int rc = check_fmt(fmt);
+    if (rc != BONSAI_OK) return rc;
+    if (F < 0 || F > kMaxDim / 2) return BONSAI_ERR_SHAPE;
+    const int64_t N = 2 * F;
+    rc = check_shape(M, N, K);
+    if (rc != BONSAI_OK) return rc;
+    if (M == 0 || F == 0) return BONSAI_OK;
+    if (!x || !packed || !scales || !h) return BONSAI_ERR_NULL;
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(h))
+        return BONSAI_ERR_ALIGN;
+    const int chosen = resolve_algo(BONSAI_ALGO_AUTO, M, N, K, fmt);
+    if (chosen < 0) return chosen;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int dev;
+    DeviceState *st;
+    rc = probe_current(&dev, &st);
+    if (rc != BONSAI_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Workspace ws;
+    if (chosen == BONSAI_ALGO_IMMA) {  // fused into the GEMV's epilogue
+        rc = ensure_workspace(*st, 0, gemv_imma_zeroed_bytes(N, K), &ws);
+        if (rc != BONSAI_OK) return rc;
+        return cuda_status(launch_gemv_imma(x, packed, scales, h, N, K, ws, s, st->info, F));
+    }
+    if (chosen == BONSAI_ALGO_GEMM) {  // fused into the GEMM's epilogue
+        rc = ensure_workspace(*st, workspace_for(chosen, M, N, K, fmt, 0, st->info), 0, &ws);
+        if (rc != BONSAI_OK) return rc;
+        return cuda_status(launch_gemm(x, packed, scales, h, M, N, K, fmt, 0, ws, s, st->info, F));
+    }
+    // otherwise: the linear layer into the tail of the workspace, then the SwiGLU kernel
+    const size_t need = (workspace_for(chosen, M, N, K, fmt, 0, st->info) + 255) / 256 * 256;
+    rc = ensure_workspace(*st, need + (size_t)M * (size_t)N * 2,
+                          chosen == BONSAI_ALGO_IMMA ? gemv_imma_zeroed_bytes(N, K) : 0, &ws);
+    if (rc != BONSAI_OK) return rc;
+    uint16_t *y = reinterpret_cast<uint16_t *>(ws.data + need);
+    Workspace inner = ws;
+    inner.data_bytes = need;
+    cudaError_t e = run_linear(chosen, x, packed, scales, y, M, N, K, fmt, 0, inner, s, st->info);
+    if (e == cudaSuccess) e = launch_swiglu(y, h, M, F, s, st->info);
+    return cuda_status(e);
 }
 
 int bonsai_launch_count(int64_t M, int64_t N, int64_t K, int fmt, int algo, int split_k) {
@@ -381,6 +433,8 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
         }
     }
     Workspace ws;
+    // + the tail in which a non-fused bonsai_ternary_linear_swiglu keeps its M x N output
+    need = (need + 255) / 256 * 256 + (size_t)M * (size_t)N * 2;
     return ensure_workspace(*st, need, zneed, &ws);
 }
 

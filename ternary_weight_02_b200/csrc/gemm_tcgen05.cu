@@ -97,6 +97,20 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                  : "memory");
 }
 
+// 32 columns of this warp's 32 TMEM lanes, the wait in the same statement.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
 // 64 columns of this warp's 32 TMEM lanes (lane i of the warp: TMEM lane 32q + i) in one
 // load; the wait is in the same statement, so no use of r can be scheduled before it.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
@@ -267,12 +281,18 @@ __device__ __forceinline__ void expand_warps_sync() { asm volatile("bar.sync 1, 
 // A continuing piece comes before anything else of its CTA's split share, and the owner's
 // piece last: the waits are short, and they only go from a CTA to later ones, which never
 // wait before they have stored (all CTAs of the grid are resident at once, one per SM).
-template <int kFmt, int kAcc>
+//
+// kSwiglu: the weight rows are a fused gate/up projection (gate rows 0 .. F-1, up rows
+// F .. 2F-1, N = 2F) and the output is h = silu(gate) * up, M x F.  A tile's
+// 256 weight rows are then gate rows 128 tn .. 128 tn + 127 followed by the matching up
+// rows, so that each epilogue warp finds gate column c and up column 128 + c of the same
+// output in its own accumulator lanes.
+template <int kFmt, int kAcc, bool kSwiglu>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap w_map,
     const uint8_t *__restrict__ packed,
     const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
-    unsigned int *__restrict__ flags, int M, int N, int K, int mt) {
+    unsigned int *__restrict__ flags, int M, int N, int K, int mt, int F) {
     using C = Cfg<kAcc>;
     constexpr int STAGES = C::kStages;
     constexpr int kSlotFloats = C::kTileM * BN;
@@ -378,9 +398,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                         tma_load_2d(sA + st * C::kAStage + a * (BM * BK * 2), &a_map, full_a + st, ks * BK,
                                     tm * C::kTileM + a * BM);
                     // PQ2_0: the stage's codes, 16 bytes of each of the tile's 256 weight rows
-                    if (kFmt == 2)
+                    if (kFmt == 2 && !kSwiglu)
                         tma_load_2d(const_cast<uint8_t *>(sCodes) + st * CODE_STAGE_BYTES, &w_map, full_a + st,
                                     ks * (BK / 4), tn * BN);
+                    if (kFmt == 2 && kSwiglu) {  // 128 gate rows, then the matching 128 up rows
+                        tma_load_2d(const_cast<uint8_t *>(sCodes) + st * CODE_STAGE_BYTES, &w_map, full_a + st,
+                                    ks * (BK / 4), tn * (BN / 2));
+                        tma_load_2d(const_cast<uint8_t *>(sCodes) + st * CODE_STAGE_BYTES + CODE_STAGE_BYTES / 2,
+                                    &w_map, full_a + st, ks * (BK / 4), F + tn * (BN / 2));
+                    }
                 }
                 v += p.ke - p.kb;
             }
@@ -440,8 +466,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
             const Piece p = piece_at(v);
             v += p.ke - p.kb;
             const int tm = p.s % mt, tn = p.s / mt;
-            const int64_t n = (int64_t)tn * BN + r;  // weight row
-            const bool valid = n < N;
+            const int64_t n = kSwiglu ? (r < BN / 2 ? (int64_t)tn * (BN / 2) + r : (int64_t)F + tn * (BN / 2) + r - BN / 2)
+                                      : (int64_t)tn * BN + r;  // weight row
+            // (SwiGLU: the last tile's gate rows past F belong to no output; their weights read as 0)
+            const bool valid = kSwiglu ? (int64_t)tn * (BN / 2) + (r & (BN / 2 - 1)) < F : n < N;
             if (live) {
                 // PTQ1_0, Q1_0: the packed bytes of the group being expanded and of the next one (in
                 // flight) come by plain loads; PQ2_0: the codes come with the stage's x' tiles
@@ -532,10 +560,105 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
             if (owner)
                 for (int c2 = cta + 1, s = u_end; s < tile_end; s = range_end(c2), c2++)
                     got = flag_wait(flags + c2) && got;
+            const int w8 = warp - 2;
+            if constexpr (kSwiglu) {
+                // h columns [64 half, +64) of the tile's 128: gate accumulator columns
+                // 64 half + 32 cc and up columns 128 + 64 half + 32 cc.  Hand-over slots are
+                // in the order (accumulator a, TMEM quadrant q, 32-column chunk of 256, float4 i,
+                // lane): writer and owner use the same mapping.
+                auto sw_slot = [&](int c2, int a, int ch) {
+                    return reinterpret_cast<float4 *>(partials + (size_t)c2 * kSlotFloats) +
+                           ((size_t)((a * 4 + q) * 8 + ch) * 8) * 32 + lane;
+                };
+                uint8_t *stage_h = sB + w8 * 4096;  // 32 rows x 64 FP16, 16-byte chunks swizzled by the row
+#pragma unroll 1
+                for (int a = 0; a < kAcc; a++) {
+#pragma unroll 1
+                    for (int cc = 0; cc < 2; cc++) {
+                        const int cg = 2 * half + cc, cu = 4 + cg;  // 32-column chunks of the 256
+                        uint32_t vg[32], vu[32];
+                        __syncwarp();
+                        if (ok) {
+                            tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 256 + 32 * cg), vg);
+                            tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 256 + 32 * cu), vu);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; i++) vg[i] = vu[i] = 0x7fc00000u;
+                        }
+                        if (continues) {
+                            float4 *dg = sw_slot(cta, a, cg), *du = sw_slot(cta, a, cu);
+#pragma unroll
+                            for (int i = 0; i < 8; i++) {
+                                dg[32 * i] = make_float4(__uint_as_float(vg[4 * i]), __uint_as_float(vg[4 * i + 1]),
+                                                         __uint_as_float(vg[4 * i + 2]), __uint_as_float(vg[4 * i + 3]));
+                                du[32 * i] = make_float4(__uint_as_float(vu[4 * i]), __uint_as_float(vu[4 * i + 1]),
+                                                         __uint_as_float(vu[4 * i + 2]), __uint_as_float(vu[4 * i + 3]));
+                            }
+                            continue;
+                        }
+                        if (owner) {
+                            for (int c2 = cta + 1, s = u_end; s < tile_end; s = range_end(c2), c2++) {
+                                const float4 *sg = sw_slot(c2, a, cg), *su = sw_slot(c2, a, cu);
+#pragma unroll
+                                for (int i = 0; i < 8; i++) {
+                                    const float4 wg = __ldcg(sg + 32 * i), wu = __ldcg(su + 32 * i);
+                                    vg[4 * i] = __float_as_uint(__uint_as_float(vg[4 * i]) + wg.x);
+                                    vg[4 * i + 1] = __float_as_uint(__uint_as_float(vg[4 * i + 1]) + wg.y);
+                                    vg[4 * i + 2] = __float_as_uint(__uint_as_float(vg[4 * i + 2]) + wg.z);
+                                    vg[4 * i + 3] = __float_as_uint(__uint_as_float(vg[4 * i + 3]) + wg.w);
+                                    vu[4 * i] = __float_as_uint(__uint_as_float(vu[4 * i]) + wu.x);
+                                    vu[4 * i + 1] = __float_as_uint(__uint_as_float(vu[4 * i + 1]) + wu.y);
+                                    vu[4 * i + 2] = __float_as_uint(__uint_as_float(vu[4 * i + 2]) + wu.z);
+                                    vu[4 * i + 3] = __float_as_uint(__uint_as_float(vu[4 * i + 3]) + wu.w);
+                                }
+                            }
+                            if (!got)
+#pragma unroll
+                                for (int i = 0; i < 32; i++) vg[i] = 0x7fc00000u;
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            uint32_t hw[4];
+#pragma unroll
+                            for (int e = 0; e < 4; e++) {
+                                float hv[2];
+#pragma unroll
+                                for (int k2 = 0; k2 < 2; k2++) {
+                                    const float g = __uint_as_float(vg[8 * j + 2 * e + k2]);
+                                    hv[k2] = g / (1.f + expf(-g)) * __uint_as_float(vu[8 * j + 2 * e + k2]);
+                                }
+                                const __half2 p2 = __floats2half2_rn(hv[0], hv[1]);
+                                hw[e] = *reinterpret_cast<const uint32_t *>(&p2);
+                            }
+                            *reinterpret_cast<uint4 *>(stage_h + lane * 128 + (((4 * cc + j) ^ (lane & 7)) << 4)) =
+                                make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                        }
+                    }
+                    if (continues) continue;
+                    __syncwarp();
+                    // four rows of 128 bytes per instruction: lane (row within four, 16-byte chunk)
+                    const int ch = lane & 7;
+                    const int64_t f0 = (int64_t)tn * (BN / 2) + half * 64 + ch * 8;
+#pragma unroll 4
+                    for (int i = 0; i < 8; i++) {
+                        const int row = 4 * i + (lane >> 3);
+                        const int m = tm * C::kTileM + a * BM + 32 * q + row;
+                        const uint4 val = *reinterpret_cast<const uint4 *>(stage_h + row * 128 + ((ch ^ (row & 7)) << 4));
+                        if (m >= M || f0 >= F) continue;
+                        uint16_t *hr = y + (int64_t)m * F + f0;
+                        if (f0 + 8 <= F && (F & 7) == 0) {
+                            *reinterpret_cast<uint4 *>(hr) = val;
+                        } else {
+                            const uint32_t wv[4] = {val.x, val.y, val.z, val.w};
+                            for (int e = 0; e < 8 && f0 + e < F; e++) hr[e] = (uint16_t)(wv[e >> 1] >> (16 * (e & 1)));
+                        }
+                    }
+                    __syncwarp();
+                }
+            } else {
             // Hand-over slots are kept in the order of the accumulator fragments (accumulator a,
             // warp, 32-column chunk c, float4 i, lane), so that writer and owner, which use the
             // same thread mapping, both move 512 contiguous bytes per warp instruction.
-            const int w8 = warp - 2;
             auto slot_at = [&](int c2, int a, int c) {
                 return reinterpret_cast<float4 *>(partials + (size_t)c2 * kSlotFloats) +
                        ((size_t)((a * kExpandWarps + w8) * 4 + c) * 8) * 32 + lane;
@@ -621,6 +744,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                 }
                 __syncwarp();  // the staging rows are rewritten by the next accumulator
             }
+            }  // kSwiglu
             // tensor memory has been read: the next piece's MMAs may overwrite it
             tc_fence_before();
             __syncwarp();
@@ -698,7 +822,9 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, const Devi
 
 cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                         uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int tile_hint,
-                        const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
+                        const Workspace &ws, cudaStream_t s, const DeviceInfo &dev, int64_t swiglu_f) {
+    const bool swiglu = swiglu_f > 0;
+    if (swiglu && N != 2 * swiglu_f) return cudaErrorInvalidValue;
     const GemmPlan plan = gemm_plan(M, N, K, tile_hint, dev.sm_count);
     if (ws.data_bytes < gemm_workspace_bytes(M, N, K, fmt, dev) || plan.ctas > kMaxTiles) return cudaErrorInvalidValue;
     uint16_t *xr = reinterpret_cast<uint16_t *>(ws.data);
@@ -725,7 +851,7 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
     if (fmt == 2) {
         const cuuint64_t wdims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
         const cuuint64_t wstrides[1] = {(cuuint64_t)(K / 4)};
-        const cuuint32_t wbox[2] = {BK / 4, BN};
+        const cuuint32_t wbox[2] = {BK / 4, swiglu ? BN / 2 : BN};
         if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), wdims, wstrides, wbox,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -735,17 +861,18 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         kern<<<plan.ctas, kThreads, smem, s>>>(map, wmap, packed, scales, y, partials, ws.counters, (int)M, (int)N,
-                                               (int)K, plan.mt);
+                                               (int)K, plan.mt, (int)swiglu_f);
         return cudaGetLastError();
     };
-    if (fmt == 1)
-        return plan.acc == 2 ? go(gemm_tcgen05_kernel<1, 2>, Cfg<2>::kSmemBytes)
-                             : go(gemm_tcgen05_kernel<1, 1>, Cfg<1>::kSmemBytes);
-    if (fmt == 3)
-        return plan.acc == 2 ? go(gemm_tcgen05_kernel<3, 2>, Cfg<2>::kSmemBytes)
-                             : go(gemm_tcgen05_kernel<3, 1>, Cfg<1>::kSmemBytes);
-    return plan.acc == 2 ? go(gemm_tcgen05_kernel<2, 2>, Cfg<2>::kSmemBytes)
-                         : go(gemm_tcgen05_kernel<2, 1>, Cfg<1>::kSmemBytes);
+    auto pick = [&](auto k1, auto k2) { return plan.acc == 2 ? go(k2, Cfg<2>::kSmemBytes) : go(k1, Cfg<1>::kSmemBytes); };
+    if (swiglu) {
+        if (fmt == 1) return pick(gemm_tcgen05_kernel<1, 1, true>, gemm_tcgen05_kernel<1, 2, true>);
+        if (fmt == 3) return pick(gemm_tcgen05_kernel<3, 1, true>, gemm_tcgen05_kernel<3, 2, true>);
+        return pick(gemm_tcgen05_kernel<2, 1, true>, gemm_tcgen05_kernel<2, 2, true>);
+    }
+    if (fmt == 1) return pick(gemm_tcgen05_kernel<1, 1, false>, gemm_tcgen05_kernel<1, 2, false>);
+    if (fmt == 3) return pick(gemm_tcgen05_kernel<3, 1, false>, gemm_tcgen05_kernel<3, 2, false>);
+    return pick(gemm_tcgen05_kernel<2, 1, false>, gemm_tcgen05_kernel<2, 2, false>);
 }
 
 }  // namespace bonsai

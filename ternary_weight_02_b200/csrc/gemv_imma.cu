@@ -253,11 +253,17 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // kAsyncScales: K is a multiple of 512, so an item's four scales of a row are 8 aligned
 // bytes, copied with cp.async as part of the item's copy; otherwise each lane loads the
 // scales it needs when it processes the item.
-template <bool kAsyncScales>
+//
+// kSwiglu: the rows are a fused gate/up projection (gate rows 0 .. F-1, up rows F .. 2F-1,
+// N = 2F) and the output is h = silu(gate) * up (F values).  Row tile v then holds gate
+// rows 16v .. 16v+15 in its rows 0..15 and up rows F + 16v .. in rows 16..31 (two 16-row
+// TMA boxes), so that the lane that finishes row r < 16 of the tile finds the matching up
+// row in lane r + 16.  (When F % 16 != 0 the last tile's rows past gate row F - 1 belong to
+// no output and are not written; its up box reads zeros past row 2F - 1.)
+template <bool kAsyncScales, bool kSwiglu>
 __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const __grid_constant__ CUtensorMap wmap, const uint16_t *__restrict__ x, const uint16_t *__restrict__ scales,
-    uint16_t *__restrict__ y, uint64_t *__restrict__ partials, int N, int K,
-    uint32_t mul2, uint32_t mul4, uint32_t mul6) {
+    uint16_t *__restrict__ y, uint64_t *__restrict__ partials, int N, int K, int F) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -269,6 +275,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const int RT = (N + kItemRows - 1) / kItemRows;
     const int I = RT * KC;  // items (host-checked to fit)
     const int C = gridDim.x;
+    // weight row of row lr (0 .. 31) of row tile rt
+    auto row_of = [&](int rt, int lr) {
+        return kSwiglu ? (lr < 16 ? 16 * rt + lr : F + 16 * rt + (lr - 16)) : rt * kItemRows + lr;
+    };
     const int c0 = (int)((int64_t)I * blockIdx.x / C), c1 = (int)((int64_t)I * (blockIdx.x + 1) / C);
     const int nq = c1 - c0 > warp ? (c1 - c0 - warp + kConsumers - 1) / kConsumers : 0;  // this warp's items
 
@@ -300,10 +310,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
             const int st = q % kStages;
             if (lane == 0) {
                 mbar_arrive_expect_tx(full + st, kItemBytes);
-                tma_load_2d(wring + st * kItemBytes, &wmap, full + st, kc * kItemRowBytes, rt * kItemRows);
+                if (kSwiglu) {  // gate rows, then the matching up rows (16-row boxes)
+                    tma_load_2d(wring + st * kItemBytes, &wmap, full + st, kc * kItemRowBytes, 16 * rt);
+                    tma_load_2d(wring + st * kItemBytes + kItemBytes / 2, &wmap, full + st, kc * kItemRowBytes,
+                                F + 16 * rt);
+                } else {
+                    tma_load_2d(wring + st * kItemBytes, &wmap, full + st, kc * kItemRowBytes, rt * kItemRows);
+                }
             }
             if (kAsyncScales) {
-                const int row = rt * kItemRows + lane;
+                const int row = row_of(rt, lane);
                 const bool v = row < N;
                 cp_async8(sring + st * kScaleRingBytes + lane * 8, scales + (v ? (int64_t)row * G + kc * 4 : 0), v);
             }
@@ -396,6 +412,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
             s = e2;
             c2++;
         }
+        if (kSwiglu) {  // h = silu(gate) * up: lanes 0..15 hold gate rows, 16..31 the up rows
+            const float up = __shfl_down_sync(0xffffffffu, sum, 16);
+            const int f = 16 * rt + lane;
+            if (lane < 16 && f < F) y[f] = float_to_half_bits(sum / (1.f + expf(-sum)) * up);
+            return;
+        }
         const int row = rt * kItemRows + lane;
         if (row < N) y[row] = float_to_half_bits(sum);
     };
@@ -427,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
             const int g = g0 + tig;
 #pragma unroll
             for (int e = 0; e < 4; e++) {
-                const int row = rt * kItemRows + 8 * e + gid;
+                const int row = row_of(rt, 8 * e + gid);
                 sc[e] = (row < N && g < G) ? (uint32_t)__ldg(scales + (int64_t)row * G + g) : 0u;
             }
         }
@@ -566,7 +588,10 @@ size_t gemv_imma_zeroed_bytes(int64_t N, int64_t K) {
 }
 
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
-                             int64_t N, int64_t K, const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
+                             int64_t N, int64_t K, const Workspace &ws, cudaStream_t s, const DeviceInfo &dev,
+                             int64_t swiglu_f) {
+    const bool swiglu = swiglu_f > 0;
+    if (swiglu && N != 2 * swiglu_f) return cudaErrorInvalidValue;
     const Layout lay = make_layout((int)K);
     if (lay.total > dev.smem_optin) return cudaErrorInvalidValue;
     // the kernel's 128-bit and barrier accesses rely on these alignments
@@ -578,7 +603,7 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
     {
         const cuuint64_t dims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
         const cuuint64_t strides[1] = {(cuuint64_t)(K / 4)};
-        const cuuint32_t box[2] = {kItemRowBytes, kItemRows};
+        const cuuint32_t box[2] = {kItemRowBytes, swiglu ? kItemRows / 2 : kItemRows};
         const cuuint32_t estr[2] = {1, 1};
         if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -589,7 +614,8 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
     if (ws.zeroed_bytes < gemv_imma_zeroed_bytes(N, K)) return cudaErrorInvalidValue;
     uint64_t *partials = reinterpret_cast<uint64_t *>(ws.zeroed);
     // K a multiple of 512: an item's scales of a row are 8 aligned bytes, copied with the item
-    auto kern = K % kItemK == 0 ? gemv_imma_kernel<true> : gemv_imma_kernel<false>;
+    auto kern = K % kItemK == 0 ? (swiglu ? gemv_imma_kernel<true, true> : gemv_imma_kernel<true, false>)
+                                : (swiglu ? gemv_imma_kernel<false, true> : gemv_imma_kernel<false, false>);
     // the attribute is set to the largest layout any K takes, so that launches of several
     // sizes captured into one graph all stay within it
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -605,8 +631,7 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, wmap, x, scales, y, partials, (int)N, (int)K, 1u << 30,
-                              1u << 28, 1u << 26);
+    return cudaLaunchKernelEx(&cfg, kern, wmap, x, scales, y, partials, (int)N, (int)K, (int)swiglu_f);
 }
 
 }  // namespace bonsai

@@ -81,7 +81,8 @@ int current_device_info(DeviceInfo *out);
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t gemv_imma_zeroed_bytes(int64_t N, int64_t K);  // of Workspace::zeroed
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
-                             int64_t N, int64_t K, const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
+                             int64_t N, int64_t K, const Workspace &ws, cudaStream_t s, const DeviceInfo &dev,
+                             int64_t swiglu_f = 0);  // > 0: fused gate/up rows, write silu(gate) * up
 
 // ---- skinny_mma.cu: 1 <= M <= 16
 bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt);
@@ -91,13 +92,19 @@ cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16
                           uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int split_k,
                           const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
 
+// ---- swiglu.cu: h = silu(y[:, :F]) * y[:, F:] for an M x 2F FP16 y
+cudaError_t launch_swiglu(const uint16_t *y, uint16_t *h, int64_t M, int64_t F, cudaStream_t s,
+                          const DeviceInfo &dev);
+
 // ---- gemm_tcgen05.cu: prefill
 bool gemm_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, const DeviceInfo &dev);
 // tile_hint: 0 automatic, 1 one 128-row accumulator per CTA, 2 two (256 rows).  Uses
 // Workspace::counters[0, SMs) as hand-over flags (zero at rest).
+// swiglu_f > 0: the N = 2 swiglu_f rows are gate then up rows and y
+// gets silu(gate) * up, M x swiglu_f.
 cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                         uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int tile_hint,
-                        const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
+                        const Workspace &ws, cudaStream_t s, const DeviceInfo &dev, int64_t swiglu_f = 0);
 
 }  // namespace bonsai

@@ -469,3 +469,113 @@ def test_small_batches_ptq1_take_the_gemm(bz, M, fmt):
     got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
+
+
+# ------------------------------------------------------------ SwiGLU after the fused gate/up projection
+
+def swiglu_ok(h, y_ref):
+    """The SwiGLU output's bar, derived from the linear layer's: with |dy| <= 1e-2 rms(y)
+    on every gate and up value (the linear bar) and |silu'| <= 1.1, each h = silu(g) u may
+    move by (1.1 |u| + |silu(g)|) 1e-2 rms(y), plus one FP16 rounding of h; and rel-L2 of h
+    <= 1e-3 as for the linear output.  Returns (ok, rel-L2, worst ratio of error to bound)."""
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    F = y_ref.shape[1] // 2
+    g, u = y_ref[:, :F], y_ref[:, F:]
+    h_ref = oracle.swiglu(y_ref)
+    rms_y = np.sqrt(np.mean(y_ref ** 2))
+    bound = (1.1 * np.abs(u) + np.abs(g / (1.0 + np.exp(-g)))) * 1e-2 * rms_y + 2.0 ** -11 * np.abs(h_ref)
+    err = np.abs(np.asarray(h, dtype=np.float64) - h_ref)
+    rel = float(np.linalg.norm(err) / max(np.linalg.norm(h_ref), 1e-300))
+    worst = float(np.max(err / np.maximum(bound, 1e-300)))
+    return rel <= 1e-3 and worst <= 1.0, rel, worst
+
+
+def _run_swiglu(bz, p, F):
+    import torch
+    x, packed, scales = p.device()
+    h = torch.full((p.M, F), float("nan"), dtype=torch.float16, device="cuda")
+    bz.bonsai_ternary_linear_swiglu(x, packed, scales, h, p.M, F, p.K, p.fmt)
+    torch.cuda.synchronize()
+    return to_numpy_f16(h)
+
+
+# (M, F, K, fmt): fused in the integer GEMV (M = 1 PQ2_0; F = 24 leaves a part-used last
+# tile; the last case is the full 27B-class gate/up) or the GEMM (tiles split between
+# CTAs; F = 200 and 1270 part-used); the other packings at M = 1 and the skinny batches
+# take the linear kernel and then the SwiGLU kernel
+SWIGLU_CASES = [(1, 16, 512, PQ2), (1, 1024, 2048, PQ2), (1, 4000, 1152, PQ2), (1, 24, 512, PQ2),
+                (1, 1024, 1024, PTQ1), (1, 1024, 2048, Q1), (4, 512, 1024, PQ2), (300, 640, 640, PQ2),
+                (300, 640, 640, Q1), (300, 384, 1152, PTQ1), (600, 1280, 384, PQ2), (300, 200, 640, PQ2), (300, 1270, 256, Q1),
+                (1, 17408, 5120, PQ2)]
+
+
+@pytest.mark.parametrize("M,F,K,fmt", SWIGLU_CASES)
+def test_linear_swiglu(bz, M, F, K, fmt):
+    p = Problem(M, 2 * F, K, fmt, seed=M + F + K)
+    got = _run_swiglu(bz, p, F)
+    assert np.all(np.isfinite(got))
+    ok, rel, worst = swiglu_ok(got, p.oracle_y())
+    assert ok, (rel, worst)
+
+
+def test_swiglu_elementwise(bz):
+    import torch
+    rng = np.random.default_rng(3)
+    M, F = 3, 1000
+    y = (rng.normal(0, 2, (M, 2 * F))).astype(np.float16)
+    h = torch.empty((M, F), dtype=torch.float16, device="cuda")
+    bz.bonsai_swiglu(torch.from_numpy(y.view(np.int16)).cuda().view(torch.float16), h, M, F)
+    torch.cuda.synchronize()
+    # exact inputs: FP32 arithmetic and one FP16 rounding of h
+    ref = oracle.swiglu(y.astype(np.float64))
+    got = to_numpy_f16(h)
+    assert np.all(np.abs(got - ref) <= 2.0 ** -10 * np.abs(ref) + 1e-6)
+
+
+def test_swiglu_fused_repeatable_and_near_unfused(bz):
+    """The fused epilogue (FP32 sums into silu) gives the same bits on every call, split
+    row tiles included, and stays within FP16 rounding of linear-then-SwiGLU."""
+    import torch
+    F, K = 17408, 5120
+    p = Problem(1, 2 * F, K, PQ2, seed=21)
+    a = _run_swiglu(bz, p, F)
+    b = _run_swiglu(bz, p, F)
+    assert np.array_equal(a, b)
+    x, packed, scales = p.device()
+    y = torch.empty((1, 2 * F), dtype=torch.float16, device="cuda")
+    bz.bonsai_ternary_linear(x, packed, scales, y, 1, 2 * F, K, PQ2)
+    h = torch.empty((1, F), dtype=torch.float16, device="cuda")
+    bz.bonsai_swiglu(y, h, 1, F)
+    torch.cuda.synchronize()
+    ok, rel, worst = swiglu_ok(to_numpy_f16(h), p.oracle_y())
+    assert ok, (rel, worst)
+    assert swiglu_ok(a, p.oracle_y())[0]
+
+
+def test_swiglu_gemm_full_size_sampled(bz):
+    """Prefill M=2048 through the fused gate/up 5120 -> 2 x 17408 with SwiGLU in the GEMM's
+    epilogue; 48 x 48 sampled outputs against the checker."""
+    import torch
+    from ternary_weight_02_b200 import inputs
+    M, F, K, seed = 2048, 17408, 5120, 8
+    dev = torch.device("cuda")
+    t = torch.from_numpy(inputs.trits(seed, 2 * F, K)).to(dev)
+    packed = bz.pack(PQ2, t)
+    del t
+    s = torch.from_numpy(inputs.scales(seed, 2 * F, K).view(np.int16)).to(dev).view(torch.float16)
+    x = torch.from_numpy(inputs.activations(seed, M, K).view(np.int16)).to(dev).view(torch.float16)
+    h = torch.full((M, F), float("nan"), dtype=torch.float16, device=dev)
+    bz.bonsai_ternary_linear_swiglu(x, packed, s, h, M, F, K, PQ2)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(7)
+    ms = np.unique(np.concatenate([[0, M - 1], rng.integers(0, M, 46)]))
+    fs = np.unique(np.concatenate([[0, F - 1], rng.integers(0, F, 46)]))
+    rows = np.concatenate([fs, F + fs])  # the gate rows, then the matching up rows
+    xr = inputs.normal_rows(seed, K, ms)
+    w = inputs.trits_rows(seed, K, rows)
+    sc = inputs.scales_rows(seed, K // 128, rows)
+    y_ref = oracle.ternary_linear(xr, oracle.pack(PQ2, w), sc, len(rows), K, PQ2)
+    got = h[torch.from_numpy(ms).to(dev)][:, torch.from_numpy(fs).to(dev)].float().cpu().numpy()
+    ok, rel, worst = swiglu_ok(got, y_ref)
+    assert ok, (rel, worst)
+    assert bool(torch.isfinite(h).all())
