@@ -334,6 +334,8 @@ def run_ours(args):
         e2e = whole_job_gbs(step_bytes(f), world, ms_e2e)
 
         launches_per_layer = sum(bz.bonsai_launch_count(1, N, K, f) for _, K, N in SHAPES)
+        if f == 2:
+            results["swiglu_decode"] = measure_swiglu_decode(stack, xs, bz, torch, stream, dev, args)
         results[f] = {
             "launches_per_layer": launches_per_layer,
             "value": value, "ms": ms, "clocks": clk, "dom_us": dom_us, "dom_gbs": dom_gbs,
@@ -377,7 +379,11 @@ def run_ours(args):
         others = {FMT_NAMES[k]: {"value": round(v["value"], 1), "unit": "GB/s",
                                  "per_token_us": round(v["ms"] * 1e3, 2),
                                  "gate_up_gbs": round(v["dom_gbs"], 1), "e2e": round(v["e2e"], 1)}
-                  for k, v in results.items() if k != fmt}
+                  for k, v in results.items() if k in FMT_NAMES and k != fmt}
+        if "swiglu_decode" in results:
+            line["swiglu"] = {"decode": results["swiglu_decode"]}
+            if prefill is not None and "swiglu_gate_up" in prefill:
+                line["swiglu"]["prefill"] = prefill.pop("swiglu_gate_up")
         if others:
             line["other_packings"] = others
         if prefill is not None:
@@ -386,6 +392,48 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return line
+
+
+def measure_swiglu_decode(stack, xs, bz, torch, stream, dev, args):
+    """The MLP's gate/up projection at M = 1 followed by SwiGLU, 64 layers per replay:
+    fused (bonsai_ternary_linear_swiglu: the integer GEMV's epilogue applies it) against
+    the linear call and then bonsai_swiglu (a second kernel)."""
+    _, K, N = SHAPES[2]
+    F = N // 2
+    h = torch.empty((1, F), dtype=torch.float16, device=dev)
+    y2 = torch.empty((1, N), dtype=torch.float16, device=dev)
+    sp = stream.cuda_stream
+    out = {}
+    for fused in (True, False):
+        def enq():
+            for layer in range(LAYERS):
+                p, s = stack[2][layer]
+                if fused:
+                    bz.bonsai_ternary_linear_swiglu(xs[2], p, s, h, 1, F, K, 2, sp)
+                else:
+                    bz.bonsai_ternary_linear(xs[2], p, s, y2, 1, N, K, 2, sp)
+                    bz.bonsai_swiglu(y2, h, 1, F, sp)
+        with torch.cuda.stream(stream):
+            enq()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                enq()
+            for _ in range(3):
+                g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = max(3, args.steps)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        out["fused_us_per_layer" if fused else "unfused_us_per_layer"] = round(
+            e0.elapsed_time(e1) * 1e3 / (reps * LAYERS), 3)
+        del g
+    out["workload"] = f"gate/up 5120 -> 2 x {F} at M=1 then SwiGLU, 64 distinct weight copies per replay, PQ2_0"
+    return out
 
 
 def run_prefill(fmt, M, dev, bz, torch, peaks, peak_kind, steps):
@@ -421,12 +469,34 @@ def run_prefill(fmt, M, dev, bz, torch, peaks, peak_kind, steps):
             total_flop += flop
             per[name] = {"us": round(us, 1), "tflops": round(flop / us / 1e6, 1)}
     layer_us = sum(v["us"] for v in per.values())
+    # gate/up then SwiGLU: fused in the GEMM's epilogue against the GEMM and bonsai_swiglu
+    sw = {}
+    name, K, N, packed, s, x, y = items[2]
+    F = N // 2
+    h = torch.empty((M, F), dtype=torch.float16, device=dev)
+    with torch.cuda.stream(stream):
+        for fused in (True, False):
+            def call():
+                if fused:
+                    bz.bonsai_ternary_linear_swiglu(x, packed, s, h, M, F, K, fmt, sp)
+                else:
+                    bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt, sp)
+                    bz.bonsai_swiglu(y, h, M, F, sp)
+            call()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(steps):
+                call()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            sw["fused_us" if fused else "unfused_us"] = round(e0.elapsed_time(e1) * 1e3 / steps, 1)
+    sw["workload"] = f"M={M} x gate/up 5120 -> 2 x {F} then SwiGLU, {FMT_NAMES[fmt]}"
     burst = float(peaks["bf16_tflops"])
     dom = per["gate_up"]
     return {
         "metric": "prefill GEMM TFLOP/s", "value": round(total_flop / layer_us / 1e6, 1), "unit": "TFLOP/s",
         "workload": f"M={M} tokens x the four 27B-class projections, {FMT_NAMES[fmt]}, FP16 x FP16 -> FP32 (tcgen05)",
-        "us_per_layer": round(layer_us, 1), "per_projection": per,
+        "us_per_layer": round(layer_us, 1), "per_projection": per, "swiglu_gate_up": sw,
         "roofline": {"bound": "tensor", "kernel": "gemm gate/up 5120->34816 (incl. FWHT pass)",
                      "achieved": dom["tflops"], "peak": burst, "peak_kind": f"{peak_kind} bf16 burst (fp16 same dense rate)",
                      "unit": "TFLOP/s", "frac": round(dom["tflops"] / burst, 4),
