@@ -23,10 +23,16 @@ LIB = os.path.join(HERE, "liboracle.so")
 FMT_PTQ1_0 = 1
 FMT_PQ2_0 = 2
 FMT_Q1_0 = 3
+FMT_PQ2_0_G64 = 4  # PQ2_0 codes, one FP16 scale per 64 weights
 GROUP = 128
 INVALID_TRIT = -128
 
 _lib = None
+
+
+def scale_group(fmt: int) -> int:
+    """Weights per FP16 scale: 64 for PQ2_0 g64, 128 for the others."""
+    return 64 if fmt == FMT_PQ2_0_G64 else GROUP
 
 
 def build(force: bool = False) -> str:
@@ -92,7 +98,7 @@ def pack(fmt: int, trits: np.ndarray) -> np.ndarray:
         raise ValueError("bad format or shape")
     out = np.zeros(nbytes, dtype=np.uint8)
     fn = {FMT_PTQ1_0: lib().oracle_pack_ptq1, FMT_PQ2_0: lib().oracle_pack_pq2,
-          FMT_Q1_0: lib().oracle_pack_q1}[fmt]
+          FMT_Q1_0: lib().oracle_pack_q1, FMT_PQ2_0_G64: lib().oracle_pack_pq2}[fmt]
     fn(_ptr(t), _ptr(out), N, K)
     return out.reshape(N, -1) if N else out.reshape(0, 0)
 
@@ -113,7 +119,7 @@ def check(fmt: int, packed: np.ndarray, N: int, K: int) -> int:
     """Number of non-canonical codes in a packed plane (0 for a valid one)."""
     p = np.ascontiguousarray(packed, dtype=np.uint8).reshape(-1)
     fn = {FMT_PTQ1_0: lib().oracle_check_ptq1, FMT_PQ2_0: lib().oracle_check_pq2,
-          FMT_Q1_0: lib().oracle_check_q1}[fmt]
+          FMT_Q1_0: lib().oracle_check_q1, FMT_PQ2_0_G64: lib().oracle_check_pq2}[fmt]
     return int(fn(_ptr(p), N, K))
 
 
@@ -141,9 +147,10 @@ def fwht_recursive(v: np.ndarray) -> np.ndarray:
 
 def ternary_linear(x: np.ndarray, packed: np.ndarray, scales: np.ndarray, N: int, K: int,
                    fmt: int, apply_hadamard: bool = True, nthreads: int = 0) -> np.ndarray:
-    """Float64 y = x' . Wdeq^T for FP16 (or float64) x (M x K) and scales (N x K/128)."""
+    """Float64 y = x' . Wdeq^T for FP16 (or float64) x (M x K) and scales (N x K/128;
+    N x K/64 for PQ2_0 g64)."""
     xd = np.ascontiguousarray(np.asarray(x).reshape(-1, K), dtype=np.float64)
-    sd = np.ascontiguousarray(np.asarray(scales).reshape(N, K // GROUP), dtype=np.float64)
+    sd = np.ascontiguousarray(np.asarray(scales).reshape(N, K // scale_group(fmt)), dtype=np.float64)
     p = np.ascontiguousarray(packed, dtype=np.uint8).reshape(-1)
     if p.size != packed_bytes(fmt, N, K):
         raise ValueError("packed size does not match N, K")

@@ -17,6 +17,9 @@
  *      "each trit in a 2-bit slot", 2.13 bits/weight); and "Bonsai把 27B 大模型
  *      塞进手机的极端量化方案到底靠不靠谱" (wmrh.cn), section 关键机制 (the
  *      5 trits / 8 bits storage bound).
+ *      PQ2_0 g64 -- PQ2_0's 2-bit slots with one FP16 scale per 64 weights instead of
+ *                per 128 (the pages' Q2_0_g64 file, wmrh.cn page, 快速上手 and 后端支持
+ *                现状): only the scale plane (N x K/64) and the group of each scale change.
  *      Q1_0   -- the 1-bit sibling: weights w in {-1, +1}, one bit each, 16 bytes
  *                per group of 128.  Source: "Bonsai把 27B 大模型塞进手机的极端量化
  *                方案到底靠不靠谱" (wmrh.cn), section 核心观点 (1-bit Bonsai, about
@@ -57,6 +60,7 @@
 #define ORACLE_FMT_PTQ1_0 1
 #define ORACLE_FMT_PQ2_0 2
 #define ORACLE_FMT_Q1_0 3
+#define ORACLE_FMT_PQ2_0_G64 4 /* PQ2_0 codes, one scale per 64 weights */
 #define ORACLE_PTQ1_GROUP_BYTES 26 /* 25 bytes x 5 trits + 1 byte x 3 trits */
 #define ORACLE_INVALID_TRIT (-128) /* written by the unpackers for an invalid code */
 
@@ -69,6 +73,7 @@ long long oracle_packed_bytes(int fmt, long long N, long long K)
     if (fmt == ORACLE_FMT_PTQ1_0) return N * (K / ORACLE_GROUP) * ORACLE_PTQ1_GROUP_BYTES;
     if (fmt == ORACLE_FMT_PQ2_0) return N * (K / 4);
     if (fmt == ORACLE_FMT_Q1_0) return N * (K / 8);
+    if (fmt == ORACLE_FMT_PQ2_0_G64) return N * (K / 4);
     return -1;
 }
 
@@ -257,6 +262,7 @@ long long oracle_unpack(int fmt, const uint8_t *packed, int8_t *trits, long long
     if (fmt == ORACLE_FMT_PTQ1_0) return oracle_unpack_ptq1(packed, trits, N, K);
     if (fmt == ORACLE_FMT_PQ2_0) return oracle_unpack_pq2(packed, trits, N, K);
     if (fmt == ORACLE_FMT_Q1_0) return oracle_unpack_q1(packed, trits, N, K);
+    if (fmt == ORACLE_FMT_PQ2_0_G64) return oracle_unpack_pq2(packed, trits, N, K);
     return -1;
 }
 
@@ -333,7 +339,8 @@ long long oracle_ternary_linear(const double *x, const uint8_t *packed, const do
 {
     long long row_bytes = oracle_packed_bytes(fmt, 1, K);
     if (row_bytes < 0 || M < 0 || N < 0) return -1;
-    long long G = K / ORACLE_GROUP;
+    const int gs = fmt == ORACLE_FMT_PQ2_0_G64 ? 64 : ORACLE_GROUP; /* weights per scale */
+    long long G = K / gs;
     double *xr = (double *)malloc(sizeof(double) * (size_t)(M * K > 0 ? M * K : 1));
     if (apply_hadamard)
         oracle_hadamard128(x, xr, M, K);
@@ -349,7 +356,7 @@ long long oracle_ternary_linear(const double *x, const uint8_t *packed, const do
         int8_t *t = (int8_t *)malloc((size_t)(K > 0 ? K : 1));
         if (fmt == ORACLE_FMT_PTQ1_0)
             bad += ptq1_unpack_row(packed + n * row_bytes, t, K);
-        else if (fmt == ORACLE_FMT_PQ2_0)
+        else if (fmt == ORACLE_FMT_PQ2_0 || fmt == ORACLE_FMT_PQ2_0_G64)
             bad += pq2_unpack_row(packed + n * row_bytes, t, K);
         else
             bad += q1_unpack_row(packed + n * row_bytes, t, K);
@@ -357,8 +364,7 @@ long long oracle_ternary_linear(const double *x, const uint8_t *packed, const do
             double acc = 0.0;
             for (long long g = 0; g < G; g++) {
                 double dot = 0.0;
-                for (int j = 0; j < ORACLE_GROUP; j++)
-                    dot += (double)t[g * ORACLE_GROUP + j] * xr[m * K + g * ORACLE_GROUP + j];
+                for (int j = 0; j < gs; j++) dot += (double)t[g * gs + j] * xr[m * K + g * gs + j];
                 acc += scales[n * G + g] * dot;
             }
             y[m * N + n] = acc;

@@ -18,6 +18,7 @@ from ternary_weight_02_b200 import inputs
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 PTQ1, PQ2, Q1 = oracle.FMT_PTQ1_0, oracle.FMT_PQ2_0, oracle.FMT_Q1_0
+G64 = oracle.FMT_PQ2_0_G64
 
 
 def _weights(fmt, seed, N, K):
@@ -345,6 +346,49 @@ def test_linear_hand_cases(fmt):
     t = np.ones((1, K), dtype=np.int8)
     y = oracle.ternary_linear(xd, oracle.pack(fmt, t), s, 1, K, fmt)
     assert np.isclose(y[0, 0], 0.25 * np.sqrt(128.0), rtol=1e-14)
+
+
+# ---------------------------------------------------------------- PQ2_0 with 64-weight scale groups
+
+def test_g64_plane_and_bits():
+    # the codes are PQ2_0's byte for byte; only the scale plane doubles
+    t = inputs.trits(2, 3, 256)
+    assert np.array_equal(oracle.pack(G64, t), oracle.pack(PQ2, t))
+    assert oracle.packed_bytes(G64, 3, 256) == oracle.packed_bytes(PQ2, 3, 256) == 192
+    assert oracle.packed_bytes(G64, 1, 5120) * 8 / 5120 + 16 / 64 == 2.25
+    assert oracle.scale_group(G64) == 64 and oracle.scale_group(PQ2) == 128
+
+
+def test_g64_hand_case_halves():
+    # all trits +1, K = 128, scales (a, b): y = a * sum x'[:64] + b * sum x'[64:]
+    x = inputs.activations(4, 1, 128)
+    xr = oracle.hadamard128(x.astype(np.float64))
+    s = np.array([[0.5, -0.125]], dtype=np.float16)
+    y = oracle.ternary_linear(x, oracle.pack(G64, np.ones((1, 128), np.int8)), s, 1, 128, G64)
+    assert np.isclose(y[0, 0], 0.5 * xr[0, :64].sum() - 0.125 * xr[0, 64:].sum(), rtol=1e-13)
+
+
+def test_g64_equals_pq2_with_paired_scales():
+    N, K, M = 9, 640, 2
+    t = inputs.trits(5, N, K)
+    S = inputs.scales(5, N, K)
+    s64 = np.repeat(S, 2, axis=1)  # both halves of a 128-group carry its scale
+    x = inputs.activations(5, M, K)
+    y2 = oracle.ternary_linear(x, oracle.pack(PQ2, t), S, N, K, PQ2)
+    y64 = oracle.ternary_linear(x, oracle.pack(G64, t), s64, N, K, G64)
+    assert np.allclose(y64, y2, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("N,K,M", [(1, 128, 1), (4, 384, 2)])
+def test_g64_brute_force_dense(N, K, M):
+    t = inputs.trits(13, N, K)
+    s = inputs.scales_rows(13, K // 64, np.arange(N))
+    x = inputs.activations(13, M, K)
+    y = oracle.ternary_linear(x, oracle.pack(G64, t), s, N, K, G64)
+    H = oracle.sylvester128()
+    xr = (x.astype(np.float64).reshape(M, K // 128, 128) @ H.T).reshape(M, K)
+    W = t.astype(np.float64) * np.repeat(s.astype(np.float64), 64, axis=1)
+    assert np.allclose(y, xr @ W.T, rtol=1e-12, atol=1e-12)
 
 
 def test_linear_q1_hand_cases():
