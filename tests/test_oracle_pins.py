@@ -199,7 +199,7 @@ def test_bits_per_weight_match_pages():
 
 def test_packed_bytes_bad_shapes():
     assert oracle.packed_bytes(PTQ1, 4, 100) == -1
-    assert oracle.packed_bytes(4, 4, 128) == -1
+    assert oracle.packed_bytes(5, 4, 128) == -1
     assert oracle.packed_bytes(PQ2, 0, 128) == 0
     assert oracle.packed_bytes(Q1, 4, 256) == 128 and oracle.packed_bytes(Q1, 1, 64) == -1
 
