@@ -19,7 +19,7 @@
  * Layouts (all row-major, all buffers owned by the caller):
  *   x       M x K   FP16 (IEEE binary16 bit patterns in uint16_t)
  *   y       M x N   FP16, round-to-nearest-even from an FP32 accumulator
- *   scales  N x K/128  FP16
+ *   scales  N x K/128  FP16 (N x K/64 for BONSAI_FMT_PQ2_0_G64)
  *   trits   N x K   int8 in {-1, 0, +1}
  *   packed  the trit plane of one of the two packings of the allhereai.com page
  *           (paragraph on the two file packings):
@@ -37,6 +37,10 @@
  *         group scale): weight k of row n is bit k%8 of byte n*K/8 + k/8, 1 for +1
  *         and 0 for -1 (every byte is valid).  Plane size N * K/8 bytes.  Same
  *         scale plane and the same rotation of x as the ternary packings.
+ *     BONSAI_FMT_PQ2_0_G64  the PQ2_0 plane (same bytes, packed by bonsai_pack_pq2)
+ *         with one FP16 scale per 64 weights: scales is N x K/64, scale g covering
+ *         weights 64g .. 64g+63 of its row (the pages' Q2_0_g64; wmrh.cn page, 快速上手
+ *         and 后端支持现状).  2.25 bits/weight with the scales.
  *
  * Conventions for every entry point:
  *   - Pointers are CUDA device pointers (any allocator) and must be 16-byte
@@ -69,7 +73,8 @@ extern "C" {
 typedef enum {
     BONSAI_FMT_PTQ1_0 = 1,
     BONSAI_FMT_PQ2_0 = 2,
-    BONSAI_FMT_Q1_0 = 3
+    BONSAI_FMT_Q1_0 = 3,
+    BONSAI_FMT_PQ2_0_G64 = 4
 } bonsai_fmt;
 
 typedef enum {
@@ -107,7 +112,7 @@ const char *bonsai_status_string(int status);
 int bonsai_check_device(void);
 
 /* Bytes of the packed trit plane for N x K weights (scales excluded: they are
- * always N * K/128 FP16 values).  Returns BONSAI_ERR_SHAPE / BONSAI_ERR_FMT
+ * N * K/128 FP16 values, N * K/64 for BONSAI_FMT_PQ2_0_G64).  Returns BONSAI_ERR_SHAPE / BONSAI_ERR_FMT
  * (negative) on a bad argument. */
 int64_t bonsai_packed_bytes(int fmt, int64_t N, int64_t K);
 
@@ -140,8 +145,9 @@ int bonsai_hadamard128(const uint16_t *x, uint16_t *x_out, int64_t M, int64_t K,
 
 /* y = x' . Wdeq^T (definitions above) for un-rotated FP16 x: the Hadamard
  * rotation of x is applied inside the call.  Dispatch on M: M == 1 -> the
- * integer tensor-core GEMV (PQ2_0, K <= 24576) or the lookup-table GEMV (PTQ1_0),
- * 2 <= M <= 16 -> skinny tensor-core kernel, larger M -> tcgen05 GEMM.  The
+ * integer tensor-core GEMV (PQ2_0, K <= 24576) or the lookup-table GEMV (PTQ1_0,
+ * Q1_0, PQ2_0 g64), 2 <= M <= 16 -> skinny tensor-core kernel (PQ2_0), otherwise
+ * (and for the other packings at 2 <= M <= 16) the tcgen05 GEMM.  The
  * integer GEMV holds each 128-group of x' as 16-bit fixed point with a power-of-two
  * scale (|x~| <= 2^14) before the exact integer products; the other kernels round
  * x' to FP16 (GEMM, skinny) or keep it in FP32 (lookup tables, plain kernel).  y must

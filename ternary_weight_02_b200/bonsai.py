@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(PKG, "libbonsai.so")
 BONSAI_FMT_PTQ1_0 = 1
 BONSAI_FMT_PQ2_0 = 2
 BONSAI_FMT_Q1_0 = 3
+BONSAI_FMT_PQ2_0_G64 = 4  # PQ2_0 codes, one FP16 scale per 64 weights
 
 BONSAI_OK = 0
 BONSAI_ERR_NULL = -1
@@ -38,7 +39,8 @@ BONSAI_ALGO_SKINNY = 3
 BONSAI_ALGO_GEMM = 4
 BONSAI_ALGO_IMMA = 5
 
-FORMATS = {"ptq1": BONSAI_FMT_PTQ1_0, "pq2": BONSAI_FMT_PQ2_0, "q1": BONSAI_FMT_Q1_0}
+FORMATS = {"ptq1": BONSAI_FMT_PTQ1_0, "pq2": BONSAI_FMT_PQ2_0, "q1": BONSAI_FMT_Q1_0,
+           "pq2g64": BONSAI_FMT_PQ2_0_G64}
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -203,7 +205,7 @@ def pack(fmt: int, trits, stream=None):
     N, K = trits.shape
     out = torch.empty(bonsai_packed_bytes(fmt, N, K), dtype=torch.uint8, device=trits.device)
     fn = {BONSAI_FMT_PTQ1_0: bonsai_pack_ptq1, BONSAI_FMT_PQ2_0: bonsai_pack_pq2,
-          BONSAI_FMT_Q1_0: bonsai_pack_q1}[fmt]
+          BONSAI_FMT_Q1_0: bonsai_pack_q1, BONSAI_FMT_PQ2_0_G64: bonsai_pack_pq2}[fmt]
     fn(trits, out, N, K, stream)
     return out.view(N, -1) if N else out
 

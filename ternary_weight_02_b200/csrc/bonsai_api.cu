@@ -124,8 +124,10 @@ int check_shape(int64_t M, int64_t N, int64_t K) {
 }
 
 int check_fmt(int fmt) {
-    return (fmt == BONSAI_FMT_PTQ1_0 || fmt == BONSAI_FMT_PQ2_0 || fmt == BONSAI_FMT_Q1_0) ? BONSAI_OK
-                                                                                         : BONSAI_ERR_FMT;
+    return (fmt == BONSAI_FMT_PTQ1_0 || fmt == BONSAI_FMT_PQ2_0 || fmt == BONSAI_FMT_Q1_0 ||
+            fmt == BONSAI_FMT_PQ2_0_G64)
+               ? BONSAI_OK
+               : BONSAI_ERR_FMT;
 }
 
 int cuda_status(cudaError_t e) {
@@ -413,7 +415,7 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
     rc = probe_current(&dev, &st);
     if (rc != BONSAI_OK) return rc;
     size_t need = simple_workspace_bytes(M, N, K), zneed = 0;
-    for (int fmt = BONSAI_FMT_PTQ1_0; fmt <= BONSAI_FMT_Q1_0; fmt++) {
+    for (int fmt = BONSAI_FMT_PTQ1_0; fmt <= BONSAI_FMT_PQ2_0_G64; fmt++) {
         size_t v;
         if (M <= 1 && gemv_supported(1, N, K, fmt)) {
             v = gemv_workspace_bytes(N, K, fmt, 0, st->info);

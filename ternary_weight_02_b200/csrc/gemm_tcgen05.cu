@@ -312,6 +312,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nk = K / BK;
     const int64_t G = K / kGroup;
+    // PQ2_0 and its 64-weight-scale variant take their codes by TMA with the x' stage
+    constexpr bool kTma = kFmt == 2 || kFmt == 4;
+    const int64_t G64 = K / 64;  // PQ2_0 g64: scales per row
     const int nctas = (int)gridDim.x, cta = (int)blockIdx.x;
     // whole-tile waves first (CTA b: tiles b, b + C, ...), then the last one or two
     // waves' worth of tiles split by units
@@ -392,16 +395,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                         *abort_flag = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(full_a + st, C::kAStage + (kFmt == 2 ? CODE_STAGE_BYTES : 0));
+                    mbar_arrive_expect_tx(full_a + st, C::kAStage + (kTma ? CODE_STAGE_BYTES : 0));
 #pragma unroll
                     for (int a = 0; a < kAcc; a++)
                         tma_load_2d(sA + st * C::kAStage + a * (BM * BK * 2), &a_map, full_a + st, ks * BK,
                                     tm * C::kTileM + a * BM);
                     // PQ2_0: the stage's codes, 16 bytes of each of the tile's 256 weight rows
-                    if (kFmt == 2 && !kSwiglu)
+                    if (kTma && !kSwiglu)
                         tma_load_2d(const_cast<uint8_t *>(sCodes) + st * CODE_STAGE_BYTES, &w_map, full_a + st,
                                     ks * (BK / 4), tn * BN);
-                    if (kFmt == 2 && kSwiglu) {  // 128 gate rows, then the matching 128 up rows
+                    if (kTma && kSwiglu) {  // 128 gate rows, then the matching 128 up rows
                         tma_load_2d(const_cast<uint8_t *>(sCodes) + st * CODE_STAGE_BYTES, &w_map, full_a + st,
                                     ks * (BK / 4), tn * (BN / 2));
                         tma_load_2d(const_cast<uint8_t *>(sCodes) + st * CODE_STAGE_BYTES + CODE_STAGE_BYTES / 2,
@@ -477,13 +480,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                 GroupRaw cur, nxt;
                 const int g_last = (p.ke - 1) >> 1;
                 uint32_t sc = 0u;
-                if (kFmt != 2 && valid) load_group<kFmt>(packed, scales, n, G, p.kb >> 1, cur);
+                if (!kTma && valid) load_group<kFmt>(packed, scales, n, G, p.kb >> 1, cur);
                 if (kFmt == 2 && valid) sc = __ldg(scales + n * G + (p.kb >> 1));
+                if (kFmt == 4 && valid) sc = __ldg(scales + n * G64 + p.kb);  // one scale per stage
                 uint32_t cw[8];
                 uint32_t tneg = 0u, tpos = 0u;  // the group's value table {-s, 0, +s}
                 for (int ks = p.kb; ks < p.ke; ks++, it++) {
                     const int g = ks >> 1, hf = ks & 1;  // a 128-weight group fills two 64-wide stages
-                    if (ks == p.kb || hf == 0) {
+                    if (kFmt == 4) {  // a 64-weight scale group is one stage
+                        tneg = valid ? sc ^ 0x8000u : 0u;
+                        tpos = valid ? sc : 0u;
+                        if (valid && ks + 1 < p.ke) sc = __ldg(scales + n * G64 + ks + 1);
+                    } else if (ks == p.kb || hf == 0) {
                         if (kFmt == 2) {
                             tneg = valid ? sc ^ 0x8000u : 0u;
                             tpos = valid ? sc : 0u;
@@ -507,14 +515,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                     // every lane acquires the stage itself (and, PQ2_0, its codes); the verdict
                     // is made warp-uniform
                     const bool free_ok = !*abort_flag && mbar_wait(empty + st, ph ^ 1u) &&
-                                         (kFmt != 2 || mbar_wait(full_a + st, ph));
+                                         (!kTma || mbar_wait(full_a + st, ph));
                     if (!__all_sync(0xffffffffu, free_ok)) {
                         *abort_flag = 1;
                         live = false;
                         break;
                     }
                     uint32_t w4[4];
-                    if (kFmt == 2) {
+                    if (kTma) {
                         const uint4 c4 = *reinterpret_cast<const uint4 *>(sCodes + st * CODE_STAGE_BYTES + r * 16);
                         w4[0] = c4.x, w4[1] = c4.y, w4[2] = c4.z, w4[3] = c4.w;
                     } else {
@@ -545,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
                     if (lane == 0) mbar_arrive(full_b + st);
-                    if (kFmt != 2 && hf == 1) cur = nxt;
+                    if (!kTma && hf == 1) cur = nxt;
                 }
             }
 
@@ -805,7 +813,7 @@ size_t x_rot_bytes(int64_t M, int64_t K) { return (((size_t)M * (size_t)K * 2) +
 }  // namespace
 
 bool gemm_supported(int64_t M, int64_t N, int64_t K, int fmt) {
-    if (fmt != 1 && fmt != 2 && fmt != 3) return false;
+    if (fmt < 1 || fmt > 4) return false;
     // TMA coordinates are 32-bit; the unit count of the work split must fit an int
     if (!(M >= 1 && M < (int64_t)1 << 30 && N >= 1 && N < (int64_t)1 << 30 && K % kGroup == 0 &&
           K < (int64_t)1 << 30))
@@ -848,7 +856,7 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
 
     // PQ2_0 codes: rows of K/4 bytes, a box of 16 bytes x 256 rows per 64-wide stage
     CUtensorMap wmap = map;  // (unused by PTQ1_0)
-    if (fmt == 2) {
+    if (fmt == 2 || fmt == 4) {
         const cuuint64_t wdims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
         const cuuint64_t wstrides[1] = {(cuuint64_t)(K / 4)};
         const cuuint32_t wbox[2] = {BK / 4, swiglu ? BN / 2 : BN};
@@ -868,10 +876,12 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
     if (swiglu) {
         if (fmt == 1) return pick(gemm_tcgen05_kernel<1, 1, true>, gemm_tcgen05_kernel<1, 2, true>);
         if (fmt == 3) return pick(gemm_tcgen05_kernel<3, 1, true>, gemm_tcgen05_kernel<3, 2, true>);
+        if (fmt == 4) return pick(gemm_tcgen05_kernel<4, 1, true>, gemm_tcgen05_kernel<4, 2, true>);
         return pick(gemm_tcgen05_kernel<2, 1, true>, gemm_tcgen05_kernel<2, 2, true>);
     }
     if (fmt == 1) return pick(gemm_tcgen05_kernel<1, 1, false>, gemm_tcgen05_kernel<1, 2, false>);
     if (fmt == 3) return pick(gemm_tcgen05_kernel<3, 1, false>, gemm_tcgen05_kernel<3, 2, false>);
+    if (fmt == 4) return pick(gemm_tcgen05_kernel<4, 1, false>, gemm_tcgen05_kernel<4, 2, false>);
     return pick(gemm_tcgen05_kernel<2, 1, false>, gemm_tcgen05_kernel<2, 2, false>);
 }
 

@@ -75,6 +75,7 @@ template <>
 struct Fmt<2> {  // PQ2_0
     static constexpr int kSliceK = 512;       // activations per K slice
     static constexpr int kLanesPerGroup = 8;  // lanes whose words cover one scale group
+    static constexpr int kScaleGroup = 128;   // weights per FP16 scale
     static constexpr int kSliceBytes = 128;
     __device__ static int64_t row_bytes(int64_t K) { return K / 4; }
     // byte offset of the lane's word inside a row's slice segment
@@ -85,6 +86,7 @@ template <>
 struct Fmt<1> {  // PTQ1_0
     static constexpr int kSliceK = 512;
     static constexpr int kLanesPerGroup = 8;
+    static constexpr int kScaleGroup = 128;
     static constexpr int kSliceBytes = 4 * kPtq1GroupBytes;  // 104
     __device__ static int64_t row_bytes(int64_t K) { return (K / kGroup) * kPtq1GroupBytes; }
     // the 8th lane of a group reads a valid word too; its tables are all zero
@@ -98,8 +100,19 @@ template <>
 struct Fmt<3> {  // Q1_0: a byte holds 8 signs, so a 128-byte row slice covers 1024 activations
     static constexpr int kSliceK = 1024;
     static constexpr int kLanesPerGroup = 4;
+    static constexpr int kScaleGroup = 128;
     static constexpr int kSliceBytes = 128;
     __device__ static int64_t row_bytes(int64_t K) { return K / 8; }
+    __device__ static int lane_offset(int lane) { return 4 * lane; }
+};
+
+template <>
+struct Fmt<4> {  // PQ2_0 with one scale per 64 weights: PQ2_0's tables, 4 lanes per scale group
+    static constexpr int kSliceK = 512;
+    static constexpr int kLanesPerGroup = 4;
+    static constexpr int kScaleGroup = 64;
+    static constexpr int kSliceBytes = 128;
+    __device__ static int64_t row_bytes(int64_t K) { return K / 4; }
     __device__ static int lane_offset(int lane) { return 4 * lane; }
 };
 
@@ -163,7 +176,7 @@ __device__ __forceinline__ void build_tables(const float *xr, uint8_t *tables, i
     const int lane = t & 31, j = (t >> 5) & 3, q = t >> 7;
     const float *xa;
     int n, place;  // trits in the chunk, place value of one digit (4: 2-bit slots, 3: base 3)
-    if (kFmt == 2) {
+    if (kFmt == 2 || kFmt == 4) {
         xa = xr + 4 * (4 * lane + j);  // chunk 4*lane + j covers activations 4c .. 4c+3
         n = 4;
         place = 4;
@@ -177,7 +190,7 @@ __device__ __forceinline__ void build_tables(const float *xr, uint8_t *tables, i
     int combos = 1;
     for (int i = 2; i < n; i++) combos *= 3;
     float xs[5];
-    if (kFmt == 2) {
+    if (kFmt == 2 || kFmt == 4) {
         const float4 q4 = *reinterpret_cast<const float4 *>(xa);
         xs[0] = q4.x, xs[1] = q4.y, xs[2] = q4.z, xs[3] = q4.w, xs[4] = 0.f;
     } else {
@@ -292,10 +305,10 @@ __device__ __forceinline__ float2 task_group_sums(const uint32_t (&w)[kRows], co
     return make_float2(v[0] * half_bits_to_float(sc[0]), v[1] * half_bits_to_float(sc[1]));
 }
 
-// Q1_0: lookups of one task, the reduction over the 4 lanes of each of the slice's 8
-// scale groups, the scales, then the sum over the groups.  Lanes L and L + 16 end with
-// row L & 15 of the task.
-__device__ __forceinline__ float task_total_q1(const uint32_t (&w)[kRows], const uint16_t (&sc)[4],
+// Q1_0 and PQ2_0 g64 (4 lanes per scale group): lookups of one task, the reduction over
+// the 4 lanes of each of the slice's 8 scale groups, the scales, then the sum over the
+// groups.  Lanes L and L + 16 end with row L & 15 of the task.
+__device__ __forceinline__ float task_total_4lane(const uint32_t (&w)[kRows], const uint16_t (&sc)[4],
                                                const uint32_t (&pbase)[4], int lane) {
     float v[kRows];
 #pragma unroll
@@ -347,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
     pdl_launch_dependents();
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t G = K / kGroup;
+    const int64_t G = K / Fmt<kFmt>::kScaleGroup;  // scales per row
     constexpr int kSK = Fmt<kFmt>::kSliceK, kLPG = Fmt<kFmt>::kLanesPerGroup, kNS = kRows / kLPG;
     const int S = (int)(K / kSK);
     const int64_t RB = (N + kRows - 1) / kRows;
@@ -357,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
     const uint32_t row_bytes = (uint32_t)Fmt<kFmt>::row_bytes(K);
     const int lane_off = Fmt<kFmt>::lane_offset(lane);
     const uint8_t *slice_base = packed + (int64_t)slice * Fmt<kFmt>::kSliceBytes;
-    const int64_t gcol = (int64_t)slice * (kSK / kGroup) + lane / kLPG;
+    const int64_t gcol = (int64_t)slice * (kSK / Fmt<kFmt>::kScaleGroup) + lane / kLPG;
 
     zero_phantom_tables<kFmt>(tables, lane, warp);
     pdl_wait();  // x, the workspace and y may belong to the previous kernel
@@ -383,8 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_split_kernel(
     // one slice's sums go straight to y (S == 1) or to the FP32 partials, which
     // gemv_reduce_kernel adds up in slice order
     auto task_total = [&](const uint32_t(&w)[kRows], const uint16_t(&sc)[kNS]) -> float {
-        if constexpr (kFmt == 3)
-            return task_total_q1(w, sc, pbase, lane);
+        if constexpr (kLPG == 4)
+            return task_total_4lane(w, sc, pbase, lane);
         else
             return groups_total(task_group_sums(w, sc, pbase, lane), lane);
     };
@@ -529,7 +542,7 @@ bool use_rows_mode(int64_t N, int64_t K, int fmt, const DeviceInfo &dev) {
 
 // Split mode: rows of the weight matrix are split into `parts` ranges per K slice so that
 // the grid (slices x parts) fills the SMs once.
-int slice_k(int fmt) { return fmt == 3 ? Fmt<3>::kSliceK : kSliceK; }
+int slice_k(int fmt) { return fmt == 3 ? Fmt<3>::kSliceK : kSliceK; }  // (PQ2_0 g64: 512)
 
 int gemv_parts(int64_t N, int64_t K, int fmt, const DeviceInfo &dev) {
     const int64_t S = K / slice_k(fmt);
@@ -577,6 +590,7 @@ cudaError_t launch_split(const uint16_t *x, const uint8_t *packed, const uint16_
     if (grid > 0x7fffffff) return cudaErrorInvalidValue;
     cudaError_t e = fmt == 1   ? launch_pdl(gemv_split_kernel<1>, (int)grid, s, x, packed, scales, y, partials, N, K, parts)
                     : fmt == 3 ? launch_pdl(gemv_split_kernel<3>, (int)grid, s, x, packed, scales, y, partials, N, K, parts)
+                    : fmt == 4 ? launch_pdl(gemv_split_kernel<4>, (int)grid, s, x, packed, scales, y, partials, N, K, parts)
                                : launch_pdl(gemv_split_kernel<2>, (int)grid, s, x, packed, scales, y, partials, N, K, parts);
     if (e != cudaSuccess || S == 1) return e;
     const int64_t rgrid64 = (N + 255) / 256;
@@ -587,14 +601,14 @@ cudaError_t launch_split(const uint16_t *x, const uint8_t *packed, const uint16_
 }  // namespace
 
 bool gemv_supported(int64_t M, int64_t N, int64_t K, int fmt) {
-    if (M != 1 || (fmt != 1 && fmt != 2 && fmt != 3) || K % slice_k(fmt) != 0) return false;
+    if (M != 1 || fmt < 1 || fmt > 4 || K % slice_k(fmt) != 0) return false;
     if ((N + kRows - 1) / kRows > kMaxTiles) return false;
     return true;
 }
 
 // Schedule: split_k 0 = automatic, 1 = rows mode (when the shape allows it), >= 2 = split mode.
 bool pick_rows_mode(int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev) {
-    if (fmt == 3) return false;  // Q1_0: split mode only
+    if (fmt == 3 || fmt == 4) return false;  // Q1_0, PQ2_0 g64: split mode only
     if (split_k == 1) return K <= kRowsModeMaxK && K / kSliceK >= 2;
     if (split_k >= 2) return false;
     return use_rows_mode(N, K, fmt, dev);

@@ -34,6 +34,7 @@ __global__ void __launch_bounds__(256) linear_simple_kernel(
         float acc[kTokensPerWarp] = {0.f, 0.f, 0.f, 0.f};
         for (int64_t g = lane; g < G; g += 32) {
             float dot[kTokensPerWarp] = {0.f, 0.f, 0.f, 0.f};
+            float dot_hi[kTokensPerWarp] = {0.f, 0.f, 0.f, 0.f};  // PQ2_0 g64: weights 64 .. 127
             for (int j = 0; j < kGroup; j++) {
                 int t;
                 if (kFmt == 1) {
@@ -48,10 +49,22 @@ __global__ void __launch_bounds__(256) linear_simple_kernel(
                     t = ((v >> (2 * (j % 4))) & 3) - 1;
                 }
                 for (int i = 0; i < kTokensPerWarp; i++)
-                    if (m0 + i < M) dot[i] += (float)t * xr[(m0 + i) * K + g * kGroup + j];
+                    if (m0 + i < M) {
+                        const float p = (float)t * xr[(m0 + i) * K + g * kGroup + j];
+                        if (kFmt == 4 && j >= 64)
+                            dot_hi[i] += p;
+                        else
+                            dot[i] += p;
+                    }
             }
-            const float sc = half_bits_to_float(scales[n * G + g]);
-            for (int i = 0; i < kTokensPerWarp; i++) acc[i] += sc * dot[i];
+            if (kFmt == 4) {  // two scales per 128 weights
+                const float s0 = half_bits_to_float(scales[n * 2 * G + 2 * g]);
+                const float s1 = half_bits_to_float(scales[n * 2 * G + 2 * g + 1]);
+                for (int i = 0; i < kTokensPerWarp; i++) acc[i] += s0 * dot[i] + s1 * dot_hi[i];
+            } else {
+                const float sc = half_bits_to_float(scales[n * G + g]);
+                for (int i = 0; i < kTokensPerWarp; i++) acc[i] += sc * dot[i];
+            }
         }
         for (int i = 0; i < kTokensPerWarp; i++) {
             const float total = warp_sum(acc[i]);
@@ -81,6 +94,8 @@ cudaError_t launch_linear_simple(const uint16_t *x, const uint8_t *packed, const
         linear_simple_kernel<1><<<grid, 256, 0, s>>>(xr, packed, scales, y, M, N, K);
     else if (fmt == 3)
         linear_simple_kernel<3><<<grid, 256, 0, s>>>(xr, packed, scales, y, M, N, K);
+    else if (fmt == 4)
+        linear_simple_kernel<4><<<grid, 256, 0, s>>>(xr, packed, scales, y, M, N, K);
     else
         linear_simple_kernel<2><<<grid, 256, 0, s>>>(xr, packed, scales, y, M, N, K);
     return cudaGetLastError();

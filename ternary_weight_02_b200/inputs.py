@@ -124,9 +124,9 @@ def scales_rows(seed: int, G: int, rows, stream_id: int = STREAM_SCALES) -> np.n
     return (SCALE_LO + (SCALE_HI - SCALE_LO) * u).astype(np.float16)
 
 
-def scales(seed: int, N: int, K: int, stream_id: int = STREAM_SCALES) -> np.ndarray:
-    """N x (K/128) FP16 scales, row-major."""
-    return scales_rows(seed, K // 128, np.arange(N), stream_id)
+def scales(seed: int, N: int, K: int, stream_id: int = STREAM_SCALES, group: int = 128) -> np.ndarray:
+    """N x (K/group) FP16 scales, row-major (one scale per `group` weights of a row)."""
+    return scales_rows(seed, K // group, np.arange(N), stream_id)
 
 
 def normal_rows(seed: int, K: int, rows, stream_id: int = STREAM_X) -> np.ndarray:

@@ -16,7 +16,7 @@ class Problem:
         self.M, self.N, self.K, self.fmt, self.seed = M, N, K, fmt, seed
         # the 1-bit Q1_0 packing holds weights +-1 only
         self.trits = inputs.signs(seed, N, K) if fmt == oracle.FMT_Q1_0 else inputs.trits(seed, N, K)
-        self.scales = inputs.scales(seed, N, K)
+        self.scales = inputs.scales(seed, N, K, group=oracle.scale_group(fmt))
         self.x = inputs.activations(seed, M, K) if M > 0 else np.zeros((0, K), np.float16)
 
     # checker side

@@ -43,6 +43,7 @@ def test_packed_bytes_host_arithmetic(bz):
     assert bz.bonsai_packed_bytes(bz.BONSAI_FMT_PTQ1_0, 5120, 17408) == 5120 * 136 * 26
     assert bz.bonsai_packed_bytes(bz.BONSAI_FMT_PQ2_0, 34816, 5120) == 34816 * 1280
     assert bz.bonsai_packed_bytes(bz.BONSAI_FMT_Q1_0, 34816, 5120) == 34816 * 640
+    assert bz.bonsai_packed_bytes(bz.BONSAI_FMT_PQ2_0_G64, 34816, 5120) == 34816 * 1280  # PQ2_0's plane
     assert bz.raw().bonsai_packed_bytes(bz.BONSAI_FMT_PQ2_0, 4, 100) == bz.BONSAI_ERR_SHAPE
     assert bz.raw().bonsai_packed_bytes(7, 4, 128) == bz.BONSAI_ERR_FMT
     assert bz.raw().bonsai_packed_bytes(1, -1, 128) == bz.BONSAI_ERR_SHAPE
@@ -62,7 +63,7 @@ def test_host_validation_needs_no_gpu(bz):
     assert L.bonsai_hadamard128(good, good, 2, 64, None) == bz.BONSAI_ERR_SHAPE
     # format
     assert L.bonsai_ternary_linear(good, good, good, good, 1, 8, 128, 0, None) == bz.BONSAI_ERR_FMT
-    assert L.bonsai_unpack(4, good, good, 1, 128, None) == bz.BONSAI_ERR_FMT
+    assert L.bonsai_unpack(5, good, good, 1, 128, None) == bz.BONSAI_ERR_FMT
     # alignment
     assert L.bonsai_ternary_linear(good + 2, good, good, good, 1, 8, 128, 2, None) == bz.BONSAI_ERR_ALIGN
     assert L.bonsai_pack_ptq1(good, good + 8, 4, 128, None) == bz.BONSAI_ERR_ALIGN

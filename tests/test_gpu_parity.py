@@ -11,7 +11,7 @@ from tests.gpu_util import Problem, to_numpy_f16
 
 pytestmark = pytest.mark.gpu
 
-PTQ1, PQ2, Q1 = oracle.FMT_PTQ1_0, oracle.FMT_PQ2_0, oracle.FMT_Q1_0
+PTQ1, PQ2, Q1, G64 = oracle.FMT_PTQ1_0, oracle.FMT_PQ2_0, oracle.FMT_Q1_0, oracle.FMT_PQ2_0_G64
 
 
 @pytest.fixture(scope="module")
@@ -125,7 +125,7 @@ def _run(bz, p, algo, split_k=0):
 SIMPLE_CASES = [(1, 1, 128), (1, 33, 384), (3, 100, 1024), (17, 65, 640), (1, 1024, 1024)]
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1, G64])
 @pytest.mark.parametrize("M,N,K", SIMPLE_CASES)
 def test_linear_simple(bz, fmt, M, N, K):
     p = Problem(M, N, K, fmt, seed=M * 7 + N)
@@ -134,7 +134,7 @@ def test_linear_simple(bz, fmt, M, N, K):
     assert ok, (rel, mx)
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1, G64])
 def test_linear_auto_config1(bz, fmt):
     """Single ternary linear, M=1, K=1024 -> N=1024, seed 0, through the default entry point."""
     import torch
@@ -171,7 +171,7 @@ def test_argument_errors_on_device(bz):
 GEMV_CASES = [(1, 512), (33, 512), (100, 1024), (1024, 1024), (1000, 2048), (37, 17408)]
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, G64])
 @pytest.mark.parametrize("N,K", GEMV_CASES)
 def test_gemv_small(bz, fmt, N, K):
     p = Problem(1, N, K, fmt, seed=N + 3 * K)
@@ -206,7 +206,7 @@ def test_q1_k_not_multiple_of_1024(bz):
 DECODE_SHAPES = [(5120, 7168), (5120, 5120), (5120, 34816), (17408, 5120)]
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1, G64])
 @pytest.mark.parametrize("K,N", DECODE_SHAPES)
 def test_gemv_decode_shapes_full(bz, fmt, K, N):
     """Every output of the full-size M=1 projections against the float64 checker."""
@@ -214,7 +214,7 @@ def test_gemv_decode_shapes_full(bz, fmt, K, N):
     got = _run(bz, p, bz.BONSAI_ALGO_GEMV)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
-    if fmt in (PTQ1, Q1):  # through the default entry point too (M == 1 PTQ1_0, Q1_0 dispatch here)
+    if fmt in (PTQ1, Q1, G64):  # through the default entry point too (M == 1 dispatches here)
         import torch
         x, packed, scales = p.device()
         y = torch.empty((1, N), dtype=torch.float16, device="cuda")
@@ -223,7 +223,7 @@ def test_gemv_decode_shapes_full(bz, fmt, K, N):
         assert np.array_equal(to_numpy_f16(y), got)
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1, G64])
 def test_gemv_repeatable_and_counters_reset(bz, fmt):
     """Split-K arrival counters return to zero: back-to-back calls on different shapes
     give bit-identical results (the slice-ordered reduction is deterministic)."""
@@ -353,7 +353,7 @@ GEMM_SMALL = [(1, 64, 128), (17, 256, 128), (130, 300, 384), (256, 512, 1024), (
               (600, 2000, 1152), (1000, 3000, 2048), (2000, 9500, 256)]
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1, G64])
 @pytest.mark.parametrize("M,N,K", GEMM_SMALL)
 @pytest.mark.parametrize("tile", [1, 2])
 def test_gemm_small(bz, fmt, M, N, K, tile):
@@ -365,7 +365,7 @@ def test_gemm_small(bz, fmt, M, N, K, tile):
     assert ok, (rel, mx)
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1, G64])
 def test_gemm_split_tiles_repeatable(bz, fmt):
     """Split tiles hand their partial sums over through flags that the owner clears:
     the same call twice, and after a differently split shape, gives the same bits."""
@@ -387,7 +387,7 @@ def _sampled_reference(fmt, M, N, K, seed, ms, ns):
     um, un = np.unique(ms), np.unique(ns)
     x = inputs.normal_rows(seed, K, um)
     t = inputs.signs_rows(seed, K, un) if fmt == Q1 else inputs.trits_rows(seed, K, un)
-    s = inputs.scales_rows(seed, K // 128, un)
+    s = inputs.scales_rows(seed, K // oracle.scale_group(fmt), un)
     y = oracle.ternary_linear(x, oracle.pack(fmt, t), s, len(un), K, fmt)
     return y, um, un
 
@@ -396,7 +396,7 @@ def _sampled_reference(fmt, M, N, K, seed, ms, ns):
 PREFILL = [(2048, 5120, 34816), (512, 17408, 5120), (8192, 5120, 7168)]
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1, G64])
 @pytest.mark.parametrize("M,K,N", PREFILL)
 def test_gemm_prefill_full_size_sampled(bz, fmt, M, K, N):
     """Full-size GEMM on the device; 64 x 64 sampled outputs against the checker."""
@@ -409,7 +409,8 @@ def test_gemm_prefill_full_size_sampled(bz, fmt, M, K, N):
     del w
     packed = bz.pack(fmt, t)
     del t
-    s = torch.from_numpy(inputs.scales(seed, N, K).view(np.int16)).to(dev).view(torch.float16)
+    s = torch.from_numpy(inputs.scales(seed, N, K, group=oracle.scale_group(fmt)).view(np.int16))
+    s = s.to(dev).view(torch.float16)
     x = torch.from_numpy(inputs.activations(seed, M, K).view(np.int16)).to(dev).view(torch.float16)
     y = torch.full((M, N), float("nan"), dtype=torch.float16, device=dev)
     bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt)
@@ -463,7 +464,7 @@ def test_skinny_split_is_deterministic(bz):
 
 
 @pytest.mark.parametrize("M", [2, 5, 16])
-@pytest.mark.parametrize("fmt", [PTQ1, Q1])
+@pytest.mark.parametrize("fmt", [PTQ1, Q1, G64])
 def test_small_batches_ptq1_take_the_gemm(bz, M, fmt):
     p = Problem(M, 300, 1024, fmt, seed=M)
     got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
@@ -506,7 +507,7 @@ def _run_swiglu(bz, p, F):
 SWIGLU_CASES = [(1, 16, 512, PQ2), (1, 1024, 2048, PQ2), (1, 4000, 1152, PQ2), (1, 24, 512, PQ2),
                 (1, 1024, 1024, PTQ1), (1, 1024, 2048, Q1), (4, 512, 1024, PQ2), (300, 640, 640, PQ2),
                 (300, 640, 640, Q1), (300, 384, 1152, PTQ1), (600, 1280, 384, PQ2), (300, 200, 640, PQ2), (300, 1270, 256, Q1),
-                (1, 17408, 5120, PQ2)]
+                (1, 1024, 2048, G64), (300, 200, 640, G64), (600, 1280, 384, G64), (1, 17408, 5120, PQ2)]
 
 
 @pytest.mark.parametrize("M,F,K,fmt", SWIGLU_CASES)
