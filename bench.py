@@ -40,19 +40,31 @@ sys.path.insert(0, ROOT)
 METRIC = "batch-1 ternary GEMV HBM GB/s (% of 8 TB/s); prefill GEMM TFLOPS (% peak)"
 SHAPES = [("qkv", 5120, 7168), ("o", 5120, 5120), ("gate_up", 5120, 34816), ("down", 17408, 5120)]
 LAYERS = 64
-FMT_NAMES = {1: "PTQ1_0", 2: "PQ2_0", 3: "Q1_0"}
-FMTS = {"ptq1": 1, "pq2": 2, "q1": 3}
+FMT_NAMES = {1: "PTQ1_0", 2: "PQ2_0", 3: "Q1_0", 4: "PQ2_0_g64"}
+FMTS = {"ptq1": 1, "pq2": 2, "q1": 3, "pq2g64": 4}
 # the kernel a batch-1 call runs for each packing, and its source file
 DOM_KERNEL = {1: "lookup-table GEMV (gemv_split_kernel + in-order reduction)",
               2: "integer tensor-core GEMV (gemv_imma_kernel)",
-              3: "lookup-table GEMV (gemv_split_kernel, 1-bit tables + in-order reduction)"}
-DOM_SOURCE = {1: "gemv_lut.cu", 2: "gemv_imma.cu", 3: "gemv_lut.cu"}
+              3: "lookup-table GEMV (gemv_split_kernel, 1-bit tables + in-order reduction)",
+              4: "lookup-table GEMV (gemv_split_kernel, 64-weight scale groups + in-order reduction)"}
+DOM_SOURCE = {1: "gemv_lut.cu", 2: "gemv_imma.cu", 3: "gemv_lut.cu", 4: "gemv_lut.cu"}
 
 
 def weights(fmt, seed, N, K):
     """Seeded weights of the workload: trits, or signs for the 1-bit Q1_0 packing."""
     from ternary_weight_02_b200 import inputs
     return inputs.signs(seed, N, K) if fmt == 3 else inputs.trits(seed, N, K)
+
+
+def scale_group(fmt):
+    """Weights per FP16 scale: 64 for the g64 variant of PQ2_0, else 128."""
+    return 64 if fmt == 4 else 128
+
+
+def scales(fmt, seed, N, K):
+    """Seeded N x K/group FP16 scale plane of the workload."""
+    from ternary_weight_02_b200 import inputs
+    return inputs.scales(seed, N, K, group=scale_group(fmt))
 
 
 def measured_peaks():
@@ -66,7 +78,7 @@ def measured_peaks():
 
 def plane_bytes(fmt, N, K):
     trit = N * (K // 128) * 26 if fmt == 1 else (N * K // 8 if fmt == 3 else N * K // 4)
-    return trit + N * (K // 128) * 2
+    return trit + N * (K // scale_group(fmt)) * 2
 
 
 def step_bytes(fmt):
@@ -175,7 +187,7 @@ def run_reference(args):
     probs = []
     for i, (name, K, N) in enumerate(SHAPES):
         t = weights(fmt, i, N, K)
-        probs.append((inputs.activations(i, 1, K), oracle.pack(fmt, t), inputs.scales(i, N, K), N, K))
+        probs.append((inputs.activations(i, 1, K), oracle.pack(fmt, t), scales(fmt, i, N, K), N, K))
     threads = oracle.max_threads()
 
     def one_step():
@@ -216,7 +228,7 @@ def build_stack(fmt, dev, bz, torch):
         t = torch.from_numpy(weights(fmt, i, N, K)).to(dev)
         packed = bz.pack(fmt, t)
         del t
-        s = torch.from_numpy(inputs.scales(i, N, K).view(np.int16)).to(dev).view(torch.float16)
+        s = torch.from_numpy(scales(fmt, i, N, K).view(np.int16)).to(dev).view(torch.float16)
         copies = [(packed.clone(), s.clone()) for _ in range(LAYERS)]
         del packed, s
         stack.append(copies)
@@ -242,7 +254,7 @@ def run_ours(args):
     bz.bonsai_reserve(1, 34816, 17408)
 
     results = {}
-    for f in ([fmt] + [o for o in (2, 1, 3) if o != fmt]) if args.both else [fmt]:
+    for f in ([fmt] + [o for o in (2, 1, 3, 4) if o != fmt]) if args.both else [fmt]:
         stack, xs, ys = build_stack(f, dev, bz, torch)
         stream = torch.cuda.Stream(device=dev)
         sp = stream.cuda_stream
@@ -445,7 +457,7 @@ def run_prefill(fmt, M, dev, bz, torch, peaks, peak_kind, steps):
         t = torch.from_numpy(weights(fmt, i, N, K)).to(dev)
         packed = bz.pack(fmt, t)
         del t
-        s = torch.from_numpy(inputs.scales(i, N, K).view(np.int16)).to(dev).view(torch.float16)
+        s = torch.from_numpy(scales(fmt, i, N, K).view(np.int16)).to(dev).view(torch.float16)
         x = torch.randn((M, K), device=dev, generator=torch.Generator(device=dev).manual_seed(i)).half()
         items.append((name, K, N, packed, s, x, torch.empty((M, N), dtype=torch.float16, device=dev)))
         bz.bonsai_reserve(M, N, K)
@@ -512,7 +524,7 @@ def cpu_baseline(fmt):
     probs = []
     for i, (name, K, N) in enumerate(SHAPES):
         probs.append((inputs.activations(i, 1, K), oracle.pack(fmt, weights(fmt, i, N, K)),
-                      inputs.scales(i, N, K), N, K))
+                      scales(fmt, i, N, K), N, K))
     t0 = time.perf_counter()
     for x, p, s, N, K in probs:
         oracle.ternary_linear(x, p, s, N, K, fmt)
@@ -535,7 +547,7 @@ def run_case(args):
     t = torch.from_numpy(weights(fmt, i, N, K)).to(dev)
     packed = bz.pack(fmt, t)
     del t
-    s = torch.from_numpy(inputs.scales(i, N, K).view(np.int16)).to(dev).view(torch.float16)
+    s = torch.from_numpy(scales(fmt, i, N, K).view(np.int16)).to(dev).view(torch.float16)
     x = torch.from_numpy(inputs.activations(i, M, K).view(np.int16)).to(dev).view(torch.float16)
     y = torch.empty((M, N), dtype=torch.float16, device=dev)
     algo = {"gemv": bz.BONSAI_ALGO_GEMV, "imma": bz.BONSAI_ALGO_IMMA, "gemm": bz.BONSAI_ALGO_GEMM}[args.case]
@@ -558,7 +570,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--fmt", choices=["pq2", "ptq1", "q1"], default="pq2")
+    ap.add_argument("--fmt", choices=list(FMTS), default="pq2")
     ap.add_argument("--both", type=int, default=1, help="also measure the other packing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-m", type=int, default=2048, help="tokens of the prefill GEMM line (0: skip)")
