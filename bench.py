@@ -46,8 +46,8 @@ FMTS = {"ptq1": 1, "pq2": 2, "q1": 3, "pq2g64": 4}
 DOM_KERNEL = {1: "lookup-table GEMV (gemv_split_kernel + in-order reduction)",
               2: "integer tensor-core GEMV (gemv_imma_kernel)",
               3: "lookup-table GEMV (gemv_split_kernel, 1-bit tables + in-order reduction)",
-              4: "lookup-table GEMV (gemv_split_kernel, 64-weight scale groups + in-order reduction)"}
-DOM_SOURCE = {1: "gemv_lut.cu", 2: "gemv_imma.cu", 3: "gemv_lut.cu", 4: "gemv_lut.cu"}
+              4: "integer tensor-core GEMV (gemv_imma_kernel, 64-weight scale groups)"}
+DOM_SOURCE = {1: "gemv_lut.cu", 2: "gemv_imma.cu", 3: "gemv_lut.cu", 4: "gemv_imma.cu"}
 
 
 def weights(fmt, seed, N, K):

@@ -97,7 +97,8 @@ typedef enum {
     BONSAI_ALGO_GEMV = 2,    /* batch-1 lookup-table GEMV with split-K; M == 1 only       */
     BONSAI_ALGO_SKINNY = 3,  /* register-dequant tensor-core kernel; 1 <= M <= 16         */
     BONSAI_ALGO_GEMM = 4,    /* tcgen05/TMEM prefill GEMM on FP16 tiles; any M            */
-    BONSAI_ALGO_IMMA = 5     /* batch-1 GEMV on the integer tensor cores; M == 1, PQ2_0   */
+    BONSAI_ALGO_IMMA = 5     /* batch-1 GEMV on the integer tensor cores; M == 1, PQ2_0
+                                and PQ2_0 g64                                             */
 } bonsai_algo;
 
 /* Library version, (major << 16) | (minor << 8) | patch. */
@@ -145,8 +146,8 @@ int bonsai_hadamard128(const uint16_t *x, uint16_t *x_out, int64_t M, int64_t K,
 
 /* y = x' . Wdeq^T (definitions above) for un-rotated FP16 x: the Hadamard
  * rotation of x is applied inside the call.  Dispatch on M: M == 1 -> the
- * integer tensor-core GEMV (PQ2_0, K <= 24576) or the lookup-table GEMV (PTQ1_0,
- * Q1_0, PQ2_0 g64), 2 <= M <= 16 -> skinny tensor-core kernel (PQ2_0), otherwise
+ * integer tensor-core GEMV (PQ2_0 and PQ2_0 g64, K <= 24576) or the lookup-table GEMV
+ * (PTQ1_0, Q1_0), 2 <= M <= 16 -> skinny tensor-core kernel (PQ2_0), otherwise
  * (and for the other packings at 2 <= M <= 16) the tcgen05 GEMM.  The
  * integer GEMV holds each 128-group of x' as 16-bit fixed point with a power-of-two
  * scale (|x~| <= 2^14) before the exact integer products; the other kernels round
@@ -182,7 +183,7 @@ int bonsai_swiglu(const uint16_t *y, uint16_t *h, int64_t M, int64_t F, void *st
 /* The fused gate/up linear layer followed by SwiGLU: packed and scales hold 2F weight rows
  * (gate rows first, then up rows: the N = 2F plane of bonsai_ternary_linear) and h gets
  * the M x F result of bonsai_swiglu applied to their product with x'.  On the integer
- * tensor-core GEMV (M = 1 PQ2_0) and the prefill GEMM the step runs in the kernel's
+ * tensor-core GEMV (M = 1 PQ2_0, PQ2_0 g64) and the prefill GEMM the step runs in the kernel's
  * epilogue on the FP32 sums; the lookup-table GEMV, the skinny and the plain kernel write
  * the product to the library's workspace in FP16 and bonsai_swiglu follows. */
 int bonsai_ternary_linear_swiglu(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,

@@ -163,7 +163,7 @@ cudaError_t run_linear(int chosen, const uint16_t *x, const uint8_t *packed, con
         case BONSAI_ALGO_GEMV: return launch_gemv(x, packed, scales, y, N, K, fmt, split_k, ws, s, info);
         case BONSAI_ALGO_SKINNY: return launch_skinny(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, info);
         case BONSAI_ALGO_GEMM: return launch_gemm(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, info);
-        case BONSAI_ALGO_IMMA: return launch_gemv_imma(x, packed, scales, y, N, K, ws, s, info);
+        case BONSAI_ALGO_IMMA: return launch_gemv_imma(x, packed, scales, y, N, K, fmt, ws, s, info);
         default: return launch_linear_simple(x, packed, scales, y, M, N, K, fmt, ws, s, info);
     }
 }
@@ -366,7 +366,7 @@ int bonsai_ternary_linear_swiglu(const uint16_t *x, const uint8_t *packed, const
     if (chosen == BONSAI_ALGO_IMMA) {  // fused into the GEMV's epilogue
         rc = ensure_workspace(*st, 0, gemv_imma_zeroed_bytes(N, K), &ws);
         if (rc != BONSAI_OK) return rc;
-        return cuda_status(launch_gemv_imma(x, packed, scales, h, N, K, ws, s, st->info, F));
+        return cuda_status(launch_gemv_imma(x, packed, scales, h, N, K, fmt, ws, s, st->info, F));
     }
     if (chosen == BONSAI_ALGO_GEMM) {  // fused into the GEMM's epilogue
         rc = ensure_workspace(*st, workspace_for(chosen, M, N, K, fmt, 0, st->info), 0, &ws);

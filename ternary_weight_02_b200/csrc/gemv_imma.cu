@@ -1,7 +1,10 @@
-// gemv_imma.cu -- batch-1 (M == 1) ternary GEMV for PQ2_0 on the integer tensor cores,
-// with the block Hadamard rotation of x fused in.
+// gemv_imma.cu -- batch-1 (M == 1) ternary GEMV for PQ2_0 (one FP16 scale per 128 or per
+// 64 weights) on the integer tensor cores, with the block Hadamard rotation of x fused in.
 //
-// Operation: y[n] = sum_g s[n][g] * sum_j t[n][128g+j] * x'[128g+j], x' = blockdiag(Hn) x.
+// Operation: y[n] = sum_g s[n][g] * sum_j t[n][128g+j] * x'[128g+j], x' = blockdiag(Hn) x;
+// with 64-weight scale groups each 128-group's sum splits into two halves, each with its
+// own scale (PQ2_0 g64, the Q2_0_g64 files of "Bonsai把 27B 大模型塞进手机的极端量化方案
+// 到底靠不靠谱" (wmrh.cn), sections 快速上手 and 后端支持现状).
 // Sources: "27B 模型压到 5.95GB，推理能力还保住 98%" (allhereai.com): method paragraph
 // (trits, FP16 scale per 128 weights, block Hadamard), paragraph on running the files
 // (activation-side Hadamard), paragraph on the two packings (PQ2_0: one trit per 2-bit
@@ -20,7 +23,10 @@
 //   With c = t + 1 the PQ2_0 code of a weight, the MMA gives sum c*hi and sum c*lo
 //   exactly in int32, so sum t*x~ = 256*Dhi + Dlo - sum x~ exactly; one FP32 multiply by
 //   s * 2^-e per (row, group) follows.  (The rounding of x' to x~ is the only
-//   approximation; it is finer than FP16 for every element of the group.)
+//   approximation; it is finer than FP16 for every element of the group.)  With 64-weight
+//   scales the MMA chain runs over the group's first two 32-weight subslots, is folded
+//   with the first half's sum of x~ and scale, then over the last two: the same
+//   accumulator registers, one more fold per group.
 // * One launch.  16 warps per CTA, each feeding its own ring of item buffers (a TMA
 //   box of trits, and the item's scales by cp.async).  After waiting for the previous
 //   kernel, every CTA loads all of x (each CTA starting at a different group quad), then
@@ -55,7 +61,7 @@ constexpr int kItemRows = 32;
 constexpr int kItemK = 512;
 constexpr int kItemRowBytes = kItemK / 4;               // 128 bytes of PQ2_0 codes
 constexpr int kItemBytes = kItemRows * kItemRowBytes;   // 4096
-constexpr int kScaleRingBytes = kItemRows * 8;          // per stage: the item's 4 scales of each row
+constexpr int kScaleRingBytes = kItemRows * 16;         // per stage: the item's 4 (g64: 8) scales of each row
 constexpr int kXHalfBytes = 144;                        // one part (hi or lo) of a group's fragments, padded
 constexpr int kXGroupBytes = 2 * kXHalfBytes;
 constexpr int kStages = 2;
@@ -69,11 +75,11 @@ constexpr uint32_t kCodeMask = 0x03030303u;
 
 // Shared memory, from a 1024-byte aligned base (each 4 KB weight buffer stays 1024-byte
 // aligned, as the 128-byte swizzle of its TMA box requires):
-// [weight rings: kConsumers x kStages x 4096][scale rings: kConsumers x kStages x 256]
-// [x~ fragments G4 x 288][(64 sum x~, 2^-e / 64) x G4][slots kMaxCtaItems x 128][256 zero bytes]
-// [full barriers]
+// [weight rings: kConsumers x kStages x 4096][scale rings: kConsumers x kStages x 512]
+// [x~ fragments G4 x 288][(64 sum x~, 2^-e / 64) x G4][64 sum of the first 64 x~ x G4]
+// [slots kMaxCtaItems x 128][256 zero bytes][full barriers]
 struct Layout {
-    int sring, xfrag, sxf, slots, tcnt, zero, full, total;
+    int sring, xfrag, sxf, sxl, slots, tcnt, zero, full, total;
 };
 
 // Alignment: the weight buffers 1024 bytes (swizzled TMA destinations), the fragment,
@@ -84,7 +90,8 @@ __host__ __device__ inline Layout make_layout(int K) {
     L.sring = kConsumers * kStages * kItemBytes;
     L.xfrag = L.sring + kConsumers * kStages * kScaleRingBytes;
     L.sxf = L.xfrag + G4 * kXGroupBytes;
-    L.slots = L.sxf + G4 * 8;
+    L.sxl = L.sxf + G4 * 8;
+    L.slots = L.sxl + ((G4 * 4 + 15) & ~15);
     L.tcnt = L.slots + kMaxCtaItems * kItemRows * 4;
     L.zero = (L.tcnt + kMaxCtaTiles * 4 + 15) & ~15;  // 128-bit loads read the zero bytes
     L.full = L.zero + 256;
@@ -132,8 +139,10 @@ __device__ __forceinline__ void load_x8(const uint16_t *__restrict__ x, int g, i
 // padding per half-block put the eight lanes that load one chunk of four consecutive
 // groups on distinct shared-memory banks.  Lane l = 2*s + hb writes whole words.
 // Rotates and quantises group g (its x in r0, r1 of the group's 8 lanes) into the
-// fragment area and (64 * sum x~, 2^-e / 64) into sxf[g].
-__device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag, int2 *sxf, int g, int lane) {
+// fragment area, (64 * sum x~, 2^-e / 64) into sxf[g] and 64 * the sum of its first 64
+// x~ (lanes 0..3 of the group) into sxl[g].
+__device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag, int2 *sxf, int *sxl, int g,
+                                             int lane) {
     const int l = lane & 7;
     const unsigned int gmask = 0xffu << (lane & 24);
     float v[16];
@@ -192,8 +201,10 @@ __device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag,
         qa[i] = (int)(__float_as_uint(fmaf(v[i], sc, 12583040.0f)) - 0x4B400000u);
         sum += qa[i];
     }
-#pragma unroll
-    for (int b = 1; b < 8; b <<= 1) sum += __shfl_xor_sync(gmask, sum, b);
+    sum += __shfl_xor_sync(gmask, sum, 1);
+    sum += __shfl_xor_sync(gmask, sum, 2);
+    const int sum_lo = sum - 128 * (kGroup / 2);  // lane 0: elements 0..63
+    sum += __shfl_xor_sync(gmask, sum, 4);
     sum -= 128 * kGroup;  // the 128 added to each of the group's q
     // lane l = 2s + hb: chunk 2s + (j >> 1), byte 8 (j & 1) + 4 hb + i (element 16l + 4i + j)
     uint8_t *dst = xfrag + g * kXGroupBytes + (l >> 1) * 32 + (l & 1) * 4;
@@ -208,7 +219,10 @@ __device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag,
         *reinterpret_cast<uint32_t *>(dst + off) = whi;
         *reinterpret_cast<uint32_t *>(dst + kXHalfBytes + off) = wlo;
     }
-    if (l == 0) sxf[g] = make_int2(sum * 64, __float_as_int(f));
+    if (l == 0) {
+        sxf[g] = make_int2(sum * 64, __float_as_int(f));
+        sxl[g] = sum_lo * 64;
+    }
 }
 
 // ---------------------------------------------------------------- the GEMV
@@ -245,14 +259,20 @@ __device__ __forceinline__ void cp_async8(void *dst, const void *src, bool valid
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(saddr(dst)), "l"(src), "r"(valid ? 8 : 0)
                  : "memory");
 }
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int kPending>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// kAsyncScales: K is a multiple of 512, so an item's four scales of a row are 8 aligned
-// bytes, copied with cp.async as part of the item's copy; otherwise each lane loads the
-// scales it needs when it processes the item.
+// kAsyncScales: K is a multiple of 512, so an item's four (g64: eight) scales of a row are
+// 8 (16) aligned bytes, copied with cp.async as part of the item's copy; otherwise each
+// lane loads the scales it needs when it processes the item.
+//
+// kG64: one scale per 64 weights (scales N x K/64).
 //
 // kSwiglu: the rows are a fused gate/up projection (gate rows 0 .. F-1, up rows F .. 2F-1,
 // N = 2F) and the output is h = silu(gate) * up (F values).  Row tile v then holds gate
@@ -260,7 +280,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // TMA boxes), so that the lane that finishes row r < 16 of the tile finds the matching up
 // row in lane r + 16.  (When F % 16 != 0 the last tile's rows past gate row F - 1 belong to
 // no output and are not written; its up box reads zeros past row 2F - 1.)
-template <bool kAsyncScales, bool kSwiglu>
+template <bool kAsyncScales, bool kSwiglu, bool kG64>
 __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const __grid_constant__ CUtensorMap wmap, const uint16_t *__restrict__ x, const uint16_t *__restrict__ scales,
     uint16_t *__restrict__ y, uint64_t *__restrict__ partials, int N, int K, int F) {
@@ -270,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const int gid = lane >> 2, tig = lane & 3;
     const Layout L = make_layout(K);
     const int G = K / kGroup;
+    const int GS = kG64 ? 2 * G : G;  // scales per row
     const int KC = (K + kItemK - 1) / kItemK;
     const int G4 = KC * 4;
     const int RT = (N + kItemRows - 1) / kItemRows;
@@ -283,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const int nq = c1 - c0 > warp ? (c1 - c0 - warp + kConsumers - 1) / kConsumers : 0;  // this warp's items
 
     uint8_t *wring = smem + warp * kStages * kItemBytes;
-    uint8_t *sring = smem + L.sring + warp * kStages * kScaleRingBytes;  // [stage][item row][4 scales]
+    uint8_t *sring = smem + L.sring + warp * kStages * kScaleRingBytes;  // [stage][item row][16 bytes]
     uint8_t *xf = smem + L.xfrag;
     const int2 *sxf = reinterpret_cast<const int2 *>(smem + L.sxf);
     float *slots = reinterpret_cast<float *>(smem + L.slots);
@@ -321,7 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
             if (kAsyncScales) {
                 const int row = row_of(rt, lane);
                 const bool v = row < N;
-                cp_async8(sring + st * kScaleRingBytes + lane * 8, scales + (v ? (int64_t)row * G + kc * 4 : 0), v);
+                if (kG64)
+                    cp_async16(sring + st * kScaleRingBytes + lane * 16, scales + (v ? (int64_t)row * GS + kc * 8 : 0), v);
+                else
+                    cp_async8(sring + st * kScaleRingBytes + lane * 16, scales + (v ? (int64_t)row * GS + kc * 4 : 0), v);
             }
             n_issued++;
         }
@@ -362,8 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
             int pq = quad + rot;
             if (pq >= nquads) pq -= nquads;
             if (quad < nquads)  // whole warps
-                build_group8(xr[r][0], xr[r][1], xf, reinterpret_cast<int2 *>(smem + L.sxf), pq * 4 + (lane >> 3),
-                             lane);
+                build_group8(xr[r][0], xr[r][1], xf, reinterpret_cast<int2 *>(smem + L.sxf),
+                             reinterpret_cast<int *>(smem + L.sxl), pq * 4 + (lane >> 3), lane);
         }
         for (int q = kFirstIssue; q < kStages; q++) issue(q);
     }
@@ -438,19 +462,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
                 raw[t][h][1] = *reinterpret_cast<const uint4 *>(sb + loff1 + 2048 * t + 1024 * h);
             }
         const int g0 = kc * 4;
-        uint32_t sc[4];  // (t, h) = (e >> 1, e & 1): scale of row 16t + 8h + gid, group g0 + tig
+        // (t, h) = (e >> 1, e & 1): scale of row 16t + 8h + gid, group g0 + tig (g64: the
+        // group's two half scales, first half in the low 16 bits)
+        uint32_t sc[4];
         if (kAsyncScales) {
             cp_async_wait<kStages - 1>();  // this item's scales have landed (own copies)
             __syncwarp();                  // ... and every lane's
-            const uint8_t *sp = sring + st * kScaleRingBytes + gid * 8 + tig * 2;
+            const uint8_t *sp = sring + st * kScaleRingBytes + gid * 16 + tig * (kG64 ? 4 : 2);
 #pragma unroll
-            for (int e = 0; e < 4; e++) sc[e] = *reinterpret_cast<const uint16_t *>(sp + e * 64);
+            for (int e = 0; e < 4; e++)
+                sc[e] = kG64 ? *reinterpret_cast<const uint32_t *>(sp + e * 128)
+                             : (uint32_t)*reinterpret_cast<const uint16_t *>(sp + e * 128);
         } else {
             const int g = g0 + tig;
 #pragma unroll
             for (int e = 0; e < 4; e++) {
                 const int row = row_of(rt, 8 * e + gid);
-                sc[e] = (row < N && g < G) ? (uint32_t)__ldg(scales + (int64_t)row * G + g) : 0u;
+                const bool v = row < N && g < G;
+                if (kG64)
+                    sc[e] = v ? (uint32_t)__ldg(scales + (int64_t)row * GS + 2 * g) |
+                                    ((uint32_t)__ldg(scales + (int64_t)row * GS + 2 * g + 1) << 16)
+                              : 0u;
+                else
+                    sc[e] = v ? (uint32_t)__ldg(scales + (int64_t)row * GS + g) : 0u;
             }
         }
         __syncwarp();
@@ -463,11 +497,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
 
         // Codes stay in place: (w & 0x03030303 << 2j) gives code slot j of the four bytes of
         // a word as u8 values c * 4^j.  One accumulator per (tile, j); the 4^j factors are
-        // undone once per item (the sums come out 64 times too large, folded into 2^-e).
+        // undone once per fold (the sums come out 64 times too large, folded into 2^-e).
+        // One fold per group, or (g64) one per 64-weight half: subslots 0, 1 then 2, 3.
+        constexpr int kFolds = kG64 ? 2 : 1, kSubPerFold = 4 / kFolds;
         int d[2][4][4];
         const uint8_t *xb = xb_lane + g0 * xb_stride;
+        const int2 sf = sxf[g0 + tig];  // (64 * sum x~, 2^-e / 64)
+        const float fg = __int_as_float(sf.y);
+        const int sfl = kG64 ? reinterpret_cast<const int *>(smem + L.sxl)[g0 + tig] : 0;  // first half's
+        float v[4] = {0.f, 0.f, 0.f, 0.f};  // (t, h) = (e >> 1, e & 1)
 #pragma unroll
-        for (int s = 0; s < 4; s++) {
+        for (int fold = 0; fold < kFolds; fold++) {
+#pragma unroll
+        for (int s = fold * kSubPerFold; s < (fold + 1) * kSubPerFold; s++) {
             const uint4 b01 = *reinterpret_cast<const uint4 *>(xb + 32 * s);       // code slots 0, 1
             const uint4 b23 = *reinterpret_cast<const uint4 *>(xb + 32 * s + 16);  // code slots 2, 3
 #pragma unroll
@@ -481,26 +523,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
                     const uint4 &r0 = raw[t][0][s >> 1], &r1 = raw[t][1][s >> 1];
                     const uint32_t w0 = (s & 1) ? r0.z : r0.x, w2 = (s & 1) ? r0.w : r0.y;
                     const uint32_t w1 = (s & 1) ? r1.z : r1.x, w3 = (s & 1) ? r1.w : r1.y;
-                    if (s == 0)
+                    if (s == fold * kSubPerFold)
                         imma0(d[t][j], w0 & mask, w1 & mask, w2 & mask, w3 & mask, bx, by);
                     else
                         imma(d[t][j], w0 & mask, w1 & mask, w2 & mask, w3 & mask, bx, by);
                 }
             }
         }
-        // lane (gid, tig) holds columns 2tig (hi) and 2tig+1 (lo): group g0 + tig of rows
-        // gid (d[t][j][0..1]) and gid + 8 (d[t][j][2..3])
-        const int2 sf = sxf[g0 + tig];  // (64 * sum x~, 2^-e / 64)
-        const float fg = __int_as_float(sf.y);
-        float v[4];  // (t, h) = (e >> 1, e & 1)
+        // lane (gid, tig) holds columns 2tig (hi) and 2tig+1 (lo): group g0 + tig (g64: its
+        // half `fold`) of rows gid (d[t][j][0..1]) and gid + 8 (d[t][j][2..3])
+        const int sx = kG64 ? (fold == 0 ? sfl : sf.x - sfl) : sf.x;  // 64 * sum of the fold's x~
 #pragma unroll
         for (int e = 0; e < 4; e++) {
             const int t = e >> 1, h = e & 1;
             const int H = ((d[t][0][2 * h] * 4 + d[t][1][2 * h]) * 4 + d[t][2][2 * h]) * 4 + d[t][3][2 * h];
             const int Lo = ((d[t][0][2 * h + 1] * 4 + d[t][1][2 * h + 1]) * 4 + d[t][2][2 * h + 1]) * 4 +
                            d[t][3][2 * h + 1];
-            const int T64 = H * 256 + Lo - sf.x;
-            v[e] = (float)T64 * (half_bits_to_float((uint16_t)sc[e]) * fg);
+            const int T64 = H * 256 + Lo - sx;
+            const uint16_t sbits = (uint16_t)(kG64 && fold == 1 ? sc[e] >> 16 : sc[e]);
+            v[e] = fmaf((float)T64, half_bits_to_float(sbits) * fg, v[e]);
+        }
         }
         // sum over the four groups (lanes of the quad) and leave (t, h) = (tig >> 1, tig & 1)
         // in lane tig: keep the pair whose h is the lane's, then the t
@@ -567,13 +609,13 @@ Shape shape_of(int64_t N, int64_t K, int sm_count) {
 
 }  // namespace
 
-static_assert(kConsumers * kStages * (kItemBytes + kScaleRingBytes) + (kMaxK / kItemK) * 4 * (kXGroupBytes + 8) +
+static_assert(kConsumers * kStages * (kItemBytes + kScaleRingBytes) + (kMaxK / kItemK) * 4 * (kXGroupBytes + 12) +
                   kMaxCtaItems * kItemRows * 4 + kMaxCtaTiles * 4 + 15 + 256 + kConsumers * kStages * 8 + 1024 <=
                   232448,
               "shared-memory layout exceeds the per-CTA limit at the largest K");
 
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt) {
-    if (fmt != 2 || M != 1 || N < 1 || K < kGroup || K % kGroup != 0 || K > kMaxK) return false;
+    if ((fmt != 2 && fmt != 4) || M != 1 || N < 1 || K < kGroup || K % kGroup != 0 || K > kMaxK) return false;
     const int64_t RT = (N + kItemRows - 1) / kItemRows;
     return RT * ((K + kItemK - 1) / kItemK) < ((int64_t)1 << 30);
 }
@@ -588,8 +630,9 @@ size_t gemv_imma_zeroed_bytes(int64_t N, int64_t K) {
 }
 
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
-                             int64_t N, int64_t K, const Workspace &ws, cudaStream_t s, const DeviceInfo &dev,
-                             int64_t swiglu_f) {
+                             int64_t N, int64_t K, int fmt, const Workspace &ws, cudaStream_t s,
+                             const DeviceInfo &dev, int64_t swiglu_f) {
+    if (fmt != 2 && fmt != 4) return cudaErrorInvalidValue;
     const bool swiglu = swiglu_f > 0;
     if (swiglu && N != 2 * swiglu_f) return cudaErrorInvalidValue;
     const Layout lay = make_layout((int)K);
@@ -603,7 +646,7 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
     {
         const cuuint64_t dims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
         const cuuint64_t strides[1] = {(cuuint64_t)(K / 4)};
-        const cuuint32_t box[2] = {kItemRowBytes, swiglu ? kItemRows / 2 : kItemRows};
+        const cuuint32_t box[2] = {(cuuint32_t)kItemRowBytes, (cuuint32_t)(swiglu ? kItemRows / 2 : kItemRows)};
         const cuuint32_t estr[2] = {1, 1};
         if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -613,9 +656,17 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
     const Shape sh = shape_of(N, K, dev.sm_count);
     if (ws.zeroed_bytes < gemv_imma_zeroed_bytes(N, K)) return cudaErrorInvalidValue;
     uint64_t *partials = reinterpret_cast<uint64_t *>(ws.zeroed);
-    // K a multiple of 512: an item's scales of a row are 8 aligned bytes, copied with the item
-    auto kern = K % kItemK == 0 ? (swiglu ? gemv_imma_kernel<true, true> : gemv_imma_kernel<true, false>)
-                                : (swiglu ? gemv_imma_kernel<false, true> : gemv_imma_kernel<false, false>);
+    // K a multiple of 512: an item's scales of a row are 8 (g64: 16) aligned bytes, copied
+    // with the item
+    using Kern = decltype(&gemv_imma_kernel<true, true, true>);
+    const bool async = K % kItemK == 0;
+    Kern kern;
+    if (fmt == 4)
+        kern = async ? (swiglu ? gemv_imma_kernel<true, true, true> : gemv_imma_kernel<true, false, true>)
+                     : (swiglu ? gemv_imma_kernel<false, true, true> : gemv_imma_kernel<false, false, true>);
+    else
+        kern = async ? (swiglu ? gemv_imma_kernel<true, true, false> : gemv_imma_kernel<true, false, false>)
+                     : (swiglu ? gemv_imma_kernel<false, true, false> : gemv_imma_kernel<false, false, false>);
     // the attribute is set to the largest layout any K takes, so that launches of several
     // sizes captured into one graph all stay within it
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -81,8 +81,8 @@ int current_device_info(DeviceInfo *out);
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t gemv_imma_zeroed_bytes(int64_t N, int64_t K);  // of Workspace::zeroed
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
-                             int64_t N, int64_t K, const Workspace &ws, cudaStream_t s, const DeviceInfo &dev,
-                             int64_t swiglu_f = 0);  // > 0: fused gate/up rows, write silu(gate) * up
+                             int64_t N, int64_t K, int fmt, const Workspace &ws, cudaStream_t s,
+                             const DeviceInfo &dev, int64_t swiglu_f = 0);  // > 0: fused gate/up rows, write silu(gate) * up
 
 // ---- skinny_mma.cu: 1 <= M <= 16
 bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt);

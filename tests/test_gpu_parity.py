@@ -214,7 +214,7 @@ def test_gemv_decode_shapes_full(bz, fmt, K, N):
     got = _run(bz, p, bz.BONSAI_ALGO_GEMV)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
-    if fmt in (PTQ1, Q1, G64):  # through the default entry point too (M == 1 dispatches here)
+    if fmt in (PTQ1, Q1):  # through the default entry point too (M == 1 dispatches here)
         import torch
         x, packed, scales = p.device()
         y = torch.empty((1, N), dtype=torch.float16, device="cuda")
@@ -268,29 +268,31 @@ IMMA_CASES = [(1, 128), (33, 384), (31, 640), (100, 1024), (1024, 1024), (1000, 
               (20000, 8192), (12000, 10752)]
 
 
+@pytest.mark.parametrize("fmt", [PQ2, G64])
 @pytest.mark.parametrize("N,K", IMMA_CASES)
-def test_imma_small(bz, N, K):
-    p = Problem(1, N, K, PQ2, seed=N + 5 * K)
+def test_imma_small(bz, fmt, N, K):
+    p = Problem(1, N, K, fmt, seed=N + 5 * K)
     got = _run(bz, p, bz.BONSAI_ALGO_IMMA)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
 
 
+@pytest.mark.parametrize("fmt", [PQ2, G64])
 @pytest.mark.parametrize("K,N", DECODE_SHAPES)
-def test_imma_decode_shapes_full(bz, K, N):
-    """Every output of the full-size M=1 PQ2_0 projections against the float64 checker,
-    and the default entry point (which dispatches M == 1 PQ2_0 here) bit-equal to it."""
+def test_imma_decode_shapes_full(bz, fmt, K, N):
+    """Every output of the full-size M=1 PQ2_0 (and g64) projections against the float64
+    checker, and the default entry point (which dispatches M == 1 here) bit-equal to it."""
     import torch
-    p = Problem(1, N, K, PQ2, seed=0)
+    p = Problem(1, N, K, fmt, seed=0)
     got = _run(bz, p, bz.BONSAI_ALGO_IMMA)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
     x, packed, scales = p.device()
     y = torch.empty((1, N), dtype=torch.float16, device="cuda")
-    bz.bonsai_ternary_linear(x, packed, scales, y, 1, N, K, PQ2)
+    bz.bonsai_ternary_linear(x, packed, scales, y, 1, N, K, fmt)
     torch.cuda.synchronize()
     assert np.array_equal(to_numpy_f16(y), got)
-    assert bz.bonsai_launch_count(1, N, K, PQ2) == 1
+    assert bz.bonsai_launch_count(1, N, K, fmt) == 1
 
 
 def test_imma_repeatable_and_counters_reset(bz):
@@ -301,13 +303,14 @@ def test_imma_repeatable_and_counters_reset(bz):
     import torch
     probs = [Problem(1, 3000, 5120, PQ2, seed=1), Problem(1, 77, 17408, PQ2, seed=2),
              Problem(1, 34816, 5120, PQ2, seed=4), Problem(1, 5120, 17408, PQ2, seed=3),
-             Problem(1, 20000, 8192, PQ2, seed=5)]
+             Problem(1, 20000, 8192, PQ2, seed=5), Problem(1, 34816, 5120, G64, seed=6),
+             Problem(1, 5000, 1152, G64, seed=7)]
     devs = [p.device() for p in probs]
     outs = []
     for _ in range(3):
         for p, (x, packed, scales) in zip(probs, devs):
             y = torch.empty((1, p.N), dtype=torch.float16, device="cuda")
-            bz.bonsai_ternary_linear_algo(x, packed, scales, y, 1, p.N, p.K, PQ2, bz.BONSAI_ALGO_IMMA, 0)
+            bz.bonsai_ternary_linear_algo(x, packed, scales, y, 1, p.N, p.K, p.fmt, bz.BONSAI_ALGO_IMMA, 0)
             outs.append(y)
     torch.cuda.synchronize()
     n = len(probs)
@@ -317,10 +320,10 @@ def test_imma_repeatable_and_counters_reset(bz):
         assert oracle.compare(to_numpy_f16(outs[i]), p.oracle_y())[0]
 
 
-def test_imma_input_with_large_and_small_groups(bz):
+@pytest.mark.parametrize("fmt", [PQ2, G64])
+def test_imma_input_with_large_and_small_groups(bz, fmt):
     """Groups of x whose magnitudes differ by 2^20 get their own power-of-two scales."""
-    import torch
-    p = Problem(1, 256, 2048, PQ2, seed=9)
+    p = Problem(1, 256, 2048, fmt, seed=9)
     xs = p.x.astype(np.float32)
     for g in range(16):
         xs[:, 128 * g:128 * (g + 1)] *= 2.0 ** (5 if g % 2 else -15)
@@ -500,14 +503,15 @@ def _run_swiglu(bz, p, F):
     return to_numpy_f16(h)
 
 
-# (M, F, K, fmt): fused in the integer GEMV (M = 1 PQ2_0; F = 24 leaves a part-used last
+# (M, F, K, fmt): fused in the integer GEMV (M = 1 PQ2_0 and g64; F = 24 leaves a part-used last
 # tile; the last case is the full 27B-class gate/up) or the GEMM (tiles split between
 # CTAs; F = 200 and 1270 part-used); the other packings at M = 1 and the skinny batches
 # take the linear kernel and then the SwiGLU kernel
 SWIGLU_CASES = [(1, 16, 512, PQ2), (1, 1024, 2048, PQ2), (1, 4000, 1152, PQ2), (1, 24, 512, PQ2),
                 (1, 1024, 1024, PTQ1), (1, 1024, 2048, Q1), (4, 512, 1024, PQ2), (300, 640, 640, PQ2),
                 (300, 640, 640, Q1), (300, 384, 1152, PTQ1), (600, 1280, 384, PQ2), (300, 200, 640, PQ2), (300, 1270, 256, Q1),
-                (1, 1024, 2048, G64), (300, 200, 640, G64), (600, 1280, 384, G64), (1, 17408, 5120, PQ2)]
+                (1, 1024, 2048, G64), (1, 24, 512, G64), (1, 4000, 1152, G64), (300, 200, 640, G64),
+                (600, 1280, 384, G64), (1, 17408, 5120, PQ2), (1, 17408, 5120, G64)]
 
 
 @pytest.mark.parametrize("M,F,K,fmt", SWIGLU_CASES)
