@@ -550,7 +550,8 @@ def run_case(args):
     s = torch.from_numpy(scales(fmt, i, N, K).view(np.int16)).to(dev).view(torch.float16)
     x = torch.from_numpy(inputs.activations(i, M, K).view(np.int16)).to(dev).view(torch.float16)
     y = torch.empty((M, N), dtype=torch.float16, device=dev)
-    algo = {"gemv": bz.BONSAI_ALGO_GEMV, "imma": bz.BONSAI_ALGO_IMMA, "gemm": bz.BONSAI_ALGO_GEMM}[args.case]
+    algo = {"gemv": bz.BONSAI_ALGO_GEMV, "imma": bz.BONSAI_ALGO_IMMA, "gemm": bz.BONSAI_ALGO_GEMM,
+            "skinny": bz.BONSAI_ALGO_SKINNY}[args.case]
     bz.bonsai_reserve(M, N, K)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -574,9 +575,9 @@ def main():
     ap.add_argument("--both", type=int, default=1, help="also measure the other packing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-m", type=int, default=2048, help="tokens of the prefill GEMM line (0: skip)")
-    ap.add_argument("--case", choices=["gemv", "imma", "gemm"], help="run one projection only (profiler case)")
+    ap.add_argument("--case", choices=["gemv", "imma", "gemm", "skinny"], help="run one projection only (profiler case)")
     ap.add_argument("--shape", choices=[n for n, _, _ in SHAPES], default="gate_up")
-    ap.add_argument("--m", type=int, default=2048, help="tokens for --case gemm")
+    ap.add_argument("--m", type=int, default=2048, help="tokens for --case gemm / skinny (skinny: at most 16)")
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

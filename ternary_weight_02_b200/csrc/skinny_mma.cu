@@ -1,4 +1,5 @@
-// skinny_mma.cu -- ternary linear layer for small batches (1 <= M <= 16 tokens), PQ2_0.
+// skinny_mma.cu -- ternary linear layer for small batches (1 <= M <= 16 tokens), PQ2_0
+// with one FP16 scale per 128 or per 64 weights.
 //
 // y[m][n] = sum_g s[n][g] * sum_j t[n][128g+j] * x'[m][128g+j].  Sources: "27B 模型压到
 // 5.95GB，推理能力还保住 98%" (allhereai.com): method paragraph (trits, FP16 group
@@ -27,6 +28,11 @@
 // * A warp owns 16 weight rows; a CTA 128 rows and one K chunk.  Split-K: chunks
 //   write FP32 partials; the warp that brings a row block's last chunk sums them in
 //   chunk order (deterministic) and writes y.
+// * 64-weight scales (PQ2_0 g64, the Q2_0_g64 files of "Bonsai把 27B 大模型塞进手机的极端
+//   量化方案到底靠不靠谱" (wmrh.cn), sections 快速上手 and 后端支持现状): lane quad member tq
+//   takes words tq and tq + 4 of the group instead of 2tq and 2tq + 1, so that MMAs 0-3
+//   cover the group's first 64 weights and MMAs 4-7 the last 64; each half has its own
+//   accumulator, scale and sum of x'.
 #include "common.cuh"
 #include "internal.h"
 
@@ -43,7 +49,8 @@ template <int NT>
 constexpr int sub_groups() { return NT == 1 ? 48 : 24; }
 
 // One 128-weight group of the warp's rows r0 = gid and r1 = gid + 8, as lane (gid, tq)
-// holds it: words 2tq and 2tq + 1 (8 bytes) of each row, and the two FP16 scales.
+// holds it: words 2tq and 2tq + 1 (g64: tq and tq + 4) of each row, and the rows' FP16
+// scales (g64: both halves' scales, the first in the low 16 bits).
 struct Grp {
     uint2 a, b;
     uint32_t s0, s1;
@@ -60,16 +67,20 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 
 // K order of the MMAs: MMA i of a group takes, from lane quad member tq, byte (i & 3) of
 // group word 2tq + (i >> 2), i.e. the four weights 32tq + 16(i >> 2) + 4(i & 3) + c,
-// c = 0..3, which sit at B slots 4tq + c of the MMA's 16-half row of x'.
+// c = 0..3, which sit at B slots 4tq + c of the MMA's 16-half row of x'.  g64: byte
+// (i & 3) of word tq + 4(i >> 2), weights 64(i >> 2) + 16tq + 4(i & 3) + c.
+template <bool kG64>
 __device__ __forceinline__ int64_t skinny_k(int64_t group, int step, int tq) {
-    return group * kGroup + 32 * tq + 16 * (step >> 2) + 4 * (step & 3);
+    return kG64 ? group * kGroup + 64 * (step >> 2) + 16 * tq + 4 * (step & 3)
+                : group * kGroup + 32 * tq + 16 * (step >> 2) + 4 * (step & 3);
 }
 
 // The rotation pass of this kernel: one warp per (group g, token m < MT).  It writes x'
 // (FP16, nearest) of the block in the layout the MMAs read, [g][step][token][16] with
 // slot 4tq + c = element skinny_k(g, step, tq) + c scaled by 4^-c, zeros for the padding
-// tokens m >= M, and the FP32 sum of the block's FP16 x' values to gsum[g][m].
-template <int MT>
+// tokens m >= M, and the FP32 sum of the block's FP16 x' values to gsum[g][m] (g64: the
+// sums of its two 64-element halves to gsum[g][h][m]).
+template <int MT, bool kG64>
 __global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ xs,
                                                           float *__restrict__ gsum, int M, int64_t K) {
     const int lane = threadIdx.x & 31;
@@ -85,17 +96,28 @@ __global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__rest
     }
     const __half2 h01 = __floats2half2_rn(v[0], v[1]), h23 = __floats2half2_rn(v[2], v[3]);
     const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-    const float sum = warp_sum((f01.x + f01.y) + (f23.x + f23.y));
+    float sum = (f01.x + f01.y) + (f23.x + f23.y);
+    if (kG64) {  // lanes 0..15 hold the first 64 elements, 16..31 the last 64
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    } else {
+        sum = warp_sum(sum);
+    }
     // lane l holds elements 4l .. 4l+3 = skinny_k(g, i, tq) + c with tq = l >> 3 and
-    // i = 4 ((l >> 2) & 1) + (l & 3)
-    const int tq = lane >> 3, i = 4 * ((lane >> 2) & 1) + (lane & 3);
+    // i = 4 ((l >> 2) & 1) + (l & 3) (g64: tq = (l >> 2) & 3, i = 4 (l >> 4) + (l & 3))
+    const int tq = kG64 ? (lane >> 2) & 3 : lane >> 3;
+    const int i = kG64 ? 4 * (lane >> 4) + (lane & 3) : 4 * ((lane >> 2) & 1) + (lane & 3);
     const __half2 s01 = __hmul2(h01, __floats2half2_rn(1.f, 0.25f));
     const __half2 s23 = __hmul2(h23, __floats2half2_rn(0.0625f, 0.015625f));
     uint2 out;
     out.x = *reinterpret_cast<const uint32_t *>(&s01);
     out.y = *reinterpret_cast<const uint32_t *>(&s23);
     *reinterpret_cast<uint2 *>(xs + ((g * 8 + i) * MT + m) * 16 + 4 * tq) = out;
-    if (lane == 0) gsum[g * MT + m] = sum;
+    if (kG64) {
+        if ((lane & 15) == 0) gsum[(g * 2 + (lane >> 4)) * MT + m] = sum;
+    } else if (lane == 0) {
+        gsum[g * MT + m] = sum;
+    }
 }
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
@@ -104,7 +126,7 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
                  : "memory");
 }
 
-template <int NT>  // n8 token tiles: 1 (M <= 8) or 2 (M <= 16)
+template <int NT, bool kG64>  // n8 token tiles: 1 (M <= 8) or 2 (M <= 16); 64-weight scales
 __global__ void __launch_bounds__(kThreads) skinny_kernel(
     const uint16_t *__restrict__ xsg, const float *__restrict__ gsg, const uint8_t *__restrict__ packed,
     const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
@@ -114,8 +136,9 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
     // groups staged at a time: the whole chunk when it fits (shared memory is sized so)
     const int kSub = gpc < sub_groups<NT>() ? gpc : sub_groups<NT>();
     extern __shared__ __align__(16) uint8_t smem[];
+    constexpr int kHalves = kG64 ? 2 : 1;  // scale groups per 128 weights
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [kSub * 8 steps][MT][16]
-    float *gsum = reinterpret_cast<float *>(smem + kSub * 8 * MT * 32);  // [MT][kSub]
+    float *gsum = reinterpret_cast<float *>(smem + kSub * 8 * MT * 32);  // [MT][kSub][kHalves]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tq = lane & 3;
@@ -133,16 +156,27 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
 #pragma unroll
         for (int e = 0; e < 4; e++) acc[nt][e] = 0.f;
 
+    auto row_words = [&](int64_t r, int g) -> uint2 {
+        const uint8_t *p = packed + (r * G + g) * kPq2GroupBytes;
+        if (kG64)
+            return make_uint2(__ldcs(reinterpret_cast<const unsigned int *>(p) + tq),
+                              __ldcs(reinterpret_cast<const unsigned int *>(p) + tq + 4));
+        return __ldcs(reinterpret_cast<const uint2 *>(p) + tq);
+    };
+    auto row_scales = [&](int64_t r, int g) -> uint32_t {
+        if (kG64) return __ldg(reinterpret_cast<const unsigned int *>(scales + r * 2 * G + 2 * g));
+        return __ldg(scales + r * G + g);
+    };
     auto load = [&](int g, Grp &q) {
         if (v0) {
-            q.a = __ldcs(reinterpret_cast<const uint2 *>(packed + (r0 * G + g) * kPq2GroupBytes) + tq);
-            q.s0 = __ldg(scales + r0 * G + g);
+            q.a = row_words(r0, g);
+            q.s0 = row_scales(r0, g);
         } else {
             q.a = make_uint2(0x55555555u, 0x55555555u), q.s0 = 0u;  // trits 0
         }
         if (v1) {
-            q.b = __ldcs(reinterpret_cast<const uint2 *>(packed + (r1 * G + g) * kPq2GroupBytes) + tq);
-            q.s1 = __ldg(scales + r1 * G + g);
+            q.b = row_words(r1, g);
+            q.s1 = row_scales(r1, g);
         } else {
             q.b = make_uint2(0x55555555u, 0x55555555u), q.s1 = 0u;
         }
@@ -165,9 +199,9 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
             for (int off = tid * 16; off < bytes; off += kThreads * 16)
                 cp_async16(reinterpret_cast<uint8_t *>(xs) + off, src + off);
             asm volatile("cp.async.commit_group;" ::: "memory");
-            for (int idx = tid; idx < nsub * MT; idx += kThreads) {
-                const int gl = idx / MT, m = idx % MT;
-                gsum[m * kSub + gl] = gsg[(int64_t)(sub + gl) * MT + m];
+            for (int idx = tid; idx < nsub * MT * kHalves; idx += kThreads) {
+                const int gh = idx / MT, m = idx % MT;  // gh = kHalves * gl + h
+                gsum[m * kSub * kHalves + gh] = gsg[((int64_t)sub * kHalves + gh) * MT + m];
             }
             asm volatile("cp.async.wait_all;" ::: "memory");
         }
@@ -179,11 +213,13 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
                 const int gl = gl0 + u;
                 if (gl >= nsub) break;
                 Grp &cur = ring[u];
-                float d[NT][4];
+                float d[kHalves][NT][4];  // g64: MMAs 0-3 and 4-7 fill the two halves
 #pragma unroll
-                for (int nt = 0; nt < NT; nt++)
+                for (int h = 0; h < kHalves; h++)
 #pragma unroll
-                    for (int e = 0; e < 4; e++) d[nt][e] = 0.f;
+                    for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+                        for (int e = 0; e < 4; e++) d[h][nt][e] = 0.f;
 #pragma unroll
                 for (int i = 0; i < 8; i++) {
                     // byte (i & 3) of the lane's word i >> 2, in both halves: (c0, c1) and
@@ -197,19 +233,24 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
 #pragma unroll
                     for (int nt = 0; nt < NT; nt++) {
                         const uint2 b = *reinterpret_cast<const uint2 *>(xs + ((ks * MT + nt * 8 + gid) * 16 + tq * 4));
-                        mma16816(d[nt], a0, a1, a2, a3, b.x, b.y);
+                        mma16816(d[kG64 ? i >> 2 : 0][nt], a0, a1, a2, a3, b.x, b.y);
                     }
                 }
-                const float cs0 = half_bits_to_float((uint16_t)cur.s0), cs1 = half_bits_to_float((uint16_t)cur.s1);
 #pragma unroll
-                for (int nt = 0; nt < NT; nt++) {
-                    const int m0 = nt * 8 + 2 * tq;
-                    const float gs0 = gsum[m0 * kSub + gl], gs1 = gsum[(m0 + 1) * kSub + gl];
-                    // d[0], d[1]: row r0, tokens m0, m0+1; d[2], d[3]: row r1
-                    acc[nt][0] = fmaf(cs0, fmaf(d[nt][0], 16777216.f, -gs0), acc[nt][0]);
-                    acc[nt][1] = fmaf(cs0, fmaf(d[nt][1], 16777216.f, -gs1), acc[nt][1]);
-                    acc[nt][2] = fmaf(cs1, fmaf(d[nt][2], 16777216.f, -gs0), acc[nt][2]);
-                    acc[nt][3] = fmaf(cs1, fmaf(d[nt][3], 16777216.f, -gs1), acc[nt][3]);
+                for (int h = 0; h < kHalves; h++) {
+                    const float cs0 = half_bits_to_float((uint16_t)(cur.s0 >> (16 * h)));
+                    const float cs1 = half_bits_to_float((uint16_t)(cur.s1 >> (16 * h)));
+#pragma unroll
+                    for (int nt = 0; nt < NT; nt++) {
+                        const int m0 = nt * 8 + 2 * tq;
+                        const float gs0 = gsum[m0 * kSub * kHalves + gl * kHalves + h];
+                        const float gs1 = gsum[(m0 + 1) * kSub * kHalves + gl * kHalves + h];
+                        // d[h][nt][0], [1]: row r0, tokens m0, m0+1; [2], [3]: row r1
+                        acc[nt][0] = fmaf(cs0, fmaf(d[h][nt][0], 16777216.f, -gs0), acc[nt][0]);
+                        acc[nt][1] = fmaf(cs0, fmaf(d[h][nt][1], 16777216.f, -gs1), acc[nt][1]);
+                        acc[nt][2] = fmaf(cs1, fmaf(d[h][nt][2], 16777216.f, -gs0), acc[nt][2]);
+                        acc[nt][3] = fmaf(cs1, fmaf(d[h][nt][3], 16777216.f, -gs1), acc[nt][3]);
+                    }
                 }
                 const int g = sub + gl;
                 if (g + kRing < g_end) load(g + kRing, cur);  // refill the slot
@@ -258,10 +299,10 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
     if (lane == 0) counters[rb] = 0u;
 }
 
-int smem_bytes(int NT, int gpc) {
+int smem_bytes(int NT, int gpc, bool g64) {
     int sub = NT == 1 ? sub_groups<1>() : sub_groups<2>();
     sub = gpc < sub ? gpc : sub;
-    return sub * 8 * NT * 8 * 32 + NT * 8 * sub * 4;
+    return sub * 8 * NT * 8 * 32 + NT * 8 * sub * 4 * (g64 ? 2 : 1);
 }
 
 // K chunks: about as many CTAs as fit on the GPU at once (one wave; a CTA's registers
@@ -277,21 +318,21 @@ void choose_split(int64_t N, int64_t K, int split_k, const DeviceInfo &dev, int 
     *S = (int)((G + per - 1) / per);
 }
 
-// Workspace: the staged x' ([G][8][MT][16] FP16), the group sums ([G][MT] FP32), then the
-// split-K partials.
+// Workspace: the staged x' ([G][8][MT][16] FP16), the group sums ([G][MT] FP32; g64
+// [G][2][MT]), then the split-K partials.
 size_t staged_bytes(int64_t M, int64_t K) {
     const int64_t MT = M <= 8 ? 8 : 16;
     return ((size_t)(K / kGroup) * 8 * MT * 32 + 255) / 256 * 256;
 }
-size_t gsum_bytes(int64_t M, int64_t K) {
+size_t gsum_bytes(int64_t M, int64_t K) {  // room for the g64 half sums
     const int64_t MT = M <= 8 ? 8 : 16;
-    return ((size_t)(K / kGroup) * MT * 4 + 255) / 256 * 256;
+    return ((size_t)(K / kGroup) * 2 * MT * 4 + 255) / 256 * 256;
 }
 
 }  // namespace
 
 bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt) {
-    return fmt == 2 && M >= 1 && M <= 16 && K % kGroup == 0 && (N + 15) / 16 <= kMaxTiles &&
+    return (fmt == 2 || fmt == 4) && M >= 1 && M <= 16 && K % kGroup == 0 && (N + 15) / 16 <= kMaxTiles &&
            K < ((int64_t)1 << 31);
 }
 
@@ -305,7 +346,7 @@ size_t skinny_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int spli
 cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                           uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int split_k,
                           const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
-    (void)fmt;
+    if (fmt != 2 && fmt != 4) return cudaErrorInvalidValue;
     uint16_t *xsg = reinterpret_cast<uint16_t *>(ws.data);
     float *gsg = reinterpret_cast<float *>(ws.data + staged_bytes(M, K));
     float *partials = reinterpret_cast<float *>(ws.data + staged_bytes(M, K) + gsum_bytes(M, K));
@@ -313,21 +354,20 @@ cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16
     choose_split(N, K, split_k, dev, &S, &gpc);
     const dim3 grid((unsigned)((N + kRowsPerCta - 1) / kRowsPerCta), (unsigned)S);
     const int64_t G = K / kGroup;
-    cudaError_t err;
-    if (M <= 8) {
-        skinny_prep_kernel<8><<<(unsigned)((G * 8 + 7) / 8), 256, 0, s>>>(x, xsg, gsg, (int)M, K);
-        err = cudaFuncSetAttribute(skinny_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(1, gpc));
+    const bool g64 = fmt == 4;
+    auto run = [&](auto prep, auto kern, int MT, int NT) -> cudaError_t {
+        prep<<<(unsigned)((G * MT + 7) / 8), 256, 0, s>>>(x, xsg, gsg, (int)M, K);
+        const int smem = smem_bytes(NT, gpc, g64);
+        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err != cudaSuccess) return err;
-        skinny_kernel<1><<<grid, kThreads, smem_bytes(1, gpc), s>>>(xsg, gsg, packed, scales, y, partials, ws.counters,
-                                                               (int)M, N, K, S, gpc);
-    } else {
-        skinny_prep_kernel<16><<<(unsigned)((G * 16 + 7) / 8), 256, 0, s>>>(x, xsg, gsg, (int)M, K);
-        err = cudaFuncSetAttribute(skinny_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes(2, gpc));
-        if (err != cudaSuccess) return err;
-        skinny_kernel<2><<<grid, kThreads, smem_bytes(2, gpc), s>>>(xsg, gsg, packed, scales, y, partials, ws.counters,
-                                                               (int)M, N, K, S, gpc);
-    }
-    return cudaGetLastError();
+        kern<<<grid, kThreads, smem, s>>>(xsg, gsg, packed, scales, y, partials, ws.counters, (int)M, N, K, S, gpc);
+        return cudaGetLastError();
+    };
+    if (M <= 8)
+        return g64 ? run(skinny_prep_kernel<8, true>, skinny_kernel<1, true>, 8, 1)
+                   : run(skinny_prep_kernel<8, false>, skinny_kernel<1, false>, 8, 1);
+    return g64 ? run(skinny_prep_kernel<16, true>, skinny_kernel<2, true>, 16, 2)
+               : run(skinny_prep_kernel<16, false>, skinny_kernel<2, false>, 16, 2);
 }
 
 }  // namespace bonsai
