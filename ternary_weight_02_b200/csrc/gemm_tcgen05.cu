@@ -22,7 +22,8 @@
 //     - warps 2..9 (256 threads, one weight row each): expand the packed trits of a
 //       128-weight group times its FP16 scale into two 64-wide FP16 B stages, written
 //       in the same 128-byte-swizzled K-major layout the MMA descriptors describe
-//       (t * s is exact in FP16); after each piece of a tile, the epilogue:
+//       (t * s is exact in FP16; PQ2_0 g64 takes a new scale with every 64-wide
+//       stage); after each piece of a tile, the epilogue:
 //       tcgen05.ld of the accumulator, then FP16 (nearest even) stores to y, or the
 //       FP32 hand-over of a split tile.
 // Every wait is bounded: if one gives up, the CTA stops issuing work, waits for the

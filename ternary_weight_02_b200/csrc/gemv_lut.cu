@@ -2,6 +2,9 @@
 // Hadamard rotation of x fused in.  Q1_0 (1-bit, "Bonsai把 27B 大模型塞进手机的极端量化方案
 // 到底靠不靠谱" (wmrh.cn), sections 核心观点 and 关键机制): a byte holds 8 signs, so its
 // table covers 8 activations and a 128-byte row slice covers 1024 (split mode only).
+// PQ2_0 g64 (one scale per 64 weights, the Q2_0_g64 files of the same wmrh.cn page,
+// sections 快速上手 and 后端支持现状): PQ2_0's tables, with 4 lanes per scale group (split
+// mode only; batch-1 calls take the integer GEMV by default, this kernel on request).
 //
 // Operation: y[n] = sum_g s[n][g] * sum_j t[n][128g+j] * x'[128g+j], x' = blockdiag(Hn) x.
 // Sources: "27B 模型压到 5.95GB，推理能力还保住 98%" (allhereai.com): method paragraph

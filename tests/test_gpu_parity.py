@@ -25,7 +25,7 @@ def bz():
 
 # ------------------------------------------------------------ codec
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1, G64])
 @pytest.mark.parametrize("N,K", [(1, 128), (3, 384), (37, 1024), (64, 5120), (5, 17408)])
 def test_pack_bit_exact(bz, fmt, N, K):
     import torch
@@ -37,7 +37,7 @@ def test_pack_bit_exact(bz, fmt, N, K):
     assert np.array_equal(got, want)
 
 
-@pytest.mark.parametrize("fmt", [PTQ1, PQ2])
+@pytest.mark.parametrize("fmt", [PTQ1, PQ2, G64])
 def test_unpack_bit_exact_and_invalid_codes(bz, fmt):
     import torch
     N, K = 9, 640

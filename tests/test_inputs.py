@@ -43,6 +43,9 @@ def test_rows_are_order_independent():
     assert np.array_equal(inputs.normal_rows(3, 256, [5, 0]), xs[[5, 0]])
     ss = inputs.scales(3, 10, 512)
     assert np.array_equal(inputs.scales_rows(3, 4, [9]), ss[[9]])
+    # one scale per 64 weights: a 10 x 8 plane whose rows regenerate alone
+    s64 = inputs.scales(3, 10, 512, group=64)
+    assert s64.shape == (10, 8) and np.array_equal(inputs.scales_rows(3, 8, [9, 0]), s64[[9, 0]])
 
 
 def test_distributions():
