@@ -21,8 +21,9 @@
  *   y       M x N   FP16, round-to-nearest-even from an FP32 accumulator
  *   scales  N x K/128  FP16 (N x K/64 for BONSAI_FMT_PQ2_0_G64)
  *   trits   N x K   int8 in {-1, 0, +1}
- *   packed  the trit plane of one of the two packings of the allhereai.com page
- *           (paragraph on the two file packings):
+ *   packed  the plane of one of the formats below: the two packings of the
+ *           allhereai.com page (paragraph on the two file packings) and two
+ *           variants the wmrh.cn page names:
  *     BONSAI_FMT_PTQ1_0  "compact trits", 1.75 bits/weight with the scale:
  *         row n, group g (128 weights) occupies 26 bytes at (n*K/128 + g)*26;
  *         byte b < 25 holds weights 128g+5b .. 128g+5b+4, byte 25 the last
