@@ -48,6 +48,9 @@ DOM_KERNEL = {1: "lookup-table GEMV (gemv_split_kernel + in-order reduction)",
               3: "lookup-table GEMV (gemv_split_kernel, 1-bit tables + in-order reduction)",
               4: "integer tensor-core GEMV (gemv_imma_kernel, 64-weight scale groups)"}
 DOM_SOURCE = {1: "gemv_lut.cu", 2: "gemv_imma.cu", 3: "gemv_lut.cu", 4: "gemv_imma.cu"}
+# the arithmetic of that kernel: integer MMA (u8 codes x s8 bytes of 16-bit fixed-point x',
+# s32 sums, then FP32 group scaling), or FP32 table sums
+DECODE_DTYPE = {1: "f32", 2: "int8", 3: "f32", 4: "int8"}
 
 
 def weights(fmt, seed, N, K):
@@ -367,7 +370,7 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms"], 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DECODE_DTYPE[fmt],
             "data": "synthetic (seeded SplitMix64 trits P(0)=.38, FP16 scales U[.01,.05], FP16 x N(0,1))",
             "config": {
                 "workload": (f"64-layer 27B-class linear stack at M=1 (qkv 5120->7168, o 5120->5120, "
