@@ -59,6 +59,12 @@ def weights(fmt, seed, N, K):
     return inputs.signs(seed, N, K) if fmt == 3 else inputs.trits(seed, N, K)
 
 
+def stack_workload(fmt):
+    """The decode workload both arms report: the 64-layer linear stack, one token per step."""
+    return (f"64-layer 27B-class linear stack at M=1 (qkv 5120->7168, o 5120->5120, "
+            f"gate/up 5120->34816, down 17408->5120), {FMT_NAMES[fmt]}, one token per step")
+
+
 def scale_group(fmt):
     """Weights per FP16 scale: 64 for the g64 variant of PQ2_0, else 128."""
     return 64 if fmt == 4 else 128
@@ -211,8 +217,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"27B-class decode projections, M=1, {FMT_NAMES[fmt]}, one layer per step",
-                   "l2": "n/a (CPU)"},
+        "config": {"workload": stack_workload(fmt), "sample": sample, "l2": "n/a (CPU)"},
         "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -373,8 +378,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DECODE_DTYPE[fmt],
             "data": "synthetic (seeded SplitMix64 trits P(0)=.38, FP16 scales U[.01,.05], FP16 x N(0,1))",
             "config": {
-                "workload": (f"64-layer 27B-class linear stack at M=1 (qkv 5120->7168, o 5120->5120, "
-                             f"gate/up 5120->34816, down 17408->5120), {FMT_NAMES[fmt]}, one token per step"),
+                "workload": stack_workload(fmt),
                 "packing": FMT_NAMES[fmt], "layers": LAYERS, "tokens_per_step": 1,
                 "bytes_per_step": step_bytes(fmt), "l2": "inputs larger than L2 (weights re-read every step)",
                 "per_token_us": round(r["ms"] * 1e3, 2), "frac_of_8TBps": round(r["value"] / 8000.0, 4),
