@@ -148,8 +148,8 @@ int bonsai_hadamard128(const uint16_t *x, uint16_t *x_out, int64_t M, int64_t K,
 /* y = x' . Wdeq^T (definitions above) for un-rotated FP16 x: the Hadamard
  * rotation of x is applied inside the call.  Dispatch on M: M == 1 -> the
  * integer tensor-core GEMV (PQ2_0 and PQ2_0 g64, K <= 24576) or the lookup-table GEMV
- * (PTQ1_0, Q1_0), 2 <= M <= 16 -> skinny tensor-core kernel (PQ2_0), otherwise
- * (and for the other packings at 2 <= M <= 16) the tcgen05 GEMM.  The
+ * (PTQ1_0, Q1_0), 2 <= M <= 16 -> skinny tensor-core kernel (PQ2_0, PQ2_0 g64,
+ * Q1_0), otherwise (and for PTQ1_0 at 2 <= M <= 16) the tcgen05 GEMM.  The
  * integer GEMV holds each 128-group of x' as 16-bit fixed point with a power-of-two
  * scale (|x~| <= 2^14) before the exact integer products; the other kernels round
  * x' to FP16 (GEMM, skinny) or keep it in FP32 (lookup tables, plain kernel).  y must

@@ -1,5 +1,5 @@
-// skinny_mma.cu -- ternary linear layer for small batches (1 <= M <= 16 tokens), PQ2_0
-// with one FP16 scale per 128 or per 64 weights.
+// skinny_mma.cu -- ternary linear layer for small batches (1 <= M <= 16 tokens): PQ2_0
+// with one FP16 scale per 128 or per 64 weights, and the 1-bit Q1_0 packing.
 //
 // y[m][n] = sum_g s[n][g] * sum_j t[n][128g+j] * x'[m][128g+j].  Sources: "27B 模型压到
 // 5.95GB，推理能力还保住 98%" (allhereai.com): method paragraph (trits, FP16 group
@@ -33,6 +33,11 @@
 //   takes words tq and tq + 4 of the group instead of 2tq and 2tq + 1, so that MMAs 0-3
 //   cover the group's first 64 weights and MMAs 4-7 the last 64; each half has its own
 //   accumulator, scale and sum of x'.
+// * Q1_0 (weights +-1 as bits, "Bonsai把 27B 大模型塞进手机的极端量化方案到底靠不靠谱"
+//   (wmrh.cn), sections 核心观点 and 关键机制): lane quad member tq takes word tq of the
+//   16-byte group; MMA i uses nibble i & 1 of byte i >> 1, bits left in place as FP16
+//   subnormals b * 2^j * 2^-24 (j = 0..7 within the byte) against x' pre-scaled by 2^-j,
+//   and the epilogue adds s * (2 * 2^24 * D - sum x'), which turns bits b into 2b - 1.
 #include "common.cuh"
 #include "internal.h"
 
@@ -68,19 +73,22 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // K order of the MMAs: MMA i of a group takes, from lane quad member tq, byte (i & 3) of
 // group word 2tq + (i >> 2), i.e. the four weights 32tq + 16(i >> 2) + 4(i & 3) + c,
 // c = 0..3, which sit at B slots 4tq + c of the MMA's 16-half row of x'.  g64: byte
-// (i & 3) of word tq + 4(i >> 2), weights 64(i >> 2) + 16tq + 4(i & 3) + c.
-template <bool kG64>
+// (i & 3) of word tq + 4(i >> 2), weights 64(i >> 2) + 16tq + 4(i & 3) + c.  Q1_0:
+// nibble i & 1 of byte i >> 1 of word tq, weights 32tq + 4i + c.
+template <int kFmt>
 __device__ __forceinline__ int64_t skinny_k(int64_t group, int step, int tq) {
-    return kG64 ? group * kGroup + 64 * (step >> 2) + 16 * tq + 4 * (step & 3)
-                : group * kGroup + 32 * tq + 16 * (step >> 2) + 4 * (step & 3);
+    return kFmt == 4   ? group * kGroup + 64 * (step >> 2) + 16 * tq + 4 * (step & 3)
+           : kFmt == 3 ? group * kGroup + 32 * tq + 4 * step
+                       : group * kGroup + 32 * tq + 16 * (step >> 2) + 4 * (step & 3);
 }
 
 // The rotation pass of this kernel: one warp per (group g, token m < MT).  It writes x'
 // (FP16, nearest) of the block in the layout the MMAs read, [g][step][token][16] with
-// slot 4tq + c = element skinny_k(g, step, tq) + c scaled by 4^-c, zeros for the padding
+// slot 4tq + c = element skinny_k(g, step, tq) + c scaled by 4^-c (Q1_0: by 2^-c for an
+// even step, 2^-(4 + c) for an odd one), zeros for the padding
 // tokens m >= M, and the FP32 sum of the block's FP16 x' values to gsum[g][m] (g64: the
 // sums of its two 64-element halves to gsum[g][h][m]).
-template <int MT, bool kG64>
+template <int MT, int kFmt>
 __global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ xs,
                                                           float *__restrict__ gsum, int M, int64_t K) {
     const int lane = threadIdx.x & 31;
@@ -96,6 +104,7 @@ __global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__rest
     }
     const __half2 h01 = __floats2half2_rn(v[0], v[1]), h23 = __floats2half2_rn(v[2], v[3]);
     const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+    constexpr bool kG64 = kFmt == 4;
     float sum = (f01.x + f01.y) + (f23.x + f23.y);
     if (kG64) {  // lanes 0..15 hold the first 64 elements, 16..31 the last 64
 #pragma unroll
@@ -104,11 +113,19 @@ __global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__rest
         sum = warp_sum(sum);
     }
     // lane l holds elements 4l .. 4l+3 = skinny_k(g, i, tq) + c with tq = l >> 3 and
-    // i = 4 ((l >> 2) & 1) + (l & 3) (g64: tq = (l >> 2) & 3, i = 4 (l >> 4) + (l & 3))
+    // i = 4 ((l >> 2) & 1) + (l & 3) (g64: tq = (l >> 2) & 3, i = 4 (l >> 4) + (l & 3);
+    // Q1_0: tq = l >> 3, i = l & 7)
     const int tq = kG64 ? (lane >> 2) & 3 : lane >> 3;
-    const int i = kG64 ? 4 * (lane >> 4) + (lane & 3) : 4 * ((lane >> 2) & 1) + (lane & 3);
-    const __half2 s01 = __hmul2(h01, __floats2half2_rn(1.f, 0.25f));
-    const __half2 s23 = __hmul2(h23, __floats2half2_rn(0.0625f, 0.015625f));
+    const int i = kG64 ? 4 * (lane >> 4) + (lane & 3) : (kFmt == 3 ? lane & 7 : 4 * ((lane >> 2) & 1) + (lane & 3));
+    __half2 s01, s23;
+    if (kFmt == 3) {  // 2^-c, or 2^-(4 + c) for the high nibble (odd step)
+        const float f = (i & 1) ? 0.0625f : 1.f;
+        s01 = __hmul2(h01, __floats2half2_rn(f, 0.5f * f));
+        s23 = __hmul2(h23, __floats2half2_rn(0.25f * f, 0.125f * f));
+    } else {
+        s01 = __hmul2(h01, __floats2half2_rn(1.f, 0.25f));
+        s23 = __hmul2(h23, __floats2half2_rn(0.0625f, 0.015625f));
+    }
     uint2 out;
     out.x = *reinterpret_cast<const uint32_t *>(&s01);
     out.y = *reinterpret_cast<const uint32_t *>(&s23);
@@ -126,7 +143,8 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
                  : "memory");
 }
 
-template <int NT, bool kG64>  // n8 token tiles: 1 (M <= 8) or 2 (M <= 16); 64-weight scales
+// kFmt: 2 PQ2_0, 4 PQ2_0 g64 (64-weight scales), 3 Q1_0
+template <int NT, int kFmt>  // n8 token tiles: 1 (M <= 8) or 2 (M <= 16)
 __global__ void __launch_bounds__(kThreads) skinny_kernel(
     const uint16_t *__restrict__ xsg, const float *__restrict__ gsg, const uint8_t *__restrict__ packed,
     const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
@@ -136,6 +154,7 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
     // groups staged at a time: the whole chunk when it fits (shared memory is sized so)
     const int kSub = gpc < sub_groups<NT>() ? gpc : sub_groups<NT>();
     extern __shared__ __align__(16) uint8_t smem[];
+    constexpr bool kG64 = kFmt == 4, kQ1 = kFmt == 3;
     constexpr int kHalves = kG64 ? 2 : 1;  // scale groups per 128 weights
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [kSub * 8 steps][MT][16]
     float *gsum = reinterpret_cast<float *>(smem + kSub * 8 * MT * 32);  // [MT][kSub][kHalves]
@@ -157,6 +176,9 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
         for (int e = 0; e < 4; e++) acc[nt][e] = 0.f;
 
     auto row_words = [&](int64_t r, int g) -> uint2 {
+        if (kQ1)  // word tq of the row's 16-byte group
+            return make_uint2(__ldcs(reinterpret_cast<const unsigned int *>(packed + (r * G + g) * kQ1GroupBytes) + tq),
+                              0u);
         const uint8_t *p = packed + (r * G + g) * kPq2GroupBytes;
         if (kG64)
             return make_uint2(__ldcs(reinterpret_cast<const unsigned int *>(p) + tq),
@@ -223,12 +245,18 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
 #pragma unroll
                 for (int i = 0; i < 8; i++) {
                     // byte (i & 3) of the lane's word i >> 2, in both halves: (c0, c1) and
-                    // (c2, c3) left in place as FP16 subnormals c * 4^j * 2^-24
-                    const uint32_t sel = 0x4040u | (uint32_t)(i & 3) | ((uint32_t)(i & 3) << 8);
-                    const uint32_t p0 = __byte_perm((i >> 2) ? cur.a.y : cur.a.x, 0u, sel);
-                    const uint32_t p1 = __byte_perm((i >> 2) ? cur.b.y : cur.b.x, 0u, sel);
-                    const uint32_t a0 = p0 & 0x000C0003u, a1 = p1 & 0x000C0003u;
-                    const uint32_t a2 = p0 & 0x00C00030u, a3 = p1 & 0x00C00030u;
+                    // (c2, c3) left in place as FP16 subnormals c * 4^j * 2^-24.  Q1_0: byte
+                    // i >> 1 of the word, bits 4(i & 1) + (0, 1) and + (2, 3) left in place
+                    const int byte = kQ1 ? i >> 1 : i & 3;
+                    const uint32_t sel = 0x4040u | (uint32_t)byte | ((uint32_t)byte << 8);
+                    const uint32_t w0 = kQ1 ? cur.a.x : ((i >> 2) ? cur.a.y : cur.a.x);
+                    const uint32_t w1 = kQ1 ? cur.b.x : ((i >> 2) ? cur.b.y : cur.b.x);
+                    const uint32_t p0 = __byte_perm(w0, 0u, sel);
+                    const uint32_t p1 = __byte_perm(w1, 0u, sel);
+                    const uint32_t m01 = kQ1 ? ((i & 1) ? 0x00200010u : 0x00020001u) : 0x000C0003u;
+                    const uint32_t m23 = kQ1 ? ((i & 1) ? 0x00800040u : 0x00080004u) : 0x00C00030u;
+                    const uint32_t a0 = p0 & m01, a1 = p1 & m01;
+                    const uint32_t a2 = p0 & m23, a3 = p1 & m23;
                     const int ks = gl * 8 + i;
 #pragma unroll
                     for (int nt = 0; nt < NT; nt++) {
@@ -245,11 +273,13 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
                         const int m0 = nt * 8 + 2 * tq;
                         const float gs0 = gsum[m0 * kSub * kHalves + gl * kHalves + h];
                         const float gs1 = gsum[(m0 + 1) * kSub * kHalves + gl * kHalves + h];
-                        // d[h][nt][0], [1]: row r0, tokens m0, m0+1; [2], [3]: row r1
-                        acc[nt][0] = fmaf(cs0, fmaf(d[h][nt][0], 16777216.f, -gs0), acc[nt][0]);
-                        acc[nt][1] = fmaf(cs0, fmaf(d[h][nt][1], 16777216.f, -gs1), acc[nt][1]);
-                        acc[nt][2] = fmaf(cs1, fmaf(d[h][nt][2], 16777216.f, -gs0), acc[nt][2]);
-                        acc[nt][3] = fmaf(cs1, fmaf(d[h][nt][3], 16777216.f, -gs1), acc[nt][3]);
+                        // d[h][nt][0], [1]: row r0, tokens m0, m0+1; [2], [3]: row r1.  Codes c
+                        // give sum c x' - sum x'; Q1_0 bits b give 2 sum b x' - sum x'
+                        constexpr float kUnit = kQ1 ? 33554432.f : 16777216.f;
+                        acc[nt][0] = fmaf(cs0, fmaf(d[h][nt][0], kUnit, -gs0), acc[nt][0]);
+                        acc[nt][1] = fmaf(cs0, fmaf(d[h][nt][1], kUnit, -gs1), acc[nt][1]);
+                        acc[nt][2] = fmaf(cs1, fmaf(d[h][nt][2], kUnit, -gs0), acc[nt][2]);
+                        acc[nt][3] = fmaf(cs1, fmaf(d[h][nt][3], kUnit, -gs1), acc[nt][3]);
                     }
                 }
                 const int g = sub + gl;
@@ -332,7 +362,7 @@ size_t gsum_bytes(int64_t M, int64_t K) {  // room for the g64 half sums
 }  // namespace
 
 bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt) {
-    return (fmt == 2 || fmt == 4) && M >= 1 && M <= 16 && K % kGroup == 0 && (N + 15) / 16 <= kMaxTiles &&
+    return (fmt == 2 || fmt == 3 || fmt == 4) && M >= 1 && M <= 16 && K % kGroup == 0 && (N + 15) / 16 <= kMaxTiles &&
            K < ((int64_t)1 << 31);
 }
 
@@ -346,7 +376,7 @@ size_t skinny_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int spli
 cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                           uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int split_k,
                           const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
-    if (fmt != 2 && fmt != 4) return cudaErrorInvalidValue;
+    if (fmt != 2 && fmt != 3 && fmt != 4) return cudaErrorInvalidValue;
     uint16_t *xsg = reinterpret_cast<uint16_t *>(ws.data);
     float *gsg = reinterpret_cast<float *>(ws.data + staged_bytes(M, K));
     float *partials = reinterpret_cast<float *>(ws.data + staged_bytes(M, K) + gsum_bytes(M, K));
@@ -363,11 +393,14 @@ cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16
         kern<<<grid, kThreads, smem, s>>>(xsg, gsg, packed, scales, y, partials, ws.counters, (int)M, N, K, S, gpc);
         return cudaGetLastError();
     };
-    if (M <= 8)
-        return g64 ? run(skinny_prep_kernel<8, true>, skinny_kernel<1, true>, 8, 1)
-                   : run(skinny_prep_kernel<8, false>, skinny_kernel<1, false>, 8, 1);
-    return g64 ? run(skinny_prep_kernel<16, true>, skinny_kernel<2, true>, 16, 2)
-               : run(skinny_prep_kernel<16, false>, skinny_kernel<2, false>, 16, 2);
+    if (M <= 8) {
+        if (g64) return run(skinny_prep_kernel<8, 4>, skinny_kernel<1, 4>, 8, 1);
+        if (fmt == 3) return run(skinny_prep_kernel<8, 3>, skinny_kernel<1, 3>, 8, 1);
+        return run(skinny_prep_kernel<8, 2>, skinny_kernel<1, 2>, 8, 1);
+    }
+    if (g64) return run(skinny_prep_kernel<16, 4>, skinny_kernel<2, 4>, 16, 2);
+    if (fmt == 3) return run(skinny_prep_kernel<16, 3>, skinny_kernel<2, 3>, 16, 2);
+    return run(skinny_prep_kernel<16, 2>, skinny_kernel<2, 2>, 16, 2);
 }
 
 }  // namespace bonsai

@@ -433,7 +433,7 @@ def test_gemm_prefill_full_size_sampled(bz, fmt, M, K, N):
 SKINNY_SMALL = [(2, 64, 128), (3, 129, 384), (8, 300, 1024), (9, 100, 640), (16, 257, 2048)]
 
 
-@pytest.mark.parametrize("fmt", [PQ2, G64])
+@pytest.mark.parametrize("fmt", [PQ2, G64, Q1])
 @pytest.mark.parametrize("M,N,K", SKINNY_SMALL)
 @pytest.mark.parametrize("split_k", [0, 1, 3])
 def test_skinny_small(bz, fmt, M, N, K, split_k):
@@ -443,19 +443,19 @@ def test_skinny_small(bz, fmt, M, N, K, split_k):
     assert ok, (rel, mx)
 
 
-@pytest.mark.parametrize("fmt", [PQ2, G64])
+@pytest.mark.parametrize("fmt", [PQ2, G64, Q1])
 @pytest.mark.parametrize("M", [2, 4, 8, 16])
 @pytest.mark.parametrize("K,N", [(5120, 5120), (17408, 5120), (5120, 34816)])
 def test_skinny_decode_shapes_full(bz, fmt, M, K, N):
     """Skinny decode batches on 27B-class projections, every output against the checker
-    (the default entry point takes the skinny kernel for both packings)."""
+    (the default entry point takes the skinny kernel for these packings)."""
     p = Problem(M, N, K, fmt, seed=M)
     got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
 
 
-@pytest.mark.parametrize("fmt", [PQ2, G64])
+@pytest.mark.parametrize("fmt", [PQ2, G64, Q1])
 def test_skinny_split_is_deterministic(bz, fmt):
     import torch
     p = Problem(8, 5120, 17408, fmt, seed=3)
@@ -471,7 +471,7 @@ def test_skinny_split_is_deterministic(bz, fmt):
 
 
 @pytest.mark.parametrize("M", [2, 5, 16])
-@pytest.mark.parametrize("fmt", [PTQ1, Q1])
+@pytest.mark.parametrize("fmt", [PTQ1])
 def test_small_batches_ptq1_take_the_gemm(bz, M, fmt):
     p = Problem(M, 300, 1024, fmt, seed=M)
     got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
@@ -515,7 +515,7 @@ SWIGLU_CASES = [(1, 16, 512, PQ2), (1, 1024, 2048, PQ2), (1, 4000, 1152, PQ2), (
                 (1, 1024, 1024, PTQ1), (1, 1024, 2048, Q1), (4, 512, 1024, PQ2), (300, 640, 640, PQ2),
                 (300, 640, 640, Q1), (300, 384, 1152, PTQ1), (600, 1280, 384, PQ2), (300, 200, 640, PQ2), (300, 1270, 256, Q1),
                 (1, 1024, 2048, G64), (1, 24, 512, G64), (1, 4000, 1152, G64), (300, 200, 640, G64),
-                (600, 1280, 384, G64), (4, 512, 1024, G64), (1, 17408, 5120, PQ2), (1, 17408, 5120, G64)]
+                (600, 1280, 384, G64), (4, 512, 1024, G64), (4, 512, 1024, Q1), (1, 17408, 5120, PQ2), (1, 17408, 5120, G64)]
 
 
 @pytest.mark.parametrize("M,F,K,fmt", SWIGLU_CASES)
