@@ -860,7 +860,7 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
     if (fmt == 2 || fmt == 4) {
         const cuuint64_t wdims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
         const cuuint64_t wstrides[1] = {(cuuint64_t)(K / 4)};
-        const cuuint32_t wbox[2] = {BK / 4, swiglu ? BN / 2 : BN};
+        const cuuint32_t wbox[2] = {(cuuint32_t)(BK / 4), (cuuint32_t)(swiglu ? BN / 2 : BN)};
         if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), wdims, wstrides, wbox,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)

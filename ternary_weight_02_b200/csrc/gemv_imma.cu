@@ -99,8 +99,6 @@ __host__ __device__ inline Layout make_layout(int K) {
     return L;
 }
 
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 // D += A * B, A 16 x 32 u8 (row-major fragments), B 32 x 8 s8, D int32.
 __device__ __forceinline__ void imma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -255,18 +253,6 @@ __device__ __forceinline__ float wait_pairs(uint64_t *p, int lane) {
     return __int_as_float(0x7fc00000);
 }
 
-__device__ __forceinline__ void cp_async8(void *dst, const void *src, bool valid) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(saddr(dst)), "l"(src), "r"(valid ? 8 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src), "r"(valid ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int kPending>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // kAsyncScales: K is a multiple of 512, so an item's four (g64: eight) scales of a row are
 // 8 (16) aligned bytes, copied with cp.async as part of the item's copy; otherwise each
@@ -343,9 +329,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
                 const int row = row_of(rt, lane);
                 const bool v = row < N;
                 if (kG64)
-                    cp_async16(sring + st * kScaleRingBytes + lane * 16, scales + (v ? (int64_t)row * GS + kc * 8 : 0), v);
+                    cp_async16_zfill(sring + st * kScaleRingBytes + lane * 16, scales + (v ? (int64_t)row * GS + kc * 8 : 0), v);
                 else
-                    cp_async8(sring + st * kScaleRingBytes + lane * 16, scales + (v ? (int64_t)row * GS + kc * 4 : 0), v);
+                    cp_async8_zfill(sring + st * kScaleRingBytes + lane * 16, scales + (v ? (int64_t)row * GS + kc * 4 : 0), v);
             }
             n_issued++;
         }

@@ -68,8 +68,6 @@ constexpr int kSmemBytes = 0x30000;
 constexpr int kRowsModeMaxK = 12288;        // x' of all K must fit below the tables
 constexpr int kMaxTasksPerWarp = 32;        // split mode: row blocks per warp (host-checked)
 
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 template <int kFmt>
 struct Fmt;
@@ -231,11 +229,12 @@ __device__ __forceinline__ void build_tables(const float *xr, uint8_t *tables, i
 // nothing: a valid byte never reaches an unwritten entry.
 template <int kFmt>
 __device__ __forceinline__ void zero_phantom_tables(uint8_t *tables, int lane, int warp) {
-    if (kFmt != 1) return;
-    for (int e = warp; e < 256; e += kWarps)
+    if constexpr (kFmt == 1) {
+        for (int e = warp; e < 256; e += kWarps)
 #pragma unroll
-        for (int j = 0; j < 4; j++)
-            if (ptq1_slot_pos(lane, j) < 0) *reinterpret_cast<float *>(tables + table_offset(lane, j, e)) = 0.f;
+            for (int j = 0; j < 4; j++)
+                if (ptq1_slot_pos(lane, j) < 0) *reinterpret_cast<float *>(tables + table_offset(lane, j, e)) = 0.f;
+    }
 }
 
 // Loads one warp task: register i <- the lane's word of row n0 + i (each load

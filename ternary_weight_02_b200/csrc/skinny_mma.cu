@@ -137,11 +137,6 @@ __global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__rest
     }
 }
 
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src)
-                 : "memory");
-}
 
 // kFmt: 2 PQ2_0, 4 PQ2_0 g64 (64-weight scales), 3 Q1_0
 template <int NT, int kFmt>  // n8 token tiles: 1 (M <= 8) or 2 (M <= 16)
@@ -220,12 +215,12 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
             const int bytes = nsub * 8 * MT * 32;
             for (int off = tid * 16; off < bytes; off += kThreads * 16)
                 cp_async16(reinterpret_cast<uint8_t *>(xs) + off, src + off);
-            asm volatile("cp.async.commit_group;" ::: "memory");
+            cp_async_commit();
             for (int idx = tid; idx < nsub * MT * kHalves; idx += kThreads) {
                 const int gh = idx / MT, m = idx % MT;  // gh = kHalves * gl + h
                 gsum[m * kSub * kHalves + gh] = gsg[((int64_t)sub * kHalves + gh) * MT + m];
             }
-            asm volatile("cp.async.wait_all;" ::: "memory");
+            cp_async_wait_all();
         }
         __syncthreads();
 

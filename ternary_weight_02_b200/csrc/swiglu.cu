@@ -17,8 +17,8 @@ namespace {
 
 __global__ void __launch_bounds__(256) swiglu_kernel(const uint16_t *__restrict__ y, uint16_t *__restrict__ h,
                                                      int64_t M, int64_t F) {
-    asm volatile("griddepcontrol.launch_dependents;");
-    asm volatile("griddepcontrol.wait;" ::: "memory");  // y may belong to the previous kernel
+    pdl_launch_dependents();
+    pdl_wait();  // y may belong to the previous kernel
     const int64_t total = M * F;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t m = i / F, f = i - m * F;
