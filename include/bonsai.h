@@ -108,7 +108,7 @@ int bonsai_version(void);
 /* Human-readable text for a bonsai_status value (static storage). */
 const char *bonsai_status_string(int status);
 
-/* BONSAI_OK if the current CUDA device is an sm_100 part this build can run on,
+/* BONSAI_OK if the current CUDA device is an sm_100 part the library was compiled for,
  * BONSAI_ERR_ARCH if it is another architecture, BONSAI_ERR_CUDA if there is no
  * usable device. */
 int bonsai_check_device(void);
