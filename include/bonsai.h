@@ -60,6 +60,10 @@
  *     them on one stream); bonsai_reserve() sizes it ahead of stream capture.
  *   - Invalid codes in a packed plane (PTQ1_0 bytes >= 243, PQ2_0 code 3)
  *     produce unspecified output values but never out-of-bounds accesses.
+ *   - Every wait inside a kernel (a barrier on a copy in flight, a hand-over
+ *     between CTAs of the same grid) gives up after a bounded number of polls;
+ *     the call then writes NaN to the outputs it could not finish instead of
+ *     hanging the GPU, and later calls run normally.
  */
 #ifndef BONSAI_H
 #define BONSAI_H
