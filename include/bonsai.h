@@ -63,7 +63,9 @@
  *   - Every wait inside a kernel (a barrier on a copy in flight, a hand-over
  *     between CTAs of the same grid) gives up after a bounded number of polls;
  *     the call then writes NaN to the outputs it could not finish instead of
- *     hanging the GPU, and later calls run normally.
+ *     hanging the GPU.  Such a call may leave hand-over state behind in the
+ *     workspace, so after NaN outputs of this kind call bonsai_shutdown(): the
+ *     next call re-creates the workspace, zeroed.
  */
 #ifndef BONSAI_H
 #define BONSAI_H
