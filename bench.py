@@ -251,10 +251,11 @@ def run_ours(args):
     from ternary_weight_02_b200 import bonsai as bz
 
     world, rank, local = dist_setup()
-    if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    # bind this rank to its GPU before the process group so that NCCL uses it
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     if bz.bonsai_check_device() != bz.BONSAI_OK:
         raise RuntimeError("libbonsai: not an sm_100 device")
     peaks, peak_kind = measured_peaks()
