@@ -90,3 +90,13 @@ def test_no_device_reports_cuda_error(bz):
     good = 1 << 20
     assert bz.bonsai_check_device() == bz.BONSAI_ERR_CUDA
     assert bz.raw().bonsai_ternary_linear(good, good, good, good, 1, 8, 128, 2, None) == bz.BONSAI_ERR_CUDA
+
+
+def test_every_entry_point_is_documented():
+    """Each function the header declares is preceded by its own comment block (the
+    operation, argument layouts, ownership and error behaviour live there)."""
+    text = open(HEADER).read()
+    for name in declared_functions():
+        m = re.search(r"(/\*(?:(?!\*/).)*\*/)\s*(?:[A-Za-z_][A-Za-z0-9_ ]*[ *])" + name + r"\s*\(", text, flags=re.S)
+        assert m is not None, f"{name} has no comment block right before its declaration"
+        assert len(m.group(1)) > 40, name
