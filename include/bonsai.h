@@ -153,7 +153,8 @@ int bonsai_hadamard128(const uint16_t *x, uint16_t *x_out, int64_t M, int64_t K,
 
 /* y = x' . Wdeq^T (definitions above) for un-rotated FP16 x: the Hadamard
  * rotation of x is applied inside the call.  Dispatch on M: M == 1 -> the
- * integer tensor-core GEMV (PQ2_0 and PQ2_0 g64, K <= 24576) or the lookup-table GEMV
+ * integer tensor-core GEMV (PQ2_0 and PQ2_0 g64, K <= 24576, and a grid of at most one
+ * CTA per SM: up to about 14,000 items of 32 rows x 512 weights on 148 SMs) or the lookup-table GEMV
  * (PTQ1_0, Q1_0), 2 <= M <= 16 -> skinny tensor-core kernel (PQ2_0, PQ2_0 g64,
  * Q1_0), otherwise (and for PTQ1_0 at 2 <= M <= 16) the tcgen05 GEMM.  The
  * integer GEMV holds each 128-group of x' as 16-bit fixed point with a power-of-two

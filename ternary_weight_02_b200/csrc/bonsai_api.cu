@@ -136,10 +136,13 @@ int cuda_status(cudaError_t e) {
     return BONSAI_ERR_CUDA;
 }
 
-// Picks the kernel for AUTO, or checks an explicit choice.
-int resolve_algo(int algo, int64_t M, int64_t N, int64_t K, int fmt) {
+// Picks the kernel for AUTO, or checks an explicit choice.  Without the device (argument
+// checks before the device is probed) AUTO assumes the integer GEMV's grid fits; callers
+// resolve AUTO again with the device once it is known.
+int resolve_algo(int algo, int64_t M, int64_t N, int64_t K, int fmt, const DeviceInfo *dev = nullptr) {
     if (algo == BONSAI_ALGO_AUTO) {
-        if (M == 1 && gemv_imma_supported(M, N, K, fmt)) return BONSAI_ALGO_IMMA;
+        if (M == 1 && gemv_imma_supported(M, N, K, fmt) && (dev == nullptr || gemv_imma_grid_fits(N, K, *dev)))
+            return BONSAI_ALGO_IMMA;
         if (M == 1 && gemv_supported(M, N, K, fmt)) return BONSAI_ALGO_GEMV;
         if (M <= 16 && skinny_supported(M, N, K, fmt)) return BONSAI_ALGO_SKINNY;
         if (gemm_supported(M, N, K, fmt)) return BONSAI_ALGO_GEMM;
@@ -307,7 +310,7 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
     if (!x || !packed || !scales || !y) return BONSAI_ERR_NULL;
     if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(y))
         return BONSAI_ERR_ALIGN;
-    const int chosen = resolve_algo(algo, M, N, K, fmt);
+    int chosen = resolve_algo(algo, M, N, K, fmt);
     if (chosen < 0) return chosen;
 
     std::lock_guard<std::mutex> lock(g_mutex);
@@ -315,6 +318,7 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
     DeviceState *st;
     rc = probe_current(&dev, &st);
     if (rc != BONSAI_OK) return rc;
+    if (algo == BONSAI_ALGO_AUTO) chosen = resolve_algo(algo, M, N, K, fmt, &st->info);
     Workspace ws;
     rc = ensure_workspace(*st, workspace_for(chosen, M, N, K, fmt, split_k, st->info),
                           chosen == BONSAI_ALGO_IMMA ? gemv_imma_zeroed_bytes(N, K) : 0, &ws);
@@ -354,13 +358,14 @@ int bonsai_ternary_linear_swiglu(const uint16_t *x, const uint8_t *packed, const
     if (!x || !packed || !scales || !h) return BONSAI_ERR_NULL;
     if (!aligned16(x) || !aligned16(packed) || !aligned16(scales) || !aligned16(h))
         return BONSAI_ERR_ALIGN;
-    const int chosen = resolve_algo(BONSAI_ALGO_AUTO, M, N, K, fmt);
+    int chosen = resolve_algo(BONSAI_ALGO_AUTO, M, N, K, fmt);
     if (chosen < 0) return chosen;
     std::lock_guard<std::mutex> lock(g_mutex);
     int dev;
     DeviceState *st;
     rc = probe_current(&dev, &st);
     if (rc != BONSAI_OK) return rc;
+    chosen = resolve_algo(BONSAI_ALGO_AUTO, M, N, K, fmt, &st->info);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Workspace ws;
     if (chosen == BONSAI_ALGO_IMMA) {  // fused into the GEMV's epilogue
@@ -392,13 +397,14 @@ int bonsai_launch_count(int64_t M, int64_t N, int64_t K, int fmt, int algo, int 
     rc = check_shape(M, N, K);
     if (rc != BONSAI_OK) return rc;
     if (M == 0 || N == 0) return 0;
-    const int chosen = resolve_algo(algo, M, N, K, fmt);
+    int chosen = resolve_algo(algo, M, N, K, fmt);
     if (chosen < 0) return chosen;
     std::lock_guard<std::mutex> lock(g_mutex);
     int dev;
     DeviceState *st;
     rc = probe_current(&dev, &st);
     if (rc != BONSAI_OK) return rc;
+    if (algo == BONSAI_ALGO_AUTO) chosen = resolve_algo(algo, M, N, K, fmt, &st->info);
     switch (chosen) {
         case BONSAI_ALGO_GEMV: return gemv_launches(N, K, fmt, split_k, st->info);
         case BONSAI_ALGO_IMMA: return 1;  // the rotation and quantisation of x are fused

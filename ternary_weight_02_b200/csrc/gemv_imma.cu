@@ -606,6 +606,14 @@ bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt) {
     return RT * ((K + kItemK - 1) / kItemK) < ((int64_t)1 << 30);
 }
 
+// True when the call's grid fits on the GPU at once (at most one CTA per SM), which the
+// hand-over between CTAs assumes: a CTA holds at most kMaxCtaItems items, so shapes with
+// more than sm_count x kMaxCtaItems items are left to the other batch-1 kernels by the
+// automatic choice.
+bool gemv_imma_grid_fits(int64_t N, int64_t K, const DeviceInfo &dev) {
+    return shape_of(N, K, dev.sm_count).grid <= dev.sm_count;
+}
+
 // the zero-initialised workspace region: (value, epoch) pairs of the pieces of row tiles
 // split between CTAs, indexed by the piece's first item: items x 32 x 8 bytes.  Every
 // pair a call stores is cleared again by its reader.
