@@ -96,59 +96,84 @@ def step_bytes(fmt):
     return LAYERS * per_layer
 
 
-class Clocks:
-    """Samples nvidia-smi during the timed region (SM clock, throttle reasons)."""
-
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-
-    def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        return parse_clock_samples(out)
+# NVML clock-event reason bits that the timing rules name (nvmlClocksEventReason*)
+CLOCK_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
 
-def parse_clock_samples(out):
-    """Median SM clock, max clock and the throttle reasons seen in nvidia-smi's
-    `Clocks.FIELDS` lines (csv, noheader, nounits); None without a valid sample."""
-    sm, smax, reasons = [], [], set()
-    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-    for line in out.strip().splitlines():
-        parts = [p.strip() for p in line.split(",")]
-        if len(parts) < 9:
-            continue
-        try:
-            sm.append(float(parts[1]))
-            smax.append(float(parts[2]))
-        except ValueError:
-            continue
-        for name, val in zip(names, parts[5:9]):
-            if val.lower() == "active":
-                reasons.add(name)
+def summarize_clock_samples(samples):
+    """Median SM clock, max SM clock and the throttle reasons seen in a list of
+    (sm_mhz, sm_max_mhz, reasons_bitmask) samples; None without a valid sample."""
+    sm = [float(a) for a, b, r in samples if a is not None and a > 0]
+    smax = [float(b) for a, b, r in samples if b is not None and b > 0]
     if not sm:
         return None
-    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-            "samples": len(sm)}
+    reasons = sorted({name for _, _, r in samples for bit, name in CLOCK_REASONS.items() if r & bit})
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax) if smax else None,
+            "reasons": reasons, "samples": len(sm)}
+
+
+class Clocks:
+    """Samples the GPU's SM clock and clock-event reasons through NVML in a background
+    thread (every 10 ms) while a timed region runs.  The NVML device is the one whose
+    UUID matches the torch device, so a CUDA_VISIBLE_DEVICES remap cannot mislead it."""
+
+    def __init__(self, torch_device_index):
+        self.index = torch_device_index
+        self.samples = []
+        self.thread = None
+        self.stop_flag = None
+        self.handle = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            want = str(torch.cuda.get_device_properties(self.index).uuid).lower().replace("gpu-", "")
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = (u.decode() if isinstance(u, bytes) else u).lower().replace("gpu-", "")
+                if u == want:
+                    self.handle = h
+                    break
+            self.nvml = pynvml
+        except Exception:  # no NVML or no match: the line's clocks stay null
+            self.handle = None
+
+    def _sample(self):
+        n = self.nvml
+        try:
+            sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+            smax = n.nvmlDeviceGetMaxClockInfo(self.handle, n.NVML_CLOCK_SM)
+            reasons = n.nvmlDeviceGetCurrentClocksThrottleReasons(self.handle)
+            self.samples.append((sm, smax, int(reasons)))
+        except Exception:
+            pass
+
+    def start(self):
+        if self.handle is None:
+            return
+        import threading
+        self.samples = []
+        self.stop_flag = threading.Event()
+
+        def loop():
+            while not self.stop_flag.is_set():
+                self._sample()
+                self.stop_flag.wait(0.01)
+
+        self._sample()
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.thread is None:
+            return None
+        self._sample()
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        self.thread = None
+        return summarize_clock_samples(self.samples)
 
 
 def dist_setup():
@@ -232,23 +257,194 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ our arm
 
-def build_stack(fmt, dev, bz, torch):
-    """Weights of the 64-layer stack: seeded trits/scales per shape, packed on the GPU,
-    copied into 64 distinct buffers per shape; x per shape."""
+def nvtx(torch, name):
+    """A named NVTX range around a bench phase (visible to profilers; no cost otherwise)."""
+    import contextlib
+
+    @contextlib.contextmanager
+    def rng():
+        torch.cuda.nvtx.range_push(name)
+        try:
+            yield
+        finally:
+            torch.cuda.nvtx.range_pop()
+    return rng()
+
+
+def base_planes(fmt, dev, bz, torch):
+    """One seeded packed plane, scale plane and FP16 x (M = 1) per projection shape."""
     from ternary_weight_02_b200 import inputs
-    stack = []
-    xs, ys = [], []
+    out = []
     for i, (name, K, N) in enumerate(SHAPES):
         t = torch.from_numpy(weights(fmt, i, N, K)).to(dev)
         packed = bz.pack(fmt, t)
         del t
         s = torch.from_numpy(scales(fmt, i, N, K).view(np.int16)).to(dev).view(torch.float16)
-        copies = [(packed.clone(), s.clone()) for _ in range(LAYERS)]
-        del packed, s
-        stack.append(copies)
+        out.append((packed, s))
+    return out
+
+
+def build_stack(fmt, base, dev, torch):
+    """Weights of the 64-layer stack: LAYERS distinct copies of each shape's planes (far
+    more than L2 holds, so every step streams them from HBM); x and y per shape."""
+    from ternary_weight_02_b200 import inputs
+    stack, xs, ys = [], [], []
+    for i, (name, K, N) in enumerate(SHAPES):
+        packed, s = base[i]
+        stack.append([(packed.clone(), s.clone()) for _ in range(LAYERS)])
         xs.append(torch.from_numpy(inputs.activations(i, 1, K).view(np.int16)).to(dev).view(torch.float16))
         ys.append(torch.empty((1, N), dtype=torch.float16, device=dev))
     return stack, xs, ys
+
+
+def capture(torch, stream, fn):
+    """fn() enqueued once eagerly (first-use set-up), then captured into a CUDA graph."""
+    with torch.cuda.stream(stream):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(torch, stream, g, reps, warmup=3):
+    """Device time of one replay of g in ms: CUDA events on its stream around reps replays."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def measure_decode(f, base, dev, bz, torch, args, world, hbm):
+    """The decode stack of packing f (step time, e2e), each projection's batch-1 call
+    time in a graph of LAYERS calls on distinct weight copies, and the live timing of the
+    dominant (gate/up) kernel."""
+    stack, xs, ys = build_stack(f, base, dev, torch)
+    stream = torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+
+    def enqueue(only=None):
+        for layer in range(LAYERS):
+            for i, (name, K, N) in enumerate(SHAPES):
+                if only is not None and i != only:
+                    continue
+                p, s = stack[i][layer]
+                bz.bonsai_ternary_linear(xs[i], p, s, ys[i], 1, N, K, f, sp)
+
+    g = capture(torch, stream, enqueue)
+    # ---- device-resident timing of the whole step
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    clocks = Clocks(dev.index)
+    clocks.start()
+    with nvtx(torch, f"decode stack {FMT_NAMES[f]}"):
+        ms = time_graph(torch, stream, g, args.steps, warmup=0)
+    clk = clocks.stop()
+    ms = max_over_ranks(ms, dev)
+    value = whole_job_gbs(step_bytes(f), world, ms)
+
+    # ---- each projection alone: LAYERS calls per replay, each on its own weight copy
+    per = {}
+    with nvtx(torch, f"per-projection {FMT_NAMES[f]}"):
+        for i, (name, K, N) in enumerate(SHAPES):
+            gi = capture(torch, stream, lambda i=i: enqueue(only=i))
+            reps = max(3, args.steps)
+            us = time_graph(torch, stream, gi, reps) * 1e3 / LAYERS
+            b = plane_bytes(f, N, K) + 2 * K + 2 * N
+            per[name] = {"K": K, "N": N, "us": round(us, 3), "gbs": round(b / (us * 1e-6) / 1e9, 1),
+                         "frac": round(b / (us * 1e-6) / 1e9 / hbm, 4), "bytes": b,
+                         "launches": bz.bonsai_launch_count(1, N, K, f)}
+            del gi
+
+    # ---- end to end through the C ABI with host buffers
+    hx = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in xs]
+    for h, x in zip(hx, xs):
+        h.copy_(x.cpu())
+    hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
+    h2d = sum(h.numel() * h.element_size() for h in hx)
+    d2h = sum(h.numel() * h.element_size() for h in hy)
+
+    def e2e_step():
+        for h, x in zip(hx, xs):
+            x.copy_(h, non_blocking=True)
+        g.replay()
+        for h, y in zip(hy, ys):
+            h.copy_(y, non_blocking=True)
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with nvtx(torch, f"e2e {FMT_NAMES[f]}"), torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+    e2e = whole_job_gbs(step_bytes(f), world, ms_e2e)
+
+    launches_per_layer = sum(bz.bonsai_launch_count(1, N, K, f) for _, K, N in SHAPES)
+    out = {"launches_per_layer": launches_per_layer, "value": value, "ms": ms, "clocks": clk,
+           "per_projection": per, "e2e": e2e, "h2d": h2d, "d2h": d2h, "traffic": kernel_traffic(f)}
+    if f == 2:
+        out["swiglu_decode"] = measure_swiglu_decode(stack, xs, bz, torch, stream, dev, args)
+    if args.skinny and f in (1, 2):
+        out["skinny_grid"] = measure_skinny_grid(f, stack, dev, bz, torch, stream, args, hbm)
+    del stack, g
+    torch.cuda.synchronize()
+    return out
+
+
+def measure_skinny_grid(f, stack, dev, bz, torch, stream, args, hbm):
+    """Decode batches of M in {1, 2, 4, 8, 16} tokens on each projection: the automatic
+    choice, the skinny kernel without split-K, and the prefill GEMM, each as LAYERS calls
+    on distinct weight copies per replay.  GB/s counts the weight, scale, x and y bytes."""
+    from ternary_weight_02_b200 import inputs
+    sp = stream.cuda_stream
+    grid = {}
+    variants = [("auto", bz.BONSAI_ALGO_AUTO, 0), ("skinny_no_split", bz.BONSAI_ALGO_SKINNY, 1),
+                ("gemm", bz.BONSAI_ALGO_GEMM, 0)]
+    with nvtx(torch, f"skinny grid {FMT_NAMES[f]}"):
+        for M in (1, 2, 4, 8, 16):
+            for i, (name, K, N) in enumerate(SHAPES):
+                x = torch.from_numpy(inputs.activations(100 + i, M, K).view(np.int16)).to(dev).view(torch.float16)
+                y = torch.empty((M, N), dtype=torch.float16, device=dev)
+                b = plane_bytes(f, N, K) + 2 * M * K + 2 * M * N
+                row = {}
+                for vname, algo, sk in variants:
+                    try:
+                        bz.bonsai_launch_count(M, N, K, f, algo, sk)
+                    except bz.BonsaiError:
+                        continue  # this kernel does not take the shape or packing
+
+                    def enq(algo=algo, sk=sk):
+                        for layer in range(LAYERS):
+                            p, s = stack[i][layer]
+                            bz.bonsai_ternary_linear_algo(x, p, s, y, M, N, K, f, algo, sk, sp)
+                    gi = capture(torch, stream, enq)
+                    us = time_graph(torch, stream, gi, max(3, args.steps // 4)) * 1e3 / LAYERS
+                    row[vname] = {"us": round(us, 2), "gbs": round(b / (us * 1e-6) / 1e9, 1),
+                                  "frac": round(b / (us * 1e-6) / 1e9 / hbm, 4)}
+                    del gi
+                grid[f"M{M}_{name}"] = row
+    return {"workload": (f"M in {{1,2,4,8,16}} tokens x the four 27B-class projections, {FMT_NAMES[f]}, "
+                         f"{LAYERS} distinct weight copies per replay (weights re-read from HBM)"),
+            "unit": "us per call", "grid": grid}
 
 
 def run_ours(args):
@@ -265,120 +461,26 @@ def run_ours(args):
     if bz.bonsai_check_device() != bz.BONSAI_OK:
         raise RuntimeError("libbonsai: not an sm_100 device")
     peaks, peak_kind = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
     fmt = FMTS[args.fmt]
-    bz.bonsai_reserve(1, 34816, 17408)
+    bz.bonsai_reserve(16, 34816, 17408)
 
     results = {}
+    prefill = None
     for f in ([fmt] + [o for o in (2, 1, 3, 4) if o != fmt]) if args.both else [fmt]:
-        stack, xs, ys = build_stack(f, dev, bz, torch)
-        stream = torch.cuda.Stream(device=dev)
-        sp = stream.cuda_stream
-
-        def enqueue(only=None):
-            for layer in range(LAYERS):
-                for i, (name, K, N) in enumerate(SHAPES):
-                    if only is not None and i != only:
-                        continue
-                    p, s = stack[i][layer]
-                    bz.bonsai_ternary_linear(xs[i], p, s, ys[i], 1, N, K, f, sp)
-
-        with torch.cuda.stream(stream):
-            for _ in range(2):
-                enqueue()
-            torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                enqueue()
-            g_dom = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_dom, stream=stream):
-                enqueue(only=2)
-        torch.cuda.synchronize()
-
-        # ---- device-resident timing
-        with torch.cuda.stream(stream):
-            for _ in range(args.warmup):
-                g.replay()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        clocks = Clocks(local)
-        clocks.start()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            torch.cuda.synchronize()
-            e0.record(stream)
-            for _ in range(args.steps):
-                g.replay()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / args.steps
-        clk = clocks.stop()
-        ms = max_over_ranks(ms, dev)
-        value = whole_job_gbs(step_bytes(f), world, ms)
-
-        # ---- dominant kernel (gate/up GEMV), 64 launches per replay
-        with torch.cuda.stream(stream):
-            g_dom.replay()
-            torch.cuda.synchronize()
-            e0.record(stream)
-            for _ in range(max(3, args.steps)):
-                g_dom.replay()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        dom_launches = LAYERS * max(3, args.steps)
-        dom_us = e0.elapsed_time(e1) * 1e3 / dom_launches
-        _, Kd, Nd = SHAPES[2]
-        dom_bytes = plane_bytes(f, Nd, Kd) + 2 * Kd + 2 * Nd
-        dom_gbs = dom_bytes / (dom_us * 1e-6) / 1e9
-        traffic = kernel_traffic(f)
-
-        # ---- end to end through the C ABI with host buffers
-        hx = [torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in xs]
-        for h, x in zip(hx, xs):
-            h.copy_(x.cpu())
-        hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
-        h2d = sum(h.numel() * h.element_size() for h in hx)
-        d2h = sum(h.numel() * h.element_size() for h in hy)
-
-        def e2e_step():
-            for h, x in zip(hx, xs):
-                x.copy_(h, non_blocking=True)
-            g.replay()
-            for h, y in zip(hy, ys):
-                h.copy_(y, non_blocking=True)
-
-        with torch.cuda.stream(stream):
-            for _ in range(args.warmup):
-                e2e_step()
-            torch.cuda.synchronize()
-            e0.record(stream)
-            for _ in range(args.steps):
-                e2e_step()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
-        e2e = whole_job_gbs(step_bytes(f), world, ms_e2e)
-
-        launches_per_layer = sum(bz.bonsai_launch_count(1, N, K, f) for _, K, N in SHAPES)
-        if f == 2:
-            results["swiglu_decode"] = measure_swiglu_decode(stack, xs, bz, torch, stream, dev, args)
-        results[f] = {
-            "launches_per_layer": launches_per_layer,
-            "value": value, "ms": ms, "clocks": clk, "dom_us": dom_us, "dom_gbs": dom_gbs,
-            "dom_bytes": dom_bytes, "traffic": traffic, "e2e": e2e, "h2d": h2d, "d2h": d2h,
-        }
-        del stack, g, g_dom
+        base = base_planes(f, dev, bz, torch)
+        results[f] = measure_decode(f, base, dev, bz, torch, args, world, hbm)
+        if args.prefill_m > 0 and f in (1, 2) and (args.both or f == fmt):
+            pg = measure_prefill(f, base, dev, bz, torch, args, peaks, peak_kind)
+            prefill = pg if prefill is None else {**prefill, "grid": {**prefill["grid"], **pg["grid"]}}
+        del base
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
-
-    prefill = run_prefill(fmt, args.prefill_m, dev, bz, torch, peaks, peak_kind, max(3, args.steps // 20)) \
-        if args.prefill_m > 0 else None
 
     r = results[fmt]
     line = None
     if rank == 0:
-        hbm = float(peaks["hbm_gbs"])
+        dom = r["per_projection"]["gate_up"]
         line = {
             "metric": METRIC, "value": round(r["value"], 1), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(r["ms"], 4),
@@ -392,27 +494,33 @@ def run_ours(args):
                 "frac_of_measured_hbm": round(r["value"] / hbm, 4), "parallelism": f"replicas x{world}",
             },
             "roofline": {
-                "bound": "hbm", "kernel": f"{DOM_KERNEL[fmt]}, gate/up 5120->34816", "achieved": round(r["dom_gbs"], 1),
-                "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(r["dom_gbs"] / hbm, 4),
-                "traffic": r["traffic"], "algorithmic_bytes_per_launch": r["dom_bytes"],
-                "avg_launch_us": round(r["dom_us"], 3),
+                "bound": "hbm", "kernel": f"{DOM_KERNEL[fmt]}, gate/up 5120->34816", "achieved": dom["gbs"],
+                "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(dom["gbs"] / hbm, 4),
+                "traffic": r["traffic"], "algorithmic_bytes_per_launch": dom["bytes"],
+                "avg_launch_us": dom["us"],
             },
             "e2e": {"value": round(r["e2e"], 1), "unit": "GB/s", "h2d_bytes_per_step": r["h2d"],
                     "d2h_bytes_per_step": r["d2h"]},
             "gpu_launches": LAYERS * r["launches_per_layer"] * args.steps,
             "clocks": r["clocks"],
+            "per_projection": {FMT_NAMES[k]: v["per_projection"] for k, v in results.items()},
         }
         others = {FMT_NAMES[k]: {"value": round(v["value"], 1), "unit": "GB/s",
                                  "per_token_us": round(v["ms"] * 1e3, 2),
-                                 "gate_up_gbs": round(v["dom_gbs"], 1), "e2e": round(v["e2e"], 1)}
-                  for k, v in results.items() if k in FMT_NAMES and k != fmt}
-        if "swiglu_decode" in results:
-            line["swiglu"] = {"decode": results["swiglu_decode"]}
-            if prefill is not None and "swiglu_gate_up" in prefill:
-                line["swiglu"]["prefill"] = prefill.pop("swiglu_gate_up")
+                                 "gate_up_gbs": v["per_projection"]["gate_up"]["gbs"], "e2e": round(v["e2e"], 1),
+                                 "clocks": v["clocks"]}
+                  for k, v in results.items() if k != fmt}
         if others:
             line["other_packings"] = others
+        grids = {FMT_NAMES[k]: v["skinny_grid"] for k, v in results.items() if "skinny_grid" in v}
+        if grids:
+            line["skinny"] = grids
+        sw = next((v["swiglu_decode"] for v in results.values() if "swiglu_decode" in v), None)
+        if sw is not None:
+            line["swiglu"] = {"decode": sw}
         if prefill is not None:
+            if "swiglu_gate_up" in prefill:
+                line.setdefault("swiglu", {})["prefill"] = prefill.pop("swiglu_gate_up")
             line["prefill"] = prefill
     if world > 1:
         dist.barrier()
@@ -439,113 +547,138 @@ def measure_swiglu_decode(stack, xs, bz, torch, stream, dev, args):
                 else:
                     bz.bonsai_ternary_linear(xs[2], p, s, y2, 1, N, K, 2, sp)
                     bz.bonsai_swiglu(y2, h, 1, F, sp)
-        with torch.cuda.stream(stream):
-            enq()
-            torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                enq()
-            for _ in range(3):
-                g.replay()
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = max(3, args.steps)
-            e0.record(stream)
-            for _ in range(reps):
-                g.replay()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        out["fused_us_per_layer" if fused else "unfused_us_per_layer"] = round(
-            e0.elapsed_time(e1) * 1e3 / (reps * LAYERS), 3)
+        g = capture(torch, stream, enq)
+        us = time_graph(torch, stream, g, max(3, args.steps)) * 1e3 / LAYERS
+        out["fused_us_per_layer" if fused else "unfused_us_per_layer"] = round(us, 3)
         del g
     out["workload"] = f"gate/up 5120 -> 2 x {F} at M=1 then SwiGLU, 64 distinct weight copies per replay, PQ2_0"
     return out
 
 
-def run_prefill(fmt, M, dev, bz, torch, peaks, peak_kind, steps):
-    """Prefill: M tokens through one layer's four projections (tcgen05 GEMM + FWHT pass)."""
+PREFILL_MS = (512, 2048, 8192)
+
+
+def measure_prefill(fmt, base, dev, bz, torch, args, peaks, peak_kind):
+    """Prefill: M tokens through each of the four projections (tcgen05 GEMM with the
+    rotation of x), for M in PREFILL_MS.  Every call is timed on its own with CUDA events,
+    after a write of twice the L2 size that evicts the previous call's data; at least 20
+    calls per (M, projection)."""
     from ternary_weight_02_b200 import inputs
     stream = torch.cuda.Stream(device=dev)
-    items = []
-    for i, (name, K, N) in enumerate(SHAPES):
-        t = torch.from_numpy(weights(fmt, i, N, K)).to(dev)
-        packed = bz.pack(fmt, t)
-        del t
-        s = torch.from_numpy(scales(fmt, i, N, K).view(np.int16)).to(dev).view(torch.float16)
-        x = torch.randn((M, K), device=dev, generator=torch.Generator(device=dev).manual_seed(i)).half()
-        items.append((name, K, N, packed, s, x, torch.empty((M, N), dtype=torch.float16, device=dev)))
-        bz.bonsai_reserve(M, N, K)
     sp = stream.cuda_stream
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    per = {}
-    total_flop = 0
-    with torch.cuda.stream(stream):
-        for name, K, N, packed, s, x, y in items:
-            for _ in range(2):
-                bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt, sp)
+    flush = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size, dtype=torch.uint8, device=dev)
+    calls = max(20, args.steps)
+    burst = float(peaks["bf16_tflops"])
+    grid = {}
+    summary = None
+    for M in PREFILL_MS:
+        per = {}
+        total_flop, layer_us = 0, 0.0
+        for i, (name, K, N) in enumerate(SHAPES):
+            packed, s = base[i]
+            x = torch.from_numpy(inputs.activations(200 + i, M, K).view(np.int16)).to(dev).view(torch.float16)
+            y = torch.empty((M, N), dtype=torch.float16, device=dev)
+            bz.bonsai_reserve(M, N, K)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
+            with nvtx(torch, f"prefill M={M} {name} {FMT_NAMES[fmt]}"), torch.cuda.stream(stream):
+                for _ in range(2):
+                    bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt, sp)
+                for a, b in ev:
+                    flush.fill_(1)
+                    a.record(stream)
+                    bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt, sp)
+                    b.record(stream)
             torch.cuda.synchronize()
-            e0.record(stream)
-            for _ in range(steps):
-                bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt, sp)
-            e1.record(stream)
-            torch.cuda.synchronize()
-            us = e0.elapsed_time(e1) * 1e3 / steps
+            us = sum(a.elapsed_time(b) for a, b in ev) * 1e3 / calls
             flop = 2 * M * N * K
             total_flop += flop
-            per[name] = {"us": round(us, 1), "tflops": round(flop / us / 1e6, 1)}
-    layer_us = sum(v["us"] for v in per.values())
-    # gate/up then SwiGLU: fused in the GEMM's epilogue against the GEMM and bonsai_swiglu
-    sw = {}
-    name, K, N, packed, s, x, y = items[2]
+            layer_us += us
+            per[name] = {"us": round(us, 1), "tflops": round(flop / us / 1e6, 1),
+                         "frac": round(flop / us / 1e6 / burst, 4), "calls": calls,
+                         "launches": bz.bonsai_launch_count(M, N, K, fmt)}
+            del x, y
+        grid[f"{FMT_NAMES[fmt]}_M{M}"] = {"per_projection": per, "us_per_layer": round(layer_us, 1),
+                                          "tflops": round(total_flop / layer_us / 1e6, 1)}
+        if M == args.prefill_m:
+            dom = per["gate_up"]
+            summary = {
+                "metric": "prefill GEMM TFLOP/s", "value": round(total_flop / layer_us / 1e6, 1), "unit": "TFLOP/s",
+                "workload": f"M={M} tokens x the four 27B-class projections, {FMT_NAMES[fmt]}, "
+                            f"FP16 x FP16 -> FP32 (tcgen05)",
+                "us_per_layer": round(layer_us, 1), "per_projection": per,
+                "roofline": {"bound": "tensor", "kernel": "gemm gate/up 5120->34816 (incl. the rotation of x)",
+                             "achieved": dom["tflops"], "peak": burst,
+                             "peak_kind": f"{peak_kind} bf16 burst (fp16 same dense rate)",
+                             "unit": "TFLOP/s", "frac": round(dom["tflops"] / burst, 4),
+                             "frac_of_sustained": round(dom["tflops"] / float(peaks["bf16_tflops_sustained"]), 4),
+                             "traffic": None},
+            }
+    out = {"grid": grid, "l2": "every call after a write of 2x the L2 size", "calls_per_entry": calls}
+    if summary is not None:
+        out.update(summary)
+    if fmt == 2 and args.prefill_m in PREFILL_MS:
+        out["swiglu_gate_up"] = measure_swiglu_prefill(fmt, base, dev, bz, torch, args.prefill_m, calls, flush)
+    return out
+
+
+def measure_swiglu_prefill(fmt, base, dev, bz, torch, M, calls, flush):
+    """gate/up then SwiGLU at M tokens: fused in the GEMM's epilogue against the GEMM and
+    bonsai_swiglu."""
+    from ternary_weight_02_b200 import inputs
+    stream = torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+    name, K, N = SHAPES[2]
+    packed, s = base[2]
     F = N // 2
+    x = torch.from_numpy(inputs.activations(202, M, K).view(np.int16)).to(dev).view(torch.float16)
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
     h = torch.empty((M, F), dtype=torch.float16, device=dev)
-    with torch.cuda.stream(stream):
-        for fused in (True, False):
-            def call():
-                if fused:
-                    bz.bonsai_ternary_linear_swiglu(x, packed, s, h, M, F, K, fmt, sp)
-                else:
-                    bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt, sp)
-                    bz.bonsai_swiglu(y, h, M, F, sp)
+    sw = {}
+    for fused in (True, False):
+        def call():
+            if fused:
+                bz.bonsai_ternary_linear_swiglu(x, packed, s, h, M, F, K, fmt, sp)
+            else:
+                bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt, sp)
+                bz.bonsai_swiglu(y, h, M, F, sp)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
+        with torch.cuda.stream(stream):
             call()
-            torch.cuda.synchronize()
-            e0.record(stream)
-            for _ in range(steps):
+            for a, b in ev:
+                flush.fill_(1)
+                a.record(stream)
                 call()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            sw["fused_us" if fused else "unfused_us"] = round(e0.elapsed_time(e1) * 1e3 / steps, 1)
+                b.record(stream)
+        torch.cuda.synchronize()
+        sw["fused_us" if fused else "unfused_us"] = round(sum(a.elapsed_time(b) for a, b in ev) * 1e3 / calls, 1)
     sw["workload"] = f"M={M} x gate/up 5120 -> 2 x {F} then SwiGLU, {FMT_NAMES[fmt]}"
-    burst = float(peaks["bf16_tflops"])
-    dom = per["gate_up"]
-    return {
-        "metric": "prefill GEMM TFLOP/s", "value": round(total_flop / layer_us / 1e6, 1), "unit": "TFLOP/s",
-        "workload": f"M={M} tokens x the four 27B-class projections, {FMT_NAMES[fmt]}, FP16 x FP16 -> FP32 (tcgen05)",
-        "us_per_layer": round(layer_us, 1), "per_projection": per, "swiglu_gate_up": sw,
-        "roofline": {"bound": "tensor", "kernel": "gemm gate/up 5120->34816 (incl. FWHT pass)",
-                     "achieved": dom["tflops"], "peak": burst, "peak_kind": f"{peak_kind} bf16 burst (fp16 same dense rate)",
-                     "unit": "TFLOP/s", "frac": round(dom["tflops"] / burst, 4),
-                     "frac_of_sustained": round(dom["tflops"] / float(peaks["bf16_tflops_sustained"]), 4),
-                     "traffic": None},
-    }
+    return sw
 
 
 def cpu_baseline(fmt):
-    """The checker on one layer of the stack (rank 0, N = 1): bounded CPU sample."""
+    """The checker on one layer of the stack (rank 0, N = 1): a bounded CPU sample, timed
+    on all host cores and on one."""
     import oracle
     from ternary_weight_02_b200 import inputs
     probs = []
     for i, (name, K, N) in enumerate(SHAPES):
         probs.append((inputs.activations(i, 1, K), oracle.pack(fmt, weights(fmt, i, N, K)),
                       scales(fmt, i, N, K), N, K))
-    t0 = time.perf_counter()
-    for x, p, s, N, K in probs:
-        oracle.ternary_linear(x, p, s, N, K, fmt)
-    dt = time.perf_counter() - t0
-    return {"value": round(step_bytes(fmt) / LAYERS / dt / 1e9, 3), "unit": "GB/s",
-            "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": f"one layer (4 projections, M=1, {FMT_NAMES[fmt]}) of the 64-layer stack, float64"}
+
+    def timed(threads):
+        t0 = time.perf_counter()
+        for x, p, s, N, K in probs:
+            oracle.ternary_linear(x, p, s, N, K, fmt, nthreads=threads)
+        return time.perf_counter() - t0
+
+    cores = oracle.max_threads()
+    dt_all, dt_one = timed(cores), timed(1)
+    layer = step_bytes(fmt) / LAYERS
+    sample = f"one layer (4 projections, M=1, {FMT_NAMES[fmt]}) of the 64-layer stack, float64"
+    return {"value": round(layer / dt_all / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": sample,
+            "single_thread": {"value": round(layer / dt_one / 1e9, 4), "unit": "GB/s", "cores": 1,
+                              "kind": "oracle", "sample": sample}}
 
 
 def run_case(args):
@@ -588,7 +721,9 @@ def main():
     ap.add_argument("--fmt", choices=list(FMTS), default="pq2")
     ap.add_argument("--both", type=int, default=1, help="also measure the other packing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--prefill-m", type=int, default=2048, help="tokens of the prefill GEMM line (0: skip)")
+    ap.add_argument("--prefill-m", type=int, default=2048,
+                    help="tokens of the prefill summary line, one of 512, 2048, 8192 (0: skip the prefill grid)")
+    ap.add_argument("--skinny", type=int, default=1, help="measure the M = 1..16 decode grid (PQ2_0, PTQ1_0)")
     ap.add_argument("--case", choices=["gemv", "imma", "gemm", "skinny"], help="run one projection only (profiler case)")
     ap.add_argument("--shape", choices=[n for n, _, _ in SHAPES], default="gate_up")
     ap.add_argument("--m", type=int, default=2048, help="tokens for --case gemm / skinny (skinny: at most 16)")

@@ -175,7 +175,9 @@ int bonsai_ternary_linear(const uint16_t *x, const uint8_t *packed, const uint16
  * partials, 0 = automatic.  BONSAI_ALGO_IMMA ignores it (its work split is fixed
  * by the shape and the SM count, so results are bitwise repeatable).
  * Returns BONSAI_ERR_ALGO if the chosen kernel cannot run the shape (e.g.
- * BONSAI_ALGO_GEMV with M > 1).  For measurement and testing of each kernel. */
+ * BONSAI_ALGO_GEMV with M > 1, or BONSAI_ALGO_IMMA on a shape whose grid would not fit
+ * on the current device at once, the limit the automatic choice also applies).  For
+ * measurement and testing of each kernel. */
 int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                                uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int algo,
                                int split_k, void *stream);
@@ -214,24 +216,27 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K);
  * Some callers cannot call cudaMalloc: code that runs while a CUDA graph is being
  * captured, allocators that must own every byte on the device, or hosts that forbid
  * allocation after start-up.  This entry point computes the same y as
- * bonsai_ternary_linear for M == 1 (the split-K lookup-table GEMV) but takes its
- * scratch -- split-K arrival counters and FP32 partial sums -- from one fixed array in
- * device memory that is part of the library image, instead of the per-device
- * workspace.  It never calls cudaMalloc, cudaFree or any allocating routine.  The
- * pages this library follows describe no such variant: it exists only for these
+ * bonsai_ternary_linear for M == 1 with the split-K lookup-table GEMV, but takes that
+ * kernel's scratch -- one FP32 partial sum per (512-weight K slice, output row) -- from
+ * one fixed array in device memory that is part of the library image, instead of the
+ * per-device workspace.  It never calls cudaMalloc, cudaFree or any allocating routine.
+ * The pages this library follows describe no such variant: it exists only for these
  * callers.
  *
- * Limits: M must be 1, K a multiple of 512, N <= 1048576, and (K / 512) * N <= 1048576
- * (the array holds 65536 counters and 2^20 FP32 partials, 4.25 MiB, kept by every
- * GPU that loads the library until the process exits); larger problems return
- * BONSAI_ERR_TOO_LARGE and launch nothing.  Inputs and output are caller-owned
- * device memory as for bonsai_ternary_linear.
+ * Formats: BONSAI_FMT_PTQ1_0 and BONSAI_FMT_PQ2_0 only; BONSAI_FMT_Q1_0 and
+ * BONSAI_FMT_PQ2_0_G64 return BONSAI_ERR_FMT.
+ * Limits: M must be 1, K a multiple of 512 and (K / 512) * N <= 1048576 (the array holds
+ * 2^20 FP32 partials, 4 MiB, kept by every GPU that loads the library until the process
+ * exits); other shapes return BONSAI_ERR_TOO_LARGE and launch nothing.  Checks run in
+ * the order format, shape, NULL pointer, alignment, then these limits.  Inputs and
+ * output are caller-owned device memory as for bonsai_ternary_linear.
  *
  * Set-up: the first call on each device looks up that device's copy of the array
  * (with that device current); make that first call before capturing any stream.
- * Every call shares the one array: it clears the counters it uses on `stream` before
- * its kernel, and calls whose work overlaps on the GPU (different streams, or
- * concurrent host threads) race on the array -- serialise them. */
+ * Every call shares the one array and leaves its partial sums there; each call writes
+ * every partial it reads before reading it, so nothing needs clearing between calls.
+ * Calls whose work overlaps on the GPU (different streams, or concurrent host threads)
+ * race on the array -- serialise them. */
 int bonsai_ternary_linear_noalloc(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                                   uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, void *stream);
 

@@ -47,7 +47,8 @@ int probe_current(int *dev_out, DeviceState **st_out) {
             cudaDeviceGetAttribute(&info.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&info.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&info.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&info.l2_bytes, cudaDevAttrL2CacheSize, dev) != cudaSuccess) {
+            cudaDeviceGetAttribute(&info.l2_bytes, cudaDevAttrL2CacheSize, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&info.smem_reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) {
             cudaGetLastError();
             return BONSAI_ERR_CUDA;
         }
@@ -319,6 +320,8 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
     rc = probe_current(&dev, &st);
     if (rc != BONSAI_OK) return rc;
     if (algo == BONSAI_ALGO_AUTO) chosen = resolve_algo(algo, M, N, K, fmt, &st->info);
+    // the integer GEMV's hand-over between CTAs needs its whole grid on the GPU at once
+    if (chosen == BONSAI_ALGO_IMMA && !gemv_imma_grid_fits(N, K, st->info)) return BONSAI_ERR_ALGO;
     Workspace ws;
     rc = ensure_workspace(*st, workspace_for(chosen, M, N, K, fmt, split_k, st->info),
                           chosen == BONSAI_ALGO_IMMA ? gemv_imma_zeroed_bytes(N, K) : 0, &ws);
@@ -405,6 +408,7 @@ int bonsai_launch_count(int64_t M, int64_t N, int64_t K, int fmt, int algo, int 
     rc = probe_current(&dev, &st);
     if (rc != BONSAI_OK) return rc;
     if (algo == BONSAI_ALGO_AUTO) chosen = resolve_algo(algo, M, N, K, fmt, &st->info);
+    if (chosen == BONSAI_ALGO_IMMA && !gemv_imma_grid_fits(N, K, st->info)) return BONSAI_ERR_ALGO;
     switch (chosen) {
         case BONSAI_ALGO_GEMV: return gemv_launches(N, K, fmt, split_k, st->info);
         case BONSAI_ALGO_IMMA: return 1;  // the rotation and quantisation of x are fused

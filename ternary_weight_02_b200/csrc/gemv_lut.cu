@@ -632,10 +632,7 @@ cudaError_t launch_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t
                         const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
     // the dynamic allocation must start below kTableAddr - kMiscBytes in the shared
     // window; it starts right after the per-block reserved area (no static shared memory)
-    static int reserved = -1;
-    if (reserved < 0 && cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, 0) != cudaSuccess)
-        return cudaErrorUnknown;
-    if (reserved + kMiscBytes > (int)kTableAddr) return cudaErrorNotSupported;
+    if (dev.smem_reserved + kMiscBytes > (int)kTableAddr) return cudaErrorNotSupported;
     if (pick_rows_mode(N, K, fmt, split_k, dev)) {
         const int64_t RB = (N + kRows - 1) / kRows;
         const int grid = (int)(RB < dev.sm_count ? RB : dev.sm_count);
@@ -645,24 +642,19 @@ cudaError_t launch_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t
     return launch_split(x, packed, scales, y, reinterpret_cast<float *>(ws.data), N, K, fmt, s, dev);
 }
 
-// Split-mode launch with caller-provided scratch (counters and partials), whatever the
-// shape; used by the no-allocation entry point.  partial_floats is the space the
-// scratch holds after its counters; returns cudaErrorInvalidValue if the shape needs more.
+// Split-mode launch with caller-provided scratch for the FP32 partials, whatever the shape;
+// used by the no-allocation entry point.  partial_floats is the space the scratch holds;
+// returns cudaErrorInvalidValue if the shape needs more.
 size_t gemv_split_partial_floats(int64_t N, int64_t K) {
     const int64_t S = K / kSliceK;  // PTQ1_0 / PQ2_0 (the no-allocation entry point's formats)
     return S > 1 ? (size_t)S * (size_t)N : 0;
 }
 
 cudaError_t launch_gemv_split_scratch(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
-                                      uint16_t *y, int64_t N, int64_t K, int fmt, unsigned int *counters,
-                                      float *partials, size_t partial_floats, cudaStream_t s,
-                                      const DeviceInfo &dev) {
+                                      uint16_t *y, int64_t N, int64_t K, int fmt, float *partials,
+                                      size_t partial_floats, cudaStream_t s, const DeviceInfo &dev) {
     if (gemv_split_partial_floats(N, K) > partial_floats) return cudaErrorInvalidValue;
-    static int reserved = -1;
-    if (reserved < 0 && cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, 0) != cudaSuccess)
-        return cudaErrorUnknown;
-    if (reserved + kMiscBytes > (int)kTableAddr) return cudaErrorNotSupported;
-    (void)counters;  // the in-order reduction kernel needs no arrival counters
+    if (dev.smem_reserved + kMiscBytes > (int)kTableAddr) return cudaErrorNotSupported;
     return launch_split(x, packed, scales, y, partials, N, K, fmt, s, dev);
 }
 

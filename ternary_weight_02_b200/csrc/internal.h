@@ -13,6 +13,7 @@ struct DeviceInfo {
     int major = 0, minor = 0;
     int smem_optin = 0;  // max dynamic shared memory per block (opt-in), bytes
     int l2_bytes = 0;
+    int smem_reserved = 0;  // shared memory the system reserves per block, bytes
 };
 
 // Split-K bookkeeping lives at the start of the workspace: kMaxTiles arrival
@@ -68,12 +69,11 @@ cudaError_t launch_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t
                         uint16_t *y, int64_t N, int64_t K, int fmt, int split_k,
                         const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
 
-// split-mode GEMV on caller-provided scratch (no-allocation entry point)
+// split-mode GEMV on caller-provided scratch for its FP32 partials (no-allocation entry point)
 size_t gemv_split_partial_floats(int64_t N, int64_t K);
 cudaError_t launch_gemv_split_scratch(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
-                                      uint16_t *y, int64_t N, int64_t K, int fmt, unsigned int *counters,
-                                      float *partials, size_t partial_floats, cudaStream_t s,
-                                      const DeviceInfo &dev);
+                                      uint16_t *y, int64_t N, int64_t K, int fmt, float *partials,
+                                      size_t partial_floats, cudaStream_t s, const DeviceInfo &dev);
 // current device's properties (the same probe the other entry points use)
 int current_device_info(DeviceInfo *out);
 

@@ -3,10 +3,11 @@
 // captured, allocators that must own every byte of the device, hosts that forbid
 // allocation after start-up).
 //
-// The split-K GEMV needs scratch: one arrival counter per 16-row block and one FP32
-// partial per (K slice, row).  Here that scratch is a fixed array in the library's own
-// device image instead of the per-device workspace, so the call never allocates.
-// Every GPU that loads the library holds the array (4.25 MiB) until the process exits.
+// The split-K GEMV needs scratch: one FP32 partial per (512-weight K slice, row), summed
+// in slice order by its second kernel.  Here that scratch is a fixed array in the
+// library's own device image instead of the per-device workspace, so the call never
+// allocates.  Every GPU that loads the library holds the array (4 MiB) until the process
+// exits.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -17,18 +18,16 @@
 namespace bonsai {
 namespace {
 
-constexpr int kScratchCounters = 65536;      // one per 16-row block: N <= 1048576
 constexpr int kScratchPartials = 1 << 20;    // FP32 partials: (K / 512) * N <= 2^20
 constexpr int kMaxDevices = 64;
 
-// [counters (kScratchCounters x uint32) | partials (kScratchPartials x FP32)]
-static __device__ __align__(256) unsigned int g_scratch[kScratchCounters + kScratchPartials];
+static __device__ __align__(256) float g_scratch[kScratchPartials];
 
 std::mutex g_setup_mutex;
-unsigned int *g_scratch_addr[kMaxDevices];  // device address of g_scratch, per device
+float *g_scratch_addr[kMaxDevices];  // device address of g_scratch, per device
 
 // Looks up the current device's copy of the array once (that device must be current).
-int scratch_for_current_device(unsigned int **out) {
+int scratch_for_current_device(float **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         cudaGetLastError();
@@ -41,7 +40,7 @@ int scratch_for_current_device(unsigned int **out) {
             cudaGetLastError();
             return BONSAI_ERR_CUDA;
         }
-        g_scratch_addr[dev] = static_cast<unsigned int *>(p);
+        g_scratch_addr[dev] = static_cast<float *>(p);
     }
     *out = g_scratch_addr[dev];
     return BONSAI_OK;
@@ -58,31 +57,23 @@ extern "C" int bonsai_ternary_linear_noalloc(const uint16_t *x, const uint8_t *p
     if (fmt != BONSAI_FMT_PTQ1_0 && fmt != BONSAI_FMT_PQ2_0) return BONSAI_ERR_FMT;
     if (M < 0 || N < 0 || K <= 0 || K % 128 != 0) return BONSAI_ERR_SHAPE;
     if (M == 0 || N == 0) return BONSAI_OK;
-    if (M != 1 || K % 512 != 0) return BONSAI_ERR_TOO_LARGE;
-    if ((N + 15) / 16 > kScratchCounters || gemv_split_partial_floats(N, K) > (size_t)kScratchPartials)
-        return BONSAI_ERR_TOO_LARGE;
     if (!x || !packed || !scales || !y) return BONSAI_ERR_NULL;
     const uintptr_t mis = reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(packed) |
                           reinterpret_cast<uintptr_t>(scales) | reinterpret_cast<uintptr_t>(y);
     if (mis & 15u) return BONSAI_ERR_ALIGN;
+    if (M != 1 || K % 512 != 0 || gemv_split_partial_floats(N, K) > (size_t)kScratchPartials)
+        return BONSAI_ERR_TOO_LARGE;
 
     DeviceInfo info;
     int rc = current_device_info(&info);
     if (rc != BONSAI_OK) return rc;
-    unsigned int *scratch = nullptr;
-    rc = scratch_for_current_device(&scratch);
+    float *partials = nullptr;
+    rc = scratch_for_current_device(&partials);
     if (rc != BONSAI_OK) return rc;
-
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the counters must start at zero; the array keeps whatever the last call left
-    const size_t counter_bytes = (size_t)((N + 15) / 16) * sizeof(unsigned int);
-    if (cudaMemsetAsync(scratch, 0, counter_bytes, s) != cudaSuccess) {
-        cudaGetLastError();
-        return BONSAI_ERR_CUDA;
-    }
-    float *partials = reinterpret_cast<float *>(scratch + kScratchCounters);
-    const cudaError_t e = launch_gemv_split_scratch(x, packed, scales, y, N, K, fmt, scratch, partials,
-                                                    (size_t)kScratchPartials, s, info);
+    // Every partial the reduction reads is written by the same call first, so nothing in
+    // the array needs clearing; the array keeps whatever the last call left.
+    const cudaError_t e = launch_gemv_split_scratch(x, packed, scales, y, N, K, fmt, partials,
+                                                    (size_t)kScratchPartials, static_cast<cudaStream_t>(stream), info);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return BONSAI_ERR_CUDA;

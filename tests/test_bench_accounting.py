@@ -42,16 +42,12 @@ def test_whole_job_rate():
     assert abs(bench.whole_job_gbs(10**9, 8, 1.0) - 8000.0) < 1e-9
 
 
-def test_clock_samples_parse_reasons_and_median():
-    out = "\n".join([
-        "0, 1965, 1965, 812.4, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
-        "0, 1950, 1965, 990.1, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
-        "0, 1965, 1965, 1001.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
-        "garbage line",
-        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
-    ])
-    c = bench.parse_clock_samples(out)
+def test_clock_samples_median_and_reasons():
+    idle, cap = 0x1, 0x4
+    samples = [(1965, 1965, 0), (1950, 1965, cap), (1965, 1965, cap | idle), (0, 1965, 0), (None, None, 0)]
+    c = bench.summarize_clock_samples(samples)
     assert c == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
-    thermal = "0, 1400, 1965, 700, 0x48, Active, Not Active, Active, Not Active"
-    assert bench.parse_clock_samples(thermal)["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
-    assert bench.parse_clock_samples("") is None
+    thermal = [(1400, 1965, 0x8 | 0x40 | 0x20)]
+    assert bench.summarize_clock_samples(thermal)["reasons"] == [
+        "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"]
+    assert bench.summarize_clock_samples([]) is None

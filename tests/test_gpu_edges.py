@@ -1,0 +1,167 @@
+"""GPU parity on inputs that stress one kernel's number format or its dispatch, against
+the float64 checker with the parity bar (rel-L2 <= 1e-3, max abs <= 1e-2 * rms).
+
+* A dominant element inside every 128-block: x = c * Hn e_j + N(0,1) noise, so that the
+  rotated block is c e_j plus noise.  The rotation exists to spread such outliers
+  ("Bonsai 2，把27B压进6个G", section 它怎么做到的); here the outlier is what the rotation
+  produces.  The integer GEMV holds each rotated block as 16-bit fixed point scaled to
+  its largest element, so the noise elements keep only about 4 significant bits: the rows
+  whose trit at j is 0 carry exactly that coarse part.  Every linear kernel gets it.
+* The skinny batches at the full qkv shape, and PTQ1_0 batches of 2 and 16 tokens at
+  full 27B-class shapes (they take the prefill GEMM).
+* The automatic choice at batch 1 on both sides of the integer GEMV's grid limit.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from tests.gpu_util import Problem, to_numpy_f16
+
+pytestmark = pytest.mark.gpu
+
+PTQ1, PQ2, Q1, G64 = oracle.FMT_PTQ1_0, oracle.FMT_PQ2_0, oracle.FMT_Q1_0, oracle.FMT_PQ2_0_G64
+
+
+@pytest.fixture(scope="module")
+def bz():
+    import torch
+    from ternary_weight_02_b200 import bonsai
+    assert bonsai.bonsai_check_device() == bonsai.BONSAI_OK
+    torch.cuda.init()
+    return bonsai
+
+
+def _run(bz, p, algo, split_k=0):
+    import torch
+    x, packed, scales = p.device()
+    y = torch.full((p.M, p.N), float("nan"), dtype=torch.float16, device="cuda")
+    bz.bonsai_ternary_linear_algo(x, packed, scales, y, p.M, p.N, p.K, p.fmt, algo, split_k)
+    torch.cuda.synchronize()
+    return to_numpy_f16(y)
+
+
+def dominant_problem(M, N, K, fmt, c=1000.0, seed=21):
+    """Seeded problem whose x has, in every 128-block b of every token, the column
+    j_b = (37 b + 11 m) mod 128 of the normalised Hadamard matrix times c added to
+    N(0,1) noise: after the rotation that block is c at j_b plus rotated noise."""
+    p = Problem(M, N, K, fmt, seed=seed)
+    G = K // 128
+    delta = np.zeros((M, K), dtype=np.float64)
+    for m in range(M):
+        for b in range(G):
+            delta[m, 128 * b + (37 * b + 11 * m) % 128] = c
+    spike = oracle.hadamard128(delta)  # Hn is its own inverse: rotating spike gives delta
+    p.x = (p.x.astype(np.float64) + spike).astype(np.float16)
+    return p
+
+
+def _rotated_peaks(p):
+    """Per token and block: the rotated block's largest magnitude over its median one."""
+    xr = oracle.hadamard128(p.x.astype(np.float64)).reshape(p.M, -1, 128)
+    a = np.abs(xr)
+    return a.max(axis=2) / np.median(a, axis=2)
+
+
+DOMINANT_CASES = [
+    # (algo, fmt, M, N, K): the integer GEMV, the lookup-table GEMV, the skinny kernel,
+    # the prefill GEMM and the plain kernel, each on every packing it takes
+    ("IMMA", PQ2, 1, 1000, 2048), ("IMMA", G64, 1, 1000, 2048), ("IMMA", PQ2, 1, 7168, 5120),
+    ("GEMV", PTQ1, 1, 1000, 2048), ("GEMV", PQ2, 1, 1000, 2048), ("GEMV", Q1, 1, 1000, 2048),
+    ("GEMV", G64, 1, 1000, 2048),
+    ("SKINNY", PQ2, 4, 1000, 2048), ("SKINNY", G64, 4, 1000, 2048), ("SKINNY", Q1, 4, 1000, 2048),
+    ("SKINNY", PQ2, 16, 700, 1024),
+    ("GEMM", PTQ1, 200, 600, 1024), ("GEMM", PQ2, 200, 600, 1024), ("GEMM", Q1, 200, 600, 1024),
+    ("GEMM", G64, 200, 600, 1024),
+    ("SIMPLE", PTQ1, 3, 300, 1024), ("SIMPLE", PQ2, 3, 300, 1024), ("SIMPLE", Q1, 3, 300, 1024),
+    ("SIMPLE", G64, 3, 300, 1024),
+]
+
+
+@pytest.mark.parametrize("algo,fmt,M,N,K", DOMINANT_CASES)
+def test_dominant_element_in_every_block(bz, algo, fmt, M, N, K):
+    p = dominant_problem(M, N, K, fmt)
+    # the input really is what the test claims: one element per rotated block stands
+    # hundreds of times above the block's typical element
+    assert np.all(_rotated_peaks(p) > 300)
+    got = _run(bz, p, getattr(bz, f"BONSAI_ALGO_{algo}"))
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+@pytest.mark.parametrize("fmt", [PQ2, G64])
+@pytest.mark.parametrize("c", [1.0, 1000.0])
+def test_imma_error_within_the_fixed_point_step(bz, fmt, c):
+    """Every output of the integer GEMV lies within the error its arithmetic allows.  The
+    kernel holds rotated block g as integers q = rint(x' 2^e), with 2^e the power of two
+    that puts the block's largest |x'| in [2^13, 2^14); every product and sum after that is
+    exact, so each element is off by at most half a step 2^-e, and y[n] by at most
+    sum_g s[n,g] * (nonzero trits of row n in g) * 2^-e / 2, plus the FP16 rounding of y.
+    (The bound takes the next power of two up for 2^-e, in case the kernel's FP32 maximum
+    lands on the other side of a power of two.)  With c = 1000 the noise elements of each
+    block keep only about four significant bits, so rows whose trits skip the dominant
+    positions carry an error near this bound."""
+    M, N, K = 1, 4096, 1024
+    p = dominant_problem(M, N, K, fmt, c=c)
+    got = _run(bz, p, bz.BONSAI_ALGO_IMMA)[0]
+    ref = p.oracle_y()[0]
+    G = K // 128
+    xr = oracle.hadamard128(p.x.astype(np.float64))[0].reshape(G, 128)
+    E = np.floor(np.log2(np.abs(xr).max(axis=1)))
+    step = 2.0 ** (E - 12)  # one power of two above the kernel's step
+    gs = oracle.scale_group(fmt)
+    s = p.scales.astype(np.float64).reshape(N, K // gs)
+    nz = (p.trits != 0).reshape(N, K // gs, gs).sum(axis=2)
+    bound = (s * nz * np.repeat(step, 128 // gs)[None, :]).sum(axis=1) * 0.5 * 1.001
+    bound += 2.0 ** -11 * np.abs(ref) + 2.0 ** -24
+    err = np.abs(got - ref)
+    assert np.all(err <= bound), float(np.max(err / bound))
+    ok, rel, mx = oracle.compare(got[None, :], ref[None, :])
+    assert ok, (rel, mx)
+
+
+@pytest.mark.parametrize("fmt", [PQ2, G64, Q1])
+@pytest.mark.parametrize("M", [2, 16])
+def test_skinny_full_qkv_shape(bz, fmt, M):
+    """The qkv projection (5120 -> 7168) in skinny batches, every output."""
+    p = Problem(M, 7168, 5120, fmt, seed=40 + M)
+    got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+@pytest.mark.parametrize("M", [2, 16])
+@pytest.mark.parametrize("K,N", [(5120, 7168), (17408, 5120), (5120, 34816)])
+def test_ptq1_small_batches_full_shapes(bz, M, K, N):
+    """PTQ1_0 batches of 2 and 16 tokens at full 27B-class shapes through the default
+    entry point, every output."""
+    p = Problem(M, N, K, PTQ1, seed=50 + M)
+    got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+def test_auto_batch1_on_both_sides_of_the_imma_grid_limit(bz):
+    """At batch 1, PQ2_0, the automatic choice takes the integer GEMV only while its grid
+    fits on the GPU at once.  N = 45440 at K = 5120 is 14,200 items of 32 rows x 512
+    weights (fits on 148 SMs at 96 items each); N = 46080 is 14,400 (does not), and goes
+    to the lookup-table GEMV.  Both against the checker; an explicit integer-GEMV request
+    past the limit is refused."""
+    import torch
+    props = torch.cuda.get_device_properties(0)
+    limit = props.multi_processor_count * 96
+    K = 5120
+    for N in (45440, 46080):
+        items = (N // 32) * (K // 512)
+        fits = items <= limit
+        launches = bz.bonsai_launch_count(1, N, K, PQ2)
+        want = 1 if fits else bz.bonsai_launch_count(1, N, K, PQ2, bz.BONSAI_ALGO_GEMV)
+        assert launches == want, (N, items, limit, launches)
+        p = Problem(1, N, K, PQ2, seed=N)
+        got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
+        ok, rel, mx = oracle.compare(got, p.oracle_y())
+        assert ok, (N, rel, mx)
+        if not fits:
+            x, packed, scales = p.device()
+            y = torch.empty((1, N), dtype=torch.float16, device="cuda")
+            with pytest.raises(bz.BonsaiError):
+                bz.bonsai_ternary_linear_algo(x, packed, scales, y, 1, N, K, PQ2, bz.BONSAI_ALGO_IMMA)

@@ -2,7 +2,8 @@
 (code running during CUDA-graph capture, allocators that own every byte of the
 device, hosts that forbid allocation after start-up).  It runs the batch-1 layer on
 a fixed scratch array inside the library's device image; its output must match the
-regular entry point's within the parity bar, call after call."""
+regular entry point's and the float64 checker's within the parity bar, call after
+call."""
 import numpy as np
 import pytest
 
@@ -32,6 +33,8 @@ def test_noalloc_matches_regular_entry_point_two_calls(fmt):
         got, want = to_numpy_f16(y_na), to_numpy_f16(y_reg)
         ok, rel, mx = oracle.compare(got, want)
         assert ok, (N, K, rel, mx)
+        ok, rel, mx = oracle.compare(got, p.oracle_y())
+        assert ok, ("checker", N, K, rel, mx)
 
 
 def test_noalloc_rejects_beyond_its_scratch():
@@ -47,3 +50,7 @@ def test_noalloc_rejects_beyond_its_scratch():
     assert L.bonsai_ternary_linear_noalloc(p, p, p, p, 2, 64, 512, 2, stream) == bz.BONSAI_ERR_TOO_LARGE
     assert L.bonsai_ternary_linear_noalloc(p, p, p, p, 1, 64, 384, 2, stream) == bz.BONSAI_ERR_TOO_LARGE
     assert "scratch" in bz.bonsai_status_string(bz.BONSAI_ERR_TOO_LARGE)
+    # only PTQ1_0 and PQ2_0; a NULL pointer is reported before the size limit
+    assert L.bonsai_ternary_linear_noalloc(p, p, p, p, 1, 64, 512, 3, stream) == bz.BONSAI_ERR_FMT
+    assert L.bonsai_ternary_linear_noalloc(p, p, p, p, 1, 64, 512, 4, stream) == bz.BONSAI_ERR_FMT
+    assert L.bonsai_ternary_linear_noalloc(p, None, p, p, 1, 40000, 17408, 2, stream) == bz.BONSAI_ERR_NULL
