@@ -63,9 +63,10 @@
  *   - Every wait inside a kernel (a barrier on a copy in flight, a hand-over
  *     between CTAs of the same grid) gives up after a bounded number of polls;
  *     the call then writes NaN to the outputs it could not finish instead of
- *     hanging the GPU.  Such a call may leave hand-over state behind in the
- *     workspace, so after NaN outputs of this kind call bonsai_shutdown(): the
- *     next call re-creates the workspace, zeroed.
+ *     hanging the GPU, and sets a bit in the device status word that
+ *     bonsai_device_status() reads.  Hand-over data carries the number of the call
+ *     that wrote it, so a piece that arrives after its reader gave up is never taken
+ *     for a later call's: the next call runs normally.
  */
 #ifndef BONSAI_H
 #define BONSAI_H
@@ -239,6 +240,28 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K);
  * race on the array -- serialise them. */
 int bonsai_ternary_linear_noalloc(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                                   uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, void *stream);
+
+/* Device status bits, set by a kernel whose bounded wait gave up (the call then wrote
+ * NaN for the outputs it could not finish; see the conventions above).  They stay set
+ * until cleared by bonsai_device_status. */
+#define BONSAI_DEVICE_GEMV_COPY_TIMEOUT 1u  /* integer GEMV: a weight copy never landed      */
+#define BONSAI_DEVICE_GEMV_PIECE_TIMEOUT 2u /* integer GEMV: a split tile's later piece, or  */
+                                            /* its hand-over, never came                      */
+#define BONSAI_DEVICE_GEMM_TIMEOUT 4u       /* prefill GEMM: a barrier or hand-over wait gave up */
+
+/* Reads the calling device's status bits into *bits after synchronising `stream` (the
+ * stream of the calls in question), and clears them when `clear` is non-zero.  *bits is 0
+ * when no call has run on the device yet.  Returns BONSAI_ERR_NULL for a NULL bits,
+ * BONSAI_ERR_CUDA if the copy or the synchronisation fails.  The pages describe no such
+ * call; it reports the bounded waits of this implementation. */
+int bonsai_device_status(void *stream, uint32_t *bits, int clear);
+
+/* Test hook.  While enabled (enable != 0), the waits of the integer tensor-core GEMV for
+ * the later pieces of its split row tiles, and of the prefill GEMM for its hand-over
+ * flags, look for a call number that no CTA writes and give up after 64 polls: the calls
+ * then write NaN for those tiles and set the status bits, without any fault, so that the
+ * timeout path can be tested.  Off by default; applies to calls launched while enabled. */
+int bonsai_debug_force_timeouts(int enable);
 
 /* Frees the workspaces of every device (after synchronising each).  The
  * library stays usable: the next call allocates again. */

@@ -32,6 +32,10 @@ BONSAI_ERR_NOMEM = -7
 BONSAI_ERR_ALGO = -8
 BONSAI_ERR_TOO_LARGE = -9
 
+BONSAI_DEVICE_GEMV_COPY_TIMEOUT = 1
+BONSAI_DEVICE_GEMV_PIECE_TIMEOUT = 2
+BONSAI_DEVICE_GEMM_TIMEOUT = 4
+
 BONSAI_ALGO_AUTO = 0
 BONSAI_ALGO_SIMPLE = 1
 BONSAI_ALGO_GEMV = 2
@@ -67,6 +71,8 @@ _SIGS = {
     "bonsai_swiglu": (_int, [_p, _p, _i64, _i64, _p]),
     "bonsai_ternary_linear_swiglu": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _int, _p]),
     "bonsai_reserve": (_int, [_i64, _i64, _i64]),
+    "bonsai_device_status": (_int, [_p, ctypes.POINTER(ctypes.c_uint32), _int]),
+    "bonsai_debug_force_timeouts": (_int, [_int]),
     "bonsai_shutdown": (None, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -182,6 +188,19 @@ def bonsai_launch_count(M: int, N: int, K: int, fmt: int, algo: int = BONSAI_ALG
 
 def bonsai_reserve(M: int, N: int, K: int) -> None:
     _check(_lib.bonsai_reserve(M, N, K), "bonsai_reserve")
+
+
+def bonsai_device_status(stream=None, clear: bool = False) -> int:
+    """The calling device's status bits (BONSAI_DEVICE_*), after synchronising `stream`."""
+    bits = ctypes.c_uint32(0)
+    _check(_lib.bonsai_device_status(_stream(stream), ctypes.byref(bits), 1 if clear else 0),
+           "bonsai_device_status")
+    return int(bits.value)
+
+
+def bonsai_debug_force_timeouts(enable: bool) -> None:
+    """Test hook: cross-CTA waits give up (NaN outputs, status bits) while enabled."""
+    _check(_lib.bonsai_debug_force_timeouts(1 if enable else 0), "bonsai_debug_force_timeouts")
 
 
 def bonsai_shutdown() -> None:

@@ -33,6 +33,7 @@ struct DeviceState {
 
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
+bool g_force_wait_timeouts = false;  // test hook (bonsai_debug_force_timeouts)
 
 int probe_current(int *dev_out, DeviceState **st_out) {
     int dev = -1;
@@ -57,6 +58,7 @@ int probe_current(int *dev_out, DeviceState **st_out) {
         st.status = (info.major == 10 && info.minor == 0) ? BONSAI_OK : BONSAI_ERR_ARCH;
         st.probed = true;
     }
+    st.info.force_wait_timeouts = g_force_wait_timeouts;
     *dev_out = dev;
     *st_out = &st;
     return st.status;
@@ -67,6 +69,8 @@ int probe_current(int *dev_out, DeviceState **st_out) {
 // work in flight may still use the old buffer).
 int ensure_workspace(DeviceState &st, size_t data_bytes, size_t zeroed_bytes, Workspace *ws) {
     const size_t need = kCounterBytes + ((data_bytes + 255) / 256) * 256;
+    // the zeroed region always holds at least the control words (the device status word)
+    if (zeroed_bytes < kCtlRegionBytes) zeroed_bytes = kCtlRegionBytes;
     if (st.ws_bytes < need) {
         if (st.ws_base) {
             if (cudaDeviceSynchronize() != cudaSuccess) return BONSAI_ERR_CUDA;
@@ -448,6 +452,34 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
     // + the tail in which a non-fused bonsai_ternary_linear_swiglu keeps its M x N output
     need = (need + 255) / 256 * 256 + (size_t)M * (size_t)N * 2;
     return ensure_workspace(*st, need, zneed, &ws);
+}
+
+int bonsai_device_status(void *stream, uint32_t *bits, int clear) {
+    if (!bits) return BONSAI_ERR_NULL;
+    *bits = 0;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    int dev;
+    DeviceState *st;
+    int rc = probe_current(&dev, &st);
+    if (rc != BONSAI_OK) return rc;
+    if (!st->zb_base) return BONSAI_OK;  // no call has run on this device: nothing to report
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int *word = static_cast<unsigned int *>(st->zb_base) + kCtlStatus;
+    unsigned int host = 0;
+    if (cudaMemcpyAsync(&host, word, sizeof(host), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        (clear && cudaMemsetAsync(word, 0, sizeof(unsigned int), s) != cudaSuccess) ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return BONSAI_ERR_CUDA;
+    }
+    *bits = host;
+    return BONSAI_OK;
+}
+
+int bonsai_debug_force_timeouts(int enable) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    g_force_wait_timeouts = enable != 0;
+    return BONSAI_OK;
 }
 
 void bonsai_shutdown(void) {

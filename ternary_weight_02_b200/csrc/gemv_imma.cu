@@ -19,14 +19,17 @@
 //   the weights of group gl meet a B operand that is non-zero in columns 2gl, 2gl+1
 //   only, so four groups accumulate side by side in one fragment.
 // * Activations as 16-bit block fixed point.  Per 128-group, x~ = rint(x' * 2^e) with
-//   the power of two chosen so that |x~| <= 2^14, stored as signed bytes hi * 256 + lo.
-//   With c = t + 1 the PQ2_0 code of a weight, the MMA gives sum c*hi and sum c*lo
-//   exactly in int32, so sum t*x~ = 256*Dhi + Dlo - sum x~ exactly; one FP32 multiply by
-//   s * 2^-e per (row, group) follows.  (The rounding of x' to x~ is the only
-//   approximation; it is finer than FP16 for every element of the group.)  With 64-weight
-//   scales the MMA chain runs over the group's first two 32-weight subslots, is folded
-//   with the first half's sum of x~ and scale, then over the last two: the same
-//   accumulator registers, one more fold per group.
+//   the power of two chosen so that the group's largest |x'| * 2^e lies in [2^13, 2^14),
+//   stored as signed bytes hi * 256 + lo.  With c = t + 1 the PQ2_0 code of a weight, the
+//   MMA gives sum c*hi and sum c*lo exactly in int32, so sum t*x~ = 256*Dhi + Dlo - sum x~
+//   exactly; one FP32 multiply by s * 2^-e per (row, group) follows.  The rounding of x'
+//   to x~ is the only approximation: every element is off by at most half a step 2^-e,
+//   2^-15 to 2^-14 of the group's largest element.  That is finer than FP16 for the
+//   group's elements above about 1/8 of its largest and coarser for those below (an
+//   element 1000 times smaller than the group's largest keeps about 4 significant bits).
+//   With 64-weight scales the MMA chain runs over the group's first two 32-weight
+//   subslots, is folded with the first half's sum of x~ and scale, then over the last
+//   two: the same accumulator registers, one more fold per group.
 // * One launch.  16 warps per CTA, each feeding its own ring of item buffers (a TMA
 //   box of trits, and the item's scales by cp.async).  After waiting for the previous
 //   kernel, every CTA loads all of x (each CTA starting at a different group quad), then
@@ -41,13 +44,17 @@
 //   bank conflicts).
 // * Work split.  Items are ordered (row tile, K chunk); each CTA takes one contiguous
 //   range, dealt round-robin to its consumer warps.  Every item's 32 row sums go to a
-//   slot in shared memory; at the end each row tile's slots are added in K order.  A
-//   tile shared with a neighbouring CTA goes through FP32 partials in the workspace:
-//   the CTA whose arrival completes the tile adds the pieces in K order (deterministic)
-//   and resets the tile's counter to zero for the next call.
-// * Every mbarrier wait is bounded.  A warp whose wait gives up stops refilling, turns
+//   slot in shared memory; the warp that completes the CTA's part of a row tile adds its
+//   slots in K order.  A tile shared with the following CTAs goes through 64-bit
+//   (value, epoch) pairs in the workspace: the CTA holding the tile's first item adds
+//   the later pieces in K order (deterministic).  The epoch is a call number kept in
+//   the workspace's control words, so stored pairs never need clearing and a late pair
+//   can never be taken for a later call's.
+// * Every wait is bounded.  A warp whose mbarrier wait gives up stops refilling, turns
 //   its results into NaN (keeping the partial-sum protocol intact) and, before the
-//   CTA exits, waits (again bounded) for the copies it had started.
+//   CTA exits, waits (again bounded) for the copies it had started; an owner whose wait
+//   for a later piece gives up writes NaN for that tile.  Both set a bit in the
+//   workspace's device status word.
 #include "common.cuh"
 #include "internal.h"
 #include "tma.cuh"
@@ -95,7 +102,7 @@ __host__ __device__ inline Layout make_layout(int K) {
     L.tcnt = L.slots + kMaxCtaItems * kItemRows * 4;
     L.zero = (L.tcnt + kMaxCtaTiles * 4 + 15) & ~15;  // 128-bit loads read the zero bytes
     L.full = L.zero + 256;
-    L.total = L.full + kConsumers * kStages * 8 + 1024;  // + room to align the base
+    L.total = L.full + kConsumers * kStages * 8 + 16 + 1024;  // + the epoch word, room to align the base
     return L;
 }
 
@@ -226,10 +233,10 @@ __device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag,
 // ---------------------------------------------------------------- the GEMV
 
 // A later piece's partial sums travel as 64-bit (value, epoch) pairs, one per row: an
-// aligned 64-bit access is single-copy atomic, so a reader that sees epoch 1 sees the
-// value stored with it -- no fence on either side.
-__device__ __forceinline__ void st_pair(uint64_t *p, float v) {
-    const uint64_t w = (uint64_t)__float_as_uint(v) | ((uint64_t)1 << 32);
+// aligned 64-bit access is single-copy atomic, so a reader that sees this call's epoch
+// sees the value stored with it -- no fence on either side.
+__device__ __forceinline__ void st_pair(uint64_t *p, float v, uint32_t epoch) {
+    const uint64_t w = (uint64_t)__float_as_uint(v) | ((uint64_t)epoch << 32);
     asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
 }
 __device__ __forceinline__ uint64_t ld_pair(const uint64_t *p) {
@@ -237,21 +244,21 @@ __device__ __forceinline__ uint64_t ld_pair(const uint64_t *p) {
     asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
     return w;
 }
-// Bounded wait, by the whole warp, for the 32 pairs at p (one per lane) to carry epoch 1;
-// returns this lane's value, or NaN if they did not all come within kSpinLimit polls.
-// The pairs are written by a CTA with a higher index, which writes them before it waits
-// on anything itself.
-__device__ __forceinline__ float wait_pairs(uint64_t *p, int lane) {
-    for (uint32_t i = 0; i < kSpinLimit; i++) {
+// Bounded wait, by the whole warp, for the 32 pairs at p (one per lane) to carry the
+// epoch `want`; returns this lane's value, or NaN (and sets the status bit) if they did
+// not all come within `limit` polls.  The pairs are written by a CTA with a higher index,
+// which writes them before it waits on anything itself.
+__device__ __forceinline__ float wait_pairs(const uint64_t *p, int lane, uint32_t want, uint32_t limit,
+                                            unsigned int *status) {
+    for (uint32_t i = 0; i < limit; i++) {
         const uint64_t w = ld_pair(p + lane);
-        if (__all_sync(0xffffffffu, (w >> 32) == 1u)) {
-            asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p + lane), "l"((uint64_t)0) : "memory");
-            return __uint_as_float((uint32_t)w);  // (cleared for the next call)
-        }
+        if (__all_sync(0xffffffffu, (uint32_t)(w >> 32) == want)) return __uint_as_float((uint32_t)w);
         __nanosleep(32);
     }
+    if (lane == 0) atomicOr(status, kDevStatusGemvPieceTimeout);
     return __int_as_float(0x7fc00000);
 }
+
 
 
 // kAsyncScales: K is a multiple of 512, so an item's four (g64: eight) scales of a row are
@@ -266,10 +273,17 @@ __device__ __forceinline__ float wait_pairs(uint64_t *p, int lane) {
 // TMA boxes), so that the lane that finishes row r < 16 of the tile finds the matching up
 // row in lane r + 16.  (When F % 16 != 0 the last tile's rows past gate row F - 1 belong to
 // no output and are not written; its up box reads zeros past row 2F - 1.)
+//
+// ctl: the workspace's control words: the 64-bit call counter (calls counted so far in
+// its high half, CTAs of the running call that have read it in its low half) and the
+// sticky status bits.  wait_limit and epoch_skew are the polls of a wait for a later piece
+// and an offset added to the epoch it waits for: kSpinLimit and 0, except under the test
+// hook that makes those waits give up.
 template <bool kAsyncScales, bool kSwiglu, bool kG64>
 __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const __grid_constant__ CUtensorMap wmap, const uint16_t *__restrict__ x, const uint16_t *__restrict__ scales,
-    uint16_t *__restrict__ y, uint64_t *__restrict__ partials, int N, int K, int F) {
+    uint16_t *__restrict__ y, uint64_t *__restrict__ partials, unsigned int *__restrict__ ctl, int N, int K, int F,
+    uint32_t wait_limit, uint32_t epoch_skew) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -297,6 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     int *tile_cnt = reinterpret_cast<int *>(smem + L.tcnt);  // items done, per row tile of the range
     uint8_t *zero = smem + L.zero;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.full) + warp * kStages;
+    uint32_t *epoch_s = reinterpret_cast<uint32_t *>(smem + L.full + kConsumers * kStages * 8);
+    unsigned int *status = ctl + kCtlStatus;
 
     // item q of this warp: c0 + warp + q * kConsumers -> ring stage q % kStages.  Lane 0
     // starts the TMA box; lane r copies the item's four scales of row r (cp.async); one
@@ -350,6 +366,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     // and the call's time is set by its slowest CTA (measured: faster on every shape).
     pdl_launch_dependents();
     pdl_wait();  // x, y and the workspace may belong to the previous kernel
+    // This call's epoch is one more than the calls counted so far.  One atomic add reads the
+    // count and counts this CTA in the same 64-bit word, so every CTA sees the same count;
+    // the last CTA to arrive advances it for the next call (its result is needed only after
+    // the x~ build, which hides its latency).
+    unsigned long long ctr = 0;
+    if (tid == 0) ctr = atomicAdd(reinterpret_cast<unsigned long long *>(ctl + kCtlCalls), 1ull);
     // x -> x~ fragments, four groups (a quad) per warp and round: all of this warp's x
     // first.  Every CTA reads all of x at the same moment, so each starts at a different
     // quad: the simultaneous requests spread over the lines of x instead of piling up.
@@ -377,7 +399,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
         }
         for (int q = kFirstIssue; q < kStages; q++) issue(q);
     }
+    if (tid == 0) {
+        const uint32_t calls = (uint32_t)(ctr >> 32);
+        *epoch_s = calls + 1u;  // the count skips 0xffffffff, so the epoch is never 0
+        if ((uint32_t)ctr == (uint32_t)C - 1u) {  // the last CTA: every CTA has its epoch
+            const unsigned long long step = calls + 1u == 0xffffffffu ? 2ull : 1ull;
+            atomicAdd(reinterpret_cast<unsigned long long *>(ctl + kCtlCalls), (step << 32) - (unsigned long long)C);
+        }
+    }
     __syncthreads();
+    const uint32_t epoch = *epoch_s;
 
     // Lane (gid, tig) works on scale group tig of the item: MMA rows gid and gid + 8 of
     // each 16-row tile t are shared-memory rows r = 16t + gid (+ 8), whose group tig is
@@ -411,14 +442,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
         float sum = 0.f;
         for (int i = a; i < b; i++) sum += slots[(i - c0) * kItemRows + lane];
         if (a > tile_first) {
-            st_pair(partials + (int64_t)a * kItemRows + lane, sum);
+            st_pair(partials + (int64_t)a * kItemRows + lane, sum, epoch);
             return;
         }
         int s = b, c2 = (int)blockIdx.x + 1;
         while (s < tile_end) {
             int e2 = (int)((int64_t)I * (c2 + 1) / C);  // the piece of CTA c2 is [s, e2)
             e2 = e2 < tile_end ? e2 : tile_end;
-            sum += wait_pairs(partials + (int64_t)s * kItemRows, lane);
+            sum += wait_pairs(partials + (int64_t)s * kItemRows, lane, epoch + epoch_skew, wait_limit, status);
             s = e2;
             c2++;
         }
@@ -436,7 +467,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
         const int i = c0 + warp + q * kConsumers;
         if (ok) {
             ok = __all_sync(0xffffffffu, mbar_wait(full + st, phase));
-            if (ok) n_waited++;
+            if (ok)
+                n_waited++;
+            else if (lane == 0)
+                atomicOr(status, kDevStatusGemvCopyTimeout);
         }
         const uint8_t *sb = wring + st * kItemBytes;
         uint4 raw[2][2][2];  // [t][h][16-byte half of the lane's 32 bytes]
@@ -596,7 +630,7 @@ Shape shape_of(int64_t N, int64_t K, int sm_count) {
 }  // namespace
 
 static_assert(kConsumers * kStages * (kItemBytes + kScaleRingBytes) + (kMaxK / kItemK) * 4 * (kXGroupBytes + 12) +
-                  kMaxCtaItems * kItemRows * 4 + kMaxCtaTiles * 4 + 15 + 256 + kConsumers * kStages * 8 + 1024 <=
+                  kMaxCtaItems * kItemRows * 4 + kMaxCtaTiles * 4 + 15 + 256 + kConsumers * kStages * 8 + 16 + 1024 <=
                   232448,
               "shared-memory layout exceeds the per-CTA limit at the largest K");
 
@@ -614,13 +648,13 @@ bool gemv_imma_grid_fits(int64_t N, int64_t K, const DeviceInfo &dev) {
     return shape_of(N, K, dev.sm_count).grid <= dev.sm_count;
 }
 
-// the zero-initialised workspace region: (value, epoch) pairs of the pieces of row tiles
-// split between CTAs, indexed by the piece's first item: items x 32 x 8 bytes.  Every
-// pair a call stores is cleared again by its reader.
+// the zero-initialised workspace region: the control words, then the (value, epoch) pairs
+// of the pieces of row tiles split between CTAs, indexed by the piece's first item:
+// items x 32 x 8 bytes.
 size_t gemv_imma_zeroed_bytes(int64_t N, int64_t K) {
     const int64_t KC = (K + kItemK - 1) / kItemK;
     const int64_t items = ((N + kItemRows - 1) / kItemRows) * KC;
-    return (size_t)items * kItemRows * sizeof(uint64_t);
+    return kCtlRegionBytes + (size_t)items * kItemRows * sizeof(uint64_t);
 }
 
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
@@ -649,7 +683,8 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
     }
     const Shape sh = shape_of(N, K, dev.sm_count);
     if (ws.zeroed_bytes < gemv_imma_zeroed_bytes(N, K)) return cudaErrorInvalidValue;
-    uint64_t *partials = reinterpret_cast<uint64_t *>(ws.zeroed);
+    unsigned int *ctl = reinterpret_cast<unsigned int *>(ws.zeroed);
+    uint64_t *partials = reinterpret_cast<uint64_t *>(ws.zeroed + kCtlRegionBytes);
     // K a multiple of 512: an item's scales of a row are 8 (g64: 16) aligned bytes, copied
     // with the item
     using Kern = decltype(&gemv_imma_kernel<true, true, true>);
@@ -676,7 +711,10 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, wmap, x, scales, y, partials, (int)N, (int)K, (int)swiglu_f);
+    const uint32_t limit = dev.force_wait_timeouts ? kForcedWaitPolls : kSpinLimit;
+    const uint32_t skew = dev.force_wait_timeouts ? 0x80000000u : 0u;
+    return cudaLaunchKernelEx(&cfg, kern, wmap, x, scales, y, partials, ctl, (int)N, (int)K, (int)swiglu_f, limit,
+                              skew);
 }
 
 }  // namespace bonsai

@@ -14,7 +14,11 @@ struct DeviceInfo {
     int smem_optin = 0;  // max dynamic shared memory per block (opt-in), bytes
     int l2_bytes = 0;
     int smem_reserved = 0;  // shared memory the system reserves per block, bytes
+    // test hook (bonsai_debug_force_timeouts): cross-CTA waits look for a value nobody
+    // writes and give up after kForcedWaitPolls polls
+    bool force_wait_timeouts = false;
 };
+constexpr uint32_t kForcedWaitPolls = 64;
 
 // Split-K bookkeeping lives at the start of the workspace: kMaxTiles arrival
 // counters, zero when the workspace is created and returned to zero by the
@@ -77,13 +81,25 @@ cudaError_t launch_gemv_split_scratch(const uint16_t *x, const uint8_t *packed, 
 // current device's properties (the same probe the other entry points use)
 int current_device_info(DeviceInfo *out);
 
+// The zero-initialised workspace region starts with control words that kernels keep across
+// calls, as 32-bit words: [kCtlCalls, +1] a 64-bit call counter (low half: CTAs of the
+// running call that have read it; high half: calls counted so far, the epoch of the
+// cross-CTA hand-over data being one more), [kCtlStatus] sticky device status bits.
+constexpr int kCtlCalls = 0, kCtlStatus = 2;
+constexpr size_t kCtlRegionBytes = 256;
+// device status bits (kCtlStatus); the same values are public in bonsai.h
+constexpr unsigned int kDevStatusGemvCopyTimeout = 1u;   // integer GEMV: a weight copy never landed
+constexpr unsigned int kDevStatusGemvPieceTimeout = 2u;  // integer GEMV: a split tile's later piece never came
+constexpr unsigned int kDevStatusGemmTimeout = 4u;       // prefill GEMM: a barrier or hand-over wait gave up
+
 // ---- gemv_imma.cu: M == 1, PQ2_0, integer tensor cores
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t gemv_imma_zeroed_bytes(int64_t N, int64_t K);  // of Workspace::zeroed
 bool gemv_imma_grid_fits(int64_t N, int64_t K, const DeviceInfo &dev);
+// swiglu_f > 0: fused gate/up rows, write silu(gate) * up.
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
                              int64_t N, int64_t K, int fmt, const Workspace &ws, cudaStream_t s,
-                             const DeviceInfo &dev, int64_t swiglu_f = 0);  // > 0: fused gate/up rows, write silu(gate) * up
+                             const DeviceInfo &dev, int64_t swiglu_f = 0);
 
 // ---- skinny_mma.cu: 1 <= M <= 16
 bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt);

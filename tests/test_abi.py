@@ -70,6 +70,8 @@ def test_host_validation_needs_no_gpu(bz):
     # algorithm choice that cannot take the shape
     assert (L.bonsai_ternary_linear_algo(good, good, good, good, 1, 8, 128, 2, 99, 0, None)
             == bz.BONSAI_ERR_ALGO)
+    # the status query needs somewhere to write
+    assert L.bonsai_device_status(None, None, 0) == bz.BONSAI_ERR_NULL
     # empty problems are accepted and launch nothing
     assert L.bonsai_ternary_linear(None, None, None, None, 0, 8, 128, 2, None) == bz.BONSAI_OK
     assert L.bonsai_pack_pq2(None, None, 0, 128, None) == bz.BONSAI_OK

@@ -1,0 +1,85 @@
+"""The bounded waits' failure path, without any GPU fault: the library's test hook makes
+the integer GEMV's waits for the later pieces of its split row tiles look for a call
+number that nobody writes, so they give up after a few polls.  The call must then write
+NaN for exactly the row tiles split between CTAs, set the device status bit, and leave
+nothing behind that a following call could mistake for its own data."""
+import numpy as np
+import pytest
+
+import oracle
+from tests.gpu_util import Problem, to_numpy_f16
+
+pytestmark = pytest.mark.gpu
+
+PQ2 = oracle.FMT_PQ2_0
+
+
+@pytest.fixture(scope="module")
+def bz():
+    import torch
+    from ternary_weight_02_b200 import bonsai
+    assert bonsai.bonsai_check_device() == bonsai.BONSAI_OK
+    torch.cuda.init()
+    return bonsai
+
+
+def imma_split_tiles(N, K, sms):
+    """Row tiles (32 rows) of the integer GEMV whose 512-weight items fall to two or more
+    CTAs, from its work split: items (row tile, K chunk), CTA b taking items
+    [I b / C, I (b + 1) / C), C = max(ceil(I / 96), min(ceil(I / 16), SMs))."""
+    KC, RT = (K + 511) // 512, (N + 31) // 32
+    I = RT * KC
+    C = max(-(-I // 96), min(-(-I // 16), sms))
+    bounds = {I * b // C for b in range(1, C)}
+    return sorted({c // KC for c in bounds if c % KC != 0})
+
+
+def _run(bz, x, packed, scales, N, K):
+    import torch
+    y = torch.full((1, N), 7.0, dtype=torch.float16, device="cuda")
+    bz.bonsai_ternary_linear_algo(x, packed, scales, y, 1, N, K, PQ2, bz.BONSAI_ALGO_IMMA)
+    torch.cuda.synchronize()
+    return to_numpy_f16(y)[0]
+
+
+@pytest.mark.parametrize("N,K", [(7168, 5120), (5120, 17408)])
+def test_forced_piece_timeouts_nan_status_and_recovery(bz, N, K):
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    p = Problem(1, N, K, PQ2, seed=N + K)
+    x, packed, scales = p.device()
+    ref = p.oracle_y()[0]
+    split = imma_split_tiles(N, K, sms)
+    assert len(split) > 0
+    bz.bonsai_device_status(clear=True)
+    bz.bonsai_debug_force_timeouts(True)
+    try:
+        got = _run(bz, x, packed, scales, N, K)
+    finally:
+        bz.bonsai_debug_force_timeouts(False)
+    status = bz.bonsai_device_status(clear=True)
+    assert status & bz.BONSAI_DEVICE_GEMV_PIECE_TIMEOUT
+    assert not status & bz.BONSAI_DEVICE_GEMV_COPY_TIMEOUT
+    bad = np.zeros(N, dtype=bool)
+    for t in split:
+        bad[32 * t:min(32 * t + 32, N)] = True
+    assert np.all(np.isnan(got[bad]))
+    assert np.all(np.isfinite(got[~bad]))
+    ok, rel, mx = oracle.compare(got[~bad], ref[~bad])
+    assert ok, (rel, mx)
+    # the pieces that arrived after their reader gave up carry that call's number: the
+    # next call (hook off) takes none of them
+    for _ in range(2):
+        again = _run(bz, x, packed, scales, N, K)
+        ok, rel, mx = oracle.compare(again, ref)
+        assert ok, (rel, mx)
+    assert bz.bonsai_device_status() == 0
+
+
+def test_status_is_clear_after_normal_calls(bz):
+    p = Problem(1, 3000, 5120, PQ2, seed=3)
+    x, packed, scales = p.device()
+    bz.bonsai_device_status(clear=True)
+    got = _run(bz, x, packed, scales, 3000, 5120)
+    assert oracle.compare(got, p.oracle_y()[0])[0]
+    assert bz.bonsai_device_status() == 0
