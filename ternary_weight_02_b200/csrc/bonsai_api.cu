@@ -416,6 +416,11 @@ int bonsai_launch_count(int64_t M, int64_t N, int64_t K, int fmt, int algo, int 
     switch (chosen) {
         case BONSAI_ALGO_GEMV: return gemv_launches(N, K, fmt, split_k, st->info);
         case BONSAI_ALGO_IMMA: return 1;  // the rotation and quantisation of x are fused
+        case BONSAI_ALGO_GEMM: return 1;  // the rotation is the kernel's first phase
+        case BONSAI_ALGO_SKINNY: {  // fused when its grid is resident at once
+            const int n = skinny_launches(M, N, K, fmt, split_k, st->info);
+            return n < 0 ? BONSAI_ERR_CUDA : n;
+        }
         default: return 2;  // the rotation pass, then the kernel
     }
 }

@@ -99,6 +99,59 @@ __device__ __forceinline__ void store_half4(uint16_t *p, const float v[4]) {
     *reinterpret_cast<uint2 *>(p) = raw;
 }
 
+// One 128-block of x rotated by a warp into FP16 (nearest even), lane l storing outputs
+// 4l .. 4l+3 of the block.  kPerm: 0 natural order; 8: each 8 consecutive outputs in the
+// order [0, 4, 1, 5, 2, 6, 3, 7]; 16: each 16 in the order [0, 8, 1, 9, ..., 7, 15].  The
+// prefill GEMM expands its PQ2_0 (8) or Q1_0 (16) weights in the same order within each
+// block (a contraction does not depend on the order of its terms), which lets it build
+// two FP16 weights with one byte permute.
+// rotate_store_f16 takes the lane's four inputs already loaded (as load_half4 gives them).
+template <int kPerm>
+__device__ __forceinline__ void rotate_store_f16(float (&v)[4], uint16_t *__restrict__ out, int64_t blk, int lane) {
+    fwht128_warp(v, lane);
+    float o[4];
+    if (kPerm == 16) {
+        // lanes 4b .. 4b+3 hold outputs 16b .. 16b+15; lane r of the four stores
+        // (e, e + 8, e + 1, e + 9) with e = 4 (r >> 1) + 2 (r & 1): elements e, e + 1
+        // of lane r >> 1 and of lane 2 + (r >> 1)
+        const int base = lane & ~3, r = lane & 3;
+        const int la = base + (r >> 1), lb = base + 2 + (r >> 1);
+        float a[4], b[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            a[k] = __shfl_sync(0xffffffffu, v[k], la);
+            b[k] = __shfl_sync(0xffffffffu, v[k], lb);
+        }
+        const bool odd = r & 1;
+        o[0] = odd ? a[2] : a[0];
+        o[1] = odd ? b[2] : b[0];
+        o[2] = odd ? a[3] : a[1];
+        o[3] = odd ? b[3] : b[1];
+    } else if (kPerm == 8) {
+        // lanes 2b, 2b + 1 hold outputs 8b .. 8b + 7; the even lane stores
+        // (0, 4, 1, 5), the odd one (2, 6, 3, 7)
+        const bool odd = lane & 1;
+        const float r0 = __shfl_xor_sync(0xffffffffu, odd ? v[0] : v[2], 1);
+        const float r1 = __shfl_xor_sync(0xffffffffu, odd ? v[1] : v[3], 1);
+        if (odd) {
+            o[0] = r0, o[1] = v[2], o[2] = r1, o[3] = v[3];
+        } else {
+            o[0] = v[0], o[1] = r0, o[2] = v[1], o[3] = r1;
+        }
+    } else {
+        o[0] = v[0], o[1] = v[1], o[2] = v[2], o[3] = v[3];
+    }
+    store_half4(out + blk * kGroup + 4 * lane, o);
+}
+
+template <int kPerm>
+__device__ __forceinline__ void rotate_block_f16(const uint16_t *__restrict__ x, uint16_t *__restrict__ out,
+                                                 int64_t blk, int lane) {
+    float v[4];
+    load_half4(x + blk * kGroup + 4 * lane, v);
+    rotate_store_f16<kPerm>(v, out, blk, lane);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -7,12 +7,16 @@
 // Hadamard), packings paragraph (PQ2_0 wins prompt processing); "Bonsai 2，把27B压进6个G"
 // (10100.com), section 它怎么做到的 (the input takes the matching transform).
 //
-// Two launches per call:
-//  1. the block-Hadamard rotation x -> x' (FP16, round to nearest) into the workspace
-//     (hadamard.cu), each 8 columns in the K order of the expanded weights.  Rotating inside the GEMM would redo each 128 x 128 A tile's FWHT
-//     for every one of the N/256 column tiles; as a pass it costs one read and one
-//     write of x, under 1% of the GEMM's time at these shapes.
-//  2. this kernel, persistent: at most one CTA per SM, each taking whole tiles in waves
+// One launch per call, persistent (at most one CTA per SM, all resident at once):
+//  1. every CTA rotates its share of the 128-blocks of x into x' (FP16, round to
+//     nearest) in the workspace, each 8 columns (Q1_0: 16) in the K order of the expanded
+//     weights.  Rotating per tile would redo each 128 x 128 x' tile's FWHT for every one
+//     of the N/256 column tiles; done once, it costs one read and one write of x.  The
+//     CTAs then meet at a grid-wide barrier: each counts itself in the workspace's call
+//     counter with one atomic add, the last one advances the counter, and only the
+//     thread that issues the TMA loads of x' waits for that (bounded), while the rest of
+//     the CTA sets up its barriers and tensor memory.
+//  2. the tiles: each CTA takes whole tiles in waves
 //     and then an even share of the last tiles' 64-wide K stages (stream-K, below), so
 //     that no SM idles in a partial last wave.  A tile is kAcc x 128 rows x 256
 //     columns of y; per stage (3- or 4-deep rings):
@@ -28,7 +32,7 @@
 //       FP32 hand-over of a split tile.
 // Every wait is bounded: if one gives up, the CTA stops issuing work, waits for the
 // copies and MMAs it started, frees its tensor memory and writes NaN to its tiles (and
-// hands NaN over for a split one).
+// hands NaN over for a split one), and sets its bit in the device status word.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -58,7 +62,7 @@ struct Cfg {
     static constexpr int kOffB = kStages * kAStage;
     static constexpr int kOffCodes = kOffB + kStages * B_STAGE_BYTES;
     static constexpr int kOffBar = kOffCodes + kStages * CODE_STAGE_BYTES;
-    static constexpr int kNumBars = 3 * kStages + 3;  // full_a, full_b, empty, done, tmem_free, fin
+    static constexpr int kNumBars = 3 * kStages + 6;  // full_a, full_b, empty, done, tmem_free, fin, 3 rotation
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 8;
     static constexpr int kOffLut = kOffAbort + 8;
@@ -241,9 +245,10 @@ __device__ __forceinline__ void group_codes(const GroupRaw &raw, const uint32_t 
 // ---------------------------------------------------------------- cross-CTA hand-over
 
 // A tile piece's FP32 partial sums go to the CTA's own slot in the workspace; a flag
-// word per CTA (zero at rest) says that the slot is complete.  The writer's threads
-// fence, meet at a named barrier, and one of them releases the flag; the owner acquires
-// it (every lane polls, bounded), reads the slot through L2 and later clears the flag.
+// word per CTA says that the slot is complete by holding this call's epoch (the call
+// counter's value plus one), so flags never need clearing.  The writer's threads fence,
+// meet at a named barrier, and one of them releases the flag; the owner acquires it
+// (every lane polls, bounded) and reads the slot through L2.
 __device__ __forceinline__ void flag_release(unsigned int *p, unsigned int v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -252,13 +257,18 @@ __device__ __forceinline__ unsigned int flag_acquire(const unsigned int *p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-// Bounded wait of a whole warp for *p == 1.
-__device__ __forceinline__ bool flag_wait(const unsigned int *p) {
-    for (uint32_t i = 0; i < kSpinLimit; i++) {
-        if (__all_sync(0xffffffffu, flag_acquire(p) == 1u)) return true;
+// Bounded wait of a whole warp for *p == want.
+__device__ __forceinline__ bool flag_wait(const unsigned int *p, unsigned int want, uint32_t limit) {
+    for (uint32_t i = 0; i < limit; i++) {
+        if (__all_sync(0xffffffffu, flag_acquire(p) == want)) return true;
         __nanosleep(64);
     }
     return false;
+}
+__device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int *p) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 // The eight expansion/epilogue warps (256 threads) meet here; barrier 0 is __syncthreads.
 __device__ __forceinline__ void expand_warps_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
@@ -283,6 +293,12 @@ __device__ __forceinline__ void expand_warps_sync() { asm volatile("bar.sync 1, 
 // piece last: the waits are short, and they only go from a CTA to later ones, which never
 // wait before they have stored (all CTAs of the grid are resident at once, one per SM).
 //
+// x: the un-rotated input (M x K); xr: the workspace's x' (nblocks 128-blocks).  ctl: the
+// workspace's control words (call counter, status word, hand-over flags from kCtlGemmFlags
+// on).  wait_limit and epoch_skew: the polls of an owner's wait for a flag and an offset
+// added to the epoch it waits for (kSpinLimit and 0 except under the test hook that makes
+// those waits give up).
+//
 // kSwiglu: the weight rows are a fused gate/up projection (gate rows 0 .. F-1, up rows
 // F .. 2F-1, N = 2F) and the output is h = silu(gate) * up, M x F.  A tile's
 // 256 weight rows are then gate rows 128 tn .. 128 tn + 127 followed by the matching up
@@ -293,7 +309,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap w_map,
     const uint8_t *__restrict__ packed,
     const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
-    unsigned int *__restrict__ flags, int M, int N, int K, int mt, int F) {
+    const uint16_t *__restrict__ x, uint16_t *__restrict__ xr, int64_t nblocks, unsigned int *__restrict__ ctl,
+    uint32_t wait_limit, uint32_t epoch_skew, int M, int N, int K, int mt, int F) {
     using C = Cfg<kAcc>;
     constexpr int STAGES = C::kStages;
     constexpr int kSlotFloats = C::kTileM * BN;
@@ -307,6 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     uint64_t *full_a = bars, *full_b = bars + STAGES, *empty = bars + 2 * STAGES;
     uint64_t *done = bars + 3 * STAGES, *tmem_free = done + 1, *fin = done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmemSlot);
+    uint32_t *epoch_s = tmem_slot + 1;  // the second word of the slot's 8 bytes
+    unsigned int *flags = ctl + kCtlGemmFlags;
+    unsigned int *status = ctl + kCtlStatus;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffAbort);
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem + C::kOffLut);
 
@@ -348,6 +368,64 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
         return p;
     };
 
+    // ---- rotation of this CTA's share of x, then its arrival at the grid barrier.  The
+    // CTA's 128-blocks (a contiguous run of x) stream through the tile rings' shared memory,
+    // idle until the tiles start, in 64 KB bulk copies three deep; each warp rotates blocks
+    // from there and stores x'.
+    bool rot_fail = false;
+    {
+        constexpr int kWarps = kThreads / 32;
+        constexpr int kRotBufBytes = 64 * 1024, kRotBufs = 3, kRotBlocks = kRotBufBytes / (kGroup * 2);
+        static_assert(kRotBufs * kRotBufBytes <= C::kOffCodes, "rotation buffers lie inside the A and B rings");
+        uint64_t *rot_bar = bars + 3 * STAGES + 3;
+        const int64_t rb0 = nblocks * cta / nctas, rb1 = nblocks * (cta + 1) / nctas;
+        const int nchunks = (int)((rb1 - rb0 + kRotBlocks - 1) / kRotBlocks);
+        auto issue_chunk = [&](int c) {  // one thread
+            const int64_t b = rb0 + (int64_t)c * kRotBlocks;
+            const int64_t e = b + kRotBlocks < rb1 ? b + kRotBlocks : rb1;
+            const uint32_t bytes = (uint32_t)((e - b) * kGroup * 2);
+            mbar_arrive_expect_tx(rot_bar + c % kRotBufs, bytes);
+            bulk_load(smem + (c % kRotBufs) * kRotBufBytes, x + b * kGroup, bytes, rot_bar + c % kRotBufs);
+        };
+        if (tid == 0) {
+            for (int i = 0; i < kRotBufs; i++) mbar_init(rot_bar + i, 1);
+            mbar_init_fence();
+            for (int c = 0; c < kRotBufs && c < nchunks; c++) issue_chunk(c);
+        }
+        __syncthreads();
+        int c = 0;
+        for (; c < nchunks; c++) {
+            const bool got = mbar_wait(rot_bar + c % kRotBufs, (uint32_t)(c / kRotBufs) & 1u);
+            if (__syncthreads_or(!got)) {
+                rot_fail = true;
+                break;
+            }
+            const int64_t b = rb0 + (int64_t)c * kRotBlocks;
+            const int64_t e = b + kRotBlocks < rb1 ? b + kRotBlocks : rb1;
+            const uint8_t *buf = smem + (c % kRotBufs) * kRotBufBytes;
+            for (int64_t blk = b + warp; blk < e; blk += kWarps) {
+                const uint2 raw = *reinterpret_cast<const uint2 *>(buf + (blk - b) * (kGroup * 2) + lane * 8);
+                const float2 f01 = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
+                const float2 f23 = __half22float2(*reinterpret_cast<const __half2 *>(&raw.y));
+                float v[4] = {f01.x, f01.y, f23.x, f23.y};
+                rotate_store_f16<kFmt == 3 ? 16 : 8>(v, xr, blk, lane);
+            }
+            // these reads of the buffer before the copy that refills it
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncthreads();
+            if (tid == 0 && c + kRotBufs < nchunks) issue_chunk(c + kRotBufs);
+        }
+        if (rot_fail && tid == 0)  // let the copies in flight land before the rings are reused
+            for (int c2 = c; c2 < nchunks && c2 < c + kRotBufs; c2++)
+                mbar_wait(rot_bar + c2 % kRotBufs, (uint32_t)(c2 / kRotBufs) & 1u);
+        // these generic-proxy stores before the async-proxy (TMA) loads of any CTA
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+    }
+    __syncthreads();
+    unsigned long long arrival = 0;
+    if (tid == 0) arrival = atomicAdd(reinterpret_cast<unsigned long long *>(ctl + kCtlCalls), 1ull);
+
     if (tid == 0) {
         for (int st = 0; st < STAGES; st++) {
             mbar_init(full_a + st, 1);
@@ -357,8 +435,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
         mbar_init(done, 1);
         mbar_init(tmem_free, kExpandWarps);
         mbar_init(fin, 1);
-        *abort_flag = 0;
+        *abort_flag = rot_fail ? 1 : 0;
         mbar_init_fence();
+        // this call's epoch; the last CTA to arrive advances the counter (skipping
+        // 0xffffffff, so that the epoch is never 0), which releases the barrier
+        const uint32_t calls = (uint32_t)(arrival >> 32);
+        *epoch_s = calls + 1u;
+        if ((uint32_t)arrival == (uint32_t)nctas - 1u) {
+            const unsigned long long step = calls + 1u == 0xffffffffu ? 2ull : 1ull;
+            atomicAdd(reinterpret_cast<unsigned long long *>(ctl + kCtlCalls),
+                      (step << 32) - (unsigned long long)nctas);
+        }
     }
     if (kFmt == 1) {  // byte -> its five base-3 digits as 2-bit codes (code i at bits 2i)
         for (int b = tid; b < 256; b += kThreads) {
@@ -381,10 +468,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const uint32_t epoch = *epoch_s;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (x' tiles)
         if (lane == 0) {
+            // every CTA's x' is written: the call counter has moved past this call's arrivals
+            {
+                uint32_t i = 0;
+                for (; i < kSpinLimit; i++) {
+                    if (ld_acquire_u32(ctl + kCtlCalls + 1) != epoch - 1u) break;
+                    __nanosleep(32);
+                }
+                if (i == kSpinLimit) *abort_flag = 1;
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+            }
             int it = 0;  // units issued: ring position
             for (int v = 0; v < n_mine && !*abort_flag;) {
                 const Piece p = piece_at(v);
@@ -568,7 +666,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
             bool got = true;  // the later pieces all arrived (owner)
             if (owner)
                 for (int c2 = cta + 1, s = u_end; s < tile_end; s = range_end(c2), c2++)
-                    got = flag_wait(flags + c2) && got;
+                    got = flag_wait(flags + c2, epoch + epoch_skew, wait_limit) && got;
+            if (!got && r == 0) atomicOr(status, kDevStatusGemmTimeout);
             const int w8 = warp - 2;
             if constexpr (kSwiglu) {
                 // h columns [64 half, +64) of the tile's 128: gate accumulator columns
@@ -761,11 +860,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
             if (continues) {
                 __threadfence();
                 expand_warps_sync();
-                if (r == 0) flag_release(flags + cta, 1u);
+                if (r == 0) flag_release(flags + cta, epoch);
             } else if (owner) {
                 expand_warps_sync();  // every warp has read the later pieces and its staging rows
-                if (r == 0)
-                    for (int c2 = cta + 1, s = u_end; s < tile_end; s = range_end(c2), c2++) flags[c2] = 0u;
             } else {
                 // the next piece's expansion writes the B ring, where other warps may still
                 // be reading their staging rows
@@ -776,6 +873,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
 
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && *abort_flag) atomicOr(status, kDevStatusGemmTimeout);
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
@@ -835,13 +933,15 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
     const bool swiglu = swiglu_f > 0;
     if (swiglu && N != 2 * swiglu_f) return cudaErrorInvalidValue;
     const GemmPlan plan = gemm_plan(M, N, K, tile_hint, dev.sm_count);
-    if (ws.data_bytes < gemm_workspace_bytes(M, N, K, fmt, dev) || plan.ctas > kMaxTiles) return cudaErrorInvalidValue;
+    if (ws.data_bytes < gemm_workspace_bytes(M, N, K, fmt, dev) || plan.ctas > kCtlGemmMaxCtas ||
+        ws.zeroed_bytes < kCtlRegionBytes)
+        return cudaErrorInvalidValue;
     uint16_t *xr = reinterpret_cast<uint16_t *>(ws.data);
     float *partials = reinterpret_cast<float *>(ws.data + x_rot_bytes(M, K));
-    // x' in the expansion's K order
-    cudaError_t err = fmt == 3 ? launch_hadamard_f16_perm16(x, xr, M, K, s, dev)
-                               : launch_hadamard_f16_perm8(x, xr, M, K, s, dev);
-    if (err != cudaSuccess) return err;
+    unsigned int *ctl = reinterpret_cast<unsigned int *>(ws.zeroed);
+    const int64_t nblocks = M * (K / kGroup);
+    const uint32_t limit = dev.force_wait_timeouts ? kForcedWaitPolls : kSpinLimit;
+    const uint32_t skew = dev.force_wait_timeouts ? 0x80000000u : 0u;
 
     EncodeTiledFn encode = encode_fn();
     if (!encode) return cudaErrorNotSupported;
@@ -869,8 +969,8 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
     auto go = [&](auto kern, int smem) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        kern<<<plan.ctas, kThreads, smem, s>>>(map, wmap, packed, scales, y, partials, ws.counters, (int)M, (int)N,
-                                               (int)K, plan.mt, (int)swiglu_f);
+        kern<<<plan.ctas, kThreads, smem, s>>>(map, wmap, packed, scales, y, partials, x, xr, nblocks, ctl, limit,
+                                               skew, (int)M, (int)N, (int)K, plan.mt, (int)swiglu_f);
         return cudaGetLastError();
     };
     auto pick = [&](auto k1, auto k2) { return plan.acc == 2 ? go(k2, Cfg<2>::kSmemBytes) : go(k1, Cfg<1>::kSmemBytes); };

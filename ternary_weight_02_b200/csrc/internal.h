@@ -51,13 +51,6 @@ cudaError_t launch_hadamard_f16(const uint16_t *x, uint16_t *out, int64_t M, int
                                 cudaStream_t s, const DeviceInfo &dev);
 cudaError_t launch_hadamard_f32(const uint16_t *x, float *out, int64_t M, int64_t K,
                                 cudaStream_t s, const DeviceInfo &dev);
-// As launch_hadamard_f16, each 8 outputs stored in the order [0, 4, 1, 5, 2, 6, 3, 7]
-// (the K order of the prefill GEMM's expanded weight tiles).
-cudaError_t launch_hadamard_f16_perm8(const uint16_t *x, uint16_t *out, int64_t M, int64_t K,
-                                      cudaStream_t s, const DeviceInfo &dev);
-// The same, each 16 outputs in the order [0, 8, 1, 9, ..., 7, 15] (Q1_0 tiles).
-cudaError_t launch_hadamard_f16_perm16(const uint16_t *x, uint16_t *out, int64_t M, int64_t K,
-                                       cudaStream_t s, const DeviceInfo &dev);
 
 // ---- linear_simple.cu: x' (FP32, M x K) in the workspace, then one warp per row
 size_t simple_workspace_bytes(int64_t M, int64_t N, int64_t K);
@@ -85,12 +78,15 @@ int current_device_info(DeviceInfo *out);
 // calls, as 32-bit words: [kCtlCalls, +1] a 64-bit call counter (low half: CTAs of the
 // running call that have read it; high half: calls counted so far, the epoch of the
 // cross-CTA hand-over data being one more), [kCtlStatus] sticky device status bits.
-constexpr int kCtlCalls = 0, kCtlStatus = 2;
-constexpr size_t kCtlRegionBytes = 256;
+// [kCtlGemmFlags, + kCtlGemmMaxCtas): the prefill GEMM's hand-over flags, one per CTA.
+constexpr int kCtlCalls = 0, kCtlStatus = 2, kCtlGemmFlags = 64;
+constexpr int kCtlGemmMaxCtas = 960;
+constexpr size_t kCtlRegionBytes = 4096;
 // device status bits (kCtlStatus); the same values are public in bonsai.h
 constexpr unsigned int kDevStatusGemvCopyTimeout = 1u;   // integer GEMV: a weight copy never landed
 constexpr unsigned int kDevStatusGemvPieceTimeout = 2u;  // integer GEMV: a split tile's later piece never came
 constexpr unsigned int kDevStatusGemmTimeout = 4u;       // prefill GEMM: a barrier or hand-over wait gave up
+constexpr unsigned int kDevStatusSkinnyTimeout = 8u;     // skinny kernel: the wait for the rotated x gave up
 
 // ---- gemv_imma.cu: M == 1, PQ2_0, integer tensor cores
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt);
@@ -101,10 +97,12 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
                              int64_t N, int64_t K, int fmt, const Workspace &ws, cudaStream_t s,
                              const DeviceInfo &dev, int64_t swiglu_f = 0);
 
-// ---- skinny_mma.cu: 1 <= M <= 16
+// ---- skinny_mma.cu: 1 <= M <= 16 (one launch when its grid is resident at once: the
+// rotation, a barrier on the call counter in Workspace::zeroed, the kernel; else two)
 bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t skinny_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int split_k,
                               const DeviceInfo &dev);
+int skinny_launches(int64_t M, int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev);
 cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                           uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int split_k,
                           const Workspace &ws, cudaStream_t s, const DeviceInfo &dev);
@@ -116,8 +114,9 @@ cudaError_t launch_swiglu(const uint16_t *y, uint16_t *h, int64_t M, int64_t F, 
 // ---- gemm_tcgen05.cu: prefill
 bool gemm_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, const DeviceInfo &dev);
-// tile_hint: 0 automatic, 1 one 128-row accumulator per CTA, 2 two (256 rows).  Uses
-// Workspace::counters[0, SMs) as hand-over flags (zero at rest).
+// tile_hint: 0 automatic, 1 one 128-row accumulator per CTA, 2 two (256 rows).  One launch:
+// the rotation of x into the workspace, a grid barrier, the tiles; hand-over flags and the
+// barrier live in the control words of Workspace::zeroed.
 // swiglu_f > 0: the N = 2 swiglu_f rows are gate then up rows and y
 // gets silu(gate) * up, M x swiglu_f.
 cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,

@@ -38,8 +38,15 @@
 //   16-byte group; MMA i uses nibble i & 1 of byte i >> 1, bits left in place as FP16
 //   subnormals b * 2^j * 2^-24 (j = 0..7 within the byte) against x' pre-scaled by 2^-j,
 //   and the epilogue adds s * (2 * 2^24 * D - sum x'), which turns bits b into 2b - 1.
+// * PTQ1_0 (5 trits per base-3 byte, 26 bytes per 128-weight group; the allhereai.com
+//   page's packings paragraph).  A byte's base-3 digits are the trits plus one, i.e.
+//   PQ2_0's codes, so a 256-entry shared-memory table turns each byte into its five 2-bit
+//   codes and the lane assembles the same two code words (weights 32tq .. 32tq + 31) the
+//   PQ2_0 path loads; everything after that is PQ2_0's.  The lane's 7 or 8 bytes of a row's
+//   group (from byte 32tq / 5) come as three aligned 32-bit loads.
 #include "common.cuh"
 #include "internal.h"
+#include "tma.cuh"  // kSpinLimit: the bound of every wait
 
 namespace bonsai {
 namespace {
@@ -59,7 +66,35 @@ constexpr int sub_groups() { return NT == 1 ? 48 : 24; }
 struct Grp {
     uint2 a, b;
     uint32_t s0, s1;
+    uint32_t a2, b2;  // PTQ1_0: the third raw word of each row (a, b hold the first two)
 };
+
+// PTQ1_0: the first of the group's bytes that hold lane quad member tq's weights 32tq ..
+// 32tq + 31, and the digit of that byte where weight 32tq sits.
+__device__ __forceinline__ int ptq1_first_byte(int tq) { return (32 * tq) / 5; }
+__device__ __forceinline__ int ptq1_first_digit(int tq) { return (32 * tq) % 5; }
+
+// PTQ1_0 -> the lane's two PQ2_0 code words: w0..w2 are the aligned 32-bit words that hold
+// its bytes from byte offset `shift` on; lut[b] holds the five 2-bit codes (digits) of byte b.
+__device__ __forceinline__ uint2 ptq1_codes(uint32_t w0, uint32_t w1, uint32_t w2, int shift, int tq,
+                                            const uint16_t *lut) {
+    const uint32_t lo = __funnelshift_r(w0, w1, 8 * shift), hi = __funnelshift_r(w1, w2, 8 * shift);
+    const uint64_t v0 = (uint64_t)lut[lo & 0xffu] | ((uint64_t)lut[(lo >> 8) & 0xffu] << 10) |
+                        ((uint64_t)lut[(lo >> 16) & 0xffu] << 20) | ((uint64_t)lut[lo >> 24] << 30) |
+                        ((uint64_t)lut[hi & 0xffu] << 40) | ((uint64_t)lut[(hi >> 8) & 0xffu] << 50);
+    const uint64_t v1 = (uint64_t)lut[(hi >> 16) & 0xffu] | ((uint64_t)lut[hi >> 24] << 10);
+    const int off = 2 * ptq1_first_digit(tq);  // bits of the digits before weight 32tq
+    const uint64_t r = (v0 >> off) | (v1 << (60 - off));
+    return make_uint2((uint32_t)r, (uint32_t)(r >> 32));
+}
+
+// 32-bit word at byte offset o (a multiple of 4) of a plane of `end` bytes (even): the bytes
+// past the end read as zero and are never accessed.
+__device__ __forceinline__ uint32_t ld_word_clamped(const uint8_t *p, int64_t o, int64_t end) {
+    if (o + 4 <= end) return __ldcs(reinterpret_cast<const unsigned int *>(p + o));
+    if (o + 2 <= end) return (uint32_t)__ldcs(reinterpret_cast<const unsigned short *>(p + o));
+    return 0u;
+}
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -89,13 +124,9 @@ __device__ __forceinline__ int64_t skinny_k(int64_t group, int step, int tq) {
 // tokens m >= M, and the FP32 sum of the block's FP16 x' values to gsum[g][m] (g64: the
 // sums of its two 64-element halves to gsum[g][h][m]).
 template <int MT, int kFmt>
-__global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ xs,
-                                                          float *__restrict__ gsum, int M, int64_t K) {
-    const int lane = threadIdx.x & 31;
-    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // (g, m) = (w / MT, w % MT)
-    const int64_t G = K / kGroup;
-    if (w >= G * MT) return;
-    const int64_t g = w / MT;
+__device__ __forceinline__ void prep_task(const uint16_t *__restrict__ x, uint16_t *__restrict__ xs,
+                                          float *__restrict__ gsum, int M, int64_t K, int64_t w, int lane) {
+    const int64_t g = w / MT;  // (g, m) = (w / MT, w % MT)
     const int m = (int)(w % MT);
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     if (m < M) {
@@ -137,20 +168,37 @@ __global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__rest
     }
 }
 
+template <int MT, int kFmt>
+__global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__restrict__ x, uint16_t *__restrict__ xs,
+                                                          float *__restrict__ gsum, int M, int64_t K) {
+    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (w >= (K / kGroup) * MT) return;
+    prep_task<MT, kFmt>(x, xs, gsum, M, K, w, threadIdx.x & 31);
+}
 
-// kFmt: 2 PQ2_0, 4 PQ2_0 g64 (64-weight scales), 3 Q1_0
+
+// kFmt: 2 PQ2_0, 4 PQ2_0 g64 (64-weight scales), 3 Q1_0, 1 PTQ1_0 (transcoded to PQ2_0 codes)
+//
+// x != nullptr: the rotation is the kernel's first phase.  Every CTA rotates its share of
+// the (group, token) blocks into the staged layout (as the rotation pass does), counts
+// itself in the workspace's call counter (ctl) and requests its first weights; before
+// staging x' it waits (bounded) until the last CTA has advanced the counter.  The grid
+// is then resident at once (the launcher checks the occupancy).  If that wait gives up,
+// the CTA writes NaN and sets the status bit.
 template <int NT, int kFmt>  // n8 token tiles: 1 (M <= 8) or 2 (M <= 16)
 __global__ void __launch_bounds__(kThreads) skinny_kernel(
-    const uint16_t *__restrict__ xsg, const float *__restrict__ gsg, const uint8_t *__restrict__ packed,
+    uint16_t *__restrict__ xsg, float *__restrict__ gsg, const uint8_t *__restrict__ packed,
     const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
-    unsigned int *__restrict__ counters, int M, int64_t N, int64_t K, int S, int gpc) {
+    unsigned int *__restrict__ counters, int M, int64_t N, int64_t K, int S, int gpc,
+    const uint16_t *__restrict__ x, unsigned int *__restrict__ ctl) {
     constexpr int MT = NT * 8;  // tokens padded
     static_assert(sub_groups<NT>() % kRing == 0, "ring slots follow the group index");
     // groups staged at a time: the whole chunk when it fits (shared memory is sized so)
     const int kSub = gpc < sub_groups<NT>() ? gpc : sub_groups<NT>();
     extern __shared__ __align__(16) uint8_t smem[];
-    constexpr bool kG64 = kFmt == 4, kQ1 = kFmt == 3;
+    constexpr bool kG64 = kFmt == 4, kQ1 = kFmt == 3, kP1 = kFmt == 1;
     constexpr int kHalves = kG64 ? 2 : 1;  // scale groups per 128 weights
+    __shared__ uint16_t lut3[kP1 ? 256 : 1];  // PTQ1_0: byte -> its five digits as 2-bit codes
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [kSub * 8 steps][MT][16]
     float *gsum = reinterpret_cast<float *>(smem + kSub * 8 * MT * 32);  // [MT][kSub][kHalves]
 
@@ -170,6 +218,39 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
 #pragma unroll
         for (int e = 0; e < 4; e++) acc[nt][e] = 0.f;
 
+    // ---- the rotation phase and this CTA's arrival (fused launch)
+    unsigned long long arrival = 0;
+    if (x != nullptr) {
+        const int64_t ncta = (int64_t)gridDim.x * gridDim.y;
+        const int64_t b = (int64_t)blockIdx.y * gridDim.x + blockIdx.x;
+        for (int64_t w = b * kWarps + warp; w < G * MT; w += ncta * kWarps)
+            prep_task<MT, kFmt>(x, xsg, gsg, M, K, w, lane);
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            arrival = atomicAdd(reinterpret_cast<unsigned long long *>(ctl + kCtlCalls), 1ull);
+            const uint32_t calls = (uint32_t)(arrival >> 32);
+            if ((uint32_t)arrival == (uint32_t)ncta - 1u) {  // the last CTA releases the others
+                const unsigned long long step = calls + 1u == 0xffffffffu ? 2ull : 1ull;
+                atomicAdd(reinterpret_cast<unsigned long long *>(ctl + kCtlCalls),
+                          (step << 32) - (unsigned long long)ncta);
+            }
+        }
+    }
+
+    const int64_t plane_end = N * G * kPtq1GroupBytes;  // PTQ1_0 plane size
+    // PTQ1_0: the three aligned words holding the lane's bytes of row r's group g
+    auto row_words3 = [&](int64_t r, int g, uint2 &w01, uint32_t &w2) {
+        const int64_t a = ((r * G + g) * kPtq1GroupBytes + ptq1_first_byte(tq)) & ~(int64_t)3;
+        if (a + 12 <= plane_end) {
+            const unsigned int *p = reinterpret_cast<const unsigned int *>(packed + a);
+            w01 = make_uint2(__ldcs(p), __ldcs(p + 1));
+            w2 = __ldcs(p + 2);
+        } else {  // the plane's last group
+            w01 = make_uint2(ld_word_clamped(packed, a, plane_end), ld_word_clamped(packed, a + 4, plane_end));
+            w2 = ld_word_clamped(packed, a + 8, plane_end);
+        }
+    };
     auto row_words = [&](int64_t r, int g) -> uint2 {
         if (kQ1)  // word tq of the row's 16-byte group
             return make_uint2(__ldcs(reinterpret_cast<const unsigned int *>(packed + (r * G + g) * kQ1GroupBytes) + tq),
@@ -186,18 +267,37 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
     };
     auto load = [&](int g, Grp &q) {
         if (v0) {
-            q.a = row_words(r0, g);
+            if (kP1)
+                row_words3(r0, g, q.a, q.a2);
+            else
+                q.a = row_words(r0, g);
             q.s0 = row_scales(r0, g);
         } else {
             q.a = make_uint2(0x55555555u, 0x55555555u), q.s0 = 0u;  // trits 0
+            q.a2 = 0u;
         }
         if (v1) {
-            q.b = row_words(r1, g);
+            if (kP1)
+                row_words3(r1, g, q.b, q.b2);
+            else
+                q.b = row_words(r1, g);
             q.s1 = row_scales(r1, g);
         } else {
             q.b = make_uint2(0x55555555u, 0x55555555u), q.s1 = 0u;
+            q.b2 = 0u;
         }
     };
+    if (kP1) {  // the byte -> codes table; the barrier before the first staging of x' publishes it
+        for (int b = tid; b < 256; b += kThreads) {
+            uint32_t f = 0;
+            int v = b < 243 ? b : 0;
+            for (int i = 0; i < 5; i++) {
+                f |= (uint32_t)(v % 3) << (2 * i);
+                v /= 3;
+            }
+            lut3[b] = (uint16_t)f;
+        }
+    }
 
     // group g of the chunk lives in ring slot (g - g_begin) % kRing; the first kRing are
     // requested before x' is staged
@@ -205,6 +305,25 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
 #pragma unroll
     for (int u = 0; u < kRing; u++)
         if (g_begin + u < g_end) load(g_begin + u, ring[u]);
+
+    bool barrier_ok = true;
+    if (x != nullptr) {  // every CTA's x' is staged once the counter has moved on
+        __shared__ int ok_s;
+        if (tid == 0) {
+            const uint32_t calls = (uint32_t)(arrival >> 32);
+            uint32_t i = 0;
+            for (; i < kSpinLimit; i++) {
+                uint32_t hi;
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(hi) : "l"(ctl + kCtlCalls + 1) : "memory");
+                if (hi != calls) break;
+                __nanosleep(32);
+            }
+            ok_s = i < kSpinLimit;
+            if (i == kSpinLimit) atomicOr(ctl + kCtlStatus, kDevStatusSkinnyTimeout);
+        }
+        __syncthreads();
+        barrier_ok = ok_s != 0;
+    }
 
     for (int sub = g_begin; sub < g_end; sub += kSub) {
         const int nsub = g_end - sub < kSub ? g_end - sub : kSub;
@@ -218,7 +337,8 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
             cp_async_commit();
             for (int idx = tid; idx < nsub * MT * kHalves; idx += kThreads) {
                 const int gh = idx / MT, m = idx % MT;  // gh = kHalves * gl + h
-                gsum[m * kSub * kHalves + gh] = gsg[((int64_t)sub * kHalves + gh) * MT + m];
+                // (through L2: in the fused launch other CTAs wrote these sums)
+                gsum[m * kSub * kHalves + gh] = __ldcg(gsg + ((int64_t)sub * kHalves + gh) * MT + m);
             }
             cp_async_wait_all();
         }
@@ -230,6 +350,13 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
                 const int gl = gl0 + u;
                 if (gl >= nsub) break;
                 Grp &cur = ring[u];
+                if (kP1) {  // base-3 bytes -> the PQ2_0 code words of weights 32tq .. 32tq + 31
+                    const int g = sub + gl;
+                    const int sh0 = (int)(((r0 * G + g) * kPtq1GroupBytes + ptq1_first_byte(tq)) & 3);
+                    const int sh1 = (int)(((r1 * G + g) * kPtq1GroupBytes + ptq1_first_byte(tq)) & 3);
+                    if (v0) cur.a = ptq1_codes(cur.a.x, cur.a.y, cur.a2, sh0, tq, lut3);
+                    if (v1) cur.b = ptq1_codes(cur.b.x, cur.b.y, cur.b2, sh1, tq, lut3);
+                }
                 float d[kHalves][NT][4];  // g64: MMAs 0-3 and 4-7 fill the two halves
 #pragma unroll
                 for (int h = 0; h < kHalves; h++)
@@ -283,6 +410,11 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
         }
     }
 
+    if (!barrier_ok)
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int e = 0; e < 4; e++) acc[nt][e] = __int_as_float(0x7fc00000);
     // ---- output (warps wholly past N do nothing; every CTA of the row block agrees)
     if (n0 >= N) return;
     if (S == 1) {
@@ -354,10 +486,41 @@ size_t gsum_bytes(int64_t M, int64_t K) {  // room for the g64 half sums
     return ((size_t)(K / kGroup) * 2 * MT * 4 + 255) / 256 * 256;
 }
 
+// The kernel instance for (M, fmt), its shared memory, and whether its grid is resident
+// on the GPU at once (then the rotation runs inside it: one launch).
+template <int NT, int kFmt>
+cudaError_t kernel_fits(int64_t grid_ctas, int smem, const DeviceInfo &dev, bool *fits) {
+    auto kern = skinny_kernel<NT, kFmt>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (err != cudaSuccess) return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+    if (err != cudaSuccess) return err;
+    *fits = grid_ctas <= (int64_t)per_sm * dev.sm_count;
+    return cudaSuccess;
+}
+
+cudaError_t grid_fits(int64_t M, int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev, bool *fits) {
+    int S, gpc;
+    choose_split(N, K, split_k, dev, &S, &gpc);
+    const int64_t ctas = ((N + kRowsPerCta - 1) / kRowsPerCta) * S;
+    const int NT = M <= 8 ? 1 : 2;
+    const int smem = smem_bytes(NT, gpc, fmt == 4);
+    if (NT == 1)
+        return fmt == 4   ? kernel_fits<1, 4>(ctas, smem, dev, fits)
+               : fmt == 3 ? kernel_fits<1, 3>(ctas, smem, dev, fits)
+               : fmt == 1 ? kernel_fits<1, 1>(ctas, smem, dev, fits)
+                          : kernel_fits<1, 2>(ctas, smem, dev, fits);
+    return fmt == 4   ? kernel_fits<2, 4>(ctas, smem, dev, fits)
+           : fmt == 3 ? kernel_fits<2, 3>(ctas, smem, dev, fits)
+           : fmt == 1 ? kernel_fits<2, 1>(ctas, smem, dev, fits)
+                      : kernel_fits<2, 2>(ctas, smem, dev, fits);
+}
+
 }  // namespace
 
 bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt) {
-    return (fmt == 2 || fmt == 3 || fmt == 4) && M >= 1 && M <= 16 && K % kGroup == 0 && (N + 15) / 16 <= kMaxTiles &&
+    return fmt >= 1 && fmt <= 4 && M >= 1 && M <= 16 && K % kGroup == 0 && (N + 15) / 16 <= kMaxTiles &&
            K < ((int64_t)1 << 31);
 }
 
@@ -368,10 +531,16 @@ size_t skinny_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int spli
     return staged_bytes(M, K) + gsum_bytes(M, K) + (S > 1 ? (size_t)S * (size_t)M * (size_t)N * sizeof(float) : 0);
 }
 
+int skinny_launches(int64_t M, int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev) {
+    bool fits = false;
+    if (grid_fits(M, N, K, fmt, split_k, dev, &fits) != cudaSuccess) return -1;
+    return fits ? 1 : 2;
+}
+
 cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                           uint16_t *y, int64_t M, int64_t N, int64_t K, int fmt, int split_k,
                           const Workspace &ws, cudaStream_t s, const DeviceInfo &dev) {
-    if (fmt != 2 && fmt != 3 && fmt != 4) return cudaErrorInvalidValue;
+    if (fmt < 1 || fmt > 4) return cudaErrorInvalidValue;
     uint16_t *xsg = reinterpret_cast<uint16_t *>(ws.data);
     float *gsg = reinterpret_cast<float *>(ws.data + staged_bytes(M, K));
     float *partials = reinterpret_cast<float *>(ws.data + staged_bytes(M, K) + gsum_bytes(M, K));
@@ -380,21 +549,30 @@ cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16
     const dim3 grid((unsigned)((N + kRowsPerCta - 1) / kRowsPerCta), (unsigned)S);
     const int64_t G = K / kGroup;
     const bool g64 = fmt == 4;
+    // one launch when the whole grid is resident at once (its CTAs meet at a barrier after
+    // rotating x), else the rotation pass first
+    bool fits = false;
+    cudaError_t ferr = grid_fits(M, N, K, fmt, split_k, dev, &fits);
+    if (ferr != cudaSuccess) return ferr;
+    const bool fused = fits && ws.zeroed != nullptr && ws.zeroed_bytes >= kCtlRegionBytes;
     auto run = [&](auto prep, auto kern, int MT, int NT) -> cudaError_t {
-        prep<<<(unsigned)((G * MT + 7) / 8), 256, 0, s>>>(x, xsg, gsg, (int)M, K);
         const int smem = smem_bytes(NT, gpc, g64);
         cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err != cudaSuccess) return err;
-        kern<<<grid, kThreads, smem, s>>>(xsg, gsg, packed, scales, y, partials, ws.counters, (int)M, N, K, S, gpc);
+        if (!fused) prep<<<(unsigned)((G * MT + 7) / 8), 256, 0, s>>>(x, xsg, gsg, (int)M, K);
+        kern<<<grid, kThreads, smem, s>>>(xsg, gsg, packed, scales, y, partials, ws.counters, (int)M, N, K, S, gpc,
+                                          fused ? x : nullptr, reinterpret_cast<unsigned int *>(ws.zeroed));
         return cudaGetLastError();
     };
     if (M <= 8) {
         if (g64) return run(skinny_prep_kernel<8, 4>, skinny_kernel<1, 4>, 8, 1);
         if (fmt == 3) return run(skinny_prep_kernel<8, 3>, skinny_kernel<1, 3>, 8, 1);
+        if (fmt == 1) return run(skinny_prep_kernel<8, 1>, skinny_kernel<1, 1>, 8, 1);
         return run(skinny_prep_kernel<8, 2>, skinny_kernel<1, 2>, 8, 1);
     }
     if (g64) return run(skinny_prep_kernel<16, 4>, skinny_kernel<2, 4>, 16, 2);
     if (fmt == 3) return run(skinny_prep_kernel<16, 3>, skinny_kernel<2, 3>, 16, 2);
+    if (fmt == 1) return run(skinny_prep_kernel<16, 1>, skinny_kernel<2, 1>, 16, 2);
     return run(skinny_prep_kernel<16, 2>, skinny_kernel<2, 2>, 16, 2);
 }
 

@@ -8,7 +8,7 @@ the float64 checker with the parity bar (rel-L2 <= 1e-3, max abs <= 1e-2 * rms).
   its largest element, so the noise elements keep only about 4 significant bits: the rows
   whose trit at j is 0 carry exactly that coarse part.  Every linear kernel gets it.
 * The skinny batches at the full qkv shape, and PTQ1_0 batches of 2 and 16 tokens at
-  full 27B-class shapes (they take the prefill GEMM).
+  full 27B-class shapes.
 * The automatic choice at batch 1 on both sides of the integer GEMV's grid limit.
 """
 import numpy as np
@@ -69,6 +69,7 @@ DOMINANT_CASES = [
     ("GEMV", PTQ1, 1, 1000, 2048), ("GEMV", PQ2, 1, 1000, 2048), ("GEMV", Q1, 1, 1000, 2048),
     ("GEMV", G64, 1, 1000, 2048),
     ("SKINNY", PQ2, 4, 1000, 2048), ("SKINNY", G64, 4, 1000, 2048), ("SKINNY", Q1, 4, 1000, 2048),
+    ("SKINNY", PTQ1, 4, 1000, 2048),
     ("SKINNY", PQ2, 16, 700, 1024),
     ("GEMM", PTQ1, 200, 600, 1024), ("GEMM", PQ2, 200, 600, 1024), ("GEMM", Q1, 200, 600, 1024),
     ("GEMM", G64, 200, 600, 1024),
@@ -119,7 +120,7 @@ def test_imma_error_within_the_fixed_point_step(bz, fmt, c):
     assert ok, (rel, mx)
 
 
-@pytest.mark.parametrize("fmt", [PQ2, G64, Q1])
+@pytest.mark.parametrize("fmt", [PQ2, G64, Q1, PTQ1])
 @pytest.mark.parametrize("M", [2, 16])
 def test_skinny_full_qkv_shape(bz, fmt, M):
     """The qkv projection (5120 -> 7168) in skinny batches, every output."""
@@ -133,7 +134,7 @@ def test_skinny_full_qkv_shape(bz, fmt, M):
 @pytest.mark.parametrize("K,N", [(5120, 7168), (17408, 5120), (5120, 34816)])
 def test_ptq1_small_batches_full_shapes(bz, M, K, N):
     """PTQ1_0 batches of 2 and 16 tokens at full 27B-class shapes through the default
-    entry point, every output."""
+    entry point (the skinny kernel), every output."""
     p = Problem(M, N, K, PTQ1, seed=50 + M)
     got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
     ok, rel, mx = oracle.compare(got, p.oracle_y())

@@ -418,6 +418,7 @@ def test_gemm_prefill_full_size_sampled(bz, fmt, M, K, N):
     y = torch.full((M, N), float("nan"), dtype=torch.float16, device=dev)
     bz.bonsai_ternary_linear(x, packed, s, y, M, N, K, fmt)
     torch.cuda.synchronize()
+    assert bz.bonsai_launch_count(M, N, K, fmt) == 1  # the rotation runs inside the GEMM
     rng = np.random.default_rng(M + N)
     ms = np.concatenate([[0, M - 1], rng.integers(0, M, 62)])
     ns = np.concatenate([[0, N - 1], rng.integers(0, N, 62)])
@@ -433,7 +434,7 @@ def test_gemm_prefill_full_size_sampled(bz, fmt, M, K, N):
 SKINNY_SMALL = [(2, 64, 128), (3, 129, 384), (8, 300, 1024), (9, 100, 640), (16, 257, 2048)]
 
 
-@pytest.mark.parametrize("fmt", [PQ2, G64, Q1])
+@pytest.mark.parametrize("fmt", [PQ2, G64, Q1, PTQ1])
 @pytest.mark.parametrize("M,N,K", SKINNY_SMALL)
 @pytest.mark.parametrize("split_k", [0, 1, 3])
 def test_skinny_small(bz, fmt, M, N, K, split_k):
@@ -443,19 +444,21 @@ def test_skinny_small(bz, fmt, M, N, K, split_k):
     assert ok, (rel, mx)
 
 
-@pytest.mark.parametrize("fmt", [PQ2, G64, Q1])
+@pytest.mark.parametrize("fmt", [PQ2, G64, Q1, PTQ1])
 @pytest.mark.parametrize("M", [2, 4, 8, 16])
-@pytest.mark.parametrize("K,N", [(5120, 5120), (17408, 5120), (5120, 34816)])
+@pytest.mark.parametrize("K,N", [(5120, 7168), (5120, 5120), (17408, 5120), (5120, 34816)])
 def test_skinny_decode_shapes_full(bz, fmt, M, K, N):
     """Skinny decode batches on 27B-class projections, every output against the checker
-    (the default entry point takes the skinny kernel for these packings)."""
+    (the default entry point takes the skinny kernel for every packing); one launch when
+    the kernel's grid is resident at once, as it is at these shapes."""
     p = Problem(M, N, K, fmt, seed=M)
     got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
+    assert bz.bonsai_launch_count(M, N, K, fmt) == 1
 
 
-@pytest.mark.parametrize("fmt", [PQ2, G64, Q1])
+@pytest.mark.parametrize("fmt", [PQ2, G64, Q1, PTQ1])
 def test_skinny_split_is_deterministic(bz, fmt):
     import torch
     p = Problem(8, 5120, 17408, fmt, seed=3)
@@ -471,12 +474,15 @@ def test_skinny_split_is_deterministic(bz, fmt):
 
 
 @pytest.mark.parametrize("M", [2, 5, 16])
-@pytest.mark.parametrize("fmt", [PTQ1])
-def test_small_batches_ptq1_take_the_gemm(bz, M, fmt):
-    p = Problem(M, 300, 1024, fmt, seed=M)
+@pytest.mark.parametrize("N,K", [(300, 1024), (3, 128), (77, 640)])
+def test_small_batches_ptq1(bz, M, N, K):
+    """PTQ1_0 batches take the skinny kernel (base-3 bytes transcoded to 2-bit codes); the
+    small N puts the plane's last group, whose lanes read its final bytes, in most warps."""
+    p = Problem(M, N, K, PTQ1, seed=M + N)
     got = _run(bz, p, bz.BONSAI_ALGO_AUTO)
     ok, rel, mx = oracle.compare(got, p.oracle_y())
     assert ok, (rel, mx)
+    assert np.array_equal(got, _run(bz, p, bz.BONSAI_ALGO_SKINNY))
 
 
 # ------------------------------------------------------------ SwiGLU after the fused gate/up projection

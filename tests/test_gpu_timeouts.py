@@ -83,3 +83,60 @@ def test_status_is_clear_after_normal_calls(bz):
     got = _run(bz, x, packed, scales, 3000, 5120)
     assert oracle.compare(got, p.oracle_y()[0])[0]
     assert bz.bonsai_device_status() == 0
+
+
+def gemm_split_tiles(M, N, K, sms):
+    """Output tiles of the prefill GEMM that are split between CTAs, from its work split:
+    tiles of 128 acc rows x 256 columns (row tile fastest), acc = 2 when M > 128; C = min(SMs,
+    ceil(units / 4)) CTAs; W = T / C - 1 whole-tile waves when T >= 2C; the remaining tiles'
+    64-wide K stages split evenly, CTA b taking units [Ur b / C, Ur (b + 1) / C)."""
+    acc = 2 if M > 128 else 1
+    mt, nt, nk = -(-M // (128 * acc)), -(-N // 256), K // 64
+    C = max(1, min(sms, -(-(mt * nt * nk) // 4)))
+    T = mt * nt
+    W = T // C - 1 if T // C >= 2 else 0
+    Ur = (T - W * C) * nk
+    split = set()
+    for b in range(1, C):
+        u = Ur * b // C
+        if u % nk != 0:
+            split.add(W * C + u // nk)
+    return [(s % mt, s // mt, acc) for s in sorted(split)]
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 1000, 640), (600, 2000, 1152)])
+def test_forced_gemm_flag_timeouts_nan_status_and_recovery(bz, M, N, K):
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    p = Problem(M, N, K, PQ2, seed=M + N)
+    x, packed, scales = p.device()
+    ref = p.oracle_y()
+    split = gemm_split_tiles(M, N, K, sms)
+    assert len(split) > 0
+
+    def run():
+        y = torch.full((M, N), 7.0, dtype=torch.float16, device="cuda")
+        bz.bonsai_ternary_linear_algo(x, packed, scales, y, M, N, K, PQ2, bz.BONSAI_ALGO_GEMM)
+        torch.cuda.synchronize()
+        return to_numpy_f16(y)
+
+    bz.bonsai_device_status(clear=True)
+    bz.bonsai_debug_force_timeouts(True)
+    try:
+        got = run()
+    finally:
+        bz.bonsai_debug_force_timeouts(False)
+    status = bz.bonsai_device_status(clear=True)
+    assert status & bz.BONSAI_DEVICE_GEMM_TIMEOUT
+    bad = np.zeros((M, N), dtype=bool)
+    for tm, tn, acc in split:
+        bad[128 * acc * tm:128 * acc * (tm + 1), 256 * tn:256 * (tn + 1)] = True
+    assert np.all(np.isnan(got[bad]))
+    assert np.all(np.isfinite(got[~bad]))
+    ok, rel, mx = oracle.compare(got[~bad], ref[~bad])
+    assert ok, (rel, mx)
+    for _ in range(2):
+        again = run()
+        ok, rel, mx = oracle.compare(again, ref)
+        assert ok, (rel, mx)
+    assert bz.bonsai_device_status() == 0
