@@ -555,7 +555,7 @@ def measure_swiglu_decode(stack, xs, bz, torch, stream, dev, args):
     return out
 
 
-PREFILL_MS = (512, 2048, 8192)
+PREFILL_MS = (512, 2048, 8192)  # the prefill workload's token counts
 
 
 def measure_prefill(fmt, base, dev, bz, torch, args, peaks, peak_kind):
@@ -571,7 +571,7 @@ def measure_prefill(fmt, base, dev, bz, torch, args, peaks, peak_kind):
     burst = float(peaks["bf16_tflops"])
     grid = {}
     summary = None
-    for M in PREFILL_MS:
+    for M in args.prefill_ms:
         per = {}
         total_flop, layer_us = 0, 0.0
         for i, (name, K, N) in enumerate(SHAPES):
@@ -616,7 +616,7 @@ def measure_prefill(fmt, base, dev, bz, torch, args, peaks, peak_kind):
     out = {"grid": grid, "l2": "every call after a write of 2x the L2 size", "calls_per_entry": calls}
     if summary is not None:
         out.update(summary)
-    if fmt == 2 and args.prefill_m in PREFILL_MS:
+    if fmt == 2 and args.prefill_m in args.prefill_ms:
         out["swiglu_gate_up"] = measure_swiglu_prefill(fmt, base, dev, bz, torch, args.prefill_m, calls, flush)
     return out
 
@@ -723,6 +723,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-m", type=int, default=2048,
                     help="tokens of the prefill summary line, one of 512, 2048, 8192 (0: skip the prefill grid)")
+    ap.add_argument("--prefill-ms", default=",".join(str(m) for m in PREFILL_MS),
+                    help="token counts of the prefill grid (comma-separated)")
     ap.add_argument("--skinny", type=int, default=1, help="measure the M = 1..16 decode grid (PQ2_0, PTQ1_0)")
     ap.add_argument("--case", choices=["gemv", "imma", "gemm", "skinny"], help="run one projection only (profiler case)")
     ap.add_argument("--shape", choices=[n for n, _, _ in SHAPES], default="gate_up")
@@ -730,6 +732,7 @@ def main():
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    args.prefill_ms = tuple(int(m) for m in args.prefill_ms.split(",") if m)
 
     world, rank, _ = dist_setup()
     if args.case:
