@@ -704,12 +704,12 @@ def run_case(args):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.reps):
-        bz.bonsai_ternary_linear_algo(x, packed, s, y, M, N, K, fmt, algo)
+        bz.bonsai_ternary_linear_algo(x, packed, s, y, M, N, K, fmt, algo, args.tile)
     e1.record()
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / args.reps
     print(json.dumps({"case": args.case, "shape": args.shape, "fmt": FMT_NAMES[fmt], "M": M, "K": K, "N": N,
-                      "reps": args.reps, "us_per_call": round(us, 2)}), flush=True)
+                      "tile": args.tile, "reps": args.reps, "us_per_call": round(us, 2)}), flush=True)
 
 
 def main():
@@ -730,6 +730,8 @@ def main():
     ap.add_argument("--shape", choices=[n for n, _, _ in SHAPES], default="gate_up")
     ap.add_argument("--m", type=int, default=2048, help="tokens for --case gemm / skinny (skinny: at most 16)")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--tile", type=int, default=0,
+                    help="--case: the kernel's split/tile argument (GEMM: 1, 2 or 3 = CTA pairs; 0 automatic)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     args.prefill_ms = tuple(int(m) for m in args.prefill_ms.split(",") if m)

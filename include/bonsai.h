@@ -170,8 +170,9 @@ int bonsai_ternary_linear(const uint16_t *x, const uint8_t *packed, const uint16
  * explicit split-K factor for the skinny kernel (0 = automatic, 1 = no split,
  * otherwise the number of K chunks, clamped to what the shape allows).  For
  * BONSAI_ALGO_GEMM the same argument picks the M tile instead: 1 = 128 rows per CTA,
- * 2 = 256 rows (two TMEM accumulators sharing each expanded weight tile), 0 =
- * automatic.  For BONSAI_ALGO_GEMV it picks the schedule: 1 = each CTA walks all K
+ * 2 = 256 rows (two TMEM accumulators sharing each expanded weight tile), 3 = CTA
+ * pairs (clusters of two SMs issuing 256-row tcgen05 MMAs together, each SM expanding
+ * half of every weight tile; an explicit choice only), 0 = automatic (1 or 2).  For BONSAI_ALGO_GEMV it picks the schedule: 1 = each CTA walks all K
  * slices of its rows (no split-K), >= 2 = one 512-wide K slice per CTA with split-K
  * partials, 0 = automatic.  BONSAI_ALGO_IMMA ignores it (its work split is fixed
  * by the shape and the SM count, so results are bitwise repeatable).

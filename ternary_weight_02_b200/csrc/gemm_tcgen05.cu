@@ -45,28 +45,33 @@ namespace {
 constexpr int BM = 128, BN = 256, BK = 64;  // BM: rows of one MMA / one TMEM accumulator
 constexpr int kExpandWarps = 8;
 constexpr int kThreads = (2 + kExpandWarps) * 32;  // 320
-constexpr int B_STAGE_BYTES = BN * BK * 2;         // 32 KB
-constexpr int CODE_STAGE_BYTES = BN * BK / 4;      // PQ2_0 codes of a B stage: 256 rows x 16 bytes
 
 // Tile configuration: kAcc accumulators of 128 rows each share every B stage (the
-// expanded weights), so the CTA covers 128 * kAcc rows of y.
-template <int kAcc>
+// expanded weights), so the CTA covers 128 * kAcc rows of y.  kPair (CTA pairs): each CTA
+// holds half of a B stage (128 weight rows), so the same shared memory takes more stages,
+// which the pair's longer round trip per stage (both CTAs' copies and expansions) needs.
+template <int kAcc, bool kPair = false>
 struct Cfg {
-    static constexpr int kStages = kAcc == 2 ? 3 : 4;
+    static constexpr int kStages = kPair ? (kAcc == 2 ? 4 : 6) : (kAcc == 2 ? 3 : 4);
     static constexpr int kTileM = BM * kAcc;
     static constexpr int kAStage = kTileM * BK * 2;  // 16 or 32 KB
+    static constexpr int kBStage = (kPair ? BN / 2 : BN) * BK * 2;   // 16 or 32 KB
+    static constexpr int kCodeStage = (kPair ? BN / 2 : BN) * BK / 4;  // PQ2_0 codes of a B stage
     static constexpr int kTmemCols = 256 * kAcc;
     // shared memory: [A stages][B stages][PQ2_0 code stages][barriers][tmem slot][abort
     // flag][PTQ1_0 LUT]
     static constexpr int kOffA = 0;
     static constexpr int kOffB = kStages * kAStage;
-    static constexpr int kOffCodes = kOffB + kStages * B_STAGE_BYTES;
-    static constexpr int kOffBar = kOffCodes + kStages * CODE_STAGE_BYTES;
+    static constexpr int kOffCodes = kOffB + kStages * kBStage;
+    static constexpr int kOffBar = kOffCodes + kStages * kCodeStage;
     static constexpr int kNumBars = 3 * kStages + 6;  // full_a, full_b, empty, done, tmem_free, fin, 3 rotation
     static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
     static constexpr int kOffAbort = kOffTmemSlot + 8;
     static constexpr int kOffLut = kOffAbort + 8;
     static constexpr int kSmemBytes = kOffLut + 256 * 4 + 1024;  // + slack for the 1024-B tile base
+    // the epilogue stages y through the B ring: 8 warps x 8 KB
+    static_assert(kStages * kBStage >= kExpandWarps * 8192, "the B ring holds the epilogue's staging rows");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -97,6 +102,59 @@ __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate));
 }
+// The same for a CTA pair (cta_group::2): M = 256, rows 0..127 of A and D in the even CTA
+// of the pair and rows 128..255 in the odd one; B's N = 256 columns split the same way
+// (columns 0..127 in the even CTA's shared memory).  Issued by the even CTA only.
+constexpr uint32_t kIdesc2 = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                             ((uint32_t)(256 >> 4) << 24);
+__device__ __forceinline__ void mma_f16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc2), "r"(accumulate));
+}
+// Arrives on the barrier at the same shared-memory offset in both CTAs of the pair once
+// every MMA the pair's issuing thread started has completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(saddr(bar)), "h"((uint16_t)3)
+        : "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+// Bounded wait with cluster-scope acquire (arrivals from the peer CTA included).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinLimit; i++) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(saddr(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(saddr(bar))
                  : "memory");
@@ -304,14 +362,25 @@ __device__ __forceinline__ void expand_warps_sync() { asm volatile("bar.sync 1, 
 // 256 weight rows are then gate rows 128 tn .. 128 tn + 127 followed by the matching up
 // rows, so that each epilogue warp finds gate column c and up column 128 + c of the same
 // output in its own accumulator lanes.
-template <int kFmt, int kAcc, bool kSwiglu>
+//
+// kPair: the CTAs work in pairs (clusters of two) on tiles of 256 kAcc rows x 256 columns
+// with tcgen05.mma.cta_group::2: CTA rank r of the pair holds x' rows a 256 + 128 r ..
+// +127 of its accumulator a and expands weight rows 128 r .. 128 r + 127 of the tile's
+// 256 (two threads per row, half a stage each), so each SM expands and reads half the B
+// operand for the same MMA work.  The even CTA issues the MMAs once both CTAs' stages
+// are ready (its full_b barrier counts its own expansion warps and one arrival that a
+// thread of the odd CTA forwards) and commits them to the barriers of both; hand-over
+// slots and flags stay per CTA, work is split per pair.  Only an explicit request takes
+// this mode: on the 27B-class projections it runs a few per cent behind single-CTA
+// tiles, whose x' traffic per MMA it shares, so halving the expansion buys nothing there.
+template <int kFmt, int kAcc, bool kSwiglu, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     const __grid_constant__ CUtensorMap a_map, const __grid_constant__ CUtensorMap w_map,
     const uint8_t *__restrict__ packed,
     const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
     const uint16_t *__restrict__ x, uint16_t *__restrict__ xr, int64_t nblocks, unsigned int *__restrict__ ctl,
     uint32_t wait_limit, uint32_t epoch_skew, int M, int N, int K, int mt, int F) {
-    using C = Cfg<kAcc>;
+    using C = Cfg<kAcc, kPair>;
     constexpr int STAGES = C::kStages;
     constexpr int kSlotFloats = C::kTileM * BN;
     extern __shared__ uint8_t smem_raw[];
@@ -337,14 +406,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     constexpr bool kTma = kFmt == 2 || kFmt == 4;
     const int64_t G64 = K / 64;  // PQ2_0 g64: scales per row
     const int nctas = (int)gridDim.x, cta = (int)blockIdx.x;
-    // whole-tile waves first (CTA b: tiles b, b + C, ...), then the last one or two
-    // waves' worth of tiles split by units
+    // the work split's unit: a CTA, or (kPair) a pair of CTAs
+    const int rank = kPair ? (int)cluster_rank() : 0;
+    const int nunits = kPair ? nctas / 2 : nctas, unit = kPair ? cta / 2 : cta;
+    auto cta_of = [&](int u) { return kPair ? 2 * u + rank : u; };  // this rank's CTA of unit u
+    constexpr int kTileRows = kPair ? 256 * kAcc : C::kTileM;      // x' rows of a tile
+    // first x' row of this CTA's accumulator a in row tile tm
+    auto acc_row0 = [&](int tm, int a) { return tm * kTileRows + (kPair ? a * 256 + rank * BM : a * BM); };
+    // whole-tile waves first (unit b: tiles b, b + C, ...), then the last one or two
+    // waves' worth of tiles split by K stages
     const int T = mt * ((N + BN - 1) / BN);
-    const int W = T / nctas >= 2 ? T / nctas - 1 : 0;
-    const int Tdp = W * nctas;
+    const int W = T / nunits >= 2 ? T / nunits - 1 : 0;
+    const int Tdp = W * nunits;
     const int Ur = (T - Tdp) * nk;
-    auto range_end = [&](int c) { return (int)((int64_t)Ur * (c + 1) / nctas); };
-    const int u_begin = (int)((int64_t)Ur * cta / nctas), u_end = range_end(cta);
+    auto range_end = [&](int c) { return (int)((int64_t)Ur * (c + 1) / nunits); };
+    const int u_begin = (int)((int64_t)Ur * unit / nunits), u_end = range_end(unit);
     const int n_mine = W * nk + (u_end - u_begin);  // this CTA's units
     // the piece that starts at this CTA's unit v: tile s (row tile fastest), stages
     // [kb, ke); tr: the tile's index among the split ones (-1 for a whole-tile wave)
@@ -354,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     auto piece_at = [&](int v) {
         Piece p;
         if (v < W * nk) {
-            p.s = cta + (v / nk) * nctas;
+            p.s = unit + (v / nk) * nunits;
             p.kb = 0;
             p.ke = nk;
             p.tr = -1;
@@ -429,11 +505,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     if (tid == 0) {
         for (int st = 0; st < STAGES; st++) {
             mbar_init(full_a + st, 1);
-            mbar_init(full_b + st, kExpandWarps);
+            // (kPair: the even CTA's barrier also takes the odd CTA's forwarded arrival)
+            mbar_init(full_b + st, kExpandWarps + (kPair && rank == 0 ? 1 : 0));
             mbar_init(empty + st, 1);
         }
         mbar_init(done, 1);
-        mbar_init(tmem_free, kExpandWarps);
+        mbar_init(tmem_free, kExpandWarps + (kPair && rank == 0 ? 1 : 0));
         mbar_init(fin, 1);
         *abort_flag = rot_fail ? 1 : 0;
         mbar_init_fence();
@@ -459,13 +536,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
         }
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)),
-                     "r"(C::kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if (kPair) {  // the same warp in both CTAs of the pair, the same slot address
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)),
+                         "r"(C::kTmemCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)),
+                         "r"(C::kTmemCols)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     tc_fence_before();
     __syncthreads();
+    // kPair: both CTAs' barriers exist before the first arrival from the peer
+    if (kPair) cluster_sync();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t epoch = *epoch_s;
@@ -494,19 +580,26 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                         *abort_flag = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(full_a + st, C::kAStage + (kTma ? CODE_STAGE_BYTES : 0));
+                    mbar_arrive_expect_tx(full_a + st,
+                                          C::kAStage + (kTma ? C::kCodeStage : 0));
 #pragma unroll
                     for (int a = 0; a < kAcc; a++)
                         tma_load_2d(sA + st * C::kAStage + a * (BM * BK * 2), &a_map, full_a + st, ks * BK,
-                                    tm * C::kTileM + a * BM);
+                                    acc_row0(tm, a));
+                    // kPair: this CTA's 128 weight rows of the tile (SwiGLU: rank 0 the gate
+                    // rows, rank 1 the matching up rows)
+                    if (kTma && kPair)
+                        tma_load_2d(const_cast<uint8_t *>(sCodes) + st * C::kCodeStage, &w_map, full_a + st,
+                                    ks * (BK / 4),
+                                    kSwiglu ? (rank == 0 ? tn * (BN / 2) : F + tn * (BN / 2)) : tn * BN + rank * 128);
                     // PQ2_0: the stage's codes, 16 bytes of each of the tile's 256 weight rows
-                    if (kTma && !kSwiglu)
-                        tma_load_2d(const_cast<uint8_t *>(sCodes) + st * CODE_STAGE_BYTES, &w_map, full_a + st,
+                    if (kTma && !kSwiglu && !kPair)
+                        tma_load_2d(const_cast<uint8_t *>(sCodes) + st * C::kCodeStage, &w_map, full_a + st,
                                     ks * (BK / 4), tn * BN);
-                    if (kTma && kSwiglu) {  // 128 gate rows, then the matching 128 up rows
-                        tma_load_2d(const_cast<uint8_t *>(sCodes) + st * CODE_STAGE_BYTES, &w_map, full_a + st,
+                    if (kTma && kSwiglu && !kPair) {  // 128 gate rows, then the matching 128 up rows
+                        tma_load_2d(const_cast<uint8_t *>(sCodes) + st * C::kCodeStage, &w_map, full_a + st,
                                     ks * (BK / 4), tn * (BN / 2));
-                        tma_load_2d(const_cast<uint8_t *>(sCodes) + st * CODE_STAGE_BYTES + CODE_STAGE_BYTES / 2,
+                        tma_load_2d(const_cast<uint8_t *>(sCodes) + st * C::kCodeStage + C::kCodeStage / 2,
                                     &w_map, full_a + st, ks * (BK / 4), F + tn * (BN / 2));
                     }
                 }
@@ -517,14 +610,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                 mbar_wait(full_a + (i % STAGES), (uint32_t)(i / STAGES) & 1u);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // ------------------------------------------------ MMA issuer (kPair: the even CTA)
+        if (lane == 0 && rank == 0) {
             int it = 0, pc = 0;
             for (int v = 0; v < n_mine && !*abort_flag; pc++) {
                 const Piece p = piece_at(v);
                 v += p.ke - p.kb;
-                // the accumulator is free once the previous piece's epilogue has read it
-                if (pc > 0 && !mbar_wait(tmem_free, (uint32_t)(pc - 1) & 1u)) {
+                // the accumulator is free once the previous piece's epilogue has read it (kPair:
+                // the epilogues of both CTAs)
+                if (pc > 0 && !(kPair ? mbar_wait_cluster(tmem_free, (uint32_t)(pc - 1) & 1u)
+                                      : mbar_wait(tmem_free, (uint32_t)(pc - 1) & 1u))) {
                     *abort_flag = 1;
                     break;
                 }
@@ -532,46 +627,103 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                 for (int ks = p.kb; ks < p.ke; ks++, it++) {
                     const int st = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    if (*abort_flag || !mbar_wait(full_a + st, ph) || !mbar_wait(full_b + st, ph)) {
+                    // kPair: full_b completes once this CTA's expansion warps have written their
+                    // B half and the odd CTA's forwarder has seen its half written and its x' in
+                    if (*abort_flag || !mbar_wait(full_a + st, ph) ||
+                        !(kPair ? mbar_wait_cluster(full_b + st, ph) : mbar_wait(full_b + st, ph))) {
                         *abort_flag = 1;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t b0 = saddr(sB + st * B_STAGE_BYTES);
+                    const uint32_t b0 = saddr(sB + st * C::kBStage);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; kk++) {
                         const uint64_t bdesc = desc_sw128(b0 + kk * 32);
 #pragma unroll
                         for (int a = 0; a < kAcc; a++) {
                             const uint32_t a0 = saddr(sA + st * C::kAStage + a * (BM * BK * 2));
-                            mma_f16(tmem + (uint32_t)(a * 256), desc_sw128(a0 + kk * 32), bdesc,
-                                    (ks > p.kb || kk > 0) ? 1u : 0u);
+                            if (kPair)
+                                mma_f16_pair(tmem + (uint32_t)(a * 256), desc_sw128(a0 + kk * 32), bdesc,
+                                             (ks > p.kb || kk > 0) ? 1u : 0u);
+                            else
+                                mma_f16(tmem + (uint32_t)(a * 256), desc_sw128(a0 + kk * 32), bdesc,
+                                        (ks > p.kb || kk > 0) ? 1u : 0u);
                         }
                     }
-                    mma_commit(empty + st);  // frees the stage when these MMAs have read it
+                    // frees the stage when these MMAs have read it (kPair: in both CTAs)
+                    if (kPair)
+                        mma_commit_pair(empty + st);
+                    else
+                        mma_commit(empty + st);
                 }
                 if (*abort_flag) break;
-                mma_commit(done);  // the piece's sums are complete in tensor memory
+                // the piece's sums are complete in tensor memory
+                if (kPair)
+                    mma_commit_pair(done);
+                else
+                    mma_commit(done);
             }
             // every MMA this thread issued has completed before tensor memory is freed
-            mma_commit(fin);
+            if (kPair)
+                mma_commit_pair(fin);
+            else
+                mma_commit(fin);
+            mbar_wait(fin, 0);
+        } else if (kPair && lane == 0) {
+            // the odd CTA: its expansion warps arrive on its own barriers, and this thread
+            // forwards each completed stage (B half written, x' and codes landed) and each
+            // freed accumulator to the even CTA's barriers with one cluster-scope arrival.
+            // (An arrival with cluster-scope release waits for all of the arriving thread's
+            // earlier memory operations; here that is one idle thread, not the expansion
+            // warps with their scale and code loads in flight.)  The events come in the
+            // order the expansion warps make them: a piece's stages, then its accumulator.
+            const uint32_t full_b_lead = cluster_addr(full_b, 0);
+            const uint32_t tmem_free_lead = cluster_addr(tmem_free, 0);
+            int it = 0;
+            bool ok = true;
+            for (int v = 0, pc = 0; v < n_mine && ok; pc++) {
+                const Piece p = piece_at(v);
+                v += p.ke - p.kb;
+                for (int ks = p.kb; ks < p.ke; ks++, it++) {
+                    const int st = it % STAGES;
+                    const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+                    if (*abort_flag || !mbar_wait(full_b + st, ph) || !mbar_wait(full_a + st, ph)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_remote(full_b_lead + (uint32_t)(st * 8));
+                }
+                if (!ok || !mbar_wait(tmem_free, (uint32_t)pc & 1u)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_remote(tmem_free_lead);
+            }
+            if (!ok) *abort_flag = 1;
+            // its shared memory and tensor memory serve the pair's MMAs until the even
+            // CTA's last commit
             mbar_wait(fin, 0);
         }
     } else {
         // ------------------------------------------------ trit expansion (one row per thread), epilogues
-        const int r = tid - 64;            // 0 .. 255: row of the B tile
+        const int r = tid - 64;            // 0 .. 255
         const int q = warp & 3;            // TMEM lane quadrant this warp may read
         const int half = (warp - 2) >> 2;  // which 128 columns of the tile it writes
+        // the B row this thread expands: its row rr of the CTA's B stage, row rb of the
+        // tile's 256, and (kPair: two threads per row) which 32 of a stage's 64 weights
+        const int rr = kPair ? (r & 127) : r;
+        const int rb = kPair ? rank * 128 + rr : r;
+        const int hsel = kPair ? (r >> 7) : 0;
         int it = 0, pc = 0;
         bool live = true;
         for (int v = 0; v < n_mine; pc++) {
             const Piece p = piece_at(v);
             v += p.ke - p.kb;
             const int tm = p.s % mt, tn = p.s / mt;
-            const int64_t n = kSwiglu ? (r < BN / 2 ? (int64_t)tn * (BN / 2) + r : (int64_t)F + tn * (BN / 2) + r - BN / 2)
-                                      : (int64_t)tn * BN + r;  // weight row
+            const int64_t n = kSwiglu ? (rb < BN / 2 ? (int64_t)tn * (BN / 2) + rb : (int64_t)F + tn * (BN / 2) + rb - BN / 2)
+                                      : (int64_t)tn * BN + rb;  // weight row
             // (SwiGLU: the last tile's gate rows past F belong to no output; their weights read as 0)
-            const bool valid = kSwiglu ? (int64_t)tn * (BN / 2) + (r & (BN / 2 - 1)) < F : n < N;
+            const bool valid = kSwiglu ? (int64_t)tn * (BN / 2) + (rb & (BN / 2 - 1)) < F : n < N;
             if (live) {
                 // PTQ1_0, Q1_0: the packed bytes of the group being expanded and of the next one (in
                 // flight) come by plain loads; PQ2_0: the codes come with the stage's x' tiles
@@ -622,29 +774,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                     }
                     uint32_t w4[4];
                     if (kTma) {
-                        const uint4 c4 = *reinterpret_cast<const uint4 *>(sCodes + st * CODE_STAGE_BYTES + r * 16);
+                        const uint4 c4 = *reinterpret_cast<const uint4 *>(sCodes + st * C::kCodeStage + rr * 16);
                         w4[0] = c4.x, w4[1] = c4.y, w4[2] = c4.z, w4[3] = c4.w;
                     } else {
 #pragma unroll
                         for (int i = 0; i < 4; i++) w4[i] = hf ? cw[4 + i] : cw[i];
                     }
-                    uint8_t *stage = sB + st * B_STAGE_BYTES;
+                    uint8_t *stage = sB + st * C::kBStage;
                     if (kFmt == 3) {
                         const uint32_t wq[2] = {hf ? cw[2] : cw[0], hf ? cw[3] : cw[1]};  // no dynamic index
 #pragma unroll
-                        for (int i = 0; i < 2; i++) {
+                        for (int i = 0; i < (kPair ? 1 : 2); i++) {
+                            const int ii = kPair ? hsel : i;  // (kPair: this thread's 32 weights)
                             uint32_t out[16];
-                            expand_word_q1(wq[i], tneg, out);  // weights 64ks + 32i .. +31
+                            expand_word_q1(ii ? wq[1] : wq[0], tneg, out);  // weights 64ks + 32ii .. +31
 #pragma unroll
-                            for (int c = 0; c < 4; c++) st_chunk(stage, r, 4 * i + c, out + 4 * c);
+                            for (int c = 0; c < 4; c++) st_chunk(stage, rr, 4 * ii + c, out + 4 * c);
                         }
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 4; i++) {
+                        for (int i = 0; i < (kPair ? 2 : 4); i++) {
+                            const int wi = kPair ? 2 * hsel + i : i;  // (kPair: this thread's 32 weights)
+                            const uint32_t wv = kPair ? (hsel ? w4[2 + i] : w4[i]) : w4[i];
                             uint32_t out[8];
-                            expand_word(w4[i], tneg, tpos, out);  // weights 64ks + 16i .. +15
-                            st_chunk(stage, r, 2 * i, out);
-                            st_chunk(stage, r, 2 * i + 1, out + 4);
+                            expand_word(wv, tneg, tpos, out);  // weights 64ks + 16wi .. +15
+                            st_chunk(stage, rr, 2 * wi, out);
+                            st_chunk(stage, rr, 2 * wi + 1, out + 4);
                         }
                     }
                     // make the generic-proxy accesses (these stores, the code loads) ordered
@@ -664,9 +819,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
             const bool owner = p.kb == 0 && p.ke < nk;        // first piece, others follow
             const int tile_end = (p.tr + 1) * nk;  // in split units
             bool got = true;  // the later pieces all arrived (owner)
-            if (owner)
-                for (int c2 = cta + 1, s = u_end; s < tile_end; s = range_end(c2), c2++)
-                    got = flag_wait(flags + c2, epoch + epoch_skew, wait_limit) && got;
+            if (owner)  // (the same rank's CTA of each later unit: its half of the tile)
+                for (int c2 = unit + 1, s = u_end; s < tile_end; s = range_end(c2), c2++)
+                    got = flag_wait(flags + cta_of(c2), epoch + epoch_skew, wait_limit) && got;
             if (!got && r == 0) atomicOr(status, kDevStatusGemmTimeout);
             const int w8 = warp - 2;
             if constexpr (kSwiglu) {
@@ -705,8 +860,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                             continue;
                         }
                         if (owner) {
-                            for (int c2 = cta + 1, s = u_end; s < tile_end; s = range_end(c2), c2++) {
-                                const float4 *sg = sw_slot(c2, a, cg), *su = sw_slot(c2, a, cu);
+                            for (int c2 = unit + 1, s = u_end; s < tile_end; s = range_end(c2), c2++) {
+                                const float4 *sg = sw_slot(cta_of(c2), a, cg), *su = sw_slot(cta_of(c2), a, cu);
 #pragma unroll
                                 for (int i = 0; i < 8; i++) {
                                     const float4 wg = __ldcg(sg + 32 * i), wu = __ldcg(su + 32 * i);
@@ -750,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
 #pragma unroll 4
                     for (int i = 0; i < 8; i++) {
                         const int row = 4 * i + (lane >> 3);
-                        const int m = tm * C::kTileM + a * BM + 32 * q + row;
+                        const int m = acc_row0(tm, a) + 32 * q + row;
                         const uint4 val = *reinterpret_cast<const uint4 *>(stage_h + row * 128 + ((ch ^ (row & 7)) << 4));
                         if (m >= M || f0 >= F) continue;
                         uint16_t *hr = y + (int64_t)m * F + f0;
@@ -799,8 +954,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                             continue;
                         }
                         if (owner) {
-                            for (int c2 = cta + 1, s = u_end; s < tile_end; s = range_end(c2), c2++) {
-                                const float4 *src = slot_at(c2, a, c);
+                            for (int c2 = unit + 1, s = u_end; s < tile_end; s = range_end(c2), c2++) {
+                                const float4 *src = slot_at(cta_of(c2), a, c);
                                 float4 w[8];
 #pragma unroll
                                 for (int i = 0; i < 8; i++) w[i] = __ldcg(src + 32 * i);
@@ -839,7 +994,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
 #pragma unroll 4
                 for (int i = 0; i < 16; i++) {
                     const int row = 2 * i + (lane >> 4);
-                    const int m = tm * C::kTileM + a * BM + 32 * q + row;
+                    const int m = acc_row0(tm, a) + 32 * q + row;
                     const uint4 val = *reinterpret_cast<const uint4 *>(stage_y + row * 256 + ((ch ^ (row & 7)) << 4));
                     if (m >= M || n0 >= N) continue;
                     uint16_t *yr = y + (int64_t)m * N + n0;
@@ -874,11 +1029,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && *abort_flag) atomicOr(status, kDevStatusGemmTimeout);
+    // kPair: neither CTA leaves (or frees its tensor memory) while the other may still
+    // arrive on its barriers or the pair's MMAs may still use its memory
+    if (kPair) cluster_sync();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
-                     : "memory");
+        if (kPair)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
+                         : "memory");
     }
 }
 
@@ -886,12 +1048,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
 
 // Tile and grid of one call.  Stream-K leaves no partial last wave, so two 128-row
 // accumulators (half the trit expansion per FLOP) are used whenever M > 128.
+// tile_hint 3: CTA pairs (cta_group::2), tiles of 256 acc rows, acc = 2 when M > 256;
+// the caller caps the pairs at the clusters that fit on the GPU at once.
 struct GemmPlan {
     int acc, mt, nt, nk, ctas;
+    bool pair;
     int64_t units;
 };
 GemmPlan gemm_plan(int64_t M, int64_t N, int64_t K, int tile_hint, int sm_count) {
     GemmPlan p;
+    p.pair = tile_hint == 3;
+    if (p.pair) {
+        p.acc = M > 2 * BM ? 2 : 1;
+        const int64_t rows = (int64_t)2 * BM * p.acc;
+        p.mt = (int)((M + rows - 1) / rows);
+        p.nt = (int)((N + BN - 1) / BN);
+        p.nk = (int)(K / BK);
+        p.units = (int64_t)p.mt * p.nt * p.nk;
+        int64_t pairs = (p.units + 3) / 4;
+        pairs = pairs < sm_count / 2 ? pairs : sm_count / 2;
+        p.ctas = (int)(2 * (pairs > 0 ? pairs : 1));
+        return p;
+    }
     p.acc = tile_hint == 1 ? 1 : tile_hint == 2 ? 2 : (M > BM ? 2 : 1);
     p.mt = (int)((M + (int64_t)BM * p.acc - 1) / ((int64_t)BM * p.acc));
     p.nt = (int)((N + BN - 1) / BN);
@@ -932,7 +1110,7 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
                         const Workspace &ws, cudaStream_t s, const DeviceInfo &dev, int64_t swiglu_f) {
     const bool swiglu = swiglu_f > 0;
     if (swiglu && N != 2 * swiglu_f) return cudaErrorInvalidValue;
-    const GemmPlan plan = gemm_plan(M, N, K, tile_hint, dev.sm_count);
+    GemmPlan plan = gemm_plan(M, N, K, tile_hint, dev.sm_count);
     if (ws.data_bytes < gemm_workspace_bytes(M, N, K, fmt, dev) || plan.ctas > kCtlGemmMaxCtas ||
         ws.zeroed_bytes < kCtlRegionBytes)
         return cudaErrorInvalidValue;
@@ -960,7 +1138,7 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
     if (fmt == 2 || fmt == 4) {
         const cuuint64_t wdims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
         const cuuint64_t wstrides[1] = {(cuuint64_t)(K / 4)};
-        const cuuint32_t wbox[2] = {(cuuint32_t)(BK / 4), (cuuint32_t)(swiglu ? BN / 2 : BN)};
+        const cuuint32_t wbox[2] = {(cuuint32_t)(BK / 4), (cuuint32_t)(swiglu || plan.pair ? BN / 2 : BN)};
         if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), wdims, wstrides, wbox,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -969,21 +1147,59 @@ cudaError_t launch_gemm(const uint16_t *x, const uint8_t *packed, const uint16_t
     auto go = [&](auto kern, int smem) -> cudaError_t {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        kern<<<plan.ctas, kThreads, smem, s>>>(map, wmap, packed, scales, y, partials, x, xr, nblocks, ctl, limit,
-                                               skew, (int)M, (int)N, (int)K, plan.mt, (int)swiglu_f);
-        return cudaGetLastError();
+        if (!plan.pair) {
+            kern<<<plan.ctas, kThreads, smem, s>>>(map, wmap, packed, scales, y, partials, x, xr, nblocks, ctl, limit,
+                                                   skew, (int)M, (int)N, (int)K, plan.mt, (int)swiglu_f);
+            return cudaGetLastError();
+        }
+        // clusters of two; only as many pairs as fit at once (the rotation phase's grid
+        // barrier and the hand-over of split tiles wait on every CTA of the grid)
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)plan.ctas);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = (size_t)smem;
+        cfg.stream = s;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+        if (e != cudaSuccess) return e;
+        if (clusters < 1) return cudaErrorInvalidConfiguration;
+        if (plan.ctas > 2 * clusters) cfg.gridDim = dim3((unsigned)(2 * clusters));
+        return cudaLaunchKernelEx(&cfg, kern, map, wmap, packed, scales, y, partials, x, xr, nblocks, ctl, limit, skew,
+                                  (int)M, (int)N, (int)K, plan.mt, (int)swiglu_f);
     };
-    auto pick = [&](auto k1, auto k2) { return plan.acc == 2 ? go(k2, Cfg<2>::kSmemBytes) : go(k1, Cfg<1>::kSmemBytes); };
-    if (swiglu) {
-        if (fmt == 1) return pick(gemm_tcgen05_kernel<1, 1, true>, gemm_tcgen05_kernel<1, 2, true>);
-        if (fmt == 3) return pick(gemm_tcgen05_kernel<3, 1, true>, gemm_tcgen05_kernel<3, 2, true>);
-        if (fmt == 4) return pick(gemm_tcgen05_kernel<4, 1, true>, gemm_tcgen05_kernel<4, 2, true>);
-        return pick(gemm_tcgen05_kernel<2, 1, true>, gemm_tcgen05_kernel<2, 2, true>);
+    auto pick = [&](auto k1, auto k2) {
+        if (plan.pair) return plan.acc == 2 ? go(k2, Cfg<2, true>::kSmemBytes) : go(k1, Cfg<1, true>::kSmemBytes);
+        return plan.acc == 2 ? go(k2, Cfg<2>::kSmemBytes) : go(k1, Cfg<1>::kSmemBytes);
+    };
+    if (plan.pair) {
+        if (swiglu) {
+            if (fmt == 1) return pick(gemm_tcgen05_kernel<1, 1, true, true>, gemm_tcgen05_kernel<1, 2, true, true>);
+            if (fmt == 3) return pick(gemm_tcgen05_kernel<3, 1, true, true>, gemm_tcgen05_kernel<3, 2, true, true>);
+            if (fmt == 4) return pick(gemm_tcgen05_kernel<4, 1, true, true>, gemm_tcgen05_kernel<4, 2, true, true>);
+            return pick(gemm_tcgen05_kernel<2, 1, true, true>, gemm_tcgen05_kernel<2, 2, true, true>);
+        }
+        if (fmt == 1) return pick(gemm_tcgen05_kernel<1, 1, false, true>, gemm_tcgen05_kernel<1, 2, false, true>);
+        if (fmt == 3) return pick(gemm_tcgen05_kernel<3, 1, false, true>, gemm_tcgen05_kernel<3, 2, false, true>);
+        if (fmt == 4) return pick(gemm_tcgen05_kernel<4, 1, false, true>, gemm_tcgen05_kernel<4, 2, false, true>);
+        return pick(gemm_tcgen05_kernel<2, 1, false, true>, gemm_tcgen05_kernel<2, 2, false, true>);
     }
-    if (fmt == 1) return pick(gemm_tcgen05_kernel<1, 1, false>, gemm_tcgen05_kernel<1, 2, false>);
-    if (fmt == 3) return pick(gemm_tcgen05_kernel<3, 1, false>, gemm_tcgen05_kernel<3, 2, false>);
-    if (fmt == 4) return pick(gemm_tcgen05_kernel<4, 1, false>, gemm_tcgen05_kernel<4, 2, false>);
-    return pick(gemm_tcgen05_kernel<2, 1, false>, gemm_tcgen05_kernel<2, 2, false>);
+    if (swiglu) {
+        if (fmt == 1) return pick(gemm_tcgen05_kernel<1, 1, true, false>, gemm_tcgen05_kernel<1, 2, true, false>);
+        if (fmt == 3) return pick(gemm_tcgen05_kernel<3, 1, true, false>, gemm_tcgen05_kernel<3, 2, true, false>);
+        if (fmt == 4) return pick(gemm_tcgen05_kernel<4, 1, true, false>, gemm_tcgen05_kernel<4, 2, true, false>);
+        return pick(gemm_tcgen05_kernel<2, 1, true, false>, gemm_tcgen05_kernel<2, 2, true, false>);
+    }
+    if (fmt == 1) return pick(gemm_tcgen05_kernel<1, 1, false, false>, gemm_tcgen05_kernel<1, 2, false, false>);
+    if (fmt == 3) return pick(gemm_tcgen05_kernel<3, 1, false, false>, gemm_tcgen05_kernel<3, 2, false, false>);
+    if (fmt == 4) return pick(gemm_tcgen05_kernel<4, 1, false, false>, gemm_tcgen05_kernel<4, 2, false, false>);
+    return pick(gemm_tcgen05_kernel<2, 1, false, false>, gemm_tcgen05_kernel<2, 2, false, false>);
 }
 
 }  // namespace bonsai

@@ -358,9 +358,10 @@ GEMM_SMALL = [(1, 64, 128), (17, 256, 128), (130, 300, 384), (256, 512, 1024), (
 
 @pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1, G64])
 @pytest.mark.parametrize("M,N,K", GEMM_SMALL)
-@pytest.mark.parametrize("tile", [1, 2])
+@pytest.mark.parametrize("tile", [1, 2, 3])
 def test_gemm_small(bz, fmt, M, N, K, tile):
-    """tile 1: one 128-row TMEM accumulator per CTA; tile 2: two (256 rows)."""
+    """tile 1: one 128-row TMEM accumulator per CTA; tile 2: two (256 rows); tile 3: CTA
+    pairs sharing each MMA (cta_group::2), 256 or 512 rows per tile."""
     p = Problem(M, N, K, fmt, seed=M + N + K)
     got = _run(bz, p, bz.BONSAI_ALGO_GEMM, tile)
     assert np.all(np.isfinite(got))
@@ -369,19 +370,18 @@ def test_gemm_small(bz, fmt, M, N, K, tile):
 
 
 @pytest.mark.parametrize("fmt", [PTQ1, PQ2, Q1, G64])
-def test_gemm_split_tiles_repeatable(bz, fmt):
-    """Split tiles hand their partial sums over through flags that the owner clears:
-    the same call twice, and after a differently split shape, gives the same bits."""
-    import torch
+@pytest.mark.parametrize("tile", [0, 3])
+def test_gemm_split_tiles_repeatable(bz, fmt, tile):
+    """Split tiles hand their partial sums over through flags that carry the call's
+    epoch: the same call twice, and after a differently split shape, gives the same bits."""
     p = Problem(2048, 8192, 384, fmt, seed=11)
     q = Problem(300, 1000, 640, fmt, seed=12)
-    a = _run(bz, p, bz.BONSAI_ALGO_GEMM)
-    _run(bz, q, bz.BONSAI_ALGO_GEMM)
-    b = _run(bz, p, bz.BONSAI_ALGO_GEMM)
+    a = _run(bz, p, bz.BONSAI_ALGO_GEMM, tile)
+    _run(bz, q, bz.BONSAI_ALGO_GEMM, tile)
+    b = _run(bz, p, bz.BONSAI_ALGO_GEMM, tile)
     assert np.array_equal(a, b)
     ok, rel, mx = oracle.compare(a, p.oracle_y())
     assert ok, (rel, mx)
-    del torch
 
 
 def _sampled_reference(fmt, M, N, K, seed, ms, ns):

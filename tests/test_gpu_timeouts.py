@@ -85,14 +85,21 @@ def test_status_is_clear_after_normal_calls(bz):
     assert bz.bonsai_device_status() == 0
 
 
-def gemm_split_tiles(M, N, K, sms):
+def gemm_split_tiles(M, N, K, sms, pair=False):
     """Output tiles of the prefill GEMM that are split between CTAs, from its work split:
     tiles of 128 acc rows x 256 columns (row tile fastest), acc = 2 when M > 128; C = min(SMs,
     ceil(units / 4)) CTAs; W = T / C - 1 whole-tile waves when T >= 2C; the remaining tiles'
-    64-wide K stages split evenly, CTA b taking units [Ur b / C, Ur (b + 1) / C)."""
-    acc = 2 if M > 128 else 1
-    mt, nt, nk = -(-M // (128 * acc)), -(-N // 256), K // 64
-    C = max(1, min(sms, -(-(mt * nt * nk) // 4)))
+    64-wide K stages split evenly, CTA b taking units [Ur b / C, Ur (b + 1) / C).  CTA pairs
+    (pair=True): tiles of 256 acc rows, acc = 2 when M > 256, and C = min(SMs / 2,
+    ceil(units / 4)) pairs in place of CTAs.  Returns (tm, tn, rows of a tile)."""
+    if pair:
+        acc = 2 if M > 256 else 1
+        rows = 256 * acc
+    else:
+        acc = 2 if M > 128 else 1
+        rows = 128 * acc
+    mt, nt, nk = -(-M // rows), -(-N // 256), K // 64
+    C = max(1, min(sms // 2 if pair else sms, -(-(mt * nt * nk) // 4)))
     T = mt * nt
     W = T // C - 1 if T // C >= 2 else 0
     Ur = (T - W * C) * nk
@@ -101,22 +108,25 @@ def gemm_split_tiles(M, N, K, sms):
         u = Ur * b // C
         if u % nk != 0:
             split.add(W * C + u // nk)
-    return [(s % mt, s // mt, acc) for s in sorted(split)]
+    return [(s % mt, s // mt, rows) for s in sorted(split)]
 
 
 @pytest.mark.parametrize("M,N,K", [(300, 1000, 640), (600, 2000, 1152)])
-def test_forced_gemm_flag_timeouts_nan_status_and_recovery(bz, M, N, K):
+@pytest.mark.parametrize("tile", [0, 3])
+def test_forced_gemm_flag_timeouts_nan_status_and_recovery(bz, M, N, K, tile):
+    """tile 0: the automatic tiles; tile 3: CTA pairs, where both CTAs of an owner pair
+    wait for their halves of the later pieces."""
     import torch
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     p = Problem(M, N, K, PQ2, seed=M + N)
     x, packed, scales = p.device()
     ref = p.oracle_y()
-    split = gemm_split_tiles(M, N, K, sms)
+    split = gemm_split_tiles(M, N, K, sms, pair=tile == 3)
     assert len(split) > 0
 
     def run():
         y = torch.full((M, N), 7.0, dtype=torch.float16, device="cuda")
-        bz.bonsai_ternary_linear_algo(x, packed, scales, y, M, N, K, PQ2, bz.BONSAI_ALGO_GEMM)
+        bz.bonsai_ternary_linear_algo(x, packed, scales, y, M, N, K, PQ2, bz.BONSAI_ALGO_GEMM, tile)
         torch.cuda.synchronize()
         return to_numpy_f16(y)
 
@@ -129,8 +139,8 @@ def test_forced_gemm_flag_timeouts_nan_status_and_recovery(bz, M, N, K):
     status = bz.bonsai_device_status(clear=True)
     assert status & bz.BONSAI_DEVICE_GEMM_TIMEOUT
     bad = np.zeros((M, N), dtype=bool)
-    for tm, tn, acc in split:
-        bad[128 * acc * tm:128 * acc * (tm + 1), 256 * tn:256 * (tn + 1)] = True
+    for tm, tn, rows in split:
+        bad[rows * tm:rows * (tm + 1), 256 * tn:256 * (tn + 1)] = True
     assert np.all(np.isnan(got[bad]))
     assert np.all(np.isfinite(got[~bad]))
     ok, rel, mx = oracle.compare(got[~bad], ref[~bad])
