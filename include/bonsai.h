@@ -105,8 +105,9 @@ typedef enum {
     BONSAI_ALGO_GEMV = 2,    /* batch-1 lookup-table GEMV with split-K; M == 1 only       */
     BONSAI_ALGO_SKINNY = 3,  /* register-dequant tensor-core kernel; 1 <= M <= 16         */
     BONSAI_ALGO_GEMM = 4,    /* tcgen05/TMEM prefill GEMM on FP16 tiles; any M            */
-    BONSAI_ALGO_IMMA = 5     /* batch-1 GEMV on the integer tensor cores; M == 1, PQ2_0
-                                and PQ2_0 g64                                             */
+    BONSAI_ALGO_IMMA = 5     /* GEMV on the integer tensor cores, PQ2_0 and PQ2_0 g64:
+                                M == 1 (K <= 24576), M == 2 (K <= 12288), and for
+                                PQ2_0 M == 3 (K <= 6144)                                  */
 } bonsai_algo;
 
 /* Library version, (major << 16) | (minor << 8) | patch. */

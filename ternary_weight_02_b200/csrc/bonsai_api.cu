@@ -146,7 +146,7 @@ int cuda_status(cudaError_t e) {
 // resolve AUTO again with the device once it is known.
 int resolve_algo(int algo, int64_t M, int64_t N, int64_t K, int fmt, const DeviceInfo *dev = nullptr) {
     if (algo == BONSAI_ALGO_AUTO) {
-        if (M == 1 && gemv_imma_supported(M, N, K, fmt) && (dev == nullptr || gemv_imma_grid_fits(N, K, *dev)))
+        if (M <= 3 && gemv_imma_supported(M, N, K, fmt) && (dev == nullptr || gemv_imma_grid_fits(N, K, *dev)))
             return BONSAI_ALGO_IMMA;
         if (M == 1 && gemv_supported(M, N, K, fmt)) return BONSAI_ALGO_GEMV;
         if (M <= 16 && skinny_supported(M, N, K, fmt)) return BONSAI_ALGO_SKINNY;
@@ -171,7 +171,7 @@ cudaError_t run_linear(int chosen, const uint16_t *x, const uint8_t *packed, con
         case BONSAI_ALGO_GEMV: return launch_gemv(x, packed, scales, y, N, K, fmt, split_k, ws, s, info);
         case BONSAI_ALGO_SKINNY: return launch_skinny(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, info);
         case BONSAI_ALGO_GEMM: return launch_gemm(x, packed, scales, y, M, N, K, fmt, split_k, ws, s, info);
-        case BONSAI_ALGO_IMMA: return launch_gemv_imma(x, packed, scales, y, N, K, fmt, ws, s, info);
+        case BONSAI_ALGO_IMMA: return launch_gemv_imma(x, packed, scales, y, M, N, K, fmt, ws, s, info);
         default: return launch_linear_simple(x, packed, scales, y, M, N, K, fmt, ws, s, info);
     }
 }
@@ -328,7 +328,7 @@ int bonsai_ternary_linear_algo(const uint16_t *x, const uint8_t *packed, const u
     if (chosen == BONSAI_ALGO_IMMA && !gemv_imma_grid_fits(N, K, st->info)) return BONSAI_ERR_ALGO;
     Workspace ws;
     rc = ensure_workspace(*st, workspace_for(chosen, M, N, K, fmt, split_k, st->info),
-                          chosen == BONSAI_ALGO_IMMA ? gemv_imma_zeroed_bytes(N, K) : 0, &ws);
+                          chosen == BONSAI_ALGO_IMMA ? gemv_imma_zeroed_bytes(M, N, K) : 0, &ws);
     if (rc != BONSAI_OK) return rc;
     return cuda_status(run_linear(chosen, x, packed, scales, y, M, N, K, fmt, split_k, ws,
                                   static_cast<cudaStream_t>(stream), st->info));
@@ -375,10 +375,10 @@ int bonsai_ternary_linear_swiglu(const uint16_t *x, const uint8_t *packed, const
     chosen = resolve_algo(BONSAI_ALGO_AUTO, M, N, K, fmt, &st->info);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Workspace ws;
-    if (chosen == BONSAI_ALGO_IMMA) {  // fused into the GEMV's epilogue
-        rc = ensure_workspace(*st, 0, gemv_imma_zeroed_bytes(N, K), &ws);
+    if (chosen == BONSAI_ALGO_IMMA && M == 1) {  // fused into the GEMV's epilogue
+        rc = ensure_workspace(*st, 0, gemv_imma_zeroed_bytes(M, N, K), &ws);
         if (rc != BONSAI_OK) return rc;
-        return cuda_status(launch_gemv_imma(x, packed, scales, h, N, K, fmt, ws, s, st->info, F));
+        return cuda_status(launch_gemv_imma(x, packed, scales, h, M, N, K, fmt, ws, s, st->info, F));
     }
     if (chosen == BONSAI_ALGO_GEMM) {  // fused into the GEMM's epilogue
         rc = ensure_workspace(*st, workspace_for(chosen, M, N, K, fmt, 0, st->info), 0, &ws);
@@ -388,7 +388,7 @@ int bonsai_ternary_linear_swiglu(const uint16_t *x, const uint8_t *packed, const
     // otherwise: the linear layer into the tail of the workspace, then the SwiGLU kernel
     const size_t need = (workspace_for(chosen, M, N, K, fmt, 0, st->info) + 255) / 256 * 256;
     rc = ensure_workspace(*st, need + (size_t)M * (size_t)N * 2,
-                          chosen == BONSAI_ALGO_IMMA ? gemv_imma_zeroed_bytes(N, K) : 0, &ws);
+                          chosen == BONSAI_ALGO_IMMA ? gemv_imma_zeroed_bytes(M, N, K) : 0, &ws);
     if (rc != BONSAI_OK) return rc;
     uint16_t *y = reinterpret_cast<uint16_t *>(ws.data + need);
     Workspace inner = ws;
@@ -440,10 +440,11 @@ int bonsai_reserve(int64_t M, int64_t N, int64_t K) {
             v = gemv_workspace_bytes(N, K, fmt, 0, st->info);
             need = v > need ? v : need;
         }
-        if (M <= 1 && gemv_imma_supported(1, N, K, fmt)) {
-            v = gemv_imma_zeroed_bytes(N, K);
-            zneed = v > zneed ? v : zneed;
-        }
+        for (int64_t m = 1; m <= 3 && m <= (M > 1 ? M : 1); m++)
+            if (gemv_imma_supported(m, N, K, fmt)) {
+                v = gemv_imma_zeroed_bytes(m, N, K);
+                zneed = v > zneed ? v : zneed;
+            }
         if (skinny_supported(M < 16 ? M : 16, N, K, fmt)) {
             v = skinny_workspace_bytes(M < 16 ? M : 16, N, K, fmt, 0, st->info);
             need = v > need ? v : need;

@@ -1,5 +1,6 @@
-// gemv_imma.cu -- batch-1 (M == 1) ternary GEMV for PQ2_0 (one FP16 scale per 128 or per
-// 64 weights) on the integer tensor cores, with the block Hadamard rotation of x fused in.
+// gemv_imma.cu -- batch-1 and batch-2 (M <= 2) ternary GEMV for PQ2_0 (one FP16 scale per
+// 128 or per 64 weights) on the integer tensor cores, with the block Hadamard rotation of
+// x fused in.
 //
 // Operation: y[n] = sum_g s[n][g] * sum_j t[n][128g+j] * x'[128g+j], x' = blockdiag(Hn) x;
 // with 64-weight scale groups each 128-group's sum splits into two halves, each with its
@@ -50,6 +51,14 @@
 //   the later pieces in K order (deterministic).  The epoch is a call number kept in
 //   the workspace's control words, so stored pairs never need clearing and a late pair
 //   can never be taken for a later call's.
+// * Several tokens (kM = 2 or 3; g64: 2).  The batch-1 layout spends an MMA's eight
+//   columns on four groups x (high, low byte), and the loop is bound by the rate of
+//   mma.sync, so more tokens there would mean more MMAs.  Instead one MMA covers one
+//   group's 32 weights of one code slot (each lane of a quad 8 bytes of the group, the
+//   same bytes for the four slots), and its columns carry (token, high/low byte); with
+//   64-weight scales (half, token, high/low byte), a column meeting only its half's
+//   weights.  The MMAs per item stay 32, the masks 128.  Each token has its own x~
+//   fragments, sums and exponents, so shared memory limits K (max_k).
 // * Every wait is bounded.  A warp whose mbarrier wait gives up stops refilling, turns
 //   its results into NaN (keeping the partial-sum protocol intact) and, before the
 //   CTA exits, waits (again bounded) for the copies it had started; an owner whose wait
@@ -77,29 +86,33 @@ constexpr int kStages = 2;
 constexpr int kFirstIssue = 1;
 constexpr int kMaxCtaItems = 96;                        // slot buffer: 96 x 32 floats
 constexpr int kMaxCtaTiles = kMaxCtaItems + 2;          // row tiles one CTA's items touch
-constexpr int64_t kMaxK = 24576;  // the layout below then fits the 227 KB a CTA may use
+constexpr int64_t kMaxK = 24576;   // the layout below then fits the 227 KB a CTA may use
+constexpr int64_t kMaxK2 = 12288;  // the same with two tokens' x~
+constexpr int64_t kMaxK3 = 6144;   // three tokens
+__host__ __device__ constexpr int64_t max_k(int M) { return M == 1 ? kMaxK : M == 2 ? kMaxK2 : kMaxK3; }
 constexpr uint32_t kCodeMask = 0x03030303u;
 
 // Shared memory, from a 1024-byte aligned base (each 4 KB weight buffer stays 1024-byte
 // aligned, as the 128-byte swizzle of its TMA box requires):
 // [weight rings: kConsumers x kStages x 4096][scale rings: kConsumers x kStages x 512]
 // [x~ fragments G4 x 288][(64 sum x~, 2^-e / 64) x G4][64 sum of the first 64 x~ x G4]
-// [slots kMaxCtaItems x 128][256 zero bytes][full barriers]
+// [slots kMaxCtaItems x 128][row-tile counts][256 zero bytes][full barriers]
 struct Layout {
     int sring, xfrag, sxf, sxl, slots, tcnt, zero, full, total;
 };
 
 // Alignment: the weight buffers 1024 bytes (swizzled TMA destinations), the fragment,
 // slot and zero areas 16 bytes (128-bit loads), the barriers 8 bytes.
-__host__ __device__ inline Layout make_layout(int K) {
+// (M tokens: M copies of the x~ areas, token-major, and M floats per item row in the slots.)
+__host__ __device__ inline Layout make_layout(int K, int M) {
     Layout L;
     const int G4 = ((K + kItemK - 1) / kItemK) * 4;
     L.sring = kConsumers * kStages * kItemBytes;
     L.xfrag = L.sring + kConsumers * kStages * kScaleRingBytes;
-    L.sxf = L.xfrag + G4 * kXGroupBytes;
-    L.sxl = L.sxf + G4 * 8;
-    L.slots = L.sxl + ((G4 * 4 + 15) & ~15);
-    L.tcnt = L.slots + kMaxCtaItems * kItemRows * 4;
+    L.sxf = L.xfrag + M * G4 * kXGroupBytes;
+    L.sxl = L.sxf + M * G4 * 8;
+    L.slots = L.sxl + ((M * G4 * 4 + 15) & ~15);
+    L.tcnt = L.slots + kMaxCtaItems * kItemRows * 4 * M;
     L.zero = (L.tcnt + kMaxCtaTiles * 4 + 15) & ~15;  // 128-bit loads read the zero bytes
     L.full = L.zero + 256;
     L.total = L.full + kConsumers * kStages * 8 + 16 + 1024;  // + the epoch word, room to align the base
@@ -142,12 +155,13 @@ __device__ __forceinline__ void load_x8(const uint16_t *__restrict__ x, int g, i
 // 8-byte subslot s: element k = 32*s + 16*hb + 4*i + j is byte (8*(j & 1) + 4*hb + i) of
 // 16-byte chunk 2*s + (j >> 1) in the 144-byte half-block (2g + p).  The 16 bytes of
 // padding per half-block put the eight lanes that load one chunk of four consecutive
-// groups on distinct shared-memory banks.  Lane l = 2*s + hb writes whole words.
+// groups on distinct shared-memory banks.  Lane l = 2*s + hb writes whole words.  With
+// several tokens the half-blocks of token m sit at 288 m within a group's gstride bytes.
 // Rotates and quantises group g (its x in r0, r1 of the group's 8 lanes) into the
 // fragment area, (64 * sum x~, 2^-e / 64) into sxf[g] and 64 * the sum of its first 64
 // x~ (lanes 0..3 of the group) into sxl[g].
-__device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag, int2 *sxf, int *sxl, int g,
-                                             int lane) {
+__device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag, int gstride, int2 *sxf, int *sxl,
+                                             int g, int lane) {
     const int l = lane & 7;
     const unsigned int gmask = 0xffu << (lane & 24);
     float v[16];
@@ -212,7 +226,7 @@ __device__ __forceinline__ void build_group8(uint4 r0, uint4 r1, uint8_t *xfrag,
     sum += __shfl_xor_sync(gmask, sum, 4);
     sum -= 128 * kGroup;  // the 128 added to each of the group's q
     // lane l = 2s + hb: chunk 2s + (j >> 1), byte 8 (j & 1) + 4 hb + i (element 16l + 4i + j)
-    uint8_t *dst = xfrag + g * kXGroupBytes + (l >> 1) * 32 + (l & 1) * 4;
+    uint8_t *dst = xfrag + g * gstride + (l >> 1) * 32 + (l & 1) * 4;
 #pragma unroll
     for (int j = 0; j < 4; j++) {
         const uint32_t a0 = (uint32_t)qa[j], a1 = (uint32_t)qa[4 + j];
@@ -279,7 +293,10 @@ __device__ __forceinline__ float wait_pairs(const uint64_t *p, int lane, uint32_
 // sticky status bits.  wait_limit and epoch_skew are the polls of a wait for a later piece
 // and an offset added to the epoch it waits for: kSpinLimit and 0, except under the test
 // hook that makes those waits give up.
-template <bool kAsyncScales, bool kSwiglu, bool kG64>
+//
+// kM: tokens (1 to 3; g64 1 or 2); x is kM x K and y kM x N, row-major.  (kSwiglu needs
+// kM = 1.)
+template <bool kAsyncScales, bool kSwiglu, bool kG64, int kM>
 __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const __grid_constant__ CUtensorMap wmap, const uint16_t *__restrict__ x, const uint16_t *__restrict__ scales,
     uint16_t *__restrict__ y, uint64_t *__restrict__ partials, unsigned int *__restrict__ ctl, int N, int K, int F,
@@ -288,7 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     uint8_t *smem = smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
-    const Layout L = make_layout(K);
+    static_assert(kM == 1 || (kM <= 3 && !kSwiglu && (!kG64 || kM == 2)),
+                  "several tokens: up to 3 (g64: 2), without the SwiGLU epilogue");
+    const Layout L = make_layout(K, kM);
     const int G = K / kGroup;
     const int GS = kG64 ? 2 * G : G;  // scales per row
     const int KC = (K + kItemK - 1) / kItemK;
@@ -373,32 +392,37 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     unsigned long long ctr = 0;
     if (tid == 0) ctr = atomicAdd(reinterpret_cast<unsigned long long *>(ctl + kCtlCalls), 1ull);
     // x -> x~ fragments, four groups (a quad) per warp and round: all of this warp's x
-    // first.  Every CTA reads all of x at the same moment, so each starts at a different
-    // quad: the simultaneous requests spread over the lines of x instead of piling up.
-    {
-        constexpr int kRounds = (int)((kMaxK / kItemK) * 4 / 4 + kConsumers - 1) / kConsumers;
+    // first (token by token).  Every CTA reads all of x at the same moment, so each starts
+    // at a different quad: the simultaneous requests spread over the lines of x instead of
+    // piling up.
+#pragma unroll
+    for (int m = 0; m < kM; m++) {
+        constexpr int kRounds = (int)((max_k(kM) / kItemK) * 4 / 4 + kConsumers - 1) / kConsumers;
         const int nquads = G4 / 4;
         const int rot = (int)(blockIdx.x % (unsigned)nquads);
+        const uint16_t *xm = x + (int64_t)m * K;
         uint4 xr[kRounds][2];
 #pragma unroll
         for (int r = 0; r < kRounds; r++) {
             const int quad = warp + r * kConsumers;
             int pq = quad + rot;
             if (pq >= nquads) pq -= nquads;
-            if (quad < nquads) load_x8(x, pq * 4 + (lane >> 3), G, lane & 7, xr[r][0], xr[r][1]);
+            if (quad < nquads) load_x8(xm, pq * 4 + (lane >> 3), G, lane & 7, xr[r][0], xr[r][1]);
         }
-        for (int q = 0; q < kFirstIssue; q++) issue(q);
+        if (m == 0)
+            for (int q = 0; q < kFirstIssue; q++) issue(q);
 #pragma unroll
         for (int r = 0; r < kRounds; r++) {
             const int quad = warp + r * kConsumers;
             int pq = quad + rot;
             if (pq >= nquads) pq -= nquads;
             if (quad < nquads)  // whole warps
-                build_group8(xr[r][0], xr[r][1], xf, reinterpret_cast<int2 *>(smem + L.sxf),
-                             reinterpret_cast<int *>(smem + L.sxl), pq * 4 + (lane >> 3), lane);
+                build_group8(xr[r][0], xr[r][1], xf + m * kXGroupBytes, kM * kXGroupBytes,
+                             reinterpret_cast<int2 *>(smem + L.sxf) + m * G4,
+                             reinterpret_cast<int *>(smem + L.sxl) + m * G4, pq * 4 + (lane >> 3), lane);
         }
-        for (int q = kFirstIssue; q < kStages; q++) issue(q);
     }
+    for (int q = kFirstIssue; q < kStages; q++) issue(q);
     if (tid == 0) {
         const uint32_t calls = (uint32_t)(ctr >> 32);
         *epoch_s = calls + 1u;  // the count skips 0xffffffff, so the epoch is never 0
@@ -436,31 +460,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const int rt_first = c0 / KC;
     // One warp per tile, one lane per row: add the CTA's items of tile rt ([a, b)) in K
     // order, then write y (whole tile), store the piece (a later piece) or collect the
-    // later pieces and write y (owned).
+    // later pieces and write y (owned); token by token.  Slots and pairs hold kM values
+    // per item row, token-major within an item.
     auto finish_tile = [&](int rt, int a, int b) {
         const int tile_first = rt * KC, tile_end = tile_first + KC;
-        float sum = 0.f;
-        for (int i = a; i < b; i++) sum += slots[(i - c0) * kItemRows + lane];
-        if (a > tile_first) {
-            st_pair(partials + (int64_t)a * kItemRows + lane, sum, epoch);
-            return;
+#pragma unroll
+        for (int m = 0; m < kM; m++) {
+            float sum = 0.f;
+            for (int i = a; i < b; i++) sum += slots[((i - c0) * kM + m) * kItemRows + lane];
+            if (a > tile_first) {
+                st_pair(partials + ((int64_t)a * kM + m) * kItemRows + lane, sum, epoch);
+                continue;
+            }
+            int s = b, c2 = (int)blockIdx.x + 1;
+            while (s < tile_end) {
+                int e2 = (int)((int64_t)I * (c2 + 1) / C);  // the piece of CTA c2 is [s, e2)
+                e2 = e2 < tile_end ? e2 : tile_end;
+                sum += wait_pairs(partials + ((int64_t)s * kM + m) * kItemRows, lane, epoch + epoch_skew, wait_limit,
+                                  status);
+                s = e2;
+                c2++;
+            }
+            if (kSwiglu) {  // h = silu(gate) * up: lanes 0..15 hold gate rows, 16..31 the up rows
+                const float up = __shfl_down_sync(0xffffffffu, sum, 16);
+                const int f = 16 * rt + lane;
+                if (lane < 16 && f < F) y[f] = float_to_half_bits(sum / (1.f + expf(-sum)) * up);
+                continue;
+            }
+            const int row = rt * kItemRows + lane;
+            if (row < N) y[(int64_t)m * N + row] = float_to_half_bits(sum);
         }
-        int s = b, c2 = (int)blockIdx.x + 1;
-        while (s < tile_end) {
-            int e2 = (int)((int64_t)I * (c2 + 1) / C);  // the piece of CTA c2 is [s, e2)
-            e2 = e2 < tile_end ? e2 : tile_end;
-            sum += wait_pairs(partials + (int64_t)s * kItemRows, lane, epoch + epoch_skew, wait_limit, status);
-            s = e2;
-            c2++;
-        }
-        if (kSwiglu) {  // h = silu(gate) * up: lanes 0..15 hold gate rows, 16..31 the up rows
-            const float up = __shfl_down_sync(0xffffffffu, sum, 16);
-            const int f = 16 * rt + lane;
-            if (lane < 16 && f < F) y[f] = float_to_half_bits(sum / (1.f + expf(-sum)) * up);
-            return;
-        }
-        const int row = rt * kItemRows + lane;
-        if (row < N) y[row] = float_to_half_bits(sum);
     };
 
     auto process = [&](int q) {
@@ -474,26 +503,60 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
         }
         const uint8_t *sb = wring + st * kItemBytes;
         uint4 raw[2][2][2];  // [t][h][16-byte half of the lane's 32 bytes]
+        // (several tokens) [t][h][group]: bytes 8 tig .. 8 tig + 7 of each of the item's
+        // four groups of row 16t + 8h + gid
+        uint2 rawg[2][2][4];
+        if constexpr (kM == 1) {
 #pragma unroll
-        for (int t = 0; t < 2; t++)
+            for (int t = 0; t < 2; t++)
 #pragma unroll
-            for (int h = 0; h < 2; h++) {
-                raw[t][h][0] = *reinterpret_cast<const uint4 *>(sb + loff0 + 2048 * t + 1024 * h);
-                raw[t][h][1] = *reinterpret_cast<const uint4 *>(sb + loff1 + 2048 * t + 1024 * h);
-            }
+                for (int h = 0; h < 2; h++) {
+                    raw[t][h][0] = *reinterpret_cast<const uint4 *>(sb + loff0 + 2048 * t + 1024 * h);
+                    raw[t][h][1] = *reinterpret_cast<const uint4 *>(sb + loff1 + 2048 * t + 1024 * h);
+                }
+        } else {
+#pragma unroll
+            for (int t = 0; t < 2; t++)
+#pragma unroll
+                for (int h = 0; h < 2; h++)
+#pragma unroll
+                    for (int g = 0; g < 4; g++)  // logical chunk 2g + tig / 2, swizzled by the row
+                        rawg[t][h][g] = *reinterpret_cast<const uint2 *>(
+                            sb + 2048 * t + 1024 * h + gid * kItemRowBytes + (((2 * g + (tig >> 1)) ^ gid) << 4) +
+                            (tig & 1) * 8);
+        }
         const int g0 = kc * 4;
         // (t, h) = (e >> 1, e & 1): scale of row 16t + 8h + gid, group g0 + tig (g64: the
         // group's two half scales, first half in the low 16 bits)
         uint32_t sc[4];
+        // (several tokens) [t][h]: the four (g64: eight) scales of row 16t + 8h + gid in
+        // this item, two to a word, the first in the low half
+        uint32_t scw[2][2][kG64 ? 4 : 2];
         if (kAsyncScales) {
             cp_async_wait<kStages - 1>();  // this item's scales have landed (own copies)
             __syncwarp();                  // ... and every lane's
-            const uint8_t *sp = sring + st * kScaleRingBytes + gid * 16 + tig * (kG64 ? 4 : 2);
+            if constexpr (kM == 1) {
+                const uint8_t *sp = sring + st * kScaleRingBytes + gid * 16 + tig * (kG64 ? 4 : 2);
 #pragma unroll
-            for (int e = 0; e < 4; e++)
-                sc[e] = kG64 ? *reinterpret_cast<const uint32_t *>(sp + e * 128)
-                             : (uint32_t)*reinterpret_cast<const uint16_t *>(sp + e * 128);
-        } else {
+                for (int e = 0; e < 4; e++)
+                    sc[e] = kG64 ? *reinterpret_cast<const uint32_t *>(sp + e * 128)
+                                 : (uint32_t)*reinterpret_cast<const uint16_t *>(sp + e * 128);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 2; t++)
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const uint8_t *sp = sring + st * kScaleRingBytes + (16 * t + 8 * h + gid) * 16;
+                        if constexpr (kG64) {
+                            const uint4 u = *reinterpret_cast<const uint4 *>(sp);
+                            scw[t][h][0] = u.x, scw[t][h][1] = u.y, scw[t][h][2] = u.z, scw[t][h][3] = u.w;
+                        } else {
+                            const uint2 u = *reinterpret_cast<const uint2 *>(sp);
+                            scw[t][h][0] = u.x, scw[t][h][1] = u.y;
+                        }
+                    }
+            }
+        } else if constexpr (kM == 1) {
             const int g = g0 + tig;
 #pragma unroll
             for (int e = 0; e < 4; e++) {
@@ -506,6 +569,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
                 else
                     sc[e] = v ? (uint32_t)__ldg(scales + (int64_t)row * GS + g) : 0u;
             }
+        } else {
+            constexpr int kPer = kG64 ? 8 : 4;  // scales of a row in one item
+#pragma unroll
+            for (int t = 0; t < 2; t++)
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    const int row = row_of(rt, 16 * t + 8 * h + gid);
+#pragma unroll
+                    for (int w = 0; w < kPer / 2; w++) {
+                        const int q0 = kPer * kc + 2 * w;  // the row's scale index
+                        const uint32_t lo = row < N && q0 < GS ? (uint32_t)__ldg(scales + (int64_t)row * GS + q0) : 0u;
+                        const uint32_t hi =
+                            row < N && q0 + 1 < GS ? (uint32_t)__ldg(scales + (int64_t)row * GS + q0 + 1) : 0u;
+                        scw[t][h][w] = lo | (hi << 16);
+                    }
+                }
         }
         __syncwarp();
         if (ok) {  // refill this buffer with the warp's item q + kStages
@@ -520,6 +599,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
         // undone once per fold (the sums come out 64 times too large, folded into 2^-e).
         // One fold per group, or (g64) one per 64-weight half: subslots 0, 1 then 2, 3.
         constexpr int kFolds = kG64 ? 2 : 1, kSubPerFold = 4 / kFolds;
+        // sum over the four groups (lanes of the quad) and leave (t, h) = (tig >> 1, tig & 1)
+        // in lane tig: keep the pair whose h is the lane's, then the t
+        auto quad_sum = [&](const float (&v)[4]) {
+            const bool b0 = tig & 1;
+            const float k0 = b0 ? v[1] : v[0], s0 = b0 ? v[0] : v[1];
+            const float k1 = b0 ? v[3] : v[2], s1 = b0 ? v[2] : v[3];
+            const float u0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 1);  // t = 0
+            const float u1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 1);  // t = 1
+            const bool b1 = tig & 2;
+            const float kk = b1 ? u1 : u0, ss = b1 ? u0 : u1;
+            return kk + __shfl_xor_sync(0xffffffffu, ss, 2);
+        };
+        if constexpr (kM == 1) {
         int d[2][4][4];
         const uint8_t *xb = xb_lane + g0 * xb_stride;
         const int2 sf = sxf[g0 + tig];  // (64 * sum x~, 2^-e / 64)
@@ -564,21 +656,68 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
             v[e] = fmaf((float)T64, half_bits_to_float(sbits) * fg, v[e]);
         }
         }
-        // sum over the four groups (lanes of the quad) and leave (t, h) = (tig >> 1, tig & 1)
-        // in lane tig: keep the pair whose h is the lane's, then the t
-        {
-            const bool b0 = tig & 1;
-            const float k0 = b0 ? v[1] : v[0], s0 = b0 ? v[0] : v[1];
-            const float k1 = b0 ? v[3] : v[2], s1 = b0 ? v[2] : v[3];
-            const float u0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 1);  // t = 0
-            const float u1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 1);  // t = 1
-            const bool b1 = tig & 2;
-            const float kk = b1 ? u1 : u0, ss = b1 ? u0 : u1;
-            v[0] = kk + __shfl_xor_sync(0xffffffffu, ss, 2);
-        }
-        float mine = v[0];
+        float mine = quad_sum(v);
         if (!ok) mine = __int_as_float(0x7fc00000);
         slots[(i - c0) * kItemRows + R] = mine;
+        } else {
+            // Several tokens: MMA (t, g, j) meets code slot j of group g0 + g of tile t with
+            // B columns (token, high/low byte) -- g64: (half, token, high/low byte), where a
+            // column meets only its half's weights (the k of lane quads 2 hf, 2 hf + 1).
+            // Lane (gid, tig) holds columns 2 tig, 2 tig + 1: token mt (g64: half ht).
+            const int mt = kG64 ? (tig & 1) : tig;
+            const int ht = kG64 ? (tig >> 1) : 0;
+            const bool valid = mt < kM;
+            const int mc = valid ? mt : 0;  // (the addresses an unused lane reads)
+            // the B column this lane supplies: column gid, for the k of lane quad tig
+            const int bm = kG64 ? ((gid >> 1) & 1) : (gid >> 1);
+            const bool bact = bm < kM && (!kG64 || (gid >> 2) == (tig >> 1));
+            const uint8_t *xbq = bact ? xf + bm * kXGroupBytes + (gid & 1) * kXHalfBytes + tig * 32 : zero;
+            const int xq_stride = bact ? kM * kXGroupBytes : 0;
+            const int2 *sxm = sxf + mc * G4;
+            const int *sxlm = reinterpret_cast<const int *>(smem + L.sxl) + mc * G4;
+            float v[2][2] = {{0.f, 0.f}, {0.f, 0.f}};  // [t][h]: row 16t + 8h + gid, token mt
+#pragma unroll
+            for (int g = 0; g < 4; g++) {
+                const uint8_t *xb = xbq + (g0 + g) * xq_stride;
+                const uint4 b01 = *reinterpret_cast<const uint4 *>(xb);       // code slots 0, 1
+                const uint4 b23 = *reinterpret_cast<const uint4 *>(xb + 16);  // code slots 2, 3
+                const int2 sf = sxm[g0 + g];  // (64 * sum x~, 2^-e / 64) of token mc
+                const float fg = __int_as_float(sf.y);
+                // 64 * the sum of x~ over the weights the lane's columns meet
+                const int sx = kG64 ? (ht == 0 ? sxlm[g0 + g] : sf.x - sxlm[g0 + g]) : sf.x;
+#pragma unroll
+                for (int t = 0; t < 2; t++) {
+                    const uint2 r0 = rawg[t][0][g], r1 = rawg[t][1][g];
+                    int d[4][4];
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const uint32_t mask = kCodeMask << (2 * j);
+                        const uint32_t bx = j == 0 ? b01.x : (j == 1 ? b01.z : (j == 2 ? b23.x : b23.z));
+                        const uint32_t by = j == 0 ? b01.y : (j == 1 ? b01.w : (j == 2 ? b23.y : b23.w));
+                        imma0(d[j], r0.x & mask, r1.x & mask, r0.y & mask, r1.y & mask, bx, by);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; h++) {
+                        const int H = ((d[0][2 * h] * 4 + d[1][2 * h]) * 4 + d[2][2 * h]) * 4 + d[3][2 * h];
+                        const int Lo =
+                            ((d[0][2 * h + 1] * 4 + d[1][2 * h + 1]) * 4 + d[2][2 * h + 1]) * 4 + d[3][2 * h + 1];
+                        const int T64 = H * 256 + Lo - sx;
+                        const int q = kG64 ? 2 * g + ht : g;  // the scale's index in the row's item
+                        const uint16_t sbits = (uint16_t)(scw[t][h][q >> 1] >> (16 * (q & 1)));
+                        v[t][h] = fmaf((float)T64, half_bits_to_float(sbits) * fg, v[t][h]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < 2; t++)
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    if (kG64) v[t][h] += __shfl_xor_sync(0xffffffffu, v[t][h], 2);  // the other half
+                    if (valid && ht == 0)
+                        slots[((i - c0) * kM + mt) * kItemRows + 16 * t + 8 * h + gid] =
+                            ok ? v[t][h] : __int_as_float(0x7fc00000);
+                }
+        }
         // the warp that completes the CTA's part of a row tile finalises it
         __syncwarp();
         int done = 0;
@@ -633,9 +772,21 @@ static_assert(kConsumers * kStages * (kItemBytes + kScaleRingBytes) + (kMaxK / k
                   kMaxCtaItems * kItemRows * 4 + kMaxCtaTiles * 4 + 15 + 256 + kConsumers * kStages * 8 + 16 + 1024 <=
                   232448,
               "shared-memory layout exceeds the per-CTA limit at the largest K");
+static_assert(kConsumers * kStages * (kItemBytes + kScaleRingBytes) + 2 * (kMaxK2 / kItemK) * 4 * (kXGroupBytes + 12) +
+                  2 * kMaxCtaItems * kItemRows * 4 + kMaxCtaTiles * 4 + 15 + 256 + kConsumers * kStages * 8 + 16 +
+                  1024 <=
+                  232448,
+              "two-token shared-memory layout exceeds the per-CTA limit at its largest K");
+static_assert(kConsumers * kStages * (kItemBytes + kScaleRingBytes) + 3 * (kMaxK3 / kItemK) * 4 * (kXGroupBytes + 12) +
+                  3 * kMaxCtaItems * kItemRows * 4 + kMaxCtaTiles * 4 + 15 + 256 + kConsumers * kStages * 8 + 16 +
+                  1024 <=
+                  232448,
+              "three-token shared-memory layout exceeds the per-CTA limit at its largest K");
 
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt) {
-    if ((fmt != 2 && fmt != 4) || M != 1 || N < 1 || K < kGroup || K % kGroup != 0 || K > kMaxK) return false;
+    if ((fmt != 2 && fmt != 4) || M < 1 || M > (fmt == 4 ? 2 : 3) || N < 1 || K < kGroup || K % kGroup != 0 ||
+        K > max_k((int)M))
+        return false;
     const int64_t RT = (N + kItemRows - 1) / kItemRows;
     return RT * ((K + kItemK - 1) / kItemK) < ((int64_t)1 << 30);
 }
@@ -650,20 +801,20 @@ bool gemv_imma_grid_fits(int64_t N, int64_t K, const DeviceInfo &dev) {
 
 // the zero-initialised workspace region: the control words, then the (value, epoch) pairs
 // of the pieces of row tiles split between CTAs, indexed by the piece's first item:
-// items x 32 x 8 bytes.
-size_t gemv_imma_zeroed_bytes(int64_t N, int64_t K) {
+// items x M x 32 x 8 bytes.
+size_t gemv_imma_zeroed_bytes(int64_t M, int64_t N, int64_t K) {
     const int64_t KC = (K + kItemK - 1) / kItemK;
     const int64_t items = ((N + kItemRows - 1) / kItemRows) * KC;
-    return kCtlRegionBytes + (size_t)items * kItemRows * sizeof(uint64_t);
+    return kCtlRegionBytes + (size_t)items * (size_t)M * kItemRows * sizeof(uint64_t);
 }
 
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
-                             int64_t N, int64_t K, int fmt, const Workspace &ws, cudaStream_t s,
+                             int64_t M, int64_t N, int64_t K, int fmt, const Workspace &ws, cudaStream_t s,
                              const DeviceInfo &dev, int64_t swiglu_f) {
-    if (fmt != 2 && fmt != 4) return cudaErrorInvalidValue;
+    if ((fmt != 2 && fmt != 4) || !gemv_imma_supported(M, N, K, fmt)) return cudaErrorInvalidValue;
     const bool swiglu = swiglu_f > 0;
-    if (swiglu && N != 2 * swiglu_f) return cudaErrorInvalidValue;
-    const Layout lay = make_layout((int)K);
+    if (swiglu && (N != 2 * swiglu_f || M != 1)) return cudaErrorInvalidValue;
+    const Layout lay = make_layout((int)K, (int)M);
     if (lay.total > dev.smem_optin) return cudaErrorInvalidValue;
     // the kernel's 128-bit and barrier accesses rely on these alignments
     if ((lay.sring | lay.xfrag | lay.sxf | lay.slots | lay.zero) % 16 != 0 || lay.full % 8 != 0)
@@ -682,24 +833,32 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
             return cudaErrorInvalidValue;
     }
     const Shape sh = shape_of(N, K, dev.sm_count);
-    if (ws.zeroed_bytes < gemv_imma_zeroed_bytes(N, K)) return cudaErrorInvalidValue;
+    if (ws.zeroed_bytes < gemv_imma_zeroed_bytes(M, N, K)) return cudaErrorInvalidValue;
     unsigned int *ctl = reinterpret_cast<unsigned int *>(ws.zeroed);
     uint64_t *partials = reinterpret_cast<uint64_t *>(ws.zeroed + kCtlRegionBytes);
     // K a multiple of 512: an item's scales of a row are 8 (g64: 16) aligned bytes, copied
     // with the item
-    using Kern = decltype(&gemv_imma_kernel<true, true, true>);
+    using Kern = decltype(&gemv_imma_kernel<true, true, true, 1>);
     const bool async = K % kItemK == 0;
     Kern kern;
-    if (fmt == 4)
-        kern = async ? (swiglu ? gemv_imma_kernel<true, true, true> : gemv_imma_kernel<true, false, true>)
-                     : (swiglu ? gemv_imma_kernel<false, true, true> : gemv_imma_kernel<false, false, true>);
-    else
-        kern = async ? (swiglu ? gemv_imma_kernel<true, true, false> : gemv_imma_kernel<true, false, false>)
-                     : (swiglu ? gemv_imma_kernel<false, true, false> : gemv_imma_kernel<false, false, false>);
+    if (M == 3) {
+        kern = async ? gemv_imma_kernel<true, false, false, 3> : gemv_imma_kernel<false, false, false, 3>;
+    } else if (M == 2) {
+        if (fmt == 4)
+            kern = async ? gemv_imma_kernel<true, false, true, 2> : gemv_imma_kernel<false, false, true, 2>;
+        else
+            kern = async ? gemv_imma_kernel<true, false, false, 2> : gemv_imma_kernel<false, false, false, 2>;
+    } else if (fmt == 4) {
+        kern = async ? (swiglu ? gemv_imma_kernel<true, true, true, 1> : gemv_imma_kernel<true, false, true, 1>)
+                     : (swiglu ? gemv_imma_kernel<false, true, true, 1> : gemv_imma_kernel<false, false, true, 1>);
+    } else {
+        kern = async ? (swiglu ? gemv_imma_kernel<true, true, false, 1> : gemv_imma_kernel<true, false, false, 1>)
+                     : (swiglu ? gemv_imma_kernel<false, true, false, 1> : gemv_imma_kernel<false, false, false, 1>);
+    }
     // the attribute is set to the largest layout any K takes, so that launches of several
     // sizes captured into one graph all stay within it
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         make_layout((int)kMaxK).total);
+                                         make_layout((int)max_k((int)M), (int)M).total);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -88,13 +88,13 @@ constexpr unsigned int kDevStatusGemvPieceTimeout = 2u;  // integer GEMV: a spli
 constexpr unsigned int kDevStatusGemmTimeout = 4u;       // prefill GEMM: a barrier or hand-over wait gave up
 constexpr unsigned int kDevStatusSkinnyTimeout = 8u;     // skinny kernel: the wait for the rotated x gave up
 
-// ---- gemv_imma.cu: M == 1, PQ2_0, integer tensor cores
+// ---- gemv_imma.cu: M <= 2, PQ2_0, integer tensor cores
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt);
-size_t gemv_imma_zeroed_bytes(int64_t N, int64_t K);  // of Workspace::zeroed
+size_t gemv_imma_zeroed_bytes(int64_t M, int64_t N, int64_t K);  // of Workspace::zeroed
 bool gemv_imma_grid_fits(int64_t N, int64_t K, const DeviceInfo &dev);
-// swiglu_f > 0: fused gate/up rows, write silu(gate) * up.
+// swiglu_f > 0 (M == 1 only): fused gate/up rows, write silu(gate) * up.
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
-                             int64_t N, int64_t K, int fmt, const Workspace &ws, cudaStream_t s,
+                             int64_t M, int64_t N, int64_t K, int fmt, const Workspace &ws, cudaStream_t s,
                              const DeviceInfo &dev, int64_t swiglu_f = 0);
 
 // ---- skinny_mma.cu: 1 <= M <= 16 (one launch when its grid is resident at once: the

@@ -66,6 +66,7 @@ DOMINANT_CASES = [
     # (algo, fmt, M, N, K): the integer GEMV, the lookup-table GEMV, the skinny kernel,
     # the prefill GEMM and the plain kernel, each on every packing it takes
     ("IMMA", PQ2, 1, 1000, 2048), ("IMMA", G64, 1, 1000, 2048), ("IMMA", PQ2, 1, 7168, 5120),
+    ("IMMA", PQ2, 2, 1000, 2048), ("IMMA", G64, 2, 1000, 2048),
     ("GEMV", PTQ1, 1, 1000, 2048), ("GEMV", PQ2, 1, 1000, 2048), ("GEMV", Q1, 1, 1000, 2048),
     ("GEMV", G64, 1, 1000, 2048),
     ("SKINNY", PQ2, 4, 1000, 2048), ("SKINNY", G64, 4, 1000, 2048), ("SKINNY", Q1, 4, 1000, 2048),

@@ -335,12 +335,12 @@ def test_imma_input_with_large_and_small_groups(bz, fmt):
 
 def test_imma_rejects_what_it_cannot_run(bz):
     import torch
-    x = torch.zeros((2, 512), dtype=torch.float16, device="cuda")
-    y = torch.zeros((2, 8), dtype=torch.float16, device="cuda")
+    x = torch.zeros((4, 512), dtype=torch.float16, device="cuda")
+    y = torch.zeros((4, 8), dtype=torch.float16, device="cuda")
     s = torch.zeros((8, 4), dtype=torch.float16, device="cuda")
     w = torch.zeros((8, 128), dtype=torch.uint8, device="cuda")
-    with pytest.raises(bz.BonsaiError):  # a batch
-        bz.bonsai_ternary_linear_algo(x, w, s, y, 2, 8, 512, PQ2, bz.BONSAI_ALGO_IMMA)
+    with pytest.raises(bz.BonsaiError):  # a batch of four
+        bz.bonsai_ternary_linear_algo(x, w, s, y, 4, 8, 512, PQ2, bz.BONSAI_ALGO_IMMA)
     with pytest.raises(bz.BonsaiError):  # PTQ1_0
         bz.bonsai_ternary_linear_algo(x[:1], w, s, y[:1], 1, 8, 512, PTQ1, bz.BONSAI_ALGO_IMMA)
 

@@ -34,35 +34,39 @@ def imma_split_tiles(N, K, sms):
     return sorted({c // KC for c in bounds if c % KC != 0})
 
 
-def _run(bz, x, packed, scales, N, K):
+def _run(bz, x, packed, scales, N, K, M=1):
     import torch
-    y = torch.full((1, N), 7.0, dtype=torch.float16, device="cuda")
-    bz.bonsai_ternary_linear_algo(x, packed, scales, y, 1, N, K, PQ2, bz.BONSAI_ALGO_IMMA)
+    y = torch.full((M, N), 7.0, dtype=torch.float16, device="cuda")
+    bz.bonsai_ternary_linear_algo(x, packed, scales, y, M, N, K, PQ2, bz.BONSAI_ALGO_IMMA)
     torch.cuda.synchronize()
-    return to_numpy_f16(y)[0]
+    got = to_numpy_f16(y)
+    return got[0] if M == 1 else got
 
 
-@pytest.mark.parametrize("N,K", [(7168, 5120), (5120, 17408)])
-def test_forced_piece_timeouts_nan_status_and_recovery(bz, N, K):
+@pytest.mark.parametrize("M,N,K", [(1, 7168, 5120), (1, 5120, 17408), (2, 7168, 5120), (3, 7168, 5120)])
+def test_forced_piece_timeouts_nan_status_and_recovery(bz, M, N, K):
+    """M = 2: both tokens' pieces go through the same waits; every split tile is NaN in
+    both rows of y."""
     import torch
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    p = Problem(1, N, K, PQ2, seed=N + K)
+    p = Problem(M, N, K, PQ2, seed=N + K)
     x, packed, scales = p.device()
-    ref = p.oracle_y()[0]
+    ref = p.oracle_y()
+    ref = ref[0] if M == 1 else ref
     split = imma_split_tiles(N, K, sms)
     assert len(split) > 0
     bz.bonsai_device_status(clear=True)
     bz.bonsai_debug_force_timeouts(True)
     try:
-        got = _run(bz, x, packed, scales, N, K)
+        got = _run(bz, x, packed, scales, N, K, M)
     finally:
         bz.bonsai_debug_force_timeouts(False)
     status = bz.bonsai_device_status(clear=True)
     assert status & bz.BONSAI_DEVICE_GEMV_PIECE_TIMEOUT
     assert not status & bz.BONSAI_DEVICE_GEMV_COPY_TIMEOUT
-    bad = np.zeros(N, dtype=bool)
+    bad = np.zeros(got.shape, dtype=bool)
     for t in split:
-        bad[32 * t:min(32 * t + 32, N)] = True
+        bad[..., 32 * t:min(32 * t + 32, N)] = True
     assert np.all(np.isnan(got[bad]))
     assert np.all(np.isfinite(got[~bad]))
     ok, rel, mx = oracle.compare(got[~bad], ref[~bad])
@@ -70,7 +74,7 @@ def test_forced_piece_timeouts_nan_status_and_recovery(bz, N, K):
     # the pieces that arrived after their reader gave up carry that call's number: the
     # next call (hook off) takes none of them
     for _ in range(2):
-        again = _run(bz, x, packed, scales, N, K)
+        again = _run(bz, x, packed, scales, N, K, M)
         ok, rel, mx = oracle.compare(again, ref)
         assert ok, (rel, mx)
     assert bz.bonsai_device_status() == 0
