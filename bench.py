@@ -412,13 +412,15 @@ def measure_decode(f, base, dev, bz, torch, args, world, hbm):
 
 def measure_skinny_grid(f, stack, dev, bz, torch, stream, args, hbm):
     """Decode batches of M in {1, 2, 4, 8, 16} tokens on each projection: the automatic
-    choice, the skinny kernel without split-K, and the prefill GEMM, each as LAYERS calls
-    on distinct weight copies per replay.  GB/s counts the weight, scale, x and y bytes."""
+    choice (the integer GEMV for PQ2_0 at M <= 2 where K allows, else the skinny kernel or
+    the lookup-table GEMV), the skinny kernel with and without split-K, and the prefill
+    GEMM, each as LAYERS calls on distinct weight copies per replay.  GB/s counts the
+    weight, scale, x and y bytes."""
     from ternary_weight_02_b200 import inputs
     sp = stream.cuda_stream
     grid = {}
-    variants = [("auto", bz.BONSAI_ALGO_AUTO, 0), ("skinny_no_split", bz.BONSAI_ALGO_SKINNY, 1),
-                ("gemm", bz.BONSAI_ALGO_GEMM, 0)]
+    variants = [("auto", bz.BONSAI_ALGO_AUTO, 0), ("skinny", bz.BONSAI_ALGO_SKINNY, 0),
+                ("skinny_no_split", bz.BONSAI_ALGO_SKINNY, 1), ("gemm", bz.BONSAI_ALGO_GEMM, 0)]
     with nvtx(torch, f"skinny grid {FMT_NAMES[f]}"):
         for M in (1, 2, 4, 8, 16):
             for i, (name, K, N) in enumerate(SHAPES):
