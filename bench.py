@@ -691,7 +691,8 @@ def run_case(args):
     fmt = FMTS[args.fmt]
     i = [n for n, _, _ in SHAPES].index(args.shape)
     _, K, N = SHAPES[i]
-    M = 1 if args.case in ("gemv", "imma") else args.m
+    # the integer GEMV takes batches of up to 3 tokens (--m); the lookup-table GEMV one
+    M = 1 if args.case == "gemv" or (args.case == "imma" and args.m > 3) else args.m
     dev = torch.device("cuda")
     t = torch.from_numpy(weights(fmt, i, N, K)).to(dev)
     packed = bz.pack(fmt, t)
@@ -730,7 +731,8 @@ def main():
     ap.add_argument("--skinny", type=int, default=1, help="measure the M = 1..16 decode grid (PQ2_0, PTQ1_0)")
     ap.add_argument("--case", choices=["gemv", "imma", "gemm", "skinny"], help="run one projection only (profiler case)")
     ap.add_argument("--shape", choices=[n for n, _, _ in SHAPES], default="gate_up")
-    ap.add_argument("--m", type=int, default=2048, help="tokens for --case gemm / skinny (skinny: at most 16)")
+    ap.add_argument("--m", type=int, default=2048,
+                    help="tokens for --case gemm / skinny / imma (skinny: at most 16; imma: 1 to 3, else 1)")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--tile", type=int, default=0,
                     help="--case: the kernel's split/tile argument (GEMM: 1, 2 or 3 = CTA pairs; 0 automatic)")
