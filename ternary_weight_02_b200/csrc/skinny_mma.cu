@@ -19,9 +19,12 @@
 //   permutation on both operands) so that its four slots are one byte of a word.
 // * Per 128-weight group the MMA starts from zero; the epilogue adds
 //   s[n][g] * (2^24 * D - sum_j x'[m][j]) (the second term turns codes into trits).
-// * Each lane loads only the 8 bytes of a row's group that its MMA slots use (words 2tq,
-//   2tq + 1), and keeps kRing groups in flight in a ring of registers whose slots are
-//   addressed by constants (no register copies that would wait for a load).
+// * Each lane reads only the 8 bytes of a row's group that its MMA slots use (words 2tq,
+//   2tq + 1).  With K a multiple of 1024 (PQ2_0, g64, Q1_0) the weights and scales come
+//   by TMA into a ring of two stages of 8 groups per warp (4 KB of codes, 128-byte
+//   swizzle), so the copies in flight hold no registers and no per-thread load slots;
+//   otherwise (and for PTQ1_0) the lane keeps kRing groups in flight in a ring of
+//   registers whose slots are addressed by constants.
 // * x' (FWHT prepass, FP16) of the CTA's K chunk sits in shared memory as
 //   [k-step][token][16 halves], 4^-(k mod 4)-scaled and in the MMAs' K order, so a
 //   lane's B fragment is one 8-byte load from a contiguous 256-byte row.
@@ -54,11 +57,22 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kRowsPerCta = kWarps * 16;
-constexpr int kRing = 8;  // groups of weights in flight per warp
+constexpr int kRing = 8;  // groups of weights in flight per warp (register ring)
 
 // groups of x' staged in shared memory at a time: 96 KB for either token tile count
 template <int NT>
 constexpr int sub_groups() { return NT == 1 ? 48 : 24; }
+
+// TMA ring (PQ2_0, g64, Q1_0 with K a multiple of 1024): per warp kTStages stages of
+// kTGroups groups of its 16 rows, each stage one mbarrier; x' staged 32 KB at a time.
+constexpr int kTStages = 2;
+constexpr int kTGroups = 8;
+template <int NT>
+constexpr int sub_groups_tma() { return NT == 1 ? 16 : 8; }
+template <int kFmt>
+constexpr int tma_wstage() { return 16 * kTGroups * (kFmt == 3 ? 16 : 32); }  // weight bytes per stage
+template <int kFmt>
+constexpr int tma_sstage() { return 16 * kTGroups * 2 * (kFmt == 4 ? 2 : 1); }  // scale bytes per stage
 
 // One 128-weight group of the warp's rows r0 = gid and r1 = gid + 8, as lane (gid, tq)
 // holds it: words 2tq and 2tq + 1 (g64: tq and tq + 4) of each row, and the rows' FP16
@@ -185,22 +199,38 @@ __global__ void __launch_bounds__(256) skinny_prep_kernel(const uint16_t *__rest
 // staging x' it waits (bounded) until the last CTA has advanced the counter.  The grid
 // is then resident at once (the launcher checks the occupancy).  If that wait gives up,
 // the CTA writes NaN and sets the status bit.
-template <int NT, int kFmt>  // n8 token tiles: 1 (M <= 8) or 2 (M <= 16)
+//
+// kTma: the weights and scales come by TMA into a ring of kTStages stages per warp (the
+// warp's 16 rows x kTGroups groups, 128-byte swizzle; scales unswizzled), one mbarrier
+// per stage, instead of the register ring: the copies in flight then do not hold
+// registers or load slots.  wmap and smap are the packed plane's and the scale plane's
+// tensor maps (unused otherwise).  Needs K a multiple of 1024 and chunks of whole stages.
+template <int NT, int kFmt, bool kTma>  // n8 token tiles: 1 (M <= 8) or 2 (M <= 16)
 __global__ void __launch_bounds__(kThreads) skinny_kernel(
     uint16_t *__restrict__ xsg, float *__restrict__ gsg, const uint8_t *__restrict__ packed,
     const uint16_t *__restrict__ scales, uint16_t *__restrict__ y, float *__restrict__ partials,
     unsigned int *__restrict__ counters, int M, int64_t N, int64_t K, int S, int gpc,
-    const uint16_t *__restrict__ x, unsigned int *__restrict__ ctl) {
+    const uint16_t *__restrict__ x, unsigned int *__restrict__ ctl, const __grid_constant__ CUtensorMap wmap,
+    const __grid_constant__ CUtensorMap smap) {
     constexpr int MT = NT * 8;  // tokens padded
     static_assert(sub_groups<NT>() % kRing == 0, "ring slots follow the group index");
+    static_assert(!kTma || (kFmt != 1 && sub_groups_tma<NT>() % kTGroups == 0), "TMA stages follow the group index");
     // groups staged at a time: the whole chunk when it fits (shared memory is sized so)
-    const int kSub = gpc < sub_groups<NT>() ? gpc : sub_groups<NT>();
-    extern __shared__ __align__(16) uint8_t smem[];
+    constexpr int kSubMax = kTma ? sub_groups_tma<NT>() : sub_groups<NT>();
+    const int kSub = gpc < kSubMax ? gpc : kSubMax;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
     constexpr bool kG64 = kFmt == 4, kQ1 = kFmt == 3, kP1 = kFmt == 1;
     constexpr int kHalves = kG64 ? 2 : 1;  // scale groups per 128 weights
+    constexpr int kWStage = tma_wstage<kFmt>(), kSStage = tma_sstage<kFmt>();
     __shared__ uint16_t lut3[kP1 ? 256 : 1];  // PTQ1_0: byte -> its five digits as 2-bit codes
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);  // [kSub * 8 steps][MT][16]
-    float *gsum = reinterpret_cast<float *>(smem + kSub * 8 * MT * 32);  // [MT][kSub][kHalves]
+    // kTma: [weight ring kWarps x kTStages x kWStage, 1024-byte aligned][scale ring
+    // kWarps x kTStages x kSStage][x'][group sums][stage barriers]; otherwise [x'][group sums]
+    uint8_t *smem = kTma ? smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u) : smem_raw;
+    uint8_t *wring = smem;
+    uint8_t *sring = smem + (kTma ? kWarps * kTStages * kWStage : 0);
+    uint8_t *xbase = sring + (kTma ? kWarps * kTStages * kSStage : 0);
+    uint16_t *xs = reinterpret_cast<uint16_t *>(xbase);  // [kSub * 8 steps][MT][16]
+    float *gsum = reinterpret_cast<float *>(xbase + kSub * 8 * MT * 32);  // [MT][kSub][kHalves]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tq = lane & 3;
@@ -299,14 +329,50 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
         }
     }
 
-    // group g of the chunk lives in ring slot (g - g_begin) % kRing; the first kRing are
-    // requested before x' is staged
-    Grp ring[kRing];
+    // Register ring: group g of the chunk lives in slot (g - g_begin) % kRing; the first
+    // kRing are requested before x' is staged.  TMA ring: stage q (groups g_begin + 8q ..)
+    // in slot q % kTStages of the warp's ring, its barrier completing with phase q / 2 & 1;
+    // the first kTStages are requested before x' is staged.  A stage past the chunk's end
+    // reads groups it does not use (zeros past the row).
+    Grp ring[kTma ? 1 : kRing];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(
+        xbase + kSub * 8 * MT * 32 + ((MT * kSub * kHalves * 4 + 7) & ~7)) + warp * kTStages;
+    const int nstages = kTma ? (g_end - g_begin + kTGroups - 1) / kTGroups : 0;
+    int n_issued = 0;
+    auto issue = [&](int q) {
+        if (q >= nstages) return;
+        const int slot = q % kTStages;
+        if (lane == 0) {
+            uint64_t *bar = bars + slot;
+            uint8_t *wdst = wring + (warp * kTStages + slot) * kWStage;
+            const int g = g_begin + q * kTGroups;
+            mbar_arrive_expect_tx(bar, (uint32_t)(kWStage + kSStage));
+            if (kQ1) {  // 8 groups x 16 bytes: one 128-byte box per row
+                tma_load_2d(wdst, &wmap, bar, g * 16, (int)n0);
+            } else {    // 8 groups x 32 bytes: two boxes of 4 groups
+                tma_load_2d(wdst, &wmap, bar, g * 32, (int)n0);
+                tma_load_2d(wdst + kWStage / 2, &wmap, bar, g * 32 + 128, (int)n0);
+            }
+            tma_load_2d(sring + (warp * kTStages + slot) * kSStage, &smap, bar, g * kHalves, (int)n0);
+        }
+        n_issued++;
+    };
+    if constexpr (kTma) {
+        if (lane == 0) {
+            for (int st = 0; st < kTStages; st++) mbar_init(bars + st, 1);
+            mbar_init_fence();
+        }
+        __syncwarp();
+        for (int q = 0; q < kTStages; q++) issue(q);
+    } else {
 #pragma unroll
-    for (int u = 0; u < kRing; u++)
-        if (g_begin + u < g_end) load(g_begin + u, ring[u]);
+        for (int u = 0; u < kRing; u++)
+            if (g_begin + u < g_end) load(g_begin + u, ring[u]);
+    }
 
     bool barrier_ok = true;
+    bool copies_ok = true;  // (kTma) every stage waited for has landed
+    int n_waited = 0;
     if (x != nullptr) {  // every CTA's x' is staged once the counter has moved on
         __shared__ int ok_s;
         if (tid == 0) {
@@ -344,73 +410,137 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
         }
         __syncthreads();
 
-        for (int gl0 = 0; gl0 < nsub; gl0 += kRing) {
-#pragma unroll
-            for (int u = 0; u < kRing; u++) {
-                const int gl = gl0 + u;
-                if (gl >= nsub) break;
-                Grp &cur = ring[u];
-                if (kP1) {  // base-3 bytes -> the PQ2_0 code words of weights 32tq .. 32tq + 31
-                    const int g = sub + gl;
-                    const int sh0 = (int)(((r0 * G + g) * kPtq1GroupBytes + ptq1_first_byte(tq)) & 3);
-                    const int sh1 = (int)(((r1 * G + g) * kPtq1GroupBytes + ptq1_first_byte(tq)) & 3);
-                    if (v0) cur.a = ptq1_codes(cur.a.x, cur.a.y, cur.a2, sh0, tq, lut3);
-                    if (v1) cur.b = ptq1_codes(cur.b.x, cur.b.y, cur.b2, sh1, tq, lut3);
-                }
-                float d[kHalves][NT][4];  // g64: MMAs 0-3 and 4-7 fill the two halves
-#pragma unroll
-                for (int h = 0; h < kHalves; h++)
-#pragma unroll
-                    for (int nt = 0; nt < NT; nt++)
-#pragma unroll
-                        for (int e = 0; e < 4; e++) d[h][nt][e] = 0.f;
-#pragma unroll
-                for (int i = 0; i < 8; i++) {
-                    // byte (i & 3) of the lane's word i >> 2, in both halves: (c0, c1) and
-                    // (c2, c3) left in place as FP16 subnormals c * 4^j * 2^-24.  Q1_0: byte
-                    // i >> 1 of the word, bits 4(i & 1) + (0, 1) and + (2, 3) left in place
-                    const int byte = kQ1 ? i >> 1 : i & 3;
-                    const uint32_t sel = 0x4040u | (uint32_t)byte | ((uint32_t)byte << 8);
-                    const uint32_t w0 = kQ1 ? cur.a.x : ((i >> 2) ? cur.a.y : cur.a.x);
-                    const uint32_t w1 = kQ1 ? cur.b.x : ((i >> 2) ? cur.b.y : cur.b.x);
-                    const uint32_t p0 = __byte_perm(w0, 0u, sel);
-                    const uint32_t p1 = __byte_perm(w1, 0u, sel);
-                    const uint32_t m01 = kQ1 ? ((i & 1) ? 0x00200010u : 0x00020001u) : 0x000C0003u;
-                    const uint32_t m23 = kQ1 ? ((i & 1) ? 0x00800040u : 0x00080004u) : 0x00C00030u;
-                    const uint32_t a0 = p0 & m01, a1 = p1 & m01;
-                    const uint32_t a2 = p0 & m23, a3 = p1 & m23;
-                    const int ks = gl * 8 + i;
-#pragma unroll
-                    for (int nt = 0; nt < NT; nt++) {
-                        const uint2 b = *reinterpret_cast<const uint2 *>(xs + ((ks * MT + nt * 8 + gid) * 16 + tq * 4));
-                        mma16816(d[kG64 ? i >> 2 : 0][nt], a0, a1, a2, a3, b.x, b.y);
-                    }
-                }
-#pragma unroll
-                for (int h = 0; h < kHalves; h++) {
-                    const float cs0 = half_bits_to_float((uint16_t)(cur.s0 >> (16 * h)));
-                    const float cs1 = half_bits_to_float((uint16_t)(cur.s1 >> (16 * h)));
-#pragma unroll
-                    for (int nt = 0; nt < NT; nt++) {
-                        const int m0 = nt * 8 + 2 * tq;
-                        const float gs0 = gsum[m0 * kSub * kHalves + gl * kHalves + h];
-                        const float gs1 = gsum[(m0 + 1) * kSub * kHalves + gl * kHalves + h];
-                        // d[h][nt][0], [1]: row r0, tokens m0, m0+1; [2], [3]: row r1.  Codes c
-                        // give sum c x' - sum x'; Q1_0 bits b give 2 sum b x' - sum x'
-                        constexpr float kUnit = kQ1 ? 33554432.f : 16777216.f;
-                        acc[nt][0] = fmaf(cs0, fmaf(d[h][nt][0], kUnit, -gs0), acc[nt][0]);
-                        acc[nt][1] = fmaf(cs0, fmaf(d[h][nt][1], kUnit, -gs1), acc[nt][1]);
-                        acc[nt][2] = fmaf(cs1, fmaf(d[h][nt][2], kUnit, -gs0), acc[nt][2]);
-                        acc[nt][3] = fmaf(cs1, fmaf(d[h][nt][3], kUnit, -gs1), acc[nt][3]);
-                    }
-                }
+        // one group of the warp's rows: decode, MMAs, fold into acc
+        auto consume = [&](Grp &cur, int gl) {
+            if (kP1) {  // base-3 bytes -> the PQ2_0 code words of weights 32tq .. 32tq + 31
                 const int g = sub + gl;
-                if (g + kRing < g_end) load(g + kRing, cur);  // refill the slot
+                const int sh0 = (int)(((r0 * G + g) * kPtq1GroupBytes + ptq1_first_byte(tq)) & 3);
+                const int sh1 = (int)(((r1 * G + g) * kPtq1GroupBytes + ptq1_first_byte(tq)) & 3);
+                if (v0) cur.a = ptq1_codes(cur.a.x, cur.a.y, cur.a2, sh0, tq, lut3);
+                if (v1) cur.b = ptq1_codes(cur.b.x, cur.b.y, cur.b2, sh1, tq, lut3);
+            }
+            float d[kHalves][NT][4];  // g64: MMAs 0-3 and 4-7 fill the two halves
+#pragma unroll
+            for (int h = 0; h < kHalves; h++)
+#pragma unroll
+                for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+                    for (int e = 0; e < 4; e++) d[h][nt][e] = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                // byte (i & 3) of the lane's word i >> 2, in both halves: (c0, c1) and
+                // (c2, c3) left in place as FP16 subnormals c * 4^j * 2^-24.  Q1_0: byte
+                // i >> 1 of the word, bits 4(i & 1) + (0, 1) and + (2, 3) left in place
+                const int byte = kQ1 ? i >> 1 : i & 3;
+                const uint32_t sel = 0x4040u | (uint32_t)byte | ((uint32_t)byte << 8);
+                const uint32_t w0 = kQ1 ? cur.a.x : ((i >> 2) ? cur.a.y : cur.a.x);
+                const uint32_t w1 = kQ1 ? cur.b.x : ((i >> 2) ? cur.b.y : cur.b.x);
+                const uint32_t p0 = __byte_perm(w0, 0u, sel);
+                const uint32_t p1 = __byte_perm(w1, 0u, sel);
+                const uint32_t m01 = kQ1 ? ((i & 1) ? 0x00200010u : 0x00020001u) : 0x000C0003u;
+                const uint32_t m23 = kQ1 ? ((i & 1) ? 0x00800040u : 0x00080004u) : 0x00C00030u;
+                const uint32_t a0 = p0 & m01, a1 = p1 & m01;
+                const uint32_t a2 = p0 & m23, a3 = p1 & m23;
+                const int ks = gl * 8 + i;
+#pragma unroll
+                for (int nt = 0; nt < NT; nt++) {
+                    const uint2 b = *reinterpret_cast<const uint2 *>(xs + ((ks * MT + nt * 8 + gid) * 16 + tq * 4));
+                    mma16816(d[kG64 ? i >> 2 : 0][nt], a0, a1, a2, a3, b.x, b.y);
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < kHalves; h++) {
+                const float cs0 = half_bits_to_float((uint16_t)(cur.s0 >> (16 * h)));
+                const float cs1 = half_bits_to_float((uint16_t)(cur.s1 >> (16 * h)));
+#pragma unroll
+                for (int nt = 0; nt < NT; nt++) {
+                    const int m0 = nt * 8 + 2 * tq;
+                    const float gs0 = gsum[m0 * kSub * kHalves + gl * kHalves + h];
+                    const float gs1 = gsum[(m0 + 1) * kSub * kHalves + gl * kHalves + h];
+                    // d[h][nt][0], [1]: row r0, tokens m0, m0+1; [2], [3]: row r1.  Codes c
+                    // give sum c x' - sum x'; Q1_0 bits b give 2 sum b x' - sum x'
+                    constexpr float kUnit = kQ1 ? 33554432.f : 16777216.f;
+                    acc[nt][0] = fmaf(cs0, fmaf(d[h][nt][0], kUnit, -gs0), acc[nt][0]);
+                    acc[nt][1] = fmaf(cs0, fmaf(d[h][nt][1], kUnit, -gs1), acc[nt][1]);
+                    acc[nt][2] = fmaf(cs1, fmaf(d[h][nt][2], kUnit, -gs0), acc[nt][2]);
+                    acc[nt][3] = fmaf(cs1, fmaf(d[h][nt][3], kUnit, -gs1), acc[nt][3]);
+                }
+            }
+        };
+        if constexpr (kTma) {
+            for (int gs = 0; gs < nsub; gs += kTGroups) {
+                const int q = (sub - g_begin + gs) / kTGroups;  // the stage
+                const int slot = q % kTStages;
+                if (copies_ok) {  // warp-uniform verdict
+                    copies_ok = __all_sync(0xffffffffu, mbar_wait(bars + slot, (uint32_t)(q / kTStages) & 1u));
+                    if (copies_ok)
+                        n_waited++;
+                    else if (lane == 0 && ctl != nullptr)
+                        atomicOr(ctl + kCtlStatus, kDevStatusSkinnyTimeout);
+                }
+                const uint8_t *wst = wring + (warp * kTStages + slot) * kWStage;
+                const uint8_t *sst = sring + (warp * kTStages + slot) * kSStage;
+#pragma unroll
+                for (int u = 0; u < kTGroups; u++) {
+                    if (gs + u >= nsub) break;
+                    // rows gid and gid + 8 of the stage (both in swizzle phase gid); the
+                    // lane's words as the register ring would load them
+                    Grp cur;
+                    if (kQ1) {  // word tq of the 16-byte group u: logical chunk u
+                        const int c = (u ^ gid) << 4;
+                        cur.a = make_uint2(*reinterpret_cast<const uint32_t *>(wst + gid * 128 + c + 4 * tq), 0u);
+                        cur.b = make_uint2(*reinterpret_cast<const uint32_t *>(wst + (gid + 8) * 128 + c + 4 * tq), 0u);
+                    } else {
+                        const uint8_t *b0 = wst + (u >> 2) * (kWStage / 2) + gid * 128;  // box of groups 4(u/4) ..
+                        const uint8_t *b1 = b0 + 8 * 128;
+                        const int qg = u & 3;
+                        if (kG64) {  // words tq and tq + 4: logical chunks 2qg and 2qg + 1
+                            const int c0 = ((2 * qg) ^ gid) << 4, c1 = ((2 * qg + 1) ^ gid) << 4;
+                            cur.a = make_uint2(*reinterpret_cast<const uint32_t *>(b0 + c0 + 4 * tq),
+                                               *reinterpret_cast<const uint32_t *>(b0 + c1 + 4 * tq));
+                            cur.b = make_uint2(*reinterpret_cast<const uint32_t *>(b1 + c0 + 4 * tq),
+                                               *reinterpret_cast<const uint32_t *>(b1 + c1 + 4 * tq));
+                        } else {  // words 2tq, 2tq + 1: logical chunk 2qg + tq / 2
+                            const int c = ((2 * qg + (tq >> 1)) ^ gid) << 4;
+                            cur.a = *reinterpret_cast<const uint2 *>(b0 + c + (tq & 1) * 8);
+                            cur.b = *reinterpret_cast<const uint2 *>(b1 + c + (tq & 1) * 8);
+                        }
+                    }
+                    if (kG64) {
+                        cur.s0 = reinterpret_cast<const uint32_t *>(sst)[gid * kTGroups + u];
+                        cur.s1 = reinterpret_cast<const uint32_t *>(sst)[(gid + 8) * kTGroups + u];
+                    } else {
+                        cur.s0 = reinterpret_cast<const uint16_t *>(sst)[gid * kTGroups + u];
+                        cur.s1 = reinterpret_cast<const uint16_t *>(sst)[(gid + 8) * kTGroups + u];
+                    }
+                    cur.a2 = cur.b2 = 0u;
+                    consume(cur, gs + u);
+                }
+                __syncwarp();  // every lane has read the stage
+                if (copies_ok) {
+                    if (lane == 0) fence_proxy_async();
+                    issue(q + kTStages);  // refill the slot
+                }
+            }
+        } else {
+            for (int gl0 = 0; gl0 < nsub; gl0 += kRing) {
+#pragma unroll
+                for (int u = 0; u < kRing; u++) {
+                    const int gl = gl0 + u;
+                    if (gl >= nsub) break;
+                    Grp &cur = ring[u];
+                    consume(cur, gl);
+                    const int g = sub + gl;
+                    if (g + kRing < g_end) load(g + kRing, cur);  // refill the slot
+                }
             }
         }
     }
 
-    if (!barrier_ok)
+    if (kTma && !copies_ok && lane == 0) {  // the copies already started land before the CTA exits
+        for (int q = n_waited; q < n_issued; q++) mbar_wait(bars + q % kTStages, (uint32_t)(q / kTStages) & 1u);
+    }
+    if (!barrier_ok || !copies_ok)
 #pragma unroll
         for (int nt = 0; nt < NT; nt++)
 #pragma unroll
@@ -456,21 +586,32 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
     if (lane == 0) counters[rb] = 0u;
 }
 
-int smem_bytes(int NT, int gpc, bool g64) {
-    int sub = NT == 1 ? sub_groups<1>() : sub_groups<2>();
+// The TMA ring takes PQ2_0, g64 and Q1_0 when a row's groups come in whole stages (its
+// plane rows and scale rows are then multiples of 16 bytes, as tensor maps need).
+bool use_tma(int64_t K, int fmt) { return fmt != 1 && (K / kGroup) % kTGroups == 0; }
+
+int smem_bytes(int NT, int gpc, int fmt, bool tma) {
+    const bool g64 = fmt == 4;
+    int sub = tma ? (NT == 1 ? sub_groups_tma<1>() : sub_groups_tma<2>()) : (NT == 1 ? sub_groups<1>() : sub_groups<2>());
     sub = gpc < sub ? gpc : sub;
-    return sub * 8 * NT * 8 * 32 + NT * 8 * sub * 4 * (g64 ? 2 : 1);
+    const int xs = sub * 8 * NT * 8 * 32, gs = NT * 8 * sub * 4 * (g64 ? 2 : 1);
+    if (!tma) return xs + gs;
+    const int ws = fmt == 3 ? tma_wstage<3>() : tma_wstage<2>();
+    const int ss = g64 ? tma_sstage<4>() : tma_sstage<2>();
+    return 1024 + kWarps * kTStages * (ws + ss) + xs + ((gs + 7) & ~7) + kWarps * kTStages * 8;
 }
 
 // K chunks: about as many CTAs as fit on the GPU at once (one wave; a CTA's registers
-// allow two per SM), unless split_k (> 0) says otherwise.
-void choose_split(int64_t N, int64_t K, int split_k, const DeviceInfo &dev, int *S, int *gpc) {
+// allow two per SM), unless split_k (> 0) says otherwise.  With the TMA ring a chunk is
+// a whole number of stages (kTGroups groups).
+void choose_split(int64_t N, int64_t K, int split_k, bool tma, const DeviceInfo &dev, int *S, int *gpc) {
     const int64_t G = K / kGroup;
     const int64_t rb = (N + kRowsPerCta - 1) / kRowsPerCta;
     int64_t s = split_k > 0 ? split_k : (2 * (int64_t)dev.sm_count) / rb;
     if (s < 1) s = 1;
     if (s > G) s = G;
-    const int64_t per = (G + s - 1) / s;
+    int64_t per = (G + s - 1) / s;
+    if (tma) per = (per + kTGroups - 1) / kTGroups * kTGroups;
     *gpc = (int)per;
     *S = (int)((G + per - 1) / per);
 }
@@ -486,11 +627,11 @@ size_t gsum_bytes(int64_t M, int64_t K) {  // room for the g64 half sums
     return ((size_t)(K / kGroup) * 2 * MT * 4 + 255) / 256 * 256;
 }
 
-// The kernel instance for (M, fmt), its shared memory, and whether its grid is resident
-// on the GPU at once (then the rotation runs inside it: one launch).
-template <int NT, int kFmt>
+// The kernel instance for (M, fmt, ring), its shared memory, and whether its grid is
+// resident on the GPU at once (then the rotation runs inside it: one launch).
+template <int NT, int kFmt, bool kTma>
 cudaError_t kernel_fits(int64_t grid_ctas, int smem, const DeviceInfo &dev, bool *fits) {
-    auto kern = skinny_kernel<NT, kFmt>;
+    auto kern = skinny_kernel<NT, kFmt, kTma>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (err != cudaSuccess) return err;
     int per_sm = 0;
@@ -500,21 +641,27 @@ cudaError_t kernel_fits(int64_t grid_ctas, int smem, const DeviceInfo &dev, bool
     return cudaSuccess;
 }
 
+template <int NT>
+cudaError_t kernel_fits_fmt(int fmt, bool tma, int64_t ctas, int smem, const DeviceInfo &dev, bool *fits) {
+    if (tma)
+        return fmt == 4   ? kernel_fits<NT, 4, true>(ctas, smem, dev, fits)
+               : fmt == 3 ? kernel_fits<NT, 3, true>(ctas, smem, dev, fits)
+                          : kernel_fits<NT, 2, true>(ctas, smem, dev, fits);
+    return fmt == 4   ? kernel_fits<NT, 4, false>(ctas, smem, dev, fits)
+           : fmt == 3 ? kernel_fits<NT, 3, false>(ctas, smem, dev, fits)
+           : fmt == 1 ? kernel_fits<NT, 1, false>(ctas, smem, dev, fits)
+                      : kernel_fits<NT, 2, false>(ctas, smem, dev, fits);
+}
+
 cudaError_t grid_fits(int64_t M, int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev, bool *fits) {
+    const bool tma = use_tma(K, fmt);
     int S, gpc;
-    choose_split(N, K, split_k, dev, &S, &gpc);
+    choose_split(N, K, split_k, tma, dev, &S, &gpc);
     const int64_t ctas = ((N + kRowsPerCta - 1) / kRowsPerCta) * S;
     const int NT = M <= 8 ? 1 : 2;
-    const int smem = smem_bytes(NT, gpc, fmt == 4);
-    if (NT == 1)
-        return fmt == 4   ? kernel_fits<1, 4>(ctas, smem, dev, fits)
-               : fmt == 3 ? kernel_fits<1, 3>(ctas, smem, dev, fits)
-               : fmt == 1 ? kernel_fits<1, 1>(ctas, smem, dev, fits)
-                          : kernel_fits<1, 2>(ctas, smem, dev, fits);
-    return fmt == 4   ? kernel_fits<2, 4>(ctas, smem, dev, fits)
-           : fmt == 3 ? kernel_fits<2, 3>(ctas, smem, dev, fits)
-           : fmt == 1 ? kernel_fits<2, 1>(ctas, smem, dev, fits)
-                      : kernel_fits<2, 2>(ctas, smem, dev, fits);
+    const int smem = smem_bytes(NT, gpc, fmt, tma);
+    return NT == 1 ? kernel_fits_fmt<1>(fmt, tma, ctas, smem, dev, fits)
+                   : kernel_fits_fmt<2>(fmt, tma, ctas, smem, dev, fits);
 }
 
 }  // namespace
@@ -525,9 +672,8 @@ bool skinny_supported(int64_t M, int64_t N, int64_t K, int fmt) {
 }
 
 size_t skinny_workspace_bytes(int64_t M, int64_t N, int64_t K, int fmt, int split_k, const DeviceInfo &dev) {
-    (void)fmt;
     int S, gpc;
-    choose_split(N, K, split_k, dev, &S, &gpc);
+    choose_split(N, K, split_k, use_tma(K, fmt), dev, &S, &gpc);
     return staged_bytes(M, K) + gsum_bytes(M, K) + (S > 1 ? (size_t)S * (size_t)M * (size_t)N * sizeof(float) : 0);
 }
 
@@ -544,11 +690,34 @@ cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16
     uint16_t *xsg = reinterpret_cast<uint16_t *>(ws.data);
     float *gsg = reinterpret_cast<float *>(ws.data + staged_bytes(M, K));
     float *partials = reinterpret_cast<float *>(ws.data + staged_bytes(M, K) + gsum_bytes(M, K));
+    const bool tma = use_tma(K, fmt);
     int S, gpc;
-    choose_split(N, K, split_k, dev, &S, &gpc);
+    choose_split(N, K, split_k, tma, dev, &S, &gpc);
     const dim3 grid((unsigned)((N + kRowsPerCta - 1) / kRowsPerCta), (unsigned)S);
     const int64_t G = K / kGroup;
-    const bool g64 = fmt == 4;
+    // tensor maps of the packed plane (rows of G x 32 bytes, Q1_0 16; boxes of 128 bytes x
+    // 16 rows, 128-byte swizzle) and of the scale plane (rows of G or 2G FP16; boxes of 8
+    // or 16 scales x 16 rows), for the TMA ring; zeros otherwise (never read)
+    CUtensorMap wmap, smap;
+    memset(&wmap, 0, sizeof(wmap));
+    memset(&smap, 0, sizeof(smap));
+    if (tma) {
+        EncodeTiledFn encode = encode_fn();
+        if (!encode) return cudaErrorNotSupported;
+        const int64_t rowb = G * (fmt == 3 ? 16 : 32), GS = G * (fmt == 4 ? 2 : 1);
+        const cuuint64_t wd[2] = {(cuuint64_t)rowb, (cuuint64_t)N}, ws_[1] = {(cuuint64_t)rowb};
+        const cuuint32_t wb[2] = {128, 16}, es[2] = {1, 1};
+        if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), wd, ws_, wb, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+        const cuuint64_t sd[2] = {(cuuint64_t)GS, (cuuint64_t)N}, ss_[1] = {(cuuint64_t)GS * 2};
+        const cuuint32_t sb[2] = {(cuuint32_t)(kTGroups * (fmt == 4 ? 2 : 1)), 16};
+        if (encode(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(scales), sd, ss_, sb, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
     // one launch when the whole grid is resident at once (its CTAs meet at a barrier after
     // rotating x), else the rotation pass first
     bool fits = false;
@@ -556,24 +725,35 @@ cudaError_t launch_skinny(const uint16_t *x, const uint8_t *packed, const uint16
     if (ferr != cudaSuccess) return ferr;
     const bool fused = fits && ws.zeroed != nullptr && ws.zeroed_bytes >= kCtlRegionBytes;
     auto run = [&](auto prep, auto kern, int MT, int NT) -> cudaError_t {
-        const int smem = smem_bytes(NT, gpc, g64);
+        const int smem = smem_bytes(NT, gpc, fmt, tma);
         cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (err != cudaSuccess) return err;
         if (!fused) prep<<<(unsigned)((G * MT + 7) / 8), 256, 0, s>>>(x, xsg, gsg, (int)M, K);
         kern<<<grid, kThreads, smem, s>>>(xsg, gsg, packed, scales, y, partials, ws.counters, (int)M, N, K, S, gpc,
-                                          fused ? x : nullptr, reinterpret_cast<unsigned int *>(ws.zeroed));
+                                          fused ? x : nullptr, reinterpret_cast<unsigned int *>(ws.zeroed), wmap,
+                                          smap);
         return cudaGetLastError();
     };
     if (M <= 8) {
-        if (g64) return run(skinny_prep_kernel<8, 4>, skinny_kernel<1, 4>, 8, 1);
-        if (fmt == 3) return run(skinny_prep_kernel<8, 3>, skinny_kernel<1, 3>, 8, 1);
-        if (fmt == 1) return run(skinny_prep_kernel<8, 1>, skinny_kernel<1, 1>, 8, 1);
-        return run(skinny_prep_kernel<8, 2>, skinny_kernel<1, 2>, 8, 1);
+        if (fmt == 4)
+            return tma ? run(skinny_prep_kernel<8, 4>, skinny_kernel<1, 4, true>, 8, 1)
+                       : run(skinny_prep_kernel<8, 4>, skinny_kernel<1, 4, false>, 8, 1);
+        if (fmt == 3)
+            return tma ? run(skinny_prep_kernel<8, 3>, skinny_kernel<1, 3, true>, 8, 1)
+                       : run(skinny_prep_kernel<8, 3>, skinny_kernel<1, 3, false>, 8, 1);
+        if (fmt == 1) return run(skinny_prep_kernel<8, 1>, skinny_kernel<1, 1, false>, 8, 1);
+        return tma ? run(skinny_prep_kernel<8, 2>, skinny_kernel<1, 2, true>, 8, 1)
+                   : run(skinny_prep_kernel<8, 2>, skinny_kernel<1, 2, false>, 8, 1);
     }
-    if (g64) return run(skinny_prep_kernel<16, 4>, skinny_kernel<2, 4>, 16, 2);
-    if (fmt == 3) return run(skinny_prep_kernel<16, 3>, skinny_kernel<2, 3>, 16, 2);
-    if (fmt == 1) return run(skinny_prep_kernel<16, 1>, skinny_kernel<2, 1>, 16, 2);
-    return run(skinny_prep_kernel<16, 2>, skinny_kernel<2, 2>, 16, 2);
+    if (fmt == 4)
+        return tma ? run(skinny_prep_kernel<16, 4>, skinny_kernel<2, 4, true>, 16, 2)
+                   : run(skinny_prep_kernel<16, 4>, skinny_kernel<2, 4, false>, 16, 2);
+    if (fmt == 3)
+        return tma ? run(skinny_prep_kernel<16, 3>, skinny_kernel<2, 3, true>, 16, 2)
+                   : run(skinny_prep_kernel<16, 3>, skinny_kernel<2, 3, false>, 16, 2);
+    if (fmt == 1) return run(skinny_prep_kernel<16, 1>, skinny_kernel<2, 1, false>, 16, 2);
+    return tma ? run(skinny_prep_kernel<16, 2>, skinny_kernel<2, 2, true>, 16, 2)
+               : run(skinny_prep_kernel<16, 2>, skinny_kernel<2, 2, false>, 16, 2);
 }
 
 }  // namespace bonsai
