@@ -77,6 +77,26 @@ def test_host_validation_needs_no_gpu(bz):
     assert L.bonsai_pack_pq2(None, None, 0, 128, None) == bz.BONSAI_OK
 
 
+def test_integer_gemv_batch_limits_on_the_host(bz):
+    """The integer tensor-core GEMV takes PQ2_0 and g64 at M = 1 (K <= 24576), M = 2
+    (K <= 12288) and, for PQ2_0, M = 3 (K <= 6144); an explicit request past those
+    limits is refused on the host, before any device is touched.  Within them the call
+    gets as far as the device (none here, or the GPU's answer)."""
+    import torch
+    L = bz.raw()
+    good = 1 << 20
+    IMMA, PQ2, G64, PTQ1 = bz.BONSAI_ALGO_IMMA, bz.BONSAI_FMT_PQ2_0, bz.BONSAI_FMT_PQ2_0_G64, bz.BONSAI_FMT_PTQ1_0
+
+    def call(M, K, fmt):
+        return L.bonsai_ternary_linear_algo(good, good, good, good, M, 64, K, fmt, IMMA, 0, None)
+    for M, K, fmt in [(4, 1024, PQ2), (2, 12288 + 128, PQ2), (3, 6144 + 128, PQ2), (3, 1024, G64),
+                      (1, 24576 + 128, PQ2), (1, 1024, PTQ1), (2, 1024, PTQ1)]:
+        assert call(M, K, fmt) == bz.BONSAI_ERR_ALGO, (M, K, fmt)
+    if not torch.cuda.is_available():
+        for M, K, fmt in [(1, 24576, PQ2), (2, 12288, PQ2), (2, 12288, G64), (3, 6144, PQ2)]:
+            assert call(M, K, fmt) == bz.BONSAI_ERR_CUDA, (M, K, fmt)
+
+
 def test_status_strings(bz):
     for code in range(-9, 1):
         s = bz.bonsai_status_string(code)
