@@ -173,9 +173,10 @@ int bonsai_ternary_linear(const uint16_t *x, const uint8_t *packed, const uint16
  * BONSAI_ALGO_GEMM the same argument picks the M tile instead: 1 = 128 rows per CTA,
  * 2 = 256 rows (two TMEM accumulators sharing each expanded weight tile), 3 = CTA
  * pairs (clusters of two SMs issuing 256-row tcgen05 MMAs together, each SM expanding
- * half of every weight tile; an explicit choice only), 0 = automatic (1 or 2).  For BONSAI_ALGO_GEMV it picks the schedule: 1 = each CTA walks all K
- * slices of its rows (no split-K), >= 2 = one 512-wide K slice per CTA with split-K
- * partials, 0 = automatic.  BONSAI_ALGO_IMMA ignores it (its work split is fixed
+ * half of every weight tile; an explicit choice only), 0 = automatic (1 or 2).  For
+ * BONSAI_ALGO_GEMV it picks the schedule: 1 = each CTA walks all K slices of its rows
+ * (no split-K), >= 2 = one 512-wide K slice per CTA with split-K partials, 0 =
+ * automatic.  BONSAI_ALGO_IMMA ignores it (its work split is fixed
  * by the shape and the SM count, so results are bitwise repeatable).
  * Returns BONSAI_ERR_ALGO if the chosen kernel cannot run the shape (e.g.
  * BONSAI_ALGO_GEMV with M > 1, or BONSAI_ALGO_IMMA on a shape whose grid would not fit
@@ -250,6 +251,8 @@ int bonsai_ternary_linear_noalloc(const uint16_t *x, const uint8_t *packed, cons
 #define BONSAI_DEVICE_GEMV_PIECE_TIMEOUT 2u /* integer GEMV: a split tile's later piece, or  */
                                             /* its hand-over, never came                      */
 #define BONSAI_DEVICE_GEMM_TIMEOUT 4u       /* prefill GEMM: a barrier or hand-over wait gave up */
+#define BONSAI_DEVICE_SKINNY_TIMEOUT 8u     /* skinny kernel: the wait after the rotation   */
+                                            /* phase, or a weight copy, never ended           */
 
 /* Reads the calling device's status bits into *bits after synchronising `stream` (the
  * stream of the calls in question), and clears them when `clear` is non-zero.  *bits is 0

@@ -35,6 +35,7 @@ BONSAI_ERR_TOO_LARGE = -9
 BONSAI_DEVICE_GEMV_COPY_TIMEOUT = 1
 BONSAI_DEVICE_GEMV_PIECE_TIMEOUT = 2
 BONSAI_DEVICE_GEMM_TIMEOUT = 4
+BONSAI_DEVICE_SKINNY_TIMEOUT = 8
 
 BONSAI_ALGO_AUTO = 0
 BONSAI_ALGO_SIMPLE = 1

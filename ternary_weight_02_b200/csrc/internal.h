@@ -86,9 +86,9 @@ constexpr size_t kCtlRegionBytes = 4096;
 constexpr unsigned int kDevStatusGemvCopyTimeout = 1u;   // integer GEMV: a weight copy never landed
 constexpr unsigned int kDevStatusGemvPieceTimeout = 2u;  // integer GEMV: a split tile's later piece never came
 constexpr unsigned int kDevStatusGemmTimeout = 4u;       // prefill GEMM: a barrier or hand-over wait gave up
-constexpr unsigned int kDevStatusSkinnyTimeout = 8u;     // skinny kernel: the wait for the rotated x gave up
+constexpr unsigned int kDevStatusSkinnyTimeout = 8u;     // skinny kernel: the wait for the rotated x, or a TMA copy, gave up
 
-// ---- gemv_imma.cu: M <= 2, PQ2_0, integer tensor cores
+// ---- gemv_imma.cu: M <= 3 (g64: 2), PQ2_0 and g64, integer tensor cores
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t gemv_imma_zeroed_bytes(int64_t M, int64_t N, int64_t K);  // of Workspace::zeroed
 bool gemv_imma_grid_fits(int64_t N, int64_t K, const DeviceInfo &dev);
