@@ -366,8 +366,9 @@ __device__ __forceinline__ void expand_warps_sync() { asm volatile("bar.sync 1, 
 // kPair: the CTAs work in pairs (clusters of two) on tiles of 256 kAcc rows x 256 columns
 // with tcgen05.mma.cta_group::2: CTA rank r of the pair holds x' rows a 256 + 128 r ..
 // +127 of its accumulator a and expands weight rows 128 r .. 128 r + 127 of the tile's
-// 256 (two threads per row, half a stage each), so each SM expands and reads half the B
-// operand for the same MMA work.  The even CTA issues the MMAs once both CTAs' stages
+// 256 (two threads per row, half a stage each), so each SM expands half the B operand for
+// the same MMA work (each SM's tensor core still reads all of B, the peer's half from the
+// peer's shared memory).  The even CTA issues the MMAs once both CTAs' stages
 // are ready (its full_b barrier counts its own expansion warps and one arrival that a
 // thread of the odd CTA forwards) and commits them to the barriers of both; hand-over
 // slots and flags stay per CTA, work is split per pair.  Only an explicit request takes
