@@ -459,6 +459,19 @@ def test_skinny_decode_shapes_full(bz, fmt, M, K, N):
 
 
 @pytest.mark.parametrize("fmt", [PQ2, G64, Q1, PTQ1])
+@pytest.mark.parametrize("M", [2, 3])
+@pytest.mark.parametrize("K,N", [(5120, 7168), (17408, 5120)])
+def test_skinny_explicit_small_batches_full(bz, fmt, M, K, N):
+    """The skinny kernel asked for explicitly at M = 2, 3 on full shapes (the default entry
+    point gives most of these to the integer GEMV; down and the explicit choice still run
+    the skinny kernel, with its TMA ring for every packing but PTQ1_0)."""
+    p = Problem(M, N, K, fmt, seed=70 + M)
+    got = _run(bz, p, bz.BONSAI_ALGO_SKINNY)
+    ok, rel, mx = oracle.compare(got, p.oracle_y())
+    assert ok, (rel, mx)
+
+
+@pytest.mark.parametrize("fmt", [PQ2, G64, Q1, PTQ1])
 def test_skinny_split_is_deterministic(bz, fmt):
     import torch
     p = Problem(8, 5120, 17408, fmt, seed=3)
