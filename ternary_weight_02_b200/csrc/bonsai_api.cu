@@ -375,7 +375,7 @@ int bonsai_ternary_linear_swiglu(const uint16_t *x, const uint8_t *packed, const
     chosen = resolve_algo(BONSAI_ALGO_AUTO, M, N, K, fmt, &st->info);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     Workspace ws;
-    if (chosen == BONSAI_ALGO_IMMA && M == 1) {  // fused into the GEMV's epilogue
+    if (chosen == BONSAI_ALGO_IMMA) {  // fused into the GEMV's epilogue
         rc = ensure_workspace(*st, 0, gemv_imma_zeroed_bytes(M, N, K), &ws);
         if (rc != BONSAI_OK) return rc;
         return cuda_status(launch_gemv_imma(x, packed, scales, h, M, N, K, fmt, ws, s, st->info, F));

@@ -294,8 +294,7 @@ __device__ __forceinline__ float wait_pairs(const uint64_t *p, int lane, uint32_
 // and an offset added to the epoch it waits for: kSpinLimit and 0, except under the test
 // hook that makes those waits give up.
 //
-// kM: tokens (1 to 3; g64 1 or 2); x is kM x K and y kM x N, row-major.  (kSwiglu needs
-// kM = 1.)
+// kM: tokens (1 to 3; g64 1 or 2); x is kM x K and y kM x N (kSwiglu: kM x F), row-major.
 template <bool kAsyncScales, bool kSwiglu, bool kG64, int kM>
 __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     const __grid_constant__ CUtensorMap wmap, const uint16_t *__restrict__ x, const uint16_t *__restrict__ scales,
@@ -305,8 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
     uint8_t *smem = smem_raw + ((1024u - (saddr(smem_raw) & 1023u)) & 1023u);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gid = lane >> 2, tig = lane & 3;
-    static_assert(kM == 1 || (kM <= 3 && !kSwiglu && (!kG64 || kM == 2)),
-                  "several tokens: up to 3 (g64: 2), without the SwiGLU epilogue");
+    static_assert(kM == 1 || (kM <= 3 && (!kG64 || kM == 2)), "several tokens: up to 3 (g64: 2)");
     const Layout L = make_layout(K, kM);
     const int G = K / kGroup;
     const int GS = kG64 ? 2 * G : G;  // scales per row
@@ -484,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_imma_kernel(
             if (kSwiglu) {  // h = silu(gate) * up: lanes 0..15 hold gate rows, 16..31 the up rows
                 const float up = __shfl_down_sync(0xffffffffu, sum, 16);
                 const int f = 16 * rt + lane;
-                if (lane < 16 && f < F) y[f] = float_to_half_bits(sum / (1.f + expf(-sum)) * up);
+                if (lane < 16 && f < F) y[(int64_t)m * F + f] = float_to_half_bits(sum / (1.f + expf(-sum)) * up);
                 continue;
             }
             const int row = rt * kItemRows + lane;
@@ -813,7 +811,7 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
                              const DeviceInfo &dev, int64_t swiglu_f) {
     if ((fmt != 2 && fmt != 4) || !gemv_imma_supported(M, N, K, fmt)) return cudaErrorInvalidValue;
     const bool swiglu = swiglu_f > 0;
-    if (swiglu && (N != 2 * swiglu_f || M != 1)) return cudaErrorInvalidValue;
+    if (swiglu && N != 2 * swiglu_f) return cudaErrorInvalidValue;
     const Layout lay = make_layout((int)K, (int)M);
     if (lay.total > dev.smem_optin) return cudaErrorInvalidValue;
     // the kernel's 128-bit and barrier accesses rely on these alignments
@@ -842,12 +840,15 @@ cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uin
     const bool async = K % kItemK == 0;
     Kern kern;
     if (M == 3) {
-        kern = async ? gemv_imma_kernel<true, false, false, 3> : gemv_imma_kernel<false, false, false, 3>;
+        kern = async ? (swiglu ? gemv_imma_kernel<true, true, false, 3> : gemv_imma_kernel<true, false, false, 3>)
+                     : (swiglu ? gemv_imma_kernel<false, true, false, 3> : gemv_imma_kernel<false, false, false, 3>);
     } else if (M == 2) {
         if (fmt == 4)
-            kern = async ? gemv_imma_kernel<true, false, true, 2> : gemv_imma_kernel<false, false, true, 2>;
+            kern = async ? (swiglu ? gemv_imma_kernel<true, true, true, 2> : gemv_imma_kernel<true, false, true, 2>)
+                         : (swiglu ? gemv_imma_kernel<false, true, true, 2> : gemv_imma_kernel<false, false, true, 2>);
         else
-            kern = async ? gemv_imma_kernel<true, false, false, 2> : gemv_imma_kernel<false, false, false, 2>;
+            kern = async ? (swiglu ? gemv_imma_kernel<true, true, false, 2> : gemv_imma_kernel<true, false, false, 2>)
+                         : (swiglu ? gemv_imma_kernel<false, true, false, 2> : gemv_imma_kernel<false, false, false, 2>);
     } else if (fmt == 4) {
         kern = async ? (swiglu ? gemv_imma_kernel<true, true, true, 1> : gemv_imma_kernel<true, false, true, 1>)
                      : (swiglu ? gemv_imma_kernel<false, true, true, 1> : gemv_imma_kernel<false, false, true, 1>);

@@ -92,7 +92,7 @@ constexpr unsigned int kDevStatusSkinnyTimeout = 8u;     // skinny kernel: the w
 bool gemv_imma_supported(int64_t M, int64_t N, int64_t K, int fmt);
 size_t gemv_imma_zeroed_bytes(int64_t M, int64_t N, int64_t K);  // of Workspace::zeroed
 bool gemv_imma_grid_fits(int64_t N, int64_t K, const DeviceInfo &dev);
-// swiglu_f > 0 (M == 1 only): fused gate/up rows, write silu(gate) * up.
+// swiglu_f > 0: fused gate/up rows, write silu(gate) * up (M x swiglu_f).
 cudaError_t launch_gemv_imma(const uint16_t *x, const uint8_t *packed, const uint16_t *scales, uint16_t *y,
                              int64_t M, int64_t N, int64_t K, int fmt, const Workspace &ws, cudaStream_t s,
                              const DeviceInfo &dev, int64_t swiglu_f = 0);

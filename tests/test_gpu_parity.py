@@ -526,15 +526,18 @@ def _run_swiglu(bz, p, F):
     return to_numpy_f16(h)
 
 
-# (M, F, K, fmt): fused in the integer GEMV (M = 1 PQ2_0 and g64; F = 24 leaves a part-used last
-# tile; the last case is the full 27B-class gate/up) or the GEMM (tiles split between
-# CTAs; F = 200 and 1270 part-used); the other packings at M = 1 and the skinny batches
-# take the linear kernel and then the SwiGLU kernel
+# (M, F, K, fmt): fused in the integer GEMV (M = 1 PQ2_0 and g64, M = 2 both, M = 3 PQ2_0;
+# F = 24 leaves a part-used last tile; the M = 1 and 2 cases at F = 17408 are the full
+# 27B-class gate/up) or the GEMM (tiles split between CTAs; F = 200 and 1270 part-used);
+# the other packings at M = 1 and the skinny batches take the linear kernel and then the
+# SwiGLU kernel
 SWIGLU_CASES = [(1, 16, 512, PQ2), (1, 1024, 2048, PQ2), (1, 4000, 1152, PQ2), (1, 24, 512, PQ2),
                 (1, 1024, 1024, PTQ1), (1, 1024, 2048, Q1), (4, 512, 1024, PQ2), (300, 640, 640, PQ2),
                 (300, 640, 640, Q1), (300, 384, 1152, PTQ1), (600, 1280, 384, PQ2), (300, 200, 640, PQ2), (300, 1270, 256, Q1),
                 (1, 1024, 2048, G64), (1, 24, 512, G64), (1, 4000, 1152, G64), (300, 200, 640, G64),
-                (600, 1280, 384, G64), (4, 512, 1024, G64), (4, 512, 1024, Q1), (1, 17408, 5120, PQ2), (1, 17408, 5120, G64)]
+                (600, 1280, 384, G64), (4, 512, 1024, G64), (4, 512, 1024, Q1), (1, 17408, 5120, PQ2), (1, 17408, 5120, G64),
+                (2, 1024, 2048, PQ2), (2, 24, 512, PQ2), (2, 4000, 1152, G64), (2, 17408, 5120, PQ2),
+                (3, 1024, 2048, PQ2), (3, 24, 640, PQ2)]
 
 
 @pytest.mark.parametrize("M,F,K,fmt", SWIGLU_CASES)
