@@ -197,9 +197,10 @@ int bonsai_swiglu(const uint16_t *y, uint16_t *h, int64_t M, int64_t F, void *st
 /* The fused gate/up linear layer followed by SwiGLU: packed and scales hold 2F weight rows
  * (gate rows first, then up rows: the N = 2F plane of bonsai_ternary_linear) and h gets
  * the M x F result of bonsai_swiglu applied to their product with x'.  On the integer
- * tensor-core GEMV (M = 1 PQ2_0, PQ2_0 g64) and the prefill GEMM the step runs in the kernel's
- * epilogue on the FP32 sums; the lookup-table GEMV, the skinny and the plain kernel write
- * the product to the library's workspace in FP16 and bonsai_swiglu follows. */
+ * tensor-core GEMV (PQ2_0 and PQ2_0 g64 at the batches and K it takes: see
+ * BONSAI_ALGO_IMMA) and the prefill GEMM the step runs in the kernel's epilogue on the
+ * FP32 sums; the lookup-table GEMV, the skinny and the plain kernel write the product to
+ * the library's workspace in FP16 and bonsai_swiglu follows. */
 int bonsai_ternary_linear_swiglu(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
                                  uint16_t *h, int64_t M, int64_t F, int64_t K, int fmt, void *stream);
 
