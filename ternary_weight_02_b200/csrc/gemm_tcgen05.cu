@@ -764,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tcgen05_kernel(
                     }
                     const int st = it % STAGES;
                     const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-                    // every lane acquires the stage itself (and, PQ2_0, its codes); the verdict
+                    // every lane acquires the stage itself (and, PQ2_0, its codes); the outcome
                     // is made warp-uniform
                     const bool free_ok = !*abort_flag && mbar_wait(empty + st, ph ^ 1u) &&
                                          (!kTma || mbar_wait(full_a + st, ph));

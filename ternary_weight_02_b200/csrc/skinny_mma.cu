@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(kThreads) skinny_kernel(
             for (int gs = 0; gs < nsub; gs += kTGroups) {
                 const int q = (sub - g_begin + gs) / kTGroups;  // the stage
                 const int slot = q % kTStages;
-                if (copies_ok) {  // warp-uniform verdict
+                if (copies_ok) {  // warp-uniform outcome
                     copies_ok = __all_sync(0xffffffffu, mbar_wait(bars + slot, (uint32_t)(q / kTStages) & 1u));
                     if (copies_ok)
                         n_waited++;
