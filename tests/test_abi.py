@@ -97,6 +97,17 @@ def test_integer_gemv_batch_limits_on_the_host(bz):
             assert call(M, K, fmt) == bz.BONSAI_ERR_CUDA, (M, K, fmt)
 
 
+def test_binding_constants_match_the_header(bz):
+    """Every enumerator and BONSAI_DEVICE_* bit the header defines has the same value in
+    the Python binding, and the binding defines no other BONSAI_ constant."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    header = {n: int(v) for n, v in re.findall(r"\b(BONSAI_[A-Z0-9_]+)\s*=\s*(-?\d+)", text)}
+    header.update({n: int(v) for n, v in re.findall(r"#define\s+(BONSAI_DEVICE_[A-Z0-9_]+)\s+(\d+)u", text)})
+    assert len(header) >= 24  # 4 formats, 10 status codes, 6 kernel choices, 4 device bits
+    binding = {n: getattr(bz, n) for n in dir(bz) if n.startswith("BONSAI_") and isinstance(getattr(bz, n), int)}
+    assert binding == header
+
+
 def test_status_strings(bz):
     for code in range(-9, 1):
         s = bz.bonsai_status_string(code)
