@@ -47,9 +47,11 @@
 //   codes and the lane assembles the same two code words (weights 32tq .. 32tq + 31) the
 //   PQ2_0 path loads; everything after that is PQ2_0's.  The lane's 7 or 8 bytes of a row's
 //   group (from byte 32tq / 5) come as three aligned 32-bit loads.
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
-#include "tma.cuh"  // kSpinLimit: the bound of every wait
+#include "tma.cuh"  // kSpinLimit: the bound of every wait; TMA and mbarrier wrappers
 
 namespace bonsai {
 namespace {
